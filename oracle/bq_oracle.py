@@ -1,0 +1,467 @@
+"""Reference quantizers and layers (float64 / int64), CPU only — test infrastructure.
+
+Conventions
+-----------
+* W [N,K] float32 weights, x [M,K] bf16-exact float32 activations, y [M,N].
+* "rn" = IEEE round-to-nearest-even (numpy ``rint``).
+* Decisions that turn floating point into an integer code (sign, rounding,
+  nearest point) are taken in float32 where the stored operands are float32,
+  exactly as written below, so the CUDA path can reach the same codes
+  bit-for-bit; every sum, mean and layer product is float64 / int64.
+* Integer accumulators are direct code products (textbook loops via int64
+  matmul): no bit-planes and no popcount, so they are independent of the
+  bit-plane arithmetic they check.
+
+Page keys ([RaBiT], [HGF], [ABQ], [BVSR], [BitNet]) are listed in the package
+docstring.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+# ---------------------------------------------------------------------------
+# shared helpers
+# ---------------------------------------------------------------------------
+
+
+def _f32(a) -> np.ndarray:
+    return np.asarray(a, dtype=np.float32)
+
+
+def bf16_round(a) -> np.ndarray:
+    """Round to the nearest bfloat16 (ties to even), returned as float32.
+
+    Used where a format stores a tensor in bf16 (the LoRA matrices of [HGF]
+    §2.1 are an fp16/bf16 correction path)."""
+    f = np.ascontiguousarray(_f32(a))
+    u = f.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000).astype(np.uint32)
+    return r.view(np.float32).reshape(f.shape)
+
+
+def sign_pm1(v) -> np.ndarray:
+    """sign(v) = +1 if v >= 0 else -1 ([BitNet] §2.1). -0.0 >= 0 holds, so
+    sign(-0.0) = +1. Pinned by tests (zero, negative zero, tiny values)."""
+    v = np.asarray(v)
+    return np.where(v >= 0, 1, -1).astype(np.int8)
+
+
+def mean_abs_f32(a) -> np.float32:
+    """mean(|a|) summed in float64, stored as float32."""
+    a64 = np.abs(np.asarray(a, dtype=np.float64))
+    if a64.size == 0:
+        return np.float32(0.0)
+    return np.float32(a64.sum() / a64.size)
+
+
+# ---------------------------------------------------------------------------
+# activation quantization
+# ---------------------------------------------------------------------------
+
+
+def quantize_act_int8(x) -> tuple[np.ndarray, np.ndarray]:
+    """Per-token absmax int8 quantization ([HGF] §1.2: activations to 8-bit
+    integers, dequantized by gamma_x/127; [BVSR] Introduction: lightweight
+    online quantization of the input).
+
+    gamma[m] = max_k |x[m,k]|;  s = 127 / gamma (float32);
+    q = clamp(rn(x * s), -127, 127) with x*s a float32 product.
+    gamma == 0 gives q == 0. Returns (q int8 [M,K], gamma float32 [M]).
+    Pinned by tests (scale endpoints map to +-127, ties, zero rows)."""
+    x = _f32(x)
+    M, K = x.shape
+    gamma = np.abs(x).max(axis=1) if K > 0 else np.zeros(M, np.float32)
+    gamma = gamma.astype(np.float32)
+    q = np.zeros((M, K), dtype=np.int8)
+    for m in range(M):
+        if gamma[m] > 0:
+            s = np.float32(127.0) / gamma[m]
+            v = (x[m] * s).astype(np.float32)
+            q[m] = np.clip(np.rint(v), -127, 127).astype(np.int8)
+    return q, gamma
+
+
+def dequant_act_int8(q, gamma) -> np.ndarray:
+    """x_hat = q * gamma / 127 in float64 ([HGF] §1.2 dequantization)."""
+    return q.astype(np.float64) * (gamma.astype(np.float64)[:, None] / 127.0)
+
+
+def quantize_rows_asym(V, bits: int) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Uniform asymmetric quantizer per row ([ABQ] §3.2 eq.(3) with the
+    compensation term off, gamma=0, and no learned clipping, alpha=beta=1 of
+    §3.1 eq.(1)):
+
+      lo = min(row), hi = max(row)                       (float32, exact)
+      Delta = max(hi - lo, 1e-5) / (2^bits - 1)          (float32 ops)
+      z = rn(-lo / Delta)                                (integer, not clamped)
+      q = clamp(rn(v / Delta) + z, 0, 2^bits - 1)
+
+    Returns (q int32 [R,L], Delta float32 [R], z int32 [R]).
+    Pinned by tests (a hand example with a rounding tie, grid round-trip)."""
+    V = _f32(V)
+    R, L = V.shape
+    qmax = (1 << bits) - 1
+    lo = V.min(axis=1).astype(np.float32)
+    hi = V.max(axis=1).astype(np.float32)
+    rng_ = np.maximum((hi - lo).astype(np.float32), np.float32(1e-5)).astype(np.float32)
+    delta = (rng_ / np.float32(qmax)).astype(np.float32)
+    z = np.rint((-lo / delta).astype(np.float32)).astype(np.int64)
+    q = np.rint((V / delta[:, None]).astype(np.float32)).astype(np.int64) + z[:, None]
+    q = np.clip(q, 0, qmax)
+    return q.astype(np.int32), delta, z.astype(np.int32)
+
+
+# ---------------------------------------------------------------------------
+# RaBiT: two residual binary paths ([RaBiT] §2.1, §2.2)
+# ---------------------------------------------------------------------------
+
+
+def rabit_pack(W, h2) -> dict:
+    """W_hat = g1*B1*h1 + g2*B2*h2 built by the residual recursion of [RaBiT]
+    §2.2: B1 = sign(W); W1 = g1 B1 h1; R1 = W - W1; B2 = sign(R1); W2 = g2 B2 h2.
+
+    The pages learn g and h; here g_p[n] = mean_k |.| of the binarized matrix
+    row (W for path 1, R1 for path 2), h1 = 1, h2 given.
+    R1 is formed from the stored float32 g1, and sign(R1) is the sign of the
+    exact difference W - g1*B1 (a float32 subtraction keeps that sign).
+    Pinned by tests (recursion-order hand example, constant-magnitude rows)."""
+    W = _f32(W)
+    N, K = W.shape
+    B1 = sign_pm1(W)
+    g1 = np.array([mean_abs_f32(W[n]) for n in range(N)], dtype=np.float32)
+    h1 = np.ones(K, dtype=np.float32)
+    R1 = W.astype(np.float64) - g1.astype(np.float64)[:, None] * B1 * h1.astype(np.float64)
+    B2 = sign_pm1(R1)
+    g2 = np.array([mean_abs_f32(R1[n]) for n in range(N)], dtype=np.float32)
+    return dict(B1=B1, B2=B2, g1=g1, g2=g2, h1=h1, h2=_f32(h2).copy())
+
+
+def rabit_weight(p) -> np.ndarray:
+    """W_hat [N,K] float64 = g1*B1*h1 + g2*B2*h2 ([RaBiT] §2.1)."""
+    g1, g2 = p["g1"].astype(np.float64), p["g2"].astype(np.float64)
+    h1, h2 = p["h1"].astype(np.float64), p["h2"].astype(np.float64)
+    return g1[:, None] * p["B1"] * h1[None, :] + g2[:, None] * p["B2"] * h2[None, :]
+
+
+def rabit_layer(p, x) -> dict:
+    """y = W_hat x in float64 with x the unquantized bf16 activations (the
+    RaBiT kernel of [RaBiT] §3.2 applies signs to the input, no activation
+    quantization). Also returns the per-path sums acc_p = sum_k B_p h_p x."""
+    x64 = _f32(x).astype(np.float64)
+    y = x64 @ rabit_weight(p).T
+    acc1 = x64 @ (p["B1"] * p["h1"].astype(np.float64)[None, :]).T
+    acc2 = x64 @ (p["B2"] * p["h2"].astype(np.float64)[None, :]).T
+    return dict(y=y, acc1=acc1, acc2=acc2)
+
+
+# ---------------------------------------------------------------------------
+# BitNet W1A8 ([BitNet] §2.1-2.3)
+# ---------------------------------------------------------------------------
+
+
+def bitnet_pack(W) -> dict:
+    """W ~= alpha * sign(W) with one alpha per matrix ([BitNet] §2.2); the page
+    learns alpha, here alpha = mean|W| over the whole tensor."""
+    W = _f32(W)
+    return dict(B=sign_pm1(W), alpha=mean_abs_f32(W))
+
+
+def bitnet_layer(p, x) -> dict:
+    """acc = sum_k B[n,k] q[m,k] (int64); y = sum_k (alpha B)(q gamma/127) in
+    float64 ([BitNet] §2.3 binary product scaled by alpha; activation scale of
+    [HGF] §1.2)."""
+    q, gamma = quantize_act_int8(x)
+    acc = q.astype(np.int64) @ p["B"].astype(np.int64).T
+    w_hat = np.float64(p["alpha"]) * p["B"].astype(np.float64)
+    y = dequant_act_int8(q, gamma) @ w_hat.T
+    return dict(q=q, gamma=gamma, acc=acc, y=y)
+
+
+# ---------------------------------------------------------------------------
+# Ternary W1.58A8 with gated low-rank correction ([HGF] §1.2, §2.1, §4.1)
+# ---------------------------------------------------------------------------
+
+
+def ternary_pack(W, lora_A=None, lora_B=None, lora_alpha: float = 0.1) -> dict:
+    """gamma = mean|W| (the code of [HGF] §1.2 uses the mean although the prose
+    says absmax); T = clamp(rn(W / gamma), -1, 1) with W/gamma a float32
+    division and rn ties-to-even (torch.round). gamma == 0 gives T == 0.
+    LoRA A [K,r], B [r,N] are stored in bf16 ([HGF] §2.1 fp16 correction path).
+    Pinned by tests (hand examples with +-0.5 ties, zero fraction of a
+    Gaussian matrix)."""
+    W = _f32(W)
+    gamma = mean_abs_f32(W)
+    if gamma > 0:
+        T = np.clip(np.rint((W / gamma).astype(np.float32)), -1, 1).astype(np.int8)
+    else:
+        T = np.zeros(W.shape, dtype=np.int8)
+    out = dict(T=T, gamma_w=gamma, lora_alpha=np.float32(lora_alpha))
+    if lora_A is not None:
+        out["A"] = bf16_round(lora_A)
+        out["B"] = bf16_round(lora_B)
+    return out
+
+
+def silu(z):
+    return z / (1.0 + np.exp(-z))
+
+
+def lora_correction(x, A, B, alpha) -> np.ndarray:
+    """tanh(alpha) * (SiLU(x @ A) @ B) in float64 ([HGF] §2.1), x unquantized."""
+    x64 = _f32(x).astype(np.float64)
+    u = silu(x64 @ A.astype(np.float64))
+    return math.tanh(float(np.float32(alpha))) * (u @ B.astype(np.float64))
+
+
+def ternary_layer(p, x) -> dict:
+    """acc = sum_k T q (int64); y = gamma_w*gamma_x/127 * acc + LoRA term,
+    the ternary part computed as a float64 product of dequantized operands
+    ([HGF] §1.2 int8 product with Y_int * gamma_x gamma_W / 127)."""
+    q, gamma = quantize_act_int8(x)
+    acc = q.astype(np.int64) @ p["T"].astype(np.int64).T
+    w_hat = np.float64(p["gamma_w"]) * p["T"].astype(np.float64)
+    y_t = dequant_act_int8(q, gamma) @ w_hat.T
+    y_l = lora_correction(x, p["A"], p["B"], p["lora_alpha"]) if "A" in p else 0.0 * y_t
+    return dict(q=q, gamma=gamma, acc=acc, y=y_t + y_l, y_ternary=y_t, y_lora=y_l)
+
+
+# ---------------------------------------------------------------------------
+# ABQ-style arbitrary-bit WxAy ([ABQ] §3.1-3.2, abstract)
+# ---------------------------------------------------------------------------
+
+
+def abq_pack(W, w_bits: int) -> dict:
+    """Per-output-row asymmetric weight codes (quantize_rows_asym)."""
+    Q, delta, z = quantize_rows_asym(W, w_bits)
+    return dict(Q=Q, delta=delta, z=z, w_bits=w_bits)
+
+
+def abq_layer(p, x, a_bits: int) -> dict:
+    """Per-token asymmetric activation codes, then
+    I = sum_k (qw - zw)(qx - zx) (int64) and y = Dw*Dx*I as the float64 product
+    of the dequantized operands."""
+    Qx, dx, zx = quantize_rows_asym(x, a_bits)
+    cw = p["Q"].astype(np.int64) - p["z"].astype(np.int64)[:, None]
+    cx = Qx.astype(np.int64) - zx.astype(np.int64)[:, None]
+    I = cx @ cw.T
+    w_hat = p["delta"].astype(np.float64)[:, None] * cw
+    x_hat = dx.astype(np.float64)[:, None] * cx
+    y = x_hat @ w_hat.T
+    return dict(Qx=Qx, delta_x=dx, z_x=zx, I=I, y=y)
+
+
+# ---------------------------------------------------------------------------
+# Bit-plane identities (what the binary AND+popcount kernels compute)
+# ---------------------------------------------------------------------------
+
+
+def popcount(v) -> np.ndarray:
+    v = np.asarray(v, dtype=np.uint64)
+    c = np.zeros(v.shape, dtype=np.int64)
+    for b in range(64):
+        c += ((v >> np.uint64(b)) & np.uint64(1)).astype(np.int64)
+    return c
+
+
+def planes_of(codes, bits: int) -> list:
+    """Bit-plane b of non-negative or two's-complement codes: a 0/1 array."""
+    c = np.asarray(codes, dtype=np.int64) & ((1 << bits) - 1)
+    return [((c >> b) & 1).astype(np.uint8) for b in range(bits)]
+
+
+def plane_weights(bits: int, signed: bool) -> list:
+    """omega_b = 2^b; for two's complement the top plane weighs -2^(bits-1)."""
+    w = [1 << b for b in range(bits)]
+    if signed:
+        w[-1] = -w[-1]
+    return w
+
+
+def pack_bits(bitvec) -> int:
+    """A 0/1 vector as one integer word, element j at bit j (LSB first)."""
+    out = 0
+    for j, b in enumerate(np.asarray(bitvec).tolist()):
+        out |= int(b) << j
+    return out
+
+
+def bitplane_dot(wc, w_bits, w_signed, xc, x_bits, x_signed) -> int:
+    """sum_b sum_c omega_b omega_c popc(W_b AND X_c) over one vector pair, the
+    arbitrary-bit product of [ABQ] (abstract: binary tensor-core equivalent
+    operations), computed literally with popcounts of packed words."""
+    wp, xp = planes_of(wc, w_bits), planes_of(xc, x_bits)
+    ww, xw = plane_weights(w_bits, w_signed), plane_weights(x_bits, x_signed)
+    tot = 0
+    for b in range(w_bits):
+        Wb = pack_bits(wp[b])
+        for c in range(x_bits):
+            Xc = pack_bits(xp[c])
+            tot += ww[b] * xw[c] * bin(Wb & Xc).count("1")
+    return tot
+
+
+def xnor_popcount_dot(a_pm1, b_pm1) -> int:
+    """[BitNet] §2.3: popcount(xnor(a, b)) for +-1 vectors coded as bit 1 <=> +1.
+    Returns 2*popc(xnor) - K, the +-1 inner product (the page's formula without
+    the affine correction is the count of agreeing positions)."""
+    a = pack_bits(np.asarray(a_pm1) > 0)
+    b = pack_bits(np.asarray(b_pm1) > 0)
+    K = len(a_pm1)
+    xnor = ~(a ^ b) & ((1 << K) - 1)
+    return 2 * bin(xnor).count("1") - K
+
+
+# ---------------------------------------------------------------------------
+# BVSR: bitvector-sum weights with cached coefficient sets ([BVSR] Introduction)
+# ---------------------------------------------------------------------------
+
+BVSR_VEC = 32
+BVSR_RATIOS = (1.5, 2.0, 2.5, 3.0)
+BVSR_GRID = 8          # lo/hi grid points per side: 4 ratios x 8 x 8 = 256 sets
+BVSR_PLANES = 4
+
+
+def nearest_rank(sorted_vals: np.ndarray, num: int, den: int):
+    """Nearest-rank quantile num/den of an ascending array: element
+    ceil(num*V/den) - 1 (integer arithmetic)."""
+    V = len(sorted_vals)
+    rank = (num * V + den - 1) // den
+    return sorted_vals[max(rank - 1, 0)]
+
+
+def bvsr_set_table(W) -> np.ndarray:
+    """The cached coefficient sets shared by all vectors of a matrix.
+
+    [BVSR] Introduction: geometric-series subset sums scaled and shifted by
+    data-dependent terms; geometric coefficient sets paired with an auxiliary
+    grid aligned to the data range; 256 sets (4 ratios x 8 x 8).
+    Reading (the page gives no formula): set s = 64*j + 8*a + b has ratio
+    r_j in {1.5, 2, 2.5, 3}, template t_i = r^i / sum_{i'<4} r^{i'},
+    lo_a = the (2a+1)/16 nearest-rank quantile of the per-vector minima,
+    hi_b = the (2b+1)/16 quantile of the per-vector maxima,
+    c_i = (hi_b - lo_a) * t_i and o = lo_a (float64, stored float32).
+    Returns table float32 [256, 5] = (c0, c1, c2, c3, o). Parity unpinned as a
+    reading; pinned by the r=2 uniform-grid case and size arithmetic."""
+    W = _f32(W)
+    N, K = W.shape
+    vecs = W.reshape(N, K // BVSR_VEC, BVSR_VEC)
+    smin = np.sort(vecs.min(axis=2).ravel())
+    smax = np.sort(vecs.max(axis=2).ravel())
+    los = [np.float64(nearest_rank(smin, 2 * a + 1, 16)) for a in range(BVSR_GRID)]
+    his = [np.float64(nearest_rank(smax, 2 * b + 1, 16)) for b in range(BVSR_GRID)]
+    table = np.zeros((len(BVSR_RATIOS) * BVSR_GRID * BVSR_GRID, 5), dtype=np.float32)
+    for j, r in enumerate(BVSR_RATIOS):
+        pw = [r ** i for i in range(BVSR_PLANES)]
+        tsum = sum(pw)
+        t = [pw[i] / tsum for i in range(BVSR_PLANES)]
+        for a in range(BVSR_GRID):
+            for b in range(BVSR_GRID):
+                s = 64 * j + 8 * a + b
+                span = his[b] - los[a]
+                for i in range(BVSR_PLANES):
+                    table[s, i] = np.float32(span * t[i])
+                table[s, 4] = np.float32(los[a])
+    return table
+
+
+def bvsr_points(table) -> np.ndarray:
+    """P[s, code] = o + c0 b0 + c1 b1 + c2 b2 + c3 b3 (b_i = bit i of code),
+    summed left to right in float64 from the float32 coefficients."""
+    t = np.asarray(table, dtype=np.float32).astype(np.float64)
+    S = t.shape[0]
+    P = np.zeros((S, 16), dtype=np.float64)
+    for code in range(16):
+        acc = t[:, 4].copy()
+        for i in range(BVSR_PLANES):
+            if (code >> i) & 1:
+                acc = acc + t[:, i]
+        P[:, code] = acc
+    return P
+
+
+def bvsr_encode_vectors(vecs, table) -> tuple[np.ndarray, np.ndarray]:
+    """Exhaustive search ([BVSR] Introduction): for every vector and every set,
+    each element takes the nearest of the set's 16 points (smallest |w - p|,
+    lowest code on a tie), the set's error is sum_e (w_e - p)^2 accumulated in
+    element order in float64, and the vector takes the set with the smallest
+    error (lowest set index on a tie).
+    vecs float32 [V, 32] -> (codes uint8 [V, 32], set index uint8 [V])."""
+    vecs = _f32(vecs)
+    V = vecs.shape[0]
+    P = bvsr_points(table)                      # [S,16]
+    codes_out = np.zeros((V, BVSR_VEC), dtype=np.uint8)
+    sets_out = np.zeros(V, dtype=np.uint8)
+    chunk = 32
+    for v0 in range(0, V, chunk):
+        w = vecs[v0:v0 + chunk].astype(np.float64)              # [c,32]
+        d = np.abs(w[:, None, :, None] - P[None, :, None, :])   # [c,S,32,16]
+        best = np.argmin(d, axis=3)                             # [c,S,32]
+        pbest = P[np.arange(P.shape[0])[None, :, None], best]   # [c,S,32]
+        err = np.zeros(best.shape[:2], dtype=np.float64)
+        for e in range(BVSR_VEC):
+            de = w[:, None, e] - pbest[:, :, e]
+            err = err + de * de
+        s = np.argmin(err, axis=1)
+        sets_out[v0:v0 + chunk] = s
+        codes_out[v0:v0 + chunk] = best[np.arange(w.shape[0]), s]
+    return codes_out, sets_out
+
+
+def bvsr_pack(W, table=None, rows=None) -> dict:
+    """BVSR 4-bit pack of W [N,K] (K % 32 == 0). ``rows`` restricts the
+    encoding to a subset of rows (the table still comes from the whole W).
+    Returns codes uint8 [R,K], set index uint8 [R,K/32], table [256,5]."""
+    W = _f32(W)
+    N, K = W.shape
+    if table is None:
+        table = bvsr_set_table(W)
+    sel = np.arange(N) if rows is None else np.asarray(rows)
+    sub = W[sel]
+    codes, sets = bvsr_encode_vectors(sub.reshape(-1, BVSR_VEC), table)
+    return dict(codes=codes.reshape(len(sel), K), sets=sets.reshape(len(sel), K // BVSR_VEC),
+                table=table, rows=sel)
+
+
+def bvsr_weight(codes, sets, table) -> np.ndarray:
+    """W_hat[n,k] = P[set(n, k/32), code(n,k)] in float64."""
+    P = bvsr_points(table)
+    R, K = codes.shape
+    s_full = np.repeat(sets.astype(np.int64), BVSR_VEC, axis=1)
+    return P[s_full, codes.astype(np.int64)]
+
+
+def bvsr_layer(codes, sets, table, x) -> dict:
+    """acc = sum_k code q (int64, code = sum_i 2^i b_i); y = sum_k W_hat x_hat in
+    float64, x_hat the per-token absmax int8 activations ([BVSR] Introduction:
+    activations quantized online, product without weight dequantization)."""
+    q, gamma = quantize_act_int8(x)
+    acc = q.astype(np.int64) @ codes.astype(np.int64).T
+    y = dequant_act_int8(q, gamma) @ bvsr_weight(codes, sets, table).T
+    return dict(q=q, gamma=gamma, acc=acc, y=y)
+
+
+# ---------------------------------------------------------------------------
+# size and bandwidth arithmetic
+# ---------------------------------------------------------------------------
+
+
+def decode_tokens_per_s(bandwidth_bytes_s: float, params: float, bits: float) -> float:
+    """Memory-wall bound T_max <= B_mem / (P * b / 8) ([HGF] §1.1)."""
+    return bandwidth_bytes_s / (params * bits / 8.0)
+
+
+def weight_bits_per_param(fmt: str, w_bits: int = 0) -> float:
+    """Storage bits per weight of the packed planes/bitvectors (scales excluded;
+    BVSR counts its 1-byte set index per 32-element vector)."""
+    return {"rabit": 2.0, "bitnet": 1.0, "ternary": 2.0, "abq": float(w_bits),
+            "bvsr": BVSR_PLANES + 8.0 / BVSR_VEC}[fmt]
+
+
+def tolerance_ok(y, y_ref, rel: float = 1e-3) -> bool:
+    """max|y - y_ref| <= rel * (||y_ref||_inf + 1e-6)."""
+    y, y_ref = np.asarray(y, np.float64), np.asarray(y_ref, np.float64)
+    if y_ref.size == 0:
+        return y.size == 0
+    return float(np.max(np.abs(y - y_ref))) <= rel * (float(np.max(np.abs(y_ref))) + 1e-6)

@@ -1,0 +1,226 @@
+"""Independent readers of the library's byte formats — test infrastructure only.
+
+These decode a host copy of a packed-weight buffer or an activation buffer,
+following the documented byte layout (declared in ``include/bq.h``), back
+into plain codes and scales that the reference layers of ``bq_oracle`` take.
+Nothing here is shared with the CUDA path; a reader bug and a writer bug
+would have to agree on the same wrong index to go unnoticed, and the golden
+fixtures in ``tests/golden`` pin single-bit positions by hand.
+
+Packed weight buffer: 256-byte header of little-endian 32-bit words, then
+sections at the header's offsets.
+
+  word  field                      word  field
+  0     magic 0x4B505142 'BQPK'    18    tile_bytes
+  1     version (1)                19    lora_rank
+  2     format (1..5)              20    lora_alpha (f32)
+  3     N                          21    tensor_scale (f32): BitNet alpha, ternary gamma_W
+  4     K                          22-23 total_bytes (u64)
+  5     N_pad (multiple of 16)     24-25 off_tiles (u64)
+  6     K_pad (multiple of 256)    26-27 off_rows  (u64)
+  7     w_bits                     28-29 off_aux   (u64)
+  8     a_bits                     30-31 off_aux2  (u64)
+  9     n_streams
+  10-13 stream field width f_s (bits per weight per stream)
+  14-17 stream shift (bit offset of the stream inside the code / plane index)
+
+Tiled weights (formats 2-5): tile (rb, kt) covers rows 16*rb .. +15 and
+k = 256*kt .. +255 and sits at off_tiles + (rb*KT + kt)*tile_bytes, with the
+streams one after another, stream s taking 512*f_s bytes laid out as
+[u < f_s][lane < 32][4 words]. In word r (0..3) of uint4 u of lane = 4g+t,
+the f-bit field j (bits f*j .. f*j+f-1) of byte b holds the weight at
+
+  row = 16*rb + g + 8*(r & 1)
+  k   = 32*(8*kt + u*(8/f) + j) + 16*(r >> 1) + 4*t + b.
+
+RaBiT (format 1) is not tiled: plane p (0,1) word w of row n is the uint32 at
+off_tiles + 4*((p*N_pad + n)*(K_pad/32) + w), bit j <-> k = 32w + j; a set bit
+means sign -1.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+PK_MAGIC = 0x4B505142
+ACT_MAGIC = 0x43415142
+FMT_RABIT, FMT_BITNET, FMT_TERNARY, FMT_ABQ, FMT_BVSR = 1, 2, 3, 4, 5
+FMT_NAMES = {1: "rabit", 2: "bitnet", 3: "ternary", 4: "abq", 5: "bvsr"}
+
+
+def _u32(buf: bytes, word: int) -> int:
+    return int(np.frombuffer(buf, dtype="<u4", count=1, offset=4 * word)[0])
+
+
+def _u64(buf: bytes, word: int) -> int:
+    return int(np.frombuffer(buf, dtype="<u8", count=1, offset=4 * word)[0])
+
+
+def _f32(buf: bytes, word: int) -> np.float32:
+    return np.frombuffer(buf, dtype="<f4", count=1, offset=4 * word)[0]
+
+
+def read_header(buf: bytes) -> dict:
+    if _u32(buf, 0) != PK_MAGIC:
+        raise ValueError("bad packed magic")
+    h = dict(version=_u32(buf, 1), fmt=_u32(buf, 2), N=_u32(buf, 3), K=_u32(buf, 4),
+             N_pad=_u32(buf, 5), K_pad=_u32(buf, 6), w_bits=_u32(buf, 7), a_bits=_u32(buf, 8),
+             n_streams=_u32(buf, 9), tile_bytes=_u32(buf, 18), lora_rank=_u32(buf, 19),
+             lora_alpha=_f32(buf, 20), tensor_scale=_f32(buf, 21), total_bytes=_u64(buf, 22),
+             off_tiles=_u64(buf, 24), off_rows=_u64(buf, 26), off_aux=_u64(buf, 28),
+             off_aux2=_u64(buf, 30))
+    h["fields"] = [_u32(buf, 10 + s) for s in range(h["n_streams"])]
+    h["shifts"] = [_u32(buf, 14 + s) for s in range(h["n_streams"])]
+    return h
+
+
+def tiled_field_index(N_pad: int, K_pad: int, f: int):
+    """For one stream of field width f, the (row, k) that each field of a tile
+    holds, as arrays over [u, lane, r, b, j] (the documented formula)."""
+    u = np.arange(f)[:, None, None, None, None]
+    lane = np.arange(32)[None, :, None, None, None]
+    r = np.arange(4)[None, None, :, None, None]
+    b = np.arange(4)[None, None, None, :, None]
+    j = np.arange(8 // f)[None, None, None, None, :]
+    g, t = lane // 4, lane % 4
+    row = g + 8 * (r & 1) + 0 * (u + b + j)
+    kk = 32 * (u * (8 // f) + j) + 16 * (r >> 1) + 4 * t + b
+    return row, kk
+
+
+def read_stream_codes(buf: bytes, h: dict, s: int) -> np.ndarray:
+    """Stream s of a tiled buffer as unsigned field values [N, K] (uint8)."""
+    f = h["fields"][s]
+    N, K, N_pad, K_pad = h["N"], h["K"], h["N_pad"], h["K_pad"]
+    RB, KT, tb = N_pad // 16, K_pad // 256, h["tile_bytes"]
+    s_off = sum(512 * h["fields"][i] for i in range(s))
+    raw = np.frombuffer(buf, dtype=np.uint8, count=RB * KT * tb, offset=h["off_tiles"])
+    tiles = raw.reshape(RB, KT, tb)[:, :, s_off:s_off + 512 * f].reshape(RB, KT, f, 32, 4, 4)
+    row_i, k_i = tiled_field_index(N_pad, K_pad, f)
+    nj = 8 // f
+    mask = (1 << f) - 1
+    # field j of every byte: [RB, KT, f, 32, 4, 4, nj]
+    vals = (tiles[..., None] >> (f * np.arange(nj))) & mask
+    out = np.zeros((N_pad, K_pad), dtype=np.uint8)
+    rb = np.arange(RB)[:, None, None, None, None, None, None]
+    kt = np.arange(KT)[None, :, None, None, None, None, None]
+    rows = 16 * rb + row_i[None, None]
+    ks = 256 * kt + k_i[None, None]
+    rows, ks = np.broadcast_arrays(rows, ks)
+    out[rows, ks] = vals
+    return out[:N, :K]
+
+
+def read_packed(buf: bytes) -> dict:
+    """Decode a packed buffer into the dict shape that bq_oracle's layers take."""
+    h = read_header(buf)
+    fmt, N, K, N_pad, K_pad = h["fmt"], h["N"], h["K"], h["N_pad"], h["K_pad"]
+    out = dict(header=h)
+    if fmt == FMT_RABIT:
+        W32 = K_pad // 32
+        raw = np.frombuffer(buf, dtype="<u4", count=2 * N_pad * W32, offset=h["off_tiles"])
+        planes = raw.reshape(2, N_pad, W32)
+        bits = ((planes[..., None] >> np.arange(32, dtype=np.uint32)) & 1).reshape(2, N_pad, K_pad)
+        out["B1"] = np.where(bits[0, :N, :K] == 1, -1, 1).astype(np.int8)
+        out["B2"] = np.where(bits[1, :N, :K] == 1, -1, 1).astype(np.int8)
+        g = np.frombuffer(buf, dtype="<f4", count=2 * N_pad, offset=h["off_rows"])
+        out["g1"], out["g2"] = g[:N].copy(), g[N_pad:N_pad + N].copy()
+        out["h1"] = np.frombuffer(buf, dtype="<f4", count=K, offset=h["off_aux"]).copy()
+        out["h2"] = np.frombuffer(buf, dtype="<f4", count=K, offset=h["off_aux2"]).copy()
+    elif fmt == FMT_BITNET:
+        neg = read_stream_codes(buf, h, 0)
+        out["B"] = np.where(neg == 1, -1, 1).astype(np.int8)
+        out["alpha"] = h["tensor_scale"]
+    elif fmt == FMT_TERNARY:
+        u = read_stream_codes(buf, h, 0).astype(np.int16)
+        out["T"] = (u - 1).astype(np.int8)
+        out["field_max"] = int(u.max()) if u.size else 0
+        out["gamma_w"] = h["tensor_scale"]
+        out["lora_alpha"] = h["lora_alpha"]
+        r = h["lora_rank"]
+        if r > 0:
+            A = np.frombuffer(buf, dtype="<u2", count=K_pad * r, offset=h["off_aux"]).reshape(K_pad, r)
+            Bt = np.frombuffer(buf, dtype="<u2", count=N_pad * r, offset=h["off_aux2"]).reshape(N_pad, r)
+            out["A"] = _bf16_to_f32(A[:K])
+            out["B"] = _bf16_to_f32(Bt[:N]).T.copy()
+    elif fmt == FMT_ABQ:
+        Q = np.zeros((N, K), dtype=np.int32)
+        for s in range(h["n_streams"]):
+            Q += read_stream_codes(buf, h, s).astype(np.int32) << h["shifts"][s]
+        out["Q"] = Q
+        rowsec = np.frombuffer(buf, dtype="<u4", count=3 * N_pad, offset=h["off_rows"])
+        out["delta"] = rowsec[:N].view("<f4").copy()
+        out["z"] = rowsec[N_pad:N_pad + N].view("<i4").copy()
+        out["S_w"] = rowsec[2 * N_pad:2 * N_pad + N].view("<i4").copy()
+        out["w_bits"] = h["w_bits"]
+        out["a_bits"] = h["a_bits"]
+    elif fmt == FMT_BVSR:
+        codes = np.zeros((N, K), dtype=np.uint8)
+        for s in range(h["n_streams"]):
+            codes |= (read_stream_codes(buf, h, s) << h["shifts"][s]).astype(np.uint8)
+        out["codes"] = codes
+        tab = np.frombuffer(buf, dtype="<f4", count=256 * 8, offset=h["off_aux"]).reshape(256, 8)
+        out["table"] = tab[:, :5].copy()
+        out["table_derived"] = tab[:, 5:].copy()
+        sets = np.frombuffer(buf, dtype=np.uint8, count=N_pad * (K_pad // 32), offset=h["off_aux2"])
+        out["sets"] = sets.reshape(N_pad, K_pad // 32)[:N, :K // 32].copy()
+    else:
+        raise ValueError(f"unknown format {fmt}")
+    return out
+
+
+def _bf16_to_f32(u16: np.ndarray) -> np.ndarray:
+    return (u16.astype(np.uint32) << 16).view(np.float32)
+
+
+# ---------------------------------------------------------------------------
+# activation buffer
+# ---------------------------------------------------------------------------
+#
+# 256-byte header of 32-bit words:
+#   0 magic 0x43415142 'BQAC'   1 version   2 format   3 M   4 K   5 K_pad
+#   6 a_bits   7 lora_rank   8-9 total_bytes   10-11 off_codes   12-13 off_tok
+#   14-15 off_gsum   16-17 off_u   18-19 off_xt
+# codes (formats 2-5): per token m and k-tile kt, 256 bytes; byte
+#   (m*KT + kt)*256 + 64*t + 8*mu + 4*h + b  holds the code of
+#   k = 32*(8*kt + mu) + 16*h + 4*t + b   (int8 for A8 formats, uint8 for ABQ).
+# tok: [M][4] words: A8 {gamma_x f32, sum_q i32, 0, 0}; ABQ {Delta_x f32, z_x i32, S_x i32, 0}
+# gsum (BVSR): int32 [M][K_pad/32] sums of q over each 32-element vector
+# u (ternary): float32 [M][lora_rank] = SiLU(x A)
+# xt (RaBiT): float32 [2][M][K_pad] = h_p * x
+
+
+def read_act(buf: bytes) -> dict:
+    if _u32(buf, 0) != ACT_MAGIC:
+        raise ValueError("bad act magic")
+    fmt, M, K, K_pad = _u32(buf, 2), _u32(buf, 3), _u32(buf, 4), _u32(buf, 5)
+    a = dict(fmt=fmt, M=M, K=K, K_pad=K_pad, a_bits=_u32(buf, 6), lora_rank=_u32(buf, 7),
+             total_bytes=_u64(buf, 8), off_codes=_u64(buf, 10), off_tok=_u64(buf, 12),
+             off_gsum=_u64(buf, 14), off_u=_u64(buf, 16), off_xt=_u64(buf, 18))
+    KT = K_pad // 256
+    if fmt == FMT_RABIT:
+        xt = np.frombuffer(buf, dtype="<f4", count=2 * M * K_pad, offset=a["off_xt"])
+        a["xt"] = xt.reshape(2, M, K_pad)[:, :, :K].copy()
+        return a
+    dt = np.uint8 if fmt == FMT_ABQ else np.int8
+    raw = np.frombuffer(buf, dtype=dt, count=M * KT * 256, offset=a["off_codes"]).reshape(M, KT, 4, 8, 2, 4)
+    t = np.arange(4)[:, None, None, None]
+    mu = np.arange(8)[None, :, None, None]
+    hh = np.arange(2)[None, None, :, None]
+    b = np.arange(4)[None, None, None, :]
+    kin = 32 * mu + 16 * hh + 4 * t + b                      # [4,8,2,4]
+    codes = np.zeros((M, K_pad), dtype=dt)
+    for kt in range(KT):
+        codes[:, 256 * kt + kin.ravel()] = raw[:, kt].reshape(M, -1)
+    a["codes"] = codes[:, :K]
+    a["codes_pad"] = codes[:, K:]
+    tok = np.frombuffer(buf, dtype="<u4", count=4 * M, offset=a["off_tok"]).reshape(M, 4)
+    a["scale"] = tok[:, 0].view("<f4").copy()
+    a["zero"] = tok[:, 1].view("<i4").copy()
+    a["sum"] = tok[:, 2].view("<i4").copy() if fmt == FMT_ABQ else tok[:, 1].view("<i4").copy()
+    if fmt == FMT_BVSR:
+        a["gsum"] = np.frombuffer(buf, dtype="<i4", count=M * (K_pad // 32),
+                                  offset=a["off_gsum"]).reshape(M, K_pad // 32)[:, :K // 32].copy()
+    if fmt == FMT_TERNARY and a["lora_rank"] > 0:
+        a["u"] = np.frombuffer(buf, dtype="<f4", count=M * a["lora_rank"],
+                               offset=a["off_u"]).reshape(M, a["lora_rank"]).copy()
+    return a

@@ -1,0 +1,51 @@
+"""The oracle's byte-format readers against hand-derived single-field positions."""
+import numpy as np
+
+from oracle import layout as L
+
+
+def _packed(fmt, N, K, fields, tile_bytes, body, tensor_scale=1.0):
+    N_pad, K_pad = -(-N // 16) * 16, -(-K // 256) * 256
+    hdr = np.zeros(64, dtype="<u4")
+    hdr[0], hdr[1], hdr[2], hdr[3], hdr[4], hdr[5], hdr[6] = L.PK_MAGIC, 1, fmt, N, K, N_pad, K_pad
+    hdr[9] = len(fields)
+    for s, f in enumerate(fields):
+        hdr[10 + s] = f
+    hdr[18] = tile_bytes
+    hdr[21] = np.array([tensor_scale], "<f4").view("<u4")[0]
+    total = 256 + len(body)
+    hdr[22], hdr[24] = total, 256
+    return hdr.tobytes() + bytes(body)
+
+
+def test_bitnet_single_negative(golden):
+    g = golden("layout_bits.json")
+    for key in ("bitnet_one_negative", "bitnet_second"):
+        c = g[key]
+        tiles = (c["N"] // 16) * (c["K"] // 256)
+        body = bytearray(tiles * c["tile_bytes"])
+        body[c["byte"]] = c["value"]
+        p = L.read_packed(_packed(L.FMT_BITNET, c["N"], c["K"], [1], c["tile_bytes"], body))
+        neg = np.argwhere(p["B"] == -1).tolist()
+        assert neg == c["neg"]
+
+
+def test_ternary_single_plus(golden):
+    c = golden("layout_bits.json")["ternary_one_plus"]
+    body = bytearray([c["fill"]]) * c["tile_bytes"]
+    body[c["byte"]] = c["value"]
+    p = L.read_packed(_packed(L.FMT_TERNARY, c["N"], c["K"], [2], c["tile_bytes"], body))
+    assert np.argwhere(p["T"] == 1).tolist() == c["plus"]
+    assert np.count_nonzero(p["T"]) == 1
+
+
+def test_act_single_code(golden):
+    c = golden("layout_bits.json")["act_one_code"]
+    hdr = np.zeros(64, dtype="<u4")
+    hdr[0], hdr[1], hdr[2], hdr[3], hdr[4], hdr[5], hdr[6] = L.ACT_MAGIC, 1, L.FMT_BITNET, 1, 256, 256, 8
+    hdr[10], hdr[12] = 256, 256 + 256
+    body = bytearray(256 + 16)
+    body[c["byte"]] = c["value"] & 0xFF
+    a = L.read_act(hdr.tobytes() + bytes(body))
+    nz = np.nonzero(a["codes"][0])[0].tolist()
+    assert nz == [c["k"]] and int(a["codes"][0, c["k"]]) == c["value"]
