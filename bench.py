@@ -1,0 +1,369 @@
+"""Benchmark: BitNet W1A8 decode GEMV (M=1) on the Llama-7B projection shapes.
+
+One step = one decode token through a 32-layer Llama-7B linear stack at
+W1A8: per decoder layer q, k, v, o [4096x4096], gate, up [11008x4096] and
+down [4096x11008], each layer call = bq_quantize_act + bq_gemv (224 calls,
+about 820 MB of packed weights, so every step streams inputs larger than L2).
+Weights ~ N(0, 0.02^2) and activations ~ N(0, 1) are synthetic (seeded torch
+generator on the device; no model or dataset).
+
+Prints one JSON line (rank 0). `value` = algorithmic HBM bytes of all ranks'
+steps / max-over-ranks device time, in GB/s; `us_per_layer` is the same run
+expressed per layer call. `--impl reference` times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "µs/layer & achieved HBM GB/s (% of B200 peak), quantized GEMV/GEMM, M=1..64"
+LLAMA7B = [("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
+           ("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008)]
+NOMINAL_HBM_GBS = 8000.0
+
+
+def layer_bytes(fmt: str, N: int, K: int, M: int = 1, w_bits: int = 1, a_bits: int = 8) -> dict:
+    """Algorithmic bytes of one layer call: packed weights + per-row/tensor scales,
+    x bf16 read by the act kernel, act codes written and read once, y fp32."""
+    bits = {"bitnet": 1, "ternary": 2, "abq": w_bits, "bvsr": 4}[fmt]
+    w = N * K * bits // 8
+    extra = {"bitnet": 4, "ternary": 4, "abq": 12 * N, "bvsr": N * K // 32 + 256 * 32}[fmt]
+    x = 2 * M * K
+    act = M * K
+    y = 4 * M * N
+    return dict(gemv=w + extra + act + y + 16 * M, act=x + act + 16 * M, total=w + extra + x + 2 * act + y + 32 * M)
+
+
+def measured_peaks() -> tuple[float, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "bit_weight_quantization_b200", "csrc")
+    for fn in sorted(os.listdir(d)):
+        with open(os.path.join(d, fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(kernel_key: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel_key)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "20", "-i", str(index)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons, pw = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1])); mx.append(float(f[2])); pw.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() in ("active", "1"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(pw), "window": "warmup+timed"}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle arm / baseline
+# ---------------------------------------------------------------------------
+def oracle_sample(seconds: float, seed: int = 0, min_calls: int = 2) -> dict:
+    """Time the CPU oracle (act quantization + reference layer) on q-projection
+    sized BitNet W1A8 layer calls (4096x4096, M=1) for about `seconds`."""
+    import bq_inputs as I
+    from oracle import bq_oracle as O
+    W = I.weights(4096, 4096, seed)
+    x = I.activations(1, 4096, seed)
+    p = O.bitnet_pack(W)
+    calls, t0 = 0, time.perf_counter()
+    while True:
+        O.bitnet_layer(p, x)
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= seconds and calls >= min_calls:
+            break
+    b = layer_bytes("bitnet", 4096, 4096)["total"]
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    return dict(seconds=el, calls=calls, gbs=calls * b / el / 1e9, us_per_layer=el / calls * 1e6, cores=cores)
+
+
+def run_reference(args) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_sample(0.0, min_calls=1)
+    res = [oracle_sample(0.0, min_calls=1) for _ in range(args.steps)]
+    el = sum(r["seconds"] for r in res)
+    calls = sum(r["calls"] for r in res)
+    b = layer_bytes("bitnet", 4096, 4096)["total"]
+    val = calls * b / el / 1e9
+    cores = res[0]["cores"]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64+f64",
+        "data": "synthetic",
+        "config": {"workload": "BitNet W1A8 decode GEMV, Llama-7B shapes, M=1 (CPU oracle sample: one "
+                               "4096x4096 layer call per step)", "seq_len": 1, "global_batch": 1},
+        "us_per_layer": el / calls * 1e6,
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{calls} BitNet W1A8 4096x4096 layer calls (act quant + layer), numpy"},
+        "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# CUDA arm
+# ---------------------------------------------------------------------------
+def build_stack(layers: int, seed: int, device):
+    import torch
+    from bit_weight_quantization_b200 import bq
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    stack = []
+    for l in range(layers):
+        for name, N, K in LLAMA7B:
+            W = torch.randn(N, K, device=device, generator=gen, dtype=torch.float32) * 0.02
+            ql = bq.QuantLinear("bitnet", W)
+            del W
+            x = torch.randn(1, K, device=device, generator=gen).to(torch.bfloat16)
+            y = torch.empty(1, N, device=device, dtype=torch.float32)
+            act = ql.act_buffer(1)
+            stack.append(dict(name=name, N=N, K=K, ql=ql, x=x, y=y, act=act))
+    torch.cuda.synchronize()
+    return stack
+
+
+def step_calls(stack, timing=None):
+    from bit_weight_quantization_b200 import bq
+    for i, L in enumerate(stack):
+        ql = L["ql"]
+        bq.bq_quantize_act(ql.layer, L["x"], 1, L["act"], L["act"].numel())
+        if timing is not None:
+            timing[i][0].record()
+        bq.bq_gemv(ql.layer, L["act"], L["y"])
+        if timing is not None:
+            timing[i][1].record()
+
+
+def run_cuda(args) -> None:
+    import torch
+    import torch.distributed as dist
+    from bit_weight_quantization_b200 import bq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    stack = build_stack(args.layers, args.seed + rank, dev)
+    per_step = sum(layer_bytes("bitnet", L["N"], L["K"])["total"] for L in stack)
+    gemv_bytes = sum(layer_bytes("bitnet", L["N"], L["K"])["gemv"] for L in stack)
+    n_layers = len(stack)
+    stream = torch.cuda.Stream(device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    with torch.cuda.stream(stream):
+        step_calls(stack)                      # eager warm-up, also loads the module
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step_calls(stack)
+        torch.cuda.synchronize()
+        bq.bq_device_check()
+
+        clocks = ClockSampler(local)
+        for _ in range(args.warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        clk = clocks.stop()
+        ms = e0.elapsed_time(e1)
+
+        # per-launch time of the GEMV kernel (the dominant one): a second capture of the
+        # same step with events around every bq_gemv, replayed as many times
+        timing = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in stack]
+        gi = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gi, stream=stream):
+            step_calls(stack, timing)
+        torch.cuda.synchronize()
+        gemv_ms = []
+        for _ in range(max(3, min(args.steps, 50))):
+            gi.replay()
+            torch.cuda.synchronize()
+            gemv_ms.append(sum(a.elapsed_time(b) for a, b in timing))
+        gemv_ms_step = statistics.median(gemv_ms)
+
+        # end to end through the public API: pinned host x -> device, the 224 calls, y -> host
+        xs_h = torch.cat([L["x"].view(-1) for L in stack]).cpu().pin_memory()
+        xs_d = torch.empty_like(xs_h, device=dev)
+        ys_h = torch.empty(sum(L["N"] for L in stack), dtype=torch.float32).pin_memory()
+        ys_d = torch.empty(ys_h.numel(), dtype=torch.float32, device=dev)
+        offs, o = [], 0
+        for L in stack:
+            offs.append(o)
+            o += L["K"]
+        yoffs, o = [], 0
+        for L in stack:
+            yoffs.append(o)
+            o += L["N"]
+
+        def e2e_step():
+            xs_d.copy_(xs_h, non_blocking=True)
+            for i, L in enumerate(stack):
+                ql = L["ql"]
+                x = xs_d[offs[i]:offs[i] + L["K"]].view(1, -1)
+                bq.bq_quantize_act(ql.layer, x, 1, L["act"], L["act"].numel())
+                bq.bq_gemv(ql.layer, L["act"], ys_d[yoffs[i]:yoffs[i] + L["N"]])
+            ys_h.copy_(ys_d, non_blocking=True)
+
+        for _ in range(max(1, min(args.warmup, 3))):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        n_e2e = max(1, min(args.steps, 50))
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = t0.elapsed_time(t1) / n_e2e
+        bq.bq_device_check()
+
+    ms_t = torch.tensor([ms, e2e_ms], device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms, e2e_ms = float(ms_t[0]), float(ms_t[1])
+    ms_step = ms / args.steps
+    value = world * per_step * args.steps / (ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    gemv_achieved = gemv_bytes / (gemv_ms_step * 1e-3) / 1e9
+    traffic = profile_traffic("bitnet_gemv_4096x4096")
+    out = None
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": "BitNet W1A8 decode GEMV, M=1: 32-layer Llama-7B linear stack "
+                                   "(q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008), "
+                                   "bq_quantize_act + bq_gemv per layer, CUDA graph per step",
+                       "layers_per_step": n_layers, "seq_len": 1, "global_batch": world,
+                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": "inputs larger than L2 (each step streams %.0f MB of distinct packed weights)"
+                             % (per_step / 1e6)},
+            "us_per_layer": ms_step * 1e3 / n_layers,
+            "frac_of_peak": value / world / peak, "frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
+            "roofline": {"bound": "hbm", "achieved": gemv_achieved, "peak": peak, "unit": "GB/s",
+                         "frac": gemv_achieved / peak, "traffic": traffic, "peak_source": peak_kind,
+                         "kernel": "k_gemv_mma<BitNet W1A8> (bq_gemv)",
+                         "us_per_launch": gemv_ms_step * 1e3 / n_layers},
+            "e2e": {"value": per_step / (e2e_ms * 1e-3) / 1e9 * world, "unit": "GB/s",
+                    "h2d_bytes_per_step": int(xs_h.numel() * 2), "d2h_bytes_per_step": int(ys_h.numel() * 4),
+                    "ms_per_step": e2e_ms, "path": "eager Python calls of the C ABI, pinned host buffers"},
+            "gpu_launches": 2 * n_layers * args.steps,
+            "clocks": clk,
+        }
+    if world > 1:
+        del g, gi
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1:
+            cb = oracle_sample(args.cpu_seconds)
+            out["cpu_baseline"] = {"value": cb["gbs"], "unit": "GB/s", "cores": cb["cores"], "kind": "oracle",
+                                   "sample": f"{cb['calls']} BitNet W1A8 4096x4096 layer calls "
+                                             f"(act quant + layer), {cb['seconds']:.1f} s"}
+        print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_cuda(args)
+
+
+if __name__ == "__main__":
+    main()

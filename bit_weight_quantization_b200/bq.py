@@ -1,0 +1,190 @@
+"""Thin ctypes binding of the C ABI in ``libbq.so`` (declared in include/bq.h).
+
+Argument marshalling only: every computation runs in the library's CUDA
+kernels. Torch tensors may be passed wherever the C call takes a device
+pointer (their ``data_ptr()`` is used); the stream defaults to torch's current
+CUDA stream. If the shared library is missing this module raises at import.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbq.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libbq.so not built at {LIB_PATH}; run bit_weight_quantization_b200.build.build()")
+_lib = ctypes.CDLL(LIB_PATH)
+
+BQ_OK, BQ_ERR_INVALID_ARG, BQ_ERR_UNSUPPORTED, BQ_ERR_SIZE = 0, 1, 2, 3
+BQ_ERR_CUDA, BQ_ERR_BAD_PACKED, BQ_ERR_DEVICE_CHECK = 4, 5, 6
+BQ_FMT_RABIT2, BQ_FMT_BITNET_W1A8, BQ_FMT_TERNARY_A8, BQ_FMT_ABQ, BQ_FMT_BVSR4 = 1, 2, 3, 4, 5
+FORMATS = {"rabit": 1, "bitnet": 2, "ternary": 3, "abq": 4, "bvsr": 5}
+
+
+class bq_pack_desc(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("w_bits", ctypes.c_int32), ("a_bits", ctypes.c_int32),
+                ("lora_rank", ctypes.c_int32), ("lora_alpha", ctypes.c_float), ("h2", ctypes.c_void_p),
+                ("lora_A", ctypes.c_void_p), ("lora_B", ctypes.c_void_p)]
+
+
+class bq_layer(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("N", ctypes.c_int32), ("K", ctypes.c_int32),
+                ("N_pad", ctypes.c_int32), ("K_pad", ctypes.c_int32), ("w_bits", ctypes.c_int32),
+                ("a_bits", ctypes.c_int32), ("lora_rank", ctypes.c_int32),
+                ("packed_bytes", ctypes.c_uint64), ("packed", ctypes.c_void_p)]
+
+
+_P = ctypes.c_void_p
+_SIGS = {
+    "bq_status_str": (ctypes.c_char_p, [ctypes.c_int]),
+    "bq_version": (ctypes.c_int32, []),
+    "bq_packed_bytes": (ctypes.c_int, [ctypes.POINTER(bq_pack_desc), ctypes.c_int32, ctypes.c_int32,
+                                       ctypes.POINTER(ctypes.c_size_t)]),
+    "bq_pack_weights": (ctypes.c_int, [ctypes.POINTER(bq_pack_desc), _P, ctypes.c_int32, ctypes.c_int32, _P,
+                                       ctypes.c_size_t, _P, ctypes.POINTER(bq_layer)]),
+    "bq_packed_validate": (ctypes.c_int, [_P, ctypes.c_size_t, _P, ctypes.POINTER(bq_layer)]),
+    "bq_act_bytes": (ctypes.c_int, [ctypes.POINTER(bq_layer), ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]),
+    "bq_quantize_act": (ctypes.c_int, [ctypes.POINTER(bq_layer), _P, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
+    "bq_gemv": (ctypes.c_int, [ctypes.POINTER(bq_layer), _P, _P, _P, _P]),
+    "bq_gemm": (ctypes.c_int, [ctypes.POINTER(bq_layer), _P, ctypes.c_int32, _P, _P, _P]),
+    "bq_device_check": (ctypes.c_int, []),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype, _f.argtypes = _res, _args
+
+EXPORTED = tuple(_SIGS)
+
+
+class BQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {bq_status_str(status)} (status {status})")
+
+
+def _ptr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return int(x.data_ptr())
+
+
+def _stream(stream):
+    if stream is not None:
+        return stream if isinstance(stream, int) else int(stream.cuda_stream)
+    import torch
+    return int(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(st: int, where: str):
+    if st != BQ_OK:
+        raise BQError(st, where)
+
+
+def bq_status_str(status: int) -> str:
+    return _lib.bq_status_str(status).decode()
+
+
+def bq_version() -> int:
+    return _lib.bq_version()
+
+
+def make_desc(fmt, w_bits=0, a_bits=0, lora_rank=0, lora_alpha=0.1, h2=None, lora_A=None, lora_B=None):
+    return bq_pack_desc(FORMATS.get(fmt, fmt), w_bits, a_bits, lora_rank, lora_alpha,
+                        _ptr(h2), _ptr(lora_A), _ptr(lora_B))
+
+
+def bq_packed_bytes(desc: bq_pack_desc, N: int, K: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(_lib.bq_packed_bytes(ctypes.byref(desc), N, K, ctypes.byref(out)), "bq_packed_bytes")
+    return out.value
+
+
+def bq_pack_weights(desc: bq_pack_desc, W, N: int, K: int, packed, packed_bytes: int, stream=None) -> bq_layer:
+    layer = bq_layer()
+    _check(_lib.bq_pack_weights(ctypes.byref(desc), _ptr(W), N, K, _ptr(packed), packed_bytes,
+                                _stream(stream), ctypes.byref(layer)), "bq_pack_weights")
+    return layer
+
+
+def bq_packed_validate(packed_host: bytes, packed_dev) -> bq_layer:
+    layer = bq_layer()
+    buf = ctypes.create_string_buffer(bytes(packed_host), len(packed_host))
+    _check(_lib.bq_packed_validate(buf, len(packed_host), _ptr(packed_dev), ctypes.byref(layer)),
+           "bq_packed_validate")
+    return layer
+
+
+def bq_act_bytes(layer: bq_layer, M: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(_lib.bq_act_bytes(ctypes.byref(layer), M, ctypes.byref(out)), "bq_act_bytes")
+    return out.value
+
+
+def bq_quantize_act(layer: bq_layer, x_bf16, M: int, act, act_bytes: int, stream=None) -> None:
+    _check(_lib.bq_quantize_act(ctypes.byref(layer), _ptr(x_bf16), M, _ptr(act), act_bytes, _stream(stream)),
+           "bq_quantize_act")
+
+
+def bq_gemv(layer: bq_layer, act, y, acc_dbg=None, stream=None) -> None:
+    _check(_lib.bq_gemv(ctypes.byref(layer), _ptr(act), _ptr(y), _ptr(acc_dbg), _stream(stream)), "bq_gemv")
+
+
+def bq_gemm(layer: bq_layer, act, M: int, y, acc_dbg=None, stream=None) -> None:
+    _check(_lib.bq_gemm(ctypes.byref(layer), _ptr(act), M, _ptr(y), _ptr(acc_dbg), _stream(stream)), "bq_gemm")
+
+
+def bq_device_check() -> None:
+    _check(_lib.bq_device_check(), "bq_device_check")
+
+
+def raw_status(name: str, *args) -> int:
+    """Call an ABI function and return its status code without raising (for fault tests)."""
+    return getattr(_lib, name)(*args)
+
+
+class QuantLinear:
+    """Device buffers (torch allocations) for one packed layer plus the calls on them.
+
+    Owns: the packed buffer. Per call: an activation buffer for M tokens and y.
+    All arithmetic happens in the library."""
+
+    def __init__(self, fmt, W, *, w_bits=0, a_bits=0, lora_rank=0, lora_alpha=0.1, h2=None,
+                 lora_A=None, lora_B=None, stream=None):
+        import torch
+        N, K = W.shape
+        self.desc = make_desc(fmt, w_bits, a_bits, lora_rank, lora_alpha, h2, lora_A, lora_B)
+        self._keep = (W, h2, lora_A, lora_B)
+        nbytes = bq_packed_bytes(self.desc, N, K)
+        self.packed = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+        self.layer = bq_pack_weights(self.desc, W, N, K, self.packed, nbytes, stream)
+        self.N, self.K = N, K
+        self._acts = {}
+
+    def act_buffer(self, M):
+        import torch
+        if M not in self._acts:
+            n = bq_act_bytes(self.layer, M)
+            self._acts[M] = torch.empty(n, dtype=torch.uint8, device=self.packed.device)
+        return self._acts[M]
+
+    def quantize_act(self, x_bf16, stream=None):
+        M = x_bf16.shape[0]
+        act = self.act_buffer(M)
+        bq_quantize_act(self.layer, x_bf16, M, act, act.numel(), stream)
+        return act
+
+    def forward(self, x_bf16, y=None, acc_dbg=None, stream=None):
+        import torch
+        M = x_bf16.shape[0]
+        act = self.quantize_act(x_bf16, stream)
+        if y is None:
+            y = torch.empty((M, self.N), dtype=torch.float32, device=x_bf16.device)
+        if M == 1:
+            bq_gemv(self.layer, act, y, acc_dbg, stream)
+        else:
+            bq_gemm(self.layer, act, M, y, acc_dbg, stream)
+        return y

@@ -1,0 +1,370 @@
+// C ABI: host-side validation, buffer layouts and kernel launches.
+#pragma once
+
+#include <algorithm>
+#include <cstring>
+
+#include "bq_act.cuh"
+#include "bq_gemv.cuh"
+#include "bq_internal.cuh"
+#include "bq_pack.cuh"
+
+namespace bqi {
+
+inline bool aligned(const void* p, size_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+
+inline bq_status check_nk(int N, int K) {
+  if (N < 1 || N > BQ_MAX_N || K < 128 || K > BQ_MAX_K || K % 128 != 0) return BQ_ERR_SIZE;
+  return BQ_OK;
+}
+
+// need_ptrs: the pack call reads the device pointers; the size query does not.
+inline bq_status check_desc(const bq_pack_desc* d, int K, bool need_ptrs) {
+  if (!d) return BQ_ERR_INVALID_ARG;
+  switch (d->fmt) {
+    case BQ_FMT_RABIT2:
+      if (need_ptrs && (!d->h2 || !aligned(d->h2, 4))) return BQ_ERR_INVALID_ARG;
+      return BQ_OK;
+    case BQ_FMT_BITNET_W1A8:
+      return BQ_OK;
+    case BQ_FMT_TERNARY_A8:
+      if (d->lora_rank < 0 || d->lora_rank > BQ_MAX_LORA_RANK) return BQ_ERR_INVALID_ARG;
+      if (need_ptrs && d->lora_rank > 0 && (!d->lora_A || !d->lora_B)) return BQ_ERR_INVALID_ARG;
+      if (!(d->lora_alpha == d->lora_alpha)) return BQ_ERR_INVALID_ARG;
+      return BQ_OK;
+    case BQ_FMT_ABQ: {
+      if (d->w_bits < 1 || d->w_bits > 8 || d->a_bits < 1 || d->a_bits > 8) return BQ_ERR_INVALID_ARG;
+      const long long bound = ((1ll << d->w_bits) - 1) * ((1ll << d->a_bits) - 1) * (long long)K;
+      if (bound >= (1ll << 31)) return BQ_ERR_SIZE;
+      return BQ_OK;
+    }
+    case BQ_FMT_BVSR4:
+      return BQ_OK;
+    default:
+      return BQ_ERR_INVALID_ARG;
+  }
+}
+
+inline bool desc_layout(const bq_pack_desc* d, int N, int K, PkLayout* L) {
+  const int rank = d->fmt == BQ_FMT_TERNARY_A8 ? d->lora_rank : 0;
+  return make_pk_layout(d->fmt, N, K, d->w_bits, d->a_bits, rank, d->lora_alpha, L);
+}
+
+inline HeaderWords header_words(const PkLayout& L) {
+  HeaderWords h{};
+  h.w[HW_MAGIC] = kPkMagic;
+  h.w[HW_VERSION] = kVersion;
+  h.w[HW_FMT] = L.fmt;
+  h.w[HW_N] = L.N;
+  h.w[HW_K] = L.K;
+  h.w[HW_NPAD] = L.N_pad;
+  h.w[HW_KPAD] = L.K_pad;
+  h.w[HW_WBITS] = L.w_bits;
+  h.w[HW_ABITS] = L.a_bits;
+  h.w[HW_NSTREAMS] = L.nstreams;
+  for (int s = 0; s < 4; s++) {
+    h.w[HW_FIELD + s] = s < L.nstreams ? L.field[s] : 0;
+    h.w[HW_SHIFT + s] = s < L.nstreams ? L.shift[s] : 0;
+  }
+  h.w[HW_TILEBYTES] = L.tile_bytes;
+  h.w[HW_LORA_RANK] = L.rank;
+  std::memcpy(&h.w[HW_LORA_ALPHA], &L.lora_alpha, 4);
+  h.w[HW_TSCALE] = 0;
+  const uint64_t q[5] = {L.total, L.off_tiles, L.off_rows, L.off_aux, L.off_aux2};
+  const int at[5] = {HW_TOTAL, HW_OFF_TILES, HW_OFF_ROWS, HW_OFF_AUX, HW_OFF_AUX2};
+  for (int i = 0; i < 5; i++) {
+    h.w[at[i]] = uint32_t(q[i]);
+    h.w[at[i] + 1] = uint32_t(q[i] >> 32);
+  }
+  return h;
+}
+
+inline bq_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+inline unsigned blocks_for(uint64_t n, unsigned threads) { return unsigned((n + threads - 1) / threads); }
+
+inline bq_status check_layer(const bq_layer* y, PkLayout* L) {
+  if (!y || !y->packed || !aligned(y->packed, 256)) return BQ_ERR_INVALID_ARG;
+  if (check_nk(y->N, y->K) != BQ_OK) return BQ_ERR_SIZE;
+  if (!layout_from_layer(y, L)) return BQ_ERR_INVALID_ARG;
+  if (L->N_pad != y->N_pad || L->K_pad != y->K_pad || L->total > y->packed_bytes) return BQ_ERR_BAD_PACKED;
+  return BQ_OK;
+}
+
+}  // namespace bqi
+
+using namespace bqi;
+
+extern "C" {
+
+const char* bq_status_str(bq_status s) {
+  switch (s) {
+    case BQ_OK: return "ok";
+    case BQ_ERR_INVALID_ARG: return "invalid argument";
+    case BQ_ERR_UNSUPPORTED: return "unsupported";
+    case BQ_ERR_SIZE: return "size out of range or buffer too small";
+    case BQ_ERR_CUDA: return "CUDA error";
+    case BQ_ERR_BAD_PACKED: return "bad packed buffer";
+    case BQ_ERR_DEVICE_CHECK: return "device-side check failed";
+    default: return "unknown status";
+  }
+}
+
+int32_t bq_version(void) { return 1; }
+
+bq_status bq_packed_bytes(const bq_pack_desc* desc, int32_t N, int32_t K, size_t* bytes) {
+  if (!bytes) return BQ_ERR_INVALID_ARG;
+  bq_status st = check_nk(N, K);
+  if (st != BQ_OK) return st;
+  if ((st = check_desc(desc, K, false)) != BQ_OK) return st;
+  PkLayout L;
+  if (!desc_layout(desc, N, K, &L)) return BQ_ERR_INVALID_ARG;
+  *bytes = size_t(L.total);
+  return BQ_OK;
+}
+
+bq_status bq_pack_weights(const bq_pack_desc* desc, const float* W, int32_t N, int32_t K, void* packed,
+                          size_t packed_bytes, void* stream, bq_layer* layer) {
+  bq_status st = check_nk(N, K);
+  if (st != BQ_OK) return st;
+  if ((st = check_desc(desc, K, true)) != BQ_OK) return st;
+  if (!W || !aligned(W, 16) || !packed || !aligned(packed, 256) || !layer) return BQ_ERR_INVALID_ARG;
+  PkLayout L;
+  if (!desc_layout(desc, N, K, &L)) return BQ_ERR_INVALID_ARG;
+  if (packed_bytes < L.total) return BQ_ERR_SIZE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* P = static_cast<uint8_t*>(packed);
+  uint32_t* hdr = reinterpret_cast<uint32_t*>(P);
+  if (cudaMemsetAsync(P, 0, L.total, s) != cudaSuccess) return BQ_ERR_CUDA;
+  k_write_header<<<1, 64, 0, s>>>(hdr, header_words(L));
+
+  FieldPackArgs fa{};
+  fa.W = W; fa.tiles = reinterpret_cast<uint32_t*>(P + L.off_tiles);
+  fa.N = N; fa.K = K; fa.KT = L.KT; fa.tile_words = L.tile_bytes / 4; fa.nstreams = L.nstreams;
+  int soff = 0;
+  for (int i = 0; i < 4; i++) {
+    fa.field[i] = L.field[i]; fa.shift[i] = L.shift[i]; fa.soff_words[i] = soff;
+    if (i < L.nstreams) soff += 128 * L.field[i];
+  }
+  fa.hdr = hdr; fa.w_bits = L.w_bits;
+  fa.total_words = uint64_t(L.RB) * L.KT * (L.tile_bytes / 4);
+
+  switch (L.fmt) {
+    case BQ_FMT_BITNET_W1A8:
+    case BQ_FMT_TERNARY_A8: {
+      double* rs = reinterpret_cast<double*>(P + L.off_tiles);   // scratch, overwritten below
+      k_row_abs_sum<<<N, 256, 0, s>>>(W, K, rs);
+      k_tensor_mean<<<1, 1024, 0, s>>>(rs, N, double(N) * double(K), hdr);
+      if (L.fmt == BQ_FMT_BITNET_W1A8)
+        k_pack_fields<BQ_FMT_BITNET_W1A8><<<blocks_for(fa.total_words, 256), 256, 0, s>>>(fa);
+      else
+        k_pack_fields<BQ_FMT_TERNARY_A8><<<blocks_for(fa.total_words, 256), 256, 0, s>>>(fa);
+      if (L.fmt == BQ_FMT_TERNARY_A8 && L.rank > 0) {
+        const uint64_t n = uint64_t(L.K_pad + L.N_pad) * L.rank;
+        k_lora_to_bf16<<<blocks_for(n, 256), 256, 0, s>>>(
+            desc->lora_A, desc->lora_B, N, K, L.N_pad, L.K_pad, L.rank, reinterpret_cast<uint16_t*>(P + L.off_aux),
+            reinterpret_cast<uint16_t*>(P + L.off_aux2));
+      }
+      break;
+    }
+    case BQ_FMT_ABQ: {
+      float* delta = reinterpret_cast<float*>(P + L.off_rows);
+      int* zero = reinterpret_cast<int*>(P + L.off_rows) + L.N_pad;
+      int* sumq = reinterpret_cast<int*>(P + L.off_rows) + 2 * L.N_pad;
+      k_abq_rows<<<N, 256, 0, s>>>(W, K, L.w_bits, delta, zero, sumq);
+      fa.abq_delta = delta; fa.abq_zero = zero;
+      k_pack_fields<BQ_FMT_ABQ><<<blocks_for(fa.total_words, 256), 256, 0, s>>>(fa);
+      break;
+    }
+    case BQ_FMT_RABIT2: {
+      k_rabit_pack<<<N, 256, 0, s>>>(W, L.N_pad, K, L.K_pad, reinterpret_cast<uint32_t*>(P + L.off_tiles),
+                                     reinterpret_cast<float*>(P + L.off_rows));
+      k_rabit_h<<<blocks_for(L.K_pad, 256), 256, 0, s>>>(desc->h2, K, L.K_pad, reinterpret_cast<float*>(P + L.off_aux),
+                                                         reinterpret_cast<float*>(P + L.off_aux2));
+      break;
+    }
+    case BQ_FMT_BVSR4: {
+      const uint64_t V = uint64_t(N) * (K / 32);
+      uint32_t* kmin = reinterpret_cast<uint32_t*>(P + L.off_tiles);   // scratch in the tile region
+      uint32_t* kmax = kmin + V;
+      uint32_t* counts = reinterpret_cast<uint32_t*>(P + L.off_aux);   // scratch in the table region
+      float* table = reinterpret_cast<float*>(P + L.off_aux);
+      k_bvsr_minmax<<<blocks_for(V, 256), 256, 0, s>>>(W, K, V, kmin, kmax);
+      const unsigned cb = unsigned(std::min<uint64_t>(blocks_for(V, 256), 148ull * 8));
+      for (int bit = 31; bit >= 0; bit--) k_bvsr_count<<<cb, 256, 0, s>>>(kmin, kmax, V, counts, bit);
+      k_bvsr_table<<<1, 256, 0, s>>>(counts, V, table);
+      if (cudaMemsetAsync(P + L.off_tiles, 0, L.off_rows - L.off_tiles, s) != cudaSuccess) return BQ_ERR_CUDA;
+      const unsigned sb = unsigned(std::min<uint64_t>(V, 148ull * 16));
+      k_bvsr_search<<<sb, 256, 0, s>>>(W, K, L.K_pad, L.KT, V, table, reinterpret_cast<uint32_t*>(P + L.off_tiles),
+                                       P + L.off_aux2);
+      break;
+    }
+    default:
+      return BQ_ERR_INVALID_ARG;
+  }
+  if ((st = launch_status()) != BQ_OK) return st;
+  layer->fmt = L.fmt; layer->N = N; layer->K = K; layer->N_pad = L.N_pad; layer->K_pad = L.K_pad;
+  layer->w_bits = L.w_bits; layer->a_bits = L.a_bits; layer->lora_rank = L.rank;
+  layer->packed_bytes = packed_bytes; layer->packed = packed;
+  return BQ_OK;
+}
+
+bq_status bq_packed_validate(const void* packed_host, size_t bytes, const void* packed_dev, bq_layer* layer) {
+  if (!packed_host || bytes < 256 || !layer || !packed_dev || !aligned(packed_dev, 256)) return BQ_ERR_INVALID_ARG;
+  uint32_t h[64];
+  std::memcpy(h, packed_host, 256);
+  if (h[HW_MAGIC] != kPkMagic || h[HW_VERSION] != kVersion) return BQ_ERR_BAD_PACKED;
+  const int fmt = int(h[HW_FMT]), N = int(h[HW_N]), K = int(h[HW_K]);
+  if (check_nk(N, K) != BQ_OK) return BQ_ERR_BAD_PACKED;
+  const int rank = int(h[HW_LORA_RANK]);
+  if (rank < 0 || rank > BQ_MAX_LORA_RANK) return BQ_ERR_BAD_PACKED;
+  float alpha;
+  std::memcpy(&alpha, &h[HW_LORA_ALPHA], 4);
+  PkLayout L;
+  if (!make_pk_layout(fmt, N, K, int(h[HW_WBITS]), int(h[HW_ABITS]), rank, alpha, &L)) return BQ_ERR_BAD_PACKED;
+  const uint64_t total = uint64_t(h[HW_TOTAL]) | (uint64_t(h[HW_TOTAL + 1]) << 32);
+  const uint64_t offs[4] = {L.off_tiles, L.off_rows, L.off_aux, L.off_aux2};
+  const int at[4] = {HW_OFF_TILES, HW_OFF_ROWS, HW_OFF_AUX, HW_OFF_AUX2};
+  for (int i = 0; i < 4; i++)
+    if ((uint64_t(h[at[i]]) | (uint64_t(h[at[i] + 1]) << 32)) != offs[i]) return BQ_ERR_BAD_PACKED;
+  if (total != L.total || int(h[HW_NPAD]) != L.N_pad || int(h[HW_KPAD]) != L.K_pad ||
+      int(h[HW_TILEBYTES]) != L.tile_bytes || int(h[HW_NSTREAMS]) != L.nstreams)
+    return BQ_ERR_BAD_PACKED;
+  if (fmt == BQ_FMT_ABQ) {
+    const long long bound = ((1ll << L.w_bits) - 1) * ((1ll << L.a_bits) - 1) * (long long)K;
+    if (bound >= (1ll << 31)) return BQ_ERR_BAD_PACKED;
+  }
+  layer->fmt = fmt; layer->N = N; layer->K = K; layer->N_pad = L.N_pad; layer->K_pad = L.K_pad;
+  layer->w_bits = L.w_bits; layer->a_bits = L.a_bits; layer->lora_rank = L.rank;
+  layer->packed_bytes = total; layer->packed = packed_dev;
+  return BQ_OK;
+}
+
+bq_status bq_act_bytes(const bq_layer* layer, int32_t M, size_t* bytes) {
+  PkLayout L;
+  bq_status st = check_layer(layer, &L);
+  if (st != BQ_OK) return st;
+  if (!bytes) return BQ_ERR_INVALID_ARG;
+  if (M < 0 || M > BQ_MAX_M) return BQ_ERR_SIZE;
+  *bytes = size_t(make_act_layout(L, M).total);
+  return BQ_OK;
+}
+
+bq_status bq_quantize_act(const bq_layer* layer, const void* x_bf16, int32_t M, void* act, size_t act_bytes,
+                          void* stream) {
+  PkLayout L;
+  bq_status st = check_layer(layer, &L);
+  if (st != BQ_OK) return st;
+  if (M < 0 || M > BQ_MAX_M) return BQ_ERR_SIZE;
+  if (M == 0) return BQ_OK;
+  if (!x_bf16 || !aligned(x_bf16, 16) || !act || !aligned(act, 256)) return BQ_ERR_INVALID_ARG;
+  const ActLayout A = make_act_layout(L, M);
+  if (act_bytes < A.total) return BQ_ERR_SIZE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint8_t* P = static_cast<const uint8_t*>(layer->packed);
+  ActArgs a{};
+  a.x = static_cast<const uint16_t*>(x_bf16);
+  a.act = static_cast<uint8_t*>(act);
+  a.M = M; a.K = L.K; a.K_pad = L.K_pad; a.KT = L.KT; a.a_bits = L.a_bits; a.rank = A.rank; a.fmt = L.fmt;
+  a.off_codes = A.off_codes; a.off_tok = A.off_tok; a.off_gsum = A.off_gsum; a.off_u = A.off_u; a.off_xt = A.off_xt;
+  a.total = A.total;
+  a.lora_A = reinterpret_cast<const uint16_t*>(P + L.off_aux);
+  a.h1 = reinterpret_cast<const float*>(P + L.off_aux);
+  a.h2 = reinterpret_cast<const float*>(P + L.off_aux2);
+  if (L.fmt == BQ_FMT_RABIT2) {
+    k_act_rabit<<<dim3(blocks_for(L.K_pad, 256), M), 256, 0, s>>>(a);
+    return launch_status();
+  }
+  const int slices_target = std::max(1, std::min(L.KT, (148 + M - 1) / M));
+  a.tiles_per_slice = (L.KT + slices_target - 1) / slices_target;
+  const int slices = (L.KT + a.tiles_per_slice - 1) / a.tiles_per_slice;
+  const dim3 grid(slices, M);
+  switch (L.fmt) {
+    case BQ_FMT_BITNET_W1A8: k_act_quant<BQ_FMT_BITNET_W1A8><<<grid, 256, 0, s>>>(a); break;
+    case BQ_FMT_TERNARY_A8: k_act_quant<BQ_FMT_TERNARY_A8><<<grid, 256, 0, s>>>(a); break;
+    case BQ_FMT_ABQ: k_act_quant<BQ_FMT_ABQ><<<grid, 256, 0, s>>>(a); break;
+    case BQ_FMT_BVSR4: k_act_quant<BQ_FMT_BVSR4><<<grid, 256, 0, s>>>(a); break;
+    default: return BQ_ERR_INVALID_ARG;
+  }
+  return launch_status();
+}
+
+bq_status bq_gemm(const bq_layer* layer, const void* act, int32_t M, float* y, int64_t* acc_dbg, void* stream) {
+  PkLayout L;
+  bq_status st = check_layer(layer, &L);
+  if (st != BQ_OK) return st;
+  if (M < 0 || M > BQ_MAX_M) return BQ_ERR_SIZE;
+  if (M == 0) return BQ_OK;
+  if (!act || !aligned(act, 256) || !y || !aligned(y, 4) || (acc_dbg && !aligned(acc_dbg, 8)))
+    return BQ_ERR_INVALID_ARG;
+  if (L.fmt == BQ_FMT_RABIT2 && acc_dbg) return BQ_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint8_t* P = static_cast<const uint8_t*>(layer->packed);
+  const uint8_t* Ab = static_cast<const uint8_t*>(act);
+  const ActLayout A = make_act_layout(L, M);
+  GemvArgs g{};
+  g.tiles = P + L.off_tiles;
+  g.pk_hdr = reinterpret_cast<const uint32_t*>(P);
+  g.row_delta = reinterpret_cast<const float*>(P + L.off_rows);
+  g.row_zero = reinterpret_cast<const int*>(P + L.off_rows) + L.N_pad;
+  g.row_sum = reinterpret_cast<const int*>(P + L.off_rows) + 2 * L.N_pad;
+  g.lora_bt = reinterpret_cast<const uint16_t*>(P + L.off_aux2);
+  g.bvsr_table = reinterpret_cast<const float*>(P + L.off_aux);
+  g.bvsr_idx = P + L.off_aux2;
+  g.rabit_planes = reinterpret_cast<const uint32_t*>(P + L.off_tiles);
+  g.rabit_g = reinterpret_cast<const float*>(P + L.off_rows);
+  g.act_hdr = reinterpret_cast<const uint32_t*>(Ab);
+  g.act_codes = Ab + A.off_codes;
+  g.act_tok = reinterpret_cast<const uint32_t*>(Ab + A.off_tok);
+  g.act_u = reinterpret_cast<const float*>(Ab + A.off_u);
+  g.act_gsum = reinterpret_cast<const int*>(Ab + A.off_gsum);
+  g.act_xt = reinterpret_cast<const float*>(Ab + A.off_xt);
+  g.y = y;
+  g.acc = reinterpret_cast<long long*>(acc_dbg);
+  g.N = L.N; g.K = L.K; g.N_pad = L.N_pad; g.K_pad = L.K_pad; g.KT = L.KT; g.M = M;
+  g.tile_bytes = L.tile_bytes; g.rank = L.fmt == BQ_FMT_TERNARY_A8 ? L.rank : 0; g.fmt = L.fmt;
+  g.shift0 = L.shift[0]; g.shift1 = L.shift[1]; g.shift2 = L.shift[2];
+  const dim3 grid(L.RB, (M + 7) / 8);
+  constexpr int NW = 4;
+  switch (L.fmt) {
+    case BQ_FMT_BITNET_W1A8: k_gemv_mma<BQ_FMT_BITNET_W1A8, 1, 0, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
+    case BQ_FMT_TERNARY_A8: k_gemv_mma<BQ_FMT_TERNARY_A8, 2, 0, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
+    case BQ_FMT_ABQ:
+      switch (L.w_bits) {
+        case 1: k_gemv_mma<BQ_FMT_ABQ, 1, 0, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
+        case 2: k_gemv_mma<BQ_FMT_ABQ, 2, 0, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
+        case 3: k_gemv_mma<BQ_FMT_ABQ, 2, 1, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
+        case 4: k_gemv_mma<BQ_FMT_ABQ, 4, 0, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
+        case 5: k_gemv_mma<BQ_FMT_ABQ, 4, 1, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
+        case 6: k_gemv_mma<BQ_FMT_ABQ, 4, 2, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
+        case 7: k_gemv_mma<BQ_FMT_ABQ, 4, 2, 1, NW><<<grid, NW * 32, 0, s>>>(g); break;
+        case 8: k_gemv_mma<BQ_FMT_ABQ, 8, 0, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
+        default: return BQ_ERR_INVALID_ARG;
+      }
+      break;
+    case BQ_FMT_BVSR4: k_gemv_bvsr<NW><<<grid, NW * 32, 0, s>>>(g); break;
+    case BQ_FMT_RABIT2: k_gemv_rabit<8><<<blocks_for(L.N, 8), 256, 0, s>>>(g); break;
+    default: return BQ_ERR_INVALID_ARG;
+  }
+  return launch_status();
+}
+
+bq_status bq_gemv(const bq_layer* layer, const void* act, float* y, int64_t* acc_dbg, void* stream) {
+  return bq_gemm(layer, act, 1, y, acc_dbg, stream);
+}
+
+bq_status bq_device_check(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return BQ_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_bq_device_error, sizeof(v)) != cudaSuccess) return BQ_ERR_CUDA;
+  if (v) {
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(g_bq_device_error, &z, sizeof(z)) != cudaSuccess) return BQ_ERR_CUDA;
+    return BQ_ERR_DEVICE_CHECK;
+  }
+  return BQ_OK;
+}
+
+}  // extern "C"

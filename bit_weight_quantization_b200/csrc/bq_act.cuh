@@ -1,0 +1,203 @@
+// Online activation quantization (one call per layer input).
+//
+// Grid (slices, M): every block re-reduces its token's whole row (max|x| or
+// min/max) from L2, which is cheap next to a cross-block exchange, then codes
+// its own slice of k-tiles into the B-operand fragment order. Block slice 0
+// also writes the per-token parameters, the sums and the LoRA input u.
+#pragma once
+
+#include "bq_internal.cuh"
+
+namespace bqi {
+
+struct ActArgs {
+  const uint16_t* x;        // bf16 [M][K]
+  uint8_t* act;             // act buffer base
+  int M, K, K_pad, KT, a_bits, rank, fmt, tiles_per_slice;
+  uint64_t off_codes, off_tok, off_gsum, off_u, off_xt, total;
+  const uint16_t* lora_A;   // ternary: bf16 [K_pad][r]
+  const float* h1;          // RaBiT: [K_pad]
+  const float* h2;
+};
+
+__device__ __forceinline__ void act_write_header(const ActArgs& a) {
+  uint32_t* h = reinterpret_cast<uint32_t*>(a.act);
+  for (int i = threadIdx.x; i < 64; i += blockDim.x) {
+    uint32_t v = 0;
+    switch (i) {
+      case AW_MAGIC: v = kActMagic; break;
+      case AW_VERSION: v = kVersion; break;
+      case AW_FMT: v = uint32_t(a.fmt); break;
+      case AW_M: v = uint32_t(a.M); break;
+      case AW_K: v = uint32_t(a.K); break;
+      case AW_KPAD: v = uint32_t(a.K_pad); break;
+      case AW_ABITS: v = uint32_t(a.a_bits); break;
+      case AW_LORA_RANK: v = uint32_t(a.rank); break;
+      case AW_TOTAL: v = uint32_t(a.total); break;
+      case AW_TOTAL + 1: v = uint32_t(a.total >> 32); break;
+      case AW_OFF_CODES: v = uint32_t(a.off_codes); break;
+      case AW_OFF_CODES + 1: v = uint32_t(a.off_codes >> 32); break;
+      case AW_OFF_TOK: v = uint32_t(a.off_tok); break;
+      case AW_OFF_TOK + 1: v = uint32_t(a.off_tok >> 32); break;
+      case AW_OFF_GSUM: v = uint32_t(a.off_gsum); break;
+      case AW_OFF_GSUM + 1: v = uint32_t(a.off_gsum >> 32); break;
+      case AW_OFF_U: v = uint32_t(a.off_u); break;
+      case AW_OFF_U + 1: v = uint32_t(a.off_u >> 32); break;
+      case AW_OFF_XT: v = uint32_t(a.off_xt); break;
+      case AW_OFF_XT + 1: v = uint32_t(a.off_xt >> 32); break;
+      default: break;
+    }
+    h[i] = v;
+  }
+}
+
+// position (in 32-bit words) of the 4 codes k = 4q .. 4q+3 inside a token's k-tile:
+// k_in = 32mu + 16h + 4t + b  ->  word 16t + 2mu + h
+__device__ __forceinline__ int code_word_in_tile(int kin) {
+  const int mu = kin >> 5, h = (kin >> 4) & 1, t = (kin >> 2) & 3;
+  return 16 * t + 2 * mu + h;
+}
+
+__device__ __forceinline__ void load4(const uint16_t* xr, int k, int K, float v[4]) {
+  if (k + 3 < K) {
+    const uint2 p = *reinterpret_cast<const uint2*>(xr + k);
+    v[0] = __uint_as_float(p.x << 16);
+    v[1] = __uint_as_float(p.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(p.y << 16);
+    v[3] = __uint_as_float(p.y & 0xFFFF0000u);
+  } else {
+    for (int b = 0; b < 4; b++) v[b] = k + b < K ? bf16_bits_to_float(xr[k + b]) : 0.f;
+  }
+}
+
+// absmax int8: gamma = max|x|, s = 127/gamma, q = clamp(rn(x*s), -127, 127); gamma = 0 -> q = 0
+__device__ __forceinline__ int q_a8(float x, float s) {
+  float q = rintf(__fmul_rn(x, s));
+  q = fminf(fmaxf(q, -127.f), 127.f);
+  return int(q);
+}
+// asymmetric a-bit: q = clamp(rn(x/Delta) + z, 0, 2^a - 1)
+__device__ __forceinline__ int q_asym(float x, float d, int z, int qmax) {
+  long long q = (long long)rintf(__fdiv_rn(x, d)) + z;
+  q = q < 0 ? 0 : q;
+  q = q > qmax ? qmax : q;
+  return int(q);
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(256) k_act_quant(ActArgs a) {
+  __shared__ float shf[32];
+  __shared__ int shi[32];
+  __shared__ float u_part[8][64];
+  const int m = blockIdx.y, slice = blockIdx.x;
+  const uint16_t* xr = a.x + size_t(m) * a.K;
+  if (slice == 0 && m == 0) act_write_header(a);
+
+  // --- per-token scale (whole row) ---
+  float scale = 0.f, delta = 0.f;
+  int zero = 0;
+  const int qmax = (1 << a.a_bits) - 1;
+  if (FMT == BQ_FMT_ABQ) {
+    float lo = INFINITY, hi = -INFINITY;
+    for (int k = threadIdx.x * 4; k < a.K; k += blockDim.x * 4) {
+      float v[4];
+      load4(xr, k, a.K, v);
+      for (int b = 0; b < 4; b++) if (k + b < a.K) { lo = fminf(lo, v[b]); hi = fmaxf(hi, v[b]); }
+    }
+    lo = block_min(lo, shf);
+    hi = block_max(hi, shf);
+    delta = __fdiv_rn(fmaxf(__fsub_rn(hi, lo), 1e-5f), float(qmax));
+    zero = int(rintf(__fdiv_rn(-lo, delta)));
+  } else {
+    float mx = 0.f;
+    for (int k = threadIdx.x * 4; k < a.K; k += blockDim.x * 4) {
+      float v[4];
+      load4(xr, k, a.K, v);
+      for (int b = 0; b < 4; b++) mx = fmaxf(mx, fabsf(v[b]));
+    }
+    mx = block_max(mx, shf);
+    scale = mx;                                            // gamma_x
+    delta = mx > 0.f ? __fdiv_rn(127.f, mx) : 0.f;         // s = 127/gamma
+  }
+
+  // --- codes for this slice of k-tiles ---
+  uint32_t* codes = reinterpret_cast<uint32_t*>(a.act + a.off_codes) + size_t(m) * a.KT * 64;
+  int* gsum = reinterpret_cast<int*>(a.act + a.off_gsum) + size_t(m) * (a.K_pad / 32);
+  const int kt0 = slice * a.tiles_per_slice;
+  const int kt1 = min(a.KT, kt0 + a.tiles_per_slice);
+  for (int q4 = kt0 * 64 + threadIdx.x; q4 < kt1 * 64; q4 += blockDim.x) {
+    const int k = q4 * 4;
+    float v[4];
+    load4(xr, k, a.K, v);
+    uint32_t word = 0;
+    int qs = 0;
+    for (int b = 0; b < 4; b++) {
+      int q = 0;
+      if (k + b < a.K) q = FMT == BQ_FMT_ABQ ? q_asym(v[b], delta, zero, qmax) : q_a8(v[b], delta);
+      qs += q;
+      word |= (uint32_t(q) & 0xFFu) << (8 * b);
+    }
+    const int kt = k >> 8;
+    codes[kt * 64 + code_word_in_tile(k & 255)] = word;
+    if (FMT == BQ_FMT_BVSR4) {
+      // 8 consecutive threads cover one 32-element vector (blockDim and 64 are multiples of 8)
+      qs += __shfl_xor_sync(0xffffffffu, qs, 1);
+      qs += __shfl_xor_sync(0xffffffffu, qs, 2);
+      qs += __shfl_xor_sync(0xffffffffu, qs, 4);
+      if ((q4 & 7) == 0) gsum[k >> 5] = qs;
+    }
+  }
+
+  if (slice != 0) return;
+  // --- per-token parameters: sum of codes over the whole row ---
+  int s = 0;
+  for (int k = threadIdx.x * 4; k < a.K; k += blockDim.x * 4) {
+    float v[4];
+    load4(xr, k, a.K, v);
+    for (int b = 0; b < 4; b++)
+      if (k + b < a.K) s += FMT == BQ_FMT_ABQ ? q_asym(v[b], delta, zero, qmax) : q_a8(v[b], delta);
+  }
+  s = block_sum(s, shi);
+  uint32_t* tok = reinterpret_cast<uint32_t*>(a.act + a.off_tok) + 4 * m;
+  if (threadIdx.x == 0) {
+    if (FMT == BQ_FMT_ABQ) {
+      tok[0] = __float_as_uint(delta); tok[1] = uint32_t(zero); tok[2] = uint32_t(s); tok[3] = 0;
+    } else {
+      tok[0] = __float_as_uint(scale); tok[1] = uint32_t(s); tok[2] = 0; tok[3] = 0;
+    }
+  }
+  // --- ternary: u = SiLU(x A) from the unquantized x ---
+  if (FMT == BQ_FMT_TERNARY_A8 && a.rank > 0) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int r0 = 0; r0 < a.rank; r0 += 32) {
+      const int r = r0 + lane;
+      float acc = 0.f;
+      if (r < a.rank)
+        for (int k = warp; k < a.K; k += 8)
+          acc = fmaf(bf16_bits_to_float(xr[k]), bf16_bits_to_float(a.lora_A[size_t(k) * a.rank + r]), acc);
+      u_part[warp][lane] = acc;
+      __syncthreads();
+      if (warp == 0 && r < a.rank) {
+        float z = 0.f;
+        for (int w = 0; w < 8; w++) z += u_part[w][lane];
+        float* u = reinterpret_cast<float*>(a.act + a.off_u) + size_t(m) * a.rank;
+        u[r] = z / (1.f + expf(-z));
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// RaBiT: xt_p = h_p * x in float32, no quantization.
+__global__ void k_act_rabit(ActArgs a) {
+  const int m = blockIdx.y;
+  if (blockIdx.x == 0 && m == 0) act_write_header(a);
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= a.K_pad) return;
+  float* xt = reinterpret_cast<float*>(a.act + a.off_xt);
+  const float x = k < a.K ? bf16_bits_to_float(a.x[size_t(m) * a.K + k]) : 0.f;
+  xt[size_t(m) * a.K_pad + k] = k < a.K ? __fmul_rn(a.h1[k], x) : 0.f;
+  xt[(size_t(a.M) + m) * a.K_pad + k] = k < a.K ? __fmul_rn(a.h2[k], x) : 0.f;
+}
+
+}  // namespace bqi

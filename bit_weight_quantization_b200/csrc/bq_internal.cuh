@@ -1,0 +1,221 @@
+// Internal definitions shared by the pack, activation and GEMV kernels:
+// header word indices, the byte layouts of the packed-weight and activation
+// buffers (documented in include/bq.h), and small device helpers.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cmath>
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "bq.h"
+
+namespace bqi {
+
+constexpr uint32_t kPkMagic = 0x4B505142u;   // 'BQPK'
+constexpr uint32_t kActMagic = 0x43415142u;  // 'BQAC'
+constexpr uint32_t kVersion = 1;
+
+// packed-buffer header words
+enum : int {
+  HW_MAGIC = 0, HW_VERSION = 1, HW_FMT = 2, HW_N = 3, HW_K = 4, HW_NPAD = 5, HW_KPAD = 6,
+  HW_WBITS = 7, HW_ABITS = 8, HW_NSTREAMS = 9, HW_FIELD = 10, HW_SHIFT = 14, HW_TILEBYTES = 18,
+  HW_LORA_RANK = 19, HW_LORA_ALPHA = 20, HW_TSCALE = 21, HW_TOTAL = 22, HW_OFF_TILES = 24,
+  HW_OFF_ROWS = 26, HW_OFF_AUX = 28, HW_OFF_AUX2 = 30, HW_COUNT = 32
+};
+// activation-buffer header words
+enum : int {
+  AW_MAGIC = 0, AW_VERSION = 1, AW_FMT = 2, AW_M = 3, AW_K = 4, AW_KPAD = 5, AW_ABITS = 6,
+  AW_LORA_RANK = 7, AW_TOTAL = 8, AW_OFF_CODES = 10, AW_OFF_TOK = 12, AW_OFF_GSUM = 14,
+  AW_OFF_U = 16, AW_OFF_XT = 18, AW_COUNT = 20
+};
+
+constexpr int kBvsrSets = 256;
+constexpr int kBvsrTableStride = 8;  // floats per set: c0 c1 c2 c3 o sc ratio_index 0
+
+struct PkLayout {
+  int fmt, N, K, N_pad, K_pad, RB, KT, w_bits, a_bits, nstreams;
+  int field[4], shift[4];
+  int tile_bytes, rank;
+  float lora_alpha;
+  uint64_t off_tiles, off_rows, off_aux, off_aux2, total;
+};
+
+struct ActLayout {
+  int fmt, M, K, K_pad, KT, a_bits, rank;
+  uint64_t off_codes, off_tok, off_gsum, off_u, off_xt, total;
+};
+
+inline uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
+
+// Returns false for an unknown format or bit width.
+inline bool make_pk_layout(int fmt, int N, int K, int w_bits, int a_bits, int rank, float alpha,
+                           PkLayout* L) {
+  PkLayout l{};
+  l.fmt = fmt; l.N = N; l.K = K;
+  l.N_pad = (N + 15) / 16 * 16;
+  l.K_pad = (K + 255) / 256 * 256;
+  l.RB = l.N_pad / 16; l.KT = l.K_pad / 256;
+  uint64_t tiles = 0, rows = 0, aux = 0, aux2 = 0;
+  switch (fmt) {
+    case BQ_FMT_RABIT2:
+      l.w_bits = 2; l.a_bits = 16; l.nstreams = 2;
+      l.field[0] = l.field[1] = 1; l.shift[0] = 0; l.shift[1] = 1;
+      l.tile_bytes = 0;
+      tiles = 2ull * l.N_pad * (l.K_pad / 8);
+      rows = 2ull * l.N_pad * 4; aux = uint64_t(l.K_pad) * 4; aux2 = uint64_t(l.K_pad) * 4;
+      break;
+    case BQ_FMT_BITNET_W1A8:
+      l.w_bits = 1; l.a_bits = 8; l.nstreams = 1; l.field[0] = 1; l.tile_bytes = 512;
+      break;
+    case BQ_FMT_TERNARY_A8:
+      l.w_bits = 2; l.a_bits = 8; l.nstreams = 1; l.field[0] = 2; l.tile_bytes = 1024;
+      l.rank = rank; l.lora_alpha = alpha;
+      aux = uint64_t(l.K_pad) * rank * 2; aux2 = uint64_t(l.N_pad) * rank * 2;
+      break;
+    case BQ_FMT_ABQ: {
+      if (w_bits < 1 || w_bits > 8 || a_bits < 1 || a_bits > 8) return false;
+      l.w_bits = w_bits; l.a_bits = a_bits;
+      int rem = w_bits, sh = 0;
+      while (rem > 0) {  // fields of 8/4/2/1 bits from the low end of the code
+        int f = rem >= 8 ? 8 : rem >= 4 ? 4 : rem >= 2 ? 2 : 1;
+        l.field[l.nstreams] = f; l.shift[l.nstreams] = sh; l.nstreams++;
+        rem -= f; sh += f;
+      }
+      l.tile_bytes = 512 * w_bits;
+      rows = 3ull * l.N_pad * 4;
+      break;
+    }
+    case BQ_FMT_BVSR4:
+      l.w_bits = 4; l.a_bits = 8; l.nstreams = 4;
+      for (int s = 0; s < 4; s++) { l.field[s] = 1; l.shift[s] = s; }
+      l.tile_bytes = 2048;
+      aux = uint64_t(kBvsrSets) * kBvsrTableStride * 4;
+      aux2 = uint64_t(l.N_pad) * (l.K_pad / 32);
+      break;
+    default:
+      return false;
+  }
+  if (fmt != BQ_FMT_RABIT2) tiles = uint64_t(l.RB) * l.KT * l.tile_bytes;
+  l.off_tiles = 256;
+  l.off_rows = align256(l.off_tiles + tiles);
+  l.off_aux = align256(l.off_rows + rows);
+  l.off_aux2 = align256(l.off_aux + aux);
+  l.total = align256(l.off_aux2 + aux2);
+  *L = l;
+  return true;
+}
+
+inline ActLayout make_act_layout(const PkLayout& L, int M) {
+  ActLayout a{};
+  a.fmt = L.fmt; a.M = M; a.K = L.K; a.K_pad = L.K_pad; a.KT = L.KT; a.a_bits = L.a_bits;
+  a.rank = L.fmt == BQ_FMT_TERNARY_A8 ? L.rank : 0;
+  uint64_t codes = L.fmt == BQ_FMT_RABIT2 ? 0 : uint64_t(M) * L.KT * 256;
+  uint64_t tok = uint64_t(M) * 16;
+  uint64_t gsum = L.fmt == BQ_FMT_BVSR4 ? uint64_t(M) * (L.K_pad / 32) * 4 : 0;
+  uint64_t u = uint64_t(M) * a.rank * 4;
+  uint64_t xt = L.fmt == BQ_FMT_RABIT2 ? 2ull * M * L.K_pad * 4 : 0;
+  a.off_codes = 256;
+  a.off_tok = align256(a.off_codes + codes);
+  a.off_gsum = align256(a.off_tok + tok);
+  a.off_u = align256(a.off_gsum + gsum);
+  a.off_xt = align256(a.off_u + u);
+  a.total = align256(a.off_xt + xt);
+  return a;
+}
+
+inline bool layout_from_layer(const bq_layer* y, PkLayout* L) {
+  return make_pk_layout(y->fmt, y->N, y->K, y->w_bits, y->a_bits, y->lora_rank, 0.f, L);
+}
+
+// ---------------------------------------------------------------------------
+// device helpers
+// ---------------------------------------------------------------------------
+
+// Order-preserving map of a float to uint32 (total order on non-NaN values).
+__device__ __forceinline__ uint32_t float_key(float f) {
+  uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_float(uint32_t k) {
+  uint32_t b = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+  return __uint_as_float(b);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
+  return __uint_as_float(uint32_t(h) << 16);
+}
+
+// Round a float to bf16 (nearest, ties to even) and return the 16-bit storage.
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+  uint32_t u = __float_as_uint(f);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return uint16_t(u >> 16);
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Block-wide reductions for blockDim.x a multiple of 32 (<= 1024). `sh` needs 32 slots.
+template <typename T>
+__device__ T block_sum(T v, T* sh) {
+  int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) sh[w] = v;
+  __syncthreads();
+  T r = T(0);
+  if (w == 0) {
+    r = lane < nw ? sh[lane] : T(0);
+    r = warp_sum(r);
+    if (lane == 0) sh[0] = r;
+  }
+  __syncthreads();
+  return sh[0];
+}
+__device__ inline float block_max(float v, float* sh) {
+  int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_max(v);
+  __syncthreads();
+  if (lane == 0) sh[w] = v;
+  __syncthreads();
+  if (w == 0) {
+    float r = lane < nw ? sh[lane] : -INFINITY;
+    r = warp_max(r);
+    if (lane == 0) sh[0] = r;
+  }
+  __syncthreads();
+  return sh[0];
+}
+__device__ inline float block_min(float v, float* sh) {
+  int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_min(v);
+  __syncthreads();
+  if (lane == 0) sh[w] = v;
+  __syncthreads();
+  if (w == 0) {
+    float r = lane < nw ? sh[lane] : INFINITY;
+    r = warp_min(r);
+    if (lane == 0) sh[0] = r;
+  }
+  __syncthreads();
+  return sh[0];
+}
+
+}  // namespace bqi

@@ -1,0 +1,411 @@
+// Weight quantize + pack kernels (offline step of the layer).
+//
+// Every quantizer decision that turns a float into a code is taken in float32
+// with IEEE round-to-nearest operations (__fdiv_rn, rintf) or in float64 with
+// explicitly rounded operations (__dadd_rn / __dmul_rn, no FMA contraction),
+// so that the codes are reproducible bit for bit. Reductions (means) run in
+// float64 and are stored as float32.
+#pragma once
+
+#include "bq_internal.cuh"
+
+namespace bqi {
+
+struct HeaderWords {
+  uint32_t w[HW_COUNT];
+};
+
+__global__ void k_write_header(uint32_t* hdr, HeaderWords h) {
+  int i = threadIdx.x;
+  if (i < 64) hdr[i] = i < HW_COUNT ? h.w[i] : 0u;
+}
+
+// ---------------------------------------------------------------------------
+// mean |W| over a tensor: per-row float64 sums, then one fixed-order total
+// ---------------------------------------------------------------------------
+__global__ void k_row_abs_sum(const float* __restrict__ W, int K, double* __restrict__ row_sum) {
+  __shared__ double sh[32];
+  const float* w = W + size_t(blockIdx.x) * K;
+  double s = 0.0;
+  for (int k = threadIdx.x * 4; k < K; k += blockDim.x * 4) {
+    float4 v = *reinterpret_cast<const float4*>(w + k);
+    s = __dadd_rn(s, fabs(double(v.x)));
+    s = __dadd_rn(s, fabs(double(v.y)));
+    s = __dadd_rn(s, fabs(double(v.z)));
+    s = __dadd_rn(s, fabs(double(v.w)));
+  }
+  s = block_sum(s, sh);
+  if (threadIdx.x == 0) row_sum[blockIdx.x] = s;
+}
+
+__global__ void k_tensor_mean(const double* __restrict__ row_sum, int N, double count,
+                              uint32_t* __restrict__ hdr) {
+  __shared__ double sh[32];
+  double s = 0.0;
+  for (int n = threadIdx.x; n < N; n += blockDim.x) s = __dadd_rn(s, row_sum[n]);
+  s = block_sum(s, sh);
+  if (threadIdx.x == 0) {
+    float m = count > 0 ? __double2float_rn(__ddiv_rn(s, count)) : 0.f;
+    hdr[HW_TSCALE] = __float_as_uint(m);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// ABQ per-row asymmetric quantizer parameters: Delta, z, S_w = sum_k q
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int abq_code(float w, float delta, int z, int qmax) {
+  float r = rintf(__fdiv_rn(w, delta));
+  long long q = (long long)r + z;
+  q = q < 0 ? 0 : q;
+  q = q > qmax ? qmax : q;
+  return int(q);
+}
+
+__global__ void k_abq_rows(const float* __restrict__ W, int K, int w_bits, float* __restrict__ delta,
+                           int* __restrict__ zero, int* __restrict__ sumq) {
+  __shared__ float shf[32];
+  __shared__ int shi[32];
+  const float* w = W + size_t(blockIdx.x) * K;
+  float lo = INFINITY, hi = -INFINITY;
+  for (int k = threadIdx.x; k < K; k += blockDim.x) {
+    float v = w[k];
+    lo = fminf(lo, v);
+    hi = fmaxf(hi, v);
+  }
+  lo = block_min(lo, shf);
+  hi = block_max(hi, shf);
+  const int qmax = (1 << w_bits) - 1;
+  float rng = fmaxf(__fsub_rn(hi, lo), 1e-5f);
+  float d = __fdiv_rn(rng, float(qmax));
+  int z = int(rintf(__fdiv_rn(-lo, d)));
+  int s = 0;
+  for (int k = threadIdx.x; k < K; k += blockDim.x) s += abq_code(w[k], d, z, qmax);
+  s = block_sum(s, shi);
+  if (threadIdx.x == 0) {
+    delta[blockIdx.x] = d;
+    zero[blockIdx.x] = z;
+    sumq[blockIdx.x] = s;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Tiled field packer for BitNet / ternary / ABQ: one thread per 32-bit word.
+// ---------------------------------------------------------------------------
+struct FieldPackArgs {
+  const float* W;
+  uint32_t* tiles;
+  int N, K, KT, tile_words, nstreams;
+  int field[4], shift[4], soff_words[4];
+  const uint32_t* hdr;      // for the tensor scale (ternary gamma_W)
+  const float* abq_delta;   // ABQ row params
+  const int* abq_zero;
+  int w_bits;
+  uint64_t total_words;
+};
+
+template <int FMT>
+__global__ void k_pack_fields(FieldPackArgs a) {
+  uint64_t idx = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= a.total_words) return;
+  const int tw = a.tile_words;
+  const uint64_t tile = idx / tw;
+  const int wt = int(idx - tile * tw);
+  const int rb = int(tile / a.KT), kt = int(tile - uint64_t(rb) * a.KT);
+  int s = 0;
+  while (s + 1 < a.nstreams && wt >= a.soff_words[s + 1]) s++;
+  const int f = a.field[s];
+  const int ws = wt - a.soff_words[s];      // word within stream: [u][lane][r]
+  const int u = ws / 128, lane = (ws >> 2) & 31, r = ws & 3;
+  const int g = lane >> 2, t = lane & 3;
+  const int row = rb * 16 + g + 8 * (r & 1);
+  const int nj = 8 / f;
+  float gamma = 0.f;
+  if (FMT == BQ_FMT_TERNARY_A8) gamma = __uint_as_float(a.hdr[HW_TSCALE]);
+  float d = 0.f;
+  int z = 0;
+  const int qmax = (1 << a.w_bits) - 1;
+  if (FMT == BQ_FMT_ABQ && row < a.N) { d = a.abq_delta[row]; z = a.abq_zero[row]; }
+  uint32_t word = 0;
+  for (int j = 0; j < nj; j++) {
+    const int kb = 32 * (8 * kt + u * nj + j) + 16 * (r >> 1) + 4 * t;
+    for (int b = 0; b < 4; b++) {
+      const int k = kb + b;
+      uint32_t field;
+      const bool in = row < a.N && k < a.K;
+      const float w = in ? a.W[size_t(row) * a.K + k] : 0.f;
+      if (FMT == BQ_FMT_BITNET_W1A8) {
+        field = in ? (w >= 0.f ? 0u : 1u) : 0u;               // bit set <=> sign -1
+      } else if (FMT == BQ_FMT_TERNARY_A8) {
+        int T = 0;
+        if (in && gamma > 0.f) {
+          float q = rintf(__fdiv_rn(w, gamma));
+          T = q > 1.f ? 1 : (q < -1.f ? -1 : int(q));
+        }
+        field = uint32_t(T + 1);                              // {0,1,2}
+      } else {                                                // ABQ
+        int q = in ? abq_code(w, d, z, qmax) : 0;
+        field = (uint32_t(q) >> a.shift[s]) & ((1u << f) - 1u);
+      }
+      word |= field << (8 * b + f * j);
+    }
+  }
+  a.tiles[idx] = word;
+}
+
+// ---------------------------------------------------------------------------
+// RaBiT: B1 = sign(W), g1 = mean|W|, R1 = W - g1 B1 (h1 = 1), B2 = sign(R1),
+// g2 = mean|R1|; one block per row.
+// ---------------------------------------------------------------------------
+__global__ void k_rabit_pack(const float* __restrict__ W, int N_pad, int K, int K_pad,
+                             uint32_t* __restrict__ planes, float* __restrict__ g) {
+  __shared__ double sh[32];
+  const int n = blockIdx.x;
+  const float* w = W + size_t(n) * K;
+  double s1 = 0.0;
+  for (int k = threadIdx.x; k < K; k += blockDim.x) s1 = __dadd_rn(s1, fabs(double(w[k])));
+  s1 = block_sum(s1, sh);
+  const float g1 = __double2float_rn(__ddiv_rn(s1, double(K)));
+  const double g1d = double(g1);
+  const int W32 = K_pad / 32;
+  double s2 = 0.0;
+  for (int wd = threadIdx.x; wd < W32; wd += blockDim.x) {
+    uint32_t p1 = 0, p2 = 0;
+    for (int j = 0; j < 32; j++) {
+      const int k = wd * 32 + j;
+      if (k >= K) break;
+      const float v = w[k];
+      const bool neg1 = !(v >= 0.f);
+      const double r1 = __dsub_rn(double(v), neg1 ? -g1d : g1d);
+      const bool neg2 = !(r1 >= 0.0);
+      s2 = __dadd_rn(s2, fabs(r1));
+      p1 |= uint32_t(neg1) << j;
+      p2 |= uint32_t(neg2) << j;
+    }
+    planes[size_t(n) * W32 + wd] = p1;
+    planes[(size_t(N_pad) + n) * W32 + wd] = p2;
+  }
+  s2 = block_sum(s2, sh);
+  if (threadIdx.x == 0) {
+    g[n] = g1;
+    g[N_pad + n] = __double2float_rn(__ddiv_rn(s2, double(K)));
+  }
+}
+
+__global__ void k_rabit_h(const float* __restrict__ h2, int K, int K_pad, float* __restrict__ h1_out,
+                          float* __restrict__ h2_out) {
+  int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= K_pad) return;
+  h1_out[k] = k < K ? 1.f : 0.f;
+  h2_out[k] = k < K ? h2[k] : 0.f;
+}
+
+// ---------------------------------------------------------------------------
+// Ternary LoRA matrices to bf16: A [K][r] -> [K_pad][r], B [r][N] -> B^T [N_pad][r]
+// ---------------------------------------------------------------------------
+__global__ void k_lora_to_bf16(const float* __restrict__ A, const float* __restrict__ B, int N, int K,
+                               int N_pad, int K_pad, int r, uint16_t* __restrict__ A16,
+                               uint16_t* __restrict__ Bt16) {
+  uint64_t i = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const uint64_t na = uint64_t(K_pad) * r, nb = uint64_t(N_pad) * r;
+  if (i < na) {
+    int k = int(i / r), c = int(i % r);
+    A16[i] = k < K ? float_to_bf16_bits(A[size_t(k) * r + c]) : 0;
+  } else if (i < na + nb) {
+    uint64_t j = i - na;
+    int n = int(j / r), c = int(j % r);
+    Bt16[j] = n < N ? float_to_bf16_bits(B[size_t(c) * N + n]) : 0;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// BVSR: per-vector min/max keys, nearest-rank quantiles by a 32-step bitwise
+// selection, the 256-set table, then the exhaustive search per vector.
+// ---------------------------------------------------------------------------
+__global__ void k_bvsr_minmax(const float* __restrict__ W, int K, uint64_t V, uint32_t* __restrict__ kmin,
+                              uint32_t* __restrict__ kmax) {
+  uint64_t v = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (v >= V) return;
+  const int vpr = K / 32;
+  const uint64_t n = v / vpr, kv = v % vpr;
+  const float4* p = reinterpret_cast<const float4*>(W + n * K + kv * 32);
+  float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 8; i++) {
+    float4 q = p[i];
+    lo = fminf(fminf(lo, q.x), fminf(q.y, fminf(q.z, q.w)));
+    hi = fmaxf(fmaxf(hi, q.x), fmaxf(q.y, fmaxf(q.z, q.w)));
+  }
+  kmin[v] = float_key(lo);
+  kmax[v] = float_key(hi);
+}
+
+// target t < 8: (2t+1)/16 quantile of the minima; t >= 8: (2(t-8)+1)/16 of the maxima
+__device__ __forceinline__ uint64_t bvsr_rank(int t, uint64_t V) {
+  uint64_t num = 2 * (t & 7) + 1;
+  uint64_t r = (num * V + 15) / 16;
+  return r < 1 ? 1 : r;
+}
+
+__device__ __forceinline__ uint32_t bvsr_answer(const uint32_t* counts, int t, uint64_t V, int from_bit) {
+  uint32_t ans = 0;
+  const uint64_t rk = bvsr_rank(t, V);
+  for (int b = 31; b >= from_bit; b--)
+    if (uint64_t(counts[b * 16 + t]) < rk) ans |= 1u << b;
+  return ans;
+}
+
+// counts[bit][t] = #{keys <= ans_t(bits above) | (2^bit - 1)}
+__global__ void k_bvsr_count(const uint32_t* __restrict__ kmin, const uint32_t* __restrict__ kmax,
+                             uint64_t V, uint32_t* __restrict__ counts, int bit) {
+  __shared__ uint32_t thr_sh[16];
+  if (threadIdx.x < 16) thr_sh[threadIdx.x] = bvsr_answer(counts, threadIdx.x, V, bit + 1) | ((1u << bit) - 1u);
+  __syncthreads();
+  uint32_t thr[16];
+#pragma unroll
+  for (int t = 0; t < 16; t++) thr[t] = thr_sh[t];
+  uint32_t c[16];
+#pragma unroll
+  for (int t = 0; t < 16; t++) c[t] = 0;
+  for (uint64_t v = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x; v < V;
+       v += uint64_t(gridDim.x) * blockDim.x) {
+    const uint32_t a = kmin[v], b = kmax[v];
+#pragma unroll
+    for (int t = 0; t < 8; t++) c[t] += a <= thr[t];
+#pragma unroll
+    for (int t = 8; t < 16; t++) c[t] += b <= thr[t];
+  }
+#pragma unroll
+  for (int t = 0; t < 16; t++) {
+    uint32_t s = warp_sum(c[t]);
+    if ((threadIdx.x & 31) == 0 && s) atomicAdd(&counts[bit * 16 + t], s);
+  }
+}
+
+// One block of 256 threads: set s = 64j + 8a + b.
+__global__ void k_bvsr_table(const uint32_t* counts_in, uint64_t V, float* table) {
+  __shared__ uint32_t cnt[32 * 16];
+  __shared__ float lo[8], hi[8];
+  for (int i = threadIdx.x; i < 32 * 16; i += blockDim.x) cnt[i] = counts_in[i];
+  __syncthreads();   // every read of the counts (which share the table's memory) is done
+  if (threadIdx.x < 16) {
+    const float v = key_float(bvsr_answer(cnt, threadIdx.x, V, 0));
+    if (threadIdx.x < 8) lo[threadIdx.x] = v; else hi[threadIdx.x - 8] = v;
+  }
+  __syncthreads();
+  const int s = threadIdx.x;
+  const int j = s >> 6, a = (s >> 3) & 7, b = s & 7;
+  const double r = 1.5 + 0.5 * j;
+  const double pw[4] = {1.0, r, r * r, r * r * r};
+  const double tsum = __dadd_rn(__dadd_rn(__dadd_rn(pw[0], pw[1]), pw[2]), pw[3]);
+  const double span = __dsub_rn(double(hi[b]), double(lo[a]));
+  float* row = table + s * kBvsrTableStride;
+  for (int i = 0; i < 4; i++) row[i] = __double2float_rn(__dmul_rn(span, __ddiv_rn(pw[i], tsum)));
+  row[4] = lo[a];
+  // derived kernel constants: c_i = (hi - lo) R_i / sum R for the integer templates R
+  const double rsum[4] = {65.0, 15.0, 203.0, 40.0};
+  row[5] = __double2float_rn(__ddiv_rn(span, rsum[j]));
+  row[6] = float(j);
+  row[7] = 0.f;
+}
+
+// Points of set s, o + c0 b0 + c1 b1 + c2 b2 + c3 b3 summed left to right in float64.
+__device__ __forceinline__ void bvsr_points(const float* __restrict__ row, double P[16]) {
+  const double o = row[4], c0 = row[0], c1 = row[1], c2 = row[2], c3 = row[3];
+#pragma unroll
+  for (int code = 0; code < 16; code++) {
+    double acc = o;
+    if (code & 1) acc = __dadd_rn(acc, c0);
+    if (code & 2) acc = __dadd_rn(acc, c1);
+    if (code & 4) acc = __dadd_rn(acc, c2);
+    if (code & 8) acc = __dadd_rn(acc, c3);
+    P[code] = acc;
+  }
+}
+
+// nearest point: smallest |w - p|, lowest code on an exact tie
+__device__ __forceinline__ int bvsr_nearest(double w, const double P[16], double* p_out) {
+  double best = INFINITY, bp = P[0];
+  int bc = 0;
+#pragma unroll
+  for (int code = 0; code < 16; code++) {
+    const double d = fabs(__dsub_rn(w, P[code]));
+    if (d < best) { best = d; bc = code; bp = P[code]; }
+  }
+  *p_out = bp;
+  return bc;
+}
+
+// One block of 256 threads (thread = set) per vector, grid-stride over vectors.
+__global__ void __launch_bounds__(256) k_bvsr_search(const float* __restrict__ W, int K, int K_pad, int KT,
+                                                     uint64_t V, const float* __restrict__ table,
+                                                     uint32_t* __restrict__ tiles32, uint8_t* __restrict__ setidx) {
+  __shared__ float wv[32];
+  __shared__ double red_e[8];
+  __shared__ int red_s[8];
+  __shared__ int s_best_sh;
+  const int s = threadIdx.x, lane = s & 31, warp = s >> 5;
+  double P[16];
+  bvsr_points(table + s * kBvsrTableStride, P);
+  const int vpr = K / 32;
+  for (uint64_t v = blockIdx.x; v < V; v += gridDim.x) {
+    const uint64_t n = v / vpr;
+    const int kv = int(v % vpr);
+    __syncthreads();
+    if (s < 32) wv[s] = W[n * K + uint64_t(kv) * 32 + s];
+    __syncthreads();
+    double err = 0.0;
+    for (int e = 0; e < 32; e++) {
+      const double w = double(wv[e]);
+      double p;
+      bvsr_nearest(w, P, &p);
+      const double de = __dsub_rn(w, p);
+      err = __dadd_rn(err, __dmul_rn(de, de));
+    }
+    // argmin over sets, lowest index on a tie
+    int sb = s;
+    double eb = err;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const double e2 = __shfl_xor_sync(0xffffffffu, eb, o);
+      const int s2 = __shfl_xor_sync(0xffffffffu, sb, o);
+      if (e2 < eb || (e2 == eb && s2 < sb)) { eb = e2; sb = s2; }
+    }
+    if (lane == 0) { red_e[warp] = eb; red_s[warp] = sb; }
+    __syncthreads();
+    if (warp == 0) {
+      eb = lane < 8 ? red_e[lane] : INFINITY;
+      sb = lane < 8 ? red_s[lane] : 0x7fffffff;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double e2 = __shfl_xor_sync(0xffffffffu, eb, o);
+        const int s2 = __shfl_xor_sync(0xffffffffu, sb, o);
+        if (e2 < eb || (e2 == eb && s2 < sb)) { eb = e2; sb = s2; }
+      }
+      if (lane == 0) s_best_sh = sb;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const int sbest = s_best_sh;
+      double Pb[16];
+      bvsr_points(table + sbest * kBvsrTableStride, Pb);
+      double p;
+      const int code = bvsr_nearest(double(wv[lane]), Pb, &p);
+      // tile position of element e = lane of vector (n, kv)
+      const int rb = int(n >> 4), rho = int(n & 15), g = rho & 7, rbit = rho >> 3;
+      const int kt = kv >> 3, j = kv & 7;
+      const int e = lane, rh = e >> 4, t = (e >> 2) & 3, b = e & 3;
+      const int r = 2 * rh + rbit, tl = 4 * g + t;
+      const uint64_t base_w = (uint64_t(rb) * KT + kt) * (2048 / 4) + tl * 4 + r;
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        uint32_t val = uint32_t((code >> i) & 1) << (8 * b + j);
+        val |= __shfl_xor_sync(0xffffffffu, val, 1);
+        val |= __shfl_xor_sync(0xffffffffu, val, 2);
+        if (b == 0 && val) atomicOr(&tiles32[base_w + i * 128], val);
+      }
+      if (lane == 0) setidx[n * (K_pad / 32) + kv] = uint8_t(sbest);
+    }
+  }
+}
+
+}  // namespace bqi

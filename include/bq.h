@@ -1,0 +1,185 @@
+/*
+ * bq.h -- C ABI of the bit-plane quantized linear layer for NVIDIA B200 (sm_100a).
+ *
+ * One computation, y = sum_k scales (.) (B_k . x), for five weight formats
+ * whose weights are stored as binary planes or bitvectors B_k:
+ *
+ *   BQ_FMT_RABIT2       RaBiT two-path residual binarization, W_hat = g1 B1 h1 + g2 B2 h2
+ *                       ("RaBiT框架" page, §2.1 equation and §2.2 forward()).
+ *   BQ_FMT_BITNET_W1A8  BitNet sign weights alpha*sign(W), alpha = mean|W| per tensor
+ *                       ("1-bit LLM的端侧推理革命" page, §2.1-§2.3).
+ *   BQ_FMT_TERNARY_A8   1.58-bit absmean ternary weights packed 2 bits/weight, with the
+ *                       gated rank-r correction tanh(alpha) SiLU(xA) B fused in
+ *                       ("1.58位LLM混合门控流" page, §1.2, §2.1, §4.1).
+ *   BQ_FMT_ABQ          ABQ-style arbitrary-bit WxAy: per-row / per-token asymmetric codes,
+ *                       the product decomposed over weight bit-planes
+ *                       ("ABQ-LLM" page, abstract and §3.2 eq.(3)).
+ *   BQ_FMT_BVSR4        BVSR 4-bit bitvector sums with 256 cached coefficient sets
+ *                       ("BVSR" page, Introduction).
+ *
+ * Calls (the problem the pages state: pack offline, quantize activations online,
+ * then GEMV for decode or a small-M GEMM):
+ *   bq_packed_bytes / bq_pack_weights   quantize + pack W into a self-describing buffer
+ *   bq_act_bytes / bq_quantize_act      per-token activation quantization
+ *   bq_gemv (M = 1) / bq_gemm (M >= 1)  the layer, fused scale/zero-point/LoRA epilogue
+ *
+ * Ownership: the caller allocates every buffer (device memory for packed, act, W, x, y);
+ * sizes come from the *_bytes queries. The library never allocates, frees or
+ * synchronizes (bq_packed_validate and bq_device_check excepted, which touch host memory
+ * or read one device word). All work is enqueued on the caller's stream (a cudaStream_t
+ * passed as void*; NULL = legacy default stream).
+ *
+ * Errors: arguments are validated on the host before anything is enqueued; on error
+ * nothing runs and a status is returned. A failed launch returns BQ_ERR_CUDA.
+ * The kernels check the act-buffer header against the layer (format, M, K) and on a
+ * mismatch write no output and raise a device error word that bq_device_check reports.
+ * No exception crosses this ABI, and there is no CPU fallback: every step runs on the GPU.
+ *
+ * ------------------------------------------------------------------------------------
+ * Packed weight buffer (device, 256-byte aligned), little-endian, version 1.
+ * Header: 64 x 32-bit words (256 bytes):
+ *   0 magic 0x4B505142 ('BQPK')  1 version  2 format  3 N  4 K  5 N_pad (N rounded up to 16)
+ *   6 K_pad (K rounded up to 256)  7 w_bits  8 a_bits  9 n_streams
+ *   10..13 field width f_s of stream s (bits per weight)  14..17 shift of stream s
+ *   18 tile_bytes  19 lora_rank  20 lora_alpha (f32)  21 tensor_scale (f32: BitNet alpha,
+ *   ternary gamma_W)  22-23 total_bytes (u64)  24-25 off_tiles  26-27 off_rows
+ *   28-29 off_aux  30-31 off_aux2 (u64 byte offsets from the buffer start)
+ * Tiled weights (formats 2-5). Tile (rb, kt) covers rows 16rb..16rb+15 and
+ *   k = 256kt..256kt+255, at off_tiles + (rb*(K_pad/256) + kt)*tile_bytes. Inside a tile
+ *   the streams follow one another; stream s (field width f) takes 512*f bytes laid out
+ *   as [u < f][lane < 32][4 words]. In word r (0..3) of uint4 u of lane = 4g+t, the f-bit
+ *   field j (bits f*j .. f*j+f-1) of byte b holds the weight at
+ *       row = 16rb + g + 8(r & 1),
+ *       k   = 32(8kt + u*(8/f) + j) + 16(r >> 1) + 4t + b.
+ *   This is the A-operand fragment order of the int8 m16n8k32 tensor-core MMA: one AND
+ *   with the mask of field j turns four packed words into the four A registers of one MMA.
+ *   Padding rows/columns hold zero fields (ternary: field 1, i.e. T = 0).
+ *   Streams: BitNet 1 x f=1 (bit set <=> sign -1). Ternary 1 x f=2 (field = T+1 in {0,1,2}).
+ *   ABQ: w_bits split into fields of 8/4/2/1 bits from the low end (2:[2] 4:[4] 6:[4,2]
+ *   8:[8], shift = bit offset in the code). BVSR: 4 x f=1, stream i = bitvector plane i.
+ * RaBiT (format 1) is not tiled: bit j of uint32 off_tiles + 4((p*N_pad + n)(K_pad/32) + w)
+ *   is the sign of path p (0,1), row n, k = 32w + j (1 <=> -1).
+ * Sections: RaBiT rows = g1[N_pad], g2[N_pad] f32; aux = h1[K_pad], aux2 = h2[K_pad] f32.
+ *   Ternary aux = A bf16 [K_pad][r], aux2 = B^T bf16 [N_pad][r].
+ *   ABQ rows = Delta_w f32 [N_pad], z_w i32 [N_pad], S_w = sum_k q_w i32 [N_pad].
+ *   BVSR aux = coefficient table f32 [256][8] (c0 c1 c2 c3 o; then derived kernel constants:
+ *   sc = (hi-lo)/sum_i R_i, ratio index, 0); aux2 = set index u8 [N_pad][K_pad/32].
+ *
+ * Activation buffer (device, 256-byte aligned), version 1.
+ * Header: 64 x 32-bit words: 0 magic 0x43415142 ('BQAC') 1 version 2 format 3 M 4 K 5 K_pad
+ *   6 a_bits 7 lora_rank 8-9 total_bytes 10-11 off_codes 12-13 off_tok 14-15 off_gsum
+ *   16-17 off_u 18-19 off_xt.
+ * codes (formats 2-5): per token m and k-tile kt, 256 bytes; byte
+ *   (m*(K_pad/256) + kt)*256 + 64t + 8mu + 4h + b holds the code of k = 32(8kt+mu)+16h+4t+b
+ *   (the B-operand fragment order; int8 two's complement for A8 formats, whose bits are
+ *   the activation bit-planes X_c, uint8 for ABQ). Padding k hold code 0.
+ * tok [M][4] words: A8 {gamma_x f32, sum_k q i32, 0, 0}; ABQ {Delta_x f32, z_x i32, S_x i32, 0}.
+ * gsum (BVSR): i32 [M][K_pad/32], sum of q over each 32-element vector.
+ * u (ternary): f32 [M][r] = SiLU(x A) from the unquantized bf16 x.
+ * xt (RaBiT): f32 [2][M][K_pad] = h_p * x (no activation quantization).
+ */
+#ifndef BQ_H
+#define BQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BQ_OK = 0,
+  BQ_ERR_INVALID_ARG = 1,  /* null/unaligned pointer, bad enum, inconsistent arguments */
+  BQ_ERR_UNSUPPORTED = 2,  /* a combination this build does not implement */
+  BQ_ERR_SIZE = 3,         /* N, K, M out of range or a buffer smaller than required */
+  BQ_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+  BQ_ERR_BAD_PACKED = 5,   /* packed header failed validation */
+  BQ_ERR_DEVICE_CHECK = 6  /* a kernel found an inconsistent buffer (see bq_device_check) */
+} bq_status;
+
+typedef enum {
+  BQ_FMT_RABIT2 = 1,
+  BQ_FMT_BITNET_W1A8 = 2,
+  BQ_FMT_TERNARY_A8 = 3,
+  BQ_FMT_ABQ = 4,
+  BQ_FMT_BVSR4 = 5
+} bq_format;
+
+/* Limits: 1 <= N <= 1<<20, 128 <= K <= 1<<16 with K % 128 == 0, 1 <= M <= 64 (M = 0 is
+ * a no-op). ABQ needs (2^w - 1)(2^a - 1) K < 2^31 so that the int32 plane sums are exact. */
+#define BQ_MAX_N (1 << 20)
+#define BQ_MAX_K (1 << 16)
+#define BQ_MAX_M 64
+#define BQ_MAX_LORA_RANK 64
+
+/* Pack options. Device pointers are read during bq_pack_weights only. */
+typedef struct {
+  int32_t fmt;          /* bq_format */
+  int32_t w_bits;       /* ABQ weight bits, 1..8 (ignored by the other formats) */
+  int32_t a_bits;       /* ABQ activation bits, 1..8 (ignored: the A8 formats use 8) */
+  int32_t lora_rank;    /* ternary: rank r of the correction, 0..64 (0 = none) */
+  float lora_alpha;     /* ternary: gate alpha; the correction is scaled by tanh(alpha) */
+  const float* h2;      /* RaBiT: device f32 [K], second-path input scale (h1 = 1) */
+  const float* lora_A;  /* ternary: device f32 [K][r] row-major, rounded to bf16 */
+  const float* lora_B;  /* ternary: device f32 [r][N] row-major, rounded to bf16 */
+} bq_pack_desc;
+
+/* Host-side description of a packed layer; filled by bq_pack_weights or
+ * bq_packed_validate, read by every other call (so no call reads the device header
+ * from the host). `packed` is the caller's device buffer. */
+typedef struct {
+  int32_t fmt, N, K, N_pad, K_pad, w_bits, a_bits, lora_rank;
+  uint64_t packed_bytes;
+  const void* packed;
+} bq_layer;
+
+const char* bq_status_str(bq_status s);
+int32_t bq_version(void);
+
+/* Bytes of the packed buffer for W [N,K] under `desc`. Host only. */
+bq_status bq_packed_bytes(const bq_pack_desc* desc, int32_t N, int32_t K, size_t* bytes);
+
+/* Quantize W (device f32 [N][K], row-major, 16-byte aligned) and write the packed buffer
+ * (device, >= bq_packed_bytes, 256-byte aligned). The packed buffer also serves as the
+ * pack's own scratch before it is overwritten. Weight quantizers (per format): sign with
+ * sign(0)=+1 and the residual recursion (RaBiT); alpha*sign(W), alpha = mean|W| (BitNet);
+ * T = clamp(rn(W/gamma),-1,1), gamma = mean|W| (ternary); per-row asymmetric codes
+ * q = clamp(rn(W/Delta)+z, 0, 2^w-1) (ABQ); exhaustive MSE search over the 256 cached
+ * sets (BVSR). `layer` receives the host description. Asynchronous on `stream`. */
+bq_status bq_pack_weights(const bq_pack_desc* desc, const float* W, int32_t N, int32_t K,
+                          void* packed, size_t packed_bytes, void* stream, bq_layer* layer);
+
+/* Parse and check a HOST copy of a packed buffer's header (e.g. after loading a saved
+ * buffer) and fill `layer` with packed_dev as its device pointer. Host only. */
+bq_status bq_packed_validate(const void* packed_host, size_t bytes, const void* packed_dev,
+                             bq_layer* layer);
+
+/* Bytes of the activation buffer for M tokens of `layer`. Host only. */
+bq_status bq_act_bytes(const bq_layer* layer, int32_t M, size_t* bytes);
+
+/* Quantize x (device bf16 [M][K] row-major, 16-byte aligned) per token into `act`
+ * (device, >= bq_act_bytes, 256-byte aligned): absmax int8 (A8 formats, gamma = max|x|,
+ * q = clamp(rn(x*127/gamma), -127, 127)), per-token asymmetric a-bit codes (ABQ),
+ * h_p*x in f32 (RaBiT); plus the ternary u = SiLU(xA) and the BVSR group sums. */
+bq_status bq_quantize_act(const bq_layer* layer, const void* x_bf16, int32_t M, void* act,
+                          size_t act_bytes, void* stream);
+
+/* y [M][N] f32 (device) = the layer applied to the quantized activations in `act`.
+ * acc_dbg (nullable, device int64 [M][N]) receives the exact integer accumulator:
+ * BitNet/ternary sum_k w q, ABQ sum_k (q_w - z_w)(q_x - z_x), BVSR sum_k code q
+ * (not available for RaBiT, whose path is float). bq_gemv is bq_gemm with M = 1. */
+bq_status bq_gemv(const bq_layer* layer, const void* act, float* y, int64_t* acc_dbg,
+                  void* stream);
+bq_status bq_gemm(const bq_layer* layer, const void* act, int32_t M, float* y,
+                  int64_t* acc_dbg, void* stream);
+
+/* Synchronizes the current device, then reads and clears the device error word:
+ * BQ_OK or BQ_ERR_DEVICE_CHECK. */
+bq_status bq_device_check(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BQ_H */

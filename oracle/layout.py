@@ -87,34 +87,43 @@ def tiled_field_index(N_pad: int, K_pad: int, f: int):
     return row, kk
 
 
-def read_stream_codes(buf: bytes, h: dict, s: int) -> np.ndarray:
-    """Stream s of a tiled buffer as unsigned field values [N, K] (uint8)."""
+def read_stream_codes(buf: bytes, h: dict, s: int, row_blocks=None) -> np.ndarray:
+    """Stream s of a tiled buffer as unsigned field values (uint8): [N, K], or
+    [16*len(row_blocks), K] for a subset of 16-row blocks."""
     f = h["fields"][s]
     N, K, N_pad, K_pad = h["N"], h["K"], h["N_pad"], h["K_pad"]
     RB, KT, tb = N_pad // 16, K_pad // 256, h["tile_bytes"]
     s_off = sum(512 * h["fields"][i] for i in range(s))
-    raw = np.frombuffer(buf, dtype=np.uint8, count=RB * KT * tb, offset=h["off_tiles"])
-    tiles = raw.reshape(RB, KT, tb)[:, :, s_off:s_off + 512 * f].reshape(RB, KT, f, 32, 4, 4)
+    rbs = np.arange(RB) if row_blocks is None else np.asarray(row_blocks)
+    raw = np.frombuffer(buf, dtype=np.uint8, count=RB * KT * tb, offset=h["off_tiles"]).reshape(RB, KT, tb)
+    tiles = raw[rbs][:, :, s_off:s_off + 512 * f].reshape(len(rbs), KT, f, 32, 4, 4)
     row_i, k_i = tiled_field_index(N_pad, K_pad, f)
     nj = 8 // f
     mask = (1 << f) - 1
-    # field j of every byte: [RB, KT, f, 32, 4, 4, nj]
-    vals = (tiles[..., None] >> (f * np.arange(nj))) & mask
-    out = np.zeros((N_pad, K_pad), dtype=np.uint8)
-    rb = np.arange(RB)[:, None, None, None, None, None, None]
+    vals = (tiles[..., None] >> (f * np.arange(nj))) & mask       # [R, KT, f, 32, 4, 4, nj]
+    out = np.zeros((16 * len(rbs), K_pad), dtype=np.uint8)
+    rb = np.arange(len(rbs))[:, None, None, None, None, None, None]
     kt = np.arange(KT)[None, :, None, None, None, None, None]
-    rows = 16 * rb + row_i[None, None]
-    ks = 256 * kt + k_i[None, None]
-    rows, ks = np.broadcast_arrays(rows, ks)
+    rows, ks = np.broadcast_arrays(16 * rb + row_i[None, None], 256 * kt + k_i[None, None])
     out[rows, ks] = vals
-    return out[:N, :K]
+    if row_blocks is None:
+        return out[:N, :K]
+    return out[:, :K]
 
 
-def read_packed(buf: bytes) -> dict:
-    """Decode a packed buffer into the dict shape that bq_oracle's layers take."""
+def read_packed(buf: bytes, row_blocks=None) -> dict:
+    """Decode a packed buffer into the dict shape that bq_oracle's layers take.
+    ``row_blocks`` (tiled formats) restricts the per-row arrays to those 16-row
+    blocks (rows 16*rb .. 16*rb+15, padding rows included); ``rows`` lists them."""
     h = read_header(buf)
     fmt, N, K, N_pad, K_pad = h["fmt"], h["N"], h["K"], h["N_pad"], h["K_pad"]
     out = dict(header=h)
+    rb = row_blocks
+    if rb is not None:
+        sel = (16 * np.asarray(rb)[:, None] + np.arange(16)[None, :]).ravel()
+    else:
+        sel = np.arange(N)
+    out["rows"] = sel
     if fmt == FMT_RABIT:
         W32 = K_pad // 32
         raw = np.frombuffer(buf, dtype="<u4", count=2 * N_pad * W32, offset=h["off_tiles"])
@@ -127,11 +136,11 @@ def read_packed(buf: bytes) -> dict:
         out["h1"] = np.frombuffer(buf, dtype="<f4", count=K, offset=h["off_aux"]).copy()
         out["h2"] = np.frombuffer(buf, dtype="<f4", count=K, offset=h["off_aux2"]).copy()
     elif fmt == FMT_BITNET:
-        neg = read_stream_codes(buf, h, 0)
+        neg = read_stream_codes(buf, h, 0, rb)
         out["B"] = np.where(neg == 1, -1, 1).astype(np.int8)
         out["alpha"] = h["tensor_scale"]
     elif fmt == FMT_TERNARY:
-        u = read_stream_codes(buf, h, 0).astype(np.int16)
+        u = read_stream_codes(buf, h, 0, rb).astype(np.int16)
         out["T"] = (u - 1).astype(np.int8)
         out["field_max"] = int(u.max()) if u.size else 0
         out["gamma_w"] = h["tensor_scale"]
@@ -141,28 +150,28 @@ def read_packed(buf: bytes) -> dict:
             A = np.frombuffer(buf, dtype="<u2", count=K_pad * r, offset=h["off_aux"]).reshape(K_pad, r)
             Bt = np.frombuffer(buf, dtype="<u2", count=N_pad * r, offset=h["off_aux2"]).reshape(N_pad, r)
             out["A"] = _bf16_to_f32(A[:K])
-            out["B"] = _bf16_to_f32(Bt[:N]).T.copy()
+            out["B"] = _bf16_to_f32(Bt[sel]).T.copy()
     elif fmt == FMT_ABQ:
-        Q = np.zeros((N, K), dtype=np.int32)
+        Q = np.zeros((len(sel), K), dtype=np.int32)
         for s in range(h["n_streams"]):
-            Q += read_stream_codes(buf, h, s).astype(np.int32) << h["shifts"][s]
+            Q += read_stream_codes(buf, h, s, rb).astype(np.int32) << h["shifts"][s]
         out["Q"] = Q
         rowsec = np.frombuffer(buf, dtype="<u4", count=3 * N_pad, offset=h["off_rows"])
-        out["delta"] = rowsec[:N].view("<f4").copy()
-        out["z"] = rowsec[N_pad:N_pad + N].view("<i4").copy()
-        out["S_w"] = rowsec[2 * N_pad:2 * N_pad + N].view("<i4").copy()
+        out["delta"] = rowsec[:N_pad][sel].view("<f4").copy()
+        out["z"] = rowsec[N_pad:2 * N_pad][sel].view("<i4").copy()
+        out["S_w"] = rowsec[2 * N_pad:3 * N_pad][sel].view("<i4").copy()
         out["w_bits"] = h["w_bits"]
         out["a_bits"] = h["a_bits"]
     elif fmt == FMT_BVSR:
-        codes = np.zeros((N, K), dtype=np.uint8)
+        codes = np.zeros((len(sel), K), dtype=np.uint8)
         for s in range(h["n_streams"]):
-            codes |= (read_stream_codes(buf, h, s) << h["shifts"][s]).astype(np.uint8)
+            codes |= (read_stream_codes(buf, h, s, rb) << h["shifts"][s]).astype(np.uint8)
         out["codes"] = codes
         tab = np.frombuffer(buf, dtype="<f4", count=256 * 8, offset=h["off_aux"]).reshape(256, 8)
         out["table"] = tab[:, :5].copy()
         out["table_derived"] = tab[:, 5:].copy()
         sets = np.frombuffer(buf, dtype=np.uint8, count=N_pad * (K_pad // 32), offset=h["off_aux2"])
-        out["sets"] = sets.reshape(N_pad, K_pad // 32)[:N, :K // 32].copy()
+        out["sets"] = sets.reshape(N_pad, K_pad // 32)[sel, :K // 32].copy()
     else:
         raise ValueError(f"unknown format {fmt}")
     return out

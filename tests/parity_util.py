@@ -1,0 +1,151 @@
+"""Helpers for GPU parity tests: run the CUDA path through the C ABI, read its
+buffers back with the oracle's independent readers, and compare with the
+oracle. Test infrastructure only."""
+from __future__ import annotations
+
+import numpy as np
+
+import bq_inputs as I
+from oracle import bq_oracle as O
+from oracle import layout as L
+
+RTOL = 1e-3  # max|y - y_ref| <= 1e-3 (||y_ref||_inf + 1e-6)
+
+
+def torch_mods():
+    import torch
+    from bit_weight_quantization_b200 import bq
+    return torch, bq
+
+
+def to_dev_f32(a):
+    torch, _ = torch_mods()
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def to_dev_bf16(x):
+    torch, _ = torch_mods()
+    bits = I.bf16_bits(x).view(np.int16)
+    return torch.from_numpy(np.ascontiguousarray(bits)).cuda().view(torch.bfloat16)
+
+
+def ulp_diff(a, b) -> np.ndarray:
+    a = np.asarray(a, np.float32).view(np.int32).astype(np.int64)
+    b = np.asarray(b, np.float32).view(np.int32).astype(np.int64)
+    return np.abs(a - b)
+
+
+def assert_y_close(y, y_ref, what=""):
+    y, y_ref = np.asarray(y, np.float64), np.asarray(y_ref, np.float64)
+    assert y.shape == y_ref.shape, (y.shape, y_ref.shape)
+    assert np.all(np.isfinite(y)), f"{what}: non-finite output"
+    err = float(np.max(np.abs(y - y_ref))) if y.size else 0.0
+    bound = RTOL * ((float(np.max(np.abs(y_ref))) if y_ref.size else 0.0) + 1e-6)
+    assert err <= bound, f"{what}: max|y-y_ref| = {err:.3e} > {bound:.3e}"
+
+
+class GpuLayer:
+    """One layer packed and run by the library, plus host copies of its buffers."""
+
+    def __init__(self, fmt, N, K, M, seed=0, w_bits=0, a_bits=0, lora_rank=32, lora_alpha=0.1,
+                 inputs=None, nullify_x=False):
+        torch, bq = torch_mods()
+        self.fmt, self.N, self.K, self.M = fmt, N, K, M
+        self.w_bits, self.a_bits = w_bits, a_bits
+        inp = inputs if inputs is not None else I.layer_inputs(fmt, N, K, M, seed, lora_rank)
+        if nullify_x:
+            inp["x"] = np.zeros_like(inp["x"])
+        self.inp = inp
+        self.W = to_dev_f32(inp["W"])
+        kw = {}
+        if fmt == "rabit":
+            kw["h2"] = to_dev_f32(inp["h2"])
+        if fmt == "ternary":
+            kw.update(lora_rank=lora_rank, lora_alpha=lora_alpha,
+                      lora_A=to_dev_f32(inp["lora_A"]), lora_B=to_dev_f32(inp["lora_B"]))
+        if fmt == "abq":
+            kw.update(w_bits=w_bits, a_bits=a_bits)
+        self.ql = bq.QuantLinear(fmt, self.W, **kw)
+        self.x = to_dev_bf16(inp["x"])
+        self.y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        self.acc = None
+        if fmt != "rabit":
+            self.acc = torch.full((M, N), -(1 << 62), dtype=torch.int64, device="cuda")
+        self.ql.forward(self.x, self.y, self.acc)
+        torch.cuda.synchronize()
+        bq.bq_device_check()
+        self.packed = self.ql.packed.cpu().numpy().tobytes()
+        self.act = self.ql.act_buffer(M).cpu().numpy().tobytes()
+        self.y_h = self.y.cpu().numpy()
+        self.acc_h = self.acc.cpu().numpy() if self.acc is not None else None
+
+    def read(self, row_blocks=None):
+        return L.read_packed(self.packed, row_blocks)
+
+
+def oracle_pack(fmt, inp, w_bits=0, lora_alpha=0.1, rows=None):
+    W = inp["W"]
+    if fmt == "rabit":
+        return O.rabit_pack(W, inp["h2"])
+    if fmt == "bitnet":
+        p = O.bitnet_pack(W)
+        if rows is not None:
+            p["B"] = p["B"][rows]
+        return p
+    if fmt == "ternary":
+        p = O.ternary_pack(W, inp.get("lora_A"), inp.get("lora_B"), lora_alpha)
+        if rows is not None:
+            p["T"] = p["T"][rows]
+        return p
+    if fmt == "abq":
+        sub = W if rows is None else W[rows]
+        return O.abq_pack(sub, w_bits)
+    if fmt == "bvsr":
+        return O.bvsr_pack(W, rows=rows)
+    raise ValueError(fmt)
+
+
+def oracle_layer(fmt, p, x, a_bits=0):
+    """Reference layer on the library's own decoded codes (dict from the reader)."""
+    if fmt == "rabit":
+        return O.rabit_layer(p, x)
+    if fmt == "bitnet":
+        return O.bitnet_layer(p, x)
+    if fmt == "ternary":
+        return O.ternary_layer(p, x)
+    if fmt == "abq":
+        r = O.abq_layer(p, x, a_bits)
+        r["acc"] = r["I"]
+        return r
+    if fmt == "bvsr":
+        return O.bvsr_layer(p["codes"], p["sets"], p["table"], x)
+    raise ValueError(fmt)
+
+
+def check_act(gl: GpuLayer):
+    """Activation buffer against the oracle's activation quantizer (bit-exact)."""
+    a = L.read_act(gl.act)
+    x = gl.inp["x"]
+    assert a["M"] == gl.M and a["K"] == gl.K
+    if gl.fmt == "rabit":
+        h2 = gl.inp["h2"]
+        assert np.array_equal(a["xt"][0], x.astype(np.float32))
+        assert np.array_equal(a["xt"][1], (h2[None, :] * x).astype(np.float32))
+        return
+    if gl.fmt == "abq":
+        Qx, dx, zx = O.quantize_rows_asym(x, gl.a_bits)
+        assert np.array_equal(a["codes"].astype(np.int32), Qx)
+        assert np.array_equal(a["scale"], dx) and np.array_equal(a["zero"], zx)
+        assert np.array_equal(a["sum"], Qx.sum(1).astype(np.int32))
+    else:
+        q, gamma = O.quantize_act_int8(x)
+        assert np.array_equal(a["codes"], q)
+        assert np.array_equal(a["scale"], gamma)
+        assert np.array_equal(a["sum"], q.astype(np.int64).sum(1))
+        if gl.fmt == "bvsr":
+            gs = q.astype(np.int64).reshape(gl.M, -1, 32).sum(2)
+            assert np.array_equal(a["gsum"], gs)
+        if gl.fmt == "ternary":
+            ref_u = O.silu(x.astype(np.float64) @ L.read_packed(gl.packed)["A"].astype(np.float64))
+            assert np.allclose(a["u"], ref_u, rtol=1e-4, atol=1e-5)
+    assert np.all(a["codes_pad"] == 0)

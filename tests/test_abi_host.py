@@ -1,0 +1,174 @@
+"""The C-ABI library on the host (no GPU): it loads, exports every declared
+call, sizes buffers per the documented layout, and rejects bad arguments with
+the documented status before anything is enqueued."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+from bit_weight_quantization_b200 import bq
+from oracle import layout as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "bq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bq_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 10
+    out = subprocess.run(["nm", "-D", "--defined-only", bq.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(\w+)$", out, flags=re.M))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    assert set(bq.EXPORTED) == set(names)
+
+
+def test_status_strings_and_version():
+    assert bq.bq_version() == 1
+    assert bq.bq_status_str(0) == "ok"
+    assert "device" in bq.bq_status_str(6)
+
+
+@pytest.mark.parametrize("fmt,kw,N,K,expect", [
+    ("bitnet", {}, 4096, 4096, 256 + 4096 * 4096 // 8),
+    ("bitnet", {}, 50, 384, 256 + 64 * 512 // 8),
+    ("ternary", dict(lora_rank=32), 2048, 2048, 256 + 2048 * 2048 // 4 + 2048 * 32 * 2 * 2),
+    ("abq", dict(w_bits=6, a_bits=6), 4096, 4096, 256 + 4096 * 4096 * 6 // 8 + 3 * 4096 * 4),
+    ("bvsr", {}, 5120, 5120, 256 + 5120 * 5120 // 2 + 256 * 8 * 4 + 5120 * 5120 // 32),
+])
+def test_packed_bytes_match_layout(fmt, kw, N, K, expect):
+    d = bq.make_desc(fmt, **kw)
+    assert bq.bq_packed_bytes(d, N, K) == expect
+
+
+def test_packed_bits_per_weight():
+    # 2 bits/weight ternary packing, 1 bit BitNet, w bits ABQ, 4 + 8/32 BVSR (planes + set index)
+    N = K = 4096
+    for fmt, kw, bits in [("bitnet", {}, 1), ("ternary", {}, 2), ("abq", dict(w_bits=2, a_bits=8), 2),
+                          ("abq", dict(w_bits=8, a_bits=8), 8)]:
+        tot = bq.bq_packed_bytes(bq.make_desc(fmt, **kw), N, K)
+        assert tot - 256 - (3 * N * 4 if fmt == "abq" else 0) == N * K * bits // 8
+    tot = bq.bq_packed_bytes(bq.make_desc("bvsr"), N, K)
+    assert tot - 256 - 256 * 8 * 4 == N * K * 4.25 / 8
+
+
+@pytest.mark.parametrize("N,K,status", [(0, 256, 3), (16, 0, 3), (16, 200, 3), (16, 64, 3),
+                                        ((1 << 20) + 1, 256, 3), (16, (1 << 16) + 128, 3)])
+def test_packed_bytes_rejects_sizes(N, K, status):
+    d = bq.make_desc("bitnet")
+    out = ctypes.c_size_t()
+    assert bq.raw_status("bq_packed_bytes", ctypes.byref(d), N, K, ctypes.byref(out)) == status
+
+
+def test_bad_descriptors():
+    out = ctypes.c_size_t()
+    for d, st in [(bq.make_desc(9), 1), (bq.make_desc("abq", 0, 8), 1), (bq.make_desc("abq", 8, 9), 1),
+                  (bq.make_desc("ternary", lora_rank=65, lora_A=16, lora_B=16), 1),
+                  (bq.make_desc("ternary", lora_rank=8), 0), (bq.make_desc("rabit"), 0)]:
+        assert bq.raw_status("bq_packed_bytes", ctypes.byref(d), 64, 256, ctypes.byref(out)) == st
+    # the pack call itself needs the device pointers the format reads
+    layer = bq.bq_layer()
+    fake = 1 << 40
+    for d in (bq.make_desc("rabit"), bq.make_desc("ternary", lora_rank=8)):
+        assert bq.raw_status("bq_pack_weights", ctypes.byref(d), fake, 64, 256, fake, 1 << 30, None,
+                             ctypes.byref(layer)) == 1
+    # (2^8-1)^2 * K must stay below 2^31 for exact int32 plane sums
+    d = bq.make_desc("abq", 8, 8)
+    assert bq.raw_status("bq_packed_bytes", ctypes.byref(d), 64, 33024, ctypes.byref(out)) == 0
+    assert bq.raw_status("bq_packed_bytes", ctypes.byref(d), 64, 33152, ctypes.byref(out)) == 3
+    assert bq.raw_status("bq_packed_bytes", None, 64, 256, ctypes.byref(out)) == 1
+
+
+def test_pack_rejects_before_launch():
+    d = bq.make_desc("bitnet")
+    layer = bq.bq_layer()
+    nbytes = bq.bq_packed_bytes(d, 64, 256)
+    fake = 1 << 40   # never dereferenced: validation fails first
+    args = lambda W, P, n: (ctypes.byref(d), W, 64, 256, P, n, None, ctypes.byref(layer))
+    assert bq.raw_status("bq_pack_weights", *args(None, fake, nbytes)) == 1      # null W
+    assert bq.raw_status("bq_pack_weights", *args(fake + 4, fake, nbytes)) == 1  # W not 16-aligned
+    assert bq.raw_status("bq_pack_weights", *args(fake, fake + 16, nbytes)) == 1  # packed not 256-aligned
+    assert bq.raw_status("bq_pack_weights", *args(fake, fake, nbytes - 1)) == 3  # buffer too small
+    assert bq.raw_status("bq_pack_weights", ctypes.byref(d), fake, 64, 257, fake, nbytes, None,
+                         ctypes.byref(layer)) == 3                                    # K % 128 != 0
+
+
+def _host_header(fmt, N, K, **kw):
+    """A packed header written by the oracle side from the documented layout."""
+    d = bq.make_desc(fmt, **kw)
+    total = bq.bq_packed_bytes(d, N, K)
+    N_pad, K_pad = -(-N // 16) * 16, -(-K // 256) * 256
+    h = np.zeros(64, "<u4")
+    h[0], h[1], h[2], h[3], h[4], h[5], h[6] = L.PK_MAGIC, 1, bq.FORMATS[fmt], N, K, N_pad, K_pad
+    fields = {"bitnet": [1], "ternary": [2], "bvsr": [1, 1, 1, 1]}.get(fmt)
+    if fmt == "abq":
+        w = kw["w_bits"]
+        fields, rem = [], w
+        while rem:
+            f = 8 if rem >= 8 else 4 if rem >= 4 else 2 if rem >= 2 else 1
+            fields.append(f)
+            rem -= f
+    h[7] = {"bitnet": 1, "ternary": 2, "bvsr": 4}.get(fmt, kw.get("w_bits", 0))
+    h[8] = kw.get("a_bits", 8)
+    h[9] = len(fields)
+    sh = 0
+    for i, f in enumerate(fields):
+        h[10 + i], h[14 + i] = f, (i if fmt == "bvsr" else sh)
+        sh += f
+    h[18] = 512 * sum(fields)
+    h[19] = kw.get("lora_rank", 0)
+    tiles = (N_pad // 16) * (K_pad // 256) * h[18]
+    rows = 3 * N_pad * 4 if fmt == "abq" else 0
+    a256 = lambda v: (v + 255) // 256 * 256
+    off_rows = a256(256 + tiles)
+    aux = {"ternary": K_pad * h[19] * 2, "bvsr": 256 * 8 * 4}.get(fmt, 0)
+    aux2 = {"ternary": N_pad * h[19] * 2, "bvsr": N_pad * (K_pad // 32)}.get(fmt, 0)
+    off_aux = a256(off_rows + rows)
+    off_aux2 = a256(off_aux + aux)
+    for word, v in [(22, total), (24, 256), (26, off_rows), (28, off_aux), (30, off_aux2)]:
+        h[word], h[word + 1] = v & 0xFFFFFFFF, v >> 32
+    assert a256(off_aux2 + aux2) == total
+    return h
+
+
+@pytest.mark.parametrize("fmt,kw", [("bitnet", {}), ("ternary", dict(lora_rank=32)),
+                                    ("abq", dict(w_bits=6, a_bits=6)), ("bvsr", {})])
+def test_packed_validate_host_header(fmt, kw):
+    h = _host_header(fmt, 300, 1024, **kw)
+    layer = bq.bq_packed_validate(h.tobytes(), 1 << 20)
+    assert (layer.fmt, layer.N, layer.K, layer.N_pad, layer.K_pad) == (bq.FORMATS[fmt], 300, 1024, 304, 1024)
+    assert bq.bq_act_bytes(layer, 1) > 256
+    bad = h.copy()
+    bad[26] += 256                              # wrong section offset
+    with pytest.raises(bq.BQError) as e:
+        bq.bq_packed_validate(bad.tobytes(), 1 << 20)
+    assert e.value.status == bq.BQ_ERR_BAD_PACKED
+    bad = h.copy()
+    bad[0] ^= 1                                 # wrong magic
+    with pytest.raises(bq.BQError):
+        bq.bq_packed_validate(bad.tobytes(), 1 << 20)
+
+
+def test_act_and_gemv_reject_before_launch():
+    h = _host_header("bitnet", 64, 256)
+    layer = bq.bq_packed_validate(h.tobytes(), 1 << 20)
+    nact = bq.bq_act_bytes(layer, 2)
+    assert nact == 256 + 512 + 256   # header, codes 2 x 256, token params padded to 256
+    L_ = ctypes.byref(layer)
+    fake = 1 << 40
+    assert bq.raw_status("bq_quantize_act", L_, fake, 65, fake, nact, None) == 3       # M > 64
+    assert bq.raw_status("bq_quantize_act", L_, fake + 2, 2, fake, nact, None) == 1    # x unaligned
+    assert bq.raw_status("bq_quantize_act", L_, fake, 2, fake, nact - 1, None) == 3    # act too small
+    assert bq.raw_status("bq_quantize_act", L_, fake, 0, fake, 0, None) == 0           # M = 0: no-op
+    assert bq.raw_status("bq_gemm", L_, fake + 128, 2, fake, None, None) == 1          # act unaligned
+    assert bq.raw_status("bq_gemm", L_, fake, 2, None, None, None) == 1                # null y
+    assert bq.raw_status("bq_gemm", L_, fake, 0, fake, None, None) == 0                # M = 0: no-op
+    assert bq.raw_status("bq_gemm", None, fake, 1, fake, None, None) == 1

@@ -1,0 +1,205 @@
+"""CUDA path vs the CPU oracle, through the C ABI (needs a B200).
+
+Small cases span several 16-row blocks and 256-k tiles with ragged tails
+(N not a multiple of 16, K not a multiple of 256) and several token groups;
+the oracle checks every output. Integer accumulators must be bit-exact;
+y must satisfy max|y - y_ref| <= 1e-3 (||y_ref||_inf + 1e-6).
+"""
+import numpy as np
+import pytest
+
+import bq_inputs as I
+from oracle import bq_oracle as O
+from tests.parity_util import GpuLayer, assert_y_close, check_act, oracle_layer, oracle_pack, ulp_diff
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [(16, 256), (50, 384), (97, 640), (33, 128)]
+ABQ_WA = [(2, 8), (4, 4), (6, 6), (8, 8), (1, 3), (3, 5), (5, 2), (7, 7)]
+
+
+def _pack_parity(gl: GpuLayer, fmt, w_bits=0):
+    p = gl.read()
+    ref = oracle_pack(fmt, gl.inp, w_bits)
+    if fmt == "rabit":
+        assert np.all(ulp_diff(p["g1"], ref["g1"]) <= 1)
+        assert np.array_equal(p["B1"], ref["B1"])
+        same_g1 = p["g1"] == ref["g1"]
+        assert np.array_equal(p["B2"][same_g1], ref["B2"][same_g1])
+        assert np.all(ulp_diff(p["g2"], ref["g2"]) <= 1)
+        assert np.array_equal(p["h2"], gl.inp["h2"]) and np.all(p["h1"] == 1)
+    elif fmt == "bitnet":
+        assert np.array_equal(p["B"], ref["B"])
+        assert ulp_diff(p["alpha"], ref["alpha"]) <= 1
+    elif fmt == "ternary":
+        assert ulp_diff(p["gamma_w"], ref["gamma_w"]) <= 1
+        if p["gamma_w"] == ref["gamma_w"]:
+            assert np.array_equal(p["T"], ref["T"])
+        assert p["field_max"] <= 2
+        assert np.array_equal(p["A"], ref["A"]) and np.array_equal(p["B"], ref["B"])
+        assert p["lora_alpha"] == np.float32(0.1)
+    elif fmt == "abq":
+        assert np.array_equal(p["delta"], ref["delta"])
+        assert np.array_equal(p["z"], ref["z"])
+        assert np.array_equal(p["Q"], ref["Q"])
+        assert np.array_equal(p["S_w"], ref["Q"].sum(1))
+    elif fmt == "bvsr":
+        assert np.array_equal(p["table"], ref["table"])
+        assert np.array_equal(p["sets"], ref["sets"])
+        assert np.array_equal(p["codes"], ref["codes"])
+    return p
+
+
+def _layer_parity(gl: GpuLayer, p, fmt, a_bits=0):
+    r = oracle_layer(fmt, p, gl.inp["x"], a_bits)
+    if gl.acc_h is not None:
+        assert np.array_equal(gl.acc_h, r["acc"]), "integer accumulator differs"
+    assert_y_close(gl.y_h, r["y"], fmt)
+
+
+@pytest.mark.parametrize("N,K", SMALL)
+@pytest.mark.parametrize("fmt", ["bitnet", "ternary", "bvsr", "rabit"])
+@pytest.mark.parametrize("M", [1, 3, 9])
+def test_small_parity(fmt, N, K, M):
+    if fmt == "rabit" and M > 3:
+        M = 2
+    gl = GpuLayer(fmt, N, K, M, seed=N + K + M)
+    p = _pack_parity(gl, fmt)
+    check_act(gl)
+    _layer_parity(gl, p, fmt)
+
+
+@pytest.mark.parametrize("wa", ABQ_WA)
+@pytest.mark.parametrize("N,K,M", [(50, 384, 1), (97, 640, 9), (16, 256, 8)])
+def test_small_parity_abq(wa, N, K, M):
+    w, a = wa
+    gl = GpuLayer("abq", N, K, M, seed=w * 10 + a, w_bits=w, a_bits=a)
+    p = _pack_parity(gl, "abq", w)
+    check_act(gl)
+    _layer_parity(gl, p, "abq", a)
+
+
+@pytest.mark.parametrize("fmt", ["bitnet", "ternary", "bvsr", "rabit", "abq"])
+def test_zero_activations(fmt):
+    gl = GpuLayer(fmt, 40, 256, 2, w_bits=4, a_bits=4, nullify_x=True)
+    check_act(gl)
+    if fmt == "ternary":
+        assert np.all(gl.y_h == 0)   # SiLU(0) = 0, gamma_x = 0
+    elif fmt == "abq":
+        p = gl.read()
+        _layer_parity(gl, p, "abq", 4)
+    else:
+        assert np.all(gl.y_h == 0)
+
+
+def test_ternary_m_values_and_lora():
+    for M in (1, 4, 16):
+        gl = GpuLayer("ternary", 2048, 2048, M, seed=M)
+        p = _pack_parity(gl, "ternary")
+        check_act(gl)
+        _layer_parity(gl, p, "ternary")
+
+
+def test_outlier_heavy_activations():
+    inp = I.layer_inputs("bitnet", 64, 512, 3, seed=4)
+    inp["x"] = I.bf16_round(inp["x"] * np.where(np.arange(512) % 37 == 0, 300.0, 1.0)[None, :])
+    gl = GpuLayer("bitnet", 64, 512, 3, inputs=inp)
+    check_act(gl)
+    _layer_parity(gl, gl.read(), "bitnet")
+
+
+def test_n_equals_one_and_min_k():
+    for fmt in ("bitnet", "ternary", "bvsr", "abq", "rabit"):
+        gl = GpuLayer(fmt, 1, 128, 1, w_bits=2, a_bits=8)
+        p = _pack_parity(gl, fmt, 2)
+        _layer_parity(gl, p, fmt, 8)
+
+
+def test_exact_zero_weights_are_plus_one():
+    inp = I.layer_inputs("bitnet", 16, 256, 1, seed=3)
+    inp["W"][:, ::5] = 0.0
+    inp["W"][3, ::7] = -0.0
+    gl = GpuLayer("bitnet", 16, 256, 1, inputs=inp)
+    p = gl.read()
+    assert np.all(p["B"][:, ::5][inp["W"][:, ::5] == 0] == 1)
+    _layer_parity(gl, p, "bitnet")
+
+
+# ------------------------------------------------------------------ full sizes
+def _sample_blocks(N, n=6, seed=0):
+    RB = (N + 15) // 16
+    rng = np.random.default_rng(seed)
+    return np.unique(np.concatenate([[0, RB - 1], rng.choice(RB, size=min(n, RB), replace=False)]))
+
+
+def _full_size(fmt, N, K, M, w_bits=0, a_bits=0):
+    gl = GpuLayer(fmt, N, K, M, w_bits=w_bits, a_bits=a_bits)
+    rbs = _sample_blocks(N)
+    p = gl.read(rbs)
+    rows = p["rows"]
+    keep = rows < N
+    rows = rows[keep]
+    for key in ("B", "T", "Q", "codes", "sets", "delta", "z", "S_w"):
+        if key in p:
+            p[key] = p[key][keep]
+    if "B" in p and fmt == "ternary":
+        p["B"] = p["B"][:, keep]
+    ref = oracle_pack(fmt, gl.inp, w_bits, rows=rows)
+    if fmt == "bitnet":
+        assert np.array_equal(p["B"], ref["B"]) and ulp_diff(p["alpha"], ref["alpha"]) <= 1
+    elif fmt == "ternary":
+        assert ulp_diff(p["gamma_w"], ref["gamma_w"]) <= 1
+        if p["gamma_w"] == ref["gamma_w"]:
+            assert np.array_equal(p["T"], ref["T"])
+    elif fmt == "abq":
+        assert np.array_equal(p["Q"], ref["Q"]) and np.array_equal(p["delta"], ref["delta"])
+        assert np.array_equal(p["z"], ref["z"])
+    elif fmt == "bvsr":
+        assert np.array_equal(p["table"], ref["table"])
+        assert np.array_equal(p["sets"], ref["sets"]) and np.array_equal(p["codes"], ref["codes"])
+    check_act(gl)
+    r = oracle_layer(fmt, p, gl.inp["x"], a_bits)
+    if gl.acc_h is not None:
+        assert np.array_equal(gl.acc_h[:, rows], r["acc"])
+    assert_y_close(gl.y_h[:, rows], r["y"], f"{fmt} {N}x{K}")
+    assert np.all(np.isfinite(gl.y_h))
+
+
+@pytest.mark.parametrize("N,K", [(4096, 4096), (11008, 4096), (4096, 11008)])
+def test_full_bitnet(N, K):
+    _full_size("bitnet", N, K, 1)
+
+
+@pytest.mark.parametrize("N,K", [(5120, 5120), (13824, 5120), (5120, 13824)])
+def test_full_bvsr(N, K):
+    _full_size("bvsr", N, K, 1)
+
+
+@pytest.mark.parametrize("wa", [(2, 8), (4, 4), (6, 6), (8, 8)])
+@pytest.mark.parametrize("N", [4096, 11008])
+@pytest.mark.parametrize("M", [1, 8, 64])
+def test_full_abq(wa, N, M):
+    _full_size("abq", N, 4096, M, wa[0], wa[1])
+
+
+def test_full_rabit():
+    gl = GpuLayer("rabit", 256, 512, 1)
+    p = _pack_parity(gl, "rabit")
+    check_act(gl)
+    _layer_parity(gl, p, "rabit")
+
+
+# ------------------------------------------------------------------ device checks
+def test_act_buffer_mismatch_is_reported():
+    """An act buffer quantized for M=2 used with M=1: the kernel sees the header
+    mismatch, writes nothing and raises the device error word."""
+    from tests.parity_util import torch_mods
+    torch, bq = torch_mods()
+    gl = GpuLayer("bitnet", 32, 256, 2)
+    y = torch.full((1, 32), 7.0, device="cuda")
+    bq.bq_gemv(gl.ql.layer, gl.ql.act_buffer(2), y)
+    with pytest.raises(bq.BQError) as e:
+        bq.bq_device_check()
+    assert e.value.status == bq.BQ_ERR_DEVICE_CHECK
+    assert torch.all(y == 7.0)
+    bq.bq_device_check()   # the word was cleared
