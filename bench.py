@@ -2,7 +2,8 @@
 
 One step = one decode token through a 32-layer Llama-7B linear stack at
 W1A8: per decoder layer q, k, v, o [4096x4096], gate, up [11008x4096] and
-down [4096x11008], each layer call = bq_quantize_act + bq_gemv (224 calls,
+down [4096x11008], each layer call = bq_linear, i.e. the activation quantization
+fused into the GEMV kernel (224 calls,
 about 820 MB of packed weights, so every step streams inputs larger than L2).
 Weights ~ N(0, 0.02^2) and activations ~ N(0, 1) are synthetic (seeded torch
 generator on the device; no model or dataset).
@@ -36,13 +37,23 @@ NOMINAL_HBM_GBS = 8000.0
 def layer_bytes(fmt: str, N: int, K: int, M: int = 1, w_bits: int = 1, a_bits: int = 8) -> dict:
     """Algorithmic bytes of one layer call: packed weights + per-row/tensor scales,
     x bf16 read by the act kernel, act codes written and read once, y fp32."""
+    if fmt == "rabit":
+        # 2 sign planes + g1,g2 + h1,h2; act: x bf16 in, x~1, x~2 f32 out and back in; y f32
+        w = 2 * N * K // 8 + 8 * N + 8 * K
+        return dict(gemv=w + 8 * M * K + 4 * M * N, act=2 * M * K + 8 * M * K + 8 * K,
+                    total=w + 2 * M * K + 16 * M * K + 8 * K + 4 * M * N)
     bits = {"bitnet": 1, "ternary": 2, "abq": w_bits, "bvsr": 4}[fmt]
     w = N * K * bits // 8
     extra = {"bitnet": 4, "ternary": 4, "abq": 12 * N, "bvsr": N * K // 32 + 256 * 32}[fmt]
     x = 2 * M * K
     act = M * K
     y = 4 * M * N
-    return dict(gemv=w + extra + act + y + 16 * M, act=x + act + 16 * M, total=w + extra + x + 2 * act + y + 32 * M)
+    lora_g = lora_a = 0
+    if fmt == "ternary":   # rank-32 bf16 A read by the act kernel, B^T by the GEMV, u f32 between them
+        lora_a, lora_g = 32 * K * 2 + 32 * 4 * M, 32 * N * 2 + 32 * 4 * M
+    gemv = w + extra + act + y + 16 * M + lora_g
+    actb = x + act + 16 * M + lora_a
+    return dict(gemv=gemv, act=actb, total=gemv + actb)
 
 
 def measured_peaks() -> tuple[float, str]:
@@ -191,13 +202,13 @@ def build_stack(layers: int, seed: int, device):
 
 
 def step_calls(stack, timing=None):
+    """One decode step: bq_linear (activation quantization fused into the GEMV) per layer."""
     from bit_weight_quantization_b200 import bq
     for i, L in enumerate(stack):
         ql = L["ql"]
-        bq.bq_quantize_act(ql.layer, L["x"], 1, L["act"], L["act"].numel())
         if timing is not None:
             timing[i][0].record()
-        bq.bq_gemv(ql.layer, L["act"], L["y"])
+        bq.bq_linear(ql.layer, L["x"], 1, L["y"])
         if timing is not None:
             timing[i][1].record()
 
@@ -254,7 +265,7 @@ def run_cuda(args) -> None:
 
         # per-launch time of the GEMV kernel (the dominant one): a second capture of the
         # same step with events around every bq_gemv, replayed as many times
-        timing = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in stack]
+        timing = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True)) for _ in stack]
         gi = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gi, stream=stream):
             step_calls(stack, timing)
@@ -285,8 +296,7 @@ def run_cuda(args) -> None:
             for i, L in enumerate(stack):
                 ql = L["ql"]
                 x = xs_d[offs[i]:offs[i] + L["K"]].view(1, -1)
-                bq.bq_quantize_act(ql.layer, x, 1, L["act"], L["act"].numel())
-                bq.bq_gemv(ql.layer, L["act"], ys_d[yoffs[i]:yoffs[i] + L["N"]])
+                bq.bq_linear(ql.layer, x, 1, ys_d[yoffs[i]:yoffs[i] + L["N"]])
             ys_h.copy_(ys_d, non_blocking=True)
 
         for _ in range(max(1, min(args.warmup, 3))):
@@ -320,7 +330,8 @@ def run_cuda(args) -> None:
             "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": {"workload": "BitNet W1A8 decode GEMV, M=1: 32-layer Llama-7B linear stack "
                                    "(q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008), "
-                                   "bq_quantize_act + bq_gemv per layer, CUDA graph per step",
+                                   "bq_linear (act quantization fused into the GEMV) per layer, "
+                                   "PDL between layers, CUDA graph per step",
                        "layers_per_step": n_layers, "seq_len": 1, "global_batch": world,
                        "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (each step streams %.0f MB of distinct packed weights)"
@@ -329,12 +340,12 @@ def run_cuda(args) -> None:
             "frac_of_peak": value / world / peak, "frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm", "achieved": gemv_achieved, "peak": peak, "unit": "GB/s",
                          "frac": gemv_achieved / peak, "traffic": traffic, "peak_source": peak_kind,
-                         "kernel": "k_gemv_mma<BitNet W1A8> (bq_gemv)",
+                         "kernel": "k_layer<BitNet W1A8, fused> (bq_linear)",
                          "us_per_launch": gemv_ms_step * 1e3 / n_layers},
             "e2e": {"value": per_step / (e2e_ms * 1e-3) / 1e9 * world, "unit": "GB/s",
                     "h2d_bytes_per_step": int(xs_h.numel() * 2), "d2h_bytes_per_step": int(ys_h.numel() * 4),
                     "ms_per_step": e2e_ms, "path": "eager Python calls of the C ABI, pinned host buffers"},
-            "gpu_launches": 2 * n_layers * args.steps,
+            "gpu_launches": n_layers * args.steps,
             "clocks": clk,
         }
     if world > 1:
@@ -349,6 +360,140 @@ def run_cuda(args) -> None:
         print(json.dumps(out), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# per-config measurement (every format / shape / M) and a single-layer mode
+# ---------------------------------------------------------------------------
+def make_layer(fmt, N, K, M, w_bits, a_bits, gen, device):
+    import torch
+    from bit_weight_quantization_b200 import bq
+    W = torch.randn(N, K, device=device, generator=gen) * 0.02
+    kw = {}
+    if fmt == "rabit":
+        kw["h2"] = torch.rand(K, device=device, generator=gen) + 0.5
+    if fmt == "ternary":
+        kw.update(lora_rank=32, lora_alpha=0.1,
+                  lora_A=torch.randn(K, 32, device=device, generator=gen) * 0.02,
+                  lora_B=torch.randn(32, N, device=device, generator=gen) * 0.01)
+    if fmt == "abq":
+        kw.update(w_bits=w_bits, a_bits=a_bits)
+        flat = W.view(-1)
+        idx = torch.randperm(flat.numel(), device=device, generator=gen)[: flat.numel() // 1000]
+        flat[idx] *= 20.0
+    ql = bq.QuantLinear(fmt, W, **kw)
+    x = torch.randn(M, K, device=device, generator=gen)
+    if fmt == "abq":
+        ch = torch.randperm(K, device=device, generator=gen)[: K // 100]
+        x[:, ch] *= 10.0
+    x = x.to(torch.bfloat16)
+    y = torch.empty(M, N, device=device)
+    return dict(ql=ql, x=x, y=y, act=ql.act_buffer(M), ws=ql.workspace(M), M=M, keep=kw)
+
+
+def layer_call(L, timing=None, fused=True):
+    from bit_weight_quantization_b200 import bq
+    ql, M = L["ql"], L["M"]
+    if timing is not None:
+        timing[0].record()
+    if fused:
+        bq.bq_linear(ql.layer, L["x"], M, L["y"], None, L["ws"], L["ws"].numel())
+    else:
+        bq.bq_quantize_act(ql.layer, L["x"], M, L["act"], L["act"].numel())
+        if M == 1:
+            bq.bq_gemv(ql.layer, L["act"], L["y"])
+        else:
+            bq.bq_gemm(ql.layer, L["act"], M, L["y"])
+    if timing is not None:
+        timing[1].record()
+
+
+def config_list():
+    out = [("rabit", 256, 512, 1, 0, 0)]
+    out += [("bitnet", N, K, 1, 1, 8) for N, K in [(4096, 4096), (11008, 4096), (4096, 11008)]]
+    out += [("ternary", 2048, 2048, M, 2, 8) for M in (1, 4, 16)]
+    out += [("abq", N, 4096, M, w, a) for (w, a) in [(2, 8), (4, 4), (6, 6), (8, 8)]
+            for N in (4096, 11008) for M in (1, 8, 64)]
+    out += [("bvsr", N, K, 1, 4, 8) for N, K in [(5120, 5120), (13824, 5120), (5120, 13824)]]
+    return out
+
+
+def run_configs(args) -> None:
+    """For each configuration: a CUDA graph over R distinct packed copies of the
+    layer (R copies total >= 3x L2, capped at 512) of act + gemv; reports the
+    per-layer-call time, the GEMV launch time and the algorithmic GB/s."""
+    import torch
+    from bit_weight_quantization_b200 import bq
+    dev = torch.device("cuda", 0)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(args.seed)
+    peak, peak_kind = measured_peaks()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    stream = torch.cuda.Stream(device=dev)
+    sel = config_list()
+    if args.only:
+        sel = [c for c in sel if c[0] == args.only]
+    for fmt, N, K, M, w, a in sel:
+        lb = layer_bytes(fmt, N, K, M, w, a)
+        R = int(min(512, max(2, -(-3 * l2 // lb["total"]))))
+        with torch.cuda.stream(stream):
+            Ls = [make_layer(fmt, N, K, M, w, a, gen, dev) for _ in range(R)]
+            fused = not args.unfused
+            for L in Ls:
+                layer_call(L, fused=fused)
+            torch.cuda.synchronize()
+            bq.bq_device_check()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for L in Ls:
+                    layer_call(L, fused=fused)
+            tim = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True)) for _ in Ls]
+            gi = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gi, stream=stream):
+                for L, t in zip(Ls, tim):
+                    layer_call(L, t, fused=fused)
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = max(3, int(2000 / R))
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            us_layer = e0.elapsed_time(e1) * 1e3 / (reps * R)
+            gl = []
+            for _ in range(5):
+                gi.replay()
+                torch.cuda.synchronize()
+                gl.append(statistics.mean(a_.elapsed_time(b_) for a_, b_ in tim) * 1e3)
+            us_gemv = statistics.median(gl)
+        line = dict(fmt=fmt, N=N, K=K, M=M, w_bits=w, a_bits=a, path="bq_linear" if fused else "act+gemm",
+                    copies=R, us_per_layer=us_layer,
+                    gbs=lb["total"] / (us_layer * 1e-6) / 1e9, frac_of_peak=lb["total"] / (us_layer * 1e-6) / 1e9 / peak,
+                    us_gemv=us_gemv, gemv_gbs=lb["gemv"] / (us_gemv * 1e-6) / 1e9,
+                    gemv_frac=lb["gemv"] / (us_gemv * 1e-6) / 1e9 / peak, bytes=lb["total"], peak=peak,
+                    peak_source=peak_kind)
+        print(json.dumps(line), flush=True)
+        del Ls, g, gi
+        torch.cuda.empty_cache()
+
+
+def run_layer(args) -> None:
+    """One layer, a few act + gemv calls (the target of ncu captures)."""
+    import torch
+    dev = torch.device("cuda", 0)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(args.seed)
+    N, K = (int(v) for v in args.shape.split("x"))
+    L = make_layer(args.fmt, N, K, args.M, args.w_bits, args.a_bits, gen, dev)
+    for _ in range(args.iters):
+        layer_call(L, fused=not args.unfused)
+    torch.cuda.synchronize()
+    from bit_weight_quantization_b200 import bq
+    bq.bq_device_check()
+    print(json.dumps(dict(mode="layer", fmt=args.fmt, N=N, K=K, M=args.M, iters=args.iters, ok=True)))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -358,8 +503,21 @@ def main():
     ap.add_argument("--layers", type=int, default=32)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--mode", default="bench", choices=["bench", "configs", "layer"])
+    ap.add_argument("--only", default="")
+    ap.add_argument("--fmt", default="bitnet")
+    ap.add_argument("--shape", default="11008x4096")
+    ap.add_argument("--M", type=int, default=1)
+    ap.add_argument("--w-bits", type=int, default=1)
+    ap.add_argument("--a-bits", type=int, default=8)
+    ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--unfused", action="store_true", help="bq_quantize_act + bq_gemv/gemm instead of bq_linear")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.mode == "configs":
+        run_configs(args)
+    elif args.mode == "layer":
+        run_layer(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_cuda(args)

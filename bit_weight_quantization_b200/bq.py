@@ -49,6 +49,9 @@ _SIGS = {
     "bq_quantize_act": (ctypes.c_int, [ctypes.POINTER(bq_layer), _P, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
     "bq_gemv": (ctypes.c_int, [ctypes.POINTER(bq_layer), _P, _P, _P, _P]),
     "bq_gemm": (ctypes.c_int, [ctypes.POINTER(bq_layer), _P, ctypes.c_int32, _P, _P, _P]),
+    "bq_linear_workspace_bytes": (ctypes.c_int, [ctypes.POINTER(bq_layer), ctypes.c_int32,
+                                                 ctypes.POINTER(ctypes.c_size_t)]),
+    "bq_linear": (ctypes.c_int, [ctypes.POINTER(bq_layer), _P, ctypes.c_int32, _P, _P, _P, ctypes.c_size_t, _P]),
     "bq_device_check": (ctypes.c_int, []),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -137,6 +140,18 @@ def bq_gemm(layer: bq_layer, act, M: int, y, acc_dbg=None, stream=None) -> None:
     _check(_lib.bq_gemm(ctypes.byref(layer), _ptr(act), M, _ptr(y), _ptr(acc_dbg), _stream(stream)), "bq_gemm")
 
 
+def bq_linear_workspace_bytes(layer: bq_layer, M: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(_lib.bq_linear_workspace_bytes(ctypes.byref(layer), M, ctypes.byref(out)), "bq_linear_workspace_bytes")
+    return out.value
+
+
+def bq_linear(layer: bq_layer, x_bf16, M: int, y, acc_dbg=None, workspace=None, workspace_bytes: int = 0,
+              stream=None) -> None:
+    _check(_lib.bq_linear(ctypes.byref(layer), _ptr(x_bf16), M, _ptr(y), _ptr(acc_dbg), _ptr(workspace),
+                          workspace_bytes, _stream(stream)), "bq_linear")
+
+
 def bq_device_check() -> None:
     _check(_lib.bq_device_check(), "bq_device_check")
 
@@ -157,10 +172,11 @@ class QuantLinear:
         import torch
         N, K = W.shape
         self.desc = make_desc(fmt, w_bits, a_bits, lora_rank, lora_alpha, h2, lora_A, lora_B)
-        self._keep = (W, h2, lora_A, lora_B)
         nbytes = bq_packed_bytes(self.desc, N, K)
         self.packed = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
         self.layer = bq_pack_weights(self.desc, W, N, K, self.packed, nbytes, stream)
+        # the pack reads W, h2 and the LoRA matrices asynchronously: wait before the caller may free them
+        (torch.cuda.current_stream() if stream is None else stream).synchronize()
         self.N, self.K = N, K
         self._acts = {}
 
@@ -176,6 +192,24 @@ class QuantLinear:
         act = self.act_buffer(M)
         bq_quantize_act(self.layer, x_bf16, M, act, act.numel(), stream)
         return act
+
+    def workspace(self, M):
+        import torch
+        key = ("ws", M)
+        if key not in self._acts:
+            n = bq_linear_workspace_bytes(self.layer, M)
+            self._acts[key] = torch.empty(max(n, 256), dtype=torch.uint8, device=self.packed.device)
+        return self._acts[key]
+
+    def linear(self, x_bf16, y=None, acc_dbg=None, stream=None):
+        """Fused activation quantization + layer (bq_linear)."""
+        import torch
+        M = x_bf16.shape[0]
+        if y is None:
+            y = torch.empty((M, self.N), dtype=torch.float32, device=x_bf16.device)
+        ws = self.workspace(M)
+        bq_linear(self.layer, x_bf16, M, y, acc_dbg, ws, ws.numel(), stream)
+        return y
 
     def forward(self, x_bf16, y=None, acc_dbg=None, stream=None):
         import torch

@@ -28,7 +28,7 @@ inline bq_status check_desc(const bq_pack_desc* d, int K, bool need_ptrs) {
     case BQ_FMT_BITNET_W1A8:
       return BQ_OK;
     case BQ_FMT_TERNARY_A8:
-      if (d->lora_rank < 0 || d->lora_rank > BQ_MAX_LORA_RANK) return BQ_ERR_INVALID_ARG;
+      if (d->lora_rank < 0 || d->lora_rank > BQ_MAX_LORA_RANK || d->lora_rank % 8 != 0) return BQ_ERR_INVALID_ARG;
       if (need_ptrs && d->lora_rank > 0 && (!d->lora_A || !d->lora_B)) return BQ_ERR_INVALID_ARG;
       if (!(d->lora_alpha == d->lora_alpha)) return BQ_ERR_INVALID_ARG;
       return BQ_OK;
@@ -91,6 +91,182 @@ inline bq_status check_layer(const bq_layer* y, PkLayout* L) {
   if (!layout_from_layer(y, L)) return BQ_ERR_INVALID_ARG;
   if (L->N_pad != y->N_pad || L->K_pad != y->K_pad || L->total > y->packed_bytes) return BQ_ERR_BAD_PACKED;
   return BQ_OK;
+}
+
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// bq_linear scratch: the ternary LoRA partial dot products [KT][M][r] (f32)
+inline uint64_t linear_workspace(const PkLayout& L, int M) {
+  return L.fmt == BQ_FMT_TERNARY_A8 && L.rank > 0 ? align256(uint64_t(L.KT) * M * L.rank * 4) : 0;
+}
+
+// Every field of LayerArgs that depends only on the layer, M and the outputs.
+inline LayerArgs layer_args(const PkLayout& L, const void* packed, int M, float* y, int64_t* acc) {
+  const uint8_t* P = static_cast<const uint8_t*>(packed);
+  LayerArgs g{};
+  g.tiles = P + L.off_tiles;
+  g.pk_hdr = reinterpret_cast<const uint32_t*>(P);
+  g.row_delta = reinterpret_cast<const float*>(P + L.off_rows);
+  g.row_zero = reinterpret_cast<const int*>(P + L.off_rows) + L.N_pad;
+  g.row_sum = reinterpret_cast<const int*>(P + L.off_rows) + 2 * L.N_pad;
+  g.lora_bt = reinterpret_cast<const uint16_t*>(P + L.off_aux2);
+  g.bvsr_table = reinterpret_cast<const float*>(P + L.off_aux);
+  g.rabit_planes = reinterpret_cast<const uint32_t*>(P + L.off_tiles);
+  g.rabit_g = reinterpret_cast<const float*>(P + L.off_rows);
+  g.rabit_h1 = reinterpret_cast<const float*>(P + L.off_aux);
+  g.rabit_h2 = reinterpret_cast<const float*>(P + L.off_aux2);
+  g.y = y;
+  g.acc = reinterpret_cast<long long*>(acc);
+  g.N = L.N; g.K = L.K; g.N_pad = L.N_pad; g.K_pad = L.K_pad; g.KT = L.KT; g.M = M;
+  g.RB = L.RB;
+  g.tile_bytes = L.tile_bytes; g.rank = L.fmt == BQ_FMT_TERNARY_A8 ? L.rank : 0; g.fmt = L.fmt;
+  g.a_bits = L.a_bits;
+  g.shift0 = L.shift[0]; g.shift1 = L.shift[1]; g.shift2 = L.shift[2];
+  return g;
+}
+
+inline uint32_t align128(uint64_t x) { return uint32_t((x + 127) & ~uint64_t(127)); }
+
+inline int sm_count() {
+  static int n = [] {
+    int dev = 0, v = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    return v;
+  }();
+  return n;
+}
+
+inline int pow2ceil(int v) {
+  int p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+// Work split and shared-memory carve of the persistent k_layer (NW = 8 warps):
+//  - tokens per CTA (tpc): fused, each token group of 256/pow2(tpc) threads holds its x
+//    in at most 16 16-byte chunks per thread; unfused, the code image fits in 96 KB;
+//  - about one CTA per SM, CPG CTAs per token group striding over the row blocks;
+//  - the weight ring gets what is left (at most 96 KB): S >= 2 stages of C tiles per warp.
+// Returns false when the layer does not fit this kernel.
+inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
+  constexpr int NW = 8, NT = NW * 32;
+  const int VPR = L.K_pad / 32;
+  const bool bvsr = L.fmt == BQ_FMT_BVSR4;
+  const int rank = L.fmt == BQ_FMT_TERNARY_A8 ? L.rank : 0;
+  const int npad = L.K_pad / 8;
+  g->cstride = L.KT * 256 + 16;
+  int tpc = std::min(8, M);
+  if (fused) {
+    auto J = [&](int t) { return (npad + NT / pow2ceil(t) - 1) / (NT / pow2ceil(t)); };
+    while (tpc > 1 && J(tpc) > kMaxXChunks) tpc--;
+    if (J(tpc) > kMaxXChunks) return false;
+    g->J = J(tpc);
+  } else {
+    while (tpc > 1 && uint64_t(tpc) * g->cstride > 96 * 1024) tpc--;
+    g->J = 0;
+  }
+  g->tpc = tpc;
+  g->TG = (M + tpc - 1) / tpc;
+  g->CPG = std::max(1, std::min(L.RB, (sm_count() + g->TG - 1) / g->TG));
+  g->T = (L.KT + NW - 1) / NW;
+  uint64_t off = 0;
+  auto take = [&](uint64_t bytes) {
+    const uint32_t o = uint32_t(off);
+    off = align128(off + bytes);
+    return o;
+  };
+  g->off_codes = take(uint64_t(tpc) * g->cstride);
+  g->off_tok = take(8 * 4 * 4);
+  g->off_u = take(rank > 0 ? uint64_t(tpc) * rank * 4 : 16);
+  g->off_gsum = take(bvsr ? uint64_t(tpc) * VPR * 4 : 16);
+  g->off_tab = take(bvsr ? uint64_t(kBvsrSets) * kBvsrTableStride * 4 : 16);
+  g->off_red = take(2ull * NW * 32 * 4 * 12);
+  const uint64_t fixed = off + 1024;  // + barriers
+  const uint64_t limit = 220 * 1024;
+  const uint64_t budget = std::min<uint64_t>(96 * 1024, fixed < limit ? limit - fixed : 0);
+  const uint64_t per_tile = uint64_t(NW) * L.tile_bytes;   // one tile for every warp
+  if (budget < 2 * per_tile) return false;
+  g->C = int(std::max<uint64_t>(1, std::min<uint64_t>(g->T, budget / (3 * per_tile))));
+  g->S = int(std::max<uint64_t>(2, std::min<uint64_t>(4, budget / (per_tile * g->C))));
+  g->off_ring = take(per_tile * g->C * g->S);
+  g->off_bar = take(uint64_t(NW * g->S + 2) * 8 + 16);
+  g->smem_bytes = uint32_t(off);
+  g->RB = L.RB;
+  return true;
+}
+
+// One instantiation per kernel, so the static below tracks that kernel's raised
+// dynamic shared-memory limit (processes drive one device each).
+template <int FMT, int F0, int F1, int F2, int NW, bool FUSED>
+inline cudaError_t launch_tiled_nw(const LayerArgs& g, dim3 grid, cudaStream_t s) {
+  auto k = k_layer<FMT, F0, F1, F2, NW, FUSED>;
+  static uint32_t smem_limit = 48 * 1024;
+  if (g.smem_bytes > smem_limit) {
+    const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(g.smem_bytes));
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();  // leave no stale error behind
+      return e;
+    }
+    smem_limit = g.smem_bytes;
+  }
+  return launch_pdl(k, grid, dim3(NW * 32), g.smem_bytes, s, g);
+}
+
+template <int FMT, int F0, int F1, int F2, bool FUSED>
+inline cudaError_t launch_tiled(const LayerArgs& g, int NW, dim3 grid, cudaStream_t s) {
+  (void)NW;
+  return launch_tiled_nw<FMT, F0, F1, F2, 8, FUSED>(g, grid, s);
+}
+
+template <bool FUSED>
+inline cudaError_t launch_fmt(const PkLayout& L, const LayerArgs& g, int NW, dim3 grid, cudaStream_t s) {
+  switch (L.fmt) {
+    case BQ_FMT_BITNET_W1A8: return launch_tiled<BQ_FMT_BITNET_W1A8, 1, 0, 0, FUSED>(g, NW, grid, s);
+    case BQ_FMT_TERNARY_A8: return launch_tiled<BQ_FMT_TERNARY_A8, 2, 0, 0, FUSED>(g, NW, grid, s);
+    case BQ_FMT_BVSR4: return launch_tiled<BQ_FMT_BVSR4, 1, 1, 1, FUSED>(g, NW, grid, s);
+    case BQ_FMT_ABQ:
+      switch (L.w_bits) {
+        case 1: return launch_tiled<BQ_FMT_ABQ, 1, 0, 0, FUSED>(g, NW, grid, s);
+        case 2: return launch_tiled<BQ_FMT_ABQ, 2, 0, 0, FUSED>(g, NW, grid, s);
+        case 3: return launch_tiled<BQ_FMT_ABQ, 2, 1, 0, FUSED>(g, NW, grid, s);
+        case 4: return launch_tiled<BQ_FMT_ABQ, 4, 0, 0, FUSED>(g, NW, grid, s);
+        case 5: return launch_tiled<BQ_FMT_ABQ, 4, 1, 0, FUSED>(g, NW, grid, s);
+        case 6: return launch_tiled<BQ_FMT_ABQ, 4, 2, 0, FUSED>(g, NW, grid, s);
+        case 7: return launch_tiled<BQ_FMT_ABQ, 4, 2, 1, FUSED>(g, NW, grid, s);
+        case 8: return launch_tiled<BQ_FMT_ABQ, 8, 0, 0, FUSED>(g, NW, grid, s);
+        default: return cudaErrorInvalidValue;
+      }
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+inline bq_status launch_layer(const PkLayout& L, LayerArgs& g, bool fused, cudaStream_t s) {
+  cudaError_t e;
+  if (L.fmt == BQ_FMT_RABIT2) {
+    const dim3 grid(unsigned((L.N + 7) / 8));
+    e = fused ? launch_pdl(k_rabit<8, true>, grid, dim3(256), 0, s, g)
+              : launch_pdl(k_rabit<8, false>, grid, dim3(256), 0, s, g);
+  } else {
+    if (!plan_layer(L, g.M, fused, &g)) return BQ_ERR_UNSUPPORTED;
+    const dim3 grid(unsigned(g.TG * g.CPG));
+    e = fused ? launch_fmt<true>(L, g, 8, grid, s) : launch_fmt<false>(L, g, 8, grid, s);
+  }
+  return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
 }  // namespace bqi
@@ -197,8 +373,7 @@ bq_status bq_pack_weights(const bq_pack_desc* desc, const float* W, int32_t N, i
       k_bvsr_table<<<1, 256, 0, s>>>(counts, V, table);
       if (cudaMemsetAsync(P + L.off_tiles, 0, L.off_rows - L.off_tiles, s) != cudaSuccess) return BQ_ERR_CUDA;
       const unsigned sb = unsigned(std::min<uint64_t>(V, 148ull * 16));
-      k_bvsr_search<<<sb, 256, 0, s>>>(W, K, L.K_pad, L.KT, V, table, reinterpret_cast<uint32_t*>(P + L.off_tiles),
-                                       P + L.off_aux2);
+      k_bvsr_search<<<sb, 256, 0, s>>>(W, K, L.KT, V, table, reinterpret_cast<uint32_t*>(P + L.off_tiles));
       break;
     }
     default:
@@ -274,21 +449,22 @@ bq_status bq_quantize_act(const bq_layer* layer, const void* x_bf16, int32_t M, 
   a.h1 = reinterpret_cast<const float*>(P + L.off_aux);
   a.h2 = reinterpret_cast<const float*>(P + L.off_aux2);
   if (L.fmt == BQ_FMT_RABIT2) {
-    k_act_rabit<<<dim3(blocks_for(L.K_pad, 256), M), 256, 0, s>>>(a);
-    return launch_status();
+    return launch_pdl(k_act_rabit, dim3(blocks_for(L.K_pad, 256), M), dim3(256), 0, s, a) == cudaSuccess
+               ? BQ_OK : BQ_ERR_CUDA;
   }
   const int slices_target = std::max(1, std::min(L.KT, (148 + M - 1) / M));
   a.tiles_per_slice = (L.KT + slices_target - 1) / slices_target;
   const int slices = (L.KT + a.tiles_per_slice - 1) / a.tiles_per_slice;
   const dim3 grid(slices, M);
+  cudaError_t e;
   switch (L.fmt) {
-    case BQ_FMT_BITNET_W1A8: k_act_quant<BQ_FMT_BITNET_W1A8><<<grid, 256, 0, s>>>(a); break;
-    case BQ_FMT_TERNARY_A8: k_act_quant<BQ_FMT_TERNARY_A8><<<grid, 256, 0, s>>>(a); break;
-    case BQ_FMT_ABQ: k_act_quant<BQ_FMT_ABQ><<<grid, 256, 0, s>>>(a); break;
-    case BQ_FMT_BVSR4: k_act_quant<BQ_FMT_BVSR4><<<grid, 256, 0, s>>>(a); break;
+    case BQ_FMT_BITNET_W1A8: e = launch_pdl(k_act_quant<BQ_FMT_BITNET_W1A8>, grid, dim3(256), 0, s, a); break;
+    case BQ_FMT_TERNARY_A8: e = launch_pdl(k_act_quant<BQ_FMT_TERNARY_A8>, grid, dim3(256), 0, s, a); break;
+    case BQ_FMT_ABQ: e = launch_pdl(k_act_quant<BQ_FMT_ABQ>, grid, dim3(256), 0, s, a); break;
+    case BQ_FMT_BVSR4: e = launch_pdl(k_act_quant<BQ_FMT_BVSR4>, grid, dim3(256), 0, s, a); break;
     default: return BQ_ERR_INVALID_ARG;
   }
-  return launch_status();
+  return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
 bq_status bq_gemm(const bq_layer* layer, const void* act, int32_t M, float* y, int64_t* acc_dbg, void* stream) {
@@ -300,55 +476,53 @@ bq_status bq_gemm(const bq_layer* layer, const void* act, int32_t M, float* y, i
   if (!act || !aligned(act, 256) || !y || !aligned(y, 4) || (acc_dbg && !aligned(acc_dbg, 8)))
     return BQ_ERR_INVALID_ARG;
   if (L.fmt == BQ_FMT_RABIT2 && acc_dbg) return BQ_ERR_UNSUPPORTED;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const uint8_t* P = static_cast<const uint8_t*>(layer->packed);
   const uint8_t* Ab = static_cast<const uint8_t*>(act);
   const ActLayout A = make_act_layout(L, M);
-  GemvArgs g{};
-  g.tiles = P + L.off_tiles;
-  g.pk_hdr = reinterpret_cast<const uint32_t*>(P);
-  g.row_delta = reinterpret_cast<const float*>(P + L.off_rows);
-  g.row_zero = reinterpret_cast<const int*>(P + L.off_rows) + L.N_pad;
-  g.row_sum = reinterpret_cast<const int*>(P + L.off_rows) + 2 * L.N_pad;
-  g.lora_bt = reinterpret_cast<const uint16_t*>(P + L.off_aux2);
-  g.bvsr_table = reinterpret_cast<const float*>(P + L.off_aux);
-  g.bvsr_idx = P + L.off_aux2;
-  g.rabit_planes = reinterpret_cast<const uint32_t*>(P + L.off_tiles);
-  g.rabit_g = reinterpret_cast<const float*>(P + L.off_rows);
+  LayerArgs g = layer_args(L, layer->packed, M, y, acc_dbg);
   g.act_hdr = reinterpret_cast<const uint32_t*>(Ab);
   g.act_codes = Ab + A.off_codes;
   g.act_tok = reinterpret_cast<const uint32_t*>(Ab + A.off_tok);
-  g.act_u = reinterpret_cast<const float*>(Ab + A.off_u);
+  g.u_part = reinterpret_cast<const float*>(Ab + A.off_u);
   g.act_gsum = reinterpret_cast<const int*>(Ab + A.off_gsum);
   g.act_xt = reinterpret_cast<const float*>(Ab + A.off_xt);
-  g.y = y;
-  g.acc = reinterpret_cast<long long*>(acc_dbg);
-  g.N = L.N; g.K = L.K; g.N_pad = L.N_pad; g.K_pad = L.K_pad; g.KT = L.KT; g.M = M;
-  g.tile_bytes = L.tile_bytes; g.rank = L.fmt == BQ_FMT_TERNARY_A8 ? L.rank : 0; g.fmt = L.fmt;
-  g.shift0 = L.shift[0]; g.shift1 = L.shift[1]; g.shift2 = L.shift[2];
-  const dim3 grid(L.RB, (M + 7) / 8);
-  constexpr int NW = 4;
-  switch (L.fmt) {
-    case BQ_FMT_BITNET_W1A8: k_gemv_mma<BQ_FMT_BITNET_W1A8, 1, 0, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
-    case BQ_FMT_TERNARY_A8: k_gemv_mma<BQ_FMT_TERNARY_A8, 2, 0, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
-    case BQ_FMT_ABQ:
-      switch (L.w_bits) {
-        case 1: k_gemv_mma<BQ_FMT_ABQ, 1, 0, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
-        case 2: k_gemv_mma<BQ_FMT_ABQ, 2, 0, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
-        case 3: k_gemv_mma<BQ_FMT_ABQ, 2, 1, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
-        case 4: k_gemv_mma<BQ_FMT_ABQ, 4, 0, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
-        case 5: k_gemv_mma<BQ_FMT_ABQ, 4, 1, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
-        case 6: k_gemv_mma<BQ_FMT_ABQ, 4, 2, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
-        case 7: k_gemv_mma<BQ_FMT_ABQ, 4, 2, 1, NW><<<grid, NW * 32, 0, s>>>(g); break;
-        case 8: k_gemv_mma<BQ_FMT_ABQ, 8, 0, 0, NW><<<grid, NW * 32, 0, s>>>(g); break;
-        default: return BQ_ERR_INVALID_ARG;
-      }
-      break;
-    case BQ_FMT_BVSR4: k_gemv_bvsr<NW><<<grid, NW * 32, 0, s>>>(g); break;
-    case BQ_FMT_RABIT2: k_gemv_rabit<8><<<blocks_for(L.N, 8), 256, 0, s>>>(g); break;
-    default: return BQ_ERR_INVALID_ARG;
+  return launch_layer(L, g, false, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bq_status bq_linear_workspace_bytes(const bq_layer* layer, int32_t M, size_t* bytes) {
+  PkLayout L;
+  bq_status st = check_layer(layer, &L);
+  if (st != BQ_OK) return st;
+  if (!bytes) return BQ_ERR_INVALID_ARG;
+  if (M < 0 || M > BQ_MAX_M) return BQ_ERR_SIZE;
+  *bytes = size_t(linear_workspace(L, M));
+  return BQ_OK;
+}
+
+bq_status bq_linear(const bq_layer* layer, const void* x_bf16, int32_t M, float* y, int64_t* acc_dbg,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  PkLayout L;
+  bq_status st = check_layer(layer, &L);
+  if (st != BQ_OK) return st;
+  if (M < 0 || M > BQ_MAX_M) return BQ_ERR_SIZE;
+  if (M == 0) return BQ_OK;
+  if (!x_bf16 || !aligned(x_bf16, 16) || !y || !aligned(y, 4) || (acc_dbg && !aligned(acc_dbg, 8)))
+    return BQ_ERR_INVALID_ARG;
+  if (L.fmt == BQ_FMT_RABIT2 && acc_dbg) return BQ_ERR_UNSUPPORTED;
+  const uint64_t need = linear_workspace(L, M);
+  if (need > 0 && (!workspace || !aligned(workspace, 256))) return BQ_ERR_INVALID_ARG;
+  if (workspace_bytes < need) return BQ_ERR_SIZE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint8_t* P = static_cast<const uint8_t*>(layer->packed);
+  LayerArgs g = layer_args(L, layer->packed, M, y, acc_dbg);
+  g.x = static_cast<const uint16_t*>(x_bf16);
+  if (L.fmt == BQ_FMT_TERNARY_A8 && L.rank > 0) {
+    float* up = static_cast<float*>(workspace);
+    if (launch_pdl(k_lora_partial, dim3(L.KT), dim3(256), 0, s, g.x, reinterpret_cast<const uint16_t*>(P + L.off_aux),
+                   M, L.K, L.rank, up) != cudaSuccess)
+      return BQ_ERR_CUDA;
+    g.u_part = up;
   }
-  return launch_status();
+  return launch_layer(L, g, true, s);
 }
 
 bq_status bq_gemv(const bq_layer* layer, const void* act, float* y, int64_t* acc_dbg, void* stream) {

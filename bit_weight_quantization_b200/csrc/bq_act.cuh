@@ -51,12 +51,6 @@ __device__ __forceinline__ void act_write_header(const ActArgs& a) {
   }
 }
 
-// position (in 32-bit words) of the 4 codes k = 4q .. 4q+3 inside a token's k-tile:
-// k_in = 32mu + 16h + 4t + b  ->  word 16t + 2mu + h
-__device__ __forceinline__ int code_word_in_tile(int kin) {
-  const int mu = kin >> 5, h = (kin >> 4) & 1, t = (kin >> 2) & 3;
-  return 16 * t + 2 * mu + h;
-}
 
 __device__ __forceinline__ void load4(const uint16_t* xr, int k, int K, float v[4]) {
   if (k + 3 < K) {
@@ -88,9 +82,10 @@ template <int FMT>
 __global__ void __launch_bounds__(256) k_act_quant(ActArgs a) {
   __shared__ float shf[32];
   __shared__ int shi[32];
-  __shared__ float u_part[8][64];
   const int m = blockIdx.y, slice = blockIdx.x;
   const uint16_t* xr = a.x + size_t(m) * a.K;
+  pdl_trigger();
+  pdl_wait();   // x (and this act buffer) may belong to the previous kernel
   if (slice == 0 && m == 0) act_write_header(a);
 
   // --- per-token scale (whole row) ---
@@ -148,6 +143,16 @@ __global__ void __launch_bounds__(256) k_act_quant(ActArgs a) {
     }
   }
 
+  // --- ternary: partial dot products of x and A over this slice's k-tiles (the LoRA input
+  //     u = SiLU(sum of partials) is formed by the layer kernel) ---
+  if (FMT == BQ_FMT_TERNARY_A8 && a.rank > 0) {
+    float* up = reinterpret_cast<float*>(a.act + a.off_u);
+    for (int i = threadIdx.x; i < (kt1 - kt0) * a.rank; i += blockDim.x) {
+      const int kt = kt0 + i / a.rank, r = i % a.rank;
+      up[(size_t(kt) * a.M + m) * a.rank + r] = lora_tile_dot(xr, a.lora_A, a.K, a.rank, kt, r);
+    }
+  }
+
   if (slice != 0) return;
   // --- per-token parameters: sum of codes over the whole row ---
   int s = 0;
@@ -166,31 +171,12 @@ __global__ void __launch_bounds__(256) k_act_quant(ActArgs a) {
       tok[0] = __float_as_uint(scale); tok[1] = uint32_t(s); tok[2] = 0; tok[3] = 0;
     }
   }
-  // --- ternary: u = SiLU(x A) from the unquantized x ---
-  if (FMT == BQ_FMT_TERNARY_A8 && a.rank > 0) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int r0 = 0; r0 < a.rank; r0 += 32) {
-      const int r = r0 + lane;
-      float acc = 0.f;
-      if (r < a.rank)
-        for (int k = warp; k < a.K; k += 8)
-          acc = fmaf(bf16_bits_to_float(xr[k]), bf16_bits_to_float(a.lora_A[size_t(k) * a.rank + r]), acc);
-      u_part[warp][lane] = acc;
-      __syncthreads();
-      if (warp == 0 && r < a.rank) {
-        float z = 0.f;
-        for (int w = 0; w < 8; w++) z += u_part[w][lane];
-        float* u = reinterpret_cast<float*>(a.act + a.off_u) + size_t(m) * a.rank;
-        u[r] = z / (1.f + expf(-z));
-      }
-      __syncthreads();
-    }
-  }
 }
-
 // RaBiT: xt_p = h_p * x in float32, no quantization.
 __global__ void k_act_rabit(ActArgs a) {
   const int m = blockIdx.y;
+  pdl_trigger();
+  pdl_wait();
   if (blockIdx.x == 0 && m == 0) act_write_header(a);
   const int k = blockIdx.x * blockDim.x + threadIdx.x;
   if (k >= a.K_pad) return;

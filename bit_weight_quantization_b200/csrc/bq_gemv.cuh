@@ -7,13 +7,18 @@
 // registers of one MMA whose bytes are field_value << (f*j). The int8 codes of
 // the activations (whose two's-complement bits are the activation bit-planes)
 // are the B operand, one token per B column. Each field position j keeps its
-// own int32 accumulator; at the end sum_j acc_j >> (f*j) is exactly
-// sum_k field_k * q_k, i.e. sum_b sum_c 2^(b+c) popc(W_b & X_c) over the
-// planes of the stream.
+// own int32 accumulator; sum_j acc_j >> (f*j) is exactly sum_k field_k * q_k,
+// i.e. sum_b sum_c 2^(b+c) popc(W_b & X_c) over the planes of the stream.
 //
-// Work split: CTA = one 16-row block x one group of 8 tokens, its NW warps
-// split the k-tiles; partial sums meet in shared memory, warp 0 runs the
-// fused epilogue (scales, zero points, LoRA term). No cross-CTA reduction.
+// Data movement. A CTA owns one 16-row block and up to 8 tokens; its warps
+// split the k-tiles. At entry each warp starts one bulk (TMA) copy of its
+// contiguous weight slab into shared memory (double-buffered rounds when the
+// slab is large), completing on an mbarrier. The kernel is launched with
+// programmatic dependent launch: it lets the next launch in the stream start at
+// once, and issues only the weight copies (constant data) before
+// griddepcontrol.wait; activations are read after it. The fused variant
+// (bq_linear) runs the activation quantization in the prologue. Partial sums
+// meet in shared memory and warp 0 runs the fused epilogue.
 #pragma once
 
 #include "bq_internal.cuh"
@@ -21,35 +26,55 @@
 namespace bqi {
 
 __device__ unsigned int g_bq_device_error;
+constexpr unsigned int kErrActHeader = 1u;    // act buffer does not match the layer/M
+constexpr unsigned int kErrCopyTimeout = 2u;  // a bulk copy did not complete within the wait bound
+constexpr uint32_t kMaxSpin = 1u << 22;       // try_wait rounds before a wait is abandoned
 
-struct GemvArgs {
-  const uint8_t* tiles;
-  const uint32_t* pk_hdr;
-  const float* row_delta;    // ABQ Delta_w [N_pad]
-  const int* row_zero;       // ABQ z_w
-  const int* row_sum;        // ABQ S_w
-  const uint16_t* lora_bt;   // ternary B^T bf16 [N_pad][r]
-  const float* bvsr_table;   // [256][8]
-  const uint8_t* bvsr_idx;   // [N_pad][K_pad/32]
-  const uint32_t* rabit_planes;
-  const float* rabit_g;      // g1 [N_pad], g2 [N_pad]
-  const uint32_t* act_hdr;
-  const uint8_t* act_codes;
-  const uint32_t* act_tok;
-  const float* act_u;
-  const int* act_gsum;
-  const float* act_xt;
-  float* y;
-  long long* acc;
-  int N, K, N_pad, K_pad, KT, M, tile_bytes, rank, fmt, shift0, shift1, shift2;
-};
-
-// the act buffer must come from bq_quantize_act for this layer and M
-__device__ __forceinline__ bool act_header_ok(const GemvArgs& a) {
-  const uint32_t* h = a.act_hdr;
-  return h[AW_MAGIC] == kActMagic && h[AW_FMT] == uint32_t(a.fmt) && h[AW_M] == uint32_t(a.M) &&
-         h[AW_K] == uint32_t(a.K);
+// ---------------------------------------------------------------------------
+// PTX wrappers: shared addresses, mbarrier, bulk copy, PDL
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+// global -> shared bulk copy; dst and src 16-byte aligned, bytes a multiple of 16
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// bounded wait: false (and the device error word raised) if the phase never completes
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kMaxSpin; i++)
+    if (mbar_try_wait(bar, parity)) return true;
+  atomicOr(&g_bq_device_error, kErrCopyTimeout);
+  return false;
+}
+
+__device__ __forceinline__ uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
 
 template <bool BSIGNED>
 __device__ __forceinline__ void mma_u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -62,14 +87,6 @@ __device__ __forceinline__ void mma_u8(int (&d)[4], uint32_t a0, uint32_t a1, ui
     asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
 }
 
 // B-operand word (mu, h) of this lane's 16 act words (4 uint4, words 2mu+h)
@@ -106,236 +123,529 @@ __device__ __forceinline__ void fold_stream(const int (&acc)[AN][4], int (&p)[4]
   }
 }
 
-template <int FMT, int F0, int F1, int F2, int NW>
-__global__ void __launch_bounds__(NW * 32) k_gemv_mma(GemvArgs a) {
-  constexpr bool BSIGNED = FMT != BQ_FMT_ABQ;
-  __shared__ int red[NW > 1 ? NW - 1 : 1][32][4];
-  __shared__ int bad;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane >> 2, t = lane & 3;
-  const int rb = blockIdx.x, tg = blockIdx.y;
-  if (threadIdx.x == 0) {
-    bad = act_header_ok(a) ? 0 : 1;
-    if (bad) atomicOr(&g_bq_device_error, 1u);
+struct LayerArgs {
+  // packed weights
+  const uint8_t* tiles;
+  const uint32_t* pk_hdr;
+  const float* row_delta;   // ABQ Delta_w [N_pad]
+  const int* row_zero;      // ABQ z_w
+  const int* row_sum;       // ABQ S_w
+  const uint16_t* lora_bt;  // ternary B^T bf16 [N_pad][r]
+  const float* bvsr_table;  // [256][8]
+  const uint32_t* rabit_planes;
+  const float* rabit_g;     // g1 [N_pad], g2 [N_pad]
+  const float* rabit_h1;    // [K_pad]
+  const float* rabit_h2;
+  // activations: x (fused) or the act buffer
+  const uint16_t* x;
+  const uint32_t* act_hdr;
+  const uint8_t* act_codes;
+  const uint32_t* act_tok;
+  const int* act_gsum;
+  const float* act_xt;
+  const float* u_part;      // ternary: partial x.A per 256-k tile [KT][M][r] (act buffer or workspace)
+  float* y;
+  long long* acc;
+  int N, K, N_pad, K_pad, KT, RB, M, tile_bytes, rank, fmt, a_bits, shift0, shift1, shift2;
+  // work split and shared-memory carve, computed on the host:
+  //   T  k-tiles per warp per row block,  C  tiles per ring chunk,  S  ring stages,
+  //   tpc tokens per CTA, TG token groups, CPG CTAs per token group
+  int T, C, S, tpc, TG, CPG, cstride, J;
+  uint32_t off_ring, off_codes, off_tok, off_u, off_gsum, off_tab, off_red, off_bar, smem_bytes;
+};
+
+// ---------------------------------------------------------------------------
+// activation staging into shared memory
+// ---------------------------------------------------------------------------
+constexpr int kMaxXChunks = 16;   // 16-byte chunks of x held in registers per thread
+
+// asymmetric a-bit code: clamp(rn(x / Delta) + z, 0, 2^a - 1)
+__device__ __forceinline__ int quant_asym(float x, float d, int z, int qmax) {
+  long long q = (long long)rintf(__fdiv_rn(x, d)) + z;
+  q = q < 0 ? 0 : q;
+  return int(q > qmax ? qmax : q);
+}
+
+// Reduce v over the TPT consecutive threads of a token group (TPT a power of two, 16..1024):
+// butterfly within the warp, then shared memory across the group's warps. Every thread of
+// the block calls it (it synchronizes); every thread gets its group's result.
+template <typename T, typename Op>
+__device__ __forceinline__ T group_reduce(T v, int TPT, T* sh, Op op) {
+  for (int o = min(16, TPT / 2); o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (TPT > 32) {
+    const int warp = threadIdx.x >> 5, wpg = TPT / 32, g0 = (warp / wpg) * wpg;
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) sh[warp] = v;
+    __syncthreads();
+    v = sh[g0];
+    for (int w = 1; w < wpg; w++) v = op(v, sh[g0 + w]);
+  }
+  return v;
+}
+
+// Round-to-nearest-even of a float32 product p with |p| < 2^22: adding 1.5*2^23 leaves the
+// integer in the low mantissa bits (the byte of the two's-complement code in the low byte).
+__device__ __forceinline__ uint32_t rn_biased(float p) { return __float_as_uint(__fadd_rn(p, 12582912.0f)); }
+constexpr uint32_t kRnBias = 0x4B400000u;
+
+// Fused: each token of this CTA is quantized by a group of TPT threads that hold the
+// token's x in registers (J 16-byte chunks each, loaded at once): per-token scale over
+// the whole row, codes into the fragment-order image (token stride cstride), sum of
+// codes, BVSR vector sums. Token parameters: A8 {gamma, sum q}; ABQ {Delta, z, sum q}.
+template <int FMT, int NW>
+__device__ void stage_quantize(const LayerArgs& a, uint8_t* smem, int m0, int mg) {
+  constexpr int NT = NW * 32;
+  const int tid = threadIdx.x, K = a.K;
+  float* shf = reinterpret_cast<float*>(smem + a.off_red);
+  int* shi = reinterpret_cast<int*>(smem + a.off_red) + 64;
+  int mgp = 1;
+  while (mgp < mg) mgp <<= 1;
+  const int TPT = NT / mgp;
+  const int m = tid / TPT, lt = tid - m * TPT;
+  const bool active = m < mg;
+  const int nch = K / 8, npad = a.K_pad / 8;
+  const uint4* xr = reinterpret_cast<const uint4*>(a.x + size_t(m0 + (active ? m : 0)) * K);
+  uint4 xv[kMaxXChunks];
+#pragma unroll
+  for (int j = 0; j < kMaxXChunks; j++) {
+    const int c = lt + j * TPT;
+    xv[j] = (active && j < a.J && c < nch) ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+  }
+  // pass 1: max|x| (A8) or min/max (ABQ); chunks beyond K are not real elements
+  float p0 = FMT == BQ_FMT_ABQ ? INFINITY : 0.f, p1 = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < kMaxXChunks; j++) {
+    const int c = lt + j * TPT;
+    if (active && j < a.J && c < nch) {
+      const uint32_t w[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
+#pragma unroll
+      for (int h = 0; h < 4; h++) {
+        const float lo = __uint_as_float(w[h] << 16), hi = __uint_as_float(w[h] & 0xFFFF0000u);
+        if (FMT == BQ_FMT_ABQ) { p0 = fminf(p0, fminf(lo, hi)); p1 = fmaxf(p1, fmaxf(lo, hi)); }
+        else p0 = fmaxf(p0, fmaxf(fabsf(lo), fabsf(hi)));
+      }
+    }
+  }
+  float sc = 0.f, d = 1.f;
+  int z = 0;
+  const int qmax = (1 << a.a_bits) - 1;
+  if (FMT == BQ_FMT_ABQ) {
+    p0 = group_reduce(p0, TPT, shf, [](float x, float y) { return fminf(x, y); });
+    p1 = group_reduce(p1, TPT, shf, [](float x, float y) { return fmaxf(x, y); });
+    d = __fdiv_rn(fmaxf(__fsub_rn(p1, p0), 1e-5f), float(qmax));
+    z = int(rintf(__fdiv_rn(-p0, d)));
+  } else {
+    p0 = group_reduce(p0, TPT, shf, [](float x, float y) { return fmaxf(x, y); });
+    sc = p0 > 0.f ? __fdiv_rn(127.f, p0) : 0.f;  // 127/gamma; gamma = 0 gives q = 0
+  }
+  // pass 2: codes, sums. A8: q = rn(x * sc) (|x sc| <= 127 so no clamp is reached);
+  // ABQ: q = clamp(rn(x / Delta) + z, 0, 2^a - 1).
+  uint32_t* cw = reinterpret_cast<uint32_t*>(smem + a.off_codes + size_t(active ? m : 0) * a.cstride);
+  int* gsum = reinterpret_cast<int*>(smem + a.off_gsum);
+  const int VPR = a.K_pad / 32;
+  uint32_t qsum = 0;  // A8: sum of biased codes, modulo 2^32
+  int count = 0;
+#pragma unroll
+  for (int j = 0; j < kMaxXChunks; j++) {
+    if (j >= a.J) break;
+    const int c = lt + j * TPT;
+    const int k = c * 8;
+    uint32_t word0 = 0, word1 = 0;
+    int qs = 0;
+    if (active && c < nch) {
+      const uint32_t w[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
+      uint32_t q8[8];
+#pragma unroll
+      for (int e = 0; e < 8; e++) {
+        const float xf = __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+        if (FMT == BQ_FMT_ABQ) {
+          const int q = quant_asym(xf, d, z, qmax);
+          qs += q;
+          q8[e] = uint32_t(q);
+        } else {
+          q8[e] = rn_biased(__fmul_rn(xf, sc));
+          qs += int(q8[e] - kRnBias);
+        }
+      }
+      word0 = __byte_perm(__byte_perm(q8[0], q8[1], 0x0040), __byte_perm(q8[2], q8[3], 0x0040), 0x5410);
+      word1 = __byte_perm(__byte_perm(q8[4], q8[5], 0x0040), __byte_perm(q8[6], q8[7], 0x0040), 0x5410);
+      count += 8;
+    }
+    if (active && c < npad) {
+      cw[(k >> 8) * 64 + code_word_in_tile(k & 255)] = word0;
+      cw[((k + 4) >> 8) * 64 + code_word_in_tile((k + 4) & 255)] = word1;
+    }
+    qsum += uint32_t(qs);
+    if (FMT == BQ_FMT_BVSR4) {  // 4 consecutive threads cover one 32-element vector
+      qs += __shfl_xor_sync(0xffffffffu, qs, 1);
+      qs += __shfl_xor_sync(0xffffffffu, qs, 2);
+      if (active && c < npad && (c & 3) == 0) gsum[m * VPR + (c >> 2)] = qs;
+    }
+  }
+  (void)count;
+  const int total = group_reduce(int(qsum), TPT, shi, [](int x, int y) { return x + y; });
+  uint32_t* tok = reinterpret_cast<uint32_t*>(smem + a.off_tok);
+  if (active && lt == 0) {
+    if (FMT == BQ_FMT_ABQ) {
+      tok[4 * m + 0] = __float_as_uint(d); tok[4 * m + 1] = uint32_t(z); tok[4 * m + 2] = uint32_t(total);
+    } else {
+      tok[4 * m + 0] = __float_as_uint(p0); tok[4 * m + 1] = uint32_t(total);
+    }
+  }
+}
+
+// Unfused: this CTA's tokens from the act buffer (after checking its header): the codes
+// by one bulk copy per token, token parameters and BVSR sums by plain loads.
+template <int FMT, int NW>
+__device__ bool stage_copy(const LayerArgs& a, uint8_t* smem, int m0, int mg, uint64_t* xbar) {
+  constexpr int NT = NW * 32;
+  int* bad = reinterpret_cast<int*>(smem + a.off_red);
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    const uint32_t* h = a.act_hdr;
+    const int b = !(h[AW_MAGIC] == kActMagic && h[AW_FMT] == uint32_t(a.fmt) && h[AW_M] == uint32_t(a.M) &&
+                    h[AW_K] == uint32_t(a.K));
+    *bad = b;
+    if (b) {
+      atomicOr(&g_bq_device_error, kErrActHeader);
+    } else {
+      const uint32_t per = uint32_t(a.KT) * 256u;
+      mbar_expect_tx(xbar, per * uint32_t(mg));
+      for (int m = 0; m < mg; m++)
+        bulk_g2s(smem + a.off_codes + size_t(m) * a.cstride, a.act_codes + size_t(m0 + m) * per, per, xbar);
+    }
   }
   __syncthreads();
-  if (bad) return;
+  if (*bad) return false;
+  uint32_t* tok = reinterpret_cast<uint32_t*>(smem + a.off_tok);
+  if (tid < 4 * mg) tok[tid] = a.act_tok[4 * m0 + tid];
+  if (FMT == BQ_FMT_BVSR4) {
+    const int VPR = a.K_pad / 32;
+    int* gsum = reinterpret_cast<int*>(smem + a.off_gsum);
+    for (int i = tid; i < mg * VPR; i += NT) gsum[i] = a.act_gsum[size_t(m0) * VPR + i];
+  }
+  return mbar_wait_bounded(xbar, 0);
+}
+
+// Ternary: u[m][r] = SiLU(sum over k-tiles of the partial dot products of x and A),
+// summed in tile order, into shared memory.
+__device__ void stage_lora_u(const LayerArgs& a, uint8_t* smem, int m0, int mg, int NT) {
+  float* us = reinterpret_cast<float*>(smem + a.off_u);
+  for (int i = threadIdx.x; i < mg * a.rank; i += NT) {
+    const int m = i / a.rank, r = i - m * a.rank;
+    float zsum = 0.f;
+    for (int kt = 0; kt < a.KT; kt++) zsum += a.u_part[(size_t(kt) * a.M + m0 + m) * a.rank + r];
+    us[i] = zsum / (1.f + expf(-zsum));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The layer kernel for the tiled formats (BitNet, ternary, ABQ, BVSR).
+// Persistent: CTA c serves token group c % TG and row blocks c / TG + i*CPG.
+// Warp w owns k-tiles [w*T, w*T + T) of every row block; its tiles of successive
+// row blocks stream through an S-stage ring of chunks of C tiles (bulk copies on
+// per-stage mbarriers). After each row block the warps' partial sums meet in a
+// double-buffered shared array and warp (i mod NW) runs the fused epilogue.
+// ---------------------------------------------------------------------------
+template <int FMT, int F0, int F1, int F2, int NW, bool FUSED>
+__global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr bool BSIGNED = FMT != BQ_FMT_ABQ;
+  constexpr bool BVSR = FMT == BQ_FMT_BVSR4;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
+  const int tg = blockIdx.x % a.TG, cg = blockIdx.x / a.TG;
+  const int m0 = tg * a.tpc, mg = min(a.tpc, a.M - m0);
+  const int n_items = cg < a.RB ? (a.RB - cg + a.CPG - 1) / a.CPG : 0;
+
+  // Let the next launch in the stream start; it only prefetches its own weights
+  // before its griddepcontrol.wait.
+  pdl_trigger();
+
+  // ---- weight ring. Packed weights are written only by the pack kernels, which
+  //      never trigger their dependents early, so they are complete here. ----
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.off_bar);
+  uint64_t* wbar = bars + warp * a.S;
+  uint64_t* tbar = bars + NW * a.S;       // BVSR coefficient table
+  uint64_t* xbar = tbar + 1;              // activation codes (unfused path)
+  // This warp's chunks: e = item * cpw + ci, ci < cpw = ceil(nt / C), each non-empty.
+  // Chunk e uses ring stage e mod S in phase (e / S) mod 2.
+  const int kt_begin = warp * a.T;
+  const int nt = max(0, min(a.KT, kt_begin + a.T) - kt_begin);
+  const int cpw = (nt + a.C - 1) / a.C;
+  const int n_my = n_items * cpw;
+  auto chunk_tiles = [&](int e) { return min(a.C, nt - (e % cpw) * a.C); };
+  uint8_t* ring = smem + a.off_ring + size_t(warp) * a.S * a.C * a.tile_bytes;
+  auto issue = [&](int e) {
+    const int st = e % a.S;
+    const int rb = cg + (e / cpw) * a.CPG;
+    const int kt = kt_begin + (e % cpw) * a.C;
+    const uint32_t bytes = uint32_t(chunk_tiles(e)) * uint32_t(a.tile_bytes);
+    mbar_expect_tx(&wbar[st], bytes);
+    bulk_g2s(ring + size_t(st) * a.C * a.tile_bytes, a.tiles + (size_t(rb) * a.KT + kt) * a.tile_bytes, bytes,
+             &wbar[st]);
+  };
+  const int first = min(n_my, a.S);
+  if (lane == 0) {
+    for (int st = 0; st < a.S; st++) mbar_init(&wbar[st], 1);
+    if (warp == 0) { mbar_init(tbar, 1); mbar_init(xbar, 1); }
+    fence_mbar_init();
+    for (int q = 0; q < first; q++) issue(q);
+    if (BVSR && warp == 0) {
+      mbar_expect_tx(tbar, kBvsrSets * kBvsrTableStride * 4);
+      bulk_g2s(smem + a.off_tab, a.bvsr_table, kBvsrSets * kBvsrTableStride * 4, tbar);
+    }
+  }
+  __syncthreads();
+
+  // ---- activations (they may be produced by the previous kernel) ----
+  pdl_wait();
+  bool ok = true;
+  if constexpr (FUSED) stage_quantize<FMT, NW>(a, smem, m0, mg);
+  else ok = stage_copy<FMT, NW>(a, smem, m0, mg, xbar);
+  __syncthreads();
+  if (FMT == BQ_FMT_TERNARY_A8 && a.rank > 0 && ok) stage_lora_u(a, smem, m0, mg, NW * 32);
+  if (BVSR && !mbar_wait_bounded(tbar, 0)) ok = false;
+  __syncthreads();
+
+  const uint32_t* tok = reinterpret_cast<const uint32_t*>(smem + a.off_tok);
+  const bool has_tok = g < mg;
+  const uint8_t* bsrc = smem + a.off_codes + size_t(has_tok ? g : 0) * a.cstride + t * 64;
+  const int VPR = a.K_pad / 32;
+  const int* gsum = reinterpret_cast<const int*>(smem + a.off_gsum);
+  const float* tab = reinterpret_cast<const float*>(smem + a.off_tab);
+  long long* redl = reinterpret_cast<long long*>(smem + a.off_red);                  // [2][NW][32][4]
+  float* redf = reinterpret_cast<float*>(smem + a.off_red + 2 * NW * 32 * 4 * 8);    // [2][NW][32][4]
+  const float tscale = __uint_as_float(a.pk_hdr[HW_TSCALE]);
+  const float lora_gate = FMT == BQ_FMT_TERNARY_A8 ? tanhf(__uint_as_float(a.pk_hdr[HW_LORA_ALPHA])) : 0.f;
+  bool copies_ok = true;
+  int waited = 0, issued = first;  // chunks this warp has waited for / has issued
+  int* fail = reinterpret_cast<int*>(smem + a.off_bar) + 2 * (NW * a.S + 2);  // a copy wait was abandoned
+  if (tid == 0) *fail = 0;
+  __syncthreads();
 
   constexpr int W0 = F0 > 0 ? F0 : 1, A0 = F0 > 0 ? 8 / F0 : 1;
   constexpr int W1 = F1 > 0 ? F1 : 1, A1 = F1 > 0 ? 8 / F1 : 1;
   constexpr int W2 = F2 > 0 ? F2 : 1, A2 = F2 > 0 ? 8 / F2 : 1;
-  uint4 w0[W0], w1[W1], w2[W2];
   int c0[A0][4], c1[A1][4], c2[A2][4];
-#pragma unroll
-  for (int j = 0; j < A0; j++) c0[j][0] = c0[j][1] = c0[j][2] = c0[j][3] = 0;
-#pragma unroll
-  for (int j = 0; j < A1; j++) c1[j][0] = c1[j][1] = c1[j][2] = c1[j][3] = 0;
-#pragma unroll
-  for (int j = 0; j < A2; j++) c2[j][0] = c2[j][1] = c2[j][2] = c2[j][3] = 0;
+  float yacc[4];
+  long long cacc[4];
 
-  const int tok_b = tg * 8 + g;                  // this lane's B column (token)
-  const bool has_tok = tok_b < a.M;
-  const uint4* actp = reinterpret_cast<const uint4*>(a.act_codes) + (size_t(has_tok ? tok_b : 0) * a.KT) * 16 + t * 4;
-  const uint8_t* tbase = a.tiles + size_t(rb) * a.KT * a.tile_bytes + lane * 16;
-
-  for (int kt = warp; kt < a.KT; kt += NW) {
-    const uint8_t* tp = tbase + size_t(kt) * a.tile_bytes;
-    if constexpr (F0 > 0) {
+  for (int item = 0; item < n_items; item++) {
 #pragma unroll
-      for (int u = 0; u < F0; u++) w0[u] = ldg_stream(tp + u * 512);
+    for (int j = 0; j < A0; j++) c0[j][0] = c0[j][1] = c0[j][2] = c0[j][3] = 0;
+#pragma unroll
+    for (int j = 0; j < A1; j++) c1[j][0] = c1[j][1] = c1[j][2] = c1[j][3] = 0;
+#pragma unroll
+    for (int j = 0; j < A2; j++) c2[j][0] = c2[j][1] = c2[j][2] = c2[j][3] = 0;
+#pragma unroll
+    for (int c = 0; c < 4; c++) { yacc[c] = 0.f; cacc[c] = 0; }
+    for (int ci = 0; ci < cpw; ci++) {
+    const int e = item * cpw + ci;
+    const int cnt = chunk_tiles(e);
+    const int st = e % a.S;
+    if (copies_ok) {
+      const bool got = mbar_wait_bounded(&wbar[st], uint32_t((e / a.S) & 1));
+      copies_ok = __all_sync(0xffffffffu, got);
+      if (copies_ok) waited = e + 1;
+      else *fail = 1;
     }
-    if constexpr (F1 > 0) {
+    if (copies_ok && ok) {
+      const uint8_t* sbase = ring + size_t(st) * a.C * a.tile_bytes + lane * 16;
+      const int ktc = kt_begin + ci * a.C;
+      for (int i = 0; i < cnt; i++) {
+        const int kt = ktc + i;
+        const uint8_t* tp = sbase + size_t(i) * a.tile_bytes;
+        uint4 b[4];
 #pragma unroll
-      for (int u = 0; u < F1; u++) w1[u] = ldg_stream(tp + (F0 + u) * 512);
-    }
-    if constexpr (F2 > 0) {
+        for (int qq = 0; qq < 4; qq++) b[qq] = has_tok ? lds128(bsrc + kt * 256 + qq * 16) : make_uint4(0, 0, 0, 0);
+        if constexpr (!BVSR) {
+          uint4 w0[W0], w1[W1], w2[W2];
+          if constexpr (F0 > 0) {
 #pragma unroll
-      for (int u = 0; u < F2; u++) w2[u] = ldg_stream(tp + (F0 + F1 + u) * 512);
-    }
-    uint4 b[4];
+            for (int u = 0; u < F0; u++) w0[u] = lds128(tp + u * 512);
+            stream_mma<F0, BSIGNED>(w0, b, c0);
+          }
+          if constexpr (F1 > 0) {
 #pragma unroll
-    for (int i = 0; i < 4; i++) b[i] = has_tok ? __ldg(actp + size_t(kt) * 16 + i) : make_uint4(0, 0, 0, 0);
-    if constexpr (F0 > 0) stream_mma<F0, BSIGNED>(w0, b, c0);
-    if constexpr (F1 > 0) stream_mma<F1, BSIGNED>(w1, b, c1);
-    if constexpr (F2 > 0) stream_mma<F2, BSIGNED>(w2, b, c2);
-  }
-
-  int p[4] = {0, 0, 0, 0};
-  if constexpr (F0 > 0) fold_stream<F0>(c0, p, a.shift0);
-  if constexpr (F1 > 0) fold_stream<F1>(c1, p, a.shift1);
-  if constexpr (F2 > 0) fold_stream<F2>(c2, p, a.shift2);
-
-  if (NW > 1) {
-    if (warp > 0)
+            for (int u = 0; u < F1; u++) w1[u] = lds128(tp + (F0 + u) * 512);
+            stream_mma<F1, BSIGNED>(w1, b, c1);
+          }
+          if constexpr (F2 > 0) {
 #pragma unroll
-      for (int c = 0; c < 4; c++) red[warp - 1][lane][c] = p[c];
-    __syncthreads();
-    if (warp != 0) return;
-    for (int w = 0; w < NW - 1; w++)
+            for (int u = 0; u < F2; u++) w2[u] = lds128(tp + (F0 + F1 + u) * 512);
+            stream_mma<F2, BSIGNED>(w2, b, c2);
+          }
+        } else {
+          // four 1-bit planes; each 32-k block is one vector per row with its own set
+          uint4 w[4];
 #pragma unroll
-      for (int c = 0; c < 4; c++) p[c] += red[w][lane][c];
-  }
-
-  // fused epilogue: lane holds (row g | g+8) x (token 2t | 2t+1)
-  const float tscale = __uint_as_float(a.pk_hdr[HW_TSCALE]);
+          for (int qq = 0; qq < 4; qq++) w[qq] = lds128(tp + qq * 512);
+          const uint8_t* tidx = tp - lane * 16 + 2048;
+          const uint2 i0 = *reinterpret_cast<const uint2*>(tidx + g * 8);
+          const uint2 i1 = *reinterpret_cast<const uint2*>(tidx + (g + 8) * 8);
 #pragma unroll
-  for (int c = 0; c < 4; c++) {
-    const int row = rb * 16 + g + 8 * (c >> 1);
-    const int tok = tg * 8 + 2 * t + (c & 1);
-    if (row >= a.N || tok >= a.M) continue;
-    const uint32_t* tk = a.act_tok + 4 * tok;
-    long long acc;
-    float yv;
-    if (FMT == BQ_FMT_BITNET_W1A8) {
-      // p = sum_k neg_k q_k  ->  sum_k sign_k q_k = sum q - 2p
-      acc = (long long)int(tk[1]) - 2ll * p[c];
-      yv = __fmul_rn(tscale, __fdiv_rn(__uint_as_float(tk[0]), 127.f)) * float(acc);
-    } else if (FMT == BQ_FMT_TERNARY_A8) {
-      // p = sum_k (T_k + 1) q_k  ->  sum_k T_k q_k = p - sum q
-      acc = (long long)p[c] - (long long)int(tk[1]);
-      yv = __fmul_rn(tscale, __fdiv_rn(__uint_as_float(tk[0]), 127.f)) * float(acc);
-      if (a.rank > 0) {
-        const float* u = a.act_u + size_t(tok) * a.rank;
-        const uint16_t* bt = a.lora_bt + size_t(row) * a.rank;
-        float l = 0.f;
-        for (int r = 0; r < a.rank; r++) l = fmaf(u[r], bf16_bits_to_float(bt[r]), l);
-        yv += tanhf(__uint_as_float(a.pk_hdr[HW_LORA_ALPHA])) * l;
+          for (int j = 0; j < 8; j++) {
+            const uint32_t msk = (1u << j) * 0x01010101u;
+            int d[4][4];
+#pragma unroll
+            for (int qq = 0; qq < 4; qq++) {
+              d[qq][0] = d[qq][1] = d[qq][2] = d[qq][3] = 0;
+              mma_u8<true>(d[qq], w[qq].x & msk, w[qq].y & msk, w[qq].z & msk, w[qq].w & msk, bword(b, j, 0),
+                           bword(b, j, 1));
+            }
+            const int s0 = int(((j < 4 ? i0.x : i0.y) >> (8 * (j & 3))) & 0xFFu);
+            const int s1 = int(((j < 4 ? i1.x : i1.y) >> (8 * (j & 3))) & 0xFFu);
+            const int kv = kt * 8 + j;
+            const float gs0 = 2 * t < mg ? float(gsum[2 * t * VPR + kv]) : 0.f;
+            const float gs1 = 2 * t + 1 < mg ? float(gsum[(2 * t + 1) * VPR + kv]) : 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; c++) {
+              const float* row = tab + ((c >> 1) ? s1 : s0) * kBvsrTableStride;
+              // integer templates R_i of the set's ratio (1.5, 2, 2.5, 3): c_i = sc R_i
+              const int ri = int(row[6]);
+              const uint32_t R = ri == 0 ? 0x1B120C08u : ri == 1 ? 0x08040201u : ri == 2 ? 0x7D321408u : 0x1B090301u;
+              const int E = (int(R & 0xFF) * d[0][c] + int((R >> 8) & 0xFF) * d[1][c] +
+                             int((R >> 16) & 0xFF) * d[2][c] + int(R >> 24) * d[3][c]) >> j;
+              yacc[c] = fmaf(row[5], float(E), fmaf(row[4], (c & 1) ? gs1 : gs0, yacc[c]));
+              if (a.acc) cacc[c] += (d[0][c] + 2 * d[1][c] + 4 * d[2][c] + 8 * d[3][c]) >> j;
+            }
+          }
+        }
       }
+    }
+    __syncwarp();
+    if (copies_ok && e + a.S < n_my) {
+      if (lane == 0) {
+        fence_proxy_async();  // this stage's shared reads are done before the copy overwrites it
+        issue(e + a.S);
+      }
+      issued = e + a.S + 1;
+    }
+    }
+
+    // ---- end of a row block: cross-warp sum and fused epilogue ----
+    const int buf = item & 1;
+    long long p[4] = {0, 0, 0, 0};
+    if constexpr (!BVSR) {
+      int pi[4] = {0, 0, 0, 0};
+      if constexpr (F0 > 0) fold_stream<F0>(c0, pi, a.shift0);
+      if constexpr (F1 > 0) fold_stream<F1>(c1, pi, a.shift1);
+      if constexpr (F2 > 0) fold_stream<F2>(c2, pi, a.shift2);
+#pragma unroll
+      for (int c = 0; c < 4; c++) p[c] = pi[c];
     } else {
-      // ABQ: I = P - z_x S_w - z_w S_x + K z_w z_x
-      const long long zx = int(tk[1]), sx = int(tk[2]);
-      const long long zw = a.row_zero[row], sw = a.row_sum[row];
-      acc = (long long)p[c] - zx * sw - zw * sx + (long long)a.K * zw * zx;
-      yv = __fmul_rn(a.row_delta[row], __uint_as_float(tk[0])) * float(acc);
+#pragma unroll
+      for (int c = 0; c < 4; c++) p[c] = cacc[c];
     }
-    a.y[size_t(tok) * a.N + row] = yv;
-    if (a.acc) a.acc[size_t(tok) * a.N + row] = acc;
-  }
-}
-
-// ---------------------------------------------------------------------------
-// BVSR: four 1-bit planes; every 32-k MMA block is one vector per row, with its
-// own coefficient set, so each tile folds its planes immediately:
-//   y += (gamma_x/127) [ sc_s (sum_i R_i T_i) + o_s S_v ],  T_i = acc_i >> j
-// (c_i = sc_s R_i for the integer ratio templates R of set s).
-// ---------------------------------------------------------------------------
-template <int NW>
-__global__ void __launch_bounds__(NW * 32) k_gemv_bvsr(GemvArgs a) {
-  __shared__ float tab_sc[kBvsrSets], tab_o[kBvsrSets];
-  __shared__ uint32_t tab_r[kBvsrSets];
-  __shared__ float redf[NW > 1 ? NW - 1 : 1][32][4];
-  __shared__ long long redl[NW > 1 ? NW - 1 : 1][32][4];
-  __shared__ int bad;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane >> 2, t = lane & 3;
-  const int rb = blockIdx.x, tg = blockIdx.y;
-  if (threadIdx.x == 0) {
-    bad = act_header_ok(a) ? 0 : 1;
-    if (bad) atomicOr(&g_bq_device_error, 1u);
-  }
-  for (int s = threadIdx.x; s < kBvsrSets; s += blockDim.x) {
-    const float* row = a.bvsr_table + s * kBvsrTableStride;
-    tab_sc[s] = row[5];
-    tab_o[s] = row[4];
-    const int j = int(row[6]);
-    // integer templates R_i (ratio 1.5, 2, 2.5, 3), one byte each
-    const uint32_t R[4] = {0x1B120C08u, 0x08040201u, 0x7D321408u, 0x1B090301u};
-    tab_r[s] = R[j & 3];
-  }
-  __syncthreads();
-  if (bad) return;
-
-  const int tok_b = tg * 8 + g;
-  const bool has_tok = tok_b < a.M;
-  const uint4* actp = reinterpret_cast<const uint4*>(a.act_codes) + (size_t(has_tok ? tok_b : 0) * a.KT) * 16 + t * 4;
-  const uint8_t* tbase = a.tiles + size_t(rb) * a.KT * 2048 + lane * 16;
-  const int VPR = a.K_pad / 32;
-  const int row0 = rb * 16 + g, row1 = row0 + 8;
-  const int tokc[2] = {tg * 8 + 2 * t, tg * 8 + 2 * t + 1};
-  float yacc[4] = {0.f, 0.f, 0.f, 0.f};
-  long long cacc[4] = {0, 0, 0, 0};
-
-  for (int kt = warp; kt < a.KT; kt += NW) {
-    const uint8_t* tp = tbase + size_t(kt) * 2048;
-    uint4 w[4];
+    long long* rl = redl + ((buf * NW + warp) * 32 + lane) * 4;
 #pragma unroll
-    for (int i = 0; i < 4; i++) w[i] = ldg_stream(tp + i * 512);
-    uint4 b[4];
+    for (int c = 0; c < 4; c++) rl[c] = p[c];
+    if (BVSR) {
+      float* rf = redf + ((buf * NW + warp) * 32 + lane) * 4;
 #pragma unroll
-    for (int i = 0; i < 4; i++) b[i] = has_tok ? __ldg(actp + size_t(kt) * 16 + i) : make_uint4(0, 0, 0, 0);
-    const uint2 i0 = *reinterpret_cast<const uint2*>(a.bvsr_idx + size_t(row0) * VPR + kt * 8);
-    const uint2 i1 = *reinterpret_cast<const uint2*>(a.bvsr_idx + size_t(row1) * VPR + kt * 8);
-    int gs[2][8];
-#pragma unroll
-    for (int h = 0; h < 2; h++) {
-      if (tokc[h] < a.M) {
-        const int4* gp = reinterpret_cast<const int4*>(a.act_gsum + size_t(tokc[h]) * VPR + kt * 8);
-        const int4 x0 = gp[0], x1 = gp[1];
-        gs[h][0] = x0.x; gs[h][1] = x0.y; gs[h][2] = x0.z; gs[h][3] = x0.w;
-        gs[h][4] = x1.x; gs[h][5] = x1.y; gs[h][6] = x1.z; gs[h][7] = x1.w;
-      } else {
-#pragma unroll
-        for (int j = 0; j < 8; j++) gs[h][j] = 0;
-      }
+      for (int c = 0; c < 4; c++) rf[c] = yacc[c];
     }
-#pragma unroll
-    for (int j = 0; j < 8; j++) {
-      const uint32_t m = (1u << j) * 0x01010101u;
-      int d[4][4];
-#pragma unroll
-      for (int i = 0; i < 4; i++) {
-        d[i][0] = d[i][1] = d[i][2] = d[i][3] = 0;
-        mma_u8<true>(d[i], w[i].x & m, w[i].y & m, w[i].z & m, w[i].w & m, bword(b, j, 0), bword(b, j, 1));
-      }
-      const int s0 = int(((j < 4 ? i0.x : i0.y) >> (8 * (j & 3))) & 0xFFu);
-      const int s1 = int(((j < 4 ? i1.x : i1.y) >> (8 * (j & 3))) & 0xFFu);
-#pragma unroll
-      for (int c = 0; c < 4; c++) {
-        const int s = (c >> 1) ? s1 : s0;
-        const uint32_t R = tab_r[s];
-        const int E = (int(R & 0xFF) * d[0][c] + int((R >> 8) & 0xFF) * d[1][c] +
-                       int((R >> 16) & 0xFF) * d[2][c] + int(R >> 24) * d[3][c]) >> j;
-        yacc[c] = fmaf(tab_sc[s], float(E), fmaf(tab_o[s], float(gs[c & 1][j]), yacc[c]));
-        if (a.acc) cacc[c] += (d[0][c] + 2 * d[1][c] + 4 * d[2][c] + 8 * d[3][c]) >> j;
-      }
-    }
-  }
-
-  if (NW > 1) {
-    if (warp > 0)
-#pragma unroll
-      for (int c = 0; c < 4; c++) { redf[warp - 1][lane][c] = yacc[c]; redl[warp - 1][lane][c] = cacc[c]; }
     __syncthreads();
-    if (warp != 0) return;
-    for (int w = 0; w < NW - 1; w++)
+    if (warp != item % NW || !ok || *fail) continue;
+    const int rb = cg + item * a.CPG;
+    long long pl[4] = {0, 0, 0, 0};
+    float yl[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int w = 0; w < NW; w++) {
+      const long long* r2 = redl + ((buf * NW + w) * 32 + lane) * 4;
 #pragma unroll
-      for (int c = 0; c < 4; c++) { yacc[c] += redf[w][lane][c]; cacc[c] += redl[w][lane][c]; }
+      for (int c = 0; c < 4; c++) pl[c] += r2[c];
+      if (BVSR) {
+        const float* f2 = redf + ((buf * NW + w) * 32 + lane) * 4;
+#pragma unroll
+        for (int c = 0; c < 4; c++) yl[c] += f2[c];
+      }
+    }
+    // lane holds (row g | g+8) x (token 2t | 2t+1)
+#pragma unroll
+    for (int c = 0; c < 4; c++) {
+      const int row = rb * 16 + g + 8 * (c >> 1);
+      const int tl = 2 * t + (c & 1);
+      const int tok_i = m0 + tl;
+      if (row >= a.N || tl >= mg) continue;
+      const uint32_t* tk = tok + 4 * tl;
+      long long acc;
+      float yv;
+      if (FMT == BQ_FMT_BITNET_W1A8) {
+        // p = sum_k neg_k q_k  ->  sum_k sign_k q_k = sum q - 2p
+        acc = (long long)int(tk[1]) - 2ll * pl[c];
+        yv = __fmul_rn(tscale, __fdiv_rn(__uint_as_float(tk[0]), 127.f)) * float(acc);
+      } else if (FMT == BQ_FMT_TERNARY_A8) {
+        // p = sum_k (T_k + 1) q_k  ->  sum_k T_k q_k = p - sum q
+        acc = pl[c] - (long long)int(tk[1]);
+        yv = __fmul_rn(tscale, __fdiv_rn(__uint_as_float(tk[0]), 127.f)) * float(acc);
+        if (a.rank > 0) {
+          const float* u = reinterpret_cast<const float*>(smem + a.off_u) + size_t(tl) * a.rank;
+          const uint4* bt = reinterpret_cast<const uint4*>(a.lora_bt + size_t(row) * a.rank);
+          float l = 0.f;
+          for (int q8 = 0; q8 < a.rank / 8; q8++) {
+            const uint4 v = __ldg(bt + q8);
+            const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 8; e++)
+              l = fmaf(u[q8 * 8 + e], __uint_as_float((e & 1) ? (h[e >> 1] & 0xFFFF0000u) : (h[e >> 1] << 16)), l);
+          }
+          yv += lora_gate * l;
+        }
+      } else if (FMT == BQ_FMT_ABQ) {
+        // I = P - z_x S_w - z_w S_x + K z_w z_x
+        const long long zx = int(tk[1]), sx = int(tk[2]);
+        const long long zw = a.row_zero[row], sw = a.row_sum[row];
+        acc = pl[c] - zx * sw - zw * sx + (long long)a.K * zw * zx;
+        yv = __fmul_rn(a.row_delta[row], __uint_as_float(tk[0])) * float(acc);
+      } else {
+        acc = pl[c];
+        yv = __fdiv_rn(__uint_as_float(tk[0]), 127.f) * yl[c];
+      }
+      a.y[size_t(tok_i) * a.N + row] = yv;
+      if (a.acc) a.acc[size_t(tok_i) * a.N + row] = acc;
+    }
   }
-#pragma unroll
-  for (int c = 0; c < 4; c++) {
-    const int row = rb * 16 + g + 8 * (c >> 1);
-    const int tok = tokc[c & 1];
-    if (row >= a.N || tok >= a.M) continue;
-    const float gx = __uint_as_float(a.act_tok[4 * tok]);
-    a.y[size_t(tok) * a.N + row] = __fdiv_rn(gx, 127.f) * yacc[c];
-    if (a.acc) a.acc[size_t(tok) * a.N + row] = cacc[c];
+  // copies issued but never waited for (an abandoned wait) must land before the block exits
+  if (!copies_ok)
+    for (int e = waited; e < issued; e++) (void)mbar_wait_bounded(&wbar[e % a.S], uint32_t((e / a.S) & 1));
+}
+
+// ---------------------------------------------------------------------------
+// Ternary LoRA input (fused path): partial dot products of the unquantized bf16 x
+// with A over each 256-k tile, out[kt][m][r], each summed in k order (the act kernel
+// computes the same partials for the unfused path). Grid: one CTA per k-tile.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_lora_partial(const uint16_t* __restrict__ x, const uint16_t* __restrict__ A,
+                                                      int M, int K, int rank, float* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
+  const int kt = blockIdx.x;
+  for (int i = threadIdx.x; i < M * rank; i += blockDim.x) {
+    const int m = i / rank, r = i - m * rank;
+    out[(size_t(kt) * M + m) * rank + r] = lora_tile_dot(x + size_t(m) * K, A, K, rank, kt, r);
   }
 }
 
 // ---------------------------------------------------------------------------
-// RaBiT: fp32 sign-apply, y = g1 sum_k (-1)^B1 x~1 + g2 sum_k (-1)^B2 x~2 with
-// x~p = h_p x; the sign bit of x~ is flipped by XOR with the plane bit.
-// One warp per row; lane l takes k = 32w + l.
+// RaBiT: fp32 sign-apply, y = g1 sum_k (-1)^B1 h1 x + g2 sum_k (-1)^B2 h2 x; the
+// sign bit of h_p x is flipped by XOR with the plane bit. One warp per row,
+// lane l takes k = 32w + l. Fused: reads x and h; else the act buffer's h_p x.
 // ---------------------------------------------------------------------------
-template <int NW>
-__global__ void __launch_bounds__(NW * 32) k_gemv_rabit(GemvArgs a) {
+template <int NW, bool FUSED>
+__global__ void __launch_bounds__(NW * 32) k_rabit(LayerArgs a) {
   __shared__ int bad;
-  if (threadIdx.x == 0) {
-    bad = act_header_ok(a) ? 0 : 1;
-    if (bad) atomicOr(&g_bq_device_error, 1u);
+  pdl_trigger();
+  pdl_wait();
+  if (!FUSED) {
+    if (threadIdx.x == 0) {
+      const uint32_t* h = a.act_hdr;
+      bad = !(h[AW_MAGIC] == kActMagic && h[AW_FMT] == uint32_t(a.fmt) && h[AW_M] == uint32_t(a.M) &&
+              h[AW_K] == uint32_t(a.K));
+      if (bad) atomicOr(&g_bq_device_error, kErrActHeader);
+    }
+    __syncthreads();
+    if (bad) return;
   }
-  __syncthreads();
-  if (bad) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int row = blockIdx.x * NW + warp;
   if (row >= a.N) return;
@@ -343,14 +653,21 @@ __global__ void __launch_bounds__(NW * 32) k_gemv_rabit(GemvArgs a) {
   const uint32_t* p1 = a.rabit_planes + size_t(row) * W32;
   const uint32_t* p2 = a.rabit_planes + (size_t(a.N_pad) + row) * W32;
   for (int m = 0; m < a.M; m++) {
-    const float* x1 = a.act_xt + size_t(m) * a.K_pad;
-    const float* x2 = a.act_xt + (size_t(a.M) + m) * a.K_pad;
     float acc1 = 0.f, acc2 = 0.f;
     for (int wd = 0; wd < W32; wd++) {
       const uint32_t b1 = __ldg(p1 + wd), b2 = __ldg(p2 + wd);
       const int k = wd * 32 + lane;
-      acc1 += __uint_as_float(__float_as_uint(__ldg(x1 + k)) ^ (((b1 >> lane) & 1u) << 31));
-      acc2 += __uint_as_float(__float_as_uint(__ldg(x2 + k)) ^ (((b2 >> lane) & 1u) << 31));
+      float x1, x2;
+      if (FUSED) {
+        const float xv = k < a.K ? bf16_bits_to_float(a.x[size_t(m) * a.K + k]) : 0.f;
+        x1 = __fmul_rn(__ldg(a.rabit_h1 + k), xv);
+        x2 = __fmul_rn(__ldg(a.rabit_h2 + k), xv);
+      } else {
+        x1 = __ldg(a.act_xt + size_t(m) * a.K_pad + k);
+        x2 = __ldg(a.act_xt + (size_t(a.M) + m) * a.K_pad + k);
+      }
+      acc1 += __uint_as_float(__float_as_uint(x1) ^ (((b1 >> lane) & 1u) << 31));
+      acc2 += __uint_as_float(__float_as_uint(x2) ^ (((b2 >> lane) & 1u) << 31));
     }
     acc1 = warp_sum(acc1);
     acc2 = warp_sum(acc2);

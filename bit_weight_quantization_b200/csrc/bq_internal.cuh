@@ -34,6 +34,7 @@ enum : int {
 
 constexpr int kBvsrSets = 256;
 constexpr int kBvsrTableStride = 8;  // floats per set: c0 c1 c2 c3 o sc ratio_index 0
+constexpr int kBvsrTileBytes = 4 * 512 + 16 * 8;
 
 struct PkLayout {
   int fmt, N, K, N_pad, K_pad, RB, KT, w_bits, a_bits, nstreams;
@@ -91,9 +92,8 @@ inline bool make_pk_layout(int fmt, int N, int K, int w_bits, int a_bits, int ra
     case BQ_FMT_BVSR4:
       l.w_bits = 4; l.a_bits = 8; l.nstreams = 4;
       for (int s = 0; s < 4; s++) { l.field[s] = 1; l.shift[s] = s; }
-      l.tile_bytes = 2048;
+      l.tile_bytes = kBvsrTileBytes;  // 4 planes x 512 B, then the 16 x 8 set indices
       aux = uint64_t(kBvsrSets) * kBvsrTableStride * 4;
-      aux2 = uint64_t(l.N_pad) * (l.K_pad / 32);
       break;
     default:
       return false;
@@ -115,7 +115,7 @@ inline ActLayout make_act_layout(const PkLayout& L, int M) {
   uint64_t codes = L.fmt == BQ_FMT_RABIT2 ? 0 : uint64_t(M) * L.KT * 256;
   uint64_t tok = uint64_t(M) * 16;
   uint64_t gsum = L.fmt == BQ_FMT_BVSR4 ? uint64_t(M) * (L.K_pad / 32) * 4 : 0;
-  uint64_t u = uint64_t(M) * a.rank * 4;
+  uint64_t u = uint64_t(L.KT) * M * a.rank * 4;   // LoRA partials [KT][M][r]
   uint64_t xt = L.fmt == BQ_FMT_RABIT2 ? 2ull * M * L.K_pad * 4 : 0;
   a.off_codes = 256;
   a.off_tok = align256(a.off_codes + codes);
@@ -133,6 +133,29 @@ inline bool layout_from_layer(const bq_layer* y, PkLayout* L) {
 // ---------------------------------------------------------------------------
 // device helpers
 // ---------------------------------------------------------------------------
+
+// Programmatic dependent launch: let the next kernel in the stream launch, and
+// wait until the previous one has completed and its writes are visible.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
+// Position (in 32-bit words) of the 4 activation codes k_in .. k_in+3 inside a
+// token's 256-k tile in B-fragment order: k_in = 32mu + 16h + 4t + b -> word 16t + 2mu + h.
+__device__ __forceinline__ int code_word_in_tile(int kin) {
+  const int mu = kin >> 5, h = (kin >> 4) & 1, t = (kin >> 2) & 3;
+  return 16 * t + 2 * mu + h;
+}
+
+// Partial dot product of one token's bf16 x with column r of the bf16 LoRA matrix
+// A [K_pad][rank] over the 256-k tile kt, accumulated in k order (f32).
+__device__ __forceinline__ float lora_tile_dot(const uint16_t* xr, const uint16_t* A, int K, int rank, int kt,
+                                               int r) {
+  float acc = 0.f;
+  const int k1 = min(K, kt * 256 + 256);
+  for (int k = kt * 256; k < k1; k++)
+    acc = fmaf(__uint_as_float(uint32_t(xr[k]) << 16), __uint_as_float(uint32_t(A[size_t(k) * rank + r]) << 16), acc);
+  return acc;
+}
 
 // Order-preserving map of a float to uint32 (total order on non-NaN values).
 __device__ __forceinline__ uint32_t float_key(float f) {

@@ -336,9 +336,8 @@ __device__ __forceinline__ int bvsr_nearest(double w, const double P[16], double
 }
 
 // One block of 256 threads (thread = set) per vector, grid-stride over vectors.
-__global__ void __launch_bounds__(256) k_bvsr_search(const float* __restrict__ W, int K, int K_pad, int KT,
-                                                     uint64_t V, const float* __restrict__ table,
-                                                     uint32_t* __restrict__ tiles32, uint8_t* __restrict__ setidx) {
+__global__ void __launch_bounds__(256) k_bvsr_search(const float* __restrict__ W, int K, int KT, uint64_t V,
+                                                     const float* __restrict__ table, uint32_t* __restrict__ tiles32) {
   __shared__ float wv[32];
   __shared__ double red_e[8];
   __shared__ int red_s[8];
@@ -395,7 +394,8 @@ __global__ void __launch_bounds__(256) k_bvsr_search(const float* __restrict__ W
       const int kt = kv >> 3, j = kv & 7;
       const int e = lane, rh = e >> 4, t = (e >> 2) & 3, b = e & 3;
       const int r = 2 * rh + rbit, tl = 4 * g + t;
-      const uint64_t base_w = (uint64_t(rb) * KT + kt) * (2048 / 4) + tl * 4 + r;
+      const uint64_t tile_w = (uint64_t(rb) * KT + kt) * (kBvsrTileBytes / 4);
+      const uint64_t base_w = tile_w + tl * 4 + r;
 #pragma unroll
       for (int i = 0; i < 4; i++) {
         uint32_t val = uint32_t((code >> i) & 1) << (8 * b + j);
@@ -403,7 +403,8 @@ __global__ void __launch_bounds__(256) k_bvsr_search(const float* __restrict__ W
         val |= __shfl_xor_sync(0xffffffffu, val, 2);
         if (b == 0 && val) atomicOr(&tiles32[base_w + i * 128], val);
       }
-      if (lane == 0) setidx[n * (K_pad / 32) + kv] = uint8_t(sbest);
+      // set index of (row rho, vector j of the tile) at byte 2048 + 8 rho + j of the tile
+      if (lane == 0) reinterpret_cast<uint8_t*>(tiles32 + tile_w)[2048 + rho * 8 + j] = uint8_t(sbest);
     }
   }
 }

@@ -22,6 +22,7 @@
  *   bq_packed_bytes / bq_pack_weights   quantize + pack W into a self-describing buffer
  *   bq_act_bytes / bq_quantize_act      per-token activation quantization
  *   bq_gemv (M = 1) / bq_gemm (M >= 1)  the layer, fused scale/zero-point/LoRA epilogue
+ *   bq_linear                           activation quantization + layer in one kernel (decode)
  *
  * Ownership: the caller allocates every buffer (device memory for packed, act, W, x, y);
  * sizes come from the *_bytes queries. The library never allocates, frees or
@@ -56,14 +57,16 @@
  *   Padding rows/columns hold zero fields (ternary: field 1, i.e. T = 0).
  *   Streams: BitNet 1 x f=1 (bit set <=> sign -1). Ternary 1 x f=2 (field = T+1 in {0,1,2}).
  *   ABQ: w_bits split into fields of 8/4/2/1 bits from the low end (2:[2] 4:[4] 6:[4,2]
- *   8:[8], shift = bit offset in the code). BVSR: 4 x f=1, stream i = bitvector plane i.
+ *   8:[8], shift = bit offset in the code). BVSR: 4 x f=1, stream i = bitvector plane i,
+ *   and each BVSR tile ends with 128 bytes of set indices: byte 2048 + 8g + j is the set of
+ *   row 16rb + g, vector 8kt + j (a vector is 32 contiguous k), so tile_bytes = 2176.
  * RaBiT (format 1) is not tiled: bit j of uint32 off_tiles + 4((p*N_pad + n)(K_pad/32) + w)
  *   is the sign of path p (0,1), row n, k = 32w + j (1 <=> -1).
  * Sections: RaBiT rows = g1[N_pad], g2[N_pad] f32; aux = h1[K_pad], aux2 = h2[K_pad] f32.
  *   Ternary aux = A bf16 [K_pad][r], aux2 = B^T bf16 [N_pad][r].
  *   ABQ rows = Delta_w f32 [N_pad], z_w i32 [N_pad], S_w = sum_k q_w i32 [N_pad].
  *   BVSR aux = coefficient table f32 [256][8] (c0 c1 c2 c3 o; then derived kernel constants:
- *   sc = (hi-lo)/sum_i R_i, ratio index, 0); aux2 = set index u8 [N_pad][K_pad/32].
+ *   sc = (hi-lo)/sum_i R_i, ratio index, 0).
  *
  * Activation buffer (device, 256-byte aligned), version 1.
  * Header: 64 x 32-bit words: 0 magic 0x43415142 ('BQAC') 1 version 2 format 3 M 4 K 5 K_pad
@@ -75,7 +78,8 @@
  *   the activation bit-planes X_c, uint8 for ABQ). Padding k hold code 0.
  * tok [M][4] words: A8 {gamma_x f32, sum_k q i32, 0, 0}; ABQ {Delta_x f32, z_x i32, S_x i32, 0}.
  * gsum (BVSR): i32 [M][K_pad/32], sum of q over each 32-element vector.
- * u (ternary): f32 [M][r] = SiLU(x A) from the unquantized bf16 x.
+ * u (ternary): f32 [K_pad/256][M][r] partial dot products of the unquantized bf16 x with A
+ *   over each 256-k tile (each in k order); the layer forms SiLU(sum over tiles).
  * xt (RaBiT): f32 [2][M][K_pad] = h_p * x (no activation quantization).
  */
 #ifndef BQ_H
@@ -118,7 +122,7 @@ typedef struct {
   int32_t fmt;          /* bq_format */
   int32_t w_bits;       /* ABQ weight bits, 1..8 (ignored by the other formats) */
   int32_t a_bits;       /* ABQ activation bits, 1..8 (ignored: the A8 formats use 8) */
-  int32_t lora_rank;    /* ternary: rank r of the correction, 0..64 (0 = none) */
+  int32_t lora_rank;    /* ternary: rank r of the correction, 0..64, a multiple of 8 (0 = none) */
   float lora_alpha;     /* ternary: gate alpha; the correction is scaled by tanh(alpha) */
   const float* h2;      /* RaBiT: device f32 [K], second-path input scale (h1 = 1) */
   const float* lora_A;  /* ternary: device f32 [K][r] row-major, rounded to bf16 */
@@ -173,6 +177,18 @@ bq_status bq_gemv(const bq_layer* layer, const void* act, float* y, int64_t* acc
                   void* stream);
 bq_status bq_gemm(const bq_layer* layer, const void* act, int32_t M, float* y,
                   int64_t* acc_dbg, void* stream);
+
+/* Fused layer for decode: the activation quantization of bq_quantize_act runs inside the
+ * layer kernel's prologue, so y [M][N] f32 comes from x (device bf16 [M][K], 16-byte
+ * aligned) in one launch (two for the ternary format with a LoRA term, whose
+ * partial dot products of x and A are computed first into `workspace`). Results are identical to
+ * bq_quantize_act + bq_gemm. `workspace` (device, 256-byte aligned) must hold
+ * bq_linear_workspace_bytes(layer, M) bytes; it may be NULL when that is 0.
+ * Launched with programmatic dependent launch: consecutive layer calls on one stream
+ * overlap the next layer's weight fetch with the current layer. */
+bq_status bq_linear_workspace_bytes(const bq_layer* layer, int32_t M, size_t* bytes);
+bq_status bq_linear(const bq_layer* layer, const void* x_bf16, int32_t M, float* y, int64_t* acc_dbg,
+                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronizes the current device, then reads and clears the device error word:
  * BQ_OK or BQ_ERR_DEVICE_CHECK. */

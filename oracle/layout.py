@@ -33,6 +33,9 @@ the f-bit field j (bits f*j .. f*j+f-1) of byte b holds the weight at
   row = 16*rb + g + 8*(r & 1)
   k   = 32*(8*kt + u*(8/f) + j) + 16*(r >> 1) + 4*t + b.
 
+BVSR tiles (4 one-bit planes of 512 B) end with 128 bytes of set indices: byte
+2048 + 8*g + j holds the set of row 16*rb + g, vector 8*kt + j (32 elements each).
+
 RaBiT (format 1) is not tiled: plane p (0,1) word w of row n is the uint32 at
 off_tiles + 4*((p*N_pad + n)*(K_pad/32) + w), bit j <-> k = 32w + j; a set bit
 means sign -1.
@@ -170,8 +173,13 @@ def read_packed(buf: bytes, row_blocks=None) -> dict:
         tab = np.frombuffer(buf, dtype="<f4", count=256 * 8, offset=h["off_aux"]).reshape(256, 8)
         out["table"] = tab[:, :5].copy()
         out["table_derived"] = tab[:, 5:].copy()
-        sets = np.frombuffer(buf, dtype=np.uint8, count=N_pad * (K_pad // 32), offset=h["off_aux2"])
-        out["sets"] = sets.reshape(N_pad, K_pad // 32)[sel, :K // 32].copy()
+        # set index of (row g of the tile, vector j of the tile) at byte 2048 + 8 g + j of the tile
+        RB, KT, tb = N_pad // 16, K_pad // 256, h["tile_bytes"]
+        raw = np.frombuffer(buf, dtype=np.uint8, count=RB * KT * tb, offset=h["off_tiles"]).reshape(RB, KT, tb)
+        rbs = np.arange(RB) if rb is None else np.asarray(rb)
+        idx = raw[rbs][:, :, 2048:2048 + 128].reshape(len(rbs), KT, 16, 8)
+        sets = idx.transpose(0, 2, 1, 3).reshape(16 * len(rbs), K_pad // 32)
+        out["sets"] = (sets[:N] if rb is None else sets)[:, :K // 32].copy()
     else:
         raise ValueError(f"unknown format {fmt}")
     return out
@@ -194,7 +202,8 @@ def _bf16_to_f32(u16: np.ndarray) -> np.ndarray:
 #   k = 32*(8*kt + mu) + 16*h + 4*t + b   (int8 for A8 formats, uint8 for ABQ).
 # tok: [M][4] words: A8 {gamma_x f32, sum_q i32, 0, 0}; ABQ {Delta_x f32, z_x i32, S_x i32, 0}
 # gsum (BVSR): int32 [M][K_pad/32] sums of q over each 32-element vector
-# u (ternary): float32 [M][lora_rank] = SiLU(x A)
+# u (ternary): float32 [KT][M][lora_rank] partial dot products of x and A over each
+#   256-k tile; the layer's LoRA input is SiLU(sum over tiles)
 # xt (RaBiT): float32 [2][M][K_pad] = h_p * x
 
 
@@ -230,6 +239,6 @@ def read_act(buf: bytes) -> dict:
         a["gsum"] = np.frombuffer(buf, dtype="<i4", count=M * (K_pad // 32),
                                   offset=a["off_gsum"]).reshape(M, K_pad // 32)[:, :K // 32].copy()
     if fmt == FMT_TERNARY and a["lora_rank"] > 0:
-        a["u"] = np.frombuffer(buf, dtype="<f4", count=M * a["lora_rank"],
-                               offset=a["off_u"]).reshape(M, a["lora_rank"]).copy()
+        r = a["lora_rank"]
+        a["u_part"] = np.frombuffer(buf, dtype="<f4", count=KT * M * r, offset=a["off_u"]).reshape(KT, M, r).copy()
     return a

@@ -123,14 +123,14 @@ def _host_header(fmt, N, K, **kw):
     for i, f in enumerate(fields):
         h[10 + i], h[14 + i] = f, (i if fmt == "bvsr" else sh)
         sh += f
-    h[18] = 512 * sum(fields)
+    h[18] = 512 * sum(fields) + (128 if fmt == "bvsr" else 0)
     h[19] = kw.get("lora_rank", 0)
     tiles = (N_pad // 16) * (K_pad // 256) * h[18]
     rows = 3 * N_pad * 4 if fmt == "abq" else 0
     a256 = lambda v: (v + 255) // 256 * 256
     off_rows = a256(256 + tiles)
     aux = {"ternary": K_pad * h[19] * 2, "bvsr": 256 * 8 * 4}.get(fmt, 0)
-    aux2 = {"ternary": N_pad * h[19] * 2, "bvsr": N_pad * (K_pad // 32)}.get(fmt, 0)
+    aux2 = {"ternary": N_pad * h[19] * 2}.get(fmt, 0)
     off_aux = a256(off_rows + rows)
     off_aux2 = a256(off_aux + aux)
     for word, v in [(22, total), (24, 256), (26, off_rows), (28, off_aux), (30, off_aux2)]:

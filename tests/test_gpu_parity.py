@@ -14,7 +14,8 @@ from tests.parity_util import GpuLayer, assert_y_close, check_act, oracle_layer,
 
 pytestmark = pytest.mark.gpu
 
-SMALL = [(16, 256), (50, 384), (97, 640), (33, 128)]
+# ragged N and K; (40, 2560) leaves some warps without k-tiles, (24, 6144) streams in chunks
+SMALL = [(16, 256), (50, 384), (97, 640), (33, 128), (40, 2560), (24, 6144)]
 ABQ_WA = [(2, 8), (4, 4), (6, 6), (8, 8), (1, 3), (3, 5), (5, 2), (7, 7)]
 
 
@@ -70,7 +71,7 @@ def test_small_parity(fmt, N, K, M):
 
 
 @pytest.mark.parametrize("wa", ABQ_WA)
-@pytest.mark.parametrize("N,K,M", [(50, 384, 1), (97, 640, 9), (16, 256, 8)])
+@pytest.mark.parametrize("N,K,M", [(50, 384, 1), (97, 640, 9), (16, 256, 8), (64, 6400, 2)])
 def test_small_parity_abq(wa, N, K, M):
     w, a = wa
     gl = GpuLayer("abq", N, K, M, seed=w * 10 + a, w_bits=w, a_bits=a)
