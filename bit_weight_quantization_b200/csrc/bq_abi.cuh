@@ -183,7 +183,12 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   g->tpc = tpc;
   g->TG = (M + tpc - 1) / tpc;
   g->CPG = std::max(1, std::min(L.RB, (sm_count() + g->TG - 1) / g->TG));
-  g->T = (L.KT + NW - 1) / NW;
+  // warps sharing a row block: as many as the CTA's row blocks leave idle
+  const int ipc = (L.RB + g->CPG - 1) / g->CPG;
+  int wpr = 1;
+  while (wpr * 2 <= NW && wpr * 2 * ipc <= NW) wpr *= 2;
+  g->WPR = wpr;
+  g->T = (L.KT + wpr - 1) / wpr;
   uint64_t off = 0;
   auto take = [&](uint64_t bytes) {
     const uint32_t o = uint32_t(off);
@@ -191,7 +196,7 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
     return o;
   };
   g->off_codes = take(uint64_t(tpc) * g->cstride);
-  g->off_tok = take(8 * 4 * 4);
+  g->off_tok = take(bqi::kTokWords * 4);  // per-token words, tanh(alpha), weight scale
   g->off_u = take(rank > 0 ? uint64_t(tpc) * rank * 4 : 16);
   g->off_gsum = take(bvsr ? uint64_t(tpc) * VPR * 4 : 16);
   g->off_tab = take(bvsr ? uint64_t(kBvsrSets) * kBvsrTableStride * 4 : 16);
@@ -199,11 +204,11 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   const uint64_t fixed = off + 1024;  // + barriers
   const uint64_t limit = 220 * 1024;
   const uint64_t budget = std::min<uint64_t>(96 * 1024, fixed < limit ? limit - fixed : 0);
-  const uint64_t per_tile = uint64_t(NW) * L.tile_bytes;   // one tile for every warp
-  if (budget < 2 * per_tile) return false;
-  g->C = int(std::max<uint64_t>(1, std::min<uint64_t>(g->T, budget / (3 * per_tile))));
-  g->S = int(std::max<uint64_t>(2, std::min<uint64_t>(4, budget / (per_tile * g->C))));
-  g->off_ring = take(per_tile * g->C * g->S);
+  const uint64_t per_warp = budget / NW;
+  if (per_warp < 2ull * L.tile_bytes) return false;
+  g->S = int(std::min<uint64_t>(4, std::max<uint64_t>(2, per_warp / L.tile_bytes)));
+  g->C = int(std::max<uint64_t>(1, std::min<uint64_t>(g->T, per_warp / (uint64_t(g->S) * L.tile_bytes))));
+  g->off_ring = take(uint64_t(NW) * g->S * g->C * L.tile_bytes);
   g->off_bar = take(uint64_t(NW * g->S + 2) * 8 + 16);
   g->smem_bytes = uint32_t(off);
   g->RB = L.RB;

@@ -149,8 +149,9 @@ struct LayerArgs {
   int N, K, N_pad, K_pad, KT, RB, M, tile_bytes, rank, fmt, a_bits, shift0, shift1, shift2;
   // work split and shared-memory carve, computed on the host:
   //   T  k-tiles per warp per row block,  C  tiles per ring chunk,  S  ring stages,
-  //   tpc tokens per CTA, TG token groups, CPG CTAs per token group
-  int T, C, S, tpc, TG, CPG, cstride, J;
+  //   tpc tokens per CTA, TG token groups, CPG CTAs per token group,
+  //   WPR warps sharing one row block (the k-split), a power of two dividing NW
+  int T, C, S, tpc, TG, CPG, WPR, cstride, J;
   uint32_t off_ring, off_codes, off_tok, off_u, off_gsum, off_tab, off_red, off_bar, smem_bytes;
 };
 
@@ -158,6 +159,8 @@ struct LayerArgs {
 // activation staging into shared memory
 // ---------------------------------------------------------------------------
 constexpr int kMaxXChunks = 16;   // 16-byte chunks of x held in registers per thread
+// shared token area (words): [8][4] per-token parameters, then tanh(alpha) and the weight scale
+constexpr int kTokAlpha = 32, kTokWScale = 33, kTokWords = 36;
 
 // asymmetric a-bit code: clamp(rn(x / Delta) + z, 0, 2^a - 1)
 __device__ __forceinline__ int quant_asym(float x, float d, int z, int qmax) {
@@ -167,14 +170,14 @@ __device__ __forceinline__ int quant_asym(float x, float d, int z, int qmax) {
 }
 
 // Reduce v over the TPT consecutive threads of a token group (TPT a power of two, 16..1024):
-// butterfly within the warp, then shared memory across the group's warps. Every thread of
-// the block calls it (it synchronizes); every thread gets its group's result.
+// butterfly within the warp, then, for groups wider than a warp, one exchange through
+// sh[warp] (each call needs its own sh). Every thread of the block calls it; every
+// thread gets its group's result.
 template <typename T, typename Op>
 __device__ __forceinline__ T group_reduce(T v, int TPT, T* sh, Op op) {
   for (int o = min(16, TPT / 2); o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
   if (TPT > 32) {
     const int warp = threadIdx.x >> 5, wpg = TPT / 32, g0 = (warp / wpg) * wpg;
-    __syncthreads();
     if ((threadIdx.x & 31) == 0) sh[warp] = v;
     __syncthreads();
     v = sh[g0];
@@ -188,6 +191,28 @@ __device__ __forceinline__ T group_reduce(T v, int TPT, T* sh, Op op) {
 __device__ __forceinline__ uint32_t rn_biased(float p) { return __float_as_uint(__fadd_rn(p, 12582912.0f)); }
 constexpr uint32_t kRnBias = 0x4B400000u;
 
+// L2 prefetch of this CTA's x rows, issued before griddepcontrol.wait. It only warms L2
+// (the coherent point for the previous kernel's writes); every read of x happens after the wait.
+__device__ __forceinline__ void prefetch_x(const LayerArgs& a, int m0, int mg, int NT) {
+  const char* base = reinterpret_cast<const char*>(a.x + size_t(m0) * a.K);
+  const int lines = (mg * a.K * 2 + 127) / 128;
+  for (int i = threadIdx.x; i < lines; i += NT) asm volatile("prefetch.global.L2 [%0];" ::"l"(base + size_t(i) * 128));
+}
+
+// Output scale of a token (slot 3 of its parameters): BitNet alpha gamma/127, ternary
+// gamma_W gamma/127, BVSR gamma/127, ABQ Delta_x (times Delta_w per row in the epilogue).
+// tw is the layer's weight scale (header word HW_TSCALE), read before griddepcontrol.wait.
+template <int FMT>
+__device__ __forceinline__ uint32_t token_scale(float tw, uint32_t word0) {
+  const float g0 = __uint_as_float(word0);
+  float sc;
+  if (FMT == BQ_FMT_BITNET_W1A8 || FMT == BQ_FMT_TERNARY_A8)
+    sc = __fmul_rn(tw, __fdiv_rn(g0, 127.f));
+  else if (FMT == BQ_FMT_BVSR4) sc = __fdiv_rn(g0, 127.f);
+  else sc = g0;
+  return __float_as_uint(sc);
+}
+
 // Fused: each token of this CTA is quantized by a group of TPT threads that hold the
 // token's x in registers (J 16-byte chunks each, loaded at once): per-token scale over
 // the whole row, codes into the fragment-order image (token stride cstride), sum of
@@ -196,8 +221,9 @@ template <int FMT, int NW>
 __device__ void stage_quantize(const LayerArgs& a, uint8_t* smem, int m0, int mg) {
   constexpr int NT = NW * 32;
   const int tid = threadIdx.x, K = a.K;
-  float* shf = reinterpret_cast<float*>(smem + a.off_red);
-  int* shi = reinterpret_cast<int*>(smem + a.off_red) + 64;
+  float* sh_lo = reinterpret_cast<float*>(smem + a.off_red);   // three separate exchange slots
+  float* sh_hi = sh_lo + 32;
+  int* sh_sum = reinterpret_cast<int*>(sh_lo + 64);
   int mgp = 1;
   while (mgp < mg) mgp <<= 1;
   const int TPT = NT / mgp;
@@ -230,12 +256,12 @@ __device__ void stage_quantize(const LayerArgs& a, uint8_t* smem, int m0, int mg
   int z = 0;
   const int qmax = (1 << a.a_bits) - 1;
   if (FMT == BQ_FMT_ABQ) {
-    p0 = group_reduce(p0, TPT, shf, [](float x, float y) { return fminf(x, y); });
-    p1 = group_reduce(p1, TPT, shf, [](float x, float y) { return fmaxf(x, y); });
+    p0 = group_reduce(p0, TPT, sh_lo, [](float x, float y) { return fminf(x, y); });
+    p1 = group_reduce(p1, TPT, sh_hi, [](float x, float y) { return fmaxf(x, y); });
     d = __fdiv_rn(fmaxf(__fsub_rn(p1, p0), 1e-5f), float(qmax));
     z = int(rintf(__fdiv_rn(-p0, d)));
   } else {
-    p0 = group_reduce(p0, TPT, shf, [](float x, float y) { return fmaxf(x, y); });
+    p0 = group_reduce(p0, TPT, sh_lo, [](float x, float y) { return fmaxf(x, y); });
     sc = p0 > 0.f ? __fdiv_rn(127.f, p0) : 0.f;  // 127/gamma; gamma = 0 gives q = 0
   }
   // pass 2: codes, sums. A8: q = rn(x * sc) (|x sc| <= 127 so no clamp is reached);
@@ -243,8 +269,7 @@ __device__ void stage_quantize(const LayerArgs& a, uint8_t* smem, int m0, int mg
   uint32_t* cw = reinterpret_cast<uint32_t*>(smem + a.off_codes + size_t(active ? m : 0) * a.cstride);
   int* gsum = reinterpret_cast<int*>(smem + a.off_gsum);
   const int VPR = a.K_pad / 32;
-  uint32_t qsum = 0;  // A8: sum of biased codes, modulo 2^32
-  int count = 0;
+  uint32_t qsum = 0;  // A8: sum of codes, from the biased floats, modulo 2^32
 #pragma unroll
   for (int j = 0; j < kMaxXChunks; j++) {
     if (j >= a.J) break;
@@ -269,7 +294,6 @@ __device__ void stage_quantize(const LayerArgs& a, uint8_t* smem, int m0, int mg
       }
       word0 = __byte_perm(__byte_perm(q8[0], q8[1], 0x0040), __byte_perm(q8[2], q8[3], 0x0040), 0x5410);
       word1 = __byte_perm(__byte_perm(q8[4], q8[5], 0x0040), __byte_perm(q8[6], q8[7], 0x0040), 0x5410);
-      count += 8;
     }
     if (active && c < npad) {
       cw[(k >> 8) * 64 + code_word_in_tile(k & 255)] = word0;
@@ -282,8 +306,7 @@ __device__ void stage_quantize(const LayerArgs& a, uint8_t* smem, int m0, int mg
       if (active && c < npad && (c & 3) == 0) gsum[m * VPR + (c >> 2)] = qs;
     }
   }
-  (void)count;
-  const int total = group_reduce(int(qsum), TPT, shi, [](int x, int y) { return x + y; });
+  const int total = group_reduce(int(qsum), TPT, sh_sum, [](int x, int y) { return x + y; });
   uint32_t* tok = reinterpret_cast<uint32_t*>(smem + a.off_tok);
   if (active && lt == 0) {
     if (FMT == BQ_FMT_ABQ) {
@@ -291,6 +314,7 @@ __device__ void stage_quantize(const LayerArgs& a, uint8_t* smem, int m0, int mg
     } else {
       tok[4 * m + 0] = __float_as_uint(p0); tok[4 * m + 1] = uint32_t(total);
     }
+    tok[4 * m + 3] = token_scale<FMT>(__uint_as_float(tok[kTokWScale]), tok[4 * m + 0]);
   }
 }
 
@@ -318,7 +342,8 @@ __device__ bool stage_copy(const LayerArgs& a, uint8_t* smem, int m0, int mg, ui
   __syncthreads();
   if (*bad) return false;
   uint32_t* tok = reinterpret_cast<uint32_t*>(smem + a.off_tok);
-  if (tid < 4 * mg) tok[tid] = a.act_tok[4 * m0 + tid];
+  const float tw = __uint_as_float(tok[kTokWScale]);
+  if (tid < 4 * mg) tok[tid] = (tid & 3) == 3 ? token_scale<FMT>(tw, a.act_tok[4 * m0 + tid - 3]) : a.act_tok[4 * m0 + tid];
   if (FMT == BQ_FMT_BVSR4) {
     const int VPR = a.K_pad / 32;
     int* gsum = reinterpret_cast<int*>(smem + a.off_gsum);
@@ -339,13 +364,87 @@ __device__ void stage_lora_u(const LayerArgs& a, uint8_t* smem, int m0, int mg, 
   }
 }
 
+// Fused epilogue for one 16-row block: lane holds (row g | g+8) x (token 2t | 2t+1).
+// tok[4m + 3] holds the token's output scale (alpha gamma/127, gamma_W gamma/127,
+// gamma/127 or Delta_x).
+// Per-row ABQ parameters of a row block's rows g and g + 8 (Delta_w, z_w, S_w), loaded
+// ahead of the block's tiles so the epilogue does not wait on them.
+struct RowP {
+  float d[2];
+  int z[2], s[2];
+};
+template <int FMT>
+__device__ __forceinline__ void load_rowp(const LayerArgs& a, int rb, int lane, RowP& rp) {
+  if constexpr (FMT == BQ_FMT_ABQ) {
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+      const int row = rb * 16 + (lane >> 2) + 8 * h;  // < N_pad: the arrays are padded
+      rp.d[h] = __ldg(a.row_delta + row);
+      rp.z[h] = __ldg(a.row_zero + row);
+      rp.s[h] = __ldg(a.row_sum + row);
+    }
+  }
+}
+
+template <int FMT>
+__device__ __forceinline__ void layer_epilogue(const LayerArgs& a, const uint8_t* smem, const uint32_t* tok, int rb,
+                                               int m0, int mg, int lane, const RowP& rp, const long long (&pl)[4],
+                                               const float (&yl)[4]) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int c = 0; c < 4; c++) {
+    const int row = rb * 16 + g + 8 * (c >> 1);
+    const int tl = 2 * t + (c & 1);
+    if (row >= a.N || tl >= mg) continue;
+    const uint32_t* tk = tok + 4 * tl;
+    const float scale = __uint_as_float(tk[3]);
+    long long acc;
+    float yv;
+    if (FMT == BQ_FMT_BITNET_W1A8) {
+      // p = sum_k neg_k q_k  ->  sum_k sign_k q_k = sum q - 2p
+      acc = (long long)int(tk[1]) - 2ll * pl[c];
+      yv = scale * float(acc);
+    } else if (FMT == BQ_FMT_TERNARY_A8) {
+      // p = sum_k (T_k + 1) q_k  ->  sum_k T_k q_k = p - sum q
+      acc = pl[c] - (long long)int(tk[1]);
+      yv = scale * float(acc);
+      if (a.rank > 0) {
+        const float* u = reinterpret_cast<const float*>(smem + a.off_u) + size_t(tl) * a.rank;
+        const uint4* bt = reinterpret_cast<const uint4*>(a.lora_bt + size_t(row) * a.rank);
+        float l = 0.f;
+        for (int q8 = 0; q8 < a.rank / 8; q8++) {
+          const uint4 v = __ldg(bt + q8);
+          const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 8; e++)
+            l = fmaf(u[q8 * 8 + e], __uint_as_float((e & 1) ? (h[e >> 1] & 0xFFFF0000u) : (h[e >> 1] << 16)), l);
+        }
+        yv += __uint_as_float(reinterpret_cast<const uint32_t*>(smem + a.off_tok)[kTokAlpha]) * l;  // tanh(alpha)
+      }
+    } else if (FMT == BQ_FMT_ABQ) {
+      // I = P - z_x S_w - z_w S_x + K z_w z_x
+      const long long zx = int(tk[1]), sx = int(tk[2]);
+      const long long zw = rp.z[c >> 1], sw = rp.s[c >> 1];
+      acc = pl[c] - zx * sw - zw * sx + (long long)a.K * zw * zx;
+      yv = __fmul_rn(rp.d[c >> 1], scale) * float(acc);
+    } else {
+      acc = pl[c];
+      yv = scale * yl[c];
+    }
+    a.y[size_t(m0 + tl) * a.N + row] = yv;
+    if (a.acc) a.acc[size_t(m0 + tl) * a.N + row] = acc;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // The layer kernel for the tiled formats (BitNet, ternary, ABQ, BVSR).
-// Persistent: CTA c serves token group c % TG and row blocks c / TG + i*CPG.
-// Warp w owns k-tiles [w*T, w*T + T) of every row block; its tiles of successive
-// row blocks stream through an S-stage ring of chunks of C tiles (bulk copies on
-// per-stage mbarriers). After each row block the warps' partial sums meet in a
-// double-buffered shared array and warp (i mod NW) runs the fused epilogue.
+// Persistent: CTA c serves token group c % TG and row blocks c / TG + i*CPG. Its
+// warps form G = NW/WPR groups of WPR warps; group gr takes the CTA's row blocks
+// gr, gr + G, ..., and warp w of a group owns k-tiles [w*T, w*T + T) of each. A
+// warp's tiles stream through its own S-stage ring of C-tile chunks (bulk copies on
+// per-stage mbarriers). A group's partial sums meet in shared memory behind that
+// group's named barrier (none when WPR = 1) and one of its warps runs the fused
+// epilogue: after the prologue there is no block-wide synchronization.
 // ---------------------------------------------------------------------------
 template <int FMT, int F0, int F1, int F2, int NW, bool FUSED>
 __global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
@@ -355,73 +454,83 @@ __global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
   const int tg = blockIdx.x % a.TG, cg = blockIdx.x / a.TG;
   const int m0 = tg * a.tpc, mg = min(a.tpc, a.M - m0);
-  const int n_items = cg < a.RB ? (a.RB - cg + a.CPG - 1) / a.CPG : 0;
+  const int n_items = cg < a.RB ? (a.RB - cg + a.CPG - 1) / a.CPG : 0;  // row blocks of this CTA
+  const int WPR = a.WPR, G = NW / WPR;
+  const int grp = warp / WPR, wg = warp - grp * WPR;
+  const int n_gitems = grp < n_items ? (n_items - grp + G - 1) / G : 0;  // row blocks of this group
 
   // Let the next launch in the stream start; it only prefetches its own weights
   // before its griddepcontrol.wait.
   pdl_trigger();
 
   // ---- weight ring. Packed weights are written only by the pack kernels, which
-  //      never trigger their dependents early, so they are complete here. ----
+  //      never trigger their dependents early, so they are complete here.
+  //      This warp's chunks: e = gi * cpw + ci (gi-th row block of the group, ci < cpw),
+  //      each non-empty; chunk e uses ring stage e mod S in phase (e / S) mod 2. ----
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.off_bar);
   uint64_t* wbar = bars + warp * a.S;
-  uint64_t* tbar = bars + NW * a.S;       // BVSR coefficient table
-  uint64_t* xbar = tbar + 1;              // activation codes (unfused path)
-  // This warp's chunks: e = item * cpw + ci, ci < cpw = ceil(nt / C), each non-empty.
-  // Chunk e uses ring stage e mod S in phase (e / S) mod 2.
-  const int kt_begin = warp * a.T;
+  uint64_t* tbar = bars + NW * a.S;  // BVSR coefficient table
+  uint64_t* xbar = tbar + 1;         // activation codes (unfused path)
+  const int kt_begin = wg * a.T;
   const int nt = max(0, min(a.KT, kt_begin + a.T) - kt_begin);
   const int cpw = (nt + a.C - 1) / a.C;
-  const int n_my = n_items * cpw;
+  const int n_my = n_gitems * cpw;
   auto chunk_tiles = [&](int e) { return min(a.C, nt - (e % cpw) * a.C); };
+  auto rb_of = [&](int gi) { return cg + (grp + gi * G) * a.CPG; };
   uint8_t* ring = smem + a.off_ring + size_t(warp) * a.S * a.C * a.tile_bytes;
   auto issue = [&](int e) {
     const int st = e % a.S;
-    const int rb = cg + (e / cpw) * a.CPG;
     const int kt = kt_begin + (e % cpw) * a.C;
     const uint32_t bytes = uint32_t(chunk_tiles(e)) * uint32_t(a.tile_bytes);
     mbar_expect_tx(&wbar[st], bytes);
-    bulk_g2s(ring + size_t(st) * a.C * a.tile_bytes, a.tiles + (size_t(rb) * a.KT + kt) * a.tile_bytes, bytes,
-             &wbar[st]);
+    bulk_g2s(ring + size_t(st) * a.C * a.tile_bytes,
+             a.tiles + (size_t(rb_of(e / cpw)) * a.KT + kt) * a.tile_bytes, bytes, &wbar[st]);
   };
   const int first = min(n_my, a.S);
   if (lane == 0) {
     for (int st = 0; st < a.S; st++) mbar_init(&wbar[st], 1);
     if (warp == 0) { mbar_init(tbar, 1); mbar_init(xbar, 1); }
     fence_mbar_init();
-    for (int q = 0; q < first; q++) issue(q);
+    for (int e = 0; e < first; e++) issue(e);
     if (BVSR && warp == 0) {
       mbar_expect_tx(tbar, kBvsrSets * kBvsrTableStride * 4);
       bulk_g2s(smem + a.off_tab, a.bvsr_table, kBvsrSets * kBvsrTableStride * 4, tbar);
     }
   }
+  if constexpr (FUSED) prefetch_x(a, m0, mg, NW * 32);
+  int* fail = reinterpret_cast<int*>(smem + a.off_bar) + 2 * (NW * a.S + 2);  // a copy wait was abandoned
+  if (tid == 0) {
+    *fail = 0;
+    uint32_t* tw = reinterpret_cast<uint32_t*>(smem + a.off_tok);
+    tw[kTokWScale] = a.pk_hdr[HW_TSCALE];
+    if (FMT == BQ_FMT_TERNARY_A8) tw[kTokAlpha] = __float_as_uint(tanhf(__uint_as_float(a.pk_hdr[HW_LORA_ALPHA])));
+  }
+  RowP rp;
+  if (n_gitems > 0) load_rowp<FMT>(a, rb_of(0), lane, rp);
   __syncthreads();
 
   // ---- activations (they may be produced by the previous kernel) ----
   pdl_wait();
   bool ok = true;
+  const uint32_t* tokp = reinterpret_cast<const uint32_t*>(smem + a.off_tok);
   if constexpr (FUSED) stage_quantize<FMT, NW>(a, smem, m0, mg);
   else ok = stage_copy<FMT, NW>(a, smem, m0, mg, xbar);
   __syncthreads();
-  if (FMT == BQ_FMT_TERNARY_A8 && a.rank > 0 && ok) stage_lora_u(a, smem, m0, mg, NW * 32);
+  if (FMT == BQ_FMT_TERNARY_A8 && a.rank > 0) {
+    if (ok) stage_lora_u(a, smem, m0, mg, NW * 32);
+    __syncthreads();
+  }
   if (BVSR && !mbar_wait_bounded(tbar, 0)) ok = false;
-  __syncthreads();
 
-  const uint32_t* tok = reinterpret_cast<const uint32_t*>(smem + a.off_tok);
   const bool has_tok = g < mg;
   const uint8_t* bsrc = smem + a.off_codes + size_t(has_tok ? g : 0) * a.cstride + t * 64;
   const int VPR = a.K_pad / 32;
   const int* gsum = reinterpret_cast<const int*>(smem + a.off_gsum);
   const float* tab = reinterpret_cast<const float*>(smem + a.off_tab);
-  long long* redl = reinterpret_cast<long long*>(smem + a.off_red);                  // [2][NW][32][4]
-  float* redf = reinterpret_cast<float*>(smem + a.off_red + 2 * NW * 32 * 4 * 8);    // [2][NW][32][4]
-  const float tscale = __uint_as_float(a.pk_hdr[HW_TSCALE]);
-  const float lora_gate = FMT == BQ_FMT_TERNARY_A8 ? tanhf(__uint_as_float(a.pk_hdr[HW_LORA_ALPHA])) : 0.f;
+  long long* redl = reinterpret_cast<long long*>(smem + a.off_red);                // [G][2][WPR][32][4]
+  float* redf = reinterpret_cast<float*>(smem + a.off_red + 2 * NW * 32 * 4 * 8);  // same shape
   bool copies_ok = true;
   int waited = 0, issued = first;  // chunks this warp has waited for / has issued
-  int* fail = reinterpret_cast<int*>(smem + a.off_bar) + 2 * (NW * a.S + 2);  // a copy wait was abandoned
-  if (tid == 0) *fail = 0;
-  __syncthreads();
 
   constexpr int W0 = F0 > 0 ? F0 : 1, A0 = F0 > 0 ? 8 / F0 : 1;
   constexpr int W1 = F1 > 0 ? F1 : 1, A1 = F1 > 0 ? 8 / F1 : 1;
@@ -430,7 +539,8 @@ __global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
   float yacc[4];
   long long cacc[4];
 
-  for (int item = 0; item < n_items; item++) {
+  for (int gi = 0; gi < n_gitems; gi++) {
+    if (gi > 0) load_rowp<FMT>(a, rb_of(gi), lane, rp);
 #pragma unroll
     for (int j = 0; j < A0; j++) c0[j][0] = c0[j][1] = c0[j][2] = c0[j][3] = 0;
 #pragma unroll
@@ -440,92 +550,91 @@ __global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
 #pragma unroll
     for (int c = 0; c < 4; c++) { yacc[c] = 0.f; cacc[c] = 0; }
     for (int ci = 0; ci < cpw; ci++) {
-    const int e = item * cpw + ci;
-    const int cnt = chunk_tiles(e);
-    const int st = e % a.S;
-    if (copies_ok) {
-      const bool got = mbar_wait_bounded(&wbar[st], uint32_t((e / a.S) & 1));
-      copies_ok = __all_sync(0xffffffffu, got);
-      if (copies_ok) waited = e + 1;
-      else *fail = 1;
-    }
-    if (copies_ok && ok) {
-      const uint8_t* sbase = ring + size_t(st) * a.C * a.tile_bytes + lane * 16;
-      const int ktc = kt_begin + ci * a.C;
-      for (int i = 0; i < cnt; i++) {
-        const int kt = ktc + i;
-        const uint8_t* tp = sbase + size_t(i) * a.tile_bytes;
-        uint4 b[4];
+      const int e = gi * cpw + ci;
+      const int cnt = chunk_tiles(e);
+      const int st = e % a.S;
+      if (copies_ok) {
+        const bool got = mbar_wait_bounded(&wbar[st], uint32_t((e / a.S) & 1));
+        copies_ok = __all_sync(0xffffffffu, got);
+        if (copies_ok) waited = e + 1;
+        else *fail = 1;
+      }
+      if (copies_ok && ok) {
+        const uint8_t* sbase = ring + size_t(st) * a.C * a.tile_bytes + lane * 16;
+        const int ktc = kt_begin + ci * a.C;
+        for (int i = 0; i < cnt; i++) {
+          const int kt = ktc + i;
+          const uint8_t* tp = sbase + size_t(i) * a.tile_bytes;
+          uint4 b[4];
 #pragma unroll
-        for (int qq = 0; qq < 4; qq++) b[qq] = has_tok ? lds128(bsrc + kt * 256 + qq * 16) : make_uint4(0, 0, 0, 0);
-        if constexpr (!BVSR) {
-          uint4 w0[W0], w1[W1], w2[W2];
-          if constexpr (F0 > 0) {
+          for (int qq = 0; qq < 4; qq++) b[qq] = has_tok ? lds128(bsrc + kt * 256 + qq * 16) : make_uint4(0, 0, 0, 0);
+          if constexpr (!BVSR) {
+            uint4 w0[W0], w1[W1], w2[W2];
+            if constexpr (F0 > 0) {
 #pragma unroll
-            for (int u = 0; u < F0; u++) w0[u] = lds128(tp + u * 512);
-            stream_mma<F0, BSIGNED>(w0, b, c0);
-          }
-          if constexpr (F1 > 0) {
-#pragma unroll
-            for (int u = 0; u < F1; u++) w1[u] = lds128(tp + (F0 + u) * 512);
-            stream_mma<F1, BSIGNED>(w1, b, c1);
-          }
-          if constexpr (F2 > 0) {
-#pragma unroll
-            for (int u = 0; u < F2; u++) w2[u] = lds128(tp + (F0 + F1 + u) * 512);
-            stream_mma<F2, BSIGNED>(w2, b, c2);
-          }
-        } else {
-          // four 1-bit planes; each 32-k block is one vector per row with its own set
-          uint4 w[4];
-#pragma unroll
-          for (int qq = 0; qq < 4; qq++) w[qq] = lds128(tp + qq * 512);
-          const uint8_t* tidx = tp - lane * 16 + 2048;
-          const uint2 i0 = *reinterpret_cast<const uint2*>(tidx + g * 8);
-          const uint2 i1 = *reinterpret_cast<const uint2*>(tidx + (g + 8) * 8);
-#pragma unroll
-          for (int j = 0; j < 8; j++) {
-            const uint32_t msk = (1u << j) * 0x01010101u;
-            int d[4][4];
-#pragma unroll
-            for (int qq = 0; qq < 4; qq++) {
-              d[qq][0] = d[qq][1] = d[qq][2] = d[qq][3] = 0;
-              mma_u8<true>(d[qq], w[qq].x & msk, w[qq].y & msk, w[qq].z & msk, w[qq].w & msk, bword(b, j, 0),
-                           bword(b, j, 1));
+              for (int u = 0; u < F0; u++) w0[u] = lds128(tp + u * 512);
+              stream_mma<F0, BSIGNED>(w0, b, c0);
             }
-            const int s0 = int(((j < 4 ? i0.x : i0.y) >> (8 * (j & 3))) & 0xFFu);
-            const int s1 = int(((j < 4 ? i1.x : i1.y) >> (8 * (j & 3))) & 0xFFu);
-            const int kv = kt * 8 + j;
-            const float gs0 = 2 * t < mg ? float(gsum[2 * t * VPR + kv]) : 0.f;
-            const float gs1 = 2 * t + 1 < mg ? float(gsum[(2 * t + 1) * VPR + kv]) : 0.f;
+            if constexpr (F1 > 0) {
 #pragma unroll
-            for (int c = 0; c < 4; c++) {
-              const float* row = tab + ((c >> 1) ? s1 : s0) * kBvsrTableStride;
-              // integer templates R_i of the set's ratio (1.5, 2, 2.5, 3): c_i = sc R_i
-              const int ri = int(row[6]);
-              const uint32_t R = ri == 0 ? 0x1B120C08u : ri == 1 ? 0x08040201u : ri == 2 ? 0x7D321408u : 0x1B090301u;
-              const int E = (int(R & 0xFF) * d[0][c] + int((R >> 8) & 0xFF) * d[1][c] +
-                             int((R >> 16) & 0xFF) * d[2][c] + int(R >> 24) * d[3][c]) >> j;
-              yacc[c] = fmaf(row[5], float(E), fmaf(row[4], (c & 1) ? gs1 : gs0, yacc[c]));
-              if (a.acc) cacc[c] += (d[0][c] + 2 * d[1][c] + 4 * d[2][c] + 8 * d[3][c]) >> j;
+              for (int u = 0; u < F1; u++) w1[u] = lds128(tp + (F0 + u) * 512);
+              stream_mma<F1, BSIGNED>(w1, b, c1);
+            }
+            if constexpr (F2 > 0) {
+#pragma unroll
+              for (int u = 0; u < F2; u++) w2[u] = lds128(tp + (F0 + F1 + u) * 512);
+              stream_mma<F2, BSIGNED>(w2, b, c2);
+            }
+          } else {
+            // four 1-bit planes; each 32-k block is one vector per row with its own set
+            uint4 w[4];
+#pragma unroll
+            for (int qq = 0; qq < 4; qq++) w[qq] = lds128(tp + qq * 512);
+            const uint8_t* tidx = tp - lane * 16 + 2048;
+            const uint2 i0 = *reinterpret_cast<const uint2*>(tidx + g * 8);
+            const uint2 i1 = *reinterpret_cast<const uint2*>(tidx + (g + 8) * 8);
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+              const uint32_t msk = (1u << j) * 0x01010101u;
+              int d[4][4];
+#pragma unroll
+              for (int qq = 0; qq < 4; qq++) {
+                d[qq][0] = d[qq][1] = d[qq][2] = d[qq][3] = 0;
+                mma_u8<true>(d[qq], w[qq].x & msk, w[qq].y & msk, w[qq].z & msk, w[qq].w & msk, bword(b, j, 0),
+                             bword(b, j, 1));
+              }
+              const int s0 = int(((j < 4 ? i0.x : i0.y) >> (8 * (j & 3))) & 0xFFu);
+              const int s1 = int(((j < 4 ? i1.x : i1.y) >> (8 * (j & 3))) & 0xFFu);
+              const int kv = kt * 8 + j;
+              const float gs0 = 2 * t < mg ? float(gsum[2 * t * VPR + kv]) : 0.f;
+              const float gs1 = 2 * t + 1 < mg ? float(gsum[(2 * t + 1) * VPR + kv]) : 0.f;
+#pragma unroll
+              for (int c = 0; c < 4; c++) {
+                const float* row = tab + ((c >> 1) ? s1 : s0) * kBvsrTableStride;
+                // integer templates R_i of the set's ratio (1.5, 2, 2.5, 3): c_i = sc R_i
+                const int ri = int(row[6]);
+                const uint32_t R = ri == 0 ? 0x1B120C08u : ri == 1 ? 0x08040201u : ri == 2 ? 0x7D321408u : 0x1B090301u;
+                const int E = (int(R & 0xFF) * d[0][c] + int((R >> 8) & 0xFF) * d[1][c] +
+                               int((R >> 16) & 0xFF) * d[2][c] + int(R >> 24) * d[3][c]) >> j;
+                yacc[c] = fmaf(row[5], float(E), fmaf(row[4], (c & 1) ? gs1 : gs0, yacc[c]));
+                if (a.acc) cacc[c] += (d[0][c] + 2 * d[1][c] + 4 * d[2][c] + 8 * d[3][c]) >> j;
+              }
             }
           }
         }
       }
-    }
-    __syncwarp();
-    if (copies_ok && e + a.S < n_my) {
-      if (lane == 0) {
-        fence_proxy_async();  // this stage's shared reads are done before the copy overwrites it
-        issue(e + a.S);
+      __syncwarp();
+      if (copies_ok && e + a.S < n_my) {
+        if (lane == 0) {
+          fence_proxy_async();  // this stage's shared reads are done before the copy overwrites it
+          issue(e + a.S);
+        }
+        issued = e + a.S + 1;
       }
-      issued = e + a.S + 1;
-    }
     }
 
-    // ---- end of a row block: cross-warp sum and fused epilogue ----
-    const int buf = item & 1;
-    long long p[4] = {0, 0, 0, 0};
+    // ---- end of a row block: the group's sum and the fused epilogue ----
+    long long p[4];
     if constexpr (!BVSR) {
       int pi[4] = {0, 0, 0, 0};
       if constexpr (F0 > 0) fold_stream<F0>(c0, pi, a.shift0);
@@ -537,73 +646,33 @@ __global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
 #pragma unroll
       for (int c = 0; c < 4; c++) p[c] = cacc[c];
     }
-    long long* rl = redl + ((buf * NW + warp) * 32 + lane) * 4;
-#pragma unroll
-    for (int c = 0; c < 4; c++) rl[c] = p[c];
-    if (BVSR) {
-      float* rf = redf + ((buf * NW + warp) * 32 + lane) * 4;
-#pragma unroll
-      for (int c = 0; c < 4; c++) rf[c] = yacc[c];
+    const int rb = rb_of(gi);
+    if (WPR == 1) {
+      if (ok && !*fail) layer_epilogue<FMT>(a, smem, tokp, rb, m0, mg, lane, rp, p, yacc);
+      continue;
     }
-    __syncthreads();
-    if (warp != item % NW || !ok || *fail) continue;
-    const int rb = cg + item * a.CPG;
+    const int buf = gi & 1;
+    const size_t slot = ((size_t(grp) * 2 + buf) * WPR + wg) * 32 + lane;
+#pragma unroll
+    for (int c = 0; c < 4; c++) redl[slot * 4 + c] = p[c];
+    if (BVSR) {
+#pragma unroll
+      for (int c = 0; c < 4; c++) redf[slot * 4 + c] = yacc[c];
+    }
+    asm volatile("bar.sync %0, %1;\n" ::"r"(1 + grp), "r"(WPR * 32) : "memory");
+    if (wg != gi % WPR || !ok || *fail) continue;
     long long pl[4] = {0, 0, 0, 0};
     float yl[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int w = 0; w < NW; w++) {
-      const long long* r2 = redl + ((buf * NW + w) * 32 + lane) * 4;
+    for (int w = 0; w < WPR; w++) {
+      const size_t s2 = ((size_t(grp) * 2 + buf) * WPR + w) * 32 + lane;
 #pragma unroll
-      for (int c = 0; c < 4; c++) pl[c] += r2[c];
+      for (int c = 0; c < 4; c++) pl[c] += redl[s2 * 4 + c];
       if (BVSR) {
-        const float* f2 = redf + ((buf * NW + w) * 32 + lane) * 4;
 #pragma unroll
-        for (int c = 0; c < 4; c++) yl[c] += f2[c];
+        for (int c = 0; c < 4; c++) yl[c] += redf[s2 * 4 + c];
       }
     }
-    // lane holds (row g | g+8) x (token 2t | 2t+1)
-#pragma unroll
-    for (int c = 0; c < 4; c++) {
-      const int row = rb * 16 + g + 8 * (c >> 1);
-      const int tl = 2 * t + (c & 1);
-      const int tok_i = m0 + tl;
-      if (row >= a.N || tl >= mg) continue;
-      const uint32_t* tk = tok + 4 * tl;
-      long long acc;
-      float yv;
-      if (FMT == BQ_FMT_BITNET_W1A8) {
-        // p = sum_k neg_k q_k  ->  sum_k sign_k q_k = sum q - 2p
-        acc = (long long)int(tk[1]) - 2ll * pl[c];
-        yv = __fmul_rn(tscale, __fdiv_rn(__uint_as_float(tk[0]), 127.f)) * float(acc);
-      } else if (FMT == BQ_FMT_TERNARY_A8) {
-        // p = sum_k (T_k + 1) q_k  ->  sum_k T_k q_k = p - sum q
-        acc = pl[c] - (long long)int(tk[1]);
-        yv = __fmul_rn(tscale, __fdiv_rn(__uint_as_float(tk[0]), 127.f)) * float(acc);
-        if (a.rank > 0) {
-          const float* u = reinterpret_cast<const float*>(smem + a.off_u) + size_t(tl) * a.rank;
-          const uint4* bt = reinterpret_cast<const uint4*>(a.lora_bt + size_t(row) * a.rank);
-          float l = 0.f;
-          for (int q8 = 0; q8 < a.rank / 8; q8++) {
-            const uint4 v = __ldg(bt + q8);
-            const uint32_t h[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int e = 0; e < 8; e++)
-              l = fmaf(u[q8 * 8 + e], __uint_as_float((e & 1) ? (h[e >> 1] & 0xFFFF0000u) : (h[e >> 1] << 16)), l);
-          }
-          yv += lora_gate * l;
-        }
-      } else if (FMT == BQ_FMT_ABQ) {
-        // I = P - z_x S_w - z_w S_x + K z_w z_x
-        const long long zx = int(tk[1]), sx = int(tk[2]);
-        const long long zw = a.row_zero[row], sw = a.row_sum[row];
-        acc = pl[c] - zx * sw - zw * sx + (long long)a.K * zw * zx;
-        yv = __fmul_rn(a.row_delta[row], __uint_as_float(tk[0])) * float(acc);
-      } else {
-        acc = pl[c];
-        yv = __fdiv_rn(__uint_as_float(tk[0]), 127.f) * yl[c];
-      }
-      a.y[size_t(tok_i) * a.N + row] = yv;
-      if (a.acc) a.acc[size_t(tok_i) * a.N + row] = acc;
-    }
+    layer_epilogue<FMT>(a, smem, tokp, rb, m0, mg, lane, rp, pl, yl);
   }
   // copies issued but never waited for (an abandoned wait) must land before the block exits
   if (!copies_ok)
@@ -654,6 +723,7 @@ __global__ void __launch_bounds__(NW * 32) k_rabit(LayerArgs a) {
   const uint32_t* p2 = a.rabit_planes + (size_t(a.N_pad) + row) * W32;
   for (int m = 0; m < a.M; m++) {
     float acc1 = 0.f, acc2 = 0.f;
+#pragma unroll 8
     for (int wd = 0; wd < W32; wd++) {
       const uint32_t b1 = __ldg(p1 + wd), b2 = __ldg(p2 + wd);
       const int k = wd * 32 + lane;
