@@ -522,8 +522,8 @@ bq_status bq_linear(const bq_layer* layer, const void* x_bf16, int32_t M, float*
   g.x = static_cast<const uint16_t*>(x_bf16);
   if (L.fmt == BQ_FMT_TERNARY_A8 && L.rank > 0) {
     float* up = static_cast<float*>(workspace);
-    if (launch_pdl(k_lora_partial, dim3(L.KT), dim3(256), 0, s, g.x, reinterpret_cast<const uint16_t*>(P + L.off_aux),
-                   M, L.K, L.rank, up) != cudaSuccess)
+    if (launch_pdl(k_lora_partial, dim3((L.KT * M + 7) / 8), dim3(256), 0, s, g.x,
+                   reinterpret_cast<const uint16_t*>(P + L.off_aux), M, L.K, L.KT, L.rank, up) != cudaSuccess)
       return BQ_ERR_CUDA;
     g.u_part = up;
   }

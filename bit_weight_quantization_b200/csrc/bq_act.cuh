@@ -147,10 +147,9 @@ __global__ void __launch_bounds__(256) k_act_quant(ActArgs a) {
   //     u = SiLU(sum of partials) is formed by the layer kernel) ---
   if (FMT == BQ_FMT_TERNARY_A8 && a.rank > 0) {
     float* up = reinterpret_cast<float*>(a.act + a.off_u);
-    for (int i = threadIdx.x; i < (kt1 - kt0) * a.rank; i += blockDim.x) {
-      const int kt = kt0 + i / a.rank, r = i % a.rank;
-      up[(size_t(kt) * a.M + m) * a.rank + r] = lora_tile_dot(xr, a.lora_A, a.K, a.rank, kt, r);
-    }
+    const int nw = blockDim.x >> 5, lane = threadIdx.x & 31;
+    for (int kt = kt0 + (threadIdx.x >> 5); kt < kt1; kt += nw)
+      lora_tile_partial_warp(xr, a.lora_A, a.K, a.rank, kt, lane, up + (size_t(kt) * a.M + m) * a.rank);
   }
 
   if (slice != 0) return;

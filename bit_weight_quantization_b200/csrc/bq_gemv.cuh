@@ -358,15 +358,21 @@ __device__ void stage_lora_u(const LayerArgs& a, uint8_t* smem, int m0, int mg, 
   float* us = reinterpret_cast<float*>(smem + a.off_u);
   for (int i = threadIdx.x; i < mg * a.rank; i += NT) {
     const int m = i / a.rank, r = i - m * a.rank;
+    const float* up = a.u_part + size_t(m0 + m) * a.rank + r;
+    const size_t st = size_t(a.M) * a.rank;
     float zsum = 0.f;
-    for (int kt = 0; kt < a.KT; kt++) zsum += a.u_part[(size_t(kt) * a.M + m0 + m) * a.rank + r];
+    for (int kt = 0; kt < a.KT; kt += 8) {  // loads of 8 tiles in flight, summed in tile order
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 8; e++) v[e] = kt + e < a.KT ? up[(kt + e) * st] : 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; e++)
+        if (kt + e < a.KT) zsum += v[e];
+    }
     us[i] = zsum / (1.f + expf(-zsum));
   }
 }
 
-// Fused epilogue for one 16-row block: lane holds (row g | g+8) x (token 2t | 2t+1).
-// tok[4m + 3] holds the token's output scale (alpha gamma/127, gamma_W gamma/127,
-// gamma/127 or Delta_x).
 // Per-row ABQ parameters of a row block's rows g and g + 8 (Delta_w, z_w, S_w), loaded
 // ahead of the block's tiles so the epilogue does not wait on them.
 struct RowP {
@@ -386,6 +392,9 @@ __device__ __forceinline__ void load_rowp(const LayerArgs& a, int rb, int lane, 
   }
 }
 
+// Fused epilogue for one 16-row block: lane holds (row g | g+8) x (token 2t | 2t+1).
+// tok[4m + 3] holds the token's output scale (alpha gamma/127, gamma_W gamma/127,
+// gamma/127 or Delta_x).
 template <int FMT>
 __device__ __forceinline__ void layer_epilogue(const LayerArgs& a, const uint8_t* smem, const uint32_t* tok, int rb,
                                                int m0, int mg, int lane, const RowP& rp, const long long (&pl)[4],
@@ -433,6 +442,53 @@ __device__ __forceinline__ void layer_epilogue(const LayerArgs& a, const uint8_t
     }
     a.y[size_t(m0 + tl) * a.N + row] = yv;
     if (a.acc) a.acc[size_t(m0 + tl) * a.N + row] = acc;
+  }
+}
+
+// Exact float of an integer |v| < 2^22 by the 1.5 * 2^23 bias (two full-rate ops).
+__device__ __forceinline__ float small_int_to_float(int v) {
+  return __fsub_rn(__int_as_float(int(kRnBias) + v), 12582912.0f);
+}
+
+// One BVSR tile (16 rows x 8 vectors of 32 k) for this lane's outputs. Plane i of vector j
+// is bit j of each byte of w[i]; its dot with the codes, d_i, comes from one int8 MMA
+// (scaled by 2^j). Per row and vector the set s gives the template bytes R (table word 7),
+// o and sc = span / sum R (words 4, 5): y += sc sum_i R_i d_i + o S_v, S_v the vector's
+// code sum. TWO: the CTA holds more than one token, so outputs c = 1, 3 (token 2t + 1)
+// are live too; with one token only c = 0, 2 (token 0, lanes t = 0) carry data.
+template <bool TWO>
+__device__ __forceinline__ void bvsr_tile(const uint4 (&w)[4], const uint4 (&b)[4], uint2 i0, uint2 i1,
+                                          const float* tab, const int* gs_row, int VPR, bool tok0, bool tok1,
+                                          bool want_acc, float (&yacc)[4], long long (&cacc)[4]) {
+  const uint32_t* tabu = reinterpret_cast<const uint32_t*>(tab);
+#pragma unroll
+  for (int j = 0; j < 8; j++) {
+    const uint32_t msk = (1u << j) * 0x01010101u;
+    int d[4][4];
+#pragma unroll
+    for (int qq = 0; qq < 4; qq++) {
+      d[qq][0] = d[qq][1] = d[qq][2] = d[qq][3] = 0;
+      mma_u8<true>(d[qq], w[qq].x & msk, w[qq].y & msk, w[qq].z & msk, w[qq].w & msk, bword(b, j, 0), bword(b, j, 1));
+    }
+    const int s0 = int(__byte_perm(j < 4 ? i0.x : i0.y, 0, 0x4440 + (j & 3)));
+    const int s1 = int(__byte_perm(j < 4 ? i1.x : i1.y, 0, 0x4440 + (j & 3)));
+    const uint32_t R[2] = {tabu[s0 * kBvsrTableStride + 7], tabu[s1 * kBvsrTableStride + 7]};
+    const float2 os[2] = {*reinterpret_cast<const float2*>(tab + s0 * kBvsrTableStride + 4),
+                          *reinterpret_cast<const float2*>(tab + s1 * kBvsrTableStride + 4)};
+    const float gsf[2] = {tok0 ? small_int_to_float(gs_row[j]) : 0.f,
+                          TWO && tok1 ? small_int_to_float(gs_row[VPR + j]) : 0.f};
+#pragma unroll
+    for (int h = 0; h < 2; h++) {  // row g (h = 0) or g + 8
+      const int r0 = int(R[h] & 0xFFu), r1 = int(__byte_perm(R[h], 0, 0x4441)), r2 = int(__byte_perm(R[h], 0, 0x4442)),
+                r3 = int(R[h] >> 24);
+#pragma unroll
+      for (int q = 0; q < (TWO ? 2 : 1); q++) {
+        const int c = 2 * h + q;
+        const int E = (r0 * d[0][c] + r1 * d[1][c] + r2 * d[2][c] + r3 * d[3][c]) >> j;
+        yacc[c] = fmaf(os[h].y, small_int_to_float(E), fmaf(os[h].x, gsf[q], yacc[c]));
+        if (want_acc) cacc[c] += (d[0][c] + 2 * d[1][c] + 4 * d[2][c] + 8 * d[3][c]) >> j;
+      }
+    }
   }
 }
 
@@ -498,6 +554,14 @@ __global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
     }
   }
   if constexpr (FUSED) prefetch_x(a, m0, mg, NW * 32);
+  if (FMT == BQ_FMT_TERNARY_A8 && a.rank > 0) {  // B^T rows of this CTA's row blocks, for the epilogue
+    const int lines = a.rank / 4;                 // 16 rows x rank bf16 = rank/4 lines of 128 B
+    for (int i = tid; i < n_items * lines; i += NW * 32) {
+      const int rb = cg + (i / lines) * a.CPG;
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(a.lora_bt + size_t(rb) * 16 * a.rank) +
+                                                     size_t(i % lines) * 128));
+    }
+  }
   int* fail = reinterpret_cast<int*>(smem + a.off_bar) + 2 * (NW * a.S + 2);  // a copy wait was abandoned
   if (tid == 0) {
     *fail = 0;
@@ -527,6 +591,7 @@ __global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
   const int VPR = a.K_pad / 32;
   const int* gsum = reinterpret_cast<const int*>(smem + a.off_gsum);
   const float* tab = reinterpret_cast<const float*>(smem + a.off_tab);
+  const bool want_acc = a.acc != nullptr;
   long long* redl = reinterpret_cast<long long*>(smem + a.off_red);                // [G][2][WPR][32][4]
   float* redf = reinterpret_cast<float*>(smem + a.off_red + 2 * NW * 32 * 4 * 8);  // same shape
   bool copies_ok = true;
@@ -586,40 +651,15 @@ __global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
               stream_mma<F2, BSIGNED>(w2, b, c2);
             }
           } else {
-            // four 1-bit planes; each 32-k block is one vector per row with its own set
             uint4 w[4];
 #pragma unroll
             for (int qq = 0; qq < 4; qq++) w[qq] = lds128(tp + qq * 512);
             const uint8_t* tidx = tp - lane * 16 + 2048;
             const uint2 i0 = *reinterpret_cast<const uint2*>(tidx + g * 8);
             const uint2 i1 = *reinterpret_cast<const uint2*>(tidx + (g + 8) * 8);
-#pragma unroll
-            for (int j = 0; j < 8; j++) {
-              const uint32_t msk = (1u << j) * 0x01010101u;
-              int d[4][4];
-#pragma unroll
-              for (int qq = 0; qq < 4; qq++) {
-                d[qq][0] = d[qq][1] = d[qq][2] = d[qq][3] = 0;
-                mma_u8<true>(d[qq], w[qq].x & msk, w[qq].y & msk, w[qq].z & msk, w[qq].w & msk, bword(b, j, 0),
-                             bword(b, j, 1));
-              }
-              const int s0 = int(((j < 4 ? i0.x : i0.y) >> (8 * (j & 3))) & 0xFFu);
-              const int s1 = int(((j < 4 ? i1.x : i1.y) >> (8 * (j & 3))) & 0xFFu);
-              const int kv = kt * 8 + j;
-              const float gs0 = 2 * t < mg ? float(gsum[2 * t * VPR + kv]) : 0.f;
-              const float gs1 = 2 * t + 1 < mg ? float(gsum[(2 * t + 1) * VPR + kv]) : 0.f;
-#pragma unroll
-              for (int c = 0; c < 4; c++) {
-                const float* row = tab + ((c >> 1) ? s1 : s0) * kBvsrTableStride;
-                // integer templates R_i of the set's ratio (1.5, 2, 2.5, 3): c_i = sc R_i
-                const int ri = int(row[6]);
-                const uint32_t R = ri == 0 ? 0x1B120C08u : ri == 1 ? 0x08040201u : ri == 2 ? 0x7D321408u : 0x1B090301u;
-                const int E = (int(R & 0xFF) * d[0][c] + int((R >> 8) & 0xFF) * d[1][c] +
-                               int((R >> 16) & 0xFF) * d[2][c] + int(R >> 24) * d[3][c]) >> j;
-                yacc[c] = fmaf(row[5], float(E), fmaf(row[4], (c & 1) ? gs1 : gs0, yacc[c]));
-                if (a.acc) cacc[c] += (d[0][c] + 2 * d[1][c] + 4 * d[2][c] + 8 * d[3][c]) >> j;
-              }
-            }
+            if (mg > 1) bvsr_tile<true>(w, b, i0, i1, tab, gsum + size_t(2 * t) * VPR + kt * 8, VPR, 2 * t < mg,
+                                        2 * t + 1 < mg, want_acc, yacc, cacc);
+            else bvsr_tile<false>(w, b, i0, i1, tab, gsum + kt * 8, VPR, t == 0, false, want_acc, yacc, cacc);
           }
         }
       }
@@ -681,18 +721,17 @@ __global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
 
 // ---------------------------------------------------------------------------
 // Ternary LoRA input (fused path): partial dot products of the unquantized bf16 x
-// with A over each 256-k tile, out[kt][m][r], each summed in k order (the act kernel
-// computes the same partials for the unfused path). Grid: one CTA per k-tile.
+// with A over each 256-k tile, out[kt][m][r], one warp per (kt, m) (the act kernel
+// computes the same partials with the same warp routine for the unfused path).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_lora_partial(const uint16_t* __restrict__ x, const uint16_t* __restrict__ A,
-                                                      int M, int K, int rank, float* __restrict__ out) {
+                                                      int M, int K, int KT, int rank, float* __restrict__ out) {
   pdl_trigger();
   pdl_wait();
-  const int kt = blockIdx.x;
-  for (int i = threadIdx.x; i < M * rank; i += blockDim.x) {
-    const int m = i / rank, r = i - m * rank;
-    out[(size_t(kt) * M + m) * rank + r] = lora_tile_dot(x + size_t(m) * K, A, K, rank, kt, r);
-  }
+  const int wid = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (wid >= KT * M) return;
+  const int kt = wid / M, m = wid - kt * M;
+  lora_tile_partial_warp(x + size_t(m) * K, A, K, rank, kt, threadIdx.x & 31, out + (size_t(kt) * M + m) * rank);
 }
 
 // ---------------------------------------------------------------------------

@@ -33,7 +33,7 @@ enum : int {
 };
 
 constexpr int kBvsrSets = 256;
-constexpr int kBvsrTableStride = 8;  // floats per set: c0 c1 c2 c3 o sc ratio_index 0
+constexpr int kBvsrTableStride = 8;  // words per set: c0 c1 c2 c3 o sc ratio_index, R bytes (u32)
 constexpr int kBvsrTileBytes = 4 * 512 + 16 * 8;
 
 struct PkLayout {
@@ -146,15 +146,44 @@ __device__ __forceinline__ int code_word_in_tile(int kin) {
   return 16 * t + 2 * mu + h;
 }
 
-// Partial dot product of one token's bf16 x with column r of the bf16 LoRA matrix
-// A [K_pad][rank] over the 256-k tile kt, accumulated in k order (f32).
-__device__ __forceinline__ float lora_tile_dot(const uint16_t* xr, const uint16_t* A, int K, int rank, int kt,
-                                               int r) {
-  float acc = 0.f;
-  const int k1 = min(K, kt * 256 + 256);
-  for (int k = kt * 256; k < k1; k++)
-    acc = fmaf(__uint_as_float(uint32_t(xr[k]) << 16), __uint_as_float(uint32_t(A[size_t(k) * rank + r]) << 16), acc);
-  return acc;
+// Ternary LoRA input, one 256-k tile, by one warp: out[r] = sum over the tile's k of
+// x_k A[k][r] for r < rank (K % 128 == 0, so a lane's 8 k's are all inside K or all past
+// it). Lane l takes k = 256 kt + 8l .. 8l + 7 and sums its 8 products in k order; the 32
+// lane sums meet in a fixed xor-butterfly, so every caller gets the same bits.
+__device__ __forceinline__ void lora_tile_partial_warp(const uint16_t* xr, const uint16_t* A, int K, int rank,
+                                                       int kt, int lane, float* out) {
+  const int k0 = kt * 256 + lane * 8;
+  const bool in = k0 < K;
+  float xv[8];
+  {
+    const uint4 v = in ? *reinterpret_cast<const uint4*>(xr + k0) : make_uint4(0, 0, 0, 0);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 8; e++) xv[e] = __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+  }
+  for (int rc = 0; rc < rank; rc += 8) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) acc[i] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; e++) {
+      const uint4 v = in ? *reinterpret_cast<const uint4*>(A + size_t(k0 + e) * rank + rc) : make_uint4(0, 0, 0, 0);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 8; i++)
+        acc[i] = fmaf(xv[e], __uint_as_float((i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16)), acc[i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int i = 0; i < 8; i++) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    if (lane < 8) {
+      float v = acc[0];
+#pragma unroll
+      for (int i = 1; i < 8; i++) v = lane == i ? acc[i] : v;
+      out[rc + lane] = v;
+    }
+  }
 }
 
 // Order-preserving map of a float to uint32 (total order on non-NaN values).

@@ -305,7 +305,9 @@ __global__ void k_bvsr_table(const uint32_t* counts_in, uint64_t V, float* table
   const double rsum[4] = {65.0, 15.0, 203.0, 40.0};
   row[5] = __double2float_rn(__ddiv_rn(span, rsum[j]));
   row[6] = float(j);
-  row[7] = 0.f;
+  // the integer templates R_i as bytes of one word: {8,12,18,27} {1,2,4,8} {8,20,50,125} {1,3,9,27}
+  const uint32_t rword[4] = {0x1B120C08u, 0x08040201u, 0x7D321408u, 0x1B090301u};
+  row[7] = __uint_as_float(rword[j]);
 }
 
 // Points of set s, o + c0 b0 + c1 b1 + c2 b2 + c3 b3 summed left to right in float64.

@@ -66,7 +66,8 @@
  *   Ternary aux = A bf16 [K_pad][r], aux2 = B^T bf16 [N_pad][r].
  *   ABQ rows = Delta_w f32 [N_pad], z_w i32 [N_pad], S_w = sum_k q_w i32 [N_pad].
  *   BVSR aux = coefficient table f32 [256][8] (c0 c1 c2 c3 o; then derived kernel constants:
- *   sc = (hi-lo)/sum_i R_i, ratio index, 0).
+ *   sc = (hi-lo)/sum_i R_i, ratio index, and word 7 the integer templates R_0..R_3 as the
+ *   bytes of a uint32, low byte first).
  *
  * Activation buffer (device, 256-byte aligned), version 1.
  * Header: 64 x 32-bit words: 0 magic 0x43415142 ('BQAC') 1 version 2 format 3 M 4 K 5 K_pad
