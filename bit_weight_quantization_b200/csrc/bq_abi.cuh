@@ -200,16 +200,28 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   g->off_u = take(rank > 0 ? uint64_t(tpc) * rank * 4 : 16);
   g->off_gsum = take(bvsr ? uint64_t(tpc) * VPR * 4 : 16);
   g->off_tab = take(bvsr ? uint64_t(kBvsrSets) * kBvsrTableStride * 4 : 16);
-  g->off_red = take(2ull * NW * 32 * 4 * 12);
+  // split-K exchange [G][2][WPR][32][4] of int64 (+ f32 for BVSR) when warps share a row
+  // block; at least the staging reductions' 3 x 32 words
+  g->off_red = take(wpr > 1 ? 2ull * NW * 32 * 4 * (bvsr ? 12 : 8) : 512);
+  // ternary: the B^T rows of the CTA's row blocks (32 rank bytes each) when they fit in 32 KB
+  const uint64_t lbt = uint64_t(ipc) * 32 * rank;
+  g->lbt_smem = rank > 0 && lbt <= 32 * 1024;
+  g->off_lbt = take(g->lbt_smem ? lbt : 16);
   const uint64_t fixed = off + 1024;  // + barriers
-  const uint64_t limit = 220 * 1024;
-  const uint64_t budget = std::min<uint64_t>(96 * 1024, fixed < limit ? limit - fixed : 0);
-  const uint64_t per_warp = budget / NW;
+  // two CTAs per SM (228 KB, 1 KB reserved per CTA): the next launch's CTA is resident,
+  // and prefetching its weights, while this one computes
+  // (else one CTA per SM with up to 220 KB)
+  uint64_t per_warp = 0;
+  for (const uint64_t limit : {112ull * 1024, 220ull * 1024}) {
+    const uint64_t budget = std::min<uint64_t>(96 * 1024, fixed < limit ? limit - fixed : 0);
+    per_warp = budget / NW;
+    if (per_warp >= 2ull * L.tile_bytes) break;
+  }
   if (per_warp < 2ull * L.tile_bytes) return false;
   g->S = int(std::min<uint64_t>(4, std::max<uint64_t>(2, per_warp / L.tile_bytes)));
   g->C = int(std::max<uint64_t>(1, std::min<uint64_t>(g->T, per_warp / (uint64_t(g->S) * L.tile_bytes))));
   g->off_ring = take(uint64_t(NW) * g->S * g->C * L.tile_bytes);
-  g->off_bar = take(uint64_t(NW * g->S + 2) * 8 + 16);
+  g->off_bar = take(uint64_t(NW * g->S + 3) * 8 + 16);
   g->smem_bytes = uint32_t(off);
   g->RB = L.RB;
   return true;

@@ -152,7 +152,8 @@ struct LayerArgs {
   //   tpc tokens per CTA, TG token groups, CPG CTAs per token group,
   //   WPR warps sharing one row block (the k-split), a power of two dividing NW
   int T, C, S, tpc, TG, CPG, WPR, cstride, J;
-  uint32_t off_ring, off_codes, off_tok, off_u, off_gsum, off_tab, off_red, off_bar, smem_bytes;
+  uint32_t off_ring, off_codes, off_tok, off_u, off_gsum, off_tab, off_red, off_lbt, off_bar, smem_bytes;
+  int lbt_smem;             // ternary: the CTA's B^T rows are copied to off_lbt (else read from global)
 };
 
 // ---------------------------------------------------------------------------
@@ -397,8 +398,8 @@ __device__ __forceinline__ void load_rowp(const LayerArgs& a, int rb, int lane, 
 // gamma/127 or Delta_x).
 template <int FMT>
 __device__ __forceinline__ void layer_epilogue(const LayerArgs& a, const uint8_t* smem, const uint32_t* tok, int rb,
-                                               int m0, int mg, int lane, const RowP& rp, const long long (&pl)[4],
-                                               const float (&yl)[4]) {
+                                               int m0, int mg, int lane, const RowP& rp, const uint8_t* lbt,
+                                               const long long (&pl)[4], const float (&yl)[4]) {
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
   for (int c = 0; c < 4; c++) {
@@ -419,14 +420,21 @@ __device__ __forceinline__ void layer_epilogue(const LayerArgs& a, const uint8_t
       yv = scale * float(acc);
       if (a.rank > 0) {
         const float* u = reinterpret_cast<const float*>(smem + a.off_u) + size_t(tl) * a.rank;
-        const uint4* bt = reinterpret_cast<const uint4*>(a.lora_bt + size_t(row) * a.rank);
+        const uint4* bt = a.lbt_smem ? reinterpret_cast<const uint4*>(lbt + size_t(row - rb * 16) * a.rank * 2)
+                                     : reinterpret_cast<const uint4*>(a.lora_bt + size_t(row) * a.rank);
         float l = 0.f;
-        for (int q8 = 0; q8 < a.rank / 8; q8++) {
-          const uint4 v = __ldg(bt + q8);
-          const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+        for (int q8 = 0; q8 < a.rank / 8; q8 += 4) {  // rank is a multiple of 8
+          uint4 v[4];
 #pragma unroll
-          for (int e = 0; e < 8; e++)
-            l = fmaf(u[q8 * 8 + e], __uint_as_float((e & 1) ? (h[e >> 1] & 0xFFFF0000u) : (h[e >> 1] << 16)), l);
+          for (int i = 0; i < 4; i++) v[i] = q8 + i < a.rank / 8 ? bt[q8 + i] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            if (q8 + i >= a.rank / 8) break;
+            const uint32_t h[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+            for (int e = 0; e < 8; e++)
+              l = fmaf(u[(q8 + i) * 8 + e], __uint_as_float((e & 1) ? (h[e >> 1] & 0xFFFF0000u) : (h[e >> 1] << 16)), l);
+          }
         }
         yv += __uint_as_float(reinterpret_cast<const uint32_t*>(smem + a.off_tok)[kTokAlpha]) * l;  // tanh(alpha)
       }
@@ -514,6 +522,7 @@ __global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
   const int WPR = a.WPR, G = NW / WPR;
   const int grp = warp / WPR, wg = warp - grp * WPR;
   const int n_gitems = grp < n_items ? (n_items - grp + G - 1) / G : 0;  // row blocks of this group
+  const bool LBT = FMT == BQ_FMT_TERNARY_A8 && a.rank > 0 && a.lbt_smem && n_items > 0;
 
   // Let the next launch in the stream start; it only prefetches its own weights
   // before its griddepcontrol.wait.
@@ -527,12 +536,14 @@ __global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
   uint64_t* wbar = bars + warp * a.S;
   uint64_t* tbar = bars + NW * a.S;  // BVSR coefficient table
   uint64_t* xbar = tbar + 1;         // activation codes (unfused path)
+  uint64_t* lbar = tbar + 2;         // ternary B^T rows
   const int kt_begin = wg * a.T;
   const int nt = max(0, min(a.KT, kt_begin + a.T) - kt_begin);
   const int cpw = (nt + a.C - 1) / a.C;
   const int n_my = n_gitems * cpw;
   auto chunk_tiles = [&](int e) { return min(a.C, nt - (e % cpw) * a.C); };
   auto rb_of = [&](int gi) { return cg + (grp + gi * G) * a.CPG; };
+  auto lbt_of = [&](int gi) { return smem + a.off_lbt + size_t(grp + gi * G) * 32 * a.rank; };
   uint8_t* ring = smem + a.off_ring + size_t(warp) * a.S * a.C * a.tile_bytes;
   auto issue = [&](int e) {
     const int st = e % a.S;
@@ -545,24 +556,22 @@ __global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
   const int first = min(n_my, a.S);
   if (lane == 0) {
     for (int st = 0; st < a.S; st++) mbar_init(&wbar[st], 1);
-    if (warp == 0) { mbar_init(tbar, 1); mbar_init(xbar, 1); }
+    if (warp == 0) { mbar_init(tbar, 1); mbar_init(xbar, 1); mbar_init(lbar, 1); }
     fence_mbar_init();
     for (int e = 0; e < first; e++) issue(e);
     if (BVSR && warp == 0) {
       mbar_expect_tx(tbar, kBvsrSets * kBvsrTableStride * 4);
       bulk_g2s(smem + a.off_tab, a.bvsr_table, kBvsrSets * kBvsrTableStride * 4, tbar);
     }
-  }
-  if constexpr (FUSED) prefetch_x(a, m0, mg, NW * 32);
-  if (FMT == BQ_FMT_TERNARY_A8 && a.rank > 0) {  // B^T rows of this CTA's row blocks, for the epilogue
-    const int lines = a.rank / 4;                 // 16 rows x rank bf16 = rank/4 lines of 128 B
-    for (int i = tid; i < n_items * lines; i += NW * 32) {
-      const int rb = cg + (i / lines) * a.CPG;
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(a.lora_bt + size_t(rb) * 16 * a.rank) +
-                                                     size_t(i % lines) * 128));
+    if (LBT && warp == 0) {  // the B^T rows of this CTA's row blocks (16 rows x rank bf16 each)
+      const uint32_t per = 32u * uint32_t(a.rank);
+      mbar_expect_tx(lbar, per * uint32_t(n_items));
+      for (int i = 0; i < n_items; i++)
+        bulk_g2s(smem + a.off_lbt + size_t(i) * per, a.lora_bt + size_t(cg + i * a.CPG) * 16 * a.rank, per, lbar);
     }
   }
-  int* fail = reinterpret_cast<int*>(smem + a.off_bar) + 2 * (NW * a.S + 2);  // a copy wait was abandoned
+  if constexpr (FUSED) prefetch_x(a, m0, mg, NW * 32);
+  int* fail = reinterpret_cast<int*>(smem + a.off_bar) + 2 * (NW * a.S + 3);  // a copy wait was abandoned
   if (tid == 0) {
     *fail = 0;
     uint32_t* tw = reinterpret_cast<uint32_t*>(smem + a.off_tok);
@@ -585,6 +594,7 @@ __global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
     __syncthreads();
   }
   if (BVSR && !mbar_wait_bounded(tbar, 0)) ok = false;
+  if (LBT && !mbar_wait_bounded(lbar, 0)) ok = false;
 
   const bool has_tok = g < mg;
   const uint8_t* bsrc = smem + a.off_codes + size_t(has_tok ? g : 0) * a.cstride + t * 64;
@@ -688,7 +698,7 @@ __global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
     }
     const int rb = rb_of(gi);
     if (WPR == 1) {
-      if (ok && !*fail) layer_epilogue<FMT>(a, smem, tokp, rb, m0, mg, lane, rp, p, yacc);
+      if (ok && !*fail) layer_epilogue<FMT>(a, smem, tokp, rb, m0, mg, lane, rp, lbt_of(gi), p, yacc);
       continue;
     }
     const int buf = gi & 1;
@@ -712,7 +722,7 @@ __global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
         for (int c = 0; c < 4; c++) yl[c] += redf[s2 * 4 + c];
       }
     }
-    layer_epilogue<FMT>(a, smem, tokp, rb, m0, mg, lane, rp, pl, yl);
+    layer_epilogue<FMT>(a, smem, tokp, rb, m0, mg, lane, rp, lbt_of(gi), pl, yl);
   }
   // copies issued but never waited for (an abandoned wait) must land before the block exits
   if (!copies_ok)
