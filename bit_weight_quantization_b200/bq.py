@@ -52,6 +52,7 @@ _SIGS = {
     "bq_linear_workspace_bytes": (ctypes.c_int, [ctypes.POINTER(bq_layer), ctypes.c_int32,
                                                  ctypes.POINTER(ctypes.c_size_t)]),
     "bq_linear": (ctypes.c_int, [ctypes.POINTER(bq_layer), _P, ctypes.c_int32, _P, _P, _P, ctypes.c_size_t, _P]),
+    "bq_linear_static_scratch": (ctypes.c_int, [ctypes.POINTER(bq_layer), _P, ctypes.c_int32, _P, _P, _P]),
     "bq_device_check": (ctypes.c_int, []),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -144,6 +145,15 @@ def bq_linear_workspace_bytes(layer: bq_layer, M: int) -> int:
     out = ctypes.c_size_t(0)
     _check(_lib.bq_linear_workspace_bytes(ctypes.byref(layer), M, ctypes.byref(out)), "bq_linear_workspace_bytes")
     return out.value
+
+
+BQ_STATIC_SCRATCH_BYTES = 1 << 20
+
+
+def bq_linear_static_scratch(layer: bq_layer, x_bf16, M: int, y, acc_dbg=None, stream=None) -> None:
+    """bq_linear with the library's fixed scratch array instead of a workspace."""
+    _check(_lib.bq_linear_static_scratch(ctypes.byref(layer), _ptr(x_bf16), M, _ptr(y), _ptr(acc_dbg),
+                                         _stream(stream)), "bq_linear_static_scratch")
 
 
 def bq_linear(layer: bq_layer, x_bf16, M: int, y, acc_dbg=None, workspace=None, workspace_bytes: int = 0,

@@ -1,6 +1,7 @@
 // C ABI: host-side validation, buffer layouts and kernel launches.
 #pragma once
 
+#include <mutex>
 #include <algorithm>
 #include <cstring>
 
@@ -540,6 +541,48 @@ bq_status bq_linear(const bq_layer* layer, const void* x_bf16, int32_t M, float*
     g.u_part = up;
   }
   return launch_layer(L, g, true, s);
+}
+
+// Scratch of bq_linear_static_scratch (one copy per device context).
+static __device__ __align__(256) uint8_t g_bq_static_scratch[BQ_STATIC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+
+// Device address of the scratch array on the current device, looked up once per device.
+bq_status static_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return BQ_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return BQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_bq_static_scratch) != cudaSuccess || !p) {
+      (void)cudaGetLastError();
+      return BQ_ERR_CUDA;
+    }
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return BQ_OK;
+}
+}  // namespace
+
+bq_status bq_linear_static_scratch(const bq_layer* layer, const void* x_bf16, int32_t M, float* y,
+                                   int64_t* acc_dbg, void* stream) {
+  size_t need = 0;
+  bq_status st = bq_linear_workspace_bytes(layer, M, &need);
+  if (st != BQ_OK) return st;
+  if (need > BQ_STATIC_SCRATCH_BYTES) return BQ_ERR_SIZE;
+  void* ws = nullptr;
+  st = static_scratch(&ws);
+  if (st != BQ_OK) return st;
+  return bq_linear(layer, x_bf16, M, y, acc_dbg, need > 0 ? ws : nullptr, need, stream);
 }
 
 bq_status bq_gemv(const bq_layer* layer, const void* act, float* y, int64_t* acc_dbg, void* stream) {

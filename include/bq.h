@@ -191,6 +191,30 @@ bq_status bq_linear_workspace_bytes(const bq_layer* layer, int32_t M, size_t* by
 bq_status bq_linear(const bq_layer* layer, const void* x_bf16, int32_t M, float* y, int64_t* acc_dbg,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* bq_linear with its scratch in a fixed device array inside the library instead of a
+ * caller workspace. The pages have no counterpart: this is a calling convenience, not a
+ * step of the method. It is for callers that cannot allocate device memory where they
+ * run a layer. Examples: a plain C host that owns only the packed layer and its x/y
+ * buffers and has no allocator of its own, or a decode loop that must make no allocator
+ * call between its buffers being set up and the layer running.
+ * Same arguments and results as bq_linear, without workspace and workspace_bytes.
+ *  - Scratch limit: BQ_STATIC_SCRATCH_BYTES (1 MiB). A call needing more, that is
+ *    bq_linear_workspace_bytes(layer, M) > 1 MiB, returns BQ_ERR_SIZE and enqueues
+ *    nothing. Only the ternary format with a LoRA term uses scratch, K_pad/256 * M *
+ *    rank * 4 bytes: e.g. K = 16384, M = 64, rank = 64 is exactly 1 MiB.
+ *  - Setup: the first call on a device looks up the array's device address once
+ *    (cudaGetSymbolAddress) and keeps it; a failure there returns BQ_ERR_CUDA. Make
+ *    that first call, on each device, before any stream capture begins.
+ *  - Sharing: every call on a device uses the same array. Nothing in it has to start at
+ *    zero: each call writes every scratch word before it reads it. Calls on one stream
+ *    are ordered and safe; calls whose work overlaps in time (several streams, or
+ *    several host threads each with its own stream) race on the array, so the caller
+ *    must not overlap them.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+#define BQ_STATIC_SCRATCH_BYTES (1u << 20)
+bq_status bq_linear_static_scratch(const bq_layer* layer, const void* x_bf16, int32_t M, float* y,
+                                   int64_t* acc_dbg, void* stream);
+
 /* Synchronizes the current device, then reads and clears the device error word:
  * BQ_OK or BQ_ERR_DEVICE_CHECK. */
 bq_status bq_device_check(void);

@@ -172,3 +172,8 @@ def test_act_and_gemv_reject_before_launch():
     assert bq.raw_status("bq_gemm", L_, fake, 2, None, None, None) == 1                # null y
     assert bq.raw_status("bq_gemm", L_, fake, 0, fake, None, None) == 0                # M = 0: no-op
     assert bq.raw_status("bq_gemm", None, fake, 1, fake, None, None) == 1
+
+
+def test_static_scratch_rejects_before_launch():
+    """Null layer / bad sizes are refused on the host, before any device work."""
+    assert bq.raw_status("bq_linear_static_scratch", None, None, 1, None, None, None) == bq.BQ_ERR_INVALID_ARG
