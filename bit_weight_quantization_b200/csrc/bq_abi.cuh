@@ -184,7 +184,9 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   g->tpc = tpc;
   g->TG = (M + tpc - 1) / tpc;
   g->CPG = std::max(1, std::min(L.RB, (sm_count() + g->TG - 1) / g->TG));
-  // warps sharing a row block: as many as the CTA's row blocks leave idle
+  // warps sharing a row block (the k-split): as many as the CTA's row blocks leave idle.
+  // (A split chosen to balance the SM sub-partitions' tile counts measured slower: it gives
+  // a group several row blocks, and each pays a split-K exchange and an epilogue.)
   const int ipc = (L.RB + g->CPG - 1) / g->CPG;
   int wpr = 1;
   while (wpr * 2 <= NW && wpr * 2 * ipc <= NW) wpr *= 2;
@@ -209,15 +211,13 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   g->lbt_smem = rank > 0 && lbt <= 32 * 1024;
   g->off_lbt = take(g->lbt_smem ? lbt : 16);
   const uint64_t fixed = off + 1024;  // + barriers
-  // two CTAs per SM (228 KB, 1 KB reserved per CTA): the next launch's CTA is resident,
-  // and prefetching its weights, while this one computes
-  // (else one CTA per SM with up to 220 KB)
-  uint64_t per_warp = 0;
-  for (const uint64_t limit : {112ull * 1024, 220ull * 1024}) {
-    const uint64_t budget = std::min<uint64_t>(96 * 1024, fixed < limit ? limit - fixed : 0);
-    per_warp = budget / NW;
-    if (per_warp >= 2ull * L.tile_bytes) break;
-  }
+  // The ring takes up to 96 KB. Most layers then leave room for a second CTA on the SM, so
+  // the next launch's CTA is resident, and prefetching its weights, while this one computes;
+  // a layer whose ring and fixed part exceed half of the SM runs alone. (Capping every
+  // layer at half an SM measured slower on mixed-shape layer sequences.)
+  const uint64_t limit = 220 * 1024;
+  const uint64_t budget = std::min<uint64_t>(96 * 1024, fixed < limit ? limit - fixed : 0);
+  const uint64_t per_warp = budget / NW;
   if (per_warp < 2ull * L.tile_bytes) return false;
   g->S = int(std::min<uint64_t>(4, std::max<uint64_t>(2, per_warp / L.tile_bytes)));
   g->C = int(std::max<uint64_t>(1, std::min<uint64_t>(g->T, per_warp / (uint64_t(g->S) * L.tile_bytes))));

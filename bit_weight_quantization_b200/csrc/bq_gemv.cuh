@@ -174,15 +174,29 @@ __device__ __forceinline__ int quant_asym(float x, float d, int z, int qmax) {
 // butterfly within the warp, then, for groups wider than a warp, one exchange through
 // sh[warp] (each call needs its own sh). Every thread of the block calls it; every
 // thread gets its group's result.
+// The up to 8 warp values are read back with two 16-byte loads issued together (sh is
+// 16-byte aligned, T is 4 bytes), so the exchange costs one shared-memory latency.
 template <typename T, typename Op>
 __device__ __forceinline__ T group_reduce(T v, int TPT, T* sh, Op op) {
+  static_assert(sizeof(T) == 4, "32-bit values");
   for (int o = min(16, TPT / 2); o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
   if (TPT > 32) {
     const int warp = threadIdx.x >> 5, wpg = TPT / 32, g0 = (warp / wpg) * wpg;
     if ((threadIdx.x & 31) == 0) sh[warp] = v;
     __syncthreads();
-    v = sh[g0];
-    for (int w = 1; w < wpg; w++) v = op(v, sh[g0 + w]);
+    const uint4 q0 = *reinterpret_cast<const uint4*>(sh), q1 = *reinterpret_cast<const uint4*>(sh + 4);
+    const uint32_t u[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    T e[8];
+#pragma unroll
+    for (int w = 0; w < 8; w++) memcpy(&e[w], &u[w], 4);
+    T r = e[0];
+#pragma unroll
+    for (int w = 1; w < 8; w++)
+      if (w == g0) r = e[w];
+#pragma unroll
+    for (int w = 1; w < 8; w++)
+      if (w > g0 && w < g0 + wpg) r = op(r, e[w]);  // warps g0, g0 + 1, ... in order
+    v = r;
   }
   return v;
 }
@@ -510,8 +524,10 @@ __device__ __forceinline__ void bvsr_tile(const uint4 (&w)[4], const uint4 (&b)[
 // group's named barrier (none when WPR = 1) and one of its warps runs the fused
 // epilogue: after the prologue there is no block-wide synchronization.
 // ---------------------------------------------------------------------------
+// Two CTAs per SM (at most 128 registers a thread): the next launch's CTA must fit beside
+// this one to prefetch its weights.
 template <int FMT, int F0, int F1, int F2, int NW, bool FUSED>
-__global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
+__global__ void __launch_bounds__(NW * 32, 2) k_layer(LayerArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr bool BSIGNED = FMT != BQ_FMT_ABQ;
   constexpr bool BVSR = FMT == BQ_FMT_BVSR4;
@@ -713,13 +729,14 @@ __global__ void __launch_bounds__(NW * 32) k_layer(LayerArgs a) {
     if (wg != gi % WPR || !ok || *fail) continue;
     long long pl[4] = {0, 0, 0, 0};
     float yl[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int w = 0; w < WPR; w++) {
+    for (int w = 0; w < WPR; w++) {  // in warp order
       const size_t s2 = ((size_t(grp) * 2 + buf) * WPR + w) * 32 + lane;
-#pragma unroll
-      for (int c = 0; c < 4; c++) pl[c] += redl[s2 * 4 + c];
+      const longlong2 v0 = *reinterpret_cast<const longlong2*>(redl + s2 * 4);
+      const longlong2 v1 = *reinterpret_cast<const longlong2*>(redl + s2 * 4 + 2);
+      pl[0] += v0.x; pl[1] += v0.y; pl[2] += v1.x; pl[3] += v1.y;
       if (BVSR) {
-#pragma unroll
-        for (int c = 0; c < 4; c++) yl[c] += redf[s2 * 4 + c];
+        const float4 f = *reinterpret_cast<const float4*>(redf + s2 * 4);
+        yl[0] += f.x; yl[1] += f.y; yl[2] += f.z; yl[3] += f.w;
       }
     }
     layer_epilogue<FMT>(a, smem, tokp, rb, m0, mg, lane, rp, lbt_of(gi), pl, yl);
