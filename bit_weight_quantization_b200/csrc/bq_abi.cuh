@@ -184,12 +184,30 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   g->tpc = tpc;
   g->TG = (M + tpc - 1) / tpc;
   g->CPG = std::max(1, std::min(L.RB, (sm_count() + g->TG - 1) / g->TG));
-  // warps sharing a row block (the k-split): as many as the CTA's row blocks leave idle.
-  // (A split chosen to balance the SM sub-partitions' tile counts measured slower: it gives
-  // a group several row blocks, and each pays a split-K exchange and an epilogue.)
+  // Warps sharing a row block (the k-split), a power of two: the one with the least modelled
+  // time. Warp w issues on SM sub-partition w % 4, where the MMA and field-mask issue of a
+  // tile costs about tile_c cycles (measured: ~145 per 8-MMA stream, ~900 for a BVSR tile);
+  // each row block a warp group finishes costs about epi_c cycles (split-K exchange and
+  // epilogue: ~1000 measured with a split, ~300 without). Ties go to the wider split.
   const int ipc = (L.RB + g->CPG - 1) / g->CPG;
+  const long long tile_c = bvsr ? 900 : 145ll * L.nstreams;
   int wpr = 1;
-  while (wpr * 2 <= NW && wpr * 2 * ipc <= NW) wpr *= 2;
+  long long best = -1;
+  for (int w = NW; w >= 1; w /= 2) {
+    const int G = NW / w, T = (L.KT + w - 1) / w;
+    long long load[4] = {0, 0, 0, 0};
+    int max_items = 0;
+    for (int v = 0; v < NW; v++) {
+      const int gr = v / w, wg = v % w;
+      const int items = gr < ipc ? (ipc - gr + G - 1) / G : 0;
+      const int nt = std::max(0, std::min(L.KT, wg * T + T) - wg * T);
+      load[v % 4] += (long long)items * nt * tile_c;
+      max_items = std::max(max_items, items);
+    }
+    const long long cost = std::max(std::max(load[0], load[1]), std::max(load[2], load[3])) +
+                           (long long)max_items * (w > 1 ? 1000 : 300);
+    if (best < 0 || cost < best) { best = cost; wpr = w; }
+  }
   g->WPR = wpr;
   g->T = (L.KT + wpr - 1) / wpr;
   uint64_t off = 0;
@@ -535,7 +553,7 @@ bq_status bq_linear(const bq_layer* layer, const void* x_bf16, int32_t M, float*
   g.x = static_cast<const uint16_t*>(x_bf16);
   if (L.fmt == BQ_FMT_TERNARY_A8 && L.rank > 0) {
     float* up = static_cast<float*>(workspace);
-    if (launch_pdl(k_lora_partial, dim3((L.KT * M + 7) / 8), dim3(256), 0, s, g.x,
+    if (launch_pdl(k_lora_partial, dim3((L.KT * M * (L.rank / 8) + 7) / 8), dim3(256), 0, s, g.x,
                    reinterpret_cast<const uint16_t*>(P + L.off_aux), M, L.K, L.KT, L.rank, up) != cudaSuccess)
       return BQ_ERR_CUDA;
     g.u_part = up;

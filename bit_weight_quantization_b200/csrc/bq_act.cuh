@@ -148,8 +148,11 @@ __global__ void __launch_bounds__(256) k_act_quant(ActArgs a) {
   if (FMT == BQ_FMT_TERNARY_A8 && a.rank > 0) {
     float* up = reinterpret_cast<float*>(a.act + a.off_u);
     const int nw = blockDim.x >> 5, lane = threadIdx.x & 31;
-    for (int kt = kt0 + (threadIdx.x >> 5); kt < kt1; kt += nw)
-      lora_tile_partial_warp(xr, a.lora_A, a.K, a.rank, kt, lane, up + (size_t(kt) * a.M + m) * a.rank);
+    const int nc = a.rank / 8;  // 8-rank chunks
+    for (int i = threadIdx.x >> 5; i < (kt1 - kt0) * nc; i += nw) {
+      const int kt = kt0 + i / nc, rc = (i % nc) * 8;
+      lora_tile_partial_warp(xr, a.lora_A, a.K, a.rank, kt, rc, lane, up + (size_t(kt) * a.M + m) * a.rank);
+    }
   }
 
   if (slice != 0) return;

@@ -415,6 +415,37 @@ __device__ __forceinline__ void layer_epilogue(const LayerArgs& a, const uint8_t
                                                int m0, int mg, int lane, const RowP& rp, const uint8_t* lbt,
                                                const long long (&pl)[4], const float (&yl)[4]) {
   const int g = lane >> 2, t = lane & 3;
+  // ternary: the LoRA term sum_r u[token][r] B^T[row][r] of this lane's 4 outputs, rank in
+  // steps of 8 (u and both B^T rows loaded once for all four), each sum in rank order
+  float lv[4] = {0.f, 0.f, 0.f, 0.f};
+  if (FMT == BQ_FMT_TERNARY_A8 && a.rank > 0) {
+    const float* u0 = reinterpret_cast<const float*>(smem + a.off_u) + size_t(2 * t) * a.rank;
+    const float* u1 = u0 + a.rank;
+    const bool v0 = 2 * t < mg, v1 = 2 * t + 1 < mg;
+    const int r0 = rb * 16 + g;
+    const uint4* bt0 = a.lbt_smem ? reinterpret_cast<const uint4*>(lbt + size_t(g) * a.rank * 2)
+                                  : reinterpret_cast<const uint4*>(a.lora_bt + size_t(r0) * a.rank);
+    const uint4* bt1 = bt0 + a.rank;  // row + 8: 8 rows of rank bf16 = rank uint4 further
+    for (int q8 = 0; q8 < a.rank / 8; q8++) {
+      const uint4 b0 = bt0[q8], b1 = bt1[q8];
+      const float4 ua = v0 ? *reinterpret_cast<const float4*>(u0 + q8 * 8) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 ub = v0 ? *reinterpret_cast<const float4*>(u0 + q8 * 8 + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 uc = v1 ? *reinterpret_cast<const float4*>(u1 + q8 * 8) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 ud = v1 ? *reinterpret_cast<const float4*>(u1 + q8 * 8 + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float uu0[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
+      const float uu1[8] = {uc.x, uc.y, uc.z, uc.w, ud.x, ud.y, ud.z, ud.w};
+      const uint32_t h0[4] = {b0.x, b0.y, b0.z, b0.w}, h1[4] = {b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int e = 0; e < 8; e++) {
+        const float w0 = __uint_as_float((e & 1) ? (h0[e >> 1] & 0xFFFF0000u) : (h0[e >> 1] << 16));
+        const float w1 = __uint_as_float((e & 1) ? (h1[e >> 1] & 0xFFFF0000u) : (h1[e >> 1] << 16));
+        lv[0] = fmaf(uu0[e], w0, lv[0]);
+        lv[1] = fmaf(uu1[e], w0, lv[1]);
+        lv[2] = fmaf(uu0[e], w1, lv[2]);
+        lv[3] = fmaf(uu1[e], w1, lv[3]);
+      }
+    }
+  }
 #pragma unroll
   for (int c = 0; c < 4; c++) {
     const int row = rb * 16 + g + 8 * (c >> 1);
@@ -432,26 +463,7 @@ __device__ __forceinline__ void layer_epilogue(const LayerArgs& a, const uint8_t
       // p = sum_k (T_k + 1) q_k  ->  sum_k T_k q_k = p - sum q
       acc = pl[c] - (long long)int(tk[1]);
       yv = scale * float(acc);
-      if (a.rank > 0) {
-        const float* u = reinterpret_cast<const float*>(smem + a.off_u) + size_t(tl) * a.rank;
-        const uint4* bt = a.lbt_smem ? reinterpret_cast<const uint4*>(lbt + size_t(row - rb * 16) * a.rank * 2)
-                                     : reinterpret_cast<const uint4*>(a.lora_bt + size_t(row) * a.rank);
-        float l = 0.f;
-        for (int q8 = 0; q8 < a.rank / 8; q8 += 4) {  // rank is a multiple of 8
-          uint4 v[4];
-#pragma unroll
-          for (int i = 0; i < 4; i++) v[i] = q8 + i < a.rank / 8 ? bt[q8 + i] : make_uint4(0, 0, 0, 0);
-#pragma unroll
-          for (int i = 0; i < 4; i++) {
-            if (q8 + i >= a.rank / 8) break;
-            const uint32_t h[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-            for (int e = 0; e < 8; e++)
-              l = fmaf(u[(q8 + i) * 8 + e], __uint_as_float((e & 1) ? (h[e >> 1] & 0xFFFF0000u) : (h[e >> 1] << 16)), l);
-          }
-        }
-        yv += __uint_as_float(reinterpret_cast<const uint32_t*>(smem + a.off_tok)[kTokAlpha]) * l;  // tanh(alpha)
-      }
+      if (a.rank > 0) yv += __uint_as_float(reinterpret_cast<const uint32_t*>(smem + a.off_tok)[kTokAlpha]) * lv[c];
     } else if (FMT == BQ_FMT_ABQ) {
       // I = P - z_x S_w - z_w S_x + K z_w z_x
       const long long zx = int(tk[1]), sx = int(tk[2]);
@@ -476,12 +488,11 @@ __device__ __forceinline__ float small_int_to_float(int v) {
 // is bit j of each byte of w[i]; its dot with the codes, d_i, comes from one int8 MMA
 // (scaled by 2^j). Per row and vector the set s gives the template bytes R (table word 7),
 // o and sc = span / sum R (words 4, 5): y += sc sum_i R_i d_i + o S_v, S_v the vector's
-// code sum. TWO: the CTA holds more than one token, so outputs c = 1, 3 (token 2t + 1)
-// are live too; with one token only c = 0, 2 (token 0, lanes t = 0) carry data.
-template <bool TWO>
+// code sum. TWO (warp-uniform): the CTA holds more than one token, so outputs c = 1, 3
+// (token 2t + 1) are live too; with one token only c = 0, 2 (token 0, lanes t = 0) carry data.
 __device__ __forceinline__ void bvsr_tile(const uint4 (&w)[4], const uint4 (&b)[4], uint2 i0, uint2 i1,
-                                          const float* tab, const int* gs_row, int VPR, bool tok0, bool tok1,
-                                          bool want_acc, float (&yacc)[4], long long (&cacc)[4]) {
+                                          const float* tab, const int* gs_row, int VPR, bool TWO, bool tok0,
+                                          bool tok1, bool want_acc, float (&yacc)[4], long long (&cacc)[4]) {
   const uint32_t* tabu = reinterpret_cast<const uint32_t*>(tab);
 #pragma unroll
   for (int j = 0; j < 8; j++) {
@@ -504,7 +515,8 @@ __device__ __forceinline__ void bvsr_tile(const uint4 (&w)[4], const uint4 (&b)[
       const int r0 = int(R[h] & 0xFFu), r1 = int(__byte_perm(R[h], 0, 0x4441)), r2 = int(__byte_perm(R[h], 0, 0x4442)),
                 r3 = int(R[h] >> 24);
 #pragma unroll
-      for (int q = 0; q < (TWO ? 2 : 1); q++) {
+      for (int q = 0; q < 2; q++) {
+        if (q == 1 && !TWO) break;  // warp-uniform
         const int c = 2 * h + q;
         const int E = (r0 * d[0][c] + r1 * d[1][c] + r2 * d[2][c] + r3 * d[3][c]) >> j;
         yacc[c] = fmaf(os[h].y, small_int_to_float(E), fmaf(os[h].x, gsf[q], yacc[c]));
@@ -683,9 +695,8 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(LayerArgs a) {
             const uint8_t* tidx = tp - lane * 16 + 2048;
             const uint2 i0 = *reinterpret_cast<const uint2*>(tidx + g * 8);
             const uint2 i1 = *reinterpret_cast<const uint2*>(tidx + (g + 8) * 8);
-            if (mg > 1) bvsr_tile<true>(w, b, i0, i1, tab, gsum + size_t(2 * t) * VPR + kt * 8, VPR, 2 * t < mg,
-                                        2 * t + 1 < mg, want_acc, yacc, cacc);
-            else bvsr_tile<false>(w, b, i0, i1, tab, gsum + kt * 8, VPR, t == 0, false, want_acc, yacc, cacc);
+            bvsr_tile(w, b, i0, i1, tab, gsum + size_t(2 * t) * VPR + kt * 8, VPR, mg > 1, 2 * t < mg,
+                      2 * t + 1 < mg, want_acc, yacc, cacc);
           }
         }
       }
@@ -748,17 +759,18 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(LayerArgs a) {
 
 // ---------------------------------------------------------------------------
 // Ternary LoRA input (fused path): partial dot products of the unquantized bf16 x
-// with A over each 256-k tile, out[kt][m][r], one warp per (kt, m) (the act kernel
-// computes the same partials with the same warp routine for the unfused path).
+// with A over each 256-k tile, out[kt][m][r], one warp per (kt, m, 8-rank chunk) (the act
+// kernel computes the same partials with the same warp routine for the unfused path).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_lora_partial(const uint16_t* __restrict__ x, const uint16_t* __restrict__ A,
                                                       int M, int K, int KT, int rank, float* __restrict__ out) {
   pdl_trigger();
   pdl_wait();
+  const int nc = rank / 8;  // 8-rank chunks
   const int wid = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (wid >= KT * M) return;
-  const int kt = wid / M, m = wid - kt * M;
-  lora_tile_partial_warp(x + size_t(m) * K, A, K, rank, kt, threadIdx.x & 31, out + (size_t(kt) * M + m) * rank);
+  if (wid >= KT * M * nc) return;
+  const int kt = wid / (M * nc), r2 = wid - kt * M * nc, m = r2 / nc, rc = (r2 - m * nc) * 8;
+  lora_tile_partial_warp(x + size_t(m) * K, A, K, rank, kt, rc, threadIdx.x & 31, out + (size_t(kt) * M + m) * rank);
 }
 
 // ---------------------------------------------------------------------------

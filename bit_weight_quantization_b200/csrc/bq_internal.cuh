@@ -146,43 +146,40 @@ __device__ __forceinline__ int code_word_in_tile(int kin) {
   return 16 * t + 2 * mu + h;
 }
 
-// Ternary LoRA input, one 256-k tile, by one warp: out[r] = sum over the tile's k of
-// x_k A[k][r] for r < rank (K % 128 == 0, so a lane's 8 k's are all inside K or all past
-// it). Lane l takes k = 256 kt + 8l .. 8l + 7 and sums its 8 products in k order; the 32
-// lane sums meet in a fixed xor-butterfly, so every caller gets the same bits.
+// Ternary LoRA input, one 256-k tile and 8 ranks [rc, rc + 8), by one warp: out[i] = sum
+// over the tile's k of x_k A[k][rc + i] (K % 128 == 0, so a lane's 8 k's are all inside K
+// or all past it). Lane l takes k = 256 kt + 8l .. 8l + 7 and sums its 8 products in k
+// order; the 32 lane sums meet in a fixed xor-butterfly, so every caller gets the same bits.
 __device__ __forceinline__ void lora_tile_partial_warp(const uint16_t* xr, const uint16_t* A, int K, int rank,
-                                                       int kt, int lane, float* out) {
+                                                       int kt, int rc, int lane, float* out) {
   const int k0 = kt * 256 + lane * 8;
   const bool in = k0 < K;
-  float xv[8];
-  {
-    const uint4 v = in ? *reinterpret_cast<const uint4*>(xr + k0) : make_uint4(0, 0, 0, 0);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  const uint4 xq = in ? *reinterpret_cast<const uint4*>(xr + k0) : make_uint4(0, 0, 0, 0);
+  uint4 aq[8];
 #pragma unroll
-    for (int e = 0; e < 8; e++) xv[e] = __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+  for (int e = 0; e < 8; e++)
+    aq[e] = in ? *reinterpret_cast<const uint4*>(A + size_t(k0 + e) * rank + rc) : make_uint4(0, 0, 0, 0);
+  const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; i++) acc[i] = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; e++) {
+    const float xv = __uint_as_float((e & 1) ? (xw[e >> 1] & 0xFFFF0000u) : (xw[e >> 1] << 16));
+    const uint32_t w[4] = {aq[e].x, aq[e].y, aq[e].z, aq[e].w};
+#pragma unroll
+    for (int i = 0; i < 8; i++)
+      acc[i] = fmaf(xv, __uint_as_float((i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16)), acc[i]);
   }
-  for (int rc = 0; rc < rank; rc += 8) {
-    float acc[8];
 #pragma unroll
-    for (int i = 0; i < 8; i++) acc[i] = 0.f;
+  for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-    for (int e = 0; e < 8; e++) {
-      const uint4 v = in ? *reinterpret_cast<const uint4*>(A + size_t(k0 + e) * rank + rc) : make_uint4(0, 0, 0, 0);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int i = 0; i < 8; i++) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+  if (lane < 8) {
+    float v = acc[0];
 #pragma unroll
-      for (int i = 0; i < 8; i++)
-        acc[i] = fmaf(xv[e], __uint_as_float((i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16)), acc[i]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-      for (int i = 0; i < 8; i++) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
-    if (lane < 8) {
-      float v = acc[0];
-#pragma unroll
-      for (int i = 1; i < 8; i++) v = lane == i ? acc[i] : v;
-      out[rc + lane] = v;
-    }
+    for (int i = 1; i < 8; i++) v = lane == i ? acc[i] : v;
+    out[rc + lane] = v;
   }
 }
 
