@@ -31,6 +31,8 @@ sys.path.insert(0, ROOT)
 METRIC = "µs/layer & achieved HBM GB/s (% of B200 peak), quantized GEMV/GEMM, M=1..64"
 LLAMA7B = [("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
            ("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008)]
+# projections of a decoder layer that read the same input: one grouped launch each
+LLAMA7B_CALLS = [("q", "k", "v"), ("o",), ("gate", "up"), ("down",)]
 NOMINAL_HBM_GBS = 8000.0
 
 
@@ -185,33 +187,50 @@ def run_reference(args) -> None:
 # ---------------------------------------------------------------------------
 # CUDA arm
 # ---------------------------------------------------------------------------
-def build_stack(layers: int, seed: int, device):
+def build_stack(layers: int, seed: int, device, group: bool = True):
+    """The decode step's layer calls: per decoder layer q,k,v in one grouped call on a shared
+    input, o, gate+up grouped on a shared input, down (or, ungrouped, one call per
+    projection, each with its own input)."""
     import torch
     from bit_weight_quantization_b200 import bq
     gen = torch.Generator(device=device)
     gen.manual_seed(seed)
-    stack = []
+    shapes = {n: (N, K) for n, N, K in LLAMA7B}
+    calls = []
     for l in range(layers):
+        members = {}
         for name, N, K in LLAMA7B:
             W = torch.randn(N, K, device=device, generator=gen, dtype=torch.float32) * 0.02
             ql = bq.QuantLinear("bitnet", W)
             del W
+            members[name] = dict(name=name, N=N, K=K, ql=ql, y=torch.empty(1, N, device=device, dtype=torch.float32))
+        groups = LLAMA7B_CALLS if group else [(n,) for n, _, _ in LLAMA7B]
+        for names in groups:
+            K = shapes[names[0]][1]
             x = torch.randn(1, K, device=device, generator=gen).to(torch.bfloat16)
-            y = torch.empty(1, N, device=device, dtype=torch.float32)
-            act = ql.act_buffer(1)
-            stack.append(dict(name=name, N=N, K=K, ql=ql, x=x, y=y, act=act))
+            ms = [members[n] for n in names]
+            nbytes = sum(layer_bytes("bitnet", m["N"], K)["fused"] for m in ms) - (len(ms) - 1) * 2 * K
+            calls.append(dict(members=ms, x=x, K=K, bytes=nbytes))
     torch.cuda.synchronize()
-    return stack
+    return calls
 
 
-def step_calls(stack, timing=None):
-    """One decode step: bq_linear (activation quantization fused into the GEMV) per layer."""
+def one_call(c, x=None, ys=None):
     from bit_weight_quantization_b200 import bq
-    for i, L in enumerate(stack):
-        ql = L["ql"]
+    x = c["x"] if x is None else x
+    ys = [m["y"] for m in c["members"]] if ys is None else ys
+    if len(c["members"]) == 1:
+        bq.bq_linear(c["members"][0]["ql"].layer, x, 1, ys[0])
+    else:
+        bq.bq_linear_group([m["ql"].layer for m in c["members"]], x, 1, ys)
+
+
+def step_calls(calls, timing=None):
+    """One decode step: every layer call (activation quantization fused into the layer)."""
+    for i, c in enumerate(calls):
         if timing is not None:
             timing[i][0].record()
-        bq.bq_linear(ql.layer, L["x"], 1, L["y"])
+        one_call(c)
         if timing is not None:
             timing[i][1].record()
 
@@ -230,9 +249,10 @@ def run_cuda(args) -> None:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    stack = build_stack(args.layers, args.seed + rank, dev)
-    per_step = sum(layer_bytes("bitnet", L["N"], L["K"])["fused"] for L in stack)
-    n_layers = len(stack)
+    stack = build_stack(args.layers, args.seed + rank, dev, group=not args.no_group)
+    per_step = sum(c["bytes"] for c in stack)
+    n_calls = len(stack)                               # launches per step
+    n_layers = sum(len(c["members"]) for c in stack)   # projections per step
     stream = torch.cuda.Stream(device=dev)
 
     def barrier():
@@ -279,26 +299,24 @@ def run_cuda(args) -> None:
             gemv_ms.append(sum(a.elapsed_time(b) for a, b in timing))
         gemv_ms_step = statistics.median(gemv_ms)
 
-        # end to end through the public API: pinned host x -> device, the 224 calls, y -> host
-        xs_h = torch.cat([L["x"].view(-1) for L in stack]).cpu().pin_memory()
+        # end to end through the public API: pinned host x -> device, every call, y -> host
+        xs_h = torch.cat([c["x"].view(-1) for c in stack]).cpu().pin_memory()
         xs_d = torch.empty_like(xs_h, device=dev)
-        ys_h = torch.empty(sum(L["N"] for L in stack), dtype=torch.float32).pin_memory()
+        ys_h = torch.empty(sum(m["N"] for c in stack for m in c["members"]), dtype=torch.float32).pin_memory()
         ys_d = torch.empty(ys_h.numel(), dtype=torch.float32, device=dev)
-        offs, o = [], 0
-        for L in stack:
-            offs.append(o)
-            o += L["K"]
-        yoffs, o = [], 0
-        for L in stack:
-            yoffs.append(o)
-            o += L["N"]
+        views, xo, yo = [], 0, 0
+        for c in stack:
+            yv = []
+            for m in c["members"]:
+                yv.append(ys_d[yo:yo + m["N"]].view(1, -1))
+                yo += m["N"]
+            views.append((xs_d[xo:xo + c["K"]].view(1, -1), yv))
+            xo += c["K"]
 
         def e2e_step():
             xs_d.copy_(xs_h, non_blocking=True)
-            for i, L in enumerate(stack):
-                ql = L["ql"]
-                x = xs_d[offs[i]:offs[i] + L["K"]].view(1, -1)
-                bq.bq_linear(ql.layer, x, 1, ys_d[yoffs[i]:yoffs[i] + L["N"]])
+            for c, (x, yv) in zip(stack, views):
+                one_call(c, x, yv)
             ys_h.copy_(ys_d, non_blocking=True)
 
         for _ in range(max(1, min(args.warmup, 3))):
@@ -324,9 +342,9 @@ def run_cuda(args) -> None:
     peak, peak_kind = measured_peaks()
     # every launch in the timed region is the dominant kernel (k_layer<BitNet, fused>): its
     # average launch duration is the timed region over the launches in it
-    us_launch = ms_step * 1e3 / n_layers
+    us_launch = ms_step * 1e3 / n_calls
     achieved = per_step / (ms_step * 1e-3) / 1e9
-    traffic = profile_traffic("bitnet_fused_llama7b_mix")
+    traffic = profile_traffic("bitnet_fused_llama7b_mix" if args.no_group else "bitnet_fused_llama7b_grouped")
     out = None
     if rank == 0:
         out = {
@@ -335,9 +353,13 @@ def run_cuda(args) -> None:
             "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": {"workload": "BitNet W1A8 decode GEMV, M=1: 32-layer Llama-7B linear stack "
                                    "(q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008), "
-                                   "bq_linear (act quantization fused into the GEMV) per layer, "
-                                   "PDL between layers, CUDA graph per step",
-                       "layers_per_step": n_layers, "seq_len": 1, "global_batch": world,
+                                   + ("q,k,v and gate,up each one bq_linear_group call on their shared input, "
+                                      "o and down one bq_linear call each"
+                                      if not args.no_group else "one bq_linear call per projection") +
+                                   " (act quantization fused into the layer kernel), PDL between launches, "
+                                   "CUDA graph per step",
+                       "layers_per_step": n_layers, "launches_per_step": n_calls, "seq_len": 1,
+                       "global_batch": world,
                        "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (each step streams %.0f MB of distinct packed weights)"
                              % (per_step / 1e6)},
@@ -345,13 +367,13 @@ def run_cuda(args) -> None:
             "frac_of_peak": value / world / peak, "frac_of_nominal_8tbs": value / world / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_source": peak_kind,
-                         "kernel": "k_layer<BitNet W1A8, fused> (bq_linear): all %d launches of a step" % n_layers,
-                         "bytes_per_launch": per_step / n_layers, "us_per_launch": us_launch,
-                         "serialized_us_per_launch": gemv_ms_step * 1e3 / n_layers},
+                         "kernel": "k_layer<BitNet W1A8, fused>: all %d launches of a step" % n_calls,
+                         "bytes_per_launch": per_step / n_calls, "us_per_launch": us_launch,
+                         "serialized_us_per_launch": gemv_ms_step * 1e3 / n_calls},
             "e2e": {"value": per_step / (e2e_ms * 1e-3) / 1e9 * world, "unit": "GB/s",
                     "h2d_bytes_per_step": int(xs_h.numel() * 2), "d2h_bytes_per_step": int(ys_h.numel() * 4),
                     "ms_per_step": e2e_ms, "path": "eager Python calls of the C ABI, pinned host buffers"},
-            "gpu_launches": n_layers * args.steps,
+            "gpu_launches": n_calls * args.steps,
             "clocks": clk,
         }
     if world > 1:
@@ -519,6 +541,7 @@ def main():
     ap.add_argument("--a-bits", type=int, default=8)
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--unfused", action="store_true", help="bq_quantize_act + bq_gemv/gemm instead of bq_linear")
+    ap.add_argument("--no-group", action="store_true", help="bench: one launch per projection (no bq_linear_group)")
     args = ap.parse_args()
     if args.mode == "configs":
         run_configs(args)

@@ -53,6 +53,8 @@ _SIGS = {
                                                  ctypes.POINTER(ctypes.c_size_t)]),
     "bq_linear": (ctypes.c_int, [ctypes.POINTER(bq_layer), _P, ctypes.c_int32, _P, _P, _P, ctypes.c_size_t, _P]),
     "bq_linear_static_scratch": (ctypes.c_int, [ctypes.POINTER(bq_layer), _P, ctypes.c_int32, _P, _P, _P]),
+    "bq_linear_group": (ctypes.c_int, [ctypes.POINTER(bq_layer), ctypes.c_int32, _P, ctypes.c_int32,
+                                       ctypes.POINTER(_P), ctypes.POINTER(_P), _P]),
     "bq_device_check": (ctypes.c_int, []),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -148,6 +150,16 @@ def bq_linear_workspace_bytes(layer: bq_layer, M: int) -> int:
 
 
 BQ_STATIC_SCRATCH_BYTES = 1 << 20
+BQ_MAX_GROUP = 4
+
+
+def bq_linear_group(layers, x_bf16, M: int, ys, accs=None, stream=None) -> None:
+    """Several layers sharing the input x in one launch (bq_linear_group)."""
+    n = len(layers)
+    arr = (bq_layer * n)(*layers)
+    yp = (_P * n)(*[_ptr(y) for y in ys])
+    ap = None if accs is None else (_P * n)(*[_ptr(a) for a in accs])
+    _check(_lib.bq_linear_group(arr, n, _ptr(x_bf16), M, yp, ap, _stream(stream)), "bq_linear_group")
 
 
 def bq_linear_static_scratch(layer: bq_layer, x_bf16, M: int, y, acc_dbg=None, stream=None) -> None:

@@ -117,14 +117,27 @@ inline uint64_t linear_workspace(const PkLayout& L, int M) {
 }
 
 // Every field of LayerArgs that depends only on the layer, M and the outputs.
+inline GroupLayer group_layer(const PkLayout& L, const void* packed, float* y, int64_t* acc, int rb_begin) {
+  const uint8_t* P = static_cast<const uint8_t*>(packed);
+  GroupLayer m{};
+  m.tiles = P + L.off_tiles;
+  m.hdr = reinterpret_cast<const uint32_t*>(P);
+  m.row_delta = reinterpret_cast<const float*>(P + L.off_rows);
+  m.row_zero = reinterpret_cast<const int*>(P + L.off_rows) + L.N_pad;
+  m.row_sum = reinterpret_cast<const int*>(P + L.off_rows) + 2 * L.N_pad;
+  m.y = y;
+  m.acc = reinterpret_cast<long long*>(acc);
+  m.N = L.N;
+  m.rb_end = rb_begin + L.RB;
+  return m;
+}
+
 inline LayerArgs layer_args(const PkLayout& L, const void* packed, int M, float* y, int64_t* acc) {
   const uint8_t* P = static_cast<const uint8_t*>(packed);
   LayerArgs g{};
-  g.tiles = P + L.off_tiles;
+  g.gl[0] = group_layer(L, packed, y, acc, 0);
+  g.n_grp = 1;
   g.pk_hdr = reinterpret_cast<const uint32_t*>(P);
-  g.row_delta = reinterpret_cast<const float*>(P + L.off_rows);
-  g.row_zero = reinterpret_cast<const int*>(P + L.off_rows) + L.N_pad;
-  g.row_sum = reinterpret_cast<const int*>(P + L.off_rows) + 2 * L.N_pad;
   g.lora_bt = reinterpret_cast<const uint16_t*>(P + L.off_aux2);
   g.bvsr_table = reinterpret_cast<const float*>(P + L.off_aux);
   g.rabit_planes = reinterpret_cast<const uint32_t*>(P + L.off_tiles);
@@ -601,6 +614,42 @@ bq_status bq_linear_static_scratch(const bq_layer* layer, const void* x_bf16, in
   st = static_scratch(&ws);
   if (st != BQ_OK) return st;
   return bq_linear(layer, x_bf16, M, y, acc_dbg, need > 0 ? ws : nullptr, need, stream);
+}
+
+bq_status bq_linear_group(const bq_layer* layers, int32_t n_layers, const void* x_bf16, int32_t M,
+                          float* const* y, int64_t* const* acc_dbg, void* stream) {
+  static_assert(BQ_MAX_GROUP == kMaxGroup, "group size");
+  if (!layers || !y || n_layers < 1 || n_layers > BQ_MAX_GROUP) return BQ_ERR_INVALID_ARG;
+  if (n_layers == 1) return bq_linear(&layers[0], x_bf16, M, y[0], acc_dbg ? acc_dbg[0] : nullptr, nullptr, 0, stream);
+  PkLayout Ls[BQ_MAX_GROUP];
+  for (int i = 0; i < n_layers; i++) {
+    const bq_status st = check_layer(&layers[i], &Ls[i]);
+    if (st != BQ_OK) return st;
+    if (!y[i] || !aligned(y[i], 4) || (acc_dbg && acc_dbg[i] && !aligned(acc_dbg[i], 8))) return BQ_ERR_INVALID_ARG;
+    if (Ls[i].fmt != Ls[0].fmt || Ls[i].K != Ls[0].K || Ls[i].w_bits != Ls[0].w_bits ||
+        Ls[i].a_bits != Ls[0].a_bits)
+      return BQ_ERR_INVALID_ARG;
+  }
+  const PkLayout& L0 = Ls[0];
+  const bool groupable = L0.fmt == BQ_FMT_BITNET_W1A8 || L0.fmt == BQ_FMT_ABQ ||
+                         (L0.fmt == BQ_FMT_TERNARY_A8 && L0.rank == 0);
+  for (int i = 1; i < n_layers; i++)
+    if (Ls[i].rank != L0.rank) return BQ_ERR_INVALID_ARG;
+  if (!groupable) return BQ_ERR_UNSUPPORTED;
+  if (M < 0 || M > BQ_MAX_M) return BQ_ERR_SIZE;
+  if (M == 0) return BQ_OK;
+  if (!x_bf16 || !aligned(x_bf16, 16)) return BQ_ERR_INVALID_ARG;
+  LayerArgs g = layer_args(L0, layers[0].packed, M, y[0], acc_dbg ? acc_dbg[0] : nullptr);
+  g.x = static_cast<const uint16_t*>(x_bf16);
+  int rb = L0.RB;
+  for (int i = 1; i < n_layers; i++) {
+    g.gl[i] = group_layer(Ls[i], layers[i].packed, y[i], acc_dbg ? acc_dbg[i] : nullptr, rb);
+    rb += Ls[i].RB;
+  }
+  g.n_grp = n_layers;
+  PkLayout Lg = L0;  // the work split sees the group's row blocks as one layer
+  Lg.RB = rb;
+  return launch_layer(Lg, g, true, reinterpret_cast<cudaStream_t>(stream));
 }
 
 bq_status bq_gemv(const bq_layer* layer, const void* act, float* y, int64_t* acc_dbg, void* stream) {

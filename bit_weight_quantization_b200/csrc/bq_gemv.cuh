@@ -123,13 +123,25 @@ __device__ __forceinline__ void fold_stream(const int (&acc)[AN][4], int (&p)[4]
   }
 }
 
-struct LayerArgs {
-  // packed weights
+// One layer of a group that shares its input x (same format, K and bit widths): global row
+// blocks [previous rb_end, rb_end) are its row blocks 0, 1, ...
+constexpr int kMaxGroup = 4;
+struct GroupLayer {
   const uint8_t* tiles;
-  const uint32_t* pk_hdr;
+  const uint32_t* hdr;
   const float* row_delta;   // ABQ Delta_w [N_pad]
   const int* row_zero;      // ABQ z_w
   const int* row_sum;       // ABQ S_w
+  float* y;                 // [M][N]
+  long long* acc;           // [M][N] or null
+  int N, rb_end;
+};
+
+struct LayerArgs {
+  GroupLayer gl[kMaxGroup];
+  int n_grp;
+  // packed weights (the single layer, or the group's first)
+  const uint32_t* pk_hdr;
   const uint16_t* lora_bt;  // ternary B^T bf16 [N_pad][r]
   const float* bvsr_table;  // [256][8]
   const uint32_t* rabit_planes;
@@ -161,7 +173,8 @@ struct LayerArgs {
 // ---------------------------------------------------------------------------
 constexpr int kMaxXChunks = 16;   // 16-byte chunks of x held in registers per thread
 // shared token area (words): [8][4] per-token parameters, then tanh(alpha) and the weight scale
-constexpr int kTokAlpha = 32, kTokWScale = 33, kTokWords = 36;
+// and the group members' weight scales
+constexpr int kTokAlpha = 32, kTokWScale = 33, kTokWords = 40;
 
 // asymmetric a-bit code: clamp(rn(x / Delta) + z, 0, 2^a - 1)
 __device__ __forceinline__ int quant_asym(float x, float d, int z, int qmax) {
@@ -214,18 +227,23 @@ __device__ __forceinline__ void prefetch_x(const LayerArgs& a, int m0, int mg, i
   for (int i = threadIdx.x; i < lines; i += NT) asm volatile("prefetch.global.L2 [%0];" ::"l"(base + size_t(i) * 128));
 }
 
-// Output scale of a token (slot 3 of its parameters): BitNet alpha gamma/127, ternary
-// gamma_W gamma/127, BVSR gamma/127, ABQ Delta_x (times Delta_w per row in the epilogue).
-// tw is the layer's weight scale (header word HW_TSCALE), read before griddepcontrol.wait.
+// Token part of the output scale (slot 3 of its parameters): gamma/127 for the A8 formats
+// (the epilogue multiplies BitNet alpha or ternary gamma_W in), ABQ Delta_x (times Delta_w
+// per row in the epilogue).
 template <int FMT>
-__device__ __forceinline__ uint32_t token_scale(float tw, uint32_t word0) {
+__device__ __forceinline__ uint32_t token_scale(uint32_t word0) {
   const float g0 = __uint_as_float(word0);
-  float sc;
-  if (FMT == BQ_FMT_BITNET_W1A8 || FMT == BQ_FMT_TERNARY_A8)
-    sc = __fmul_rn(tw, __fdiv_rn(g0, 127.f));
-  else if (FMT == BQ_FMT_BVSR4) sc = __fdiv_rn(g0, 127.f);
-  else sc = g0;
-  return __float_as_uint(sc);
+  return __float_as_uint(FMT == BQ_FMT_ABQ ? g0 : __fdiv_rn(g0, 127.f));
+}
+
+// The group member holding global row block rb, and rb's index inside that member.
+__device__ __forceinline__ int member_of(const LayerArgs& a, int rb, int& lrb) {
+  int l = 0;
+#pragma unroll
+  for (int i = 0; i < kMaxGroup - 1; i++)
+    if (i + 1 < a.n_grp && rb >= a.gl[i].rb_end) l = i + 1;
+  lrb = rb - (l > 0 ? a.gl[l - 1].rb_end : 0);
+  return l;
 }
 
 // Fused: each token of this CTA is quantized by a group of TPT threads that hold the
@@ -329,7 +347,7 @@ __device__ void stage_quantize(const LayerArgs& a, uint8_t* smem, int m0, int mg
     } else {
       tok[4 * m + 0] = __float_as_uint(p0); tok[4 * m + 1] = uint32_t(total);
     }
-    tok[4 * m + 3] = token_scale<FMT>(__uint_as_float(tok[kTokWScale]), tok[4 * m + 0]);
+    tok[4 * m + 3] = token_scale<FMT>(tok[4 * m + 0]);
   }
 }
 
@@ -357,8 +375,7 @@ __device__ bool stage_copy(const LayerArgs& a, uint8_t* smem, int m0, int mg, ui
   __syncthreads();
   if (*bad) return false;
   uint32_t* tok = reinterpret_cast<uint32_t*>(smem + a.off_tok);
-  const float tw = __uint_as_float(tok[kTokWScale]);
-  if (tid < 4 * mg) tok[tid] = (tid & 3) == 3 ? token_scale<FMT>(tw, a.act_tok[4 * m0 + tid - 3]) : a.act_tok[4 * m0 + tid];
+  if (tid < 4 * mg) tok[tid] = (tid & 3) == 3 ? token_scale<FMT>(a.act_tok[4 * m0 + tid - 3]) : a.act_tok[4 * m0 + tid];
   if (FMT == BQ_FMT_BVSR4) {
     const int VPR = a.K_pad / 32;
     int* gsum = reinterpret_cast<int*>(smem + a.off_gsum);
@@ -397,12 +414,14 @@ struct RowP {
 template <int FMT>
 __device__ __forceinline__ void load_rowp(const LayerArgs& a, int rb, int lane, RowP& rp) {
   if constexpr (FMT == BQ_FMT_ABQ) {
+    int lrb;
+    const GroupLayer& m = a.gl[member_of(a, rb, lrb)];
 #pragma unroll
     for (int h = 0; h < 2; h++) {
-      const int row = rb * 16 + (lane >> 2) + 8 * h;  // < N_pad: the arrays are padded
-      rp.d[h] = __ldg(a.row_delta + row);
-      rp.z[h] = __ldg(a.row_zero + row);
-      rp.s[h] = __ldg(a.row_sum + row);
+      const int row = lrb * 16 + (lane >> 2) + 8 * h;  // < N_pad: the arrays are padded
+      rp.d[h] = __ldg(m.row_delta + row);
+      rp.z[h] = __ldg(m.row_zero + row);
+      rp.s[h] = __ldg(m.row_sum + row);
     }
   }
 }
@@ -446,13 +465,19 @@ __device__ __forceinline__ void layer_epilogue(const LayerArgs& a, const uint8_t
       }
     }
   }
+  int lrb;
+  const int l = member_of(a, rb, lrb);
+  const GroupLayer& mb = a.gl[l];
+  const float tw = __uint_as_float(reinterpret_cast<const uint32_t*>(smem + a.off_tok)[kTokWScale + l]);
 #pragma unroll
   for (int c = 0; c < 4; c++) {
-    const int row = rb * 16 + g + 8 * (c >> 1);
+    const int row = lrb * 16 + g + 8 * (c >> 1);
     const int tl = 2 * t + (c & 1);
-    if (row >= a.N || tl >= mg) continue;
+    if (row >= mb.N || tl >= mg) continue;
     const uint32_t* tk = tok + 4 * tl;
-    const float scale = __uint_as_float(tk[3]);
+    const float scale = (FMT == BQ_FMT_BITNET_W1A8 || FMT == BQ_FMT_TERNARY_A8)
+                            ? __fmul_rn(tw, __uint_as_float(tk[3]))  // alpha or gamma_W times gamma/127
+                            : __uint_as_float(tk[3]);
     long long acc;
     float yv;
     if (FMT == BQ_FMT_BITNET_W1A8) {
@@ -474,8 +499,8 @@ __device__ __forceinline__ void layer_epilogue(const LayerArgs& a, const uint8_t
       acc = pl[c];
       yv = scale * yl[c];
     }
-    a.y[size_t(m0 + tl) * a.N + row] = yv;
-    if (a.acc) a.acc[size_t(m0 + tl) * a.N + row] = acc;
+    mb.y[size_t(m0 + tl) * mb.N + row] = yv;
+    if (mb.acc) mb.acc[size_t(m0 + tl) * mb.N + row] = acc;
   }
 }
 
@@ -539,7 +564,7 @@ __device__ __forceinline__ void bvsr_tile(const uint4 (&w)[4], const uint4 (&b)[
 // Two CTAs per SM (at most 128 registers a thread): the next launch's CTA must fit beside
 // this one to prefetch its weights.
 template <int FMT, int F0, int F1, int F2, int NW, bool FUSED>
-__global__ void __launch_bounds__(NW * 32, 2) k_layer(LayerArgs a) {
+__global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ LayerArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr bool BSIGNED = FMT != BQ_FMT_ABQ;
   constexpr bool BVSR = FMT == BQ_FMT_BVSR4;
@@ -577,9 +602,11 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(LayerArgs a) {
     const int st = e % a.S;
     const int kt = kt_begin + (e % cpw) * a.C;
     const uint32_t bytes = uint32_t(chunk_tiles(e)) * uint32_t(a.tile_bytes);
+    int lrb;
+    const uint8_t* tiles = a.gl[member_of(a, rb_of(e / cpw), lrb)].tiles;
     mbar_expect_tx(&wbar[st], bytes);
-    bulk_g2s(ring + size_t(st) * a.C * a.tile_bytes,
-             a.tiles + (size_t(rb_of(e / cpw)) * a.KT + kt) * a.tile_bytes, bytes, &wbar[st]);
+    bulk_g2s(ring + size_t(st) * a.C * a.tile_bytes, tiles + (size_t(lrb) * a.KT + kt) * a.tile_bytes, bytes,
+             &wbar[st]);
   };
   const int first = min(n_my, a.S);
   if (lane == 0) {
@@ -603,7 +630,7 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(LayerArgs a) {
   if (tid == 0) {
     *fail = 0;
     uint32_t* tw = reinterpret_cast<uint32_t*>(smem + a.off_tok);
-    tw[kTokWScale] = a.pk_hdr[HW_TSCALE];
+    for (int l = 0; l < a.n_grp; l++) tw[kTokWScale + l] = a.gl[l].hdr[HW_TSCALE];
     if (FMT == BQ_FMT_TERNARY_A8) tw[kTokAlpha] = __float_as_uint(tanhf(__uint_as_float(a.pk_hdr[HW_LORA_ALPHA])));
   }
   RowP rp;
@@ -629,7 +656,7 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(LayerArgs a) {
   const int VPR = a.K_pad / 32;
   const int* gsum = reinterpret_cast<const int*>(smem + a.off_gsum);
   const float* tab = reinterpret_cast<const float*>(smem + a.off_tab);
-  const bool want_acc = a.acc != nullptr;
+  const bool want_acc = a.gl[0].acc != nullptr;  // BVSR (never grouped)
   long long* redl = reinterpret_cast<long long*>(smem + a.off_red);                // [G][2][WPR][32][4]
   float* redf = reinterpret_cast<float*>(smem + a.off_red + 2 * NW * 32 * 4 * 8);  // same shape
   bool copies_ok = true;

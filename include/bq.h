@@ -191,6 +191,23 @@ bq_status bq_linear_workspace_bytes(const bq_layer* layer, int32_t M, size_t* by
 bq_status bq_linear(const bq_layer* layer, const void* x_bf16, int32_t M, float* y, int64_t* acc_dbg,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* Several layers that read the same input x, in one launch: e.g. the q, k and v projections
+ * of a decoder layer, or its gate and up projections. Each layer keeps its own packed buffer
+ * and scales; x is quantized once (as bq_linear does) and every layer's y computed from it.
+ * The pages describe one layer at a time; this is that same computation for several weight
+ * matrices sharing the input, so that the fixed cost of a launch (waiting for x, quantizing
+ * it, the epilogue drain) is paid once.
+ *  - layers: host array of n_layers (1..BQ_MAX_GROUP) descriptors, all of one format, K,
+ *    w_bits and a_bits. More than one layer is supported for BitNet, ABQ and ternary
+ *    without a LoRA term; other formats return BQ_ERR_UNSUPPORTED (use bq_linear).
+ *  - y: host array of n_layers device pointers, f32 [M][N_i] each. acc_dbg: NULL, or a host
+ *    array of n_layers nullable device int64 [M][N_i] pointers.
+ *  - Results equal separate bq_linear calls bit for bit. Same errors as bq_linear, plus
+ *    BQ_ERR_INVALID_ARG for mismatched layers. */
+#define BQ_MAX_GROUP 4
+bq_status bq_linear_group(const bq_layer* layers, int32_t n_layers, const void* x_bf16, int32_t M,
+                          float* const* y, int64_t* const* acc_dbg, void* stream);
+
 /* bq_linear with its scratch in a fixed device array inside the library instead of a
  * caller workspace. The pages have no counterpart: this is a calling convenience, not a
  * step of the method. It is for callers that cannot allocate device memory where they

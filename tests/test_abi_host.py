@@ -177,3 +177,29 @@ def test_act_and_gemv_reject_before_launch():
 def test_static_scratch_rejects_before_launch():
     """Null layer / bad sizes are refused on the host, before any device work."""
     assert bq.raw_status("bq_linear_static_scratch", None, None, 1, None, None, None) == bq.BQ_ERR_INVALID_ARG
+
+
+def test_linear_group_rejects_before_launch():
+    """Grouped layers: sizes, mismatches and unsupported formats are refused on the host."""
+    def layer(fmt, N, K, **kw):
+        return bq.bq_packed_validate(_host_header(fmt, N, K, **kw).tobytes(), 1 << 20)
+    fake = 1 << 40
+    a, b = layer("bitnet", 64, 256), layer("bitnet", 32, 256)
+    ys = [fake, fake]
+
+    def st(layers, M=1, x=fake, y=ys):
+        arr = (bq.bq_layer * len(layers))(*layers)
+        yp = (ctypes.c_void_p * len(y))(*y)
+        return bq.raw_status("bq_linear_group", arr, len(layers), x, M, yp, None, None)
+    assert st([a, b], M=0) == bq.BQ_OK                                  # nothing to do
+    assert st([a, b], M=65) == bq.BQ_ERR_SIZE
+    assert st([a, b], x=fake + 2) == bq.BQ_ERR_INVALID_ARG               # x unaligned
+    assert st([a, b], y=[fake, 0]) == bq.BQ_ERR_INVALID_ARG              # null y
+    assert st([a, layer("bitnet", 32, 512)]) == bq.BQ_ERR_INVALID_ARG    # K differs
+    assert st([a, layer("abq", 32, 256, w_bits=4, a_bits=4)]) == bq.BQ_ERR_INVALID_ARG
+    assert st([layer("bvsr", 32, 256)] * 2) == bq.BQ_ERR_UNSUPPORTED
+    assert st([layer("ternary", 32, 256, lora_rank=32)] * 2) == bq.BQ_ERR_UNSUPPORTED
+    arr = (bq.bq_layer * 5)(*([a] * 5))
+    yp = (ctypes.c_void_p * 5)(*([fake] * 5))
+    assert bq.raw_status("bq_linear_group", arr, 5, fake, 1, yp, None, None) == bq.BQ_ERR_INVALID_ARG
+    assert bq.raw_status("bq_linear_group", arr, 0, fake, 1, yp, None, None) == bq.BQ_ERR_INVALID_ARG

@@ -10,7 +10,8 @@ import pytest
 
 import bq_inputs as I
 from oracle import bq_oracle as O
-from tests.parity_util import GpuLayer, assert_y_close, check_act, oracle_layer, oracle_pack, ulp_diff
+from tests.parity_util import (GpuLayer, assert_y_close, check_act, oracle_layer, oracle_pack, to_dev_bf16,
+                               to_dev_f32, ulp_diff)
 
 pytestmark = pytest.mark.gpu
 
@@ -204,3 +205,43 @@ def test_act_buffer_mismatch_is_reported():
     assert e.value.status == bq.BQ_ERR_DEVICE_CHECK
     assert torch.all(y == 7.0)
     bq.bq_device_check()   # the word was cleared
+
+
+# ------------------------------------------------------------------ grouped layers sharing x
+@pytest.mark.parametrize("fmt,Ns,K,M,wa", [("bitnet", (64, 97, 40), 512, 1, (1, 8)),
+                                           ("bitnet", (4096, 4096, 4096), 4096, 1, (1, 8)),
+                                           ("bitnet", (33, 16), 1280, 9, (1, 8)),
+                                           ("abq", (50, 33), 384, 9, (4, 4)),
+                                           ("abq", (11008, 11008), 4096, 1, (2, 8)),
+                                           ("ternary", (48, 80, 16, 31), 640, 3, (2, 8))])
+def test_linear_group_equals_separate_calls(fmt, Ns, K, M, wa):
+    """One grouped launch gives, bit for bit, what separate bq_linear calls give (each of
+    which the other tests hold to the oracle); the first member is also checked against the
+    oracle directly."""
+    from tests.parity_util import torch_mods
+    torch, bq = torch_mods()
+    w, a = wa
+    x = to_dev_bf16(I.activations(M, K, seed=11))
+    qls, inps = [], []
+    for i, N in enumerate(Ns):
+        inp = I.layer_inputs(fmt, N, K, M, seed=20 + i, lora_rank=0)
+        kw = dict(w_bits=w, a_bits=a) if fmt == "abq" else {}
+        qls.append(bq.QuantLinear(fmt, to_dev_f32(inp["W"]), **kw))
+        inps.append(inp)
+    ys = [torch.full((M, N), float("nan"), device="cuda") for N in Ns]
+    accs = [torch.full((M, N), -(1 << 62), dtype=torch.int64, device="cuda") for N in Ns]
+    bq.bq_linear_group([q.layer for q in qls], x, M, ys, accs)
+    for q, y, acc, N in zip(qls, ys, accs, Ns):
+        y1 = torch.full((M, N), float("nan"), device="cuda")
+        a1 = torch.full((M, N), -(1 << 62), dtype=torch.int64, device="cuda")
+        q.linear(x, y1, a1)
+        torch.cuda.synchronize()
+        assert torch.equal(acc, a1)
+        assert torch.equal(y, y1)
+    bq.bq_device_check()
+    from tests.parity_util import L as layout
+    p = layout.read_packed(qls[0].packed.cpu().numpy().tobytes())
+    xh = I.activations(M, K, seed=11)
+    r = oracle_layer(fmt, p, xh, a)
+    assert np.array_equal(accs[0].cpu().numpy(), r["acc"])
+    assert_y_close(ys[0].cpu().numpy(), r["y"], f"{fmt} group member 0")
