@@ -351,6 +351,62 @@ __device__ void stage_quantize(const LayerArgs& a, uint8_t* smem, int m0, int mg
   }
 }
 
+// One token per CTA (decode), A8 formats without vector sums (BitNet, ternary): the same
+// arithmetic as stage_quantize, for all 256 threads on the one token, with JM (a compile-time
+// bound on the chunks a thread holds) unrolled. max|x| compares the bf16 bit patterns of |x|
+// as integers (exact for non-negative values); the code sum adds the packed bytes by dp4a.
+template <int FMT, int NW, int JM>
+__device__ void stage_quantize_1tok(const LayerArgs& a, uint8_t* smem, int m0) {
+  constexpr int NT = NW * 32;
+  const int tid = threadIdx.x, nch = a.K / 8, npad = a.K_pad / 8;
+  const uint4* xr = reinterpret_cast<const uint4*>(a.x + size_t(m0) * a.K);
+  uint4 xv[JM];
+#pragma unroll
+  for (int j = 0; j < JM; j++) {
+    const int c = tid + j * NT;
+    xv[j] = c < nch ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+  }
+  uint32_t mb = 0;  // f32 bit pattern of max |x| (bf16 values widened)
+#pragma unroll
+  for (int j = 0; j < JM; j++) {
+    const uint32_t w[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
+#pragma unroll
+    for (int h = 0; h < 4; h++) mb = max(mb, max(w[h] & 0x7FFF0000u, (w[h] << 16) & 0x7FFF0000u));
+  }
+  uint32_t* sh = reinterpret_cast<uint32_t*>(smem + a.off_red);
+  mb = group_reduce(mb, NT, sh, [](uint32_t x, uint32_t y) { return max(x, y); });
+  const float gmax = __uint_as_float(mb);
+  const float sc = gmax > 0.f ? __fdiv_rn(127.f, gmax) : 0.f;  // 127/gamma; gamma = 0 gives q = 0
+  uint32_t* cw = reinterpret_cast<uint32_t*>(smem + a.off_codes);
+  int qsum = 0;
+#pragma unroll
+  for (int j = 0; j < JM; j++) {
+    const int c = tid + j * NT;
+    if (c < npad) {  // chunks past K hold x = 0, so code 0
+      const uint32_t w[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
+      uint32_t q8[8];
+#pragma unroll
+      for (int e = 0; e < 8; e++)
+        q8[e] = rn_biased(__fmul_rn(__uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16)), sc));
+      const uint32_t word0 = __byte_perm(__byte_perm(q8[0], q8[1], 0x0040), __byte_perm(q8[2], q8[3], 0x0040), 0x5410);
+      const uint32_t word1 = __byte_perm(__byte_perm(q8[4], q8[5], 0x0040), __byte_perm(q8[6], q8[7], 0x0040), 0x5410);
+      qsum = __dp4a(int(word0), 0x01010101, qsum);
+      qsum = __dp4a(int(word1), 0x01010101, qsum);
+      const int k = c * 8;
+      cw[(k >> 8) * 64 + code_word_in_tile(k & 255)] = word0;
+      cw[((k + 4) >> 8) * 64 + code_word_in_tile((k + 4) & 255)] = word1;
+    }
+  }
+  int* shs = reinterpret_cast<int*>(smem + a.off_red) + 64;
+  const int total = group_reduce(qsum, NT, shs, [](int x, int y) { return x + y; });
+  if (tid == 0) {
+    uint32_t* tok = reinterpret_cast<uint32_t*>(smem + a.off_tok);
+    tok[0] = mb;
+    tok[1] = uint32_t(total);
+    tok[3] = token_scale<FMT>(mb);
+  }
+}
+
 // Unfused: this CTA's tokens from the act buffer (after checking its header): the codes
 // by one bulk copy per token, token parameters and BVSR sums by plain loads.
 template <int FMT, int NW>
@@ -641,8 +697,15 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
   pdl_wait();
   bool ok = true;
   const uint32_t* tokp = reinterpret_cast<const uint32_t*>(smem + a.off_tok);
-  if constexpr (FUSED) stage_quantize<FMT, NW>(a, smem, m0, mg);
-  else ok = stage_copy<FMT, NW>(a, smem, m0, mg, xbar);
+  if constexpr (FUSED) {
+    constexpr bool FAST = FMT == BQ_FMT_BITNET_W1A8 || FMT == BQ_FMT_TERNARY_A8;
+    if (FAST && mg == 1 && a.J <= 2) stage_quantize_1tok<FMT, NW, 2>(a, smem, m0);
+    else if (FAST && mg == 1 && a.J <= 4) stage_quantize_1tok<FMT, NW, 4>(a, smem, m0);
+    else if (FAST && mg == 1 && a.J <= 8) stage_quantize_1tok<FMT, NW, 8>(a, smem, m0);
+    else stage_quantize<FMT, NW>(a, smem, m0, mg);
+  } else {
+    ok = stage_copy<FMT, NW>(a, smem, m0, mg, xbar);
+  }
   __syncthreads();
   if (FMT == BQ_FMT_TERNARY_A8 && a.rank > 0) {
     if (ok) stage_lora_u(a, smem, m0, mg, NW * 32);
