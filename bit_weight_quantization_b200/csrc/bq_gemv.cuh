@@ -351,14 +351,16 @@ __device__ void stage_quantize(const LayerArgs& a, uint8_t* smem, int m0, int mg
   }
 }
 
-// One token per CTA (decode), A8 formats without vector sums (BitNet, ternary): the same
-// arithmetic as stage_quantize, for all 256 threads on the one token, with JM (a compile-time
-// bound on the chunks a thread holds) unrolled. max|x| compares the bf16 bit patterns of |x|
-// as integers (exact for non-negative values); the code sum adds the packed bytes by dp4a.
+// One token per CTA (decode): the same arithmetic as stage_quantize, with all 256 threads on
+// the one token and JM (a compile-time bound on the 16-byte chunks a thread holds) unrolled.
+// A8 formats: max|x| compares the bf16 bit patterns of |x| as integers (exact for
+// non-negative values); ABQ: min and max in one exchange. Code sums add the packed bytes by
+// dp4a; BVSR vector sums combine 4 neighbouring threads (32 elements).
 template <int FMT, int NW, int JM>
 __device__ void stage_quantize_1tok(const LayerArgs& a, uint8_t* smem, int m0) {
   constexpr int NT = NW * 32;
-  const int tid = threadIdx.x, nch = a.K / 8, npad = a.K_pad / 8;
+  constexpr bool ABQ = FMT == BQ_FMT_ABQ;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nch = a.K / 8, npad = a.K_pad / 8;
   const uint4* xr = reinterpret_cast<const uint4*>(a.x + size_t(m0) * a.K);
   uint4 xv[JM];
 #pragma unroll
@@ -366,44 +368,92 @@ __device__ void stage_quantize_1tok(const LayerArgs& a, uint8_t* smem, int m0) {
     const int c = tid + j * NT;
     xv[j] = c < nch ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
   }
-  uint32_t mb = 0;  // f32 bit pattern of max |x| (bf16 values widened)
+  float* shf = reinterpret_cast<float*>(smem + a.off_red);  // [0, 32) and [32, 64): the two exchanges
+  float sc = 0.f, d = 1.f;
+  int z = 0;
+  uint32_t w0 = 0;  // token word 0: gamma (A8) or Delta (ABQ)
+  const int qmax = (1 << a.a_bits) - 1;
+  if constexpr (!ABQ) {
+    uint32_t mb = 0;  // f32 bit pattern of max |x| (bf16 values widened)
 #pragma unroll
-  for (int j = 0; j < JM; j++) {
-    const uint32_t w[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
+    for (int j = 0; j < JM; j++) {
+      const uint32_t w[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
 #pragma unroll
-    for (int h = 0; h < 4; h++) mb = max(mb, max(w[h] & 0x7FFF0000u, (w[h] << 16) & 0x7FFF0000u));
+      for (int h = 0; h < 4; h++) mb = max(mb, max(w[h] & 0x7FFF0000u, (w[h] << 16) & 0x7FFF0000u));
+    }
+    mb = group_reduce(mb, NT, reinterpret_cast<uint32_t*>(shf), [](uint32_t x, uint32_t y) { return max(x, y); });
+    const float gmax = __uint_as_float(mb);
+    sc = gmax > 0.f ? __fdiv_rn(127.f, gmax) : 0.f;  // 127/gamma; gamma = 0 gives q = 0
+    w0 = mb;
+  } else {
+    float lo = INFINITY, hi = -INFINITY;  // over the real elements only
+#pragma unroll
+    for (int j = 0; j < JM; j++) {
+      if (tid + j * NT >= nch) continue;
+      const uint32_t w[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
+#pragma unroll
+      for (int h = 0; h < 4; h++) {
+        const float e0 = __uint_as_float(w[h] << 16), e1 = __uint_as_float(w[h] & 0xFFFF0000u);
+        lo = fminf(lo, fminf(e0, e1));
+        hi = fmaxf(hi, fmaxf(e0, e1));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if (lane == 0) { shf[warp] = lo; shf[32 + warp] = hi; }
+    __syncthreads();
+    const float4 l0 = *reinterpret_cast<const float4*>(shf), l1 = *reinterpret_cast<const float4*>(shf + 4);
+    const float4 h0 = *reinterpret_cast<const float4*>(shf + 32), h1 = *reinterpret_cast<const float4*>(shf + 36);
+    lo = fminf(fminf(fminf(l0.x, l0.y), fminf(l0.z, l0.w)), fminf(fminf(l1.x, l1.y), fminf(l1.z, l1.w)));
+    hi = fmaxf(fmaxf(fmaxf(h0.x, h0.y), fmaxf(h0.z, h0.w)), fmaxf(fmaxf(h1.x, h1.y), fmaxf(h1.z, h1.w)));
+    d = __fdiv_rn(fmaxf(__fsub_rn(hi, lo), 1e-5f), float(qmax));
+    z = int(rintf(__fdiv_rn(-lo, d)));
+    w0 = __float_as_uint(d);
   }
-  uint32_t* sh = reinterpret_cast<uint32_t*>(smem + a.off_red);
-  mb = group_reduce(mb, NT, sh, [](uint32_t x, uint32_t y) { return max(x, y); });
-  const float gmax = __uint_as_float(mb);
-  const float sc = gmax > 0.f ? __fdiv_rn(127.f, gmax) : 0.f;  // 127/gamma; gamma = 0 gives q = 0
   uint32_t* cw = reinterpret_cast<uint32_t*>(smem + a.off_codes);
+  int* gsum = reinterpret_cast<int*>(smem + a.off_gsum);
   int qsum = 0;
 #pragma unroll
   for (int j = 0; j < JM; j++) {
     const int c = tid + j * NT;
-    if (c < npad) {  // chunks past K hold x = 0, so code 0
+    if (j * NT >= npad) break;  // uniform: no thread has chunks left
+    uint32_t word0 = 0, word1 = 0;
+    if (c < nch) {
       const uint32_t w[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
       uint32_t q8[8];
 #pragma unroll
-      for (int e = 0; e < 8; e++)
-        q8[e] = rn_biased(__fmul_rn(__uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16)), sc));
-      const uint32_t word0 = __byte_perm(__byte_perm(q8[0], q8[1], 0x0040), __byte_perm(q8[2], q8[3], 0x0040), 0x5410);
-      const uint32_t word1 = __byte_perm(__byte_perm(q8[4], q8[5], 0x0040), __byte_perm(q8[6], q8[7], 0x0040), 0x5410);
-      qsum = __dp4a(int(word0), 0x01010101, qsum);
-      qsum = __dp4a(int(word1), 0x01010101, qsum);
+      for (int e = 0; e < 8; e++) {
+        const float xf = __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+        q8[e] = ABQ ? uint32_t(quant_asym(xf, d, z, qmax)) : rn_biased(__fmul_rn(xf, sc));
+      }
+      word0 = __byte_perm(__byte_perm(q8[0], q8[1], 0x0040), __byte_perm(q8[2], q8[3], 0x0040), 0x5410);
+      word1 = __byte_perm(__byte_perm(q8[4], q8[5], 0x0040), __byte_perm(q8[6], q8[7], 0x0040), 0x5410);
+    }
+    int qs = ABQ ? int(__dp4a(word0, 0x01010101u, __dp4a(word1, 0x01010101u, 0u)))
+                 : __dp4a(int(word0), 0x01010101, __dp4a(int(word1), 0x01010101, 0));
+    qsum += qs;
+    if (c < npad) {  // chunks past K hold code 0
       const int k = c * 8;
       cw[(k >> 8) * 64 + code_word_in_tile(k & 255)] = word0;
       cw[((k + 4) >> 8) * 64 + code_word_in_tile((k + 4) & 255)] = word1;
+    }
+    if (FMT == BQ_FMT_BVSR4) {  // 4 consecutive threads cover one 32-element vector
+      qs += __shfl_xor_sync(0xffffffffu, qs, 1);
+      qs += __shfl_xor_sync(0xffffffffu, qs, 2);
+      if (c < npad && (c & 3) == 0) gsum[c >> 2] = qs;
     }
   }
   int* shs = reinterpret_cast<int*>(smem + a.off_red) + 64;
   const int total = group_reduce(qsum, NT, shs, [](int x, int y) { return x + y; });
   if (tid == 0) {
     uint32_t* tok = reinterpret_cast<uint32_t*>(smem + a.off_tok);
-    tok[0] = mb;
-    tok[1] = uint32_t(total);
-    tok[3] = token_scale<FMT>(mb);
+    tok[0] = w0;
+    tok[1] = ABQ ? uint32_t(z) : uint32_t(total);
+    tok[2] = ABQ ? uint32_t(total) : 0u;
+    tok[3] = token_scale<FMT>(w0);
   }
 }
 
@@ -698,10 +748,9 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
   bool ok = true;
   const uint32_t* tokp = reinterpret_cast<const uint32_t*>(smem + a.off_tok);
   if constexpr (FUSED) {
-    constexpr bool FAST = FMT == BQ_FMT_BITNET_W1A8 || FMT == BQ_FMT_TERNARY_A8;
-    if (FAST && mg == 1 && a.J <= 2) stage_quantize_1tok<FMT, NW, 2>(a, smem, m0);
-    else if (FAST && mg == 1 && a.J <= 4) stage_quantize_1tok<FMT, NW, 4>(a, smem, m0);
-    else if (FAST && mg == 1 && a.J <= 8) stage_quantize_1tok<FMT, NW, 8>(a, smem, m0);
+    if (mg == 1 && a.J <= 2) stage_quantize_1tok<FMT, NW, 2>(a, smem, m0);
+    else if (mg == 1 && a.J <= 4) stage_quantize_1tok<FMT, NW, 4>(a, smem, m0);
+    else if (mg == 1 && a.J <= 8) stage_quantize_1tok<FMT, NW, 8>(a, smem, m0);
     else stage_quantize<FMT, NW>(a, smem, m0, mg);
   } else {
     ok = stage_copy<FMT, NW>(a, smem, m0, mg, xbar);
