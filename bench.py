@@ -61,6 +61,22 @@ def layer_bytes(fmt: str, N: int, K: int, M: int = 1, w_bits: int = 1, a_bits: i
     return dict(gemv=gemv, act=actb, total=gemv + actb, fused=fused)
 
 
+def reduce_max_over_ranks(values, dist=None, device=None) -> list:
+    """Each value's maximum over the ranks (a job's device time is its slowest rank's). With no
+    initialized process group, or one rank, the values come back unchanged."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist is not None and dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def job_value(bytes_per_step: float, steps: int, ms_max: float, world: int) -> float:
+    """Whole-job GB/s of `world` replicas, each streaming bytes_per_step for `steps` steps,
+    timed by the slowest rank (ms_max)."""
+    return world * bytes_per_step * steps / (ms_max * 1e-3) / 1e9
+
+
 def measured_peaks() -> tuple[float, str]:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -333,12 +349,9 @@ def run_cuda(args) -> None:
         e2e_ms = t0.elapsed_time(t1) / n_e2e
         bq.bq_device_check()
 
-    ms_t = torch.tensor([ms, e2e_ms], device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms, e2e_ms = float(ms_t[0]), float(ms_t[1])
+    ms, e2e_ms = reduce_max_over_ranks([ms, e2e_ms], dist if world > 1 else None, dev)
     ms_step = ms / args.steps
-    value = world * per_step * args.steps / (ms * 1e-3) / 1e9
+    value = job_value(per_step, args.steps, ms, world)
     peak, peak_kind = measured_peaks()
     # every launch in the timed region is the dominant kernel (k_layer<BitNet, fused>): its
     # average launch duration is the timed region over the launches in it
@@ -370,7 +383,7 @@ def run_cuda(args) -> None:
                          "kernel": "k_layer<BitNet W1A8, fused>: all %d launches of a step" % n_calls,
                          "bytes_per_launch": per_step / n_calls, "us_per_launch": us_launch,
                          "serialized_us_per_launch": gemv_ms_step * 1e3 / n_calls},
-            "e2e": {"value": per_step / (e2e_ms * 1e-3) / 1e9 * world, "unit": "GB/s",
+            "e2e": {"value": job_value(per_step, 1, e2e_ms, world), "unit": "GB/s",
                     "h2d_bytes_per_step": int(xs_h.numel() * 2), "d2h_bytes_per_step": int(ys_h.numel() * 4),
                     "ms_per_step": e2e_ms, "path": "eager Python calls of the C ABI, pinned host buffers"},
             "gpu_launches": n_calls * args.steps,
