@@ -188,8 +188,7 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   if (fused) {
     auto J = [&](int t) { return (npad + NT / pow2ceil(t) - 1) / (NT / pow2ceil(t)); };
     while (tpc > 1 && J(tpc) > kMaxXChunks) tpc--;
-    if (J(tpc) > kMaxXChunks) return false;
-    g->J = J(tpc);
+    g->J = J(tpc) > kMaxXChunks ? 0 : J(tpc);  // 0 (then tpc = 1): the staging reads x twice
   } else {
     while (tpc > 1 && uint64_t(tpc) * g->cstride > 96 * 1024) tpc--;
     g->J = 0;
@@ -261,9 +260,9 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
 
 // One instantiation per kernel, so the static below tracks that kernel's raised
 // dynamic shared-memory limit (processes drive one device each).
-template <int FMT, int F0, int F1, int F2, int NW, bool FUSED>
+template <int FMT, int F0, int F1, int F2, int NW, bool FUSED, bool T1>
 inline cudaError_t launch_tiled_nw(const LayerArgs& g, dim3 grid, cudaStream_t s) {
-  auto k = k_layer<FMT, F0, F1, F2, NW, FUSED>;
+  auto k = k_layer<FMT, F0, F1, F2, NW, FUSED, T1>;
   static uint32_t smem_limit = 48 * 1024;
   if (g.smem_bytes > smem_limit) {
     const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(g.smem_bytes));
@@ -279,7 +278,8 @@ inline cudaError_t launch_tiled_nw(const LayerArgs& g, dim3 grid, cudaStream_t s
 template <int FMT, int F0, int F1, int F2, bool FUSED>
 inline cudaError_t launch_tiled(const LayerArgs& g, int NW, dim3 grid, cudaStream_t s) {
   (void)NW;
-  return launch_tiled_nw<FMT, F0, F1, F2, 8, FUSED>(g, grid, s);
+  if (FUSED && g.tpc == 1) return launch_tiled_nw<FMT, F0, F1, F2, 8, FUSED, FUSED>(g, grid, s);
+  return launch_tiled_nw<FMT, F0, F1, F2, 8, FUSED, false>(g, grid, s);
 }
 
 template <bool FUSED>

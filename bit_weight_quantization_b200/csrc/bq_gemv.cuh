@@ -457,6 +457,97 @@ __device__ void stage_quantize_1tok(const LayerArgs& a, uint8_t* smem, int m0) {
   }
 }
 
+// Rows too long to hold in registers (more than kMaxXChunks chunks a thread, K > 32768 for
+// one token): the same arithmetic as stage_quantize, reading x twice (once for the scale,
+// once to code it).
+template <int FMT, int NW>
+__device__ void stage_quantize_reload(const LayerArgs& a, uint8_t* smem, int m0, int mg) {
+  constexpr int NT = NW * 32;
+  const int tid = threadIdx.x, K = a.K;
+  float* sh_lo = reinterpret_cast<float*>(smem + a.off_red);
+  float* sh_hi = sh_lo + 32;
+  int* sh_sum = reinterpret_cast<int*>(sh_lo + 64);
+  int mgp = 1;
+  while (mgp < mg) mgp <<= 1;
+  const int TPT = NT / mgp;
+  const int m = tid / TPT, lt = tid - m * TPT;
+  const bool active = m < mg;
+  const int nch = K / 8, npad = a.K_pad / 8;
+  const uint4* xr = reinterpret_cast<const uint4*>(a.x + size_t(m0 + (active ? m : 0)) * K);
+  float p0 = FMT == BQ_FMT_ABQ ? INFINITY : 0.f, p1 = -INFINITY;
+  for (int c = lt; active && c < nch; c += TPT) {
+    const uint4 v = __ldg(xr + c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int h = 0; h < 4; h++) {
+      const float lo = __uint_as_float(w[h] << 16), hi = __uint_as_float(w[h] & 0xFFFF0000u);
+      if (FMT == BQ_FMT_ABQ) { p0 = fminf(p0, fminf(lo, hi)); p1 = fmaxf(p1, fmaxf(lo, hi)); }
+      else p0 = fmaxf(p0, fmaxf(fabsf(lo), fabsf(hi)));
+    }
+  }
+  float sc = 0.f, d = 1.f;
+  int z = 0;
+  const int qmax = (1 << a.a_bits) - 1;
+  if (FMT == BQ_FMT_ABQ) {
+    p0 = group_reduce(p0, TPT, sh_lo, [](float x, float y) { return fminf(x, y); });
+    p1 = group_reduce(p1, TPT, sh_hi, [](float x, float y) { return fmaxf(x, y); });
+    d = __fdiv_rn(fmaxf(__fsub_rn(p1, p0), 1e-5f), float(qmax));
+    z = int(rintf(__fdiv_rn(-p0, d)));
+  } else {
+    p0 = group_reduce(p0, TPT, sh_lo, [](float x, float y) { return fmaxf(x, y); });
+    sc = p0 > 0.f ? __fdiv_rn(127.f, p0) : 0.f;
+  }
+  uint32_t* cw = reinterpret_cast<uint32_t*>(smem + a.off_codes + size_t(active ? m : 0) * a.cstride);
+  int* gsum = reinterpret_cast<int*>(smem + a.off_gsum);
+  const int VPR = a.K_pad / 32;
+  uint32_t qsum = 0;
+  for (int c0 = 0; c0 < npad; c0 += TPT) {  // uniform trip count (the BVSR sums shuffle)
+    const int c = c0 + lt;
+    uint32_t word0 = 0, word1 = 0;
+    int qs = 0;
+    if (active && c < nch) {
+      const uint4 v = __ldg(xr + c);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t q8[8];
+#pragma unroll
+      for (int e = 0; e < 8; e++) {
+        const float xf = __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+        if (FMT == BQ_FMT_ABQ) {
+          const int q = quant_asym(xf, d, z, qmax);
+          qs += q;
+          q8[e] = uint32_t(q);
+        } else {
+          q8[e] = rn_biased(__fmul_rn(xf, sc));
+          qs += int(q8[e] - kRnBias);
+        }
+      }
+      word0 = __byte_perm(__byte_perm(q8[0], q8[1], 0x0040), __byte_perm(q8[2], q8[3], 0x0040), 0x5410);
+      word1 = __byte_perm(__byte_perm(q8[4], q8[5], 0x0040), __byte_perm(q8[6], q8[7], 0x0040), 0x5410);
+    }
+    if (active && c < npad) {
+      const int k = c * 8;
+      cw[(k >> 8) * 64 + code_word_in_tile(k & 255)] = word0;
+      cw[((k + 4) >> 8) * 64 + code_word_in_tile((k + 4) & 255)] = word1;
+    }
+    qsum += uint32_t(qs);
+    if (FMT == BQ_FMT_BVSR4) {  // 4 consecutive threads cover one 32-element vector
+      qs += __shfl_xor_sync(0xffffffffu, qs, 1);
+      qs += __shfl_xor_sync(0xffffffffu, qs, 2);
+      if (active && c < npad && (c & 3) == 0) gsum[m * VPR + (c >> 2)] = qs;
+    }
+  }
+  const int total = group_reduce(int(qsum), TPT, sh_sum, [](int x, int y) { return x + y; });
+  uint32_t* tok = reinterpret_cast<uint32_t*>(smem + a.off_tok);
+  if (active && lt == 0) {
+    if (FMT == BQ_FMT_ABQ) {
+      tok[4 * m + 0] = __float_as_uint(d); tok[4 * m + 1] = uint32_t(z); tok[4 * m + 2] = uint32_t(total);
+    } else {
+      tok[4 * m + 0] = __float_as_uint(p0); tok[4 * m + 1] = uint32_t(total);
+    }
+    tok[4 * m + 3] = token_scale<FMT>(tok[4 * m + 0]);
+  }
+}
+
 // Unfused: this CTA's tokens from the act buffer (after checking its header): the codes
 // by one bulk copy per token, token parameters and BVSR sums by plain loads.
 template <int FMT, int NW>
@@ -669,7 +760,8 @@ __device__ __forceinline__ void bvsr_tile(const uint4 (&w)[4], const uint4 (&b)[
 // ---------------------------------------------------------------------------
 // Two CTAs per SM (at most 128 registers a thread): the next launch's CTA must fit beside
 // this one to prefetch its weights.
-template <int FMT, int F0, int F1, int F2, int NW, bool FUSED>
+// T1: every CTA holds one token (tpc = 1); the kernel then carries only the one-token staging.
+template <int FMT, int F0, int F1, int F2, int NW, bool FUSED, bool T1>
 __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ LayerArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr bool BSIGNED = FMT != BQ_FMT_ABQ;
@@ -748,10 +840,16 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
   bool ok = true;
   const uint32_t* tokp = reinterpret_cast<const uint32_t*>(smem + a.off_tok);
   if constexpr (FUSED) {
-    if (mg == 1 && a.J <= 2) stage_quantize_1tok<FMT, NW, 2>(a, smem, m0);
-    else if (mg == 1 && a.J <= 4) stage_quantize_1tok<FMT, NW, 4>(a, smem, m0);
-    else if (mg == 1 && a.J <= 8) stage_quantize_1tok<FMT, NW, 8>(a, smem, m0);
-    else stage_quantize<FMT, NW>(a, smem, m0, mg);
+    if (a.J == 0) {
+      stage_quantize_reload<FMT, NW>(a, smem, m0, mg);  // rows too long for registers
+    } else if constexpr (T1) {
+      if (a.J <= 2) stage_quantize_1tok<FMT, NW, 2>(a, smem, m0);
+      else if (a.J <= 4) stage_quantize_1tok<FMT, NW, 4>(a, smem, m0);
+      else if (a.J <= 8) stage_quantize_1tok<FMT, NW, 8>(a, smem, m0);
+      else stage_quantize<FMT, NW>(a, smem, m0, mg);
+    } else {
+      stage_quantize<FMT, NW>(a, smem, m0, mg);
+    }
   } else {
     ok = stage_copy<FMT, NW>(a, smem, m0, mg, xbar);
   }

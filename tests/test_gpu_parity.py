@@ -245,3 +245,17 @@ def test_linear_group_equals_separate_calls(fmt, Ns, K, M, wa):
     r = oracle_layer(fmt, p, xh, a)
     assert np.array_equal(accs[0].cpu().numpy(), r["acc"])
     assert_y_close(ys[0].cpu().numpy(), r["y"], f"{fmt} group member 0")
+
+
+# ------------------------------------------------------------------ long rows (K up to the limit)
+@pytest.mark.parametrize("fmt,N,K,M,wa", [("bitnet", 32, 65536, 1, (1, 8)), ("bitnet", 20, 40960, 3, (1, 8)),
+                                           ("abq", 24, 33024, 2, (4, 4)), ("bvsr", 16, 33024, 1, (4, 8)),
+                                           ("ternary", 16, 36864, 2, (2, 8))])
+def test_long_rows(fmt, N, K, M, wa):
+    """K past what the fused staging holds in registers (32768 for one token): the fused call
+    re-reads x and must still equal the unfused path and the oracle."""
+    w, a = wa
+    gl = GpuLayer(fmt, N, K, M, seed=K % 97, w_bits=w, a_bits=a)
+    p = _pack_parity(gl, fmt, w)
+    check_act(gl)
+    _layer_parity(gl, p, fmt, a)
