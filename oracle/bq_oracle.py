@@ -138,6 +138,61 @@ def rabit_pack(W, h2) -> dict:
     return dict(B1=B1, B2=B2, g1=g1, g2=g2, h1=h1, h2=_f32(h2).copy())
 
 
+def _seq_sum(a, axis) -> np.ndarray:
+    """float64 sum in index order (left to right) along `axis`."""
+    a = np.asarray(a, dtype=np.float64)
+    if a.shape[axis] == 0:
+        return np.zeros(np.delete(a.shape, axis), dtype=np.float64)
+    return np.take(np.add.accumulate(a, axis=axis), -1, axis=axis)
+
+
+def rabit_pack_svid(W, rounds: int = 20) -> dict:
+    """[RaBiT] §2.3 "function-aware initialization", stage 1: iterative residual SVID,
+    Gauss-Seidel alternation over the two paths (default 20 iterations, §5). Stage 2 (channel
+    importance from calibration data) is out of scope.
+
+    Reading (the page gives no formulas): path p approximates its target T_p = W - W_other by
+    sign(T_p) * (g_p h_p^T), g_p per row, h_p per column (SVID: signs times a rank-1
+    magnitude). Each round updates path 1 then path 2; a path update sets B_p = sign(T_p),
+    then one alternating least-squares step of |T_p| ~ g_p h_p^T: g first, then h.
+      g_p[i] = sum_j |T_ij| h_p[j] / sum_j h_p[j]^2        (0 if the denominator is 0)
+      h_p[j] = sum_i |T_ij| g_p[i] / sum_i g_p[i]^2        (unchanged if the denominator is 0)
+    Start: g = 0, h = 1 for both paths. Arithmetic: float64 with sums in index order;
+    g and h are rounded to float32 after every update (their storage);
+    W_p[i,j] = (g_p[i] * h_p[j]) * B_p[i,j]; sign(0) = +1.
+    Every step minimizes ||W - W_1 - W_2||^2 over its own block, so the error is non-increasing.
+    The first g-step is exactly the mean-|W| scale of rabit_pack.
+    Pinned by tests (exact signed rank-1 input, monotone error, least-squares step)."""
+    W64 = _f32(W).astype(np.float64)
+    N, K = W64.shape
+    g = [np.zeros(N, np.float32), np.zeros(N, np.float32)]
+    h = [np.ones(K, np.float32), np.ones(K, np.float32)]
+    B = [sign_pm1(W64), np.ones((N, K), np.int8)]
+
+    def path_weight(q):
+        return (g[q].astype(np.float64)[:, None] * h[q].astype(np.float64)[None, :]) * B[q]
+
+    for _ in range(rounds):
+        for q in (0, 1):
+            T = W64 - path_weight(1 - q)
+            B[q] = sign_pm1(T)
+            A = np.abs(T)
+            hq = h[q].astype(np.float64)
+            hh = _seq_sum(hq * hq, 0)
+            g[q] = (_seq_sum(A * hq[None, :], 1) / hh).astype(np.float32) if hh > 0 else np.zeros(N, np.float32)
+            gq = g[q].astype(np.float64)
+            gg = _seq_sum(gq * gq, 0)
+            if gg > 0:
+                h[q] = (_seq_sum(A * gq[:, None], 0) / gg).astype(np.float32)
+    return dict(B1=B[0], B2=B[1], g1=g[0], g2=g[1], h1=h[0], h2=h[1])
+
+
+def rabit_recon_error(p, W) -> float:
+    """||W - W_hat||^2 in float64."""
+    d = _f32(W).astype(np.float64) - rabit_weight(p)
+    return float(np.sum(d * d))
+
+
 def rabit_weight(p) -> np.ndarray:
     """W_hat [N,K] float64 = g1*B1*h1 + g2*B2*h2 ([RaBiT] §2.1)."""
     g1, g2 = p["g1"].astype(np.float64), p["g2"].astype(np.float64)

@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 
 from oracle import bq_oracle as O
+import bq_inputs as I
 
 
 # --------------------------------------------------------------------- sign
@@ -363,3 +364,48 @@ def test_bvsr_table_construction_hand_built():
                 for i in range(4):
                     assert tab[s, i] == np.float32((hi - lo) * r ** i / tot)
     assert tab[0, 4] == np.float32(-0.016) and tab[64 + 7, 0] * 15 == pytest.approx(0.030 + 0.016, rel=1e-6)
+
+
+# ------------------------------------------------------------------ RaBiT iterative residual SVID
+def test_svid_exact_signed_rank1():
+    """W = s * (a b^T) with power-of-two a, b: one round recovers W up to float32 rounding of
+    g and h (the rank-1 fit is exact in real arithmetic), and path 2 carries only that rounding."""
+    rng = np.random.default_rng(5)
+    a = 2.0 ** rng.integers(-6, -2, 16)
+    b = 2.0 ** rng.integers(-2, 2, 64)
+    s = np.where(rng.random((16, 64)) < 0.5, -1.0, 1.0)
+    W = (s * np.outer(a, b)).astype(np.float32)
+    p = O.rabit_pack_svid(W, rounds=1)
+    assert np.array_equal(p["B1"], O.sign_pm1(W))
+    w2 = float(np.sum(W.astype(np.float64) ** 2))
+    assert O.rabit_recon_error(p, W) <= 1e-12 * w2
+    p1 = dict(p, g2=np.zeros_like(p["g2"]))               # path 1 alone
+    assert O.rabit_recon_error(p1, W) <= 1e-12 * w2
+    assert np.all(np.abs(p["g2"]) <= 1e-6 * np.abs(p["g1"]).max())
+
+
+def test_svid_first_step_is_mean_abs_and_error_never_grows():
+    W = I.weights(24, 256, seed=9)
+    base = O.rabit_pack(W, np.ones(256, np.float32))
+    p1 = O.rabit_pack_svid(W, rounds=1)
+    # the first g-step from h = 1 is the mean |W| of each row, as in rabit_pack
+    g_first = np.array([O.mean_abs_f32(W[n]) for n in range(24)], dtype=np.float32)
+    assert np.array_equal(base["g1"], g_first)
+    errs = [O.rabit_recon_error(O.rabit_pack_svid(W, rounds=r), W) for r in (1, 2, 5, 20)]
+    for e0, e1 in zip(errs, errs[1:]):
+        assert e1 <= e0 * (1 + 1e-6)
+    assert errs[-1] < O.rabit_recon_error(base, W)
+
+
+def test_svid_g_step_is_least_squares():
+    """For fixed h, g from the SVID step solves min_g ||A - g h^T||^2 row by row (checked with
+    numpy's least squares on the first round's target A = |W|)."""
+    W = I.weights(8, 128, seed=3)
+    A = np.abs(W.astype(np.float64))
+    h = np.linspace(0.5, 1.5, 128)
+    g_ls = np.array([np.linalg.lstsq(h[:, None], A[i], rcond=None)[0][0] for i in range(8)])
+    g_step = (A * h[None, :]).sum(1) / (h * h).sum()
+    assert np.allclose(g_ls, g_step, rtol=1e-12)
+    p = O.rabit_pack_svid(W, rounds=1)
+    g_formula = (A.sum(1) / 128).astype(np.float32)      # h = 1 in the first step
+    assert np.allclose(p["g1"], g_formula, rtol=1e-6)
