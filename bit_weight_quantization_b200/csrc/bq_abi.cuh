@@ -22,9 +22,11 @@ inline bq_status check_nk(int N, int K) {
 // need_ptrs: the pack call reads the device pointers; the size query does not.
 inline bq_status check_desc(const bq_pack_desc* d, int K, bool need_ptrs) {
   if (!d) return BQ_ERR_INVALID_ARG;
+  if (d->fmt != BQ_FMT_RABIT2 && d->rabit_svid_rounds != 0) return BQ_ERR_INVALID_ARG;
   switch (d->fmt) {
     case BQ_FMT_RABIT2:
-      if (need_ptrs && (!d->h2 || !aligned(d->h2, 4))) return BQ_ERR_INVALID_ARG;
+      if (d->rabit_svid_rounds < 0 || d->rabit_svid_rounds > 1000) return BQ_ERR_INVALID_ARG;
+      if (need_ptrs && d->rabit_svid_rounds == 0 && (!d->h2 || !aligned(d->h2, 4))) return BQ_ERR_INVALID_ARG;
       return BQ_OK;
     case BQ_FMT_BITNET_W1A8:
       return BQ_OK;
@@ -404,10 +406,27 @@ bq_status bq_pack_weights(const bq_pack_desc* desc, const float* W, int32_t N, i
       break;
     }
     case BQ_FMT_RABIT2: {
-      k_rabit_pack<<<N, 256, 0, s>>>(W, L.N_pad, K, L.K_pad, reinterpret_cast<uint32_t*>(P + L.off_tiles),
-                                     reinterpret_cast<float*>(P + L.off_rows));
-      k_rabit_h<<<blocks_for(L.K_pad, 256), 256, 0, s>>>(desc->h2, K, L.K_pad, reinterpret_cast<float*>(P + L.off_aux),
-                                                         reinterpret_cast<float*>(P + L.off_aux2));
+      uint32_t* planes = reinterpret_cast<uint32_t*>(P + L.off_tiles);
+      float* g = reinterpret_cast<float*>(P + L.off_rows);
+      float* h1 = reinterpret_cast<float*>(P + L.off_aux);
+      float* h2 = reinterpret_cast<float*>(P + L.off_aux2);
+      if (desc->rabit_svid_rounds == 0) {
+        k_rabit_pack<<<N, 256, 0, s>>>(W, L.N_pad, K, L.K_pad, planes, g);
+        k_rabit_h<<<blocks_for(L.K_pad, 256), 256, 0, s>>>(desc->h2, K, L.K_pad, h1, h2);
+        break;
+      }
+      const uint64_t W32 = L.K_pad / 32;
+      const uint64_t init = std::max<uint64_t>(2ull * L.N_pad * W32, std::max<uint64_t>(2ull * L.N_pad, L.K_pad));
+      k_svid_init<<<blocks_for(init, 256), 256, 0, s>>>(L.N_pad, K, L.K_pad, planes, g, h1, h2);
+      uint32_t* pl[2] = {planes, planes + size_t(L.N_pad) * W32};
+      float* gp[2] = {g, g + L.N_pad};
+      float* hp[2] = {h1, h2};
+      for (int r = 0; r < desc->rabit_svid_rounds; r++)
+        for (int q = 0; q < 2; q++) {
+          const int o = 1 - q;
+          k_svid_rows<<<blocks_for(N, 128), 128, 0, s>>>(W, N, K, L.K_pad, pl[o], gp[o], hp[o], pl[q], hp[q], gp[q]);
+          k_svid_cols<<<blocks_for(K, 128), 128, 0, s>>>(W, N, K, L.K_pad, pl[o], gp[o], hp[o], gp[q], hp[q]);
+        }
       break;
     }
     case BQ_FMT_BVSR4: {

@@ -200,6 +200,84 @@ __global__ void k_rabit_h(const float* __restrict__ h2, int K, int K_pad, float*
 }
 
 // ---------------------------------------------------------------------------
+// RaBiT iterative residual SVID (pack option). Path q's target is T = W - (g_o h_o) B_o
+// from the other path's float32 g, h and sign plane; B_q = sign(T); one alternating
+// least-squares step of |T| ~ g_q h_q^T: g_q[i] = sum_j |T_ij| h_q[j] / sum_j h_q[j]^2, then
+// h_q[j] = sum_i |T_ij| g_q[i] / sum_i g_q[i]^2. float64, every sum in index order (one
+// thread per row or column, the norms by one thread per block), results rounded to float32.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ double svid_target(float w, float go, float ho, uint32_t word_o, int j) {
+  const double wo = __dmul_rn(double(go), double(ho));
+  return __dsub_rn(double(w), ((word_o >> j) & 1u) ? -wo : wo);
+}
+
+// start: planes 0 (+1), g = 0, h = 1 on the real columns (0 on padding)
+__global__ void k_svid_init(int N_pad, int K, int K_pad, uint32_t* __restrict__ planes, float* __restrict__ g,
+                            float* __restrict__ h1, float* __restrict__ h2) {
+  const uint64_t i = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const uint64_t nw = 2ull * N_pad * (K_pad / 32);
+  if (i < nw) planes[i] = 0u;
+  if (i < uint64_t(2) * N_pad) g[i] = 0.f;
+  if (i < uint64_t(K_pad)) { h1[i] = i < uint64_t(K) ? 1.f : 0.f; h2[i] = i < uint64_t(K) ? 1.f : 0.f; }
+}
+
+// sum_{i < n} v[i]^2 in index order (float64), by thread 0, shared with the block
+__device__ __forceinline__ double svid_sq_norm(const float* __restrict__ v, int n, double* sh) {
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int i = 0; i < n; i++) s = __dadd_rn(s, __dmul_rn(double(v[i]), double(v[i])));
+    *sh = s;
+  }
+  __syncthreads();
+  return *sh;
+}
+
+// one thread per row: the sign plane of path q and g_q
+__global__ void k_svid_rows(const float* __restrict__ W, int N, int K, int K_pad, const uint32_t* __restrict__ plane_o,
+                            const float* __restrict__ g_o, const float* __restrict__ h_o, uint32_t* __restrict__ plane_q,
+                            const float* __restrict__ h_q, float* __restrict__ g_q) {
+  __shared__ double hh_s;
+  const double hh = svid_sq_norm(h_q, K, &hh_s);
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= N) return;
+  const int W32 = K_pad / 32;
+  const float* w = W + size_t(i) * K;
+  const float go = g_o[i];
+  double acc = 0.0;
+  for (int wd = 0; wd < W32; wd++) {
+    const uint32_t word_o = plane_o[size_t(i) * W32 + wd];
+    uint32_t bits = 0;
+    for (int j = 0; j < 32; j++) {
+      const int k = wd * 32 + j;
+      if (k >= K) break;
+      const double t = svid_target(w[k], go, h_o[k], word_o, j);
+      bits |= uint32_t(!(t >= 0.0)) << j;
+      acc = __dadd_rn(acc, __dmul_rn(fabs(t), double(h_q[k])));
+    }
+    plane_q[size_t(i) * W32 + wd] = bits;
+  }
+  g_q[i] = hh > 0.0 ? __double2float_rn(__ddiv_rn(acc, hh)) : 0.f;
+}
+
+// one thread per column: h_q (unchanged when g_q is all zero)
+__global__ void k_svid_cols(const float* __restrict__ W, int N, int K, int K_pad, const uint32_t* __restrict__ plane_o,
+                            const float* __restrict__ g_o, const float* __restrict__ h_o, const float* __restrict__ g_q,
+                            float* __restrict__ h_q) {
+  __shared__ double gg_s;
+  const double gg = svid_sq_norm(g_q, N, &gg_s);
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= K || !(gg > 0.0)) return;
+  const int W32 = K_pad / 32, wd = k / 32, j = k % 32;
+  const float ho = h_o[k];
+  double acc = 0.0;
+  for (int i = 0; i < N; i++) {
+    const double t = svid_target(W[size_t(i) * K + k], g_o[i], ho, plane_o[size_t(i) * W32 + wd], j);
+    acc = __dadd_rn(acc, __dmul_rn(fabs(t), double(g_q[i])));
+  }
+  h_q[k] = __double2float_rn(__ddiv_rn(acc, gg));
+}
+
+// ---------------------------------------------------------------------------
 // Ternary LoRA matrices to bf16: A [K][r] -> [K_pad][r], B [r][N] -> B^T [N_pad][r]
 // ---------------------------------------------------------------------------
 __global__ void k_lora_to_bf16(const float* __restrict__ A, const float* __restrict__ B, int N, int K,

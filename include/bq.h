@@ -125,9 +125,18 @@ typedef struct {
   int32_t a_bits;       /* ABQ activation bits, 1..8 (ignored: the A8 formats use 8) */
   int32_t lora_rank;    /* ternary: rank r of the correction, 0..64, a multiple of 8 (0 = none) */
   float lora_alpha;     /* ternary: gate alpha; the correction is scaled by tanh(alpha) */
-  const float* h2;      /* RaBiT: device f32 [K], second-path input scale (h1 = 1) */
+  const float* h2;      /* RaBiT, rabit_svid_rounds = 0: device f32 [K], second-path input
+                           scale (h1 = 1); unused otherwise (may be NULL) */
   const float* lora_A;  /* ternary: device f32 [K][r] row-major, rounded to bf16 */
   const float* lora_B;  /* ternary: device f32 [r][N] row-major, rounded to bf16 */
+  int32_t rabit_svid_rounds;  /* RaBiT initialisation: 0 = the residual recursion with mean|.|
+                           row scales (h1 = 1, h2 given); R in 1..1000 = R rounds of the
+                           iterative residual SVID ("RaBiT" page, §2.3, function-aware
+                           initialisation, stage 1; its default is 20): each round fits path 1
+                           to W - W2, then path 2 to W - W1, as sign(target) * (g h^T) by one
+                           alternating least-squares step (g per row, then h per column), in
+                           float64 with sums in index order, g and h kept in float32;
+                           start g = 0, h = 1. Must be 0 for the other formats. */
 } bq_pack_desc;
 
 /* Host-side description of a packed layer; filled by bq_pack_weights or

@@ -203,3 +203,16 @@ def test_linear_group_rejects_before_launch():
     yp = (ctypes.c_void_p * 5)(*([fake] * 5))
     assert bq.raw_status("bq_linear_group", arr, 5, fake, 1, yp, None, None) == bq.BQ_ERR_INVALID_ARG
     assert bq.raw_status("bq_linear_group", arr, 0, fake, 1, yp, None, None) == bq.BQ_ERR_INVALID_ARG
+
+
+def test_svid_descriptor_checks():
+    out = ctypes.c_size_t(0)
+    for fmt, rounds, st in [("rabit", -1, bq.BQ_ERR_INVALID_ARG), ("rabit", 1001, bq.BQ_ERR_INVALID_ARG),
+                            ("rabit", 20, bq.BQ_OK), ("bitnet", 5, bq.BQ_ERR_INVALID_ARG)]:
+        d = bq.make_desc(fmt, rabit_svid_rounds=rounds)
+        assert bq.raw_status("bq_packed_bytes", ctypes.byref(d), 64, 256, ctypes.byref(out)) == st
+    # the SVID pack fits h2 itself (no h2 pointer needed); the plain recursion needs one
+    d = bq.make_desc("rabit", rabit_svid_rounds=0)
+    fake = 1 << 40
+    assert bq.raw_status("bq_pack_weights", ctypes.byref(d), fake, 64, 256, fake, 1 << 30, None,
+                         ctypes.byref(bq.bq_layer())) == bq.BQ_ERR_INVALID_ARG

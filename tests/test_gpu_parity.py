@@ -259,3 +259,32 @@ def test_long_rows(fmt, N, K, M, wa):
     p = _pack_parity(gl, fmt, w)
     check_act(gl)
     _layer_parity(gl, p, fmt, a)
+
+
+# ------------------------------------------------------------------ RaBiT SVID initialisation
+@pytest.mark.parametrize("N,K,rounds", [(40, 384, 1), (40, 384, 20), (256, 512, 20), (17, 256, 3)])
+def test_rabit_svid_pack_and_layer(N, K, rounds):
+    """The pack's iterative residual SVID gives the oracle's signs, g and h bit for bit (same
+    float64 operations in the same order); the layer on them matches the oracle's layer."""
+    from tests.parity_util import L as layout, torch_mods
+    torch, bq = torch_mods()
+    W = I.weights(N, K, seed=N + rounds)
+    x = I.activations(2, K, seed=5)
+    ql = bq.QuantLinear("rabit", to_dev_f32(W), rabit_svid_rounds=rounds)
+    p = layout.read_packed(ql.packed.cpu().numpy().tobytes())
+    ref = O.rabit_pack_svid(W, rounds)
+    for key in ("B1", "B2"):
+        assert np.array_equal(p[key], ref[key]), key
+    for key in ("g1", "g2", "h1", "h2"):
+        assert np.array_equal(p[key], ref[key]), key
+    xd = to_dev_bf16(x)
+    y = torch.full((2, N), float("nan"), device="cuda")
+    ql.linear(xd, y)
+    y2 = torch.full((2, N), float("nan"), device="cuda")
+    ql.forward(xd, y2)
+    torch.cuda.synchronize()
+    bq.bq_device_check()
+    r = O.rabit_layer(ref, x)
+    assert_y_close(y.cpu().numpy(), r["y"], "rabit svid fused")
+    assert_y_close(y2.cpu().numpy(), r["y"], "rabit svid act+gemv")
+    assert O.rabit_recon_error(ref, W) <= O.rabit_recon_error(O.rabit_pack(W, np.ones(K, np.float32)), W)
