@@ -288,3 +288,32 @@ def test_rabit_svid_pack_and_layer(N, K, rounds):
     assert_y_close(y.cpu().numpy(), r["y"], "rabit svid fused")
     assert_y_close(y2.cpu().numpy(), r["y"], "rabit svid act+gemv")
     assert O.rabit_recon_error(ref, W) <= O.rabit_recon_error(O.rabit_pack(W, np.ones(K, np.float32)), W)
+
+
+# ------------------------------------------------------------------ maximum N
+def test_max_rows_abq():
+    """N = 2^20 rows (the limit), K = 128, M = 2: ABQ's per-row codes let sampled rows be
+    checked against the oracle. W is drawn on the device; only the sampled rows come back."""
+    from tests.parity_util import L as layout, torch_mods
+    torch, bq = torch_mods()
+    N, K, M = 1 << 20, 128, 2
+    g = torch.Generator(device="cuda")
+    g.manual_seed(3)
+    W = torch.randn(N, K, device="cuda", generator=g) * 0.02
+    ql = bq.QuantLinear("abq", W, w_bits=2, a_bits=8)
+    x = I.activations(M, K, seed=4)
+    y = torch.full((M, N), float("nan"), device="cuda")
+    acc = torch.full((M, N), -(1 << 62), dtype=torch.int64, device="cuda")
+    ql.linear(to_dev_bf16(x), y, acc)
+    torch.cuda.synchronize()
+    bq.bq_device_check()
+    rbs = np.array([0, 1, 777, 40000, (N // 16) - 1])
+    p = layout.read_packed(ql.packed.cpu().numpy().tobytes(), rbs)
+    rows = p["rows"]
+    Wh = W[torch.as_tensor(rows, device="cuda")].cpu().numpy()
+    ref = O.abq_pack(Wh, 2)
+    assert np.array_equal(p["Q"], ref["Q"]) and np.array_equal(p["delta"], ref["delta"])
+    r = O.abq_layer(p, x, 8)
+    assert np.array_equal(acc.cpu().numpy()[:, rows], r["I"])
+    assert_y_close(y.cpu().numpy()[:, rows], r["y"], "abq N = 2^20")
+    assert bool(torch.isfinite(y).all())
