@@ -199,7 +199,7 @@ class QuantLinear:
         self.packed = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
         self.layer = bq_pack_weights(self.desc, W, N, K, self.packed, nbytes, stream)
         # the pack reads W, h2 and the LoRA matrices asynchronously: wait before the caller may free them
-        (torch.cuda.current_stream() if stream is None else stream).synchronize()
+        torch.cuda.synchronize(W.device)
         self.N, self.K = N, K
         self._acts = {}
 

@@ -287,6 +287,22 @@ def ternary_layer(p, x) -> dict:
 # ---------------------------------------------------------------------------
 
 
+def abq_pack_balanced(W) -> dict:
+    """[ABQ] §3.3 bit-balance strategy (W2*): INT2's four levels are asymmetric, so the
+    code space is widened to the symmetric {-2, -1, 0, 1, 2}. Reading: per row,
+    hi = max|W|, lo = -hi, Delta = max(hi - lo, 1e-5) / 4 (float32 ops, as quantize_rows_asym
+    with 4 intervals), z = 2, q = clamp(rn(W / Delta) + 2, 0, 4): a 3-bit code, so the packed
+    buffer is an ABQ w = 3 buffer whose codes take 5 values.
+    Pinned by tests (exact antisymmetry q(-W) = 4 - q(W), grid round trip, levels)."""
+    W = _f32(W)
+    hi = np.abs(W).max(axis=1).astype(np.float32)
+    rng_ = np.maximum((hi - (-hi)).astype(np.float32), np.float32(1e-5)).astype(np.float32)
+    delta = (rng_ / np.float32(4)).astype(np.float32)
+    q = np.rint((W / delta[:, None]).astype(np.float32)).astype(np.int64) + 2
+    q = np.clip(q, 0, 4)
+    return dict(Q=q.astype(np.int32), delta=delta, z=np.full(W.shape[0], 2, np.int32), w_bits=3)
+
+
 def abq_pack(W, w_bits: int) -> dict:
     """Per-output-row asymmetric weight codes (quantize_rows_asym)."""
     Q, delta, z = quantize_rows_asym(W, w_bits)

@@ -409,3 +409,27 @@ def test_svid_g_step_is_least_squares():
     p = O.rabit_pack_svid(W, rounds=1)
     g_formula = (A.sum(1) / 128).astype(np.float32)      # h = 1 in the first step
     assert np.allclose(p["g1"], g_formula, rtol=1e-6)
+
+
+# ------------------------------------------------------------------ ABQ bit balance (W2*)
+def test_bit_balance_symmetric_levels():
+    W = I.weights(12, 256, seed=21)
+    p = O.abq_pack_balanced(W)
+    pn = O.abq_pack_balanced(-W)
+    assert set(np.unique(p["Q"])) <= {0, 1, 2, 3, 4} and np.all(p["z"] == 2)
+    assert np.array_equal(pn["delta"], p["delta"])
+    assert np.array_equal(pn["Q"], 4 - p["Q"])            # rn is odd, the grid is symmetric
+    # the row extremes map to the outermost levels
+    assert np.all(p["Q"][np.arange(12), np.abs(W).argmax(1)] % 4 == 0)
+
+
+def test_bit_balance_grid_round_trip():
+    d = np.float32(0.0625)
+    levels = np.array([-2, -1, 0, 1, 2], np.float32) * d
+    rng = np.random.default_rng(2)
+    W = rng.choice(levels, size=(6, 128)).astype(np.float32)
+    W[:, 0], W[:, 1] = 2 * d, -2 * d                      # each row spans the full range
+    p = O.abq_pack_balanced(W)
+    assert np.all(p["delta"] == d)
+    deq = (p["Q"] - p["z"][:, None]).astype(np.float64) * p["delta"][:, None]
+    assert np.array_equal(deq, W.astype(np.float64))
