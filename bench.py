@@ -86,11 +86,17 @@ def measured_peaks() -> tuple[float, str]:
 
 
 def kernel_source_hash() -> str:
+    """Hash of what sets the layer kernel's DRAM traffic: its code (bq_gemv.cuh,
+    bq_internal.cuh) and its launch plan (plan_layer in bq_abi.cuh)."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "bit_weight_quantization_b200", "csrc")
-    for fn in sorted(os.listdir(d)):
+    for fn in ("bq_gemv.cuh", "bq_internal.cuh"):
         with open(os.path.join(d, fn), "rb") as f:
             h.update(f.read())
+    with open(os.path.join(d, "bq_abi.cuh")) as f:
+        src = f.read()
+    i0 = src.index("inline bool plan_layer(")
+    h.update(src[i0:src.index("\n}\n", i0)].encode())
     return h.hexdigest()[:16]
 
 

@@ -26,7 +26,8 @@ FORMATS = {"rabit": 1, "bitnet": 2, "ternary": 3, "abq": 4, "bvsr": 5}
 class bq_pack_desc(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("w_bits", ctypes.c_int32), ("a_bits", ctypes.c_int32),
                 ("lora_rank", ctypes.c_int32), ("lora_alpha", ctypes.c_float), ("h2", ctypes.c_void_p),
-                ("lora_A", ctypes.c_void_p), ("lora_B", ctypes.c_void_p), ("rabit_svid_rounds", ctypes.c_int32)]
+                ("lora_A", ctypes.c_void_p), ("lora_B", ctypes.c_void_p), ("rabit_svid_rounds", ctypes.c_int32),
+                ("abq_bit_balance", ctypes.c_int32)]
 
 
 class bq_layer(ctypes.Structure):
@@ -99,9 +100,9 @@ def bq_version() -> int:
 
 
 def make_desc(fmt, w_bits=0, a_bits=0, lora_rank=0, lora_alpha=0.1, h2=None, lora_A=None, lora_B=None,
-              rabit_svid_rounds=0):
+              rabit_svid_rounds=0, abq_bit_balance=0):
     return bq_pack_desc(FORMATS.get(fmt, fmt), w_bits, a_bits, lora_rank, lora_alpha,
-                        _ptr(h2), _ptr(lora_A), _ptr(lora_B), rabit_svid_rounds)
+                        _ptr(h2), _ptr(lora_A), _ptr(lora_B), rabit_svid_rounds, abq_bit_balance)
 
 
 def bq_packed_bytes(desc: bq_pack_desc, N: int, K: int) -> int:
@@ -191,10 +192,11 @@ class QuantLinear:
     All arithmetic happens in the library."""
 
     def __init__(self, fmt, W, *, w_bits=0, a_bits=0, lora_rank=0, lora_alpha=0.1, h2=None,
-                 lora_A=None, lora_B=None, rabit_svid_rounds=0, stream=None):
+                 lora_A=None, lora_B=None, rabit_svid_rounds=0, abq_bit_balance=0, stream=None):
         import torch
         N, K = W.shape
-        self.desc = make_desc(fmt, w_bits, a_bits, lora_rank, lora_alpha, h2, lora_A, lora_B, rabit_svid_rounds)
+        self.desc = make_desc(fmt, w_bits, a_bits, lora_rank, lora_alpha, h2, lora_A, lora_B, rabit_svid_rounds,
+                              abq_bit_balance)
         nbytes = bq_packed_bytes(self.desc, N, K)
         self.packed = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
         self.layer = bq_pack_weights(self.desc, W, N, K, self.packed, nbytes, stream)

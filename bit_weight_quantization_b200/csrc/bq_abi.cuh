@@ -23,6 +23,8 @@ inline bq_status check_nk(int N, int K) {
 inline bq_status check_desc(const bq_pack_desc* d, int K, bool need_ptrs) {
   if (!d) return BQ_ERR_INVALID_ARG;
   if (d->fmt != BQ_FMT_RABIT2 && d->rabit_svid_rounds != 0) return BQ_ERR_INVALID_ARG;
+  if (d->abq_bit_balance != 0 && (d->fmt != BQ_FMT_ABQ || d->abq_bit_balance != 1 || d->w_bits != 3))
+    return BQ_ERR_INVALID_ARG;
   switch (d->fmt) {
     case BQ_FMT_RABIT2:
       if (d->rabit_svid_rounds < 0 || d->rabit_svid_rounds > 1000) return BQ_ERR_INVALID_ARG;
@@ -400,7 +402,7 @@ bq_status bq_pack_weights(const bq_pack_desc* desc, const float* W, int32_t N, i
       float* delta = reinterpret_cast<float*>(P + L.off_rows);
       int* zero = reinterpret_cast<int*>(P + L.off_rows) + L.N_pad;
       int* sumq = reinterpret_cast<int*>(P + L.off_rows) + 2 * L.N_pad;
-      k_abq_rows<<<N, 256, 0, s>>>(W, K, L.w_bits, delta, zero, sumq);
+      k_abq_rows<<<N, 256, 0, s>>>(W, K, L.w_bits, desc->abq_bit_balance, delta, zero, sumq);
       fa.abq_delta = delta; fa.abq_zero = zero;
       k_pack_fields<BQ_FMT_ABQ><<<blocks_for(fa.total_words, 256), 256, 0, s>>>(fa);
       break;

@@ -61,7 +61,9 @@ __device__ __forceinline__ int abq_code(float w, float delta, int z, int qmax) {
   return int(q);
 }
 
-__global__ void k_abq_rows(const float* __restrict__ W, int K, int w_bits, float* __restrict__ delta,
+// balanced (W2*, w_bits = 3): symmetric range [-max|W|, max|W|] in 4 steps, z = 2; the
+// codes rn(W/Delta) + 2 then lie in 0..4 (|W/Delta| <= 2), under the same clamp.
+__global__ void k_abq_rows(const float* __restrict__ W, int K, int w_bits, int balanced, float* __restrict__ delta,
                            int* __restrict__ zero, int* __restrict__ sumq) {
   __shared__ float shf[32];
   __shared__ int shi[32];
@@ -75,9 +77,16 @@ __global__ void k_abq_rows(const float* __restrict__ W, int K, int w_bits, float
   lo = block_min(lo, shf);
   hi = block_max(hi, shf);
   const int qmax = (1 << w_bits) - 1;
-  float rng = fmaxf(__fsub_rn(hi, lo), 1e-5f);
-  float d = __fdiv_rn(rng, float(qmax));
-  int z = int(rintf(__fdiv_rn(-lo, d)));
+  float d;
+  int z;
+  if (balanced) {
+    const float hm = fmaxf(fabsf(lo), fabsf(hi));
+    d = __fdiv_rn(fmaxf(__fsub_rn(hm, -hm), 1e-5f), 4.f);
+    z = 2;
+  } else {
+    d = __fdiv_rn(fmaxf(__fsub_rn(hi, lo), 1e-5f), float(qmax));
+    z = int(rintf(__fdiv_rn(-lo, d)));
+  }
   int s = 0;
   for (int k = threadIdx.x; k < K; k += blockDim.x) s += abq_code(w[k], d, z, qmax);
   s = block_sum(s, shi);

@@ -137,6 +137,11 @@ typedef struct {
                            alternating least-squares step (g per row, then h per column), in
                            float64 with sums in index order, g and h kept in float32;
                            start g = 0, h = 1. Must be 0 for the other formats. */
+  int32_t abq_bit_balance;  /* ABQ, 1 = W2* ("ABQ-LLM" page, §3.3 bit-balance strategy): the
+                           symmetric five levels {-2..2} per row, Delta = max|W_row| / 2
+                           (max(2 max|W|, 1e-5) / 4), z = 2, code = clamp(rn(W/Delta) + 2, 0, 4)
+                           in a 3-bit field; requires w_bits = 3. The layer is the ABQ w = 3
+                           layer. 0 = the asymmetric min/max codes. Must be 0 for the others. */
 } bq_pack_desc;
 
 /* Host-side description of a packed layer; filled by bq_pack_weights or

@@ -216,3 +216,11 @@ def test_svid_descriptor_checks():
     fake = 1 << 40
     assert bq.raw_status("bq_pack_weights", ctypes.byref(d), fake, 64, 256, fake, 1 << 30, None,
                          ctypes.byref(bq.bq_layer())) == bq.BQ_ERR_INVALID_ARG
+
+
+def test_bit_balance_descriptor_checks():
+    out = ctypes.c_size_t(0)
+    for fmt, w, bal, st in [("abq", 3, 1, bq.BQ_OK), ("abq", 2, 1, bq.BQ_ERR_INVALID_ARG),
+                            ("abq", 3, 2, bq.BQ_ERR_INVALID_ARG), ("bitnet", 0, 1, bq.BQ_ERR_INVALID_ARG)]:
+        d = bq.make_desc(fmt, w_bits=w, a_bits=8, abq_bit_balance=bal)
+        assert bq.raw_status("bq_packed_bytes", ctypes.byref(d), 64, 256, ctypes.byref(out)) == st

@@ -317,3 +317,29 @@ def test_max_rows_abq():
     assert np.array_equal(acc.cpu().numpy()[:, rows], r["I"])
     assert_y_close(y.cpu().numpy()[:, rows], r["y"], "abq N = 2^20")
     assert bool(torch.isfinite(y).all())
+
+
+# ------------------------------------------------------------------ ABQ bit balance (W2*)
+@pytest.mark.parametrize("N,K,M", [(50, 384, 1), (97, 640, 9), (4096, 4096, 1)])
+def test_abq_bit_balance(N, K, M):
+    """W2*: the pack's symmetric five-level codes, Delta and z equal the oracle's; the layer (the
+    ABQ w = 3 kernels) matches the oracle's integer accumulator exactly and y within tolerance."""
+    from tests.parity_util import L as layout, torch_mods
+    torch, bq = torch_mods()
+    inp = I.layer_inputs("abq", N, K, M, seed=N + K)
+    W, x = inp["W"], inp["x"]
+    ql = bq.QuantLinear("abq", to_dev_f32(W), w_bits=3, a_bits=8, abq_bit_balance=1)
+    p = layout.read_packed(ql.packed.cpu().numpy().tobytes())
+    ref = O.abq_pack_balanced(W)
+    assert np.array_equal(p["Q"], ref["Q"]) and np.array_equal(p["delta"], ref["delta"])
+    assert np.array_equal(p["z"], ref["z"]) and np.array_equal(p["S_w"], ref["Q"].sum(1))
+    xd = to_dev_bf16(x)
+    for run in (ql.linear, ql.forward):
+        y = torch.full((M, N), float("nan"), device="cuda")
+        acc = torch.full((M, N), -(1 << 62), dtype=torch.int64, device="cuda")
+        run(xd, y, acc)
+        torch.cuda.synchronize()
+        r = O.abq_layer(p, x, 8)
+        assert np.array_equal(acc.cpu().numpy(), r["I"])
+        assert_y_close(y.cpu().numpy(), r["y"], "abq W2*")
+    bq.bq_device_check()
