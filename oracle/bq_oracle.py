@@ -34,7 +34,8 @@ def bf16_round(a) -> np.ndarray:
     """Round to the nearest bfloat16 (ties to even), returned as float32.
 
     Used where a format stores a tensor in bf16 (the LoRA matrices of [HGF]
-    §2.1 are an fp16/bf16 correction path)."""
+    §2.1 are an fp16/bf16 correction path).
+    Pinned by tests (hand values: exact, tie to even down and up, above half)."""
     f = np.ascontiguousarray(_f32(a))
     u = f.view(np.uint32).astype(np.uint64)
     r = ((u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000).astype(np.uint32)
@@ -49,7 +50,8 @@ def sign_pm1(v) -> np.ndarray:
 
 
 def mean_abs_f32(a) -> np.float32:
-    """mean(|a|) summed in float64, stored as float32."""
+    """mean(|a|) summed in float64, stored as float32.
+    Pinned by tests (BitNet alpha hand check; the SVID first g-step equals it)."""
     a64 = np.abs(np.asarray(a, dtype=np.float64))
     if a64.size == 0:
         return np.float32(0.0)
@@ -84,7 +86,8 @@ def quantize_act_int8(x) -> tuple[np.ndarray, np.ndarray]:
 
 
 def dequant_act_int8(q, gamma) -> np.ndarray:
-    """x_hat = q * gamma / 127 in float64 ([HGF] §1.2 dequantization)."""
+    """x_hat = q * gamma / 127 in float64 ([HGF] §1.2 dequantization).
+    Pinned by tests (act endpoints and range: q gamma / 127 recovers the row extremes)."""
     return q.astype(np.float64) * (gamma.astype(np.float64)[:, None] / 127.0)
 
 
@@ -188,13 +191,15 @@ def rabit_pack_svid(W, rounds: int = 20) -> dict:
 
 
 def rabit_recon_error(p, W) -> float:
-    """||W - W_hat||^2 in float64."""
+    """||W - W_hat||^2 in float64.
+    Pinned by tests (zero error on the exact signed rank-1 input to rounding)."""
     d = _f32(W).astype(np.float64) - rabit_weight(p)
     return float(np.sum(d * d))
 
 
 def rabit_weight(p) -> np.ndarray:
-    """W_hat [N,K] float64 = g1*B1*h1 + g2*B2*h2 ([RaBiT] §2.1)."""
+    """W_hat [N,K] float64 = g1*B1*h1 + g2*B2*h2 ([RaBiT] §2.1).
+    Pinned by tests (RaBiT hand recursion, constant-magnitude rows reconstruct exactly)."""
     g1, g2 = p["g1"].astype(np.float64), p["g2"].astype(np.float64)
     h1, h2 = p["h1"].astype(np.float64), p["h2"].astype(np.float64)
     return g1[:, None] * p["B1"] * h1[None, :] + g2[:, None] * p["B2"] * h2[None, :]
@@ -203,7 +208,8 @@ def rabit_weight(p) -> np.ndarray:
 def rabit_layer(p, x) -> dict:
     """y = W_hat x in float64 with x the unquantized bf16 activations (the
     RaBiT kernel of [RaBiT] §3.2 applies signs to the input, no activation
-    quantization). Also returns the per-path sums acc_p = sum_k B_p h_p x."""
+    quantization). Also returns the per-path sums acc_p = sum_k B_p h_p x.
+    Pinned by tests (the layer equals the sum of the two sign paths, dense vs per path)."""
     x64 = _f32(x).astype(np.float64)
     y = x64 @ rabit_weight(p).T
     acc1 = x64 @ (p["B1"] * p["h1"].astype(np.float64)[None, :]).T
@@ -218,7 +224,8 @@ def rabit_layer(p, x) -> dict:
 
 def bitnet_pack(W) -> dict:
     """W ~= alpha * sign(W) with one alpha per matrix ([BitNet] §2.2); the page
-    learns alpha, here alpha = mean|W| over the whole tensor."""
+    learns alpha, here alpha = mean|W| over the whole tensor.
+    Pinned by tests (alpha = mean|W| hand check, sign(0) = +1)."""
     W = _f32(W)
     return dict(B=sign_pm1(W), alpha=mean_abs_f32(W))
 
@@ -226,7 +233,8 @@ def bitnet_pack(W) -> dict:
 def bitnet_layer(p, x) -> dict:
     """acc = sum_k B[n,k] q[m,k] (int64); y = sum_k (alpha B)(q gamma/127) in
     float64 ([BitNet] §2.3 binary product scaled by alpha; activation scale of
-    [HGF] §1.2)."""
+    [HGF] §1.2).
+    Pinned by tests (integer and dequantized-float routes agree; the W1A8 plane identity over all int8 codes)."""
     q, gamma = quantize_act_int8(x)
     acc = q.astype(np.int64) @ p["B"].astype(np.int64).T
     w_hat = np.float64(p["alpha"]) * p["B"].astype(np.float64)
@@ -260,11 +268,14 @@ def ternary_pack(W, lora_A=None, lora_B=None, lora_alpha: float = 0.1) -> dict:
 
 
 def silu(z):
+    """SiLU(z) = z / (1 + exp(-z)) ([HGF] §2.1 gate nonlinearity).
+    Pinned through lora_correction's closed form (rank 1)."""
     return z / (1.0 + np.exp(-z))
 
 
 def lora_correction(x, A, B, alpha) -> np.ndarray:
-    """tanh(alpha) * (SiLU(x @ A) @ B) in float64 ([HGF] §2.1), x unquantized."""
+    """tanh(alpha) * (SiLU(x @ A) @ B) in float64 ([HGF] §2.1), x unquantized.
+    Pinned by tests (closed form with rank 1)."""
     x64 = _f32(x).astype(np.float64)
     u = silu(x64 @ A.astype(np.float64))
     return math.tanh(float(np.float32(alpha))) * (u @ B.astype(np.float64))
@@ -273,7 +284,8 @@ def lora_correction(x, A, B, alpha) -> np.ndarray:
 def ternary_layer(p, x) -> dict:
     """acc = sum_k T q (int64); y = gamma_w*gamma_x/127 * acc + LoRA term,
     the ternary part computed as a float64 product of dequantized operands
-    ([HGF] §1.2 int8 product with Y_int * gamma_x gamma_W / 127)."""
+    ([HGF] §1.2 int8 product with Y_int * gamma_x gamma_W / 127).
+    Pinned by tests (integer route equals the dequantized route)."""
     q, gamma = quantize_act_int8(x)
     acc = q.astype(np.int64) @ p["T"].astype(np.int64).T
     w_hat = np.float64(p["gamma_w"]) * p["T"].astype(np.float64)
@@ -304,7 +316,8 @@ def abq_pack_balanced(W) -> dict:
 
 
 def abq_pack(W, w_bits: int) -> dict:
-    """Per-output-row asymmetric weight codes (quantize_rows_asym)."""
+    """Per-output-row asymmetric weight codes (quantize_rows_asym).
+    Pinned by tests (hand examples with a rounding tie, grid round trip)."""
     Q, delta, z = quantize_rows_asym(W, w_bits)
     return dict(Q=Q, delta=delta, z=z, w_bits=w_bits)
 
@@ -312,7 +325,8 @@ def abq_pack(W, w_bits: int) -> dict:
 def abq_layer(p, x, a_bits: int) -> dict:
     """Per-token asymmetric activation codes, then
     I = sum_k (qw - zw)(qx - zx) (int64) and y = Dw*Dx*I as the float64 product
-    of the dequantized operands."""
+    of the dequantized operands.
+    Pinned by tests (zero-point expansion equals the centred product; |I| bounds)."""
     Qx, dx, zx = quantize_rows_asym(x, a_bits)
     cw = p["Q"].astype(np.int64) - p["z"].astype(np.int64)[:, None]
     cx = Qx.astype(np.int64) - zx.astype(np.int64)[:, None]
@@ -329,6 +343,8 @@ def abq_layer(p, x, a_bits: int) -> dict:
 
 
 def popcount(v) -> np.ndarray:
+    """Number of set bits of each unsigned 64-bit word, counted bit by bit.
+    Pinned through the XNOR and bit-plane identities (brute force over all pairs)."""
     v = np.asarray(v, dtype=np.uint64)
     c = np.zeros(v.shape, dtype=np.int64)
     for b in range(64):
@@ -337,13 +353,15 @@ def popcount(v) -> np.ndarray:
 
 
 def planes_of(codes, bits: int) -> list:
-    """Bit-plane b of non-negative or two's-complement codes: a 0/1 array."""
+    """Bit-plane b of non-negative or two's-complement codes: a 0/1 array.
+    Pinned by tests (the W1A8 plane identity over all int8 codes)."""
     c = np.asarray(codes, dtype=np.int64) & ((1 << bits) - 1)
     return [((c >> b) & 1).astype(np.uint8) for b in range(bits)]
 
 
 def plane_weights(bits: int, signed: bool) -> list:
-    """omega_b = 2^b; for two's complement the top plane weighs -2^(bits-1)."""
+    """omega_b = 2^b; for two's complement the top plane weighs -2^(bits-1).
+    Pinned by tests (the W1A8 plane identity: plane 7 weighs -128)."""
     w = [1 << b for b in range(bits)]
     if signed:
         w[-1] = -w[-1]
@@ -351,7 +369,8 @@ def plane_weights(bits: int, signed: bool) -> list:
 
 
 def pack_bits(bitvec) -> int:
-    """A 0/1 vector as one integer word, element j at bit j (LSB first)."""
+    """A 0/1 vector as one integer word, element j at bit j (LSB first).
+    Pinned through the XNOR and bit-plane identities (brute force over all pairs)."""
     out = 0
     for j, b in enumerate(np.asarray(bitvec).tolist()):
         out |= int(b) << j
@@ -361,7 +380,8 @@ def pack_bits(bitvec) -> int:
 def bitplane_dot(wc, w_bits, w_signed, xc, x_bits, x_signed) -> int:
     """sum_b sum_c omega_b omega_c popc(W_b AND X_c) over one vector pair, the
     arbitrary-bit product of [ABQ] (abstract: binary tensor-core equivalent
-    operations), computed literally with popcounts of packed words."""
+    operations), computed literally with popcounts of packed words.
+    Pinned by tests (brute force: equals the integer dot product for every bit pair)."""
     wp, xp = planes_of(wc, w_bits), planes_of(xc, x_bits)
     ww, xw = plane_weights(w_bits, w_signed), plane_weights(x_bits, x_signed)
     tot = 0
@@ -376,7 +396,8 @@ def bitplane_dot(wc, w_bits, w_signed, xc, x_bits, x_signed) -> int:
 def xnor_popcount_dot(a_pm1, b_pm1) -> int:
     """[BitNet] §2.3: popcount(xnor(a, b)) for +-1 vectors coded as bit 1 <=> +1.
     Returns 2*popc(xnor) - K, the +-1 inner product (the page's formula without
-    the affine correction is the count of agreeing positions)."""
+    the affine correction is the count of agreeing positions).
+    Pinned by tests (brute force over all +-1 pairs: 2 popc(xnor) - K)."""
     a = pack_bits(np.asarray(a_pm1) > 0)
     b = pack_bits(np.asarray(b_pm1) > 0)
     K = len(a_pm1)
@@ -396,7 +417,8 @@ BVSR_PLANES = 4
 
 def nearest_rank(sorted_vals: np.ndarray, num: int, den: int):
     """Nearest-rank quantile num/den of an ascending array: element
-    ceil(num*V/den) - 1 (integer arithmetic)."""
+    ceil(num*V/den) - 1 (integer arithmetic).
+    Pinned by tests (hand quantiles)."""
     V = len(sorted_vals)
     rank = (num * V + den - 1) // den
     return sorted_vals[max(rank - 1, 0)]
@@ -439,7 +461,8 @@ def bvsr_set_table(W) -> np.ndarray:
 
 def bvsr_points(table) -> np.ndarray:
     """P[s, code] = o + c0 b0 + c1 b1 + c2 b2 + c3 b3 (b_i = bit i of code),
-    summed left to right in float64 from the float32 coefficients."""
+    summed left to right in float64 from the float32 coefficients.
+    Pinned by tests (ratio-2 sets are the uniform RTN grid)."""
     t = np.asarray(table, dtype=np.float32).astype(np.float64)
     S = t.shape[0]
     P = np.zeros((S, 16), dtype=np.float64)
@@ -458,7 +481,8 @@ def bvsr_encode_vectors(vecs, table) -> tuple[np.ndarray, np.ndarray]:
     lowest code on a tie), the set's error is sum_e (w_e - p)^2 accumulated in
     element order in float64, and the vector takes the set with the smallest
     error (lowest set index on a tie).
-    vecs float32 [V, 32] -> (codes uint8 [V, 32], set index uint8 [V])."""
+    vecs float32 [V, 32] -> (codes uint8 [V, 32], set index uint8 [V]).
+    Pinned by tests (matches RTN for the uniform set; exhaustive optimum on tiny inputs)."""
     vecs = _f32(vecs)
     V = vecs.shape[0]
     P = bvsr_points(table)                      # [S,16]
@@ -483,7 +507,8 @@ def bvsr_encode_vectors(vecs, table) -> tuple[np.ndarray, np.ndarray]:
 def bvsr_pack(W, table=None, rows=None) -> dict:
     """BVSR 4-bit pack of W [N,K] (K % 32 == 0). ``rows`` restricts the
     encoding to a subset of rows (the table still comes from the whole W).
-    Returns codes uint8 [R,K], set index uint8 [R,K/32], table [256,5]."""
+    Returns codes uint8 [R,K], set index uint8 [R,K/32], table [256,5].
+    Pinned by tests (layer routes agree); the set construction itself is a reading: parity unpinned."""
     W = _f32(W)
     N, K = W.shape
     if table is None:
@@ -496,7 +521,8 @@ def bvsr_pack(W, table=None, rows=None) -> dict:
 
 
 def bvsr_weight(codes, sets, table) -> np.ndarray:
-    """W_hat[n,k] = P[set(n, k/32), code(n,k)] in float64."""
+    """W_hat[n,k] = P[set(n, k/32), code(n,k)] in float64.
+    Pinned by tests (the dequantized route of bvsr_layer equals its integer route)."""
     P = bvsr_points(table)
     R, K = codes.shape
     s_full = np.repeat(sets.astype(np.int64), BVSR_VEC, axis=1)
@@ -506,7 +532,8 @@ def bvsr_weight(codes, sets, table) -> np.ndarray:
 def bvsr_layer(codes, sets, table, x) -> dict:
     """acc = sum_k code q (int64, code = sum_i 2^i b_i); y = sum_k W_hat x_hat in
     float64, x_hat the per-token absmax int8 activations ([BVSR] Introduction:
-    activations quantized online, product without weight dequantization)."""
+    activations quantized online, product without weight dequantization).
+    Pinned by tests (integer and dequantized routes agree; exact integer table case)."""
     q, gamma = quantize_act_int8(x)
     acc = q.astype(np.int64) @ codes.astype(np.int64).T
     y = dequant_act_int8(q, gamma) @ bvsr_weight(codes, sets, table).T
@@ -519,19 +546,22 @@ def bvsr_layer(codes, sets, table, x) -> dict:
 
 
 def decode_tokens_per_s(bandwidth_bytes_s: float, params: float, bits: float) -> float:
-    """Memory-wall bound T_max <= B_mem / (P * b / 8) ([HGF] §1.1)."""
+    """Memory-wall bound T_max <= B_mem / (P * b / 8) ([HGF] §1.1).
+    Pinned by tests (the HGF page's printed 35 tokens/s at FP16)."""
     return bandwidth_bytes_s / (params * bits / 8.0)
 
 
 def weight_bits_per_param(fmt: str, w_bits: int = 0) -> float:
     """Storage bits per weight of the packed planes/bitvectors (scales excluded;
-    BVSR counts its 1-byte set index per 32-element vector)."""
+    BVSR counts its 1-byte set index per 32-element vector).
+    Pinned by tests (2 bits for ternary, 4.25 for BVSR, 1 for BitNet)."""
     return {"rabit": 2.0, "bitnet": 1.0, "ternary": 2.0, "abq": float(w_bits),
             "bvsr": BVSR_PLANES + 8.0 / BVSR_VEC}[fmt]
 
 
 def tolerance_ok(y, y_ref, rel: float = 1e-3) -> bool:
-    """max|y - y_ref| <= rel * (||y_ref||_inf + 1e-6)."""
+    """max|y - y_ref| <= rel * (||y_ref||_inf + 1e-6).
+    Pinned by tests (hand cases on both sides of the bound)."""
     y, y_ref = np.asarray(y, np.float64), np.asarray(y_ref, np.float64)
     if y_ref.size == 0:
         return y.size == 0

@@ -63,6 +63,8 @@ def _f32(buf: bytes, word: int) -> np.float32:
 
 
 def read_header(buf: bytes) -> dict:
+    """The packed buffer's 64-word header as a dict (documented word layout).
+    Pinned by tests (host header fixtures; every GPU pack round trip)."""
     if _u32(buf, 0) != PK_MAGIC:
         raise ValueError("bad packed magic")
     h = dict(version=_u32(buf, 1), fmt=_u32(buf, 2), N=_u32(buf, 3), K=_u32(buf, 4),
@@ -78,7 +80,8 @@ def read_header(buf: bytes) -> dict:
 
 def tiled_field_index(N_pad: int, K_pad: int, f: int):
     """For one stream of field width f, the (row, k) that each field of a tile
-    holds, as arrays over [u, lane, r, b, j] (the documented formula)."""
+    holds, as arrays over [u, lane, r, b, j] (the documented formula).
+    Pinned by tests (single-bit layout fixtures, tests/golden/layout_bits.json)."""
     u = np.arange(f)[:, None, None, None, None]
     lane = np.arange(32)[None, :, None, None, None]
     r = np.arange(4)[None, None, :, None, None]
@@ -92,7 +95,8 @@ def tiled_field_index(N_pad: int, K_pad: int, f: int):
 
 def read_stream_codes(buf: bytes, h: dict, s: int, row_blocks=None) -> np.ndarray:
     """Stream s of a tiled buffer as unsigned field values (uint8): [N, K], or
-    [16*len(row_blocks), K] for a subset of 16-row blocks."""
+    [16*len(row_blocks), K] for a subset of 16-row blocks.
+    Pinned by tests (single-bit layout fixtures; GPU pack round trips)."""
     f = h["fields"][s]
     N, K, N_pad, K_pad = h["N"], h["K"], h["N_pad"], h["K_pad"]
     RB, KT, tb = N_pad // 16, K_pad // 256, h["tile_bytes"]
@@ -117,7 +121,8 @@ def read_stream_codes(buf: bytes, h: dict, s: int, row_blocks=None) -> np.ndarra
 def read_packed(buf: bytes, row_blocks=None) -> dict:
     """Decode a packed buffer into the dict shape that bq_oracle's layers take.
     ``row_blocks`` (tiled formats) restricts the per-row arrays to those 16-row
-    blocks (rows 16*rb .. 16*rb+15, padding rows included); ``rows`` lists them."""
+    blocks (rows 16*rb .. 16*rb+15, padding rows included); ``rows`` lists them.
+    Pinned by tests (single-bit layout fixtures; GPU pack round trips of every format)."""
     h = read_header(buf)
     fmt, N, K, N_pad, K_pad = h["fmt"], h["N"], h["K"], h["N_pad"], h["K_pad"]
     out = dict(header=h)
@@ -208,6 +213,8 @@ def _bf16_to_f32(u16: np.ndarray) -> np.ndarray:
 
 
 def read_act(buf: bytes) -> dict:
+    """An activation buffer decoded into codes, token parameters, vector sums and LoRA
+    partials. Pinned by tests (single activation-code fixture; every GPU act round trip)."""
     if _u32(buf, 0) != ACT_MAGIC:
         raise ValueError("bad act magic")
     fmt, M, K, K_pad = _u32(buf, 2), _u32(buf, 3), _u32(buf, 4), _u32(buf, 5)

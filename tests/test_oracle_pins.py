@@ -433,3 +433,13 @@ def test_bit_balance_grid_round_trip():
     assert np.all(p["delta"] == d)
     deq = (p["Q"] - p["z"][:, None]).astype(np.float64) * p["delta"][:, None]
     assert np.array_equal(deq, W.astype(np.float64))
+
+
+def test_bf16_round_hand_values():
+    """Round to nearest bf16, ties to even (hand-worked bit patterns)."""
+    vals = np.array([1.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, 1.0 + 2.0 ** -8 + 2.0 ** -20, -2.5], np.float32)
+    # 1 + 2^-8 is half-way between 1 and 1 + 2^-7: ties to the even mantissa (1.0);
+    # 1 + 3*2^-8 is half-way between 1 + 2^-7 and 1 + 2^-6: ties to 1 + 2^-6;
+    # just above half-way rounds up; -2.5 is exact
+    want = np.array([1.0, 1.0, 1.0 + 2.0 ** -6, 1.0 + 2.0 ** -7, -2.5], np.float32)
+    assert np.array_equal(O.bf16_round(vals), want)
