@@ -443,3 +443,13 @@ def test_bf16_round_hand_values():
     # just above half-way rounds up; -2.5 is exact
     want = np.array([1.0, 1.0, 1.0 + 2.0 ** -6, 1.0 + 2.0 ** -7, -2.5], np.float32)
     assert np.array_equal(O.bf16_round(vals), want)
+
+
+def test_svid_first_round_path2_g_is_mean_abs_of_residual():
+    """In round 1, path 2's g-step starts from h = 1, so g2 is the row mean of |W - W_1|
+    (W_1 from the returned path-1 state): pins the split of the magnitude between g and h."""
+    W = I.weights(10, 256, seed=13)
+    p = O.rabit_pack_svid(W, rounds=1)
+    w1 = (p["g1"].astype(np.float64)[:, None] * p["h1"].astype(np.float64)[None, :]) * p["B1"]
+    g2 = np.abs(W.astype(np.float64) - w1).mean(1)
+    assert np.allclose(p["g2"], g2, rtol=1e-6)
