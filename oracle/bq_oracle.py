@@ -197,6 +197,36 @@ def rabit_recon_error(p, W) -> float:
     return float(np.sum(d * d))
 
 
+def rabit_pack_paths(W, hs) -> dict:
+    """The residual recursion of rabit_pack with P = len(hs) paths ([RaBiT] §2.1-2.2; §6 names
+    a 3-bit, three-path version as an extension): R_0 = W; path p takes B_p = sign(R_{p-1}),
+    g_p[n] = mean_k |R_{p-1}[n,:]| (float64 sum, stored float32) and the given h_p, then
+    R_p = R_{p-1} - g_p B_p h_p in float64 from the stored g_p and h_p.
+    hs: P float32 vectors [K] (hs[0] is 1 in the two-path reading). Returns B [P,N,K] int8,
+    g [P,N] float32, h [P,K] float32. With P = 2 and hs = (1, h2) it is rabit_pack.
+    Pinned by tests (P = 2 equals rabit_pack bit for bit; with h = 1 each added path lowers
+    ||W - W_hat||^2 by K g_p^2 per row)."""
+    W = _f32(W)
+    N, K = W.shape
+    P = len(hs)
+    R = W.astype(np.float64)
+    B = np.zeros((P, N, K), np.int8)
+    g = np.zeros((P, N), np.float32)
+    h = np.stack([_f32(v) for v in hs]).astype(np.float32)
+    for p in range(P):
+        B[p] = sign_pm1(R)
+        g[p] = np.array([mean_abs_f32(R[n]) for n in range(N)], dtype=np.float32)
+        R = R - g[p].astype(np.float64)[:, None] * B[p] * h[p].astype(np.float64)[None, :]
+    return dict(B=B, g=g, h=h)
+
+
+def rabit_weight_paths(p) -> np.ndarray:
+    """W_hat [N,K] float64 = sum_p g_p B_p h_p for a rabit_pack_paths result.
+    Pinned by tests (P = 2 equals rabit_weight)."""
+    return sum(p["g"][q].astype(np.float64)[:, None] * p["B"][q] * p["h"][q].astype(np.float64)[None, :]
+               for q in range(p["B"].shape[0]))
+
+
 def rabit_weight(p) -> np.ndarray:
     """W_hat [N,K] float64 = g1*B1*h1 + g2*B2*h2 ([RaBiT] §2.1).
     Pinned by tests (RaBiT hand recursion, constant-magnitude rows reconstruct exactly)."""

@@ -453,3 +453,27 @@ def test_svid_first_round_path2_g_is_mean_abs_of_residual():
     w1 = (p["g1"].astype(np.float64)[:, None] * p["h1"].astype(np.float64)[None, :]) * p["B1"]
     g2 = np.abs(W.astype(np.float64) - w1).mean(1)
     assert np.allclose(p["g2"], g2, rtol=1e-6)
+
+
+# ------------------------------------------------------------------ RaBiT with P paths (groundwork)
+def test_rabit_paths_two_equals_rabit_pack():
+    W = I.weights(9, 256, seed=17)
+    h2 = I.uniform(256, 0.5, 1.5, seed=2, tid=3)
+    a = O.rabit_pack(W, h2)
+    b = O.rabit_pack_paths(W, [np.ones(256, np.float32), h2])
+    assert np.array_equal(b["B"][0], a["B1"]) and np.array_equal(b["B"][1], a["B2"])
+    assert np.array_equal(b["g"][0], a["g1"]) and np.array_equal(b["g"][1], a["g2"])
+    assert np.array_equal(O.rabit_weight_paths(b), O.rabit_weight(a))
+
+
+def test_rabit_third_path_lowers_error_by_k_g_squared():
+    """With h = 1: ||R - g sign(R)||^2 = ||R||^2 - K g^2 per row when g = mean|R|."""
+    W = I.weights(7, 512, seed=23)
+    ones = np.ones(512, np.float32)
+    p2 = O.rabit_pack_paths(W, [ones, ones])
+    p3 = O.rabit_pack_paths(W, [ones, ones, ones])
+    e2 = ((W.astype(np.float64) - O.rabit_weight_paths(p2)) ** 2).sum(1)
+    e3 = ((W.astype(np.float64) - O.rabit_weight_paths(p3)) ** 2).sum(1)
+    g3 = p3["g"][2].astype(np.float64)
+    assert np.allclose(e2 - e3, 512 * g3 ** 2, rtol=1e-5)
+    assert np.all(e3 < e2)
