@@ -23,10 +23,15 @@
  *   bq_act_bytes / bq_quantize_act      per-token activation quantization
  *   bq_gemv (M = 1) / bq_gemm (M >= 1)  the layer, fused scale/zero-point/LoRA epilogue
  *   bq_linear                           activation quantization + layer in one kernel (decode)
+ *   bq_linear_group                     up to 4 layers sharing their input x, one launch
+ *   bq_linear_static_scratch            bq_linear with a fixed library scratch array
+ * Pack options (bq_pack_desc): RaBiT iterative residual SVID initialisation of g and h
+ * (rabit_svid_rounds, "RaBiT框架" page §2.3); ABQ bit-balance W2* (abq_bit_balance,
+ * "ABQ-LLM" page §3.3).
  *
  * Ownership: the caller allocates every buffer (device memory for packed, act, W, x, y);
- * sizes come from the *_bytes queries. The library never allocates, frees or
- * synchronizes (bq_packed_validate and bq_device_check excepted, which touch host memory
+ * sizes come from the *_bytes queries. The library never allocates (its one static
+ * scratch array aside, see bq_linear_static_scratch), frees or synchronizes (bq_packed_validate and bq_device_check excepted, which touch host memory
  * or read one device word). All work is enqueued on the caller's stream (a cudaStream_t
  * passed as void*; NULL = legacy default stream).
  *
