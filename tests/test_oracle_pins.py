@@ -446,7 +446,7 @@ def test_bf16_round_hand_values():
 
 
 def test_svid_first_round_path2_g_is_mean_abs_of_residual():
-    """In round 1, path 2's g-step starts from h = 1, so g2 is the row mean of |W - W_1|
+    """In the first Gauss-Seidel round, path 2's g-step starts from h = 1, so g2 is the row mean of |W - W_1|
     (W_1 from the returned path-1 state): pins the split of the magnitude between g and h."""
     W = I.weights(10, 256, seed=13)
     p = O.rabit_pack_svid(W, rounds=1)
