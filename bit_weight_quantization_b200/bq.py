@@ -30,6 +30,13 @@ class bq_pack_desc(ctypes.Structure):
                 ("abq_bit_balance", ctypes.c_int32)]
 
 
+class bq_plan_info(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("tokens_per_cta", "token_groups", "ctas_per_group",
+                                              "warps_per_row_block", "tiles_per_warp", "ring_stages",
+                                              "tiles_per_stage", "x_chunks_per_thread")] + \
+               [("shared_bytes", ctypes.c_uint32)]
+
+
 class bq_layer(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("N", ctypes.c_int32), ("K", ctypes.c_int32),
                 ("N_pad", ctypes.c_int32), ("K_pad", ctypes.c_int32), ("w_bits", ctypes.c_int32),
@@ -54,6 +61,8 @@ _SIGS = {
                                                  ctypes.POINTER(ctypes.c_size_t)]),
     "bq_linear": (ctypes.c_int, [ctypes.POINTER(bq_layer), _P, ctypes.c_int32, _P, _P, _P, ctypes.c_size_t, _P]),
     "bq_linear_static_scratch": (ctypes.c_int, [ctypes.POINTER(bq_layer), _P, ctypes.c_int32, _P, _P, _P]),
+    "bq_linear_plan": (ctypes.c_int, [ctypes.POINTER(bq_layer), ctypes.c_int32, ctypes.c_int32,
+                                      ctypes.POINTER(bq_plan_info)]),
     "bq_linear_group": (ctypes.c_int, [ctypes.POINTER(bq_layer), ctypes.c_int32, _P, ctypes.c_int32,
                                        ctypes.POINTER(_P), ctypes.POINTER(_P), _P]),
     "bq_device_check": (ctypes.c_int, []),
@@ -149,6 +158,13 @@ def bq_linear_workspace_bytes(layer: bq_layer, M: int) -> int:
     out = ctypes.c_size_t(0)
     _check(_lib.bq_linear_workspace_bytes(ctypes.byref(layer), M, ctypes.byref(out)), "bq_linear_workspace_bytes")
     return out.value
+
+
+def bq_linear_plan(layer: bq_layer, M: int, fused: bool = True) -> dict:
+    """The work split of bq_linear (fused) or bq_gemm for `layer` and M tokens (host only)."""
+    info = bq_plan_info()
+    _check(_lib.bq_linear_plan(ctypes.byref(layer), M, int(fused), ctypes.byref(info)), "bq_linear_plan")
+    return {n: getattr(info, n) for n, _ in bq_plan_info._fields_}
 
 
 BQ_STATIC_SCRATCH_BYTES = 1 << 20

@@ -162,8 +162,12 @@ inline uint32_t align128(uint64_t x) { return uint32_t((x + 127) & ~uint64_t(127
 
 inline int sm_count() {
   static int n = [] {
-    int dev = 0, v = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+      cudaGetLastError();  // no device visible: plan for a B200's 148 SMs
+      v = 148;
+    }
     return v;
   }();
   return n;
@@ -671,6 +675,27 @@ bq_status bq_linear_group(const bq_layer* layers, int32_t n_layers, const void* 
   PkLayout Lg = L0;  // the work split sees the group's row blocks as one layer
   Lg.RB = rb;
   return launch_layer(Lg, g, true, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bq_status bq_linear_plan(const bq_layer* layer, int32_t M, int32_t fused, bq_plan_info* info) {
+  PkLayout L;
+  bq_status st = check_layer(layer, &L);
+  if (st != BQ_OK) return st;
+  if (!info) return BQ_ERR_INVALID_ARG;
+  if (M < 1 || M > BQ_MAX_M) return BQ_ERR_SIZE;
+  if (L.fmt == BQ_FMT_RABIT2) return BQ_ERR_UNSUPPORTED;
+  LayerArgs g{};
+  if (!plan_layer(L, M, fused != 0, &g)) return BQ_ERR_UNSUPPORTED;
+  info->tokens_per_cta = g.tpc;
+  info->token_groups = g.TG;
+  info->ctas_per_group = g.CPG;
+  info->warps_per_row_block = g.WPR;
+  info->tiles_per_warp = g.T;
+  info->ring_stages = g.S;
+  info->tiles_per_stage = g.C;
+  info->x_chunks_per_thread = g.J;
+  info->shared_bytes = g.smem_bytes;
+  return BQ_OK;
 }
 
 bq_status bq_gemv(const bq_layer* layer, const void* act, float* y, int64_t* acc_dbg, void* stream) {

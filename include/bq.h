@@ -25,6 +25,7 @@
  *   bq_linear                           activation quantization + layer in one kernel (decode)
  *   bq_linear_group                     up to 4 layers sharing their input x, one launch
  *   bq_linear_static_scratch            bq_linear with a fixed library scratch array
+ *   bq_linear_plan                      the work split of bq_linear / bq_gemm (host only)
  * Pack options (bq_pack_desc): RaBiT iterative residual SVID initialisation of g and h
  * (rabit_svid_rounds, "RaBiT框架" page §2.3); ABQ bit-balance W2* (abq_bit_balance,
  * "ABQ-LLM" page §3.3).
@@ -250,6 +251,24 @@ bq_status bq_linear_group(const bq_layer* layers, int32_t n_layers, const void* 
 #define BQ_STATIC_SCRATCH_BYTES (1u << 20)
 bq_status bq_linear_static_scratch(const bq_layer* layer, const void* x_bf16, int32_t M, float* y,
                                    int64_t* acc_dbg, void* stream);
+
+/* The work split bq_linear (fused != 0) or bq_gemm (fused = 0) would use for `layer` and M
+ * tokens, for inspection and tuning. The pages have no counterpart. Host only: nothing is
+ * enqueued. BQ_ERR_UNSUPPORTED if the layer does not fit the tiled kernel, or for RaBiT
+ * (not tiled). The SM count is the current device's (148 when no device is visible). */
+typedef struct {
+  int32_t tokens_per_cta;         /* tokens sharing a CTA's MMA columns (<= 8) */
+  int32_t token_groups;           /* CTA groups, one per tokens_per_cta tokens */
+  int32_t ctas_per_group;         /* persistent CTAs per token group (grid = product) */
+  int32_t warps_per_row_block;    /* warps splitting K over one 16-row block (power of two) */
+  int32_t tiles_per_warp;         /* 256-k tiles of a row block one warp handles */
+  int32_t ring_stages;            /* weight-ring stages per warp */
+  int32_t tiles_per_stage;        /* 256-k tiles per ring stage */
+  int32_t x_chunks_per_thread;    /* fused staging: 16-byte chunks of x a thread holds
+                                     (0: x is read twice; 0 for bq_gemm) */
+  uint32_t shared_bytes;          /* dynamic shared memory per CTA */
+} bq_plan_info;
+bq_status bq_linear_plan(const bq_layer* layer, int32_t M, int32_t fused, bq_plan_info* info);
 
 /* Synchronizes the current device, then reads and clears the device error word:
  * BQ_OK or BQ_ERR_DEVICE_CHECK. */

@@ -224,3 +224,57 @@ def test_bit_balance_descriptor_checks():
                             ("abq", 3, 2, bq.BQ_ERR_INVALID_ARG), ("bitnet", 0, 1, bq.BQ_ERR_INVALID_ARG)]:
         d = bq.make_desc(fmt, w_bits=w, a_bits=8, abq_bit_balance=bal)
         assert bq.raw_status("bq_packed_bytes", ctypes.byref(d), 64, 256, ctypes.byref(out)) == st
+
+
+def _plan_cases():
+    return [("bitnet", 4096, 4096, {}), ("bitnet", 11008, 4096, {}), ("bitnet", 4096, 11008, {}),
+            ("bitnet", 300, 40960, {}), ("ternary", 2048, 2048, dict(lora_rank=32)),
+            ("abq", 4096, 4096, dict(w_bits=2, a_bits=8)), ("abq", 11008, 4096, dict(w_bits=8, a_bits=8)),
+            ("bvsr", 5120, 13824, {}), ("bvsr", 64, 256, {})]
+
+
+@pytest.mark.parametrize("fmt,N,K,kw", _plan_cases())
+@pytest.mark.parametrize("M", [1, 3, 8, 9, 64])
+@pytest.mark.parametrize("fused", [True, False])
+def test_linear_plan_invariants(fmt, N, K, kw, M, fused):
+    """The launch plan covers every token, k tile and row block, and fits the SM (host only)."""
+    h = _host_header(fmt, N, K, **kw)
+    p = bq.bq_linear_plan(bq.bq_packed_validate(h.tobytes(), 1 << 30), M, fused)
+    K_pad, N_pad, tile_bytes = int(h[6]), int(h[5]), int(h[18])
+    KT, RB, npad = K_pad // 256, N_pad // 16, K_pad // 8
+    pow2 = lambda t: 1 << (t - 1).bit_length()
+    chunks = lambda t: -(-npad // (256 // pow2(t)))
+    tpc, J = p["tokens_per_cta"], p["x_chunks_per_thread"]
+    assert 1 <= tpc <= min(8, M) and p["token_groups"] == -(-M // tpc)
+    if fused:   # the most tokens whose x fits 16 chunks per thread; else one token read twice
+        fits = [t for t in range(1, min(8, M) + 1) if chunks(t) <= 16]
+        assert tpc == (max(fits) if fits else 1)
+        assert J == (chunks(tpc) if fits else 0)
+    else:       # the most tokens whose int8 codes fit 96 KB
+        cstride = KT * 256 + 16
+        assert J == 0 and tpc == max([t for t in range(1, min(8, M) + 1) if t * cstride <= 96 * 1024] + [1])
+    assert p["ctas_per_group"] == max(1, min(RB, -(-148 // p["token_groups"])))  # 148 SMs when no device
+    wpr, T = p["warps_per_row_block"], p["tiles_per_warp"]
+    assert wpr in (1, 2, 4, 8) and T == -(-KT // wpr)
+    S, C = p["ring_stages"], p["tiles_per_stage"]
+    assert 2 <= S <= 4 and 1 <= C <= T and 8 * S * C * tile_bytes <= 96 * 1024
+    assert p["shared_bytes"] % 128 == 0 and 8 * S * C * tile_bytes < p["shared_bytes"] <= 227 * 1024
+
+
+def test_linear_plan_of_the_measured_llama7b_layers():
+    """The decode plans of the Llama-7B BitNet layers whose timings and DRAM traffic were
+    measured; a change here means those measurements are of another plan."""
+    want = {(4096, 4096): (4, 4, 4, 2), (11008, 4096): (1, 4, 6, 2), (4096, 11008): (4, 4, 6, 6)}
+    for (N, K), (wpr, S, C, J) in want.items():
+        p = bq.bq_linear_plan(bq.bq_packed_validate(_host_header("bitnet", N, K).tobytes(), 1 << 30), 1)
+        got = (p["warps_per_row_block"], p["ring_stages"], p["tiles_per_stage"], p["x_chunks_per_thread"])
+        assert got == (wpr, S, C, J), (N, K, got)
+
+
+def test_linear_plan_rejects():
+    layer = bq.bq_packed_validate(_host_header("bitnet", 64, 256).tobytes(), 1 << 20)
+    info = bq.bq_plan_info()
+    for M, st in [(0, bq.BQ_ERR_SIZE), (65, bq.BQ_ERR_SIZE), (1, bq.BQ_OK)]:
+        assert bq.raw_status("bq_linear_plan", ctypes.byref(layer), M, 1, ctypes.byref(info)) == st
+    assert bq.raw_status("bq_linear_plan", ctypes.byref(layer), 1, 1, None) == bq.BQ_ERR_INVALID_ARG
+    assert bq.raw_status("bq_linear_plan", None, 1, 1, ctypes.byref(info)) == bq.BQ_ERR_INVALID_ARG
