@@ -16,6 +16,7 @@ import numpy as np
 
 # tensor ids: one independent stream per tensor role
 TID_W, TID_X, TID_H2, TID_LORA_A, TID_LORA_B, TID_W_OUTLIER, TID_X_CHANNEL = 1, 2, 3, 4, 5, 6, 7
+TID_COMP_A, TID_COMP_B = 8, 9
 
 
 def rng(seed: int, tensor_id: int) -> np.random.Generator:
@@ -67,6 +68,13 @@ def activations(M: int, K: int, seed: int = 0, std: float = 1.0,
 
 def uniform(n: int, lo: float, hi: float, seed: int, tid: int) -> np.ndarray:
     return rng(seed, tid).uniform(lo, hi, size=n).astype(np.float32)
+
+
+def compensation_vectors(N: int, K: int, seed: int = 0, std: float = 0.1):
+    """The ABQ distribution-compensation vectors a [N] and b [K], float32, each
+    ~ N(0, std^2), so a b^T has std std^2 (0.01 by default, half the weights' 0.02).
+    The pages fit a and b by calibration on data; these seeded draws stand in."""
+    return gaussian(N, std, seed, TID_COMP_A), gaussian(K, std, seed, TID_COMP_B)
 
 
 # ---------------------------------------------------------------------------

@@ -345,6 +345,35 @@ def abq_pack_balanced(W) -> dict:
     return dict(Q=q.astype(np.int32), delta=delta, z=np.full(W.shape[0], 2, np.int32), w_bits=3)
 
 
+def abq_compensated_weights(W, a, b) -> np.ndarray:
+    """[ABQ] §3.2 eq.(3) distribution compensation: the matrix that is quantized is
+    W + gamma a b^T, gamma = 1 (compensation on) or 0 (off). Readings: a has one entry
+    per output row n and b one per input column k, so that a b^T has the shape of W;
+    a and b are given (the page fits them by calibration); the sum is formed in float32,
+    the product a[n] b[k] rounded first, then the sum (two roundings, no fused multiply-add).
+    Pinned by tests (a = 0 leaves W unchanged; dyadic closed forms exact in float32)."""
+    W, a, b = _f32(W), _f32(a), _f32(b)
+    assert a.shape == (W.shape[0],) and b.shape == (W.shape[1],)
+    prod = (a[:, None] * b[None, :]).astype(np.float32)
+    return (W + prod).astype(np.float32)
+
+
+def abq_pack_compensated(W, a, b, w_bits: int, balanced: bool = False) -> dict:
+    """[ABQ] §3.2 eq.(3) with gamma = 1: the codes of W' = W + a b^T
+    (abq_compensated_weights). Reading: the step Delta and zero point z are those of the
+    quantizer applied to W' itself (the row range of W'), so eq.(3)'s clamp to
+    0..2^n - 1 cuts nothing but rounding overshoot; with balanced, W' gets the W2*
+    codes of abq_pack_balanced (w_bits = 3). The layer then computes y = W'_hat x with
+    the ordinary ABQ layer.
+    Pinned by tests (closed-form grid codes, exact cancellation to the degenerate row,
+    W2* antisymmetry under (W, a) -> (-W, -a))."""
+    Wc = abq_compensated_weights(W, a, b)
+    if balanced:
+        assert w_bits == 3
+        return abq_pack_balanced(Wc)
+    return abq_pack(Wc, w_bits)
+
+
 def abq_pack(W, w_bits: int) -> dict:
     """Per-output-row asymmetric weight codes (quantize_rows_asym).
     Pinned by tests (hand examples with a rounding tie, grid round trip)."""

@@ -477,3 +477,72 @@ def test_rabit_third_path_lowers_error_by_k_g_squared():
     g3 = p3["g"][2].astype(np.float64)
     assert np.allclose(e2 - e3, 512 * g3 ** 2, rtol=1e-5)
     assert np.all(e3 < e2)
+
+
+# ---------------------------------------------------------------------------
+# ABQ distribution compensation ([ABQ] §3.2 eq.(3), gamma = 1)
+# ---------------------------------------------------------------------------
+# Dyadic data: every product a[n] b[k] and every sum below is exact in float32.
+_COMP_A = np.array([1.0, -2.0, 0.5], np.float32)                                    # per output row
+_COMP_B = np.array([0.25, -0.125, 0.0625, 0.0, 0.5, -0.25, 0.125, 1.0], np.float32) / 8  # per column
+_COMP_Q0 = np.array([[0, 1, 2, 3, 3, 2, 1, 0],     # 2-bit grid codes; every row reaches 0 and 3
+                     [3, 0, 0, 1, 2, 3, 1, 2],
+                     [1, 3, 2, 0, 0, 1, 3, 2]], np.int32)
+
+
+def test_abq_compensation_closed_form():
+    """W = G - a b^T with G on the 2-bit grid Delta = 1/16, z = 1: the compensated codes
+    are the grid codes, Delta and z come back exactly; without compensation they do not."""
+    G = ((_COMP_Q0 - 1) * 0.0625).astype(np.float32)
+    W = (G - np.outer(_COMP_A, _COMP_B)).astype(np.float32)
+    assert np.array_equal((W + np.outer(_COMP_A, _COMP_B)).astype(np.float32), G)   # exact data
+    p = O.abq_pack_compensated(W, _COMP_A, _COMP_B, 2)
+    assert np.array_equal(p["Q"], _COMP_Q0)
+    assert np.all(p["delta"] == np.float32(0.0625)) and np.all(p["z"] == 1)
+    assert not np.array_equal(O.abq_pack(W, 2)["Q"], _COMP_Q0)
+    # swapping the roles of a and b cannot even be formed: W is 3 x 8
+    with pytest.raises(AssertionError):
+        O.abq_pack_compensated(W, _COMP_B, _COMP_A, 2)
+
+
+def test_abq_compensation_exact_cancellation_is_the_degenerate_row():
+    """W = -a b^T: W' = 0 exactly, every row is constant, so the 1e-5 range floor applies,
+    z = 0 and every code is 0 at any width."""
+    W = (-np.outer(_COMP_A, _COMP_B)).astype(np.float32)
+    for w in (1, 2, 4, 8):
+        p = O.abq_pack_compensated(W, _COMP_A, _COMP_B, w)
+        assert np.all(p["Q"] == 0) and np.all(p["z"] == 0)
+        assert np.all(p["delta"] > 0) and np.all(p["delta"] <= np.float32(1e-5))   # = at w = 1
+
+
+def test_abq_compensation_off_is_the_plain_pack():
+    """a = 0 (or b = 0): W + 0 = W, so the codes, Delta and z are the plain pack's."""
+    W = I.weights(37, 256, seed=5, outlier_frac=0.01)
+    a, b = I.compensation_vectors(37, 256, seed=5)
+    for w in (2, 5, 8):
+        ref = O.abq_pack(W, w)
+        for aa, bb in ((np.zeros_like(a), b), (a, np.zeros_like(b))):
+            p = O.abq_pack_compensated(W, aa, bb, w)
+            assert all(np.array_equal(p[k], ref[k]) for k in ("Q", "delta", "z"))
+    assert not np.array_equal(O.abq_pack_compensated(W, a, b, 8)["Q"], O.abq_pack(W, 8)["Q"])
+
+
+def test_abq_compensation_rounds_the_product_first():
+    """The product is rounded before the sum: (1 + 2^-12)^2 = 1 + 2^-11 + 2^-24 rounds (a tie,
+    to even) to 1 + 2^-11, so W = -(1 + 2^-11) compensates to exactly 0 (a fused
+    multiply-add would leave 2^-24)."""
+    u = np.float32(1 + 2.0 ** -12)
+    W = np.array([[-(1 + 2.0 ** -11), 1.0]], np.float32)
+    Wc = O.abq_compensated_weights(W, np.array([u]), np.array([u, 0.0], np.float32))
+    assert Wc[0, 0] == 0.0 and Wc[0, 1] == 1.0
+
+
+def test_abq_compensation_balanced_antisymmetry():
+    """W2* on W' : (W, a) -> (-W, -a) negates W' exactly, so q -> 4 - q with the same Delta."""
+    W = I.weights(29, 512, seed=7)
+    a, b = I.compensation_vectors(29, 512, seed=7)
+    p = O.abq_pack_compensated(W, a, b, 3, balanced=True)
+    m = O.abq_pack_compensated(-W, -a, b, 3, balanced=True)
+    assert np.array_equal(m["Q"], 4 - p["Q"]) and np.array_equal(m["delta"], p["delta"])
+    assert p["Q"].min() == 0 and p["Q"].max() == 4
+    assert not np.array_equal(p["Q"], O.abq_pack_balanced(W)["Q"])
