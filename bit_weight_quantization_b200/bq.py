@@ -27,7 +27,8 @@ class bq_pack_desc(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("w_bits", ctypes.c_int32), ("a_bits", ctypes.c_int32),
                 ("lora_rank", ctypes.c_int32), ("lora_alpha", ctypes.c_float), ("h2", ctypes.c_void_p),
                 ("lora_A", ctypes.c_void_p), ("lora_B", ctypes.c_void_p), ("rabit_svid_rounds", ctypes.c_int32),
-                ("abq_bit_balance", ctypes.c_int32)]
+                ("abq_bit_balance", ctypes.c_int32), ("abq_comp_a", ctypes.c_void_p),
+                ("abq_comp_b", ctypes.c_void_p)]
 
 
 class bq_plan_info(ctypes.Structure):
@@ -109,9 +110,10 @@ def bq_version() -> int:
 
 
 def make_desc(fmt, w_bits=0, a_bits=0, lora_rank=0, lora_alpha=0.1, h2=None, lora_A=None, lora_B=None,
-              rabit_svid_rounds=0, abq_bit_balance=0):
+              rabit_svid_rounds=0, abq_bit_balance=0, abq_comp_a=None, abq_comp_b=None):
     return bq_pack_desc(FORMATS.get(fmt, fmt), w_bits, a_bits, lora_rank, lora_alpha,
-                        _ptr(h2), _ptr(lora_A), _ptr(lora_B), rabit_svid_rounds, abq_bit_balance)
+                        _ptr(h2), _ptr(lora_A), _ptr(lora_B), rabit_svid_rounds, abq_bit_balance,
+                        _ptr(abq_comp_a), _ptr(abq_comp_b))
 
 
 def bq_packed_bytes(desc: bq_pack_desc, N: int, K: int) -> int:
@@ -208,15 +210,16 @@ class QuantLinear:
     All arithmetic happens in the library."""
 
     def __init__(self, fmt, W, *, w_bits=0, a_bits=0, lora_rank=0, lora_alpha=0.1, h2=None,
-                 lora_A=None, lora_B=None, rabit_svid_rounds=0, abq_bit_balance=0, stream=None):
+                 lora_A=None, lora_B=None, rabit_svid_rounds=0, abq_bit_balance=0, abq_comp_a=None,
+                 abq_comp_b=None, stream=None):
         import torch
         N, K = W.shape
         self.desc = make_desc(fmt, w_bits, a_bits, lora_rank, lora_alpha, h2, lora_A, lora_B, rabit_svid_rounds,
-                              abq_bit_balance)
+                              abq_bit_balance, abq_comp_a, abq_comp_b)
         nbytes = bq_packed_bytes(self.desc, N, K)
         self.packed = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
         self.layer = bq_pack_weights(self.desc, W, N, K, self.packed, nbytes, stream)
-        # the pack reads W, h2 and the LoRA matrices asynchronously: wait before the caller may free them
+        # the pack reads W, h2, the LoRA matrices and a, b asynchronously: wait before the caller may free them
         torch.cuda.synchronize(W.device)
         self.N, self.K = N, K
         self._acts = {}

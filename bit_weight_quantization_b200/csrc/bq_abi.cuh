@@ -25,6 +25,7 @@ inline bq_status check_desc(const bq_pack_desc* d, int K, bool need_ptrs) {
   if (d->fmt != BQ_FMT_RABIT2 && d->rabit_svid_rounds != 0) return BQ_ERR_INVALID_ARG;
   if (d->abq_bit_balance != 0 && (d->fmt != BQ_FMT_ABQ || d->abq_bit_balance != 1 || d->w_bits != 3))
     return BQ_ERR_INVALID_ARG;
+  if (d->fmt != BQ_FMT_ABQ && (d->abq_comp_a || d->abq_comp_b)) return BQ_ERR_INVALID_ARG;
   switch (d->fmt) {
     case BQ_FMT_RABIT2:
       if (d->rabit_svid_rounds < 0 || d->rabit_svid_rounds > 1000) return BQ_ERR_INVALID_ARG;
@@ -41,6 +42,9 @@ inline bq_status check_desc(const bq_pack_desc* d, int K, bool need_ptrs) {
       if (d->w_bits < 1 || d->w_bits > 8 || d->a_bits < 1 || d->a_bits > 8) return BQ_ERR_INVALID_ARG;
       const long long bound = ((1ll << d->w_bits) - 1) * ((1ll << d->a_bits) - 1) * (long long)K;
       if (bound >= (1ll << 31)) return BQ_ERR_SIZE;
+      if (need_ptrs && (!d->abq_comp_a != !d->abq_comp_b || !aligned(d->abq_comp_a, 4) ||
+                        !aligned(d->abq_comp_b, 4)))
+        return BQ_ERR_INVALID_ARG;
       return BQ_OK;
     }
     case BQ_FMT_BVSR4:
@@ -406,8 +410,10 @@ bq_status bq_pack_weights(const bq_pack_desc* desc, const float* W, int32_t N, i
       float* delta = reinterpret_cast<float*>(P + L.off_rows);
       int* zero = reinterpret_cast<int*>(P + L.off_rows) + L.N_pad;
       int* sumq = reinterpret_cast<int*>(P + L.off_rows) + 2 * L.N_pad;
-      k_abq_rows<<<N, 256, 0, s>>>(W, K, L.w_bits, desc->abq_bit_balance, delta, zero, sumq);
+      k_abq_rows<<<N, 256, 0, s>>>(W, desc->abq_comp_a, desc->abq_comp_b, K, L.w_bits, desc->abq_bit_balance,
+                                   delta, zero, sumq);
       fa.abq_delta = delta; fa.abq_zero = zero;
+      fa.abq_comp_a = desc->abq_comp_a; fa.abq_comp_b = desc->abq_comp_b;
       k_pack_fields<BQ_FMT_ABQ><<<blocks_for(fa.total_words, 256), 256, 0, s>>>(fa);
       break;
     }

@@ -61,16 +61,25 @@ __device__ __forceinline__ int abq_code(float w, float delta, int z, int qmax) {
   return int(q);
 }
 
+// The weight the ABQ codes quantize: W[n][k], or with distribution compensation (ca, cb not
+// null) W[n][k] + ca[n] * cb[k], the product rounded before the sum (ABQ-LLM §3.2 eq.(3)).
+__device__ __forceinline__ float abq_weight(float w, const float* ca, const float* cb, int n, int k) {
+  return ca ? __fadd_rn(w, __fmul_rn(ca[n], cb[k])) : w;
+}
+
 // balanced (W2*, w_bits = 3): symmetric range [-max|W|, max|W|] in 4 steps, z = 2; the
 // codes rn(W/Delta) + 2 then lie in 0..4 (|W/Delta| <= 2), under the same clamp.
-__global__ void k_abq_rows(const float* __restrict__ W, int K, int w_bits, int balanced, float* __restrict__ delta,
-                           int* __restrict__ zero, int* __restrict__ sumq) {
+// One block per row n < N; ca [N] and cb [K] are the optional compensation vectors.
+__global__ void k_abq_rows(const float* __restrict__ W, const float* __restrict__ ca, const float* __restrict__ cb,
+                           int K, int w_bits, int balanced, float* __restrict__ delta, int* __restrict__ zero,
+                           int* __restrict__ sumq) {
   __shared__ float shf[32];
   __shared__ int shi[32];
-  const float* w = W + size_t(blockIdx.x) * K;
+  const int n = blockIdx.x;
+  const float* w = W + size_t(n) * K;
   float lo = INFINITY, hi = -INFINITY;
   for (int k = threadIdx.x; k < K; k += blockDim.x) {
-    float v = w[k];
+    float v = abq_weight(w[k], ca, cb, n, k);
     lo = fminf(lo, v);
     hi = fmaxf(hi, v);
   }
@@ -88,7 +97,7 @@ __global__ void k_abq_rows(const float* __restrict__ W, int K, int w_bits, int b
     z = int(rintf(__fdiv_rn(-lo, d)));
   }
   int s = 0;
-  for (int k = threadIdx.x; k < K; k += blockDim.x) s += abq_code(w[k], d, z, qmax);
+  for (int k = threadIdx.x; k < K; k += blockDim.x) s += abq_code(abq_weight(w[k], ca, cb, n, k), d, z, qmax);
   s = block_sum(s, shi);
   if (threadIdx.x == 0) {
     delta[blockIdx.x] = d;
@@ -108,6 +117,8 @@ struct FieldPackArgs {
   const uint32_t* hdr;      // for the tensor scale (ternary gamma_W)
   const float* abq_delta;   // ABQ row params
   const int* abq_zero;
+  const float* abq_comp_a;  // ABQ distribution compensation a [N], b [K] (null: off)
+  const float* abq_comp_b;
   int w_bits;
   uint64_t total_words;
 };
@@ -152,7 +163,7 @@ __global__ void k_pack_fields(FieldPackArgs a) {
         }
         field = uint32_t(T + 1);                              // {0,1,2}
       } else {                                                // ABQ
-        int q = in ? abq_code(w, d, z, qmax) : 0;
+        int q = in ? abq_code(abq_weight(w, a.abq_comp_a, a.abq_comp_b, row, k), d, z, qmax) : 0;
         field = (uint32_t(q) >> a.shift[s]) & ((1u << f) - 1u);
       }
       word |= field << (8 * b + f * j);

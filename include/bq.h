@@ -28,7 +28,8 @@
  *   bq_linear_plan                      the work split of bq_linear / bq_gemm (host only)
  * Pack options (bq_pack_desc): RaBiT iterative residual SVID initialisation of g and h
  * (rabit_svid_rounds, "RaBiT框架" page §2.3); ABQ bit-balance W2* (abq_bit_balance,
- * "ABQ-LLM" page §3.3).
+ * "ABQ-LLM" page §3.3); ABQ distribution compensation W + a b^T (abq_comp_a, abq_comp_b,
+ * "ABQ-LLM" page §3.2 eq.(3)).
  *
  * Ownership: the caller allocates every buffer (device memory for packed, act, W, x, y);
  * sizes come from the *_bytes queries. The library never allocates (its one static
@@ -148,6 +149,14 @@ typedef struct {
                            (max(2 max|W|, 1e-5) / 4), z = 2, code = clamp(rn(W/Delta) + 2, 0, 4)
                            in a 3-bit field; requires w_bits = 3. The layer is the ABQ w = 3
                            layer. 0 = the asymmetric min/max codes. Must be 0 for the others. */
+  const float* abq_comp_a;  /* ABQ distribution compensation ("ABQ-LLM" page, §3.2 eq.(3) with
+                           gamma = 1): device f32 a [N] (one per output row) and b [K] (one per */
+  const float* abq_comp_b;  /* input column). Both set: the matrix quantized is W + a b^T, each
+                           element formed in f32 as W[n][k] + (a[n] * b[k]) (product rounded,
+                           then the sum; no fused multiply-add), and Delta, z and the codes are
+                           those of that matrix (with abq_bit_balance too: its W2* codes). The
+                           layer then computes y = (W + a b^T)_hat x. Both NULL: off. One of
+                           them NULL, or either set for another format: BQ_ERR_INVALID_ARG. */
 } bq_pack_desc;
 
 /* Host-side description of a packed layer; filled by bq_pack_weights or

@@ -226,6 +226,22 @@ def test_bit_balance_descriptor_checks():
         assert bq.raw_status("bq_packed_bytes", ctypes.byref(d), 64, 256, ctypes.byref(out)) == st
 
 
+def test_compensation_descriptor_checks():
+    """a and b: both or neither, ABQ only, 4-byte aligned; refused before anything runs."""
+    out = ctypes.c_size_t(0)
+    fake = 1 << 40
+    d = bq.make_desc("bitnet", abq_comp_a=fake, abq_comp_b=fake)
+    assert bq.raw_status("bq_packed_bytes", ctypes.byref(d), 64, 256, ctypes.byref(out)) == bq.BQ_ERR_INVALID_ARG
+    d = bq.make_desc("abq", w_bits=4, a_bits=4, abq_comp_a=fake, abq_comp_b=fake)
+    assert bq.raw_status("bq_packed_bytes", ctypes.byref(d), 64, 256, ctypes.byref(out)) == bq.BQ_OK
+    plain = bq.make_desc("abq", w_bits=4, a_bits=4)
+    assert bq.bq_packed_bytes(d, 64, 256) == bq.bq_packed_bytes(plain, 64, 256)   # same buffer
+    for a, b in [(fake, None), (None, fake), (fake + 2, fake), (fake, fake + 1)]:
+        d = bq.make_desc("abq", w_bits=4, a_bits=4, abq_comp_a=a, abq_comp_b=b)
+        assert bq.raw_status("bq_pack_weights", ctypes.byref(d), fake, 64, 256, fake, 1 << 30, None,
+                             ctypes.byref(bq.bq_layer())) == bq.BQ_ERR_INVALID_ARG
+
+
 def _plan_cases():
     return [("bitnet", 4096, 4096, {}), ("bitnet", 11008, 4096, {}), ("bitnet", 4096, 11008, {}),
             ("bitnet", 300, 40960, {}), ("ternary", 2048, 2048, dict(lora_rank=32)),

@@ -343,3 +343,31 @@ def test_abq_bit_balance(N, K, M):
         assert np.array_equal(acc.cpu().numpy(), r["I"])
         assert_y_close(y.cpu().numpy(), r["y"], "abq W2*")
     bq.bq_device_check()
+
+
+# ------------------------------------------------------------------ ABQ distribution compensation
+@pytest.mark.parametrize("w,a,balanced", [(2, 8, False), (4, 4, False), (8, 8, False), (3, 8, True)])
+@pytest.mark.parametrize("N,K,M", [(50, 384, 1), (97, 640, 9), (4096, 4096, 1)])
+def test_abq_compensation(w, a, balanced, N, K, M):
+    """W + a b^T quantized in the pack: codes, Delta, z and S_w equal the oracle's bit for bit;
+    the unchanged ABQ layer then matches the oracle's integer accumulator exactly."""
+    from tests.parity_util import L as layout, torch_mods
+    torch, bq = torch_mods()
+    inp = I.layer_inputs("abq", N, K, M, seed=N + w)
+    W, x = inp["W"], inp["x"]
+    ca, cb = I.compensation_vectors(N, K, seed=N + w)
+    ql = bq.QuantLinear("abq", to_dev_f32(W), w_bits=w, a_bits=a, abq_bit_balance=int(balanced),
+                        abq_comp_a=to_dev_f32(ca), abq_comp_b=to_dev_f32(cb))
+    p = layout.read_packed(ql.packed.cpu().numpy().tobytes())
+    ref = O.abq_pack_compensated(W, ca, cb, w, balanced)
+    assert np.array_equal(p["delta"], ref["delta"]) and np.array_equal(p["z"], ref["z"])
+    assert np.array_equal(p["Q"], ref["Q"]) and np.array_equal(p["S_w"], ref["Q"].sum(1))
+    xd = to_dev_bf16(x)
+    y = torch.full((M, N), float("nan"), device="cuda")
+    acc = torch.full((M, N), -(1 << 62), dtype=torch.int64, device="cuda")
+    ql.linear(xd, y, acc)
+    torch.cuda.synchronize()
+    r = O.abq_layer(p, x, a)
+    assert np.array_equal(acc.cpu().numpy(), r["I"])
+    assert_y_close(y.cpu().numpy(), r["y"], "abq compensated")
+    bq.bq_device_check()
