@@ -81,6 +81,17 @@ def test_small_parity_abq(wa, N, K, M):
     _layer_parity(gl, p, "abq", a)
 
 
+@pytest.mark.parametrize("fmt", ["bitnet", "ternary", "bvsr"])
+@pytest.mark.parametrize("N,K", [(97, 640), (40, 2560)])
+def test_max_tokens(fmt, N, K):
+    """M = 64, the largest batch: eight token groups of eight, ragged N and K; act + gemm and
+    the fused call agree bit for bit (checked in GpuLayer) and match the oracle."""
+    gl = GpuLayer(fmt, N, K, 64, seed=N + K)
+    p = _pack_parity(gl, fmt)
+    check_act(gl)
+    _layer_parity(gl, p, fmt)
+
+
 @pytest.mark.parametrize("fmt", ["bitnet", "ternary", "bvsr", "rabit", "abq"])
 def test_zero_activations(fmt):
     gl = GpuLayer(fmt, 40, 256, 2, w_bits=4, a_bits=4, nullify_x=True)
