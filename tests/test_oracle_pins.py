@@ -479,6 +479,20 @@ def test_rabit_third_path_lowers_error_by_k_g_squared():
     assert np.all(e3 < e2)
 
 
+def test_rabit_three_paths_hand_example():
+    """Three paths with non-unit h (every value dyadic, so exact), worked by hand:
+    W = [.75, -.25, .5, -1]: B1 = [+ - + -], g1 = 2.5/4 = .625, R1 = [.125, .375, -.125, -.375];
+    B2 = [+ + - -], g2 = 1/4 = .25, R2 = R1 - .25 B2 h2 with h2 = [1, 2, 1, .5]
+       = [-.125, -.125, .125, -.25]; B3 = [- - + -], g3 = .625/4 = .15625;
+    W_hat = sum_p g_p B_p h_p with h3 = [2, 1, .5, 1] = [.5625, -.28125, .453125, -.90625]."""
+    W = np.array([[0.75, -0.25, 0.5, -1.0]], np.float32)
+    hs = [np.ones(4, np.float32), np.array([1, 2, 1, 0.5], np.float32), np.array([2, 1, 0.5, 1], np.float32)]
+    p = O.rabit_pack_paths(W, hs)
+    assert p["B"][:, 0].tolist() == [[1, -1, 1, -1], [1, 1, -1, -1], [-1, -1, 1, -1]]
+    assert p["g"][:, 0].tolist() == [0.625, 0.25, 0.15625]
+    assert O.rabit_weight_paths(p)[0].tolist() == [0.5625, -0.28125, 0.453125, -0.90625]
+
+
 # ---------------------------------------------------------------------------
 # ABQ distribution compensation ([ABQ] §3.2 eq.(3), gamma = 1)
 # ---------------------------------------------------------------------------
