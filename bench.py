@@ -39,11 +39,12 @@ NOMINAL_HBM_GBS = 8000.0
 def layer_bytes(fmt: str, N: int, K: int, M: int = 1, w_bits: int = 1, a_bits: int = 8) -> dict:
     """Algorithmic bytes of one layer call: packed weights + per-row/tensor scales,
     x bf16 read by the act kernel, act codes written and read once, y fp32."""
-    if fmt == "rabit":
-        # 2 sign planes + g1,g2 + h1,h2; act: x bf16 in, x~1, x~2 f32 out and back in; y f32
-        w = 2 * N * K // 8 + 8 * N + 8 * K
-        return dict(gemv=w + 8 * M * K + 4 * M * N, act=2 * M * K + 8 * M * K + 8 * K,
-                    total=w + 2 * M * K + 16 * M * K + 8 * K + 4 * M * N, fused=w + 2 * M * K + 4 * M * N)
+    if fmt in ("rabit", "rabit3"):
+        # P sign planes + g_p + h_p; act: x bf16 in, h_p x f32 out and back in; y f32
+        P = 2 if fmt == "rabit" else 3
+        w = P * N * K // 8 + 4 * P * N + 4 * P * K
+        return dict(gemv=w + 4 * P * M * K + 4 * M * N, act=2 * M * K + 4 * P * M * K + 4 * P * K,
+                    total=w + 2 * M * K + 8 * P * M * K + 4 * P * K + 4 * M * N, fused=w + 2 * M * K + 4 * M * N)
     bits = {"bitnet": 1, "ternary": 2, "abq": w_bits, "bvsr": 4}[fmt]
     w = N * K * bits // 8
     extra = {"bitnet": 4, "ternary": 4, "abq": 12 * N, "bvsr": N * K // 32 + 256 * 32}[fmt]
@@ -415,8 +416,10 @@ def make_layer(fmt, N, K, M, w_bits, a_bits, gen, device):
     from bit_weight_quantization_b200 import bq
     W = torch.randn(N, K, device=device, generator=gen) * 0.02
     kw = {}
-    if fmt == "rabit":
+    if fmt in ("rabit", "rabit3"):
         kw["h2"] = torch.rand(K, device=device, generator=gen) + 0.5
+    if fmt == "rabit3":
+        kw["h3"] = torch.rand(K, device=device, generator=gen) + 0.5
     if fmt == "ternary":
         kw.update(lora_rank=32, lora_alpha=0.1,
                   lora_A=torch.randn(K, 32, device=device, generator=gen) * 0.02,
@@ -454,7 +457,7 @@ def layer_call(L, timing=None, fused=True):
 
 
 def config_list():
-    out = [("rabit", 256, 512, 1, 0, 0)]
+    out = [("rabit", 256, 512, 1, 0, 0), ("rabit3", 256, 512, 1, 0, 0)]
     out += [("bitnet", N, K, 1, 1, 8) for N, K in [(4096, 4096), (11008, 4096), (4096, 11008)]]
     out += [("ternary", 2048, 2048, M, 2, 8) for M in (1, 4, 16)]
     out += [("abq", N, 4096, M, w, a) for (w, a) in [(2, 8), (4, 4), (6, 6), (8, 8)]

@@ -19,8 +19,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 BQ_OK, BQ_ERR_INVALID_ARG, BQ_ERR_UNSUPPORTED, BQ_ERR_SIZE = 0, 1, 2, 3
 BQ_ERR_CUDA, BQ_ERR_BAD_PACKED, BQ_ERR_DEVICE_CHECK = 4, 5, 6
-BQ_FMT_RABIT2, BQ_FMT_BITNET_W1A8, BQ_FMT_TERNARY_A8, BQ_FMT_ABQ, BQ_FMT_BVSR4 = 1, 2, 3, 4, 5
-FORMATS = {"rabit": 1, "bitnet": 2, "ternary": 3, "abq": 4, "bvsr": 5}
+BQ_FMT_RABIT2, BQ_FMT_BITNET_W1A8, BQ_FMT_TERNARY_A8, BQ_FMT_ABQ, BQ_FMT_BVSR4, BQ_FMT_RABIT3 = 1, 2, 3, 4, 5, 6
+FORMATS = {"rabit": 1, "bitnet": 2, "ternary": 3, "abq": 4, "bvsr": 5, "rabit3": 6}
 
 
 class bq_pack_desc(ctypes.Structure):
@@ -28,7 +28,7 @@ class bq_pack_desc(ctypes.Structure):
                 ("lora_rank", ctypes.c_int32), ("lora_alpha", ctypes.c_float), ("h2", ctypes.c_void_p),
                 ("lora_A", ctypes.c_void_p), ("lora_B", ctypes.c_void_p), ("rabit_svid_rounds", ctypes.c_int32),
                 ("abq_bit_balance", ctypes.c_int32), ("abq_comp_a", ctypes.c_void_p),
-                ("abq_comp_b", ctypes.c_void_p)]
+                ("abq_comp_b", ctypes.c_void_p), ("h3", ctypes.c_void_p)]
 
 
 class bq_plan_info(ctypes.Structure):
@@ -110,10 +110,10 @@ def bq_version() -> int:
 
 
 def make_desc(fmt, w_bits=0, a_bits=0, lora_rank=0, lora_alpha=0.1, h2=None, lora_A=None, lora_B=None,
-              rabit_svid_rounds=0, abq_bit_balance=0, abq_comp_a=None, abq_comp_b=None):
+              rabit_svid_rounds=0, abq_bit_balance=0, abq_comp_a=None, abq_comp_b=None, h3=None):
     return bq_pack_desc(FORMATS.get(fmt, fmt), w_bits, a_bits, lora_rank, lora_alpha,
                         _ptr(h2), _ptr(lora_A), _ptr(lora_B), rabit_svid_rounds, abq_bit_balance,
-                        _ptr(abq_comp_a), _ptr(abq_comp_b))
+                        _ptr(abq_comp_a), _ptr(abq_comp_b), _ptr(h3))
 
 
 def bq_packed_bytes(desc: bq_pack_desc, N: int, K: int) -> int:
@@ -211,15 +211,15 @@ class QuantLinear:
 
     def __init__(self, fmt, W, *, w_bits=0, a_bits=0, lora_rank=0, lora_alpha=0.1, h2=None,
                  lora_A=None, lora_B=None, rabit_svid_rounds=0, abq_bit_balance=0, abq_comp_a=None,
-                 abq_comp_b=None, stream=None):
+                 abq_comp_b=None, h3=None, stream=None):
         import torch
         N, K = W.shape
         self.desc = make_desc(fmt, w_bits, a_bits, lora_rank, lora_alpha, h2, lora_A, lora_B, rabit_svid_rounds,
-                              abq_bit_balance, abq_comp_a, abq_comp_b)
+                              abq_bit_balance, abq_comp_a, abq_comp_b, h3)
         nbytes = bq_packed_bytes(self.desc, N, K)
         self.packed = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
         self.layer = bq_pack_weights(self.desc, W, N, K, self.packed, nbytes, stream)
-        # the pack reads W, h2, the LoRA matrices and a, b asynchronously: wait before the caller may free them
+        # the pack reads W, h2, h3, the LoRA matrices and a, b asynchronously: wait before the caller may free them
         torch.cuda.synchronize(W.device)
         self.N, self.K = N, K
         self._acts = {}

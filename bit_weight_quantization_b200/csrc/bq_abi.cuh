@@ -26,10 +26,14 @@ inline bq_status check_desc(const bq_pack_desc* d, int K, bool need_ptrs) {
   if (d->abq_bit_balance != 0 && (d->fmt != BQ_FMT_ABQ || d->abq_bit_balance != 1 || d->w_bits != 3))
     return BQ_ERR_INVALID_ARG;
   if (d->fmt != BQ_FMT_ABQ && (d->abq_comp_a || d->abq_comp_b)) return BQ_ERR_INVALID_ARG;
+  if (d->fmt != BQ_FMT_RABIT3 && d->h3) return BQ_ERR_INVALID_ARG;
   switch (d->fmt) {
     case BQ_FMT_RABIT2:
       if (d->rabit_svid_rounds < 0 || d->rabit_svid_rounds > 1000) return BQ_ERR_INVALID_ARG;
       if (need_ptrs && d->rabit_svid_rounds == 0 && (!d->h2 || !aligned(d->h2, 4))) return BQ_ERR_INVALID_ARG;
+      return BQ_OK;
+    case BQ_FMT_RABIT3:  // the residual recursion only; h2 and h3 given
+      if (need_ptrs && (!d->h2 || !aligned(d->h2, 4) || !d->h3 || !aligned(d->h3, 4))) return BQ_ERR_INVALID_ARG;
       return BQ_OK;
     case BQ_FMT_BITNET_W1A8:
       return BQ_OK;
@@ -150,8 +154,7 @@ inline LayerArgs layer_args(const PkLayout& L, const void* packed, int M, float*
   g.bvsr_table = reinterpret_cast<const float*>(P + L.off_aux);
   g.rabit_planes = reinterpret_cast<const uint32_t*>(P + L.off_tiles);
   g.rabit_g = reinterpret_cast<const float*>(P + L.off_rows);
-  g.rabit_h1 = reinterpret_cast<const float*>(P + L.off_aux);
-  g.rabit_h2 = reinterpret_cast<const float*>(P + L.off_aux2);
+  g.rabit_h = reinterpret_cast<const float*>(P + L.off_aux);
   g.y = y;
   g.acc = reinterpret_cast<long long*>(acc);
   g.N = L.N; g.K = L.K; g.N_pad = L.N_pad; g.K_pad = L.K_pad; g.KT = L.KT; g.M = M;
@@ -318,10 +321,14 @@ inline cudaError_t launch_fmt(const PkLayout& L, const LayerArgs& g, int NW, dim
 
 inline bq_status launch_layer(const PkLayout& L, LayerArgs& g, bool fused, cudaStream_t s) {
   cudaError_t e;
-  if (L.fmt == BQ_FMT_RABIT2) {
+  if (rabit_paths(L.fmt)) {
     const dim3 grid(unsigned((L.N + 7) / 8));
-    e = fused ? launch_pdl(k_rabit<8, true>, grid, dim3(256), 0, s, g)
-              : launch_pdl(k_rabit<8, false>, grid, dim3(256), 0, s, g);
+    if (rabit_paths(L.fmt) == 2)
+      e = fused ? launch_pdl(k_rabit<8, true, 2>, grid, dim3(256), 0, s, g)
+                : launch_pdl(k_rabit<8, false, 2>, grid, dim3(256), 0, s, g);
+    else
+      e = fused ? launch_pdl(k_rabit<8, true, 3>, grid, dim3(256), 0, s, g)
+                : launch_pdl(k_rabit<8, false, 3>, grid, dim3(256), 0, s, g);
   } else {
     if (!plan_layer(L, g.M, fused, &g)) return BQ_ERR_UNSUPPORTED;
     const dim3 grid(unsigned(g.TG * g.CPG));
@@ -424,7 +431,7 @@ bq_status bq_pack_weights(const bq_pack_desc* desc, const float* W, int32_t N, i
       float* h2 = reinterpret_cast<float*>(P + L.off_aux2);
       if (desc->rabit_svid_rounds == 0) {
         k_rabit_pack<<<N, 256, 0, s>>>(W, L.N_pad, K, L.K_pad, planes, g);
-        k_rabit_h<<<blocks_for(L.K_pad, 256), 256, 0, s>>>(desc->h2, K, L.K_pad, h1, h2);
+        k_rabit_h<<<blocks_for(L.K_pad, 256), 256, 0, s>>>(desc->h2, nullptr, K, L.K_pad, h1, h2, nullptr);
         break;
       }
       const uint64_t W32 = L.K_pad / 32;
@@ -439,6 +446,15 @@ bq_status bq_pack_weights(const bq_pack_desc* desc, const float* W, int32_t N, i
           k_svid_rows<<<blocks_for(N, 128), 128, 0, s>>>(W, N, K, L.K_pad, pl[o], gp[o], hp[o], pl[q], hp[q], gp[q]);
           k_svid_cols<<<blocks_for(K, 128), 128, 0, s>>>(W, N, K, L.K_pad, pl[o], gp[o], hp[o], gp[q], hp[q]);
         }
+      break;
+    }
+    case BQ_FMT_RABIT3: {  // h first: the recursion reads the packed h_p
+      uint32_t* planes = reinterpret_cast<uint32_t*>(P + L.off_tiles);
+      float* g = reinterpret_cast<float*>(P + L.off_rows);
+      float* h = reinterpret_cast<float*>(P + L.off_aux);
+      k_rabit_h<<<blocks_for(L.K_pad, 256), 256, 0, s>>>(desc->h2, desc->h3, K, L.K_pad, h, h + L.K_pad,
+                                                        h + 2 * size_t(L.K_pad));
+      k_rabit_pack_paths<3><<<N, 256, 0, s>>>(W, h, L.N_pad, K, L.K_pad, planes, g);
       break;
     }
     case BQ_FMT_BVSR4: {
@@ -526,9 +542,8 @@ bq_status bq_quantize_act(const bq_layer* layer, const void* x_bf16, int32_t M, 
   a.off_codes = A.off_codes; a.off_tok = A.off_tok; a.off_gsum = A.off_gsum; a.off_u = A.off_u; a.off_xt = A.off_xt;
   a.total = A.total;
   a.lora_A = reinterpret_cast<const uint16_t*>(P + L.off_aux);
-  a.h1 = reinterpret_cast<const float*>(P + L.off_aux);
-  a.h2 = reinterpret_cast<const float*>(P + L.off_aux2);
-  if (L.fmt == BQ_FMT_RABIT2) {
+  a.h = reinterpret_cast<const float*>(P + L.off_aux);
+  if (rabit_paths(L.fmt)) {
     return launch_pdl(k_act_rabit, dim3(blocks_for(L.K_pad, 256), M), dim3(256), 0, s, a) == cudaSuccess
                ? BQ_OK : BQ_ERR_CUDA;
   }
@@ -555,7 +570,7 @@ bq_status bq_gemm(const bq_layer* layer, const void* act, int32_t M, float* y, i
   if (M == 0) return BQ_OK;
   if (!act || !aligned(act, 256) || !y || !aligned(y, 4) || (acc_dbg && !aligned(acc_dbg, 8)))
     return BQ_ERR_INVALID_ARG;
-  if (L.fmt == BQ_FMT_RABIT2 && acc_dbg) return BQ_ERR_UNSUPPORTED;
+  if (rabit_paths(L.fmt) && acc_dbg) return BQ_ERR_UNSUPPORTED;
   const uint8_t* Ab = static_cast<const uint8_t*>(act);
   const ActLayout A = make_act_layout(L, M);
   LayerArgs g = layer_args(L, layer->packed, M, y, acc_dbg);
@@ -587,7 +602,7 @@ bq_status bq_linear(const bq_layer* layer, const void* x_bf16, int32_t M, float*
   if (M == 0) return BQ_OK;
   if (!x_bf16 || !aligned(x_bf16, 16) || !y || !aligned(y, 4) || (acc_dbg && !aligned(acc_dbg, 8)))
     return BQ_ERR_INVALID_ARG;
-  if (L.fmt == BQ_FMT_RABIT2 && acc_dbg) return BQ_ERR_UNSUPPORTED;
+  if (rabit_paths(L.fmt) && acc_dbg) return BQ_ERR_UNSUPPORTED;
   const uint64_t need = linear_workspace(L, M);
   if (need > 0 && (!workspace || !aligned(workspace, 256))) return BQ_ERR_INVALID_ARG;
   if (workspace_bytes < need) return BQ_ERR_SIZE;
@@ -689,7 +704,7 @@ bq_status bq_linear_plan(const bq_layer* layer, int32_t M, int32_t fused, bq_pla
   if (st != BQ_OK) return st;
   if (!info) return BQ_ERR_INVALID_ARG;
   if (M < 1 || M > BQ_MAX_M) return BQ_ERR_SIZE;
-  if (L.fmt == BQ_FMT_RABIT2) return BQ_ERR_UNSUPPORTED;
+  if (rabit_paths(L.fmt)) return BQ_ERR_UNSUPPORTED;
   LayerArgs g{};
   if (!plan_layer(L, M, fused != 0, &g)) return BQ_ERR_UNSUPPORTED;
   info->tokens_per_cta = g.tpc;

@@ -16,8 +16,7 @@ struct ActArgs {
   int M, K, K_pad, KT, a_bits, rank, fmt, tiles_per_slice;
   uint64_t off_codes, off_tok, off_gsum, off_u, off_xt, total;
   const uint16_t* lora_A;   // ternary: bf16 [K_pad][r]
-  const float* h1;          // RaBiT: [K_pad]
-  const float* h2;
+  const float* h;           // RaBiT: h_p at h + p K_pad, p < rabit_paths(fmt)
 };
 
 __device__ __forceinline__ void act_write_header(const ActArgs& a) {
@@ -174,7 +173,7 @@ __global__ void __launch_bounds__(256) k_act_quant(ActArgs a) {
     }
   }
 }
-// RaBiT: xt_p = h_p * x in float32, no quantization.
+// RaBiT: xt_p = h_p * x in float32 for each path p, no quantization.
 __global__ void k_act_rabit(ActArgs a) {
   const int m = blockIdx.y;
   pdl_trigger();
@@ -184,8 +183,9 @@ __global__ void k_act_rabit(ActArgs a) {
   if (k >= a.K_pad) return;
   float* xt = reinterpret_cast<float*>(a.act + a.off_xt);
   const float x = k < a.K ? bf16_bits_to_float(a.x[size_t(m) * a.K + k]) : 0.f;
-  xt[size_t(m) * a.K_pad + k] = k < a.K ? __fmul_rn(a.h1[k], x) : 0.f;
-  xt[(size_t(a.M) + m) * a.K_pad + k] = k < a.K ? __fmul_rn(a.h2[k], x) : 0.f;
+  const int P = rabit_paths(a.fmt);
+  for (int p = 0; p < P; p++)
+    xt[(size_t(p) * a.M + m) * a.K_pad + k] = k < a.K ? __fmul_rn(a.h[size_t(p) * a.K_pad + k], x) : 0.f;
 }
 
 }  // namespace bqi

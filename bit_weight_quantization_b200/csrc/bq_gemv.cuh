@@ -145,9 +145,8 @@ struct LayerArgs {
   const uint16_t* lora_bt;  // ternary B^T bf16 [N_pad][r]
   const float* bvsr_table;  // [256][8]
   const uint32_t* rabit_planes;
-  const float* rabit_g;     // g1 [N_pad], g2 [N_pad]
-  const float* rabit_h1;    // [K_pad]
-  const float* rabit_h2;
+  const float* rabit_g;     // g_p [P][N_pad]
+  const float* rabit_h;     // h_p [P][K_pad]
   // activations: x (fused) or the act buffer
   const uint16_t* x;
   const uint32_t* act_hdr;
@@ -1011,11 +1010,12 @@ __global__ void __launch_bounds__(256) k_lora_partial(const uint16_t* __restrict
 }
 
 // ---------------------------------------------------------------------------
-// RaBiT: fp32 sign-apply, y = g1 sum_k (-1)^B1 h1 x + g2 sum_k (-1)^B2 h2 x; the
+// RaBiT with P paths: fp32 sign-apply, y = sum_p g_p sum_k (-1)^B_p h_p x; the
 // sign bit of h_p x is flipped by XOR with the plane bit. One warp per row,
 // lane l takes k = 32w + l. Fused: reads x and h; else the act buffer's h_p x.
+// The scales combine from the last path down: y = fma(g1, acc1, fma(g2, acc2, g3 acc3)).
 // ---------------------------------------------------------------------------
-template <int NW, bool FUSED>
+template <int NW, bool FUSED, int P>
 __global__ void __launch_bounds__(NW * 32) k_rabit(LayerArgs a) {
   __shared__ int bad;
   pdl_trigger();
@@ -1034,29 +1034,33 @@ __global__ void __launch_bounds__(NW * 32) k_rabit(LayerArgs a) {
   const int row = blockIdx.x * NW + warp;
   if (row >= a.N) return;
   const int W32 = a.K_pad / 32;
-  const uint32_t* p1 = a.rabit_planes + size_t(row) * W32;
-  const uint32_t* p2 = a.rabit_planes + (size_t(a.N_pad) + row) * W32;
+  const uint32_t* pl = a.rabit_planes + size_t(row) * W32;   // path p: + p N_pad W32
+  const size_t pstride = size_t(a.N_pad) * W32;
   for (int m = 0; m < a.M; m++) {
-    float acc1 = 0.f, acc2 = 0.f;
+    float acc[P];
+#pragma unroll
+    for (int p = 0; p < P; p++) acc[p] = 0.f;
 #pragma unroll 8
     for (int wd = 0; wd < W32; wd++) {
-      const uint32_t b1 = __ldg(p1 + wd), b2 = __ldg(p2 + wd);
       const int k = wd * 32 + lane;
-      float x1, x2;
-      if (FUSED) {
-        const float xv = k < a.K ? bf16_bits_to_float(a.x[size_t(m) * a.K + k]) : 0.f;
-        x1 = __fmul_rn(__ldg(a.rabit_h1 + k), xv);
-        x2 = __fmul_rn(__ldg(a.rabit_h2 + k), xv);
-      } else {
-        x1 = __ldg(a.act_xt + size_t(m) * a.K_pad + k);
-        x2 = __ldg(a.act_xt + (size_t(a.M) + m) * a.K_pad + k);
+      float xv = 0.f;
+      if (FUSED) xv = k < a.K ? bf16_bits_to_float(a.x[size_t(m) * a.K + k]) : 0.f;
+#pragma unroll
+      for (int p = 0; p < P; p++) {
+        const uint32_t b = __ldg(pl + p * pstride + wd);
+        const float xp = FUSED ? __fmul_rn(__ldg(a.rabit_h + size_t(p) * a.K_pad + k), xv)
+                               : __ldg(a.act_xt + (size_t(p) * a.M + m) * a.K_pad + k);
+        acc[p] += __uint_as_float(__float_as_uint(xp) ^ (((b >> lane) & 1u) << 31));
       }
-      acc1 += __uint_as_float(__float_as_uint(x1) ^ (((b1 >> lane) & 1u) << 31));
-      acc2 += __uint_as_float(__float_as_uint(x2) ^ (((b2 >> lane) & 1u) << 31));
     }
-    acc1 = warp_sum(acc1);
-    acc2 = warp_sum(acc2);
-    if (lane == 0) a.y[size_t(m) * a.N + row] = fmaf(a.rabit_g[row], acc1, a.rabit_g[a.N_pad + row] * acc2);
+#pragma unroll
+    for (int p = 0; p < P; p++) acc[p] = warp_sum(acc[p]);
+    if (lane == 0) {
+      float yv = a.rabit_g[size_t(P - 1) * a.N_pad + row] * acc[P - 1];
+#pragma unroll
+      for (int p = P - 2; p >= 0; p--) yv = fmaf(a.rabit_g[size_t(p) * a.N_pad + row], acc[p], yv);
+      a.y[size_t(m) * a.N + row] = yv;
+    }
   }
 }
 

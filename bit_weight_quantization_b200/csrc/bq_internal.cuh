@@ -51,6 +51,11 @@ struct ActLayout {
 
 inline uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
 
+// Paths of a RaBiT format (0 for the tiled formats).
+__host__ __device__ inline int rabit_paths(int fmt) {
+  return fmt == BQ_FMT_RABIT2 ? 2 : fmt == BQ_FMT_RABIT3 ? 3 : 0;
+}
+
 // Returns false for an unknown format or bit width.
 inline bool make_pk_layout(int fmt, int N, int K, int w_bits, int a_bits, int rank, float alpha,
                            PkLayout* L) {
@@ -67,6 +72,13 @@ inline bool make_pk_layout(int fmt, int N, int K, int w_bits, int a_bits, int ra
       l.tile_bytes = 0;
       tiles = 2ull * l.N_pad * (l.K_pad / 8);
       rows = 2ull * l.N_pad * 4; aux = uint64_t(l.K_pad) * 4; aux2 = uint64_t(l.K_pad) * 4;
+      break;
+    case BQ_FMT_RABIT3:  // h2, h3 follow h1 (4 K_pad is a multiple of 256: no gaps)
+      l.w_bits = 3; l.a_bits = 16; l.nstreams = 3;
+      for (int s = 0; s < 3; s++) { l.field[s] = 1; l.shift[s] = s; }
+      l.tile_bytes = 0;
+      tiles = 3ull * l.N_pad * (l.K_pad / 8);
+      rows = 3ull * l.N_pad * 4; aux = uint64_t(l.K_pad) * 4; aux2 = 2ull * l.K_pad * 4;
       break;
     case BQ_FMT_BITNET_W1A8:
       l.w_bits = 1; l.a_bits = 8; l.nstreams = 1; l.field[0] = 1; l.tile_bytes = 512;
@@ -98,7 +110,7 @@ inline bool make_pk_layout(int fmt, int N, int K, int w_bits, int a_bits, int ra
     default:
       return false;
   }
-  if (fmt != BQ_FMT_RABIT2) tiles = uint64_t(l.RB) * l.KT * l.tile_bytes;
+  if (!rabit_paths(fmt)) tiles = uint64_t(l.RB) * l.KT * l.tile_bytes;
   l.off_tiles = 256;
   l.off_rows = align256(l.off_tiles + tiles);
   l.off_aux = align256(l.off_rows + rows);
@@ -112,11 +124,11 @@ inline ActLayout make_act_layout(const PkLayout& L, int M) {
   ActLayout a{};
   a.fmt = L.fmt; a.M = M; a.K = L.K; a.K_pad = L.K_pad; a.KT = L.KT; a.a_bits = L.a_bits;
   a.rank = L.fmt == BQ_FMT_TERNARY_A8 ? L.rank : 0;
-  uint64_t codes = L.fmt == BQ_FMT_RABIT2 ? 0 : uint64_t(M) * L.KT * 256;
+  uint64_t codes = rabit_paths(L.fmt) ? 0 : uint64_t(M) * L.KT * 256;
   uint64_t tok = uint64_t(M) * 16;
   uint64_t gsum = L.fmt == BQ_FMT_BVSR4 ? uint64_t(M) * (L.K_pad / 32) * 4 : 0;
   uint64_t u = uint64_t(L.KT) * M * a.rank * 4;   // LoRA partials [KT][M][r]
-  uint64_t xt = L.fmt == BQ_FMT_RABIT2 ? 2ull * M * L.K_pad * 4 : 0;
+  uint64_t xt = uint64_t(rabit_paths(L.fmt)) * M * L.K_pad * 4;
   a.off_codes = 256;
   a.off_tok = align256(a.off_codes + codes);
   a.off_gsum = align256(a.off_tok + tok);

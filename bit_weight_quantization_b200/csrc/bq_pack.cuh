@@ -211,12 +211,53 @@ __global__ void k_rabit_pack(const float* __restrict__ W, int N_pad, int K, int 
   }
 }
 
-__global__ void k_rabit_h(const float* __restrict__ h2, int K, int K_pad, float* __restrict__ h1_out,
-                          float* __restrict__ h2_out) {
+// h1 = 1, h2 (and h3 for three paths, when h3 is not null) copied; 0 on the padding columns.
+__global__ void k_rabit_h(const float* __restrict__ h2, const float* __restrict__ h3, int K, int K_pad,
+                          float* __restrict__ h1_out, float* __restrict__ h2_out, float* __restrict__ h3_out) {
   int k = blockIdx.x * blockDim.x + threadIdx.x;
   if (k >= K_pad) return;
   h1_out[k] = k < K ? 1.f : 0.f;
   h2_out[k] = k < K ? h2[k] : 0.f;
+  if (h3) h3_out[k] = k < K ? h3[k] : 0.f;
+}
+
+// RaBiT with P paths: R_0 = W; path p takes B_p = sign(R_{p-1}) and g_p = mean_k |R_{p-1}|
+// (float64 sum, stored float32), then R_p = R_{p-1} - g_p B_p h_p in float64 from the stored
+// g_p and h_p (their float64 product is exact). One block per row n < N; pass p replays the
+// earlier paths from W, so no residual is stored. h: the packed h_p [P][K_pad] (h1 = 1).
+template <int P>
+__global__ void k_rabit_pack_paths(const float* __restrict__ W, const float* __restrict__ h, int N_pad, int K,
+                                   int K_pad, uint32_t* __restrict__ planes, float* __restrict__ g) {
+  __shared__ double sh[32];
+  __shared__ float gs[P];
+  const int n = blockIdx.x;
+  const float* w = W + size_t(n) * K;
+  const int W32 = K_pad / 32;
+  for (int p = 0; p < P; p++) {
+    double s = 0.0;
+    for (int wd = threadIdx.x; wd < W32; wd += blockDim.x) {
+      uint32_t bits = 0;
+      for (int j = 0; j < 32; j++) {
+        const int k = wd * 32 + j;
+        if (k >= K) break;
+        double r = double(w[k]);
+        for (int q = 0; q < p; q++) {
+          const double gh = __dmul_rn(double(gs[q]), double(h[size_t(q) * K_pad + k]));
+          r = __dsub_rn(r, r >= 0.0 ? gh : -gh);
+        }
+        s = __dadd_rn(s, fabs(r));
+        bits |= uint32_t(!(r >= 0.0)) << j;
+      }
+      planes[(size_t(p) * N_pad + n) * W32 + wd] = bits;
+    }
+    s = block_sum(s, sh);
+    if (threadIdx.x == 0) {
+      const float gp = __double2float_rn(__ddiv_rn(s, double(K)));
+      gs[p] = gp;
+      g[size_t(p) * N_pad + n] = gp;
+    }
+    __syncthreads();
+  }
 }
 
 // ---------------------------------------------------------------------------

@@ -17,6 +17,7 @@ import numpy as np
 # tensor ids: one independent stream per tensor role
 TID_W, TID_X, TID_H2, TID_LORA_A, TID_LORA_B, TID_W_OUTLIER, TID_X_CHANNEL = 1, 2, 3, 4, 5, 6, 7
 TID_COMP_A, TID_COMP_B = 8, 9
+TID_H3 = 10
 
 
 def rng(seed: int, tensor_id: int) -> np.random.Generator:
@@ -82,6 +83,7 @@ def compensation_vectors(N: int, K: int, seed: int = 0, std: float = 0.1):
 # ---------------------------------------------------------------------------
 WORKLOADS = {
     "rabit": dict(shapes=[(256, 512)], Ms=[1], w_std=0.02, h2=(0.5, 1.5)),
+    "rabit3": dict(shapes=[(256, 512)], Ms=[1], w_std=0.02, h2=(0.5, 1.5), h3=(0.5, 1.5)),
     "bitnet": dict(shapes=[(4096, 4096), (11008, 4096), (4096, 11008)], Ms=[1], w_std=0.02),
     "ternary": dict(shapes=[(2048, 2048)], Ms=[1, 4, 16], w_std=0.02, lora_rank=32,
                     lora_alpha=0.1, a_std=0.02, b_std=0.01),
@@ -104,9 +106,12 @@ def layer_inputs(fmt: str, N: int, K: int, M: int, seed: int = 0, lora_rank: int
     else:
         out["W"] = weights(N, K, seed, wl["w_std"])
         out["x"] = activations(M, K, seed, 1.0)
-    if fmt == "rabit":
+    if fmt in ("rabit", "rabit3"):
         lo, hi = wl["h2"]
         out["h2"] = uniform(K, lo, hi, seed, TID_H2)
+    if fmt == "rabit3":
+        lo, hi = wl["h3"]
+        out["h3"] = uniform(K, lo, hi, seed, TID_H3)
     if fmt == "ternary":
         out["lora_A"] = gaussian((K, lora_rank), wl["a_std"], seed, TID_LORA_A)
         out["lora_B"] = gaussian((lora_rank, N), wl["b_std"], seed, TID_LORA_B)

@@ -1,11 +1,14 @@
 /*
  * bq.h -- C ABI of the bit-plane quantized linear layer for NVIDIA B200 (sm_100a).
  *
- * One computation, y = sum_k scales (.) (B_k . x), for five weight formats
+ * One computation, y = sum_k scales (.) (B_k . x), for five weight formats (RaBiT in a
+ * two-path and a three-path variant)
  * whose weights are stored as binary planes or bitvectors B_k:
  *
  *   BQ_FMT_RABIT2       RaBiT two-path residual binarization, W_hat = g1 B1 h1 + g2 B2 h2
  *                       ("RaBiT框架" page, §2.1 equation and §2.2 forward()).
+ *   BQ_FMT_RABIT3       the same residual recursion with a third path, g3 B3 h3 (the
+ *                       3-bit, three-path extension the "RaBiT框架" page names in §6).
  *   BQ_FMT_BITNET_W1A8  BitNet sign weights alpha*sign(W), alpha = mean|W| per tensor
  *                       ("1-bit LLM的端侧推理革命" page, §2.1-§2.3).
  *   BQ_FMT_TERNARY_A8   1.58-bit absmean ternary weights packed 2 bits/weight, with the
@@ -67,9 +70,11 @@
  *   8:[8], shift = bit offset in the code). BVSR: 4 x f=1, stream i = bitvector plane i,
  *   and each BVSR tile ends with 128 bytes of set indices: byte 2048 + 8g + j is the set of
  *   row 16rb + g, vector 8kt + j (a vector is 32 contiguous k), so tile_bytes = 2176.
- * RaBiT (format 1) is not tiled: bit j of uint32 off_tiles + 4((p*N_pad + n)(K_pad/32) + w)
- *   is the sign of path p (0,1), row n, k = 32w + j (1 <=> -1).
- * Sections: RaBiT rows = g1[N_pad], g2[N_pad] f32; aux = h1[K_pad], aux2 = h2[K_pad] f32.
+ * RaBiT (formats 1 and 6, P = 2 and 3 paths) is not tiled: bit j of uint32
+ *   off_tiles + 4((p*N_pad + n)(K_pad/32) + w) is the sign of path p (0..P-1), row n,
+ *   k = 32w + j (1 <=> -1).
+ * Sections: RaBiT rows = g_p f32 [P][N_pad]; aux = h1[K_pad], aux2 = h2[K_pad] (format 6:
+ *   h2, h3 [2][K_pad]) f32, so h_p (p = 0..P-1) starts at off_aux + 4 p K_pad.
  *   Ternary aux = A bf16 [K_pad][r], aux2 = B^T bf16 [N_pad][r].
  *   ABQ rows = Delta_w f32 [N_pad], z_w i32 [N_pad], S_w = sum_k q_w i32 [N_pad].
  *   BVSR aux = coefficient table f32 [256][8] (c0 c1 c2 c3 o; then derived kernel constants:
@@ -88,7 +93,7 @@
  * gsum (BVSR): i32 [M][K_pad/32], sum of q over each 32-element vector.
  * u (ternary): f32 [K_pad/256][M][r] partial dot products of the unquantized bf16 x with A
  *   over each 256-k tile (each in k order); the layer forms SiLU(sum over tiles).
- * xt (RaBiT): f32 [2][M][K_pad] = h_p * x (no activation quantization).
+ * xt (RaBiT): f32 [P][M][K_pad] = h_p * x (no activation quantization).
  */
 #ifndef BQ_H
 #define BQ_H
@@ -115,7 +120,8 @@ typedef enum {
   BQ_FMT_BITNET_W1A8 = 2,
   BQ_FMT_TERNARY_A8 = 3,
   BQ_FMT_ABQ = 4,
-  BQ_FMT_BVSR4 = 5
+  BQ_FMT_BVSR4 = 5,
+  BQ_FMT_RABIT3 = 6
 } bq_format;
 
 /* Limits: 1 <= N <= 1<<20, 128 <= K <= 1<<16 with K % 128 == 0, 1 <= M <= 64 (M = 0 is
@@ -157,6 +163,9 @@ typedef struct {
                            those of that matrix (with abq_bit_balance too: its W2* codes). The
                            layer then computes y = (W + a b^T)_hat x. Both NULL: off. One of
                            them NULL, or either set for another format: BQ_ERR_INVALID_ARG. */
+  const float* h3;      /* RaBiT three paths (format 6): device f32 [K], the third path's input
+                           scale (h1 = 1; h2 is required too). Format 6 runs the residual
+                           recursion only (rabit_svid_rounds = 0). NULL for every other format. */
 } bq_pack_desc;
 
 /* Host-side description of a packed layer; filled by bq_pack_weights or

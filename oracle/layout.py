@@ -13,7 +13,7 @@ sections at the header's offsets.
   word  field                      word  field
   0     magic 0x4B505142 'BQPK'    18    tile_bytes
   1     version (1)                19    lora_rank
-  2     format (1..5)              20    lora_alpha (f32)
+  2     format (1..6)              20    lora_alpha (f32)
   3     N                          21    tensor_scale (f32): BitNet alpha, ternary gamma_W
   4     K                          22-23 total_bytes (u64)
   5     N_pad (multiple of 16)     24-25 off_tiles (u64)
@@ -36,9 +36,10 @@ the f-bit field j (bits f*j .. f*j+f-1) of byte b holds the weight at
 BVSR tiles (4 one-bit planes of 512 B) end with 128 bytes of set indices: byte
 2048 + 8*g + j holds the set of row 16*rb + g, vector 8*kt + j (32 elements each).
 
-RaBiT (format 1) is not tiled: plane p (0,1) word w of row n is the uint32 at
-off_tiles + 4*((p*N_pad + n)*(K_pad/32) + w), bit j <-> k = 32w + j; a set bit
-means sign -1.
+RaBiT (format 1: P = 2 paths; format 6: P = 3) is not tiled: plane p (0..P-1)
+word w of row n is the uint32 at off_tiles + 4*((p*N_pad + n)*(K_pad/32) + w),
+bit j <-> k = 32w + j; a set bit means sign -1. Rows hold g_p as f32 [P][N_pad];
+h_1 sits at off_aux and h_2 (.. h_P) at off_aux2, K_pad f32 each, one after another.
 """
 from __future__ import annotations
 
@@ -46,8 +47,8 @@ import numpy as np
 
 PK_MAGIC = 0x4B505142
 ACT_MAGIC = 0x43415142
-FMT_RABIT, FMT_BITNET, FMT_TERNARY, FMT_ABQ, FMT_BVSR = 1, 2, 3, 4, 5
-FMT_NAMES = {1: "rabit", 2: "bitnet", 3: "ternary", 4: "abq", 5: "bvsr"}
+FMT_RABIT, FMT_BITNET, FMT_TERNARY, FMT_ABQ, FMT_BVSR, FMT_RABIT3 = 1, 2, 3, 4, 5, 6
+FMT_NAMES = {1: "rabit", 2: "bitnet", 3: "ternary", 4: "abq", 5: "bvsr", 6: "rabit3"}
 
 
 def _u32(buf: bytes, word: int) -> int:
@@ -143,6 +144,16 @@ def read_packed(buf: bytes, row_blocks=None) -> dict:
         out["g1"], out["g2"] = g[:N].copy(), g[N_pad:N_pad + N].copy()
         out["h1"] = np.frombuffer(buf, dtype="<f4", count=K, offset=h["off_aux"]).copy()
         out["h2"] = np.frombuffer(buf, dtype="<f4", count=K, offset=h["off_aux2"]).copy()
+    elif fmt == FMT_RABIT3:   # the rabit_pack_paths shape: B [P,N,K], g [P,N], h [P,K]
+        P, W32 = 3, K_pad // 32
+        raw = np.frombuffer(buf, dtype="<u4", count=P * N_pad * W32, offset=h["off_tiles"])
+        bits = ((raw.reshape(P, N_pad, W32)[..., None] >> np.arange(32, dtype=np.uint32)) & 1)
+        out["B"] = np.where(bits.reshape(P, N_pad, K_pad)[:, :N, :K] == 1, -1, 1).astype(np.int8)
+        g = np.frombuffer(buf, dtype="<f4", count=P * N_pad, offset=h["off_rows"]).reshape(P, N_pad)
+        out["g"] = g[:, :N].copy()
+        h1 = np.frombuffer(buf, dtype="<f4", count=K, offset=h["off_aux"])
+        h23 = np.frombuffer(buf, dtype="<f4", count=(P - 1) * K_pad, offset=h["off_aux2"]).reshape(P - 1, K_pad)
+        out["h"] = np.concatenate([h1[None, :], h23[:, :K]]).copy()
     elif fmt == FMT_BITNET:
         neg = read_stream_codes(buf, h, 0, rb)
         out["B"] = np.where(neg == 1, -1, 1).astype(np.int8)
@@ -222,9 +233,11 @@ def read_act(buf: bytes) -> dict:
              total_bytes=_u64(buf, 8), off_codes=_u64(buf, 10), off_tok=_u64(buf, 12),
              off_gsum=_u64(buf, 14), off_u=_u64(buf, 16), off_xt=_u64(buf, 18))
     KT = K_pad // 256
-    if fmt == FMT_RABIT:
-        xt = np.frombuffer(buf, dtype="<f4", count=2 * M * K_pad, offset=a["off_xt"])
-        a["xt"] = xt.reshape(2, M, K_pad)[:, :, :K].copy()
+    if fmt in (FMT_RABIT, FMT_RABIT3):
+        P = 2 if fmt == FMT_RABIT else 3
+        xt = np.frombuffer(buf, dtype="<f4", count=P * M * K_pad, offset=a["off_xt"])
+        a["xt"] = xt.reshape(P, M, K_pad)[:, :, :K].copy()
+        a["xt_pad"] = xt.reshape(P, M, K_pad)[:, :, K:].copy()
         return a
     dt = np.uint8 if fmt == FMT_ABQ else np.int8
     raw = np.frombuffer(buf, dtype=dt, count=M * KT * 256, offset=a["off_codes"]).reshape(M, KT, 4, 8, 2, 4)

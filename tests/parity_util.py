@@ -58,8 +58,10 @@ class GpuLayer:
         self.inp = inp
         self.W = to_dev_f32(inp["W"])
         kw = {}
-        if fmt == "rabit":
+        if fmt in ("rabit", "rabit3"):
             kw["h2"] = to_dev_f32(inp["h2"])
+        if fmt == "rabit3":
+            kw["h3"] = to_dev_f32(inp["h3"])
         if fmt == "ternary":
             kw.update(lora_rank=lora_rank, lora_alpha=lora_alpha,
                       lora_A=to_dev_f32(inp["lora_A"]), lora_B=to_dev_f32(inp["lora_B"]))
@@ -69,7 +71,7 @@ class GpuLayer:
         self.x = to_dev_bf16(inp["x"])
         self.y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
         self.acc = None
-        if fmt != "rabit":
+        if fmt not in ("rabit", "rabit3"):
             self.acc = torch.full((M, N), -(1 << 62), dtype=torch.int64, device="cuda")
         self.ql.forward(self.x, self.y, self.acc)
         # the fused path (bq_linear) on the same inputs
@@ -97,6 +99,8 @@ def oracle_pack(fmt, inp, w_bits=0, lora_alpha=0.1, rows=None):
     W = inp["W"]
     if fmt == "rabit":
         return O.rabit_pack(W, inp["h2"])
+    if fmt == "rabit3":
+        return O.rabit_pack_paths(W, [np.ones(W.shape[1], np.float32), inp["h2"], inp["h3"]])
     if fmt == "bitnet":
         p = O.bitnet_pack(W)
         if rows is not None:
@@ -119,6 +123,8 @@ def oracle_layer(fmt, p, x, a_bits=0):
     """Reference layer on the library's own decoded codes (dict from the reader)."""
     if fmt == "rabit":
         return O.rabit_layer(p, x)
+    if fmt == "rabit3":
+        return dict(y=x.astype(np.float64) @ O.rabit_weight_paths(p).T)
     if fmt == "bitnet":
         return O.bitnet_layer(p, x)
     if fmt == "ternary":
@@ -137,10 +143,13 @@ def check_act(gl: GpuLayer):
     a = L.read_act(gl.act)
     x = gl.inp["x"]
     assert a["M"] == gl.M and a["K"] == gl.K
-    if gl.fmt == "rabit":
-        h2 = gl.inp["h2"]
+    if gl.fmt in ("rabit", "rabit3"):
+        hs = [gl.inp["h2"]] + ([gl.inp["h3"]] if gl.fmt == "rabit3" else [])
+        assert a["xt"].shape[0] == 1 + len(hs)
         assert np.array_equal(a["xt"][0], x.astype(np.float32))
-        assert np.array_equal(a["xt"][1], (h2[None, :] * x).astype(np.float32))
+        for p, h in enumerate(hs, start=1):
+            assert np.array_equal(a["xt"][p], (h[None, :] * x).astype(np.float32))
+        assert np.all(a["xt_pad"] == 0)
         return
     if gl.fmt == "abq":
         Qx, dx, zx = O.quantize_rows_asym(x, gl.a_bits)

@@ -43,6 +43,9 @@ def test_status_strings_and_version():
     ("ternary", dict(lora_rank=32), 2048, 2048, 256 + 2048 * 2048 // 4 + 2048 * 32 * 2 * 2),
     ("abq", dict(w_bits=6, a_bits=6), 4096, 4096, 256 + 4096 * 4096 * 6 // 8 + 3 * 4096 * 4),
     ("bvsr", {}, 5120, 5120, 256 + 5120 * 5120 // 2 + 256 * 8 * 4 + 5120 * 5120 // 32),
+    # RaBiT: P sign planes, g [P][N], h [P][K] f32
+    ("rabit", {}, 256, 512, 256 + 2 * 256 * 512 // 8 + 2 * 256 * 4 + 2 * 512 * 4),
+    ("rabit3", {}, 256, 512, 256 + 3 * 256 * 512 // 8 + 3 * 256 * 4 + 3 * 512 * 4),
 ])
 def test_packed_bytes_match_layout(fmt, kw, N, K, expect):
     d = bq.make_desc(fmt, **kw)
@@ -108,7 +111,8 @@ def _host_header(fmt, N, K, **kw):
     N_pad, K_pad = -(-N // 16) * 16, -(-K // 256) * 256
     h = np.zeros(64, "<u4")
     h[0], h[1], h[2], h[3], h[4], h[5], h[6] = L.PK_MAGIC, 1, bq.FORMATS[fmt], N, K, N_pad, K_pad
-    fields = {"bitnet": [1], "ternary": [2], "bvsr": [1, 1, 1, 1]}.get(fmt)
+    fields = {"bitnet": [1], "ternary": [2], "bvsr": [1, 1, 1, 1], "rabit": [1, 1], "rabit3": [1, 1, 1]}.get(fmt)
+    P = len(fields) if fmt.startswith("rabit") else 0
     if fmt == "abq":
         w = kw["w_bits"]
         fields, rem = [], w
@@ -116,21 +120,21 @@ def _host_header(fmt, N, K, **kw):
             f = 8 if rem >= 8 else 4 if rem >= 4 else 2 if rem >= 2 else 1
             fields.append(f)
             rem -= f
-    h[7] = {"bitnet": 1, "ternary": 2, "bvsr": 4}.get(fmt, kw.get("w_bits", 0))
-    h[8] = kw.get("a_bits", 8)
+    h[7] = {"bitnet": 1, "ternary": 2, "bvsr": 4, "rabit": 2, "rabit3": 3}.get(fmt, kw.get("w_bits", 0))
+    h[8] = 16 if P else kw.get("a_bits", 8)
     h[9] = len(fields)
     sh = 0
     for i, f in enumerate(fields):
-        h[10 + i], h[14 + i] = f, (i if fmt == "bvsr" else sh)
+        h[10 + i], h[14 + i] = f, (i if fmt == "bvsr" or P else sh)
         sh += f
-    h[18] = 512 * sum(fields) + (128 if fmt == "bvsr" else 0)
+    h[18] = 0 if P else 512 * sum(fields) + (128 if fmt == "bvsr" else 0)
     h[19] = kw.get("lora_rank", 0)
-    tiles = (N_pad // 16) * (K_pad // 256) * h[18]
-    rows = 3 * N_pad * 4 if fmt == "abq" else 0
+    tiles = P * N_pad * K_pad // 8 if P else (N_pad // 16) * (K_pad // 256) * h[18]
+    rows = 3 * N_pad * 4 if fmt == "abq" else P * N_pad * 4
     a256 = lambda v: (v + 255) // 256 * 256
     off_rows = a256(256 + tiles)
-    aux = {"ternary": K_pad * h[19] * 2, "bvsr": 256 * 8 * 4}.get(fmt, 0)
-    aux2 = {"ternary": N_pad * h[19] * 2}.get(fmt, 0)
+    aux = K_pad * 4 if P else {"ternary": K_pad * h[19] * 2, "bvsr": 256 * 8 * 4}.get(fmt, 0)
+    aux2 = (P - 1) * K_pad * 4 if P else {"ternary": N_pad * h[19] * 2}.get(fmt, 0)
     off_aux = a256(off_rows + rows)
     off_aux2 = a256(off_aux + aux)
     for word, v in [(22, total), (24, 256), (26, off_rows), (28, off_aux), (30, off_aux2)]:
@@ -238,6 +242,33 @@ def test_compensation_descriptor_checks():
     assert bq.bq_packed_bytes(d, 64, 256) == bq.bq_packed_bytes(plain, 64, 256)   # same buffer
     for a, b in [(fake, None), (None, fake), (fake + 2, fake), (fake, fake + 1)]:
         d = bq.make_desc("abq", w_bits=4, a_bits=4, abq_comp_a=a, abq_comp_b=b)
+        assert bq.raw_status("bq_pack_weights", ctypes.byref(d), fake, 64, 256, fake, 1 << 30, None,
+                             ctypes.byref(bq.bq_layer())) == bq.BQ_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("fmt", ["rabit", "rabit3"])
+def test_rabit_host_header_and_act_bytes(fmt):
+    """The documented RaBiT layout validates; the act buffer holds P x M x K_pad f32 (h_p x);
+    the layer kernel of the tiled formats has no plan for it."""
+    P = 2 if fmt == "rabit" else 3
+    layer = bq.bq_packed_validate(_host_header(fmt, 300, 640).tobytes(), 1 << 20)
+    assert (layer.fmt, layer.N_pad, layer.K_pad, layer.w_bits) == (bq.FORMATS[fmt], 304, 768, P)
+    assert bq.bq_act_bytes(layer, 5) == 256 + 256 + P * 5 * 768 * 4   # header, token words, xt
+    with pytest.raises(bq.BQError) as e:
+        bq.bq_linear_plan(layer, 1)
+    assert e.value.status == bq.BQ_ERR_UNSUPPORTED
+
+
+def test_rabit3_descriptor_checks():
+    out = ctypes.c_size_t(0)
+    fake = 1 << 40
+    for d, st in [(bq.make_desc("rabit3"), bq.BQ_OK),
+                  (bq.make_desc("rabit3", rabit_svid_rounds=20), bq.BQ_ERR_INVALID_ARG),   # recursion only
+                  (bq.make_desc("rabit", h3=fake), bq.BQ_ERR_INVALID_ARG),                 # h3: format 6 only
+                  (bq.make_desc("bitnet", h3=fake), bq.BQ_ERR_INVALID_ARG)]:
+        assert bq.raw_status("bq_packed_bytes", ctypes.byref(d), 64, 256, ctypes.byref(out)) == st
+    for h2, h3 in [(fake, None), (None, fake), (fake, fake + 2)]:
+        d = bq.make_desc("rabit3", h2=h2, h3=h3)
         assert bq.raw_status("bq_pack_weights", ctypes.byref(d), fake, 64, 256, fake, 1 << 30, None,
                              ctypes.byref(bq.bq_layer())) == bq.BQ_ERR_INVALID_ARG
 

@@ -30,6 +30,15 @@ def _pack_parity(gl: GpuLayer, fmt, w_bits=0):
         assert np.array_equal(p["B2"][same_g1], ref["B2"][same_g1])
         assert np.all(ulp_diff(p["g2"], ref["g2"]) <= 1)
         assert np.array_equal(p["h2"], gl.inp["h2"]) and np.all(p["h1"] == 1)
+    elif fmt == "rabit3":
+        # path p's signs depend on the earlier g's: compare them where those agree exactly
+        assert np.all(p["h"][0] == 1) and np.array_equal(p["h"][1:], ref["h"][1:])
+        same = np.ones(gl.N, bool)
+        for q in range(3):
+            assert np.array_equal(p["B"][q][same], ref["B"][q][same])
+            assert np.all(ulp_diff(p["g"][q][same], ref["g"][q][same]) <= 1)
+            same &= p["g"][q] == ref["g"][q]
+        assert same.sum() >= gl.N - 2
     elif fmt == "bitnet":
         assert np.array_equal(p["B"], ref["B"])
         assert ulp_diff(p["alpha"], ref["alpha"]) <= 1
@@ -92,7 +101,36 @@ def test_max_tokens(fmt, N, K):
     _layer_parity(gl, p, fmt)
 
 
-@pytest.mark.parametrize("fmt", ["bitnet", "ternary", "bvsr", "rabit", "abq"])
+@pytest.mark.parametrize("N,K", SMALL)
+@pytest.mark.parametrize("M", [1, 3])
+def test_small_parity_rabit3(N, K, M):
+    """Three residual paths: pack (signs, g, h), act (h_p x) and layer (fused and not)."""
+    gl = GpuLayer("rabit3", N, K, M, seed=N + K + M)
+    p = _pack_parity(gl, "rabit3")
+    check_act(gl)
+    _layer_parity(gl, p, "rabit3")
+
+
+def test_full_rabit3():
+    gl = GpuLayer("rabit3", 256, 512, 1)
+    p = _pack_parity(gl, "rabit3")
+    check_act(gl)
+    _layer_parity(gl, p, "rabit3")
+
+
+def test_rabit3_constant_magnitude_rows():
+    """|W| = c on a row: R_1 = 0 exactly, so paths 2 and 3 get sign +1 and g = 0, and the
+    layer is W x itself."""
+    inp = I.layer_inputs("rabit3", 40, 384, 2, seed=9)
+    c = np.float32(0.03125)
+    inp["W"] = np.where(inp["W"] >= 0, c, -c).astype(np.float32)
+    gl = GpuLayer("rabit3", 40, 384, 2, inputs=inp)
+    p = gl.read()
+    assert np.all(p["g"][0] == c) and np.all(p["g"][1:] == 0) and np.all(p["B"][1:] == 1)
+    assert_y_close(gl.y_h, inp["x"].astype(np.float64) @ inp["W"].astype(np.float64).T, "rabit3 |W| = c")
+
+
+@pytest.mark.parametrize("fmt", ["bitnet", "ternary", "bvsr", "rabit", "rabit3", "abq"])
 def test_zero_activations(fmt):
     gl = GpuLayer(fmt, 40, 256, 2, w_bits=4, a_bits=4, nullify_x=True)
     check_act(gl)
@@ -122,7 +160,7 @@ def test_outlier_heavy_activations():
 
 
 def test_n_equals_one_and_min_k():
-    for fmt in ("bitnet", "ternary", "bvsr", "abq", "rabit"):
+    for fmt in ("bitnet", "ternary", "bvsr", "abq", "rabit", "rabit3"):
         gl = GpuLayer(fmt, 1, 128, 1, w_bits=2, a_bits=8)
         p = _pack_parity(gl, fmt, 2)
         _layer_parity(gl, p, fmt, 8)
