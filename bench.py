@@ -62,6 +62,12 @@ def layer_bytes(fmt: str, N: int, K: int, M: int = 1, w_bits: int = 1, a_bits: i
     return dict(gemv=gemv, act=actb, total=gemv + actb, fused=fused)
 
 
+def call_bytes(Ns, K: int) -> int:
+    """Algorithmic bytes of one fused BitNet call (bq_linear, or bq_linear_group over several
+    layers) at M = 1: each layer's weights, scale and y, and the shared input x read once."""
+    return sum(layer_bytes("bitnet", N, K)["fused"] for N in Ns) - (len(Ns) - 1) * 2 * K
+
+
 def reduce_max_over_ranks(values, dist=None, device=None) -> list:
     """Each value's maximum over the ranks (a job's device time is its slowest rank's). With no
     initialized process group, or one rank, the values come back unchanged."""
@@ -232,8 +238,7 @@ def build_stack(layers: int, seed: int, device, group: bool = True):
             K = shapes[names[0]][1]
             x = torch.randn(1, K, device=device, generator=gen).to(torch.bfloat16)
             ms = [members[n] for n in names]
-            nbytes = sum(layer_bytes("bitnet", m["N"], K)["fused"] for m in ms) - (len(ms) - 1) * 2 * K
-            calls.append(dict(members=ms, x=x, K=K, bytes=nbytes))
+            calls.append(dict(members=ms, x=x, K=K, bytes=call_bytes([m["N"] for m in ms], K)))
     torch.cuda.synchronize()
     return calls
 
