@@ -356,7 +356,7 @@ const char* bq_status_str(bq_status s) {
   }
 }
 
-int32_t bq_version(void) { return 1; }
+int32_t bq_version(void) { return BQ_ABI_VERSION; }
 
 bq_status bq_packed_bytes(const bq_pack_desc* desc, int32_t N, int32_t K, size_t* bytes) {
   if (!bytes) return BQ_ERR_INVALID_ARG;

@@ -177,6 +177,12 @@ typedef struct {
   const void* packed;
 } bq_layer;
 
+/* ABI version: bumped whenever a struct layout or a call's meaning changes. A caller
+ * compares bq_version() with the BQ_ABI_VERSION of the header it was built against.
+ * 2: bq_pack_desc gained abq_comp_a, abq_comp_b and h3; format 6 (BQ_FMT_RABIT3). The
+ * buffer formats keep their own version word (1): no existing layout changed. */
+#define BQ_ABI_VERSION 2
+
 const char* bq_status_str(bq_status s);
 int32_t bq_version(void);
 

@@ -4,6 +4,7 @@ the documented status before anything is enqueued."""
 import ctypes
 import os
 import re
+import shutil
 import subprocess
 
 import numpy as np
@@ -32,7 +33,32 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_status_strings_and_version():
-    assert bq.bq_version() == 1
+    assert bq.bq_version() == bq.BQ_ABI_VERSION == 2
+    hdr = open(os.path.join(ROOT, "include", "bq.h")).read()
+    assert re.search(r"#define BQ_ABI_VERSION (\d+)", hdr).group(1) == str(bq.BQ_ABI_VERSION)
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+def test_binding_structs_match_the_c_header(tmp_path):
+    """Every field offset and the size of each ctypes struct equal what a C compiler makes of
+    include/bq.h."""
+    structs = {"bq_pack_desc": bq.bq_pack_desc, "bq_layer": bq.bq_layer, "bq_plan_info": bq.bq_plan_info}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "bq.h"', "int main(void) {"]
+    for name, cls in structs.items():
+        lines.append(f'  printf("{name} size %zu\\n", sizeof({name}));')
+        for f, _ in cls._fields_:
+            lines.append(f'  printf("{name} {f} %zu\\n", offsetof({name}, {f}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "offsets.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "offsets"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)], check=True)
+    got = dict(l.rsplit(" ", 1) for l in subprocess.run([str(exe)], check=True, capture_output=True,
+                                                       text=True).stdout.splitlines())
+    for name, cls in structs.items():
+        assert int(got[f"{name} size"]) == ctypes.sizeof(cls), name
+        for f, _ in cls._fields_:
+            assert int(got[f"{name} {f}"]) == getattr(cls, f).offset, (name, f)
     assert bq.bq_status_str(0) == "ok"
     assert "device" in bq.bq_status_str(6)
 
