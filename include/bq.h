@@ -7,8 +7,9 @@
  *
  *   BQ_FMT_RABIT2       RaBiT two-path residual binarization, W_hat = g1 B1 h1 + g2 B2 h2
  *                       ("RaBiT框架" page, §2.1 equation and §2.2 forward()).
- *   BQ_FMT_RABIT3       the same residual recursion with a third path, g3 B3 h3 (the
- *                       3-bit, three-path extension the "RaBiT框架" page names in §6).
+ *   BQ_FMT_RABIT3       the same residual recursion with a third path, g3 B3 h3: the 3-bit
+ *                       extension the "RaBiT框架" page lists in §6, read as one more residual
+ *                       path (one bit per path).
  *   BQ_FMT_BITNET_W1A8  BitNet sign weights alpha*sign(W), alpha = mean|W| per tensor
  *                       ("1-bit LLM的端侧推理革命" page, §2.1-§2.3).
  *   BQ_FMT_TERNARY_A8   1.58-bit absmean ternary weights packed 2 bits/weight, with the

@@ -198,8 +198,8 @@ def rabit_recon_error(p, W) -> float:
 
 
 def rabit_pack_paths(W, hs) -> dict:
-    """The residual recursion of rabit_pack with P = len(hs) paths ([RaBiT] §2.1-2.2; §6 names
-    a 3-bit, three-path version as an extension): R_0 = W; path p takes B_p = sign(R_{p-1}),
+    """The residual recursion of rabit_pack with P = len(hs) paths ([RaBiT] §2.1-2.2; §6 lists
+    a 3-bit extension, read as a third path): R_0 = W; path p takes B_p = sign(R_{p-1}),
     g_p[n] = mean_k |R_{p-1}[n,:]| (float64 sum, stored float32) and the given h_p, then
     R_p = R_{p-1} - g_p B_p h_p in float64 from the stored g_p and h_p.
     hs: P float32 vectors [K] (hs[0] is 1 in the two-path reading). Returns B [P,N,K] int8,
