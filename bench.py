@@ -474,7 +474,8 @@ def config_list():
 def run_configs(args) -> None:
     """For each configuration: a CUDA graph over R distinct packed copies of the
     layer (R copies total >= 3x L2, capped at 512) of act + gemv; reports the
-    per-layer-call time, the GEMV launch time and the algorithmic GB/s."""
+    per-layer-call time, the GEMV launch time, the algorithmic GB/s, and one cold single call
+    (no graph, L2 flushed just before; the median of three)."""
     import torch
     from bit_weight_quantization_b200 import bq
     dev = torch.device("cuda", 0)
@@ -483,6 +484,7 @@ def run_configs(args) -> None:
     peak, peak_kind = measured_peaks()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)   # twice the L2 size
     sel = config_list()
     if args.only:
         sel = [c for c in sel if c[0] == args.only]
@@ -522,12 +524,24 @@ def run_configs(args) -> None:
                 torch.cuda.synchronize()
                 gl.append(statistics.mean(a_.elapsed_time(b_) for a_, b_ in tim) * 1e3)
             us_gemv = statistics.median(gl)
+            # one cold call: outside any graph, right after writing a buffer twice the L2 size
+            cold = []
+            for L in Ls[:3]:
+                flush.zero_()
+                c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                c0.record(stream)
+                layer_call(L, fused=fused)
+                c1.record(stream)
+                torch.cuda.synchronize()
+                cold.append(c0.elapsed_time(c1) * 1e3)
+            us_cold = statistics.median(cold)
         nb = lb["fused"] if fused else lb["total"]
         line = dict(fmt=fmt, N=N, K=K, M=M, w_bits=w, a_bits=a, path="bq_linear" if fused else "act+gemm",
                     copies=R, us_per_layer=us_layer,
                     gbs=nb / (us_layer * 1e-6) / 1e9, frac_of_peak=nb / (us_layer * 1e-6) / 1e9 / peak,
                     us_gemv=us_gemv, gemv_gbs=lb["gemv"] / (us_gemv * 1e-6) / 1e9,
-                    gemv_frac=lb["gemv"] / (us_gemv * 1e-6) / 1e9 / peak, bytes=nb, peak=peak,
+                    gemv_frac=lb["gemv"] / (us_gemv * 1e-6) / 1e9 / peak, us_cold_single=us_cold,
+                    bytes=nb, peak=peak,
                     peak_source=peak_kind)
         print(json.dumps(line), flush=True)
         del Ls, g, gi
