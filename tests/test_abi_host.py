@@ -351,3 +351,10 @@ def test_linear_plan_rejects():
         assert bq.raw_status("bq_linear_plan", ctypes.byref(layer), M, 1, ctypes.byref(info)) == st
     assert bq.raw_status("bq_linear_plan", ctypes.byref(layer), 1, 1, None) == bq.BQ_ERR_INVALID_ARG
     assert bq.raw_status("bq_linear_plan", None, 1, 1, ctypes.byref(info)) == bq.BQ_ERR_INVALID_ARG
+
+
+def test_rabit3_size_matches_the_hand_fixture():
+    """The library's buffer size for the hand-derived three-path fixture's shape is the fixture's."""
+    import json
+    c = json.load(open(os.path.join(ROOT, "tests", "golden", "layout_bits.json")))["rabit3_one_bit"]
+    assert bq.bq_packed_bytes(bq.make_desc("rabit3"), c["N"], c["K"]) == c["sizes"]["total"]

@@ -49,3 +49,24 @@ def test_act_single_code(golden):
     a = L.read_act(hdr.tobytes() + bytes(body))
     nz = np.nonzero(a["codes"][0])[0].tolist()
     assert nz == [c["k"]] and int(a["codes"][0, c["k"]]) == c["value"]
+
+
+def test_rabit3_single_bit_scale_and_h(golden):
+    """Three-path RaBiT: one sign bit of path 3, one g3 and one h3 at hand-derived byte offsets."""
+    c = golden("layout_bits.json")["rabit3_one_bit"]
+    z = c["sizes"]
+    N, K = c["N"], c["K"]
+    hdr = np.zeros(64, dtype="<u4")
+    hdr[0], hdr[1], hdr[2], hdr[3], hdr[4], hdr[5], hdr[6] = L.PK_MAGIC, 1, L.FMT_RABIT3, N, K, 32, 512
+    hdr[7], hdr[8], hdr[9] = 3, 16, 3
+    for word, v in [(22, z["total"]), (24, 256), (26, z["off_rows"]), (28, z["off_aux"]), (30, z["off_aux2"])]:
+        hdr[word] = v
+    buf = bytearray(z["total"])
+    buf[:256] = hdr.tobytes()
+    buf[c["sign_byte"]] = c["sign_value"]
+    buf[c["g_byte"]:c["g_byte"] + 4] = np.array([c["g"]], "<f4").tobytes()
+    buf[c["h_byte"]:c["h_byte"] + 4] = np.array([c["h"]], "<f4").tobytes()
+    p = L.read_packed(bytes(buf))
+    assert np.argwhere(p["B"] == -1).tolist() == [c["neg"]]
+    assert np.argwhere(p["g"] != 0).tolist() == [c["neg"][:2]] and p["g"][2, 17] == c["g"]
+    assert np.argwhere(p["h"] != 0).tolist() == [[2, c["neg"][2]]] and p["h"][2, 291] == c["h"]
