@@ -151,6 +151,17 @@ def test_ternary_m_values_and_lora():
         _layer_parity(gl, p, "ternary")
 
 
+@pytest.mark.parametrize("rank", [8, 64])
+@pytest.mark.parametrize("N,K,M", [(97, 640, 1), (40, 2560, 9)])
+def test_ternary_lora_ranks(rank, N, K, M):
+    """The smallest and the largest correction rank (steps of 8 up to 64), ragged shapes."""
+    gl = GpuLayer("ternary", N, K, M, seed=rank + N, lora_rank=rank)
+    p = _pack_parity(gl, "ternary")
+    assert p["A"].shape == (K, rank) and p["B"].shape == (rank, N)
+    check_act(gl)
+    _layer_parity(gl, p, "ternary")
+
+
 def test_outlier_heavy_activations():
     inp = I.layer_inputs("bitnet", 64, 512, 3, seed=4)
     inp["x"] = I.bf16_round(inp["x"] * np.where(np.arange(512) % 37 == 0, 300.0, 1.0)[None, :])
