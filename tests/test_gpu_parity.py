@@ -17,7 +17,7 @@ pytestmark = pytest.mark.gpu
 
 # ragged N and K; (40, 2560) leaves some warps without k-tiles, (24, 6144) streams in chunks
 SMALL = [(16, 256), (50, 384), (97, 640), (33, 128), (40, 2560), (24, 6144)]
-ABQ_WA = [(2, 8), (4, 4), (6, 6), (8, 8), (1, 3), (3, 5), (5, 2), (7, 7)]
+ABQ_WA = [(2, 8), (4, 4), (6, 6), (8, 8), (1, 3), (3, 5), (5, 2), (7, 7), (1, 1), (8, 1)]
 
 
 def _pack_parity(gl: GpuLayer, fmt, w_bits=0):
