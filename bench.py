@@ -140,6 +140,12 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=10)
+        return self.parse(out)
+
+    @staticmethod
+    def parse(out: str) -> dict:
+        """Median SM clock, max clock and the throttle reasons seen, from `nvidia-smi
+        --query-gpu=FIELDS --format=csv,noheader,nounits` lines."""
         sm, mx, reasons, pw = [], [], set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in out.strip().splitlines():

@@ -38,3 +38,30 @@ def test_decode_step_bytes_match_the_traffic_record():
     assert 815e6 < step < 817e6
     # the record's per-launch DRAM figure is the mean over the four call types
     assert rec["dram_bytes_per_launch"] == sum(rec["per_call_dram_bytes"].values()) / 4
+
+
+def test_clock_parse_reads_median_max_and_reasons():
+    """Canned nvidia-smi lines (csv, noheader, nounits): median SM clock, the max clock, and
+    each throttle reason that was Active in any sample; malformed or N/A lines are skipped."""
+    out = "\n".join([
+        "2026/12/02 10:00:00.000, 1965, 1965, 640.5, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/02 10:00:00.020, 1890, 1965, 990.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "2026/12/02 10:00:00.040, 1950, 1965, 870.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/02 10:00:00.060, [N/A], 1965, 870.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+    ])
+    c = bench.ClockSampler.parse(out)
+    assert (c["sm_mhz"], c["sm_max_mhz"], c["samples"]) == (1950.0, 1965.0, 3)
+    assert c["reasons"] == ["sw_power_cap"] and c["power_w_max"] == 990.1
+    hot = out.replace("Not Active, Not Active, Not Active, Active", "Active, Not Active, Active, Not Active")
+    assert bench.ClockSampler.parse(hot)["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    assert bench.ClockSampler.parse("")["samples"] == 0
+
+
+def test_traffic_record_is_dropped_when_the_kernel_source_changes(monkeypatch):
+    rec = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))["bitnet_fused_llama7b_grouped"]
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: rec["source_hash"])
+    assert bench.profile_traffic("bitnet_fused_llama7b_grouped") == rec["dram_bytes_per_launch"]
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)
+    assert bench.profile_traffic("bitnet_fused_llama7b_grouped") is None
+    assert bench.profile_traffic("no_such_kernel") is None
