@@ -560,3 +560,14 @@ def test_abq_compensation_balanced_antisymmetry():
     assert np.array_equal(m["Q"], 4 - p["Q"]) and np.array_equal(m["delta"], p["delta"])
     assert p["Q"].min() == 0 and p["Q"].max() == 4
     assert not np.array_equal(p["Q"], O.abq_pack_balanced(W)["Q"])
+
+
+def test_every_public_oracle_function_states_its_pins():
+    """Each public function of the oracle and its layout readers says what pins it (or that its
+    parity is unpinned), so an unpinned addition cannot slip in silently."""
+    import inspect
+    from oracle import layout as Lay
+    missing = [f"{m.__name__}.{n}" for m in (O, Lay) for n, f in inspect.getmembers(m, inspect.isfunction)
+               if not n.startswith("_") and f.__module__ == m.__name__
+               and "Pinned" not in (f.__doc__ or "") and "parity unpinned" not in (f.__doc__ or "").lower()]
+    assert not missing, missing
