@@ -358,3 +358,28 @@ def test_rabit3_size_matches_the_hand_fixture():
     import json
     c = json.load(open(os.path.join(ROOT, "tests", "golden", "layout_bits.json")))["rabit3_one_bit"]
     assert bq.bq_packed_bytes(bq.make_desc("rabit3"), c["N"], c["K"]) == c["sizes"]["total"]
+
+
+def test_product_path_never_imports_the_oracle():
+    """The package (binding, build, CUDA sources) never touches oracle/ or tests/; bench.py
+    imports the oracle only inside oracle_sample (its CPU-baseline and reference legs)."""
+    import ast
+    pkg = os.path.join(ROOT, "bit_weight_quantization_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, fn), encoding="utf-8").read()
+                assert not re.search(r"\b(import|from)\s+(oracle|tests)\b|#include\s+\"[^\"]*oracle", src), fn
+    tree = ast.parse(open(os.path.join(ROOT, "bench.py")).read())
+    parent = {c: n for n in ast.walk(tree) for c in ast.iter_child_nodes(n)}
+    found = 0
+    for node in ast.walk(tree):
+        if isinstance(node, (ast.Import, ast.ImportFrom)):
+            names = [node.module or ""] if isinstance(node, ast.ImportFrom) else [a.name for a in node.names]
+            if any(n.split(".")[0] == "oracle" for n in names):
+                fn = parent.get(node)
+                while fn is not None and not isinstance(fn, ast.FunctionDef):
+                    fn = parent.get(fn)
+                assert fn is not None and fn.name == "oracle_sample", ast.dump(node)
+                found += 1
+    assert found >= 1
