@@ -40,7 +40,7 @@ inline bq_status check_desc(const bq_pack_desc* d, int K, bool need_ptrs) {
     case BQ_FMT_TERNARY_A8:
       if (d->lora_rank < 0 || d->lora_rank > BQ_MAX_LORA_RANK || d->lora_rank % 8 != 0) return BQ_ERR_INVALID_ARG;
       if (need_ptrs && d->lora_rank > 0 && (!d->lora_A || !d->lora_B)) return BQ_ERR_INVALID_ARG;
-      if (!(d->lora_alpha == d->lora_alpha)) return BQ_ERR_INVALID_ARG;
+      if (!std::isfinite(d->lora_alpha)) return BQ_ERR_INVALID_ARG;
       return BQ_OK;
     case BQ_FMT_ABQ: {
       if (d->w_bits < 1 || d->w_bits > 8 || d->a_bits < 1 || d->a_bits > 8) return BQ_ERR_INVALID_ARG;
@@ -503,6 +503,24 @@ bq_status bq_packed_validate(const void* packed_host, size_t bytes, const void* 
   if (total != L.total || int(h[HW_NPAD]) != L.N_pad || int(h[HW_KPAD]) != L.K_pad ||
       int(h[HW_TILEBYTES]) != L.tile_bytes || int(h[HW_NSTREAMS]) != L.nstreams)
     return BQ_ERR_BAD_PACKED;
+  // every word the writer derives from the layout must agree with it: the kernels take bit
+  // widths, fields and the correction rank from the layout, and load the correction rows 16
+  // bytes at a time (a rank that is not a multiple of 8 would misalign them)
+  const HeaderWords want = header_words(L);
+  for (int w = HW_WBITS; w <= HW_LORA_RANK; w++)
+    if (w != HW_TILEBYTES && h[w] != want.w[w]) return BQ_ERR_BAD_PACKED;
+  if (fmt == BQ_FMT_TERNARY_A8 && (rank % 8 != 0 || !std::isfinite(alpha))) return BQ_ERR_BAD_PACKED;
+  if (fmt != BQ_FMT_TERNARY_A8 && h[HW_LORA_ALPHA] != 0u) return BQ_ERR_BAD_PACKED;
+  // the tensor scale: mean|W| for BitNet and ternary (finite, >= 0), unused (0) otherwise
+  float tscale;
+  std::memcpy(&tscale, &h[HW_TSCALE], 4);
+  if (fmt == BQ_FMT_BITNET_W1A8 || fmt == BQ_FMT_TERNARY_A8) {
+    if (!std::isfinite(tscale) || !(tscale >= 0.f)) return BQ_ERR_BAD_PACKED;
+  } else if (h[HW_TSCALE] != 0u) {
+    return BQ_ERR_BAD_PACKED;
+  }
+  for (int w = HW_OFF_AUX2 + 2; w < 64; w++)  // reserved
+    if (h[w] != 0u) return BQ_ERR_BAD_PACKED;
   if (fmt == BQ_FMT_ABQ) {
     const long long bound = ((1ll << L.w_bits) - 1) * ((1ll << L.a_bits) - 1) * (long long)K;
     if (bound >= (1ll << 31)) return BQ_ERR_BAD_PACKED;

@@ -138,7 +138,7 @@ typedef struct {
   int32_t w_bits;       /* ABQ weight bits, 1..8 (ignored by the other formats) */
   int32_t a_bits;       /* ABQ activation bits, 1..8 (ignored: the A8 formats use 8) */
   int32_t lora_rank;    /* ternary: rank r of the correction, 0..64, a multiple of 8 (0 = none) */
-  float lora_alpha;     /* ternary: gate alpha; the correction is scaled by tanh(alpha) */
+  float lora_alpha;     /* ternary: gate alpha (finite); the correction is scaled by tanh(alpha) */
   const float* h2;      /* RaBiT, rabit_svid_rounds = 0: device f32 [K], second-path input
                            scale (h1 = 1); unused otherwise (may be NULL) */
   const float* lora_A;  /* ternary: device f32 [K][r] row-major, rounded to bf16 */
@@ -201,7 +201,12 @@ bq_status bq_pack_weights(const bq_pack_desc* desc, const float* W, int32_t N, i
                           void* packed, size_t packed_bytes, void* stream, bq_layer* layer);
 
 /* Parse and check a HOST copy of a packed buffer's header (e.g. after loading a saved
- * buffer) and fill `layer` with packed_dev as its device pointer. Host only. */
+ * buffer) and fill `layer` with packed_dev as its device pointer. Host only. The header must
+ * be exactly what bq_pack_weights writes for its format, N, K (and ABQ w/a bits, ternary
+ * rank and alpha): sizes, section offsets, bit widths, fields, shifts and rank as the layout
+ * derives them (a ternary rank a multiple of 8, alpha finite); the tensor scale finite and
+ * >= 0 for BitNet and ternary, 0 otherwise; the reserved words 32..63 zero. Anything else:
+ * BQ_ERR_BAD_PACKED (bytes < 256, a null or unaligned pointer: BQ_ERR_INVALID_ARG). */
 bq_status bq_packed_validate(const void* packed_host, size_t bytes, const void* packed_dev,
                              bq_layer* layer);
 

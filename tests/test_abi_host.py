@@ -383,3 +383,56 @@ def test_product_path_never_imports_the_oracle():
                 assert fn is not None and fn.name == "oracle_sample", ast.dump(node)
                 found += 1
     assert found >= 1
+
+
+def test_packed_validate_refuses_every_inconsistent_word():
+    """A header must be exactly what the pack writes: each single-word corruption below is
+    BQ_ERR_BAD_PACKED, including a ternary rank that is not a multiple of 8 (the kernels load
+    the correction rows 16 bytes at a time)."""
+    def bad(fmt, kw, word, value, N=64, K=256):
+        h = _host_header(fmt, N, K, **kw)
+        h[word] = value
+        with pytest.raises(bq.BQError) as e:
+            bq.bq_packed_validate(h.tobytes(), 1 << 20)
+        assert e.value.status == bq.BQ_ERR_BAD_PACKED, (fmt, word, value)
+    f32 = lambda v: int(np.array([v], "<f4").view("<u4")[0])
+    bad("bitnet", {}, 7, 2)                                  # w_bits
+    bad("bitnet", {}, 8, 4)                                  # a_bits
+    bad("bvsr", {}, 10, 2)                                   # a field width
+    bad("abq", dict(w_bits=6, a_bits=6), 15, 3)              # a stream shift
+    bad("bitnet", {}, 19, 8)                                 # a correction rank on BitNet
+    bad("ternary", dict(lora_rank=32), 19, 28)               # rank changed: sizes disagree
+    bad("ternary", dict(lora_rank=32), 20, f32(np.nan))      # gate alpha
+    bad("bitnet", {}, 20, f32(0.1))                          # alpha on a format without a correction
+    bad("bitnet", {}, 21, f32(-1.0))                         # negative tensor scale
+    bad("ternary", {}, 21, f32(np.inf))
+    bad("abq", dict(w_bits=4, a_bits=4), 21, f32(1.0))       # a tensor scale where none is used
+    bad("rabit3", {}, 40, 1)                                 # a reserved word
+    # the documented values themselves pass
+    h = _host_header("ternary", 64, 256, lora_rank=32)
+    h[20], h[21] = f32(0.1), f32(0.02)
+    bq.bq_packed_validate(h.tobytes(), 1 << 20)
+
+
+def test_packed_validate_refuses_a_rank_not_a_multiple_of_8():
+    """Ternary rank 12 with sections sized consistently for it (N 64, K 256, by hand: tiles
+    4 x 1024 at 256, A bf16 [256][12] at 4352, B^T bf16 [64][12] at align256(4352 + 6144) =
+    10496, total align256(10496 + 1536) = 12032): only the rank rule can refuse it."""
+    h = _host_header("ternary", 64, 256, lora_rank=32)
+    h[19] = 12
+    for word, v in [(22, 12032), (26, 4352), (28, 4352), (30, 10496)]:
+        h[word], h[word + 1] = v, 0
+    with pytest.raises(bq.BQError) as e:
+        bq.bq_packed_validate(h.tobytes(), 1 << 20)
+    assert e.value.status == bq.BQ_ERR_BAD_PACKED
+    h[19] = 16   # a multiple of 8 with sizes for 16 passes
+    for word, v in [(22, 256 + 4096 + 256 * 16 * 2 + 64 * 16 * 2), (26, 4352), (28, 4352), (30, 4352 + 8192)]:
+        h[word], h[word + 1] = v, 0
+    assert bq.bq_packed_validate(h.tobytes(), 1 << 20).lora_rank == 16
+
+
+def test_pack_refuses_a_non_finite_gate():
+    out = ctypes.c_size_t(0)
+    for alpha in (float("inf"), float("nan")):
+        d = bq.make_desc("ternary", lora_rank=8, lora_alpha=alpha)
+        assert bq.raw_status("bq_packed_bytes", ctypes.byref(d), 64, 256, ctypes.byref(out)) == bq.BQ_ERR_INVALID_ARG
