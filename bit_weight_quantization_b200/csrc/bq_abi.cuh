@@ -101,7 +101,14 @@ inline unsigned blocks_for(uint64_t n, unsigned threads) { return unsigned((n + 
 inline bq_status check_layer(const bq_layer* y, PkLayout* L) {
   if (!y || !y->packed || !aligned(y->packed, 256)) return BQ_ERR_INVALID_ARG;
   if (check_nk(y->N, y->K) != BQ_OK) return BQ_ERR_SIZE;
+  // the same rules as the pack: a ternary rank in 0..64 and a multiple of 8 (the correction
+  // rows are loaded 16 bytes at a time), no rank elsewhere, ABQ sums exact in int32
+  if (y->fmt == BQ_FMT_TERNARY_A8 ? (y->lora_rank < 0 || y->lora_rank > BQ_MAX_LORA_RANK || y->lora_rank % 8 != 0)
+                                  : y->lora_rank != 0)
+    return BQ_ERR_INVALID_ARG;
   if (!layout_from_layer(y, L)) return BQ_ERR_INVALID_ARG;
+  if (L->fmt == BQ_FMT_ABQ && ((1ll << L->w_bits) - 1) * ((1ll << L->a_bits) - 1) * (long long)L->K >= (1ll << 31))
+    return BQ_ERR_INVALID_ARG;
   if (L->N_pad != y->N_pad || L->K_pad != y->K_pad || L->total > y->packed_bytes) return BQ_ERR_BAD_PACKED;
   return BQ_OK;
 }

@@ -171,7 +171,10 @@ typedef struct {
 
 /* Host-side description of a packed layer; filled by bq_pack_weights or
  * bq_packed_validate, read by every other call (so no call reads the device header
- * from the host). `packed` is the caller's device buffer. */
+ * from the host). `packed` is the caller's device buffer. Every call checks it against
+ * the pack's rules (sizes, a ternary lora_rank that is a multiple of 8 within 0..64 and 0
+ * for the other formats, the ABQ int32 bound) and returns BQ_ERR_INVALID_ARG, or
+ * BQ_ERR_BAD_PACKED for sizes that disagree, before anything runs. */
 typedef struct {
   int32_t fmt, N, K, N_pad, K_pad, w_bits, a_bits, lora_rank;
   uint64_t packed_bytes;

@@ -436,3 +436,23 @@ def test_pack_refuses_a_non_finite_gate():
     for alpha in (float("inf"), float("nan")):
         d = bq.make_desc("ternary", lora_rank=8, lora_alpha=alpha)
         assert bq.raw_status("bq_packed_bytes", ctypes.byref(d), 64, 256, ctypes.byref(out)) == bq.BQ_ERR_INVALID_ARG
+
+
+def test_hand_made_layer_descriptors_follow_the_pack_rules():
+    """A bq_layer built or edited by hand meets the pack's rules in every call: ternary rank a
+    multiple of 8 within 0..64, no rank for other formats, ABQ within the int32 bound."""
+    def status(layer):
+        out = ctypes.c_size_t(0)
+        return bq.raw_status("bq_act_bytes", ctypes.byref(layer), 1, ctypes.byref(out))
+    t = bq.bq_packed_validate(_host_header("ternary", 64, 256, lora_rank=32).tobytes(), 1 << 20)
+    assert status(t) == bq.BQ_OK
+    for r in (12, -8, 72):
+        t.lora_rank = r
+        assert status(t) == bq.BQ_ERR_INVALID_ARG, r
+    b = bq.bq_packed_validate(_host_header("bitnet", 64, 256).tobytes(), 1 << 20)
+    b.lora_rank = 8
+    assert status(b) == bq.BQ_ERR_INVALID_ARG
+    a = bq.bq_packed_validate(_host_header("abq", 64, 65536, w_bits=8, a_bits=7).tobytes(), 1 << 30)
+    assert status(a) == bq.BQ_OK                     # 255 * 127 * 65536 = 2,122,383,360 < 2^31
+    a.a_bits = 8
+    assert status(a) == bq.BQ_ERR_INVALID_ARG        # 255 * 255 * 65536 = 4,261,478,400 >= 2^31
