@@ -456,3 +456,58 @@ def test_hand_made_layer_descriptors_follow_the_pack_rules():
     assert status(a) == bq.BQ_OK                     # 255 * 127 * 65536 = 2,122,383,360 < 2^31
     a.a_bits = 8
     assert status(a) == bq.BQ_ERR_INVALID_ARG        # 255 * 255 * 65536 = 4,261,478,400 >= 2^31
+
+
+def _rand_int(rng):
+    return rng.choice([rng.randint(-3, 10), rng.randint(-100, 70000), rng.getrandbits(31), -rng.getrandbits(31)])
+
+
+def test_host_queries_under_random_arguments():
+    """Seeded fuzz of the host-only calls: random descriptors, sizes and hand-edited layer
+    descriptors always get a status back, and whatever is accepted has sane sizes (256-byte
+    multiples, a plan that fits the SM)."""
+    import random
+    rng = random.Random(1234)
+    layers = [("bitnet", {}), ("ternary", dict(lora_rank=32)), ("abq", dict(w_bits=4, a_bits=4)),
+              ("bvsr", {}), ("rabit", {}), ("rabit3", {})]
+    for _ in range(1500):
+        d = bq.bq_pack_desc(rng.randint(-1, 8), _rand_int(rng), _rand_int(rng), _rand_int(rng),
+                            rng.choice([0.1, float("nan"), float("inf")]), None, None, None,
+                            _rand_int(rng) if rng.random() < 0.3 else 0, _rand_int(rng) if rng.random() < 0.3 else 0,
+                            None, None, None)
+        out = ctypes.c_size_t(0)
+        K = rng.choice([_rand_int(rng), 128 * rng.randint(1, 600)])
+        if bq.raw_status("bq_packed_bytes", ctypes.byref(d), _rand_int(rng), K, ctypes.byref(out)) == bq.BQ_OK:
+            assert out.value >= 256 and out.value % 256 == 0
+        fmt, kw = rng.choice(layers)
+        L_ = bq.bq_packed_validate(_host_header(fmt, rng.randint(1, 3000), 128 * rng.randint(1, 64), **kw).tobytes(),
+                                   1 << 30)
+        for f in rng.sample(["fmt", "N", "K", "N_pad", "K_pad", "w_bits", "a_bits", "lora_rank"], rng.randint(0, 2)):
+            setattr(L_, f, _rand_int(rng))
+        o = ctypes.c_size_t(0)
+        if bq.raw_status("bq_act_bytes", ctypes.byref(L_), rng.choice([0, 1, 64, 65]), ctypes.byref(o)) == bq.BQ_OK:
+            assert o.value % 256 == 0
+        info = bq.bq_plan_info()
+        if bq.raw_status("bq_linear_plan", ctypes.byref(L_), rng.choice([1, 8, 64]), 1, ctypes.byref(info)) == bq.BQ_OK:
+            assert 0 < info.shared_bytes <= 227 * 1024 and info.ring_stages >= 2
+
+
+def test_packed_validate_under_mutated_headers():
+    """Seeded fuzz: valid headers with one to three words overwritten are either refused with
+    BQ_ERR_BAD_PACKED or describe a layer the host queries accept."""
+    import random
+    rng = random.Random(99)
+    layers = [("bitnet", {}), ("ternary", dict(lora_rank=32)), ("abq", dict(w_bits=3, a_bits=5)), ("bvsr", {}),
+              ("rabit", {}), ("rabit3", {})]
+    for _ in range(1500):
+        fmt, kw = rng.choice(layers)
+        h = _host_header(fmt, rng.randint(1, 5000), 128 * rng.randint(1, 100), **kw)
+        for _ in range(rng.randint(1, 3)):
+            w = rng.randint(1, 63)
+            h[w] = rng.choice([0, 1, 0xFFFFFFFF, rng.getrandbits(32), (int(h[w]) + rng.choice([-256, -1, 1, 256])) & 0xFFFFFFFF])
+        try:
+            layer = bq.bq_packed_validate(h.tobytes(), 1 << 20)
+        except bq.BQError as e:
+            assert e.status == bq.BQ_ERR_BAD_PACKED
+            continue
+        assert bq.bq_act_bytes(layer, 1) % 256 == 0
