@@ -605,6 +605,7 @@ bq_status bq_gemm(const bq_layer* layer, const void* act, int32_t M, float* y, i
   g.u_part = reinterpret_cast<const float*>(Ab + A.off_u);
   g.act_gsum = reinterpret_cast<const int*>(Ab + A.off_gsum);
   g.act_xt = reinterpret_cast<const float*>(Ab + A.off_xt);
+  g.act_total = A.total;
   return launch_layer(L, g, false, reinterpret_cast<cudaStream_t>(stream));
 }
 

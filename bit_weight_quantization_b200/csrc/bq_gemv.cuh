@@ -155,6 +155,7 @@ struct LayerArgs {
   const int* act_gsum;
   const float* act_xt;
   const float* u_part;      // ternary: partial x.A per 256-k tile [KT][M][r] (act buffer or workspace)
+  unsigned long long act_total;  // unfused: the act buffer's size for this layer and M
   float* y;
   long long* acc;
   int N, K, N_pad, K_pad, KT, RB, M, tile_bytes, rank, fmt, a_bits, shift0, shift1, shift2;
@@ -547,6 +548,16 @@ __device__ void stage_quantize_reload(const LayerArgs& a, uint8_t* smem, int m0,
   }
 }
 
+// The act buffer was written for this layer and M: every header word its layout depends on
+// (the format, M, K, activation bits, correction rank) and its total size agree, so every
+// section read below lies inside it.
+__device__ __forceinline__ bool act_header_ok(const uint32_t* h, const LayerArgs& a) {
+  return h[AW_MAGIC] == kActMagic && h[AW_VERSION] == kVersion && h[AW_FMT] == uint32_t(a.fmt) &&
+         h[AW_M] == uint32_t(a.M) && h[AW_K] == uint32_t(a.K) && h[AW_ABITS] == uint32_t(a.a_bits) &&
+         h[AW_LORA_RANK] == uint32_t(a.rank) && h[AW_TOTAL] == uint32_t(a.act_total) &&
+         h[AW_TOTAL + 1] == uint32_t(a.act_total >> 32);
+}
+
 // Unfused: this CTA's tokens from the act buffer (after checking its header): the codes
 // by one bulk copy per token, token parameters and BVSR sums by plain loads.
 template <int FMT, int NW>
@@ -555,9 +566,7 @@ __device__ bool stage_copy(const LayerArgs& a, uint8_t* smem, int m0, int mg, ui
   int* bad = reinterpret_cast<int*>(smem + a.off_red);
   const int tid = threadIdx.x;
   if (tid == 0) {
-    const uint32_t* h = a.act_hdr;
-    const int b = !(h[AW_MAGIC] == kActMagic && h[AW_FMT] == uint32_t(a.fmt) && h[AW_M] == uint32_t(a.M) &&
-                    h[AW_K] == uint32_t(a.K));
+    const int b = !act_header_ok(a.act_hdr, a);
     *bad = b;
     if (b) {
       atomicOr(&g_bq_device_error, kErrActHeader);
@@ -1022,9 +1031,7 @@ __global__ void __launch_bounds__(NW * 32) k_rabit(LayerArgs a) {
   pdl_wait();
   if (!FUSED) {
     if (threadIdx.x == 0) {
-      const uint32_t* h = a.act_hdr;
-      bad = !(h[AW_MAGIC] == kActMagic && h[AW_FMT] == uint32_t(a.fmt) && h[AW_M] == uint32_t(a.M) &&
-              h[AW_K] == uint32_t(a.K));
+      bad = !act_header_ok(a.act_hdr, a);
       if (bad) atomicOr(&g_bq_device_error, kErrActHeader);
     }
     __syncthreads();

@@ -43,8 +43,10 @@
  *
  * Errors: arguments are validated on the host before anything is enqueued; on error
  * nothing runs and a status is returned. A failed launch returns BQ_ERR_CUDA.
- * The kernels check the act-buffer header against the layer (format, M, K) and on a
- * mismatch write no output and raise a device error word that bq_device_check reports.
+ * The kernels check the act-buffer header against the layer (version, format, M, K,
+ * activation bits, correction rank and total size, so that every section they read lies
+ * inside the buffer) before reading anything else from it; on a mismatch they write no
+ * output and raise a device error word that bq_device_check reports.
  * No exception crosses this ABI, and there is no CPU fallback: every step runs on the GPU.
  *
  * ------------------------------------------------------------------------------------

@@ -267,6 +267,25 @@ def test_act_buffer_mismatch_is_reported():
     bq.bq_device_check()   # the word was cleared
 
 
+@pytest.mark.parametrize("fmt,kw_act,kw_layer", [("ternary", dict(lora_rank=8), dict(lora_rank=32)),
+                                                  ("abq", dict(w_bits=4, a_bits=4), dict(w_bits=4, a_bits=8))])
+def test_act_buffer_of_another_layer_config_is_refused(fmt, kw_act, kw_layer):
+    """An act buffer quantized for a layer of the same format, N, K and M but another correction
+    rank (its sections are smaller) or activation width: the kernel reads only its header,
+    writes nothing and raises the device error word."""
+    from tests.parity_util import torch_mods
+    torch, bq = torch_mods()
+    src = GpuLayer(fmt, 32, 256, 1, **kw_act)
+    dst = GpuLayer(fmt, 32, 256, 1, **kw_layer)
+    y = torch.full((1, 32), 7.0, device="cuda")
+    bq.bq_gemv(dst.ql.layer, src.ql.act_buffer(1), y)
+    with pytest.raises(bq.BQError) as e:
+        bq.bq_device_check()
+    assert e.value.status == bq.BQ_ERR_DEVICE_CHECK
+    assert torch.all(y == 7.0)
+    bq.bq_device_check()
+
+
 # ------------------------------------------------------------------ grouped layers sharing x
 @pytest.mark.parametrize("fmt,Ns,K,M,wa", [("bitnet", (64, 97, 40), 512, 1, (1, 8)),
                                            ("bitnet", (4096, 4096, 4096), 4096, 1, (1, 8)),
