@@ -39,7 +39,9 @@ inline bq_status check_desc(const bq_pack_desc* d, int K, bool need_ptrs) {
       return BQ_OK;
     case BQ_FMT_TERNARY_A8:
       if (d->lora_rank < 0 || d->lora_rank > BQ_MAX_LORA_RANK || d->lora_rank % 8 != 0) return BQ_ERR_INVALID_ARG;
-      if (need_ptrs && d->lora_rank > 0 && (!d->lora_A || !d->lora_B)) return BQ_ERR_INVALID_ARG;
+      if (need_ptrs && d->lora_rank > 0 &&
+          (!d->lora_A || !d->lora_B || !aligned(d->lora_A, 4) || !aligned(d->lora_B, 4)))
+        return BQ_ERR_INVALID_ARG;
       if (!std::isfinite(d->lora_alpha)) return BQ_ERR_INVALID_ARG;
       return BQ_OK;
     case BQ_FMT_ABQ: {

@@ -143,8 +143,8 @@ typedef struct {
   float lora_alpha;     /* ternary: gate alpha (finite); the correction is scaled by tanh(alpha) */
   const float* h2;      /* RaBiT, rabit_svid_rounds = 0: device f32 [K], second-path input
                            scale (h1 = 1); unused otherwise (may be NULL) */
-  const float* lora_A;  /* ternary: device f32 [K][r] row-major, rounded to bf16 */
-  const float* lora_B;  /* ternary: device f32 [r][N] row-major, rounded to bf16 */
+  const float* lora_A;  /* ternary: device f32 [K][r] row-major, 4-byte aligned, rounded to bf16 */
+  const float* lora_B;  /* ternary: device f32 [r][N] row-major, 4-byte aligned, rounded to bf16 */
   int32_t rabit_svid_rounds;  /* RaBiT initialisation: 0 = the residual recursion with mean|.|
                            row scales (h1 = 1, h2 given); R in 1..1000 = R rounds of the
                            iterative residual SVID ("RaBiT" page, §2.3, function-aware

@@ -511,3 +511,11 @@ def test_packed_validate_under_mutated_headers():
             assert e.status == bq.BQ_ERR_BAD_PACKED
             continue
         assert bq.bq_act_bytes(layer, 1) % 256 == 0
+
+
+def test_pack_refuses_unaligned_or_missing_correction_matrices():
+    fake = 1 << 40
+    for A, B in [(None, fake), (fake, None), (fake + 2, fake), (fake, fake + 1)]:
+        d = bq.make_desc("ternary", lora_rank=8, lora_A=A, lora_B=B)
+        assert bq.raw_status("bq_pack_weights", ctypes.byref(d), fake, 64, 256, fake, 1 << 30, None,
+                             ctypes.byref(bq.bq_layer())) == bq.BQ_ERR_INVALID_ARG
