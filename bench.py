@@ -555,7 +555,8 @@ def run_configs(args) -> None:
 
 
 def run_layer(args) -> None:
-    """One layer, a few act + gemv calls (the target of ncu captures)."""
+    """One layer, a few calls (the target of ncu captures): bq_linear (fused) by default,
+    bq_quantize_act + bq_gemv/bq_gemm with --unfused."""
     import torch
     dev = torch.device("cuda", 0)
     gen = torch.Generator(device=dev)
