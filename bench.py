@@ -84,6 +84,20 @@ def job_value(bytes_per_step: float, steps: int, ms_max: float, world: int) -> f
     return world * bytes_per_step * steps / (ms_max * 1e-3) / 1e9
 
 
+def clock_record(clk: dict) -> dict:
+    """The bench line's clocks: the SM clock median and reasons of the timed window when it
+    holds samples, else of the soak and timed windows together (the whole sampled run)."""
+    t = clk.get("timed") or {}
+    s = clk.get("soak") or {}
+    src = t if t.get("samples") else clk
+    out = {"sm_mhz": src.get("sm_mhz"), "sm_max_mhz": clk.get("sm_max_mhz"),
+           "reasons": sorted(set(clk.get("reasons", [])) | set(t.get("reasons", [])) | set(s.get("reasons", []))),
+           "samples": clk.get("samples", 0), "timed_samples": t.get("samples", 0), "soak_samples": s.get("samples", 0),
+           "soak_sm_mhz": s.get("sm_mhz"), "timed_sm_mhz": t.get("sm_mhz"), "power_w_max": clk.get("power_w_max"),
+           "window": "timed regions" if t.get("samples") else "soak + timed"}
+    return out
+
+
 def measured_peaks() -> tuple[float, str]:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -122,25 +136,54 @@ def profile_traffic(kernel_key: str):
 
 
 class ClockSampler:
+    """nvidia-smi sampled every `period_ms` in a background reader; each line is stamped with
+    the host time it arrived, so samples can be assigned to the soak and timed windows."""
     FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
-        self.proc = None
+    def __init__(self, index: int, period_ms: int = 100):
+        import threading
+        self.proc, self.lines, self.windows = None, [], {}
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "20", "-i", str(index)], stdout=subprocess.PIPE,
+                                          "-lms", str(period_ms), "-i", str(index)], stdout=subprocess.PIPE,
                                          stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line))
+
+    def wait_first(self, timeout: float = 5.0) -> bool:
+        """Block until the first sample has arrived (or `timeout` s)."""
+        t0 = time.time()
+        while self.proc is not None and not self.lines and time.time() - t0 < timeout:
+            time.sleep(0.01)
+        return bool(self.lines)
+
+    def window(self, name: str, t0: float, t1: float):
+        self.windows[name] = (t0, t1)
 
     def stop(self) -> dict:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)   # one more period after the last window
         self.proc.terminate()
-        out, _ = self.proc.communicate(timeout=10)
-        return self.parse(out)
+        try:
+            self.proc.wait(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        out = self.parse("".join(l for _, l in self.lines))
+        for name, (t0, t1) in self.windows.items():
+            sel = "".join(l for t, l in self.lines if t0 <= t <= t1 + 0.15)
+            out[name] = self.parse(sel)
+        return out
 
     @staticmethod
     def parse(out: str) -> dict:
@@ -162,37 +205,65 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm), "power_w_max": max(pw), "window": "warmup+timed"}
+                "samples": len(sm), "power_w_max": max(pw)}
 
 
 # ---------------------------------------------------------------------------
 # CPU oracle arm / baseline
 # ---------------------------------------------------------------------------
-def oracle_sample(seconds: float, seed: int = 0, min_calls: int = 2) -> dict:
-    """Time the CPU oracle (act quantization + reference layer) on q-projection
-    sized BitNet W1A8 layer calls (4096x4096, M=1) for about `seconds`."""
+def cpu_model() -> str:
+    """The host CPU's model name (first processor in /proc/cpuinfo), or the platform string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
+def oracle_sample(seconds: float, seed: int = 0, min_calls: int = 2, threads: int = 0) -> dict:
+    """Time the C++ oracle (act quantization + reference layer, oracle/bq_ref.cpp) on
+    q-projection sized BitNet W1A8 layer calls (4096x4096, M=1) for about `seconds`, on
+    `threads` OpenMP threads (0: all host cores). Returns the sample's GB/s over all calls and the
+    best single call (time.perf_counter around each call)."""
     import bq_inputs as I
-    from oracle import bq_oracle as O
+    from oracle import cref as O
+    O.set_threads(threads if threads > 0 else (os.cpu_count() or 1))
     W = I.weights(4096, 4096, seed)
     x = I.activations(1, 4096, seed)
     p = O.bitnet_pack(W)
-    calls, t0 = 0, time.perf_counter()
+    calls, times, t0 = 0, [], time.perf_counter()
     while True:
+        c0 = time.perf_counter()
         O.bitnet_layer(p, x)
+        times.append(time.perf_counter() - c0)
         calls += 1
         el = time.perf_counter() - t0
         if el >= seconds and calls >= min_calls:
             break
     b = layer_bytes("bitnet", 4096, 4096)["fused"]
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = 1
-    return dict(seconds=el, calls=calls, gbs=calls * b / el / 1e9, us_per_layer=el / calls * 1e6, cores=cores)
+    return dict(seconds=el, calls=calls, gbs=calls * b / el / 1e9, us_per_layer=el / calls * 1e6,
+                best_us=min(times) * 1e6, best3_us=sorted(times)[min(2, len(times) - 1)] * 1e6,
+                cores=O.threads(), cpu=cpu_model(), nproc=os.cpu_count())
+
+
+def cpu_baseline_record(all_cores: dict, one_core: dict) -> dict:
+    """The bench line's cpu_baseline: the oracle on all host cores (the value) and on one core."""
+    return {"value": all_cores["gbs"], "unit": "GB/s", "cores": all_cores["cores"], "kind": "oracle (C++)",
+            "cpu": all_cores["cpu"], "nproc": all_cores["nproc"],
+            "sample": f"{all_cores['calls']} BitNet W1A8 4096x4096 layer calls (act quant + layer) of the C++ "
+                      f"oracle in {all_cores['seconds']:.1f} s; best call {all_cores['best_us']:.0f} us",
+            "one_core": {"value": one_core["gbs"], "unit": "GB/s", "cores": one_core["cores"],
+                         "calls": one_core["calls"], "seconds": one_core["seconds"],
+                         "best_us": one_core["best_us"]}}
 
 
 def run_reference(args) -> None:
+    """The reference arm: the C++ oracle on the host cores, one BitNet W1A8 4096x4096 layer call
+    (act quantization + layer) per step, on all cores; a one-core sample beside it."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -203,17 +274,21 @@ def run_reference(args) -> None:
     calls = sum(r["calls"] for r in res)
     b = layer_bytes("bitnet", 4096, 4096)["fused"]
     val = calls * b / el / 1e9
+    one = oracle_sample(min(args.cpu_seconds, 3.0), min_calls=2, threads=1)
     cores = res[0]["cores"]
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64+f64",
         "data": "synthetic",
-        "config": {"workload": "BitNet W1A8 decode GEMV, Llama-7B shapes, M=1 (CPU oracle sample: one "
+        "config": {"workload": "BitNet W1A8 decode GEMV, Llama-7B shapes, M=1 (C++ CPU oracle sample: one "
                                "4096x4096 layer call per step)", "seq_len": 1, "global_batch": 1},
         "us_per_layer": el / calls * 1e6,
-        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{calls} BitNet W1A8 4096x4096 layer calls (act quant + layer), numpy"},
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": cores, "kind": "oracle (C++)", "cpu": res[0]["cpu"],
+                         "nproc": res[0]["nproc"],
+                         "sample": f"{calls} BitNet W1A8 4096x4096 layer calls (act quant + layer) of the C++ oracle",
+                         "one_core": {"value": one["gbs"], "unit": "GB/s", "cores": one["cores"],
+                                      "calls": one["calls"], "best_us": one["best_us"]}},
         "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -302,22 +377,47 @@ def run_cuda(args) -> None:
         torch.cuda.synchronize()
         bq.bq_device_check()
 
+        # clocks: the sampler runs from before the soak to after the last timed region
         clocks = ClockSampler(local)
+        clocks.wait_first()
+        # soak: the same step replayed for about --soak-seconds (untimed) so that the clocks
+        # sampled are those of this workload under load
+        ts0 = time.time()
+        n_soak = 0
+        while time.time() - ts0 < args.soak_seconds or n_soak == 0:
+            for _ in range(8):
+                g.replay()
+            torch.cuda.synchronize()
+            n_soak += 8
+        ts1 = time.time()
+        host_ms_step = (ts1 - ts0) * 1e3 / n_soak
         for _ in range(args.warmup):
             g.replay()
         torch.cuda.synchronize()
-        barrier()
-        torch.cuda.synchronize()
+        # timed: R back-to-back regions of exactly K steps each, every region bracketed by a
+        # barrier and a synchronize, so that together they last about --timed-seconds
+        R = int(reduce_max_over_ranks([max(1, min(200, -(-args.timed_seconds * 1e3 // (host_ms_step * args.steps))))],
+                                      dist if world > 1 else None, dev)[0])
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            g.replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        torch.cuda.synchronize()
+        region_ms = []
+        tt0 = time.time()
+        for _ in range(R):
+            barrier()
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(args.steps):
+                g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            torch.cuda.synchronize()
+            region_ms.append(e0.elapsed_time(e1))
+        tt1 = time.time()
+        clocks.window("soak", ts0, ts1)
+        clocks.window("timed", tt0, tt1)
         clk = clocks.stop()
-        ms = e0.elapsed_time(e1)
+        region_ms = reduce_max_over_ranks(region_ms, dist if world > 1 else None, dev)
+        ms = statistics.median(region_ms)
 
         # serialized per-launch time (context only): a second capture of the same step with
         # events around every bq_linear; the events between launches remove the PDL overlap
@@ -367,7 +467,7 @@ def run_cuda(args) -> None:
         e2e_ms = t0.elapsed_time(t1) / n_e2e
         bq.bq_device_check()
 
-    ms, e2e_ms = reduce_max_over_ranks([ms, e2e_ms], dist if world > 1 else None, dev)
+    e2e_ms = reduce_max_over_ranks([e2e_ms], dist if world > 1 else None, dev)[0]
     ms_step = ms / args.steps
     value = job_value(per_step, args.steps, ms, world)
     peak, peak_kind = measured_peaks()
@@ -390,6 +490,10 @@ def run_cuda(args) -> None:
                                    " (act quantization fused into the layer kernel), PDL between launches, "
                                    "CUDA graph per step",
                        "layers_per_step": n_layers, "launches_per_step": n_calls, "seq_len": 1,
+                       "timing": "median of %d back-to-back timed regions of %d steps each (CUDA events; "
+                                 "region ms min %.3f, median %.3f, max %.3f); %.1f s untimed soak before the "
+                                 "warm-up" % (len(region_ms), args.steps, min(region_ms), ms, max(region_ms),
+                                              args.soak_seconds),
                        "global_batch": world,
                        "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (each step streams %.0f MB of distinct packed weights)"
@@ -405,17 +509,15 @@ def run_cuda(args) -> None:
                     "h2d_bytes_per_step": int(xs_h.numel() * 2), "d2h_bytes_per_step": int(ys_h.numel() * 4),
                     "ms_per_step": e2e_ms, "path": "eager Python calls of the C ABI, pinned host buffers"},
             "gpu_launches": n_calls * args.steps,
-            "clocks": clk,
+            "clocks": clock_record(clk),
         }
     if world > 1:
         del g, gi
         dist.destroy_process_group()
     if rank == 0:
         if world == 1:
-            cb = oracle_sample(args.cpu_seconds)
-            out["cpu_baseline"] = {"value": cb["gbs"], "unit": "GB/s", "cores": cb["cores"], "kind": "oracle",
-                                   "sample": f"{cb['calls']} BitNet W1A8 4096x4096 layer calls "
-                                             f"(act quant + layer), {cb['seconds']:.1f} s"}
+            out["cpu_baseline"] = cpu_baseline_record(oracle_sample(args.cpu_seconds),
+                                                      oracle_sample(args.cpu_seconds / 2, threads=1))
         print(json.dumps(out), flush=True)
 
 
@@ -580,6 +682,10 @@ def main():
     ap.add_argument("--layers", type=int, default=32)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--soak-seconds", type=float, default=1.5,
+                    help="untimed replays before the warm-up, while the clocks are sampled")
+    ap.add_argument("--timed-seconds", type=float, default=1.0,
+                    help="the timed regions (K steps each) repeat until they last about this long")
     ap.add_argument("--mode", default="bench", choices=["bench", "configs", "layer"])
     ap.add_argument("--only", default="")
     ap.add_argument("--fmt", default="bitnet")

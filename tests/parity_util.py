@@ -1,12 +1,13 @@
 """Helpers for GPU parity tests: run the CUDA path through the C ABI, read its
 buffers back with the oracle's independent readers, and compare with the
-oracle. Test infrastructure only."""
+oracle (the C++ reference, oracle/bq_ref.cpp through oracle/cref.py). Test
+infrastructure only."""
 from __future__ import annotations
 
 import numpy as np
 
 import bq_inputs as I
-from oracle import bq_oracle as O
+from oracle import cref as O
 from oracle import layout as L
 
 RTOL = 1e-3  # max|y - y_ref| <= 1e-3 (||y_ref||_inf + 1e-6)
@@ -33,6 +34,54 @@ def ulp_diff(a, b) -> np.ndarray:
     a = np.asarray(a, np.float32).view(np.int32).astype(np.int64)
     b = np.asarray(b, np.float32).view(np.int32).astype(np.int64)
     return np.abs(a - b)
+
+
+NEAR_TIE_ULPS = 4          # a code may differ only this close (float32 ulps) to its boundary
+NEAR_TIE_LOG: list = []    # (what, codes compared, codes that differ, near-tie codes)
+
+
+def assert_codes_near_tie(got, ref, near, what):
+    """Pack parity where several results are correct: every code is compared, and a code may
+    differ from the oracle's only where ``near`` marks the quantity that decides it within
+    NEAR_TIE_ULPS float32 ulps of its rounding or selection boundary (the GPU reduces the scale
+    that feeds the decision in another order than the oracle). Every differing code is counted
+    and reported; the count is returned."""
+    got, ref, near = np.asarray(got), np.asarray(ref), np.asarray(near, bool)
+    assert got.shape == ref.shape == near.shape, (got.shape, ref.shape, near.shape)
+    diff = got != ref
+    n_diff, n_far = int(diff.sum()), int((diff & ~near).sum())
+    NEAR_TIE_LOG.append((what, int(got.size), n_diff, int(near.sum())))
+    if n_diff:
+        print(f"[near-tie] {what}: {n_diff} of {got.size} codes differ from the oracle "
+              f"({n_diff - n_far} within {NEAR_TIE_ULPS} ulps of a boundary)")
+    assert n_far == 0, f"{what}: {n_far} codes differ from the oracle away from any decision boundary"
+    return n_diff
+
+
+def ulps_of(v) -> np.ndarray:
+    """float32 spacing at |v| (one ulp)."""
+    return np.spacing(np.abs(np.asarray(v, np.float32))).astype(np.float64)
+
+
+def ternary_near(W, gamma_ref) -> np.ndarray:
+    """Ternary codes are decided by W / gamma (float32) against the rounding boundaries +-0.5."""
+    d = (np.asarray(W, np.float32) / np.float32(gamma_ref)).astype(np.float32).astype(np.float64)
+    return np.abs(np.abs(d) - 0.5) <= NEAR_TIE_ULPS * float(np.spacing(np.float32(0.5)))
+
+
+def rabit_near(W, B, g, h) -> list:
+    """RaBiT path p (p >= 1) signs are decided by the residual R_{p-1} = W - sum_{q<p} g_q B_q h_q
+    (float64) against 0; its inputs move by about one ulp of each g_q h_q when the GPU's g_q
+    differs from the oracle's by one ulp. Masks for paths 1.. (path 0, sign(W), has no scale)."""
+    W64 = np.asarray(W, np.float64)
+    R = W64.copy()
+    tol = np.zeros(W64.shape[0])
+    out = []
+    for q in range(len(B) - 1):
+        R = R - (g[q].astype(np.float64)[:, None] * B[q]) * h[q].astype(np.float64)[None, :]
+        tol = tol + ulps_of(g[q]) * float(np.max(np.abs(h[q])))
+        out.append(np.abs(R) <= NEAR_TIE_ULPS * tol[:, None])
+    return out
 
 
 def assert_y_close(y, y_ref, what=""):
@@ -124,7 +173,7 @@ def oracle_layer(fmt, p, x, a_bits=0):
     if fmt == "rabit":
         return O.rabit_layer(p, x)
     if fmt == "rabit3":
-        return dict(y=x.astype(np.float64) @ O.rabit_weight_paths(p).T)
+        return O.rabit_layer(p, x)
     if fmt == "bitnet":
         return O.bitnet_layer(p, x)
     if fmt == "ternary":

@@ -65,3 +65,16 @@ def test_traffic_record_is_dropped_when_the_kernel_source_changes(monkeypatch):
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)
     assert bench.profile_traffic("bitnet_fused_llama7b_grouped") is None
     assert bench.profile_traffic("no_such_kernel") is None
+
+
+def test_clock_record_prefers_the_timed_window():
+    """The bench line's clocks come from the samples inside the timed regions when there are
+    any, else from the whole sampled run; reasons seen in any window are kept."""
+    timed = {"sm_mhz": 1890.0, "samples": 4, "reasons": ["sw_power_cap"]}
+    soak = {"sm_mhz": 1965.0, "samples": 9, "reasons": []}
+    whole = {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "samples": 14, "reasons": ["sw_power_cap"], "power_w_max": 900.0}
+    r = bench.clock_record(dict(whole, timed=timed, soak=soak))
+    assert (r["sm_mhz"], r["window"], r["timed_samples"], r["soak_samples"]) == (1890.0, "timed regions", 4, 9)
+    assert r["reasons"] == ["sw_power_cap"] and r["sm_max_mhz"] == 1965.0
+    r = bench.clock_record(dict(whole, timed={"samples": 0}, soak=soak))
+    assert (r["sm_mhz"], r["window"]) == (1950.0, "soak + timed")

@@ -1,5 +1,7 @@
 """Pins of the CPU oracle against what the pages and the mathematics fix.
 
+Every test runs on both implementations of the oracle: the C++ reference (oracle/bq_ref.cpp,
+through oracle/cref.py) and the numpy one (oracle/bq_oracle.py), through the fixture ``O``.
 Each test checks the oracle against something other than itself: values
 worked by hand from a page's formula (tests/golden, with citations), closed
 forms, brute force over tiny inputs, invariants and special cases. A planted
@@ -11,26 +13,35 @@ import math
 import numpy as np
 import pytest
 
-from oracle import bq_oracle as O
 import bq_inputs as I
 
 
+@pytest.fixture(params=["cpp", "numpy"])
+def O(request):
+    """The oracle implementation under test: the C++ reference or the numpy one."""
+    if request.param == "cpp":
+        from oracle import cref
+        return cref
+    from oracle import bq_oracle
+    return bq_oracle
+
+
 # --------------------------------------------------------------------- sign
-def test_sign_zero_is_plus_one(golden):
+def test_sign_zero_is_plus_one(O, golden):
     g = golden("sign_zero.json")
     got = O.sign_pm1(np.array(g["inputs"], dtype=np.float32))
     assert got.tolist() == g["expect"]
 
 
 # ------------------------------------------------------- activation int8
-def test_act_int8_hand_values(golden):
+def test_act_int8_hand_values(O, golden):
     g = golden("act_int8_handpicked.json")
     q, gamma = O.quantize_act_int8(np.array(g["x"], dtype=np.float32))
     assert q.tolist() == g["q"]
     assert gamma.tolist() == g["gamma"]
 
 
-def test_act_int8_endpoints_and_range():
+def test_act_int8_endpoints_and_range(O):
     rng = np.random.default_rng(5)
     x = (rng.standard_normal((16, 300)) * rng.uniform(0.1, 50, (16, 1))).astype(np.float32)
     q, gamma = O.quantize_act_int8(x)
@@ -46,7 +57,7 @@ def test_act_int8_endpoints_and_range():
 
 
 # -------------------------------------------------------------------- RaBiT
-def test_rabit_recursion_hand_example(golden):
+def test_rabit_recursion_hand_example(O, golden):
     g = golden("rabit_recursion.json")
     p = O.rabit_pack(np.array(g["W"], np.float32), np.array(g["h2"], np.float32))
     assert p["B1"].tolist() == g["B1"]
@@ -56,7 +67,7 @@ def test_rabit_recursion_hand_example(golden):
     assert O.rabit_weight(p).tolist() == g["W_hat"]
 
 
-def test_rabit_constant_magnitude_rows_reconstruct_exactly():
+def test_rabit_constant_magnitude_rows_reconstruct_exactly(O):
     # |W[n,k]| = c_n for all k -> g1 = c_n, R1 == 0, B2 = sign(0) = +1, g2 = 0, W_hat = W
     rng = np.random.default_rng(1)
     c = np.array([0.5, 0.25, 0.125, 2.0], np.float32)
@@ -69,7 +80,7 @@ def test_rabit_constant_magnitude_rows_reconstruct_exactly():
     assert np.array_equal(O.rabit_weight(p), W.astype(np.float64))
 
 
-def test_rabit_layer_is_sum_of_two_sign_paths():
+def test_rabit_layer_is_sum_of_two_sign_paths(O):
     rng = np.random.default_rng(2)
     W = (rng.standard_normal((8, 96)) * 0.02).astype(np.float32)
     h2 = rng.uniform(0.5, 1.5, 96).astype(np.float32)
@@ -90,14 +101,14 @@ def test_rabit_layer_is_sum_of_two_sign_paths():
 
 
 # ------------------------------------------------------------------- BitNet
-def test_bitnet_alpha_is_mean_abs():
+def test_bitnet_alpha_is_mean_abs(O):
     W = np.array([[0.5, -0.25], [-1.0, 0.25]], np.float32)
     p = O.bitnet_pack(W)
     assert p["alpha"] == np.float32(0.5)
     assert p["B"].tolist() == [[1, -1], [-1, 1]]
 
 
-def test_xnor_popcount_identity_all_pairs():
+def test_xnor_popcount_identity_all_pairs(O):
     # BitNet §2.3 binary product: for +-1 vectors, sum a*b = 2*popc(xnor(a,b)) - K
     K = 8
     vals = [[1 if (v >> j) & 1 else -1 for j in range(K)] for v in range(1 << K)]
@@ -106,7 +117,7 @@ def test_xnor_popcount_identity_all_pairs():
             assert O.xnor_popcount_dot(a, b) == sum(x * y for x, y in zip(a, b))
 
 
-def test_w1a8_plane_identity_all_int8_codes():
+def test_w1a8_plane_identity_all_int8_codes(O):
     # sum_k B_k q_k = sum q - 2 * sum_c omega_c popc(NEG & X_c) for every int8 code value
     rng = np.random.default_rng(3)
     codes = np.arange(-127, 128)
@@ -123,7 +134,7 @@ def test_w1a8_plane_identity_all_int8_codes():
         assert sum(w * int(p[0]) for w, p in zip(O.plane_weights(8, True), pl)) == v
 
 
-def test_bitnet_layer_integer_and_float_routes_agree():
+def test_bitnet_layer_integer_and_float_routes_agree(O):
     rng = np.random.default_rng(4)
     W = (rng.standard_normal((24, 128)) * 0.02).astype(np.float32)
     x = rng.standard_normal((2, 128)).astype(np.float32)
@@ -137,14 +148,14 @@ def test_bitnet_layer_integer_and_float_routes_agree():
 
 
 # ------------------------------------------------------------------ ternary
-def test_ternary_hand_examples(golden):
+def test_ternary_hand_examples(O, golden):
     for c in golden("ternary_handpicked.json")["cases"]:
         p = O.ternary_pack(np.array(c["W"], np.float32))
         assert float(p["gamma_w"]) == c["gamma"]
         assert p["T"].tolist() == c["T"]
 
 
-def test_ternary_zero_fraction_of_gaussian():
+def test_ternary_zero_fraction_of_gaussian(O):
     # threshold 0.5*gamma with gamma = sigma*sqrt(2/pi): P(|Z| < 0.5 sqrt(2/pi)) = erf(0.5/sqrt(pi))
     W = (np.random.default_rng(6).standard_normal((1024, 1024)) * 0.02).astype(np.float32)
     p = O.ternary_pack(W)
@@ -153,7 +164,7 @@ def test_ternary_zero_fraction_of_gaussian():
     assert abs(float(np.mean(p["T"] == 1)) - float(np.mean(p["T"] == -1))) < 0.003
 
 
-def test_ternary_int_route_equals_dequant_route():
+def test_ternary_int_route_equals_dequant_route(O):
     # HGF §1.2: Y = Y_int * gamma_x gamma_W / 127
     rng = np.random.default_rng(7)
     W = (rng.standard_normal((16, 64)) * 0.02).astype(np.float32)
@@ -164,7 +175,7 @@ def test_ternary_int_route_equals_dequant_route():
     assert np.allclose(r["y_ternary"], y_int, rtol=1e-12, atol=1e-15)
 
 
-def test_lora_correction_closed_form():
+def test_lora_correction_closed_form(O):
     # tanh(ln 2) = 3/5 and SiLU(ln 3) = ln 3 * sigmoid(ln 3) = 0.75 ln 3
     A = np.array([[math.log(3.0)]])
     B = np.array([[1.0, -2.0, 0.5]])
@@ -181,7 +192,7 @@ def test_lora_correction_closed_form():
 
 
 # ---------------------------------------------------------------------- ABQ
-def test_abq_hand_examples(golden):
+def test_abq_hand_examples(O, golden):
     for c in golden("abq_handpicked.json")["cases"]:
         q, d, z = O.quantize_rows_asym(np.array([c["row"]], np.float32), c["bits"])
         assert q[0].tolist() == c["q"]
@@ -190,7 +201,7 @@ def test_abq_hand_examples(golden):
 
 
 @pytest.mark.parametrize("bits", [2, 4, 6, 8])
-def test_abq_grid_round_trip(bits):
+def test_abq_grid_round_trip(O, bits):
     # values already on a binary-exact grid lo + Delta*i dequantize exactly
     L = 1 << bits
     delta = 2.0 ** -6
@@ -202,7 +213,7 @@ def test_abq_grid_round_trip(bits):
 
 
 @pytest.mark.parametrize("w,a", [(w, a) for w in (2, 4, 6, 8) for a in (2, 4, 6, 8)])
-def test_abq_bitplane_identity_brute_force(w, a):
+def test_abq_bitplane_identity_brute_force(O, w, a):
     # sum_b sum_c 2^(b+c) popc(W_b & X_c) == sum q_w q_x for unsigned codes
     rng = np.random.default_rng(w * 10 + a)
     for _ in range(3):
@@ -211,7 +222,7 @@ def test_abq_bitplane_identity_brute_force(w, a):
         assert O.bitplane_dot(qw, w, False, qx, a, False) == int(np.dot(qw, qx))
 
 
-def test_abq_zero_point_expansion_and_bounds():
+def test_abq_zero_point_expansion_and_bounds(O):
     rng = np.random.default_rng(8)
     W = (rng.standard_normal((12, 256)) * 0.02).astype(np.float32)
     x = (rng.standard_normal((3, 256)) * 3).astype(np.float32)
@@ -232,14 +243,14 @@ def test_abq_zero_point_expansion_and_bounds():
 
 
 # --------------------------------------------------------------------- BVSR
-def test_nearest_rank_quantile():
+def test_nearest_rank_quantile(O):
     v = np.arange(16.0)
     assert [O.nearest_rank(v, 2 * a + 1, 16) for a in range(8)] == [2.0 * a for a in range(8)]
     v = np.arange(10.0)  # ceil(1*10/16) = 1 -> v[0]; ceil(15*10/16) = 10 -> v[9]
     assert O.nearest_rank(v, 1, 16) == 0.0 and O.nearest_rank(v, 15, 16) == 9.0
 
 
-def test_bvsr_ratio2_sets_are_the_uniform_rtn_grid():
+def test_bvsr_ratio2_sets_are_the_uniform_rtn_grid(O):
     # r = 2: subset sums of {1,2,4,8}/15 scaled to [lo, hi] are lo + (hi-lo) i/15, i = 0..15
     W = (np.random.default_rng(9).standard_normal((32, 256)) * 0.02).astype(np.float32)
     tab = O.bvsr_set_table(W)
@@ -251,7 +262,7 @@ def test_bvsr_ratio2_sets_are_the_uniform_rtn_grid():
         assert np.all(np.diff(P[s]) > 0)
 
 
-def test_bvsr_encoding_matches_rtn_for_uniform_set():
+def test_bvsr_encoding_matches_rtn_for_uniform_set(O):
     # a table whose only set is the uniform grid on [lo, hi]: codes are round((w-lo)/Delta) clamped
     lo, hi = -0.06, 0.09
     span = hi - lo
@@ -268,7 +279,7 @@ def test_bvsr_encoding_matches_rtn_for_uniform_set():
     assert np.all(sets == 0)            # equal errors everywhere: lowest set index
 
 
-def test_bvsr_exact_integer_table():
+def test_bvsr_exact_integer_table(O):
     # c = {1,2,4,8}, o = 0 makes the 16 points the integers 0..15: integer weights encode exactly
     tab = np.zeros((256, 5), np.float32)
     tab[:, :4] = [50.0, 60.0, 70.0, 80.0]
@@ -280,7 +291,7 @@ def test_bvsr_exact_integer_table():
     assert np.array_equal(codes, w.astype(np.uint8))
 
 
-def test_bvsr_search_is_exhaustive_optimum():
+def test_bvsr_search_is_exhaustive_optimum(O):
     # no other set, and no single-element code change, gives a smaller squared error
     W = (np.random.default_rng(12).standard_normal((4, 64)) * 0.02).astype(np.float32)
     tab = O.bvsr_set_table(W)
@@ -302,7 +313,7 @@ def test_bvsr_search_is_exhaustive_optimum():
                 assert (w[e_i] - P[sets[v], c]) ** 2 >= (w[e_i] - P[sets[v], codes[v, e_i]]) ** 2 - 1e-18
 
 
-def test_bvsr_layer_routes_agree():
+def test_bvsr_layer_routes_agree(O):
     rng = np.random.default_rng(13)
     W = (rng.standard_normal((6, 128)) * 0.02).astype(np.float32)
     x = rng.standard_normal((2, 128)).astype(np.float32)
@@ -324,7 +335,7 @@ def test_bvsr_layer_routes_agree():
 
 
 # ---------------------------------------------------------- size / memory wall
-def test_memory_wall_and_sizes(golden):
+def test_memory_wall_and_sizes(O, golden):
     g = golden("memory_wall.json")
     w = g["wall"]
     tps = O.decode_tokens_per_s(w["bandwidth_Bps"], w["params"], w["bits"])
@@ -336,13 +347,13 @@ def test_memory_wall_and_sizes(golden):
     assert O.weight_bits_per_param("abq", 6) == 6.0
 
 
-def test_tolerance_helper():
+def test_tolerance_helper(O):
     y_ref = np.array([1.0, -2.0, 0.5])
     assert O.tolerance_ok(y_ref + 1.9e-3, y_ref)
     assert not O.tolerance_ok(y_ref + 2.1e-3, y_ref)
 
 
-def test_bvsr_table_construction_hand_built():
+def test_bvsr_table_construction_hand_built(O):
     # 16 vectors whose minima are -(v+1)/1000 and maxima (v+1)/500, every other element 0.
     # Nearest-rank (2a+1)/16 quantile of 16 values is the (2a+1)-th smallest: lo_a = -(16-2a)/1000,
     # hi_b = (2b+1)/500. Set 64j + 8a + b: o = lo_a, c_i = (hi_b - lo_a) r_j^i / sum_i' r_j^i'.
@@ -367,7 +378,7 @@ def test_bvsr_table_construction_hand_built():
 
 
 # ------------------------------------------------------------------ RaBiT iterative residual SVID
-def test_svid_exact_signed_rank1():
+def test_svid_exact_signed_rank1(O):
     """W = s * (a b^T) with power-of-two a, b: one round recovers W up to float32 rounding of
     g and h (the rank-1 fit is exact in real arithmetic), and path 2 carries only that rounding."""
     rng = np.random.default_rng(5)
@@ -384,7 +395,7 @@ def test_svid_exact_signed_rank1():
     assert np.all(np.abs(p["g2"]) <= 1e-6 * np.abs(p["g1"]).max())
 
 
-def test_svid_first_step_is_mean_abs_and_error_never_grows():
+def test_svid_first_step_is_mean_abs_and_error_never_grows(O):
     W = I.weights(24, 256, seed=9)
     base = O.rabit_pack(W, np.ones(256, np.float32))
     p1 = O.rabit_pack_svid(W, rounds=1)
@@ -397,7 +408,7 @@ def test_svid_first_step_is_mean_abs_and_error_never_grows():
     assert errs[-1] < O.rabit_recon_error(base, W)
 
 
-def test_svid_g_step_is_least_squares():
+def test_svid_g_step_is_least_squares(O):
     """For fixed h, g from the SVID step solves min_g ||A - g h^T||^2 row by row (checked with
     numpy's least squares on the first round's target A = |W|)."""
     W = I.weights(8, 128, seed=3)
@@ -412,7 +423,7 @@ def test_svid_g_step_is_least_squares():
 
 
 # ------------------------------------------------------------------ ABQ bit balance (W2*)
-def test_bit_balance_symmetric_levels():
+def test_bit_balance_symmetric_levels(O):
     W = I.weights(12, 256, seed=21)
     p = O.abq_pack_balanced(W)
     pn = O.abq_pack_balanced(-W)
@@ -423,7 +434,7 @@ def test_bit_balance_symmetric_levels():
     assert np.all(p["Q"][np.arange(12), np.abs(W).argmax(1)] % 4 == 0)
 
 
-def test_bit_balance_grid_round_trip():
+def test_bit_balance_grid_round_trip(O):
     d = np.float32(0.0625)
     levels = np.array([-2, -1, 0, 1, 2], np.float32) * d
     rng = np.random.default_rng(2)
@@ -435,7 +446,7 @@ def test_bit_balance_grid_round_trip():
     assert np.array_equal(deq, W.astype(np.float64))
 
 
-def test_bf16_round_hand_values():
+def test_bf16_round_hand_values(O):
     """Round to nearest bf16, ties to even (hand-worked bit patterns)."""
     vals = np.array([1.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, 1.0 + 2.0 ** -8 + 2.0 ** -20, -2.5], np.float32)
     # 1 + 2^-8 is half-way between 1 and 1 + 2^-7: ties to the even mantissa (1.0);
@@ -445,7 +456,7 @@ def test_bf16_round_hand_values():
     assert np.array_equal(O.bf16_round(vals), want)
 
 
-def test_svid_first_round_path2_g_is_mean_abs_of_residual():
+def test_svid_first_round_path2_g_is_mean_abs_of_residual(O):
     """In the first Gauss-Seidel round, path 2's g-step starts from h = 1, so g2 is the row mean of |W - W_1|
     (W_1 from the returned path-1 state): pins the split of the magnitude between g and h."""
     W = I.weights(10, 256, seed=13)
@@ -456,7 +467,7 @@ def test_svid_first_round_path2_g_is_mean_abs_of_residual():
 
 
 # ------------------------------------------------------------------ RaBiT with P paths (groundwork)
-def test_rabit_paths_two_equals_rabit_pack():
+def test_rabit_paths_two_equals_rabit_pack(O):
     W = I.weights(9, 256, seed=17)
     h2 = I.uniform(256, 0.5, 1.5, seed=2, tid=3)
     a = O.rabit_pack(W, h2)
@@ -466,7 +477,7 @@ def test_rabit_paths_two_equals_rabit_pack():
     assert np.array_equal(O.rabit_weight_paths(b), O.rabit_weight(a))
 
 
-def test_rabit_third_path_lowers_error_by_k_g_squared():
+def test_rabit_third_path_lowers_error_by_k_g_squared(O):
     """With h = 1: ||R - g sign(R)||^2 = ||R||^2 - K g^2 per row when g = mean|R|."""
     W = I.weights(7, 512, seed=23)
     ones = np.ones(512, np.float32)
@@ -479,7 +490,7 @@ def test_rabit_third_path_lowers_error_by_k_g_squared():
     assert np.all(e3 < e2)
 
 
-def test_rabit_three_paths_hand_example():
+def test_rabit_three_paths_hand_example(O):
     """Three paths with non-unit h (every value dyadic, so exact), worked by hand:
     W = [.75, -.25, .5, -1]: B1 = [+ - + -], g1 = 2.5/4 = .625, R1 = [.125, .375, -.125, -.375];
     B2 = [+ + - -], g2 = 1/4 = .25, R2 = R1 - .25 B2 h2 with h2 = [1, 2, 1, .5]
@@ -504,7 +515,7 @@ _COMP_Q0 = np.array([[0, 1, 2, 3, 3, 2, 1, 0],     # 2-bit grid codes; every row
                      [1, 3, 2, 0, 0, 1, 3, 2]], np.int32)
 
 
-def test_abq_compensation_closed_form():
+def test_abq_compensation_closed_form(O):
     """W = G - a b^T with G on the 2-bit grid Delta = 1/16, z = 1: the compensated codes
     are the grid codes, Delta and z come back exactly; without compensation they do not."""
     G = ((_COMP_Q0 - 1) * 0.0625).astype(np.float32)
@@ -519,7 +530,7 @@ def test_abq_compensation_closed_form():
         O.abq_pack_compensated(W, _COMP_B, _COMP_A, 2)
 
 
-def test_abq_compensation_exact_cancellation_is_the_degenerate_row():
+def test_abq_compensation_exact_cancellation_is_the_degenerate_row(O):
     """W = -a b^T: W' = 0 exactly, every row is constant, so the 1e-5 range floor applies,
     z = 0 and every code is 0 at any width."""
     W = (-np.outer(_COMP_A, _COMP_B)).astype(np.float32)
@@ -529,7 +540,7 @@ def test_abq_compensation_exact_cancellation_is_the_degenerate_row():
         assert np.all(p["delta"] > 0) and np.all(p["delta"] <= np.float32(1e-5))   # = at w = 1
 
 
-def test_abq_compensation_off_is_the_plain_pack():
+def test_abq_compensation_off_is_the_plain_pack(O):
     """a = 0 (or b = 0): W + 0 = W, so the codes, Delta and z are the plain pack's."""
     W = I.weights(37, 256, seed=5, outlier_frac=0.01)
     a, b = I.compensation_vectors(37, 256, seed=5)
@@ -541,7 +552,7 @@ def test_abq_compensation_off_is_the_plain_pack():
     assert not np.array_equal(O.abq_pack_compensated(W, a, b, 8)["Q"], O.abq_pack(W, 8)["Q"])
 
 
-def test_abq_compensation_rounds_the_product_first():
+def test_abq_compensation_rounds_the_product_first(O):
     """The product is rounded before the sum: (1 + 2^-12)^2 = 1 + 2^-11 + 2^-24 rounds (a tie,
     to even) to 1 + 2^-11, so W = -(1 + 2^-11) compensates to exactly 0 (a fused
     multiply-add would leave 2^-24)."""
@@ -551,7 +562,7 @@ def test_abq_compensation_rounds_the_product_first():
     assert Wc[0, 0] == 0.0 and Wc[0, 1] == 1.0
 
 
-def test_abq_compensation_balanced_antisymmetry():
+def test_abq_compensation_balanced_antisymmetry(O):
     """W2* on W' : (W, a) -> (-W, -a) negates W' exactly, so q -> 4 - q with the same Delta."""
     W = I.weights(29, 512, seed=7)
     a, b = I.compensation_vectors(29, 512, seed=7)
@@ -562,7 +573,7 @@ def test_abq_compensation_balanced_antisymmetry():
     assert not np.array_equal(p["Q"], O.abq_pack_balanced(W)["Q"])
 
 
-def test_every_public_oracle_function_states_its_pins():
+def test_every_public_oracle_function_states_its_pins(O):
     """Each public function of the oracle and its layout readers says what pins it (or that its
     parity is unpinned), so an unpinned addition cannot slip in silently."""
     import inspect
