@@ -1,6 +1,7 @@
 // C ABI: host-side validation, buffer layouts and kernel launches.
 #pragma once
 
+#include <cuda.h>  // CUcontext and CUresult types only; the driver calls are resolved at run time
 #include <mutex>
 #include <algorithm>
 #include <cstring>
@@ -176,6 +177,35 @@ inline LayerArgs layer_args(const PkLayout& L, const void* packed, int M, float*
 
 inline uint32_t align128(uint64_t x) { return uint32_t((x + 127) & ~uint64_t(127)); }
 
+// Unique id of the calling thread's current CUDA context (cuCtxGetId), or 0 when there is
+// none or the driver cannot tell. Context ids are never reused within a process, so a context
+// created after cudaDeviceReset, or another context on the same device, has a new id. The two
+// driver entry points are resolved once through the runtime, so the library does not link the
+// driver library (it still loads on a machine without one).
+inline unsigned long long current_context_id() {
+  typedef CUresult (*GetCurrent)(CUcontext*);
+  typedef CUresult (*GetId)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(f);
+    (void)cudaGetLastError();
+  });
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 inline int sm_count() {
   static int n = [] {
     int dev = 0, v = 0;
@@ -282,19 +312,28 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   return true;
 }
 
-// One instantiation per kernel, so the static below tracks that kernel's raised
-// dynamic shared-memory limit (processes drive one device each).
+// One instantiation per kernel, so the statics below track that kernel's raised dynamic
+// shared-memory limit in the context that raised it; a launch in another context (another
+// device, or a context created after a reset) raises it again there.
 template <int FMT, int F0, int F1, int F2, int NW, bool FUSED, bool T1>
 inline cudaError_t launch_tiled_nw(const LayerArgs& g, dim3 grid, cudaStream_t s) {
   auto k = k_layer<FMT, F0, F1, F2, NW, FUSED, T1>;
+  static std::mutex mu;
+  static unsigned long long limit_ctx = 0;
   static uint32_t smem_limit = 48 * 1024;
-  if (g.smem_bytes > smem_limit) {
-    const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(g.smem_bytes));
-    if (e != cudaSuccess) {
-      (void)cudaGetLastError();  // leave no stale error behind
-      return e;
+  if (g.smem_bytes > 48 * 1024) {
+    const unsigned long long ctx = current_context_id();
+    std::lock_guard<std::mutex> lock(mu);
+    if (ctx == 0 || ctx != limit_ctx || g.smem_bytes > smem_limit) {
+      const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(g.smem_bytes));
+      if (e != cudaSuccess) {
+        (void)cudaGetLastError();  // leave no stale error behind
+        return e;
+      }
+      if (ctx != limit_ctx) smem_limit = 48 * 1024;
+      limit_ctx = ctx;
+      smem_limit = std::max(smem_limit, g.smem_bytes);
     }
-    smem_limit = g.smem_bytes;
   }
   return launch_pdl(k, grid, dim3(NW * 32), g.smem_bytes, s, g);
 }
@@ -654,10 +693,16 @@ static __device__ __align__(256) uint8_t g_bq_static_scratch[BQ_STATIC_SCRATCH_B
 namespace {
 constexpr int kMaxDevices = 64;
 
-// Device address of the scratch array on the current device, looked up once per device.
+// Device address of the scratch array in the current context. The address belongs to the
+// context the library's module was loaded into, so it is cached per device together with that
+// context's id, and looked up again (cudaGetSymbolAddress, with the device current) whenever
+// the current context is not the one it was looked up in: after cudaDeviceReset, or under
+// another context on the same device. Without a context id (none current yet, or a driver that
+// cannot tell) it is looked up on every call.
 bq_status static_scratch(void** out) {
   static std::mutex mu;
   static void* addr[kMaxDevices] = {};
+  static unsigned long long ctx_of[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
     (void)cudaGetLastError();
@@ -665,13 +710,15 @@ bq_status static_scratch(void** out) {
   }
   if (dev < 0 || dev >= kMaxDevices) return BQ_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  const unsigned long long ctx = current_context_id();
+  if (!addr[dev] || ctx == 0 || ctx != ctx_of[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_bq_static_scratch) != cudaSuccess || !p) {
       (void)cudaGetLastError();
       return BQ_ERR_CUDA;
     }
     addr[dev] = p;
+    ctx_of[dev] = current_context_id();  // the lookup makes the device's context current
   }
   *out = addr[dev];
   return BQ_OK;

@@ -274,9 +274,13 @@ bq_status bq_linear_group(const bq_layer* layers, int32_t n_layers, const void* 
  *    bq_linear_workspace_bytes(layer, M) > 1 MiB, returns BQ_ERR_SIZE and enqueues
  *    nothing. Only the ternary format with a LoRA term uses scratch, K_pad/256 * M *
  *    rank * 4 bytes: e.g. K = 16384, M = 64, rank = 64 is exactly 1 MiB.
- *  - Setup: the first call on a device looks up the array's device address once
- *    (cudaGetSymbolAddress) and keeps it; a failure there returns BQ_ERR_CUDA. Make
- *    that first call, on each device, before any stream capture begins.
+ *  - Setup: the first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and keeps it together with the
+ *    current context's id; a failure there returns BQ_ERR_CUDA. The address belongs to
+ *    that context, so a call under another context (one created after cudaDeviceReset,
+ *    or a second context on the same device) looks it up again for that context. Make
+ *    the first call on each device, and the first call after any such change of
+ *    context, before any stream capture begins.
  *  - Sharing: every call on a device uses the same array. Nothing in it has to start at
  *    zero: each call writes every scratch word before it reads it. Calls on one stream
  *    are ordered and safe; calls whose work overlaps in time (several streams, or
