@@ -28,7 +28,7 @@ class bq_pack_desc(ctypes.Structure):
                 ("lora_rank", ctypes.c_int32), ("lora_alpha", ctypes.c_float), ("h2", ctypes.c_void_p),
                 ("lora_A", ctypes.c_void_p), ("lora_B", ctypes.c_void_p), ("rabit_svid_rounds", ctypes.c_int32),
                 ("abq_bit_balance", ctypes.c_int32), ("abq_comp_a", ctypes.c_void_p),
-                ("abq_comp_b", ctypes.c_void_p), ("h3", ctypes.c_void_p)]
+                ("abq_comp_b", ctypes.c_void_p), ("h3", ctypes.c_void_p), ("bvsr_cluster_rounds", ctypes.c_int32)]
 
 
 class bq_plan_info(ctypes.Structure):
@@ -75,7 +75,7 @@ for _name, (_res, _args) in _SIGS.items():
 EXPORTED = tuple(_SIGS)
 
 # the struct layouts below are those of this ABI version of include/bq.h
-BQ_ABI_VERSION = 2
+BQ_ABI_VERSION = 3
 if _lib.bq_version() != BQ_ABI_VERSION:
     raise ImportError(f"{LIB_PATH} has ABI version {_lib.bq_version()}, this binding needs {BQ_ABI_VERSION}; "
                       "rebuild it with bit_weight_quantization_b200.build.build(force=True)")
@@ -116,10 +116,11 @@ def bq_version() -> int:
 
 
 def make_desc(fmt, w_bits=0, a_bits=0, lora_rank=0, lora_alpha=0.1, h2=None, lora_A=None, lora_B=None,
-              rabit_svid_rounds=0, abq_bit_balance=0, abq_comp_a=None, abq_comp_b=None, h3=None):
+              rabit_svid_rounds=0, abq_bit_balance=0, abq_comp_a=None, abq_comp_b=None, h3=None,
+              bvsr_cluster_rounds=0):
     return bq_pack_desc(FORMATS.get(fmt, fmt), w_bits, a_bits, lora_rank, lora_alpha,
                         _ptr(h2), _ptr(lora_A), _ptr(lora_B), rabit_svid_rounds, abq_bit_balance,
-                        _ptr(abq_comp_a), _ptr(abq_comp_b), _ptr(h3))
+                        _ptr(abq_comp_a), _ptr(abq_comp_b), _ptr(h3), bvsr_cluster_rounds)
 
 
 def bq_packed_bytes(desc: bq_pack_desc, N: int, K: int) -> int:
@@ -217,11 +218,11 @@ class QuantLinear:
 
     def __init__(self, fmt, W, *, w_bits=0, a_bits=0, lora_rank=0, lora_alpha=0.1, h2=None,
                  lora_A=None, lora_B=None, rabit_svid_rounds=0, abq_bit_balance=0, abq_comp_a=None,
-                 abq_comp_b=None, h3=None, stream=None):
+                 abq_comp_b=None, h3=None, bvsr_cluster_rounds=0, stream=None):
         import torch
         N, K = W.shape
         self.desc = make_desc(fmt, w_bits, a_bits, lora_rank, lora_alpha, h2, lora_A, lora_B, rabit_svid_rounds,
-                              abq_bit_balance, abq_comp_a, abq_comp_b, h3)
+                              abq_bit_balance, abq_comp_a, abq_comp_b, h3, bvsr_cluster_rounds)
         nbytes = bq_packed_bytes(self.desc, N, K)
         self.packed = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
         self.layer = bq_pack_weights(self.desc, W, N, K, self.packed, nbytes, stream)

@@ -28,6 +28,9 @@ inline bq_status check_desc(const bq_pack_desc* d, int K, bool need_ptrs) {
     return BQ_ERR_INVALID_ARG;
   if (d->fmt != BQ_FMT_ABQ && (d->abq_comp_a || d->abq_comp_b)) return BQ_ERR_INVALID_ARG;
   if (d->fmt != BQ_FMT_RABIT3 && d->h3) return BQ_ERR_INVALID_ARG;
+  if (d->bvsr_cluster_rounds != 0 && (d->fmt != BQ_FMT_BVSR4 || d->bvsr_cluster_rounds < 0 ||
+                                      d->bvsr_cluster_rounds > 100))
+    return BQ_ERR_INVALID_ARG;
   switch (d->fmt) {
     case BQ_FMT_RABIT2:
       if (d->rabit_svid_rounds < 0 || d->rabit_svid_rounds > 1000) return BQ_ERR_INVALID_ARG;
@@ -133,8 +136,16 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-// bq_linear scratch: the ternary LoRA partial dot products [KT][M][r] (f32)
+// bq_linear runs an ABQ layer of more than one token as activation quantization into its
+// workspace (an act buffer) followed by the layer from that buffer: the per-token asymmetric
+// codes take a correctly rounded divide per element, which every CTA of the fused kernel would
+// otherwise repeat for its tokens.
+inline bool linear_via_act(const PkLayout& L, int M) { return L.fmt == BQ_FMT_ABQ && M >= 2; }
+
+// bq_linear scratch: the ternary LoRA partial dot products [KT][M][r] (f32), or the act buffer
+// of an ABQ layer of more than one token
 inline uint64_t linear_workspace(const PkLayout& L, int M) {
+  if (linear_via_act(L, M)) return align256(make_act_layout(L, M).total);
   return L.fmt == BQ_FMT_TERNARY_A8 && L.rank > 0 ? align256(uint64_t(L.KT) * M * L.rank * 4) : 0;
 }
 
@@ -229,7 +240,8 @@ inline int pow2ceil(int v) {
 //  - tokens per CTA (tpc): fused, each token group of 256/pow2(tpc) threads holds its x
 //    in at most 16 16-byte chunks per thread; unfused, the code image fits in 96 KB;
 //  - about one CTA per SM, CPG CTAs per token group striding over the row blocks;
-//  - the weight ring gets what is left (at most 96 KB): S >= 2 stages of C tiles per warp.
+//  - the weight ring gets what is left (at most 96 KB), split among the warps that have row
+//    blocks: S (2..4) stages of C tiles per such warp.
 // Returns false when the layer does not fit this kernel.
 inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   constexpr int NW = 8, NT = NW * 32;
@@ -249,7 +261,12 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   }
   g->tpc = tpc;
   g->TG = (M + tpc - 1) / tpc;
-  g->CPG = std::max(1, std::min(L.RB, (sm_count() + g->TG - 1) / g->TG));
+  // BVSR tiles are long latency-bound instruction chains (about 400 instructions a 2176-byte
+  // tile): at one token per CTA, two CTAs of the same launch share each SM so that 16 warps
+  // hide each other's latency; the other formats (and multi-token BVSR, whose code image is
+  // large) keep about one CTA per SM, leaving room for the next launch's.
+  const int ctas_per_sm = bvsr && tpc == 1 ? 2 : 1;
+  g->CPG = std::max(1, std::min(L.RB, (ctas_per_sm * sm_count() + g->TG - 1) / g->TG));
   // Warps sharing a row block (the k-split), a power of two: the one with the least modelled
   // time. Warp w issues on SM sub-partition w % 4, where the MMA and field-mask issue of a
   // tile costs about tile_c cycles (measured: ~145 per 8-MMA stream, ~900 for a BVSR tile);
@@ -286,7 +303,7 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   g->off_tok = take(bqi::kTokWords * 4);  // per-token words, tanh(alpha), weight scale
   g->off_u = take(rank > 0 ? uint64_t(tpc) * rank * 4 : 16);
   g->off_gsum = take(bvsr ? uint64_t(tpc) * VPR * 4 : 16);
-  g->off_tab = take(bvsr ? uint64_t(kBvsrSets) * kBvsrTableStride * 4 : 16);
+  g->off_tab = take(bvsr ? uint64_t(kBvsrSets) * kBvsrTableStride * 4 + 4 * 16 : 16);  // + the family tables
   // split-K exchange [G][2][WPR][32][4] of int64 (+ f32 for BVSR) when warps share a row
   // block; at least the staging reductions' 3 x 32 words
   g->off_red = take(wpr > 1 ? 2ull * NW * 32 * 4 * (bvsr ? 12 : 8) : 512);
@@ -299,13 +316,16 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   // the next launch's CTA is resident, and prefetching its weights, while this one computes;
   // a layer whose ring and fixed part exceed half of the SM runs alone. (Capping every
   // layer at half an SM measured slower on mixed-shape layer sequences.)
-  const uint64_t limit = 220 * 1024;
+  const uint64_t limit = ctas_per_sm == 2 ? 112 * 1024 : 220 * 1024;  // two CTAs share the SM's 228 KB
   const uint64_t budget = std::min<uint64_t>(96 * 1024, fixed < limit ? limit - fixed : 0);
-  const uint64_t per_warp = budget / NW;
+  // The ring is split among the warps that have row blocks: groups 0 .. min(G, ipc) - 1, i.e.
+  // warps 0 .. active - 1 (a CTA never holds more than ipc row blocks); idle warps get none.
+  const int active = std::min(NW / wpr, ipc) * wpr;
+  const uint64_t per_warp = budget / uint64_t(std::max(1, active));
   if (per_warp < 2ull * L.tile_bytes) return false;
   g->S = int(std::min<uint64_t>(4, std::max<uint64_t>(2, per_warp / L.tile_bytes)));
   g->C = int(std::max<uint64_t>(1, std::min<uint64_t>(g->T, per_warp / (uint64_t(g->S) * L.tile_bytes))));
-  g->off_ring = take(uint64_t(NW) * g->S * g->C * L.tile_bytes);
+  g->off_ring = take(uint64_t(std::max(1, active)) * g->S * g->C * L.tile_bytes);
   g->off_bar = take(uint64_t(NW * g->S + 3) * 8 + 16);
   g->smem_bytes = uint32_t(off);
   g->RB = L.RB;
@@ -514,7 +534,21 @@ bq_status bq_pack_weights(const bq_pack_desc* desc, const float* W, int32_t N, i
       k_bvsr_minmax<<<blocks_for(V, 256), 256, 0, s>>>(W, K, V, kmin, kmax);
       const unsigned cb = unsigned(std::min<uint64_t>(blocks_for(V, 256), 148ull * 8));
       for (int bit = 31; bit >= 0; bit--) k_bvsr_count<<<cb, 256, 0, s>>>(kmin, kmax, V, counts, bit);
-      k_bvsr_table<<<1, 256, 0, s>>>(counts, V, table);
+      const int rounds = desc->bvsr_cluster_rounds;
+      double* cen = rounds > 0 ? reinterpret_cast<double*>(P + L.off_aux + kBvsrSets * kBvsrTableStride * 4) : nullptr;
+      k_bvsr_table<<<1, 256, 0, s>>>(counts, V, table, cen);
+      if (rounds > 0) {  // the clustering reading of the coefficient cache
+        unsigned long long* acc = reinterpret_cast<unsigned long long*>(cen + 2 * kBvsrSets);
+        uint8_t* fam = reinterpret_cast<uint8_t*>(kmax + V);  // scratch in the tile region (9 V <= 17 V bytes)
+        k_bvsr_grid_families<<<1, 128, 0, s>>>(cen);
+        k_bvsr_family<<<blocks_for(4 * V, 256), 256, 0, s>>>(W, K, V, fam);
+        for (int r = 0; r < rounds; r++) {
+          if (cudaMemsetAsync(acc, 0, kBvsrSets * 3 * 8, s) != cudaSuccess) return BQ_ERR_CUDA;
+          k_bvsr_assign<<<blocks_for(V, 256), 256, 0, s>>>(kmin, kmax, fam, V, cen, acc);
+          k_bvsr_update<<<1, 256, 0, s>>>(acc, cen);
+        }
+        k_bvsr_cluster_sets<<<1, 256, 0, s>>>(cen, table);
+      }
       if (cudaMemsetAsync(P + L.off_tiles, 0, L.off_rows - L.off_tiles, s) != cudaSuccess) return BQ_ERR_CUDA;
       const unsigned sb = unsigned(std::min<uint64_t>(V, 148ull * 16));
       k_bvsr_search<<<sb, 256, 0, s>>>(W, K, L.KT, V, table, reinterpret_cast<uint32_t*>(P + L.off_tiles));
@@ -673,6 +707,10 @@ bq_status bq_linear(const bq_layer* layer, const void* x_bf16, int32_t M, float*
   const uint64_t need = linear_workspace(L, M);
   if (need > 0 && (!workspace || !aligned(workspace, 256))) return BQ_ERR_INVALID_ARG;
   if (workspace_bytes < need) return BQ_ERR_SIZE;
+  if (linear_via_act(L, M)) {
+    st = bq_quantize_act(layer, x_bf16, M, workspace, workspace_bytes, stream);
+    return st != BQ_OK ? st : bq_gemm(layer, workspace, M, y, acc_dbg, stream);
+  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const uint8_t* P = static_cast<const uint8_t*>(layer->packed);
   LayerArgs g = layer_args(L, layer->packed, M, y, acc_dbg);
@@ -781,7 +819,7 @@ bq_status bq_linear_plan(const bq_layer* layer, int32_t M, int32_t fused, bq_pla
   if (M < 1 || M > BQ_MAX_M) return BQ_ERR_SIZE;
   if (rabit_paths(L.fmt)) return BQ_ERR_UNSUPPORTED;
   LayerArgs g{};
-  if (!plan_layer(L, M, fused != 0, &g)) return BQ_ERR_UNSUPPORTED;
+  if (!plan_layer(L, M, fused != 0 && !linear_via_act(L, M), &g)) return BQ_ERR_UNSUPPORTED;
   info->tokens_per_cta = g.tpc;
   info->token_groups = g.TG;
   info->ctas_per_group = g.CPG;

@@ -714,43 +714,76 @@ __device__ __forceinline__ float small_int_to_float(int v) {
   return __fsub_rn(__int_as_float(int(kRnBias) + v), 12582912.0f);
 }
 
-// One BVSR tile (16 rows x 8 vectors of 32 k) for this lane's outputs. Plane i of vector j
-// is bit j of each byte of w[i]; its dot with the codes, d_i, comes from one int8 MMA
-// (scaled by 2^j). Per row and vector the set s gives the template bytes R (table word 7),
-// o and sc = span / sum R (words 4, 5): y += sc sum_i R_i d_i + o S_v, S_v the vector's
-// code sum. TWO (warp-uniform): the CTA holds more than one token, so outputs c = 1, 3
-// (token 2t + 1) are live too; with one token only c = 0, 2 (token 0, lanes t = 0) carry data.
+// prmt.b32 in its default mode: byte i of the result is byte (s >> 4i) & 7 of the pair
+// {a (bytes 0-3), b (bytes 4-7)}, or, when bit 3 of that selector nibble is set, the sign
+// bit of that byte copied over all eight bits. Only the low 16 bits of s are read.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Per family of coefficient sets (set index >> 6, one geometric ratio each), from its integer
+// template R_0..R_3 (proportional to r^i): lo/hi = the bytes L3(c) = R_0 b_0 + R_1 b_1 + R_2 b_2
+// for c = 0..3 / 4..7 (b_i the bits of c), r3 = R_3 in every byte. All entries are below 128.
+struct BvsrFam {
+  uint32_t lo, hi, r3, pad;
+};
+
+// One BVSR tile (16 rows x 8 vectors of 32 k) for this lane's outputs. For vector j the lane
+// holds two words: the 4-bit codes of A registers a0 (row g) and a1 (row g + 8) in the low and
+// high half of the first, a2 and a3 in the second, nibble b of a half being byte b of the
+// register. With the set's integer template, L(c) = sum_i R_i b_i(c) = L3(c & 7) + R_3 [c >= 8]
+// (at most 203, one u8 byte), and E = sum_k L(code_k) q_k comes exactly from two int8 MMAs:
+// bytes L3(c & 7) (the family table selected by the code with its bit 3 cleared) and bytes
+// R_3 [c >= 8] (R_3 selected with bit 3 flipped, so that codes below 8 copy the sign of
+// R_3 < 128, i.e. 0). Per row and vector the set s gives o and sc = span / sum R (table words
+// 4, 5): y += sc E + o S_v, S_v the vector's code sum. TWO (warp-uniform): the CTA holds more
+// than one token, so outputs c = 1, 3 (token 2t + 1) are live too; with one token only c = 0, 2.
+// want_acc adds sum_k code_k q_k (a third MMA on the code bytes).
 __device__ __forceinline__ void bvsr_tile(const uint4 (&w)[4], const uint4 (&b)[4], uint2 i0, uint2 i1,
-                                          const float* tab, const int* gs_row, int VPR, bool TWO, bool tok0,
-                                          bool tok1, bool want_acc, float (&yacc)[4], long long (&cacc)[4]) {
-  const uint32_t* tabu = reinterpret_cast<const uint32_t*>(tab);
+                                          const float* tab, const BvsrFam* fam, const int* gs_row, int VPR,
+                                          bool TWO, bool tok0, bool tok1, bool want_acc, float (&yacc)[4],
+                                          long long (&cacc)[4]) {
 #pragma unroll
   for (int j = 0; j < 8; j++) {
-    const uint32_t msk = (1u << j) * 0x01010101u;
-    int d[4][4];
-#pragma unroll
-    for (int qq = 0; qq < 4; qq++) {
-      d[qq][0] = d[qq][1] = d[qq][2] = d[qq][3] = 0;
-      mma_u8<true>(d[qq], w[qq].x & msk, w[qq].y & msk, w[qq].z & msk, w[qq].w & msk, bword(b, j, 0), bword(b, j, 1));
-    }
+    const uint4& q = w[j >> 1];
+    const uint32_t w0 = (j & 1) ? q.z : q.x, w1 = (j & 1) ? q.w : q.y;
+    const uint32_t sel[4] = {w0, w0 >> 16, w1, w1 >> 16};  // a0 (row g), a1 (g + 8), a2 (g), a3 (g + 8)
     const int s0 = int(__byte_perm(j < 4 ? i0.x : i0.y, 0, 0x4440 + (j & 3)));
     const int s1 = int(__byte_perm(j < 4 ? i1.x : i1.y, 0, 0x4440 + (j & 3)));
-    const uint32_t R[2] = {tabu[s0 * kBvsrTableStride + 7], tabu[s1 * kBvsrTableStride + 7]};
+    const BvsrFam f0 = fam[s0 >> 6], f1 = fam[s1 >> 6];
+    uint32_t a1[4], a2[4];
+#pragma unroll
+    for (int r = 0; r < 4; r++) {
+      const BvsrFam& f = (r & 1) ? f1 : f0;
+      a1[r] = prmt(f.lo, f.hi, sel[r] & 0x7777u);
+      a2[r] = prmt(f.r3, f.r3, sel[r] ^ 0x8888u);
+    }
+    int d1[4] = {0, 0, 0, 0}, d2[4] = {0, 0, 0, 0};
+    mma_u8<true>(d1, a1[0], a1[1], a1[2], a1[3], bword(b, j, 0), bword(b, j, 1));
+    mma_u8<true>(d2, a2[0], a2[1], a2[2], a2[3], bword(b, j, 0), bword(b, j, 1));
+    if (want_acc) {  // the code bytes: c & 7 plus 8 [c >= 8]
+      uint32_t a3[4];
+#pragma unroll
+      for (int r = 0; r < 4; r++)
+        a3[r] = prmt(0x03020100u, 0x07060504u, sel[r] & 0x7777u) + prmt(0x08080808u, 0x08080808u, sel[r] ^ 0x8888u);
+      int d3[4] = {0, 0, 0, 0};
+      mma_u8<true>(d3, a3[0], a3[1], a3[2], a3[3], bword(b, j, 0), bword(b, j, 1));
+#pragma unroll
+      for (int c = 0; c < 4; c++) cacc[c] += d3[c];
+    }
     const float2 os[2] = {*reinterpret_cast<const float2*>(tab + s0 * kBvsrTableStride + 4),
                           *reinterpret_cast<const float2*>(tab + s1 * kBvsrTableStride + 4)};
     const float gsf[2] = {tok0 ? small_int_to_float(gs_row[j]) : 0.f,
                           TWO && tok1 ? small_int_to_float(gs_row[VPR + j]) : 0.f};
 #pragma unroll
     for (int h = 0; h < 2; h++) {  // row g (h = 0) or g + 8
-      const int r0 = int(R[h] & 0xFFu), r1 = int(__byte_perm(R[h], 0, 0x4441)), r2 = int(__byte_perm(R[h], 0, 0x4442)),
-                r3 = int(R[h] >> 24);
 #pragma unroll
-      for (int q = 0; q < 2; q++) {
-        if (q == 1 && !TWO) break;  // warp-uniform
-        const int c = 2 * h + q;
-        const int E = (r0 * d[0][c] + r1 * d[1][c] + r2 * d[2][c] + r3 * d[3][c]) >> j;
-        yacc[c] = fmaf(os[h].y, small_int_to_float(E), fmaf(os[h].x, gsf[q], yacc[c]));
-        if (want_acc) cacc[c] += (d[0][c] + 2 * d[1][c] + 4 * d[2][c] + 8 * d[3][c]) >> j;
+      for (int qq = 0; qq < 2; qq++) {
+        if (qq == 1 && !TWO) break;  // warp-uniform
+        const int c = 2 * h + qq;
+        yacc[c] = fmaf(os[h].y, small_int_to_float(d1[c] + d2[c]), fmaf(os[h].x, gsf[qq], yacc[c]));
       }
     }
   }
@@ -866,7 +899,20 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
     if (ok) stage_lora_u(a, smem, m0, mg, NW * 32);
     __syncthreads();
   }
-  if (BVSR && !mbar_wait_bounded(tbar, 0)) ok = false;
+  if (BVSR) {
+    if (!mbar_wait_bounded(tbar, 0)) ok = false;
+    // the four families' lookup tables, from the templates of sets 0, 64, 128, 192 (word 7)
+    if (tid < 4 && ok) {
+      const uint32_t R = reinterpret_cast<const uint32_t*>(smem + a.off_tab)[(64 * tid) * kBvsrTableStride + 7];
+      const uint32_t r0 = R & 0xFFu, r1 = (R >> 8) & 0xFFu, r2 = (R >> 16) & 0xFFu, r3 = R >> 24;
+      BvsrFam* fw = reinterpret_cast<BvsrFam*>(smem + a.off_tab + kBvsrSets * kBvsrTableStride * 4);
+      fw[tid].lo = (r0 << 8) | (r1 << 16) | ((r0 + r1) << 24);
+      fw[tid].hi = r2 | ((r2 + r0) << 8) | ((r2 + r1) << 16) | ((r2 + r1 + r0) << 24);
+      fw[tid].r3 = r3 * 0x01010101u;
+      fw[tid].pad = 0;
+    }
+    __syncthreads();
+  }
   if (LBT && !mbar_wait_bounded(lbar, 0)) ok = false;
 
   const bool has_tok = g < mg;
@@ -874,6 +920,7 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
   const int VPR = a.K_pad / 32;
   const int* gsum = reinterpret_cast<const int*>(smem + a.off_gsum);
   const float* tab = reinterpret_cast<const float*>(smem + a.off_tab);
+  const BvsrFam* fam = reinterpret_cast<const BvsrFam*>(smem + a.off_tab + kBvsrSets * kBvsrTableStride * 4);
   const bool want_acc = a.gl[0].acc != nullptr;  // BVSR (never grouped)
   long long* redl = reinterpret_cast<long long*>(smem + a.off_red);                // [G][2][WPR][32][4]
   float* redf = reinterpret_cast<float*>(smem + a.off_red + 2 * NW * 32 * 4 * 8);  // same shape
@@ -940,7 +987,7 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
             const uint8_t* tidx = tp - lane * 16 + 2048;
             const uint2 i0 = *reinterpret_cast<const uint2*>(tidx + g * 8);
             const uint2 i1 = *reinterpret_cast<const uint2*>(tidx + (g + 8) * 8);
-            bvsr_tile(w, b, i0, i1, tab, gsum + size_t(2 * t) * VPR + kt * 8, VPR, mg > 1, 2 * t < mg,
+            bvsr_tile(w, b, i0, i1, tab, fam, gsum + size_t(2 * t) * VPR + kt * 8, VPR, mg > 1, 2 * t < mg,
                       2 * t + 1 < mg, want_acc, yacc, cacc);
           }
         }

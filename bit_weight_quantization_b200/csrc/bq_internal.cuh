@@ -35,6 +35,8 @@ enum : int {
 constexpr int kBvsrSets = 256;
 constexpr int kBvsrTableStride = 8;  // words per set: c0 c1 c2 c3 o sc ratio_index, R bytes (u32)
 constexpr int kBvsrTileBytes = 4 * 512 + 16 * 8;
+// after the table: clustering centroids f64 [256][2] and their int64 sums [256][3]
+constexpr int kBvsrPackScratch = kBvsrSets * 2 * 8 + kBvsrSets * 3 * 8;
 
 struct PkLayout {
   int fmt, N, K, N_pad, K_pad, RB, KT, w_bits, a_bits, nstreams;
@@ -102,10 +104,11 @@ inline bool make_pk_layout(int fmt, int N, int K, int w_bits, int a_bits, int ra
       break;
     }
     case BQ_FMT_BVSR4:
-      l.w_bits = 4; l.a_bits = 8; l.nstreams = 4;
-      for (int s = 0; s < 4; s++) { l.field[s] = 1; l.shift[s] = s; }
-      l.tile_bytes = kBvsrTileBytes;  // 4 planes x 512 B, then the 16 x 8 set indices
-      aux = uint64_t(kBvsrSets) * kBvsrTableStride * 4;
+      // one stream of 4-bit codes in the nibble order of the BVSR tile (not the generic
+      // field order), then the 16 x 8 set indices
+      l.w_bits = 4; l.a_bits = 8; l.nstreams = 1; l.field[0] = 4; l.shift[0] = 0;
+      l.tile_bytes = kBvsrTileBytes;
+      aux = uint64_t(kBvsrSets) * kBvsrTableStride * 4 + kBvsrPackScratch;
       break;
     default:
       return false;

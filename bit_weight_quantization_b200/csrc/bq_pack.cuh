@@ -420,8 +420,30 @@ __global__ void k_bvsr_count(const uint32_t* __restrict__ kmin, const uint32_t* 
   }
 }
 
-// One block of 256 threads: set s = 64j + 8a + b.
-__global__ void k_bvsr_table(const uint32_t* counts_in, uint64_t V, float* table) {
+// Table row of a set of family j on the range [lo, hi] (set s = 64j + c): c_i = (hi - lo) t_i with
+// t_i = r^i / sum r^i' (float64, stored float32), o = lo; then the kernel's derived constants
+// sc = (hi - lo) / sum R, the family index and the integer templates R_0..R_3 as bytes of one
+// word: {8,12,18,27} {1,2,4,8} {8,20,50,125} {1,3,9,27}.
+__device__ __forceinline__ void bvsr_set_row(float* row, int j, double lo, double hi) {
+  const double r = 1.5 + 0.5 * j;
+  const double pw[4] = {1.0, r, r * r, r * r * r};
+  const double tsum = __dadd_rn(__dadd_rn(__dadd_rn(pw[0], pw[1]), pw[2]), pw[3]);
+  const double span = __dsub_rn(hi, lo);
+  for (int i = 0; i < 4; i++) row[i] = __double2float_rn(__dmul_rn(span, __ddiv_rn(pw[i], tsum)));
+  row[4] = __double2float_rn(lo);
+  const double rsum[4] = {65.0, 15.0, 203.0, 40.0};
+  row[5] = __double2float_rn(__ddiv_rn(span, rsum[j]));
+  row[6] = float(j);
+  const uint32_t rword[4] = {0x1B120C08u, 0x08040201u, 0x7D321408u, 0x1B090301u};
+  row[7] = __uint_as_float(rword[j]);
+}
+__device__ __forceinline__ void bvsr_write_set(float* table, int s, double lo, double hi) {
+  bvsr_set_row(table + s * kBvsrTableStride, s >> 6, lo, hi);
+}
+
+// One block of 256 threads: set s = 64j + 8a + b on the quantile grid (lo_a, hi_b). With
+// `grid` (the clustering pack) also the grid itself, grid[8a + b] = (lo_a, hi_b) in float64.
+__global__ void k_bvsr_table(const uint32_t* counts_in, uint64_t V, float* table, double* grid) {
   __shared__ uint32_t cnt[32 * 16];
   __shared__ float lo[8], hi[8];
   for (int i = threadIdx.x; i < 32 * 16; i += blockDim.x) cnt[i] = counts_in[i];
@@ -431,22 +453,12 @@ __global__ void k_bvsr_table(const uint32_t* counts_in, uint64_t V, float* table
     if (threadIdx.x < 8) lo[threadIdx.x] = v; else hi[threadIdx.x - 8] = v;
   }
   __syncthreads();
-  const int s = threadIdx.x;
-  const int j = s >> 6, a = (s >> 3) & 7, b = s & 7;
-  const double r = 1.5 + 0.5 * j;
-  const double pw[4] = {1.0, r, r * r, r * r * r};
-  const double tsum = __dadd_rn(__dadd_rn(__dadd_rn(pw[0], pw[1]), pw[2]), pw[3]);
-  const double span = __dsub_rn(double(hi[b]), double(lo[a]));
-  float* row = table + s * kBvsrTableStride;
-  for (int i = 0; i < 4; i++) row[i] = __double2float_rn(__dmul_rn(span, __ddiv_rn(pw[i], tsum)));
-  row[4] = lo[a];
-  // derived kernel constants: c_i = (hi - lo) R_i / sum R for the integer templates R
-  const double rsum[4] = {65.0, 15.0, 203.0, 40.0};
-  row[5] = __double2float_rn(__ddiv_rn(span, rsum[j]));
-  row[6] = float(j);
-  // the integer templates R_i as bytes of one word: {8,12,18,27} {1,2,4,8} {8,20,50,125} {1,3,9,27}
-  const uint32_t rword[4] = {0x1B120C08u, 0x08040201u, 0x7D321408u, 0x1B090301u};
-  row[7] = __uint_as_float(rword[j]);
+  const int s = threadIdx.x, a = (s >> 3) & 7, b = s & 7;
+  bvsr_write_set(table, s, double(lo[a]), double(hi[b]));
+  if (grid && s < 64) {
+    grid[2 * s] = double(lo[a]);
+    grid[2 * s + 1] = double(hi[b]);
+  }
 }
 
 // Points of set s, o + c0 b0 + c1 b1 + c2 b2 + c3 b3 summed left to right in float64.
@@ -530,24 +542,119 @@ __global__ void __launch_bounds__(256) k_bvsr_search(const float* __restrict__ W
       bvsr_points(table + sbest * kBvsrTableStride, Pb);
       double p;
       const int code = bvsr_nearest(double(wv[lane]), Pb, &p);
-      // tile position of element e = lane of vector (n, kv)
+      // tile position of element e = lane of vector (n, kv): word 2(j & 1) + (e >> 4) of lane
+      // 4g + t in block j >> 1, nibble b of its low (row g) or high (row g + 8) half
       const int rb = int(n >> 4), rho = int(n & 15), g = rho & 7, rbit = rho >> 3;
       const int kt = kv >> 3, j = kv & 7;
-      const int e = lane, rh = e >> 4, t = (e >> 2) & 3, b = e & 3;
-      const int r = 2 * rh + rbit, tl = 4 * g + t;
+      const int e = lane, hk = e >> 4, t = (e >> 2) & 3, b = e & 3;
       const uint64_t tile_w = (uint64_t(rb) * KT + kt) * (kBvsrTileBytes / 4);
-      const uint64_t base_w = tile_w + tl * 4 + r;
-#pragma unroll
-      for (int i = 0; i < 4; i++) {
-        uint32_t val = uint32_t((code >> i) & 1) << (8 * b + j);
-        val |= __shfl_xor_sync(0xffffffffu, val, 1);
-        val |= __shfl_xor_sync(0xffffffffu, val, 2);
-        if (b == 0 && val) atomicOr(&tiles32[base_w + i * 128], val);
-      }
+      const uint64_t word = tile_w + uint64_t((j >> 1) * 32 + 4 * g + t) * 4 + 2 * (j & 1) + hk;
+      uint32_t val = uint32_t(code) << (16 * rbit + 4 * b);
+      val |= __shfl_xor_sync(0xffffffffu, val, 1);
+      val |= __shfl_xor_sync(0xffffffffu, val, 2);
+      if (b == 0 && val) atomicOr(&tiles32[word], val);  // rows g and g + 8 share the word
       // set index of (row rho, vector j of the tile) at byte 2048 + 8 rho + j of the tile
       if (lane == 0) reinterpret_cast<uint8_t*>(tiles32 + tile_w)[2048 + rho * 8 + j] = uint8_t(sbest);
     }
   }
+}
+
+// ---------------------------------------------------------------------------
+// BVSR coefficient cache, clustering reading ("BVSR" page, Introduction): per-vector ratio
+// family on the vector's own range, then per family Lloyd k-means of the vectors' (min, max)
+// into 64 centroids started from the quantile grid; centroid means are exact (fixed-point
+// int64 sums of rn(v 2^40), so the atomic accumulation order does not matter).
+// ---------------------------------------------------------------------------
+constexpr double kBvsrFix = 1099511627776.0;              // 2^40
+constexpr double kBvsrUnfix = 9.094947017729282379150390625e-13;  // 2^-40
+
+// Per vector (4 threads, one per family): the family j whose set on the vector's own range
+// [min, max] (bvsr_write_set's c_i and o) gives the least squared error (nearest of 16 points per
+// element, the lowest code on a tie, errors added in element order); the lowest j on a tie.
+__global__ void __launch_bounds__(256) k_bvsr_family(const float* __restrict__ W, int K, uint64_t V,
+                                                     uint8_t* __restrict__ fam) {
+  const uint64_t gid = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const uint64_t v = gid >> 2;
+  const int j = int(gid & 3);
+  const bool live = v < V;
+  const int vpr = K / 32;
+  double err = INFINITY;
+  if (live) {
+    const float* w = W + (v / vpr) * uint64_t(K) + uint64_t(v % vpr) * 32;
+    float lo = w[0], hi = w[0];
+    for (int e = 1; e < 32; e++) { lo = fminf(lo, w[e]); hi = fmaxf(hi, w[e]); }
+    float row[kBvsrTableStride];
+    bvsr_set_row(row, j, double(lo), double(hi));
+    double P[16];
+    bvsr_points(row, P);
+    err = 0.0;
+    for (int e = 0; e < 32; e++) {
+      const double we = double(w[e]);
+      double p;
+      bvsr_nearest(we, P, &p);
+      const double de = __dsub_rn(we, p);
+      err = __dadd_rn(err, __dmul_rn(de, de));
+    }
+  }
+  // lowest error among the vector's 4 lanes, the lowest family on a tie
+  int bj = j;
+  double be = err;
+#pragma unroll
+  for (int o = 1; o < 4; o <<= 1) {
+    const double e2 = __shfl_xor_sync(0xffffffffu, be, o);
+    const int j2 = __shfl_xor_sync(0xffffffffu, bj, o);
+    if (e2 < be || (e2 == be && j2 < bj)) { be = e2; bj = j2; }
+  }
+  if (live && j == 0) fam[v] = uint8_t(bj);
+}
+
+// One k-means round's assignment: each vector to the nearest of its family's 64 centroids
+// (squared distance in float64, the lowest index on a tie), adding rn(v 2^40) of its min and
+// max and a count to that cluster's int64 sums (acc [256][3], zeroed before the round).
+__global__ void __launch_bounds__(256) k_bvsr_assign(const uint32_t* __restrict__ kmin,
+                                                     const uint32_t* __restrict__ kmax,
+                                                     const uint8_t* __restrict__ fam, uint64_t V,
+                                                     const double* __restrict__ cen,
+                                                     unsigned long long* __restrict__ acc) {
+  const uint64_t v = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (v >= V) return;
+  const int j = fam[v];
+  const double lo = double(key_float(kmin[v])), hi = double(key_float(kmax[v]));
+  const double* c = cen + 2 * 64 * j;
+  int bc = 0;
+  double bd = 0.0;
+  for (int k = 0; k < 64; k++) {
+    const double dl = __dsub_rn(lo, c[2 * k]), dh = __dsub_rn(hi, c[2 * k + 1]);
+    const double d = __dadd_rn(__dmul_rn(dl, dl), __dmul_rn(dh, dh));
+    if (k == 0 || d < bd) { bd = d; bc = k; }
+  }
+  unsigned long long* a = acc + 3 * (64 * j + bc);
+  atomicAdd(&a[0], (unsigned long long)__double2ll_rn(__dmul_rn(lo, kBvsrFix)));
+  atomicAdd(&a[1], (unsigned long long)__double2ll_rn(__dmul_rn(hi, kBvsrFix)));
+  atomicAdd(&a[2], 1ull);
+}
+
+// Centroid update (256 threads, one per cluster of the four families): the exact mean of the
+// round's members, sum / count / 2^40 in float64; a cluster without members keeps its centroid.
+__global__ void k_bvsr_update(const unsigned long long* __restrict__ acc, double* __restrict__ cen) {
+  const int s = threadIdx.x;
+  const long long n = (long long)acc[3 * s + 2];
+  if (n <= 0) return;
+  const double dn = __ll2double_rn(n);
+  cen[2 * s] = __dmul_rn(__ddiv_rn(__ll2double_rn((long long)acc[3 * s]), dn), kBvsrUnfix);
+  cen[2 * s + 1] = __dmul_rn(__ddiv_rn(__ll2double_rn((long long)acc[3 * s + 1]), dn), kBvsrUnfix);
+}
+
+// The clustered table: set s = 64j + c on centroid c of family j (256 threads).
+__global__ void k_bvsr_cluster_sets(const double* __restrict__ cen, float* __restrict__ table) {
+  const int s = threadIdx.x;
+  bvsr_write_set(table, s, cen[2 * s], cen[2 * s + 1]);
+}
+
+// Every family starts from the same quantile grid: copy grid [64][2] into families 1..3.
+__global__ void k_bvsr_grid_families(double* cen) {
+  const int i = threadIdx.x;  // 0 .. 127
+  for (int j = 1; j < 4; j++) cen[2 * 64 * j + i] = cen[i];
 }
 
 }  // namespace bqi

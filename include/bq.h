@@ -70,9 +70,15 @@
  *   Padding rows/columns hold zero fields (ternary: field 1, i.e. T = 0).
  *   Streams: BitNet 1 x f=1 (bit set <=> sign -1). Ternary 1 x f=2 (field = T+1 in {0,1,2}).
  *   ABQ: w_bits split into fields of 8/4/2/1 bits from the low end (2:[2] 4:[4] 6:[4,2]
- *   8:[8], shift = bit offset in the code). BVSR: 4 x f=1, stream i = bitvector plane i,
- *   and each BVSR tile ends with 128 bytes of set indices: byte 2048 + 8g + j is the set of
- *   row 16rb + g, vector 8kt + j (a vector is 32 contiguous k), so tile_bytes = 2176.
+ *   8:[8], shift = bit offset in the code). BVSR: one stream (n_streams 1, f = 4, shift 0)
+ *   of 4-bit codes (code = sum_i 2^i b_i over the four bitvectors) in its own nibble order:
+ *   2048 bytes as 4 blocks i of [lane < 32][4 words]; word 2v + h of lane 4g+t in block i
+ *   holds vector j = 2i + v of the tile, nibble b of its low half the code of row 16rb + g
+ *   and nibble b of its high half that of row 16rb + g + 8, at k = 256kt + 32j + 16h + 4t + b
+ *   (the four halves of a lane's two words are the four A registers of the vector's MMA, one
+ *   nibble per byte). Each BVSR tile ends with 128 bytes of set indices: byte 2048 + 8g + j
+ *   (g < 16) is the set of row 16rb + g, vector 8kt + j (a vector is 32 contiguous k), so
+ *   tile_bytes = 2176.
  * RaBiT (formats 1 and 6, P = 2 and 3 paths) is not tiled: bit j of uint32
  *   off_tiles + 4((p*N_pad + n)(K_pad/32) + w) is the sign of path p (0..P-1), row n,
  *   k = 32w + j (1 <=> -1).
@@ -82,7 +88,8 @@
  *   ABQ rows = Delta_w f32 [N_pad], z_w i32 [N_pad], S_w = sum_k q_w i32 [N_pad].
  *   BVSR aux = coefficient table f32 [256][8] (c0 c1 c2 c3 o; then derived kernel constants:
  *   sc = (hi-lo)/sum_i R_i, ratio index, and word 7 the integer templates R_0..R_3 as the
- *   bytes of a uint32, low byte first).
+ *   bytes of a uint32, low byte first), then 10240 bytes of pack scratch (the clustering
+ *   centroids f64 [256][2] and sums i64 [256][3]) that the layer never reads.
  *
  * Activation buffer (device, 256-byte aligned), version 1.
  * Header: 64 x 32-bit words: 0 magic 0x43415142 ('BQAC') 1 version 2 format 3 M 4 K 5 K_pad
@@ -169,6 +176,13 @@ typedef struct {
   const float* h3;      /* RaBiT three paths (format 6): device f32 [K], the third path's input
                            scale (h1 = 1; h2 is required too). Format 6 runs the residual
                            recursion only (rabit_svid_rounds = 0). NULL for every other format. */
+  int32_t bvsr_cluster_rounds;  /* BVSR coefficient cache ("BVSR" page, Introduction), clustering
+                           reading: 0 = the 256 sets on the quantile grid; R in 1..100 = the sets
+                           from R rounds of Lloyd's k-means: every vector takes the ratio family
+                           whose set on its own [min, max] fits it best, and per family the
+                           vectors' (min, max) points are clustered into 64 centroids started
+                           from the quantile grid (exact means: int64 sums of rn(v 2^40)); set
+                           64j + c spans centroid c. Must be 0 for the other formats. */
 } bq_pack_desc;
 
 /* Host-side description of a packed layer; filled by bq_pack_weights or
@@ -185,9 +199,12 @@ typedef struct {
 
 /* ABI version: bumped whenever a struct layout or a call's meaning changes. A caller
  * compares bq_version() with the BQ_ABI_VERSION of the header it was built against.
- * 2: bq_pack_desc gained abq_comp_a, abq_comp_b and h3; format 6 (BQ_FMT_RABIT3). The
- * buffer formats keep their own version word (1): no existing layout changed. */
-#define BQ_ABI_VERSION 2
+ * 2: bq_pack_desc gained abq_comp_a, abq_comp_b and h3; format 6 (BQ_FMT_RABIT3).
+ * 3: bq_pack_desc gained bvsr_cluster_rounds; the BVSR tile holds 4-bit codes in nibble order
+ * (one stream) and its aux section 10 KB of pack scratch after the table; bq_linear on ABQ
+ * with M >= 2 takes an act buffer in its workspace. The buffer version word stays 1 (a BVSR
+ * buffer of the earlier layout has 4 streams in its header and is refused). */
+#define BQ_ABI_VERSION 3
 
 const char* bq_status_str(bq_status s);
 int32_t bq_version(void);
@@ -237,8 +254,10 @@ bq_status bq_gemm(const bq_layer* layer, const void* act, int32_t M, float* y,
 /* Fused layer for decode: the activation quantization of bq_quantize_act runs inside the
  * layer kernel's prologue, so y [M][N] f32 comes from x (device bf16 [M][K], 16-byte
  * aligned) in one launch (two for the ternary format with a LoRA term, whose
- * partial dot products of x and A are computed first into `workspace`). Results are identical to
- * bq_quantize_act + bq_gemm. `workspace` (device, 256-byte aligned) must hold
+ * partial dot products of x and A are computed first into `workspace`; and two for ABQ with
+ * M >= 2, which quantizes the activations once into an act buffer in `workspace` and runs the
+ * layer from it, since its per-element divides would otherwise be repeated by every CTA).
+ * Results are identical to bq_quantize_act + bq_gemm. `workspace` (device, 256-byte aligned) must hold
  * bq_linear_workspace_bytes(layer, M) bytes; it may be NULL when that is 0.
  * Launched with programmatic dependent launch: consecutive layer calls on one stream
  * overlap the next layer's weight fetch with the current layer. */
@@ -272,8 +291,9 @@ bq_status bq_linear_group(const bq_layer* layers, int32_t n_layers, const void* 
  * Same arguments and results as bq_linear, without workspace and workspace_bytes.
  *  - Scratch limit: BQ_STATIC_SCRATCH_BYTES (1 MiB). A call needing more, that is
  *    bq_linear_workspace_bytes(layer, M) > 1 MiB, returns BQ_ERR_SIZE and enqueues
- *    nothing. Only the ternary format with a LoRA term uses scratch, K_pad/256 * M *
- *    rank * 4 bytes: e.g. K = 16384, M = 64, rank = 64 is exactly 1 MiB.
+ *    nothing. Two cases use scratch: the ternary format with a LoRA term, K_pad/256 * M *
+ *    rank * 4 bytes (e.g. K = 16384, M = 64, rank = 64 is exactly 1 MiB), and ABQ with
+ *    M >= 2, its act buffer of about M * K_pad bytes (e.g. K = 4096, M = 64: 263 KiB).
  *  - Setup: the first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current) and keeps it together with the
  *    current context's id; a failure there returns BQ_ERR_CUDA. The address belongs to

@@ -518,6 +518,79 @@ def bvsr_set_table(W) -> np.ndarray:
     return table
 
 
+def bvsr_cluster_table(W, rounds: int) -> dict:
+    """[BVSR] Introduction: the coefficient sets are shared across weight vectors by a selection
+    step the page calls the coefficient cache. Clustering reading (the page gives no procedure):
+      1. every vector takes lo = min, hi = max and the ratio family j whose set on its own range
+         (c = (hi - lo) t_j, o = lo, float32) gives it the least squared error (lowest j on a tie);
+      2. per family, Lloyd's k-means of the vectors' (lo, hi) into 64 centroids, started from the
+         8 x 8 quantile grid of bvsr_set_table (centroid 8a + b = (lo_a, hi_b)): each round assigns
+         every point to the nearest centroid (squared distance, float64, lowest index on a tie) and
+         moves each centroid with points to their mean, sum(rn(v 2^40)) / count / 2^40 with the
+         sum in int64 (exact, order-free); a centroid without points stays;
+      3. set 64 j + c: c_i = (hi_c - lo_c) t_{j,i}, o = lo_c, float32. rounds = 0 is bvsr_set_table.
+    Returns table [256,5], family [V], assign [V] (0 without rounds), centroids [4,64,2].
+    Parity unpinned as a reading; pinned by tests (rounds = 0 is bvsr_set_table, the k-means
+    objective never grows, brute-force family choice, a hand case of exact clusters)."""
+    W = _f32(W)
+    N, K = W.shape
+    vecs = W.reshape(-1, BVSR_VEC)
+    V = vecs.shape[0]
+    lo, hi = vecs.min(axis=1), vecs.max(axis=1)
+    smin, smax = np.sort(lo.astype(np.float64)), np.sort(hi.astype(np.float64))
+    los = [np.float64(nearest_rank(smin, 2 * a + 1, 16)) for a in range(BVSR_GRID)]
+    his = [np.float64(nearest_rank(smax, 2 * b + 1, 16)) for b in range(BVSR_GRID)]
+    temps = []
+    for r in BVSR_RATIOS:
+        pw = [r ** i for i in range(BVSR_PLANES)]
+        temps.append([pw[i] / sum(pw) for i in range(BVSR_PLANES)])
+    span = hi.astype(np.float64) - lo.astype(np.float64)
+    errs = np.zeros((len(BVSR_RATIOS), V))
+    for j, t in enumerate(temps):
+        sets = np.zeros((V, 5), np.float32)
+        for i in range(BVSR_PLANES):
+            sets[:, i] = (span * t[i]).astype(np.float32)
+        sets[:, 4] = lo
+        P = bvsr_points(sets)                                          # [V,16]
+        w = vecs.astype(np.float64)
+        best = np.argmin(np.abs(w[:, :, None] - P[:, None, :]), axis=2)  # [V,32]
+        pb = np.take_along_axis(P, best, axis=1)
+        e = np.zeros(V)
+        for k in range(BVSR_VEC):
+            d = w[:, k] - pb[:, k]
+            e = e + d * d
+        errs[j] = e
+    fam = np.argmin(errs, axis=0).astype(np.uint8)
+    cen = np.zeros((4, 64, 2))
+    for a in range(BVSR_GRID):
+        for b in range(BVSR_GRID):
+            cen[:, 8 * a + b] = (los[a], his[b])
+    asg = np.zeros(V, np.uint8)
+    fx = lambda v: np.rint(np.ldexp(v.astype(np.float64), 40)).astype(np.int64)
+    flo, fhi = fx(lo), fx(hi)
+    for _ in range(rounds):
+        c = cen[fam]                                                   # [V,64,2]
+        d = (lo.astype(np.float64)[:, None] - c[:, :, 0]) ** 2 + (hi.astype(np.float64)[:, None] - c[:, :, 1]) ** 2
+        asg = np.argmin(d, axis=1).astype(np.uint8)
+        idx = fam.astype(np.int64) * 64 + asg
+        sl = np.zeros(256, np.int64); sh = np.zeros(256, np.int64); cnt = np.zeros(256, np.int64)
+        np.add.at(sl, idx, flo); np.add.at(sh, idx, fhi); np.add.at(cnt, idx, 1)
+        has = cnt > 0
+        flat = cen.reshape(256, 2)
+        flat[has, 0] = np.ldexp(sl[has].astype(np.float64) / cnt[has], -40)
+        flat[has, 1] = np.ldexp(sh[has].astype(np.float64) / cnt[has], -40)
+        cen = flat.reshape(4, 64, 2)
+    table = np.zeros((256, 5), np.float32)
+    for j, t in enumerate(temps):
+        for c in range(64):
+            s = 64 * j + c
+            sp = cen[j, c, 1] - cen[j, c, 0]
+            for i in range(BVSR_PLANES):
+                table[s, i] = np.float32(sp * t[i])
+            table[s, 4] = np.float32(cen[j, c, 0])
+    return dict(table=table, family=fam, assign=asg, centroids=cen)
+
+
 def bvsr_points(table) -> np.ndarray:
     """P[s, code] = o + c0 b0 + c1 b1 + c2 b2 + c3 b3 (b_i = bit i of code),
     summed left to right in float64 from the float32 coefficients.
@@ -563,7 +636,7 @@ def bvsr_encode_vectors(vecs, table) -> tuple[np.ndarray, np.ndarray]:
     return codes_out, sets_out
 
 
-def bvsr_pack(W, table=None, rows=None) -> dict:
+def bvsr_pack(W, table=None, rows=None, cluster_rounds: int = 0) -> dict:
     """BVSR 4-bit pack of W [N,K] (K % 32 == 0). ``rows`` restricts the
     encoding to a subset of rows (the table still comes from the whole W).
     Returns codes uint8 [R,K], set index uint8 [R,K/32], table [256,5].
@@ -571,7 +644,7 @@ def bvsr_pack(W, table=None, rows=None) -> dict:
     W = _f32(W)
     N, K = W.shape
     if table is None:
-        table = bvsr_set_table(W)
+        table = bvsr_cluster_table(W, cluster_rounds)["table"] if cluster_rounds > 0 else bvsr_set_table(W)
     sel = np.arange(N) if rows is None else np.asarray(rows)
     sub = W[sel]
     codes, sets = bvsr_encode_vectors(sub.reshape(-1, BVSR_VEC), table)

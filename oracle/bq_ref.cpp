@@ -614,6 +614,162 @@ int bqref_bvsr_set_table(const float* W, int64_t N, int64_t K, float* table) {
   return 0;
 }
 
+int bqref_bvsr_points(const float* table, int S, double* P);
+
+// The quantile grid of bqref_bvsr_set_table as its raw (lo_a, hi_b) pairs: grid[8a + b] =
+// (lo_a, hi_b), float64 copies of float32 quantiles.
+static void bvsr_grid(const float* W, int64_t N, int64_t K, double* grid) {
+  const int64_t V = N * (K / kVec);
+  std::vector<double> mins(static_cast<size_t>(V)), maxs(static_cast<size_t>(V));
+  for (int64_t v = 0; v < V; v++) {
+    const float* e = W + v * kVec;
+    float lo = e[0], hi = e[0];
+    for (int i = 1; i < kVec; i++) {
+      lo = std::min(lo, e[i]);
+      hi = std::max(hi, e[i]);
+    }
+    mins[size_t(v)] = lo;
+    maxs[size_t(v)] = hi;
+  }
+  std::sort(mins.begin(), mins.end());
+  std::sort(maxs.begin(), maxs.end());
+  for (int a = 0; a < kGrid; a++)
+    for (int b = 0; b < kGrid; b++) {
+      bqref_nearest_rank(mins.data(), V, 2 * a + 1, 16, &grid[2 * (8 * a + b)]);
+      bqref_nearest_rank(maxs.data(), V, 2 * b + 1, 16, &grid[2 * (8 * a + b) + 1]);
+    }
+}
+
+// Templates t_i = r^i / sum_i' r^i' of family j (ratio r_j), float64.
+static void bvsr_templates(int j, double t[kPlanes]) {
+  double pw[kPlanes], tsum = 0.0;
+  for (int i = 0; i < kPlanes; i++) {
+    pw[i] = 1.0;
+    for (int e = 0; e < i; e++) pw[i] *= kRatios[j];
+    tsum += pw[i];
+  }
+  for (int i = 0; i < kPlanes; i++) t[i] = pw[i] / tsum;
+}
+
+// Set (c_0..c_3, o) of family j on the range [lo, hi]: c_i = (hi - lo) t_i and o = lo, stored
+// float32 (the construction of every cached set).
+static void bvsr_make_set(int j, double lo, double hi, float* row5) {
+  double t[kPlanes];
+  bvsr_templates(j, t);
+  const double span = hi - lo;
+  for (int i = 0; i < kPlanes; i++) row5[i] = float(span * t[i]);
+  row5[4] = float(lo);
+}
+
+// Squared error of one vector under one set (nearest of its 16 points per element, the lowest
+// code on a tie; errors added in element order, float64).
+static double bvsr_vector_error(const float* w, const float* row5) {
+  double P[16];
+  bqref_bvsr_points(row5, 1, P);
+  double err = 0.0;
+  for (int e = 0; e < kVec; e++) {
+    const double we = double(w[e]);
+    int bc = 0;
+    double bd = std::fabs(we - P[0]);
+    for (int c = 1; c < 16; c++) {
+      const double d = std::fabs(we - P[c]);
+      if (d < bd) { bd = d; bc = c; }
+    }
+    const double de = we - P[bc];
+    err = err + de * de;
+  }
+  return err;
+}
+
+// Fixed-point value of a vector extreme for the cluster sums: round-to-nearest of v 2^40 (the
+// scaling is exact), so that sums of any number of them are exact and independent of order.
+static int64_t bvsr_fix(float v) { return std::llrint(std::ldexp(double(v), 40)); }
+
+// [BVSR] Introduction, coefficient cache: the sets are shared by many weight vectors through a
+// selection step the page calls the coefficient cache. Clustering reading (the page gives no
+// procedure; every step below is a reading):
+//  1. each vector v takes its own range lo_v = min, hi_v = max and the ratio family j_v whose set
+//     on that range, (c = (hi_v - lo_v) t_j, o = lo_v), gives it the least squared error (the
+//     lowest j on a tie);
+//  2. per family j, the points (lo_v, hi_v) of its vectors are clustered by Lloyd's k-means into
+//     64 centroids, started from the 8 x 8 quantile grid of bqref_bvsr_set_table (centroid
+//     8a + b = (lo_a, hi_b)); a round assigns every point to the nearest centroid (squared
+//     Euclidean distance in float64, the lowest index on a tie), then moves each centroid that
+//     has points to their mean, computed exactly as sum_v fix(v) / count / 2^40 with fix(v) =
+//     rn(v 2^40) summed in int64 (order-independent); a centroid without points stays;
+//  3. set 64 j + c is the family-j set on centroid c's range: c_i = (hi_c - lo_c) t_{j,i} and
+//     o = lo_c, stored float32. With rounds = 0 this is bqref_bvsr_set_table.
+// Out: table [256][5]; family [V] (nullable): j_v; assign [V] (nullable): the cluster of the last
+// round (0 without rounds); centroids [4][64][2] (nullable): final (lo, hi) per family and cluster.
+int bqref_bvsr_cluster_table(const float* W, int64_t N, int64_t K, int rounds, float* table, uint8_t* family,
+                             uint8_t* assign, double* centroids) {
+  if (N < 1 || K < kVec || K % kVec != 0 || rounds < 0) return -1;
+  const int64_t V = N * (K / kVec);
+  double grid[2 * kGrid * kGrid];
+  bvsr_grid(W, N, K, grid);
+  std::vector<float> lo(static_cast<size_t>(V)), hi(static_cast<size_t>(V));
+  std::vector<uint8_t> fam(static_cast<size_t>(V)), asg(static_cast<size_t>(V), 0);
+#pragma omp parallel for schedule(static)
+  for (int64_t v = 0; v < V; v++) {
+    const float* e = W + v * kVec;
+    float l = e[0], h = e[0];
+    for (int i = 1; i < kVec; i++) {
+      l = std::min(l, e[i]);
+      h = std::max(h, e[i]);
+    }
+    lo[size_t(v)] = l;
+    hi[size_t(v)] = h;
+    int bj = 0;
+    double be = 0.0;
+    for (int j = 0; j < 4; j++) {
+      float row5[5];
+      bvsr_make_set(j, double(l), double(h), row5);
+      const double err = bvsr_vector_error(e, row5);
+      if (j == 0 || err < be) { be = err; bj = j; }
+    }
+    fam[size_t(v)] = uint8_t(bj);
+  }
+  double cen[4][kGrid * kGrid][2];
+  for (int j = 0; j < 4; j++)
+    for (int c = 0; c < kGrid * kGrid; c++) {
+      cen[j][c][0] = grid[2 * c];
+      cen[j][c][1] = grid[2 * c + 1];
+    }
+  for (int r = 0; r < rounds; r++) {
+#pragma omp parallel for schedule(static)
+    for (int64_t v = 0; v < V; v++) {
+      const int j = fam[size_t(v)];
+      int bc = 0;
+      double bd = 0.0;
+      for (int c = 0; c < kGrid * kGrid; c++) {
+        const double dl = double(lo[size_t(v)]) - cen[j][c][0], dh = double(hi[size_t(v)]) - cen[j][c][1];
+        const double d = dl * dl + dh * dh;
+        if (c == 0 || d < bd) { bd = d; bc = c; }
+      }
+      asg[size_t(v)] = uint8_t(bc);
+    }
+    int64_t sl[4][kGrid * kGrid] = {}, sh[4][kGrid * kGrid] = {}, cnt[4][kGrid * kGrid] = {};
+    for (int64_t v = 0; v < V; v++) {
+      const int j = fam[size_t(v)], c = asg[size_t(v)];
+      sl[j][c] += bvsr_fix(lo[size_t(v)]);
+      sh[j][c] += bvsr_fix(hi[size_t(v)]);
+      cnt[j][c] += 1;
+    }
+    for (int j = 0; j < 4; j++)
+      for (int c = 0; c < kGrid * kGrid; c++)
+        if (cnt[j][c] > 0) {
+          cen[j][c][0] = std::ldexp(double(sl[j][c]) / double(cnt[j][c]), -40);
+          cen[j][c][1] = std::ldexp(double(sh[j][c]) / double(cnt[j][c]), -40);
+        }
+  }
+  for (int j = 0; j < 4; j++)
+    for (int c = 0; c < kGrid * kGrid; c++) bvsr_make_set(j, cen[j][c][0], cen[j][c][1], table + (64 * j + c) * 5);
+  if (family) std::memcpy(family, fam.data(), size_t(V));
+  if (assign) std::memcpy(assign, asg.data(), size_t(V));
+  if (centroids) std::memcpy(centroids, cen, sizeof(cen));
+  return 0;
+}
+
 // P[s][code] = o + sum of the c_i whose bit i of code is set, added in i order in float64
 int bqref_bvsr_points(const float* table, int S, double* P) {
   if (S < 1) return -1;

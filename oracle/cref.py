@@ -52,6 +52,7 @@ _SIGS = {
     "bqref_bvsr_points": (_I, [_P, _I, _P]),
     "bqref_bvsr_encode": (_I, [_P, _I64, _P, _P, _P]),
     "bqref_bvsr_layer": (_I, [_P, _P, _P, _I64, _I64, _P, _I64, _P, _P, _P, _P]),
+    "bqref_bvsr_cluster_table": (_I, [_P, _I64, _I64, _I, _P, _P, _P, _P]),
     "bqref_decode_tokens_per_s": (_D, [_D, _D, _D]),
     "bqref_weight_bits_per_param": (_D, [_I, _I]),
     "bqref_silu": (_I, [_P, _I64, _P]),
@@ -443,6 +444,24 @@ def bvsr_set_table(W) -> np.ndarray:
     return t
 
 
+def bvsr_cluster_table(W, rounds: int) -> dict:
+    """[BVSR] Introduction, coefficient cache, clustering reading: per-vector best ratio family
+    on its own range, then per family Lloyd k-means of the vectors' (min, max) into 64 centroids
+    from the quantile grid, with exact fixed-point centroid sums; set 64 j + c spans centroid c.
+    Returns table [256,5], family [V], assign [V], centroids [4,64,2]. Parity unpinned as a
+    reading; pinned by tests (rounds = 0 is bvsr_set_table, the k-means objective never grows,
+    brute-force family choice, a hand case of exact clusters)."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    V = N * (K // BVSR_VEC)
+    t = np.empty((256, 5), np.float32)
+    fam = np.empty(V, np.uint8)
+    asg = np.empty(V, np.uint8)
+    cen = np.empty((4, 64, 2), np.float64)
+    _ok(_lib.bqref_bvsr_cluster_table(_p(W), N, K, int(rounds), _p(t), _p(fam), _p(asg), _p(cen)))
+    return dict(table=t, family=fam, assign=asg, centroids=cen)
+
+
 def bvsr_points(table) -> np.ndarray:
     """P[s, code] = o + sum of the c_i selected by the bits of code, added in i order in float64.
     Pinned by tests (ratio-2 sets are the uniform RTN grid)."""
@@ -467,13 +486,13 @@ def bvsr_encode_vectors(vecs, table):
     return codes, sets
 
 
-def bvsr_pack(W, table=None, rows=None) -> dict:
+def bvsr_pack(W, table=None, rows=None, cluster_rounds: int = 0) -> dict:
     """BVSR 4-bit pack of W (rows optionally restricted): table, codes and set indices. Pinned by
     tests (layer routes agree); the set construction itself is a reading: parity unpinned."""
     W = _c(W, np.float32)
     N, K = W.shape
     if table is None:
-        table = bvsr_set_table(W)
+        table = bvsr_cluster_table(W, cluster_rounds)["table"] if cluster_rounds > 0 else bvsr_set_table(W)
     sel = np.arange(N) if rows is None else np.asarray(rows)
     codes, sets = bvsr_encode_vectors(W[sel].reshape(-1, BVSR_VEC), table)
     return dict(codes=codes.reshape(len(sel), K), sets=sets.reshape(len(sel), K // BVSR_VEC), table=table, rows=sel)

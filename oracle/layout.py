@@ -33,8 +33,14 @@ the f-bit field j (bits f*j .. f*j+f-1) of byte b holds the weight at
   row = 16*rb + g + 8*(r & 1)
   k   = 32*(8*kt + u*(8/f) + j) + 16*(r >> 1) + 4*t + b.
 
-BVSR tiles (4 one-bit planes of 512 B) end with 128 bytes of set indices: byte
-2048 + 8*g + j holds the set of row 16*rb + g, vector 8*kt + j (32 elements each).
+BVSR tiles (one stream, n_streams = 1, field width 4) hold 4-bit codes in their own
+nibble order, not the generic field order above: the first 2048 bytes are 4 blocks
+i < 4 of [lane < 32][4 words]; word 2*v + h of lane 4g+t in block i holds, for vector
+j = 2i + v of the tile, nibble b (bits 4b..4b+3) of its low half the code of
+row 16*rb + g and of its high half the code of row 16*rb + g + 8, at
+k = 256*kt + 32*j + 16*h + 4*t + b. The tile ends with 128 bytes of set indices:
+byte 2048 + 8*g + j holds the set of row 16*rb + g (g < 16 here), vector 8*kt + j
+(32 elements each).
 
 RaBiT (format 1: P = 2 paths; format 6: P = 3) is not tiled: plane p (0..P-1)
 word w of row n is the uint32 at off_tiles + 4*((p*N_pad + n)*(K_pad/32) + w),
@@ -119,6 +125,25 @@ def read_stream_codes(buf: bytes, h: dict, s: int, row_blocks=None) -> np.ndarra
     return out[:, :K]
 
 
+def read_bvsr_codes(buf: bytes, h: dict, row_blocks=None) -> np.ndarray:
+    """The 4-bit codes of a BVSR buffer (nibble order of its tiles): uint8 [N, K], or
+    [16*len(row_blocks), K] for a subset of 16-row blocks.
+    Pinned by tests (a hand-derived nibble fixture; GPU pack round trips)."""
+    N, K, N_pad, K_pad = h["N"], h["K"], h["N_pad"], h["K_pad"]
+    RB, KT, tb = N_pad // 16, K_pad // 256, h["tile_bytes"]
+    rbs = np.arange(RB) if row_blocks is None else np.asarray(row_blocks)
+    raw = np.frombuffer(buf, dtype=np.uint8, count=RB * KT * tb, offset=h["off_tiles"]).reshape(RB, KT, tb)
+    words = np.ascontiguousarray(raw[rbs][:, :, :2048]).view("<u4")
+    w = words.reshape(len(rbs), KT, 4, 8, 4, 2, 2)               # [rb][kt][i][g][t][v][h]
+    shift = 16 * np.arange(2)[:, None] + 4 * np.arange(4)[None, :]  # [rbit][b]
+    nib = (w[..., None, None] >> shift.astype(np.uint32)) & 0xF     # [rb][kt][i][g][t][v][h][rbit][b]
+    # row = 16 rb + 8 rbit + g, k = 256 kt + 32 (2i + v) + 16 h + 4 t + b
+    arr = nib.transpose(0, 7, 3, 1, 2, 5, 6, 4, 8).reshape(16 * len(rbs), K_pad).astype(np.uint8)
+    if row_blocks is None:
+        return arr[:N, :K]
+    return arr[:, :K]
+
+
 def read_packed(buf: bytes, row_blocks=None) -> dict:
     """Decode a packed buffer into the dict shape that bq_oracle's layers take.
     ``row_blocks`` (tiled formats) restricts the per-row arrays to those 16-row
@@ -182,10 +207,7 @@ def read_packed(buf: bytes, row_blocks=None) -> dict:
         out["w_bits"] = h["w_bits"]
         out["a_bits"] = h["a_bits"]
     elif fmt == FMT_BVSR:
-        codes = np.zeros((len(sel), K), dtype=np.uint8)
-        for s in range(h["n_streams"]):
-            codes |= (read_stream_codes(buf, h, s, rb) << h["shifts"][s]).astype(np.uint8)
-        out["codes"] = codes
+        out["codes"] = read_bvsr_codes(buf, h, rb)
         tab = np.frombuffer(buf, dtype="<f4", count=256 * 8, offset=h["off_aux"]).reshape(256, 8)
         out["table"] = tab[:, :5].copy()
         out["table_derived"] = tab[:, 5:].copy()

@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_status_strings_and_version():
-    assert bq.bq_version() == bq.BQ_ABI_VERSION == 2
+    assert bq.bq_version() == bq.BQ_ABI_VERSION == 3
     hdr = open(os.path.join(ROOT, "include", "bq.h")).read()
     assert re.search(r"#define BQ_ABI_VERSION (\d+)", hdr).group(1) == str(bq.BQ_ABI_VERSION)
 
@@ -68,7 +68,7 @@ def test_binding_structs_match_the_c_header(tmp_path):
     ("bitnet", {}, 50, 384, 256 + 64 * 512 // 8),
     ("ternary", dict(lora_rank=32), 2048, 2048, 256 + 2048 * 2048 // 4 + 2048 * 32 * 2 * 2),
     ("abq", dict(w_bits=6, a_bits=6), 4096, 4096, 256 + 4096 * 4096 * 6 // 8 + 3 * 4096 * 4),
-    ("bvsr", {}, 5120, 5120, 256 + 5120 * 5120 // 2 + 256 * 8 * 4 + 5120 * 5120 // 32),
+    ("bvsr", {}, 5120, 5120, 256 + 5120 * 5120 // 2 + 256 * 8 * 4 + 10240 + 5120 * 5120 // 32),
     # RaBiT: P sign planes, g [P][N], h [P][K] f32
     ("rabit", {}, 256, 512, 256 + 2 * 256 * 512 // 8 + 2 * 256 * 4 + 2 * 512 * 4),
     ("rabit3", {}, 256, 512, 256 + 3 * 256 * 512 // 8 + 3 * 256 * 4 + 3 * 512 * 4),
@@ -86,7 +86,7 @@ def test_packed_bits_per_weight():
         tot = bq.bq_packed_bytes(bq.make_desc(fmt, **kw), N, K)
         assert tot - 256 - (3 * N * 4 if fmt == "abq" else 0) == N * K * bits // 8
     tot = bq.bq_packed_bytes(bq.make_desc("bvsr"), N, K)
-    assert tot - 256 - 256 * 8 * 4 == N * K * 4.25 / 8
+    assert tot - 256 - 256 * 8 * 4 - 10240 == N * K * 4.25 / 8   # table, then 10 KB of pack scratch
 
 
 @pytest.mark.parametrize("N,K,status", [(0, 256, 3), (16, 0, 3), (16, 200, 3), (16, 64, 3),
@@ -137,7 +137,8 @@ def _host_header(fmt, N, K, **kw):
     N_pad, K_pad = -(-N // 16) * 16, -(-K // 256) * 256
     h = np.zeros(64, "<u4")
     h[0], h[1], h[2], h[3], h[4], h[5], h[6] = L.PK_MAGIC, 1, bq.FORMATS[fmt], N, K, N_pad, K_pad
-    fields = {"bitnet": [1], "ternary": [2], "bvsr": [1, 1, 1, 1], "rabit": [1, 1], "rabit3": [1, 1, 1]}.get(fmt)
+    # BVSR: one stream of 4-bit codes in the nibble order of its tiles
+    fields = {"bitnet": [1], "ternary": [2], "bvsr": [4], "rabit": [1, 1], "rabit3": [1, 1, 1]}.get(fmt)
     P = len(fields) if fmt.startswith("rabit") else 0
     if fmt == "abq":
         w = kw["w_bits"]
@@ -151,7 +152,7 @@ def _host_header(fmt, N, K, **kw):
     h[9] = len(fields)
     sh = 0
     for i, f in enumerate(fields):
-        h[10 + i], h[14 + i] = f, (i if fmt == "bvsr" or P else sh)
+        h[10 + i], h[14 + i] = f, (i if P else sh)
         sh += f
     h[18] = 0 if P else 512 * sum(fields) + (128 if fmt == "bvsr" else 0)
     h[19] = kw.get("lora_rank", 0)
@@ -159,7 +160,7 @@ def _host_header(fmt, N, K, **kw):
     rows = 3 * N_pad * 4 if fmt == "abq" else P * N_pad * 4
     a256 = lambda v: (v + 255) // 256 * 256
     off_rows = a256(256 + tiles)
-    aux = K_pad * 4 if P else {"ternary": K_pad * h[19] * 2, "bvsr": 256 * 8 * 4}.get(fmt, 0)
+    aux = K_pad * 4 if P else {"ternary": K_pad * h[19] * 2, "bvsr": 256 * 8 * 4 + 10240}.get(fmt, 0)
     aux2 = (P - 1) * K_pad * 4 if P else {"ternary": N_pad * h[19] * 2}.get(fmt, 0)
     off_aux = a256(off_rows + rows)
     off_aux2 = a256(off_aux + aux)
@@ -319,6 +320,8 @@ def test_linear_plan_invariants(fmt, N, K, kw, M, fused):
     chunks = lambda t: -(-npad // (256 // pow2(t)))
     tpc, J = p["tokens_per_cta"], p["x_chunks_per_thread"]
     assert 1 <= tpc <= min(8, M) and p["token_groups"] == -(-M // tpc)
+    if fmt == "abq" and M >= 2:   # bq_linear quantizes once into an act buffer, then the layer
+        fused = False
     if fused:   # the most tokens whose x fits 16 chunks per thread; else one token read twice
         fits = [t for t in range(1, min(8, M) + 1) if chunks(t) <= 16]
         assert tpc == (max(fits) if fits else 1)
@@ -326,18 +329,21 @@ def test_linear_plan_invariants(fmt, N, K, kw, M, fused):
     else:       # the most tokens whose int8 codes fit 96 KB
         cstride = KT * 256 + 16
         assert J == 0 and tpc == max([t for t in range(1, min(8, M) + 1) if t * cstride <= 96 * 1024] + [1])
-    assert p["ctas_per_group"] == max(1, min(RB, -(-148 // p["token_groups"])))  # 148 SMs when no device
+    cps = 2 if fmt == "bvsr" and tpc == 1 else 1   # CTAs of one launch per SM (148 SMs when no device)
+    CPG = p["ctas_per_group"]
+    assert CPG == max(1, min(RB, -(-cps * 148 // p["token_groups"])))
     wpr, T = p["warps_per_row_block"], p["tiles_per_warp"]
     assert wpr in (1, 2, 4, 8) and T == -(-KT // wpr)
     S, C = p["ring_stages"], p["tiles_per_stage"]
-    assert 2 <= S <= 4 and 1 <= C <= T and 8 * S * C * tile_bytes <= 96 * 1024
-    assert p["shared_bytes"] % 128 == 0 and 8 * S * C * tile_bytes < p["shared_bytes"] <= 227 * 1024
+    active = min(8 // wpr, -(-RB // CPG)) * wpr   # warps that hold row blocks share the ring
+    assert 2 <= S <= 4 and 1 <= C <= T and active * S * C * tile_bytes <= 96 * 1024
+    assert p["shared_bytes"] % 128 == 0 and active * S * C * tile_bytes < p["shared_bytes"] <= 227 * 1024
 
 
 def test_linear_plan_of_the_measured_llama7b_layers():
     """The decode plans of the Llama-7B BitNet layers whose timings and DRAM traffic were
     measured; a change here means those measurements are of another plan."""
-    want = {(4096, 4096): (4, 4, 4, 2), (11008, 4096): (1, 4, 6, 2), (4096, 11008): (4, 4, 6, 6)}
+    want = {(4096, 4096): (4, 4, 4, 2), (11008, 4096): (1, 4, 9, 2), (4096, 11008): (4, 4, 6, 6)}
     for (N, K), (wpr, S, C, J) in want.items():
         p = bq.bq_linear_plan(bq.bq_packed_validate(_host_header("bitnet", N, K).tobytes(), 1 << 30), 1)
         got = (p["warps_per_row_block"], p["ring_stages"], p["tiles_per_stage"], p["x_chunks_per_thread"])
@@ -519,3 +525,16 @@ def test_pack_refuses_unaligned_or_missing_correction_matrices():
         d = bq.make_desc("ternary", lora_rank=8, lora_A=A, lora_B=B)
         assert bq.raw_status("bq_pack_weights", ctypes.byref(d), fake, 64, 256, fake, 1 << 30, None,
                              ctypes.byref(bq.bq_layer())) == bq.BQ_ERR_INVALID_ARG
+
+
+def test_bvsr_cluster_rounds_are_checked():
+    """bvsr_cluster_rounds: 0..100 for BVSR, 0 for every other format (host only)."""
+    fake = 1 << 40
+    layer = bq.bq_layer()
+    for fmt, r, ok in [("bvsr", 0, True), ("bvsr", 8, True), ("bvsr", 100, True), ("bvsr", 101, False),
+                       ("bvsr", -1, False), ("bitnet", 1, False), ("abq", 2, False)]:
+        kw = dict(w_bits=4, a_bits=4) if fmt == "abq" else {}
+        d = bq.make_desc(fmt, bvsr_cluster_rounds=r, **kw)
+        st = bq.raw_status("bq_packed_bytes", ctypes.byref(d), 64, 256, ctypes.byref(ctypes.c_size_t()))
+        assert (st == bq.BQ_OK) == ok, (fmt, r, st)
+    assert layer is not None and fake

@@ -476,3 +476,32 @@ def test_abq_compensation(w, a, balanced, N, K, M):
     assert np.array_equal(acc.cpu().numpy(), r["I"])
     assert_y_close(y.cpu().numpy(), r["y"], "abq compensated")
     bq.bq_device_check()
+
+
+# ------------------------------------------------------------------ BVSR coefficient cache by clustering
+@pytest.mark.parametrize("N,K,M,rounds", [(50, 384, 1, 1), (97, 640, 3, 4), (256, 2048, 1, 8), (5120, 5120, 1, 8)])
+def test_bvsr_cluster_pack_and_layer(N, K, M, rounds):
+    """The clustering reading of the coefficient cache: the pack's per-vector families, k-means
+    centroids (exact integer sums, so the GPU's atomic order does not matter) and resulting
+    table equal the C++ oracle's bit for bit, and so do the searched sets and codes (sampled row
+    blocks at the full size); the layer on them matches the oracle."""
+    from tests.parity_util import L as layout, torch_mods
+    torch, bq = torch_mods()
+    inp = I.layer_inputs("bvsr", N, K, M, seed=N + rounds)
+    W, x = inp["W"], inp["x"]
+    ql = bq.QuantLinear("bvsr", to_dev_f32(W), bvsr_cluster_rounds=rounds)
+    rbs = None if N <= 256 else _sample_blocks(N, n=4, seed=rounds)
+    p = layout.read_packed(ql.packed.cpu().numpy().tobytes(), rbs)
+    rows = p["rows"][p["rows"] < N]
+    ref = O.bvsr_pack(W, rows=rows, cluster_rounds=rounds)
+    assert np.array_equal(p["table"], ref["table"])
+    assert np.array_equal(p["sets"][:len(rows)], ref["sets"]) and np.array_equal(p["codes"][:len(rows)], ref["codes"])
+    xd = to_dev_bf16(x)
+    y = torch.full((M, N), float("nan"), device="cuda")
+    acc = torch.full((M, N), -(1 << 62), dtype=torch.int64, device="cuda")
+    ql.linear(xd, y, acc)
+    torch.cuda.synchronize()
+    bq.bq_device_check()
+    r = O.bvsr_layer(ref["codes"], ref["sets"], ref["table"], x)
+    assert np.array_equal(acc.cpu().numpy()[:, rows], r["acc"])
+    assert_y_close(y.cpu().numpy()[:, rows], r["y"], f"bvsr clustered {N}x{K}")

@@ -70,3 +70,24 @@ def test_rabit3_single_bit_scale_and_h(golden):
     assert np.argwhere(p["B"] == -1).tolist() == [c["neg"]]
     assert np.argwhere(p["g"] != 0).tolist() == [c["neg"][:2]] and p["g"][2, 17] == c["g"]
     assert np.argwhere(p["h"] != 0).tolist() == [[2, c["neg"][2]]] and p["h"][2, 291] == c["h"]
+
+
+def test_bvsr_single_nibble_and_set(golden):
+    """BVSR: one 4-bit code and one set index at hand-derived byte offsets of the nibble order."""
+    c = golden("layout_bits.json")["bvsr_one_nibble"]
+    z = c["sizes"]
+    N, K = c["N"], c["K"]
+    hdr = np.zeros(64, dtype="<u4")
+    hdr[0], hdr[1], hdr[2], hdr[3], hdr[4], hdr[5], hdr[6] = L.PK_MAGIC, 1, L.FMT_BVSR, N, K, 16, 256
+    hdr[7], hdr[8], hdr[9], hdr[10], hdr[18] = 4, 8, 1, 4, c["tile_bytes"]
+    for word, v in [(22, z["total"]), (24, 256), (26, z["off_aux"]), (28, z["off_aux"]), (30, z["total"])]:
+        hdr[word] = v
+    buf = bytearray(z["total"])
+    buf[:256] = hdr.tobytes()
+    buf[256 + c["byte"]] = c["value"]
+    buf[256 + c["set_byte"]] = c["set"]
+    p = L.read_packed(bytes(buf))
+    assert np.argwhere(p["codes"] != 0).tolist() == [[c["row"], c["k"]]]
+    assert int(p["codes"][c["row"], c["k"]]) == c["code"]
+    assert np.argwhere(p["sets"] != 0).tolist() == [[c["row"], c["set_vector"]]]
+    assert int(p["sets"][c["row"], c["set_vector"]]) == c["set"]

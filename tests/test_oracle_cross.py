@@ -151,3 +151,14 @@ def test_cpp_reference_runs_on_several_threads_with_the_same_results():
     _same(one["codes"], many["codes"], "codes")
     _same(one["sets"], many["sets"], "sets")
     _same(y1, ym, "y")
+
+
+@pytest.mark.parametrize("rounds", [0, 1, 4])
+def test_bvsr_cluster_table_agrees(rounds):
+    W = I.weights(48, 1024, seed=30 + rounds)
+    a, b = N.bvsr_cluster_table(W, rounds), C.bvsr_cluster_table(W, rounds)
+    for k in ("table", "family", "assign", "centroids"):
+        _same(a[k], b[k], f"cluster {k}")
+    pa, pb = N.bvsr_pack(W, rows=np.array([0, 47]), cluster_rounds=rounds), C.bvsr_pack(W, rows=np.array([0, 47]), cluster_rounds=rounds)
+    _same(pa["codes"], pb["codes"], "codes")
+    _same(pa["sets"], pb["sets"], "sets")

@@ -582,3 +582,61 @@ def test_every_public_oracle_function_states_its_pins(O):
                if not n.startswith("_") and f.__module__ == m.__name__
                and "Pinned" not in (f.__doc__ or "") and "parity unpinned" not in (f.__doc__ or "").lower()]
     assert not missing, missing
+
+
+# --------------------------------------------------------------------- BVSR coefficient cache (clustering)
+def test_bvsr_cluster_zero_rounds_is_the_quantile_table(O):
+    """Without a k-means round the centroids are the quantile grid, so the table is the grid
+    reading's table bit for bit."""
+    W = I.weights(32, 512, seed=21)
+    assert np.array_equal(O.bvsr_cluster_table(W, 0)["table"], O.bvsr_set_table(W))
+
+
+def test_bvsr_cluster_objective_never_grows(O):
+    """Lloyd rounds: each assignment and each exact mean can only lower the sum of squared
+    distances of the vectors' (min, max) to their centroid."""
+    W = I.weights(48, 1024, seed=22)
+    v = W.reshape(-1, 32)
+    pts = np.stack([v.min(1), v.max(1)], 1).astype(np.float64)
+    J = []
+    for r in range(1, 7):
+        c = O.bvsr_cluster_table(W, r)
+        cen = c["centroids"][c["family"].astype(int), c["assign"].astype(int)]
+        J.append(float(((pts - cen) ** 2).sum()))
+    assert all(b <= a * (1 + 1e-12) for a, b in zip(J, J[1:])), J
+    assert J[-1] < J[0]
+
+
+def test_bvsr_cluster_family_is_the_best_of_the_vectors_own_sets(O):
+    """A vector's family is the ratio whose set on its own range fits it best: the exhaustive
+    encoder, given a table whose sets 0..3 are the vector's own four sets (taken from the
+    quantile table of the vector alone, where every grid point is its min and max), picks set
+    index == family."""
+    W = I.weights(8, 256, seed=23)
+    c = O.bvsr_cluster_table(W, 2)
+    vecs = W.reshape(-1, 32)
+    for vi in range(0, vecs.shape[0], 7):
+        own = O.bvsr_set_table(vecs[vi:vi + 1])
+        tab = np.repeat(own[[192]], 256, axis=0)
+        tab[:4] = own[[0, 64, 128, 192]]
+        _, sets = O.bvsr_encode_vectors(vecs[vi:vi + 1], tab)
+        assert int(sets[0]) == int(c["family"][vi])
+
+
+def test_bvsr_cluster_exact_grid_vectors():
+    """Hand case: every vector holds -1/2 + k/16 for k = 0..15 (each twice). The ratio-2 set on
+    its range [-1/2, 7/16] has exactly those points (c = 1/16, 2/16, 4/16, 8/16), so the family is
+    1 (ratio 2, error 0); all vectors share one range, so after a round their centroid is that
+    range exactly, and the cluster's set is (1/16, 1/8, 1/4, 1/2, -1/2)."""
+    from oracle import bq_oracle as Nmp, cref as Cpp
+    row = (-0.5 + np.arange(16) / 16.0).astype(np.float32)
+    W = np.tile(np.concatenate([row, row[::-1]]), (4, 2)).astype(np.float32)  # 4 rows x 64: 8 vectors
+    for O in (Cpp, Nmp):
+        c = O.bvsr_cluster_table(W, 1)
+        assert np.all(c["family"] == 1)
+        cl = int(c["assign"][0])
+        assert np.all(c["assign"] == cl)
+        assert c["centroids"][1, cl].tolist() == [-0.5, 0.4375]
+        assert c["table"][64 + cl].tolist() == [0.0625, 0.125, 0.25, 0.5, -0.5]
+        codes, sets = O.bvsr_encode_vectors(W.reshape(-1, 32), c["table"])
+        assert np.all(sets == 64 + cl) and codes[0].tolist() == list(range(16)) + list(range(15, -1, -1))
