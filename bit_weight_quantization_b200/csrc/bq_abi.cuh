@@ -10,6 +10,7 @@
 #include "bq_gemv.cuh"
 #include "bq_internal.cuh"
 #include "bq_pack.cuh"
+#include "bq_tc.cuh"
 
 namespace bqi {
 
@@ -240,7 +241,8 @@ inline int pow2ceil(int v) {
 //  - tokens per CTA (tpc): fused, each token group of 256/pow2(tpc) threads holds its x
 //    in at most 16 16-byte chunks per thread; unfused, the code image fits in 96 KB;
 //  - about one CTA per SM, CPG CTAs per token group striding over the row blocks;
-//  - the weight ring gets what is left (at most 96 KB), split among the warps that have row
+//  - the weight ring gets what is left (at most 96 KB; a CTA whose weight slab exceeds 128 KB
+//    takes the whole SM), split among the warps that have row
 //    blocks: S (2..4) stages of C tiles per such warp.
 // Returns false when the layer does not fit this kernel.
 inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
@@ -317,7 +319,11 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   // a layer whose ring and fixed part exceed half of the SM runs alone. (Capping every
   // layer at half an SM measured slower on mixed-shape layer sequences.)
   const uint64_t limit = ctas_per_sm == 2 ? 112 * 1024 : 220 * 1024;  // two CTAs share the SM's 228 KB
-  const uint64_t budget = std::min<uint64_t>(96 * 1024, fixed < limit ? limit - fixed : 0);
+  // A layer whose weight slab per CTA is large (more than 128 KB) streams most of it after the
+  // wait whatever the ring: it gets the whole SM for its ring (one CTA per SM, more bytes in
+  // flight) instead of leaving room for the next launch's CTA.
+  const bool big = uint64_t(ipc) * L.KT * L.tile_bytes > 128 * 1024 && ctas_per_sm == 1;
+  const uint64_t budget = std::min<uint64_t>(big ? limit : 96 * 1024, fixed < limit ? limit - fixed : 0);
   // The ring is split among the warps that have row blocks: groups 0 .. min(G, ipc) - 1, i.e.
   // warps 0 .. active - 1 (a CTA never holds more than ipc row blocks); idle warps get none.
   const int active = std::min(NW / wpr, ipc) * wpr;
@@ -385,6 +391,43 @@ inline cudaError_t launch_fmt(const PkLayout& L, const LayerArgs& g, int NW, dim
       }
     default: return cudaErrorInvalidValue;
   }
+}
+
+// ABQ with 8-bit weight codes and 16..64 tokens (from an act buffer) runs on the tensor cores.
+inline bool tc_eligible(const PkLayout& L, int M) { return tc_layer(L.fmt, L.w_bits, M); }
+
+inline bq_status launch_abq_tc(const PkLayout& L, const void* packed, const void* act, int M, float* y,
+                               int64_t* acc, cudaStream_t s) {
+  const uint8_t* P = static_cast<const uint8_t*>(packed);
+  const uint8_t* Ab = static_cast<const uint8_t*>(act);
+  const ActLayout A = make_act_layout(L, M);
+  TcArgs t{};
+  t.tiles = P + L.off_tiles;
+  t.row_delta = reinterpret_cast<const float*>(P + L.off_rows);
+  t.row_zero = reinterpret_cast<const int*>(P + L.off_rows + 4ull * L.N_pad);
+  t.row_sum = reinterpret_cast<const int*>(P + L.off_rows + 8ull * L.N_pad);
+  t.act_hdr = reinterpret_cast<const uint32_t*>(Ab);
+  t.act_codes = Ab + A.off_ct;
+  t.act_tok = reinterpret_cast<const uint32_t*>(Ab + A.off_tok);
+  t.act_total = A.total;
+  t.y = y;
+  t.acc = reinterpret_cast<long long*>(acc);
+  t.N = L.N; t.K = L.K; t.KT = L.KT; t.RB = L.RB; t.M = M; t.Nmma = (M + 15) / 16 * 16; t.a_bits = L.a_bits;
+  static std::mutex mu;
+  static unsigned long long set_ctx = 0;
+  {
+    const unsigned long long ctx = current_context_id();
+    std::lock_guard<std::mutex> lock(mu);
+    if (ctx == 0 || ctx != set_ctx) {
+      if (cudaFuncSetAttribute(k_abq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return BQ_ERR_CUDA;
+      }
+      set_ctx = ctx;
+    }
+  }
+  return launch_pdl(k_abq_tc, dim3((L.RB + kTcRb - 1) / kTcRb), dim3(kTcThreads), kTcSmem, s, t) == cudaSuccess
+             ? BQ_OK : BQ_ERR_CUDA;
 }
 
 inline bq_status launch_layer(const PkLayout& L, LayerArgs& g, bool fused, cudaStream_t s) {
@@ -640,6 +683,7 @@ bq_status bq_quantize_act(const bq_layer* layer, const void* x_bf16, int32_t M, 
   a.act = static_cast<uint8_t*>(act);
   a.M = M; a.K = L.K; a.K_pad = L.K_pad; a.KT = L.KT; a.a_bits = L.a_bits; a.rank = A.rank; a.fmt = L.fmt;
   a.off_codes = A.off_codes; a.off_tok = A.off_tok; a.off_gsum = A.off_gsum; a.off_u = A.off_u; a.off_xt = A.off_xt;
+  a.off_ct = A.off_ct;
   a.total = A.total;
   a.lora_A = reinterpret_cast<const uint16_t*>(P + L.off_aux);
   a.h = reinterpret_cast<const float*>(P + L.off_aux);
@@ -653,10 +697,10 @@ bq_status bq_quantize_act(const bq_layer* layer, const void* x_bf16, int32_t M, 
   const dim3 grid(slices, M);
   cudaError_t e;
   switch (L.fmt) {
-    case BQ_FMT_BITNET_W1A8: e = launch_pdl(k_act_quant<BQ_FMT_BITNET_W1A8>, grid, dim3(256), 0, s, a); break;
-    case BQ_FMT_TERNARY_A8: e = launch_pdl(k_act_quant<BQ_FMT_TERNARY_A8>, grid, dim3(256), 0, s, a); break;
-    case BQ_FMT_ABQ: e = launch_pdl(k_act_quant<BQ_FMT_ABQ>, grid, dim3(256), 0, s, a); break;
-    case BQ_FMT_BVSR4: e = launch_pdl(k_act_quant<BQ_FMT_BVSR4>, grid, dim3(256), 0, s, a); break;
+    case BQ_FMT_BITNET_W1A8: e = launch_pdl(k_act_quant<BQ_FMT_BITNET_W1A8>, grid, dim3(1024), 0, s, a); break;
+    case BQ_FMT_TERNARY_A8: e = launch_pdl(k_act_quant<BQ_FMT_TERNARY_A8>, grid, dim3(1024), 0, s, a); break;
+    case BQ_FMT_ABQ: e = launch_pdl(k_act_quant<BQ_FMT_ABQ>, grid, dim3(1024), 0, s, a); break;
+    case BQ_FMT_BVSR4: e = launch_pdl(k_act_quant<BQ_FMT_BVSR4>, grid, dim3(1024), 0, s, a); break;
     default: return BQ_ERR_INVALID_ARG;
   }
   return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
@@ -671,6 +715,7 @@ bq_status bq_gemm(const bq_layer* layer, const void* act, int32_t M, float* y, i
   if (!act || !aligned(act, 256) || !y || !aligned(y, 4) || (acc_dbg && !aligned(acc_dbg, 8)))
     return BQ_ERR_INVALID_ARG;
   if (rabit_paths(L.fmt) && acc_dbg) return BQ_ERR_UNSUPPORTED;
+  if (tc_eligible(L, M)) return launch_abq_tc(L, layer->packed, act, M, y, acc_dbg, reinterpret_cast<cudaStream_t>(stream));
   const uint8_t* Ab = static_cast<const uint8_t*>(act);
   const ActLayout A = make_act_layout(L, M);
   LayerArgs g = layer_args(L, layer->packed, M, y, acc_dbg);

@@ -14,7 +14,7 @@ struct ActArgs {
   const uint16_t* x;        // bf16 [M][K]
   uint8_t* act;             // act buffer base
   int M, K, K_pad, KT, a_bits, rank, fmt, tiles_per_slice;
-  uint64_t off_codes, off_tok, off_gsum, off_u, off_xt, total;
+  uint64_t off_codes, off_tok, off_gsum, off_u, off_xt, off_ct, total;
   const uint16_t* lora_A;   // ternary: bf16 [K_pad][r]
   const float* h;           // RaBiT: h_p at h + p K_pad, p < rabit_paths(fmt)
 };
@@ -44,6 +44,8 @@ __device__ __forceinline__ void act_write_header(const ActArgs& a) {
       case AW_OFF_U + 1: v = uint32_t(a.off_u >> 32); break;
       case AW_OFF_XT: v = uint32_t(a.off_xt); break;
       case AW_OFF_XT + 1: v = uint32_t(a.off_xt >> 32); break;
+      case AW_OFF_CT: v = uint32_t(a.off_ct); break;
+      case AW_OFF_CT + 1: v = uint32_t(a.off_ct >> 32); break;
       default: break;
     }
     h[i] = v;
@@ -77,8 +79,10 @@ __device__ __forceinline__ int q_asym(float x, float d, int z, int qmax) {
   return int(q);
 }
 
+// 1024 threads a block: slice 0 also codes the whole row for the token's code sum, which for
+// ABQ is a correctly rounded divide per element on that block's critical path.
 template <int FMT>
-__global__ void __launch_bounds__(256) k_act_quant(ActArgs a) {
+__global__ void __launch_bounds__(1024) k_act_quant(ActArgs a) {
   __shared__ float shf[32];
   __shared__ int shi[32];
   const int m = blockIdx.y, slice = blockIdx.x;
@@ -133,6 +137,8 @@ __global__ void __launch_bounds__(256) k_act_quant(ActArgs a) {
     }
     const int kt = k >> 8;
     codes[kt * 64 + code_word_in_tile(k & 255)] = word;
+    if (a.off_ct)  // the tile-major copy: tile kt of token m at (kt M + m) 256
+      reinterpret_cast<uint32_t*>(a.act + a.off_ct)[(size_t(kt) * a.M + m) * 64 + code_word_in_tile(k & 255)] = word;
     if (FMT == BQ_FMT_BVSR4) {
       // 8 consecutive threads cover one 32-element vector (blockDim and 64 are multiples of 8)
       qs += __shfl_xor_sync(0xffffffffu, qs, 1);

@@ -741,49 +741,59 @@ struct BvsrFam {
 // 4, 5): y += sc E + o S_v, S_v the vector's code sum. TWO (warp-uniform): the CTA holds more
 // than one token, so outputs c = 1, 3 (token 2t + 1) are live too; with one token only c = 0, 2.
 // want_acc adds sum_k code_k q_k (a third MMA on the code bytes).
-__device__ __forceinline__ void bvsr_tile(const uint4 (&w)[4], const uint4 (&b)[4], uint2 i0, uint2 i1,
+// The tile is walked as a loop over its four vector pairs (the weight words and the act codes
+// of a pair are one 16-byte load each), so that the loop body stays small in the instruction
+// cache; the tile's set bytes for rows g and g + 8 are i0, i1 (byte j of the pair of words).
+__device__ __forceinline__ void bvsr_tile(const uint8_t* tp, const uint8_t* bp, bool has_tok, uint2 i0, uint2 i1,
                                           const float* tab, const BvsrFam* fam, const int* gs_row, int VPR,
                                           bool TWO, bool tok0, bool tok1, bool want_acc, float (&yacc)[4],
                                           long long (&cacc)[4]) {
+#pragma unroll 1
+  for (int jp = 0; jp < 4; jp++) {
+    const uint4 q = lds128(tp + jp * 512);
+    const uint4 bq = has_tok ? lds128(bp + jp * 16) : make_uint4(0, 0, 0, 0);
+    const uint32_t iw0 = jp < 2 ? i0.x : i0.y, iw1 = jp < 2 ? i1.x : i1.y;
 #pragma unroll
-  for (int j = 0; j < 8; j++) {
-    const uint4& q = w[j >> 1];
-    const uint32_t w0 = (j & 1) ? q.z : q.x, w1 = (j & 1) ? q.w : q.y;
-    const uint32_t sel[4] = {w0, w0 >> 16, w1, w1 >> 16};  // a0 (row g), a1 (g + 8), a2 (g), a3 (g + 8)
-    const int s0 = int(__byte_perm(j < 4 ? i0.x : i0.y, 0, 0x4440 + (j & 3)));
-    const int s1 = int(__byte_perm(j < 4 ? i1.x : i1.y, 0, 0x4440 + (j & 3)));
-    const BvsrFam f0 = fam[s0 >> 6], f1 = fam[s1 >> 6];
-    uint32_t a1[4], a2[4];
+    for (int v = 0; v < 2; v++) {
+      const int j = 2 * jp + v;
+      const uint32_t w0 = v ? q.z : q.x, w1 = v ? q.w : q.y;
+      const uint32_t b0 = v ? bq.z : bq.x, b1 = v ? bq.w : bq.y;
+      const uint32_t sel[4] = {w0, w0 >> 16, w1, w1 >> 16};  // a0 (row g), a1 (g + 8), a2 (g), a3 (g + 8)
+      const int s0 = int(__byte_perm(iw0, 0, 0x4440u | uint32_t(j & 3)));
+      const int s1 = int(__byte_perm(iw1, 0, 0x4440u | uint32_t(j & 3)));
+      const BvsrFam f0 = fam[s0 >> 6], f1 = fam[s1 >> 6];
+      uint32_t a1[4], a2[4];
 #pragma unroll
-    for (int r = 0; r < 4; r++) {
-      const BvsrFam& f = (r & 1) ? f1 : f0;
-      a1[r] = prmt(f.lo, f.hi, sel[r] & 0x7777u);
-      a2[r] = prmt(f.r3, f.r3, sel[r] ^ 0x8888u);
-    }
-    int d1[4] = {0, 0, 0, 0}, d2[4] = {0, 0, 0, 0};
-    mma_u8<true>(d1, a1[0], a1[1], a1[2], a1[3], bword(b, j, 0), bword(b, j, 1));
-    mma_u8<true>(d2, a2[0], a2[1], a2[2], a2[3], bword(b, j, 0), bword(b, j, 1));
-    if (want_acc) {  // the code bytes: c & 7 plus 8 [c >= 8]
-      uint32_t a3[4];
+      for (int r = 0; r < 4; r++) {
+        const BvsrFam& f = (r & 1) ? f1 : f0;
+        a1[r] = prmt(f.lo, f.hi, sel[r] & 0x7777u);
+        a2[r] = prmt(f.r3, f.r3, sel[r] ^ 0x8888u);
+      }
+      int d1[4] = {0, 0, 0, 0}, d2[4] = {0, 0, 0, 0};
+      mma_u8<true>(d1, a1[0], a1[1], a1[2], a1[3], b0, b1);
+      mma_u8<true>(d2, a2[0], a2[1], a2[2], a2[3], b0, b1);
+      if (want_acc) {  // the code bytes: c & 7 plus 8 [c >= 8]
+        uint32_t a3[4];
 #pragma unroll
-      for (int r = 0; r < 4; r++)
-        a3[r] = prmt(0x03020100u, 0x07060504u, sel[r] & 0x7777u) + prmt(0x08080808u, 0x08080808u, sel[r] ^ 0x8888u);
-      int d3[4] = {0, 0, 0, 0};
-      mma_u8<true>(d3, a3[0], a3[1], a3[2], a3[3], bword(b, j, 0), bword(b, j, 1));
+        for (int r = 0; r < 4; r++)
+          a3[r] = prmt(0x03020100u, 0x07060504u, sel[r] & 0x7777u) + prmt(0x08080808u, 0x08080808u, sel[r] ^ 0x8888u);
+        int d3[4] = {0, 0, 0, 0};
+        mma_u8<true>(d3, a3[0], a3[1], a3[2], a3[3], b0, b1);
 #pragma unroll
-      for (int c = 0; c < 4; c++) cacc[c] += d3[c];
-    }
-    const float2 os[2] = {*reinterpret_cast<const float2*>(tab + s0 * kBvsrTableStride + 4),
-                          *reinterpret_cast<const float2*>(tab + s1 * kBvsrTableStride + 4)};
-    const float gsf[2] = {tok0 ? small_int_to_float(gs_row[j]) : 0.f,
-                          TWO && tok1 ? small_int_to_float(gs_row[VPR + j]) : 0.f};
+        for (int c = 0; c < 4; c++) cacc[c] += d3[c];
+      }
+      const float2 os[2] = {*reinterpret_cast<const float2*>(tab + s0 * kBvsrTableStride + 4),
+                            *reinterpret_cast<const float2*>(tab + s1 * kBvsrTableStride + 4)};
+      const float gsf[2] = {tok0 ? small_int_to_float(gs_row[j]) : 0.f,
+                            TWO && tok1 ? small_int_to_float(gs_row[VPR + j]) : 0.f};
 #pragma unroll
-    for (int h = 0; h < 2; h++) {  // row g (h = 0) or g + 8
+      for (int h = 0; h < 2; h++) {  // row g (h = 0) or g + 8
 #pragma unroll
-      for (int qq = 0; qq < 2; qq++) {
-        if (qq == 1 && !TWO) break;  // warp-uniform
-        const int c = 2 * h + qq;
-        yacc[c] = fmaf(os[h].y, small_int_to_float(d1[c] + d2[c]), fmaf(os[h].x, gsf[qq], yacc[c]));
+        for (int qq = 0; qq < 2; qq++) {
+          if (qq == 1 && !TWO) break;  // warp-uniform
+          const int c = 2 * h + qq;
+          yacc[c] = fmaf(os[h].y, small_int_to_float(d1[c] + d2[c]), fmaf(os[h].x, gsf[qq], yacc[c]));
+        }
       }
     }
   }
@@ -960,10 +970,10 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
         for (int i = 0; i < cnt; i++) {
           const int kt = ktc + i;
           const uint8_t* tp = sbase + size_t(i) * a.tile_bytes;
-          uint4 b[4];
-#pragma unroll
-          for (int qq = 0; qq < 4; qq++) b[qq] = has_tok ? lds128(bsrc + kt * 256 + qq * 16) : make_uint4(0, 0, 0, 0);
           if constexpr (!BVSR) {
+            uint4 b[4];
+#pragma unroll
+            for (int qq = 0; qq < 4; qq++) b[qq] = has_tok ? lds128(bsrc + kt * 256 + qq * 16) : make_uint4(0, 0, 0, 0);
             uint4 w0[W0], w1[W1], w2[W2];
             if constexpr (F0 > 0) {
 #pragma unroll
@@ -981,13 +991,10 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
               stream_mma<F2, BSIGNED>(w2, b, c2);
             }
           } else {
-            uint4 w[4];
-#pragma unroll
-            for (int qq = 0; qq < 4; qq++) w[qq] = lds128(tp + qq * 512);
             const uint8_t* tidx = tp - lane * 16 + 2048;
             const uint2 i0 = *reinterpret_cast<const uint2*>(tidx + g * 8);
             const uint2 i1 = *reinterpret_cast<const uint2*>(tidx + (g + 8) * 8);
-            bvsr_tile(w, b, i0, i1, tab, fam, gsum + size_t(2 * t) * VPR + kt * 8, VPR, mg > 1, 2 * t < mg,
+            bvsr_tile(tp, bsrc + kt * 256, has_tok, i0, i1, tab, fam, gsum + size_t(2 * t) * VPR + kt * 8, VPR, mg > 1, 2 * t < mg,
                       2 * t + 1 < mg, want_acc, yacc, cacc);
           }
         }

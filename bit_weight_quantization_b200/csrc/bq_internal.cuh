@@ -29,7 +29,7 @@ enum : int {
 enum : int {
   AW_MAGIC = 0, AW_VERSION = 1, AW_FMT = 2, AW_M = 3, AW_K = 4, AW_KPAD = 5, AW_ABITS = 6,
   AW_LORA_RANK = 7, AW_TOTAL = 8, AW_OFF_CODES = 10, AW_OFF_TOK = 12, AW_OFF_GSUM = 14,
-  AW_OFF_U = 16, AW_OFF_XT = 18, AW_COUNT = 20
+  AW_OFF_U = 16, AW_OFF_XT = 18, AW_OFF_CT = 20, AW_COUNT = 22
 };
 
 constexpr int kBvsrSets = 256;
@@ -48,8 +48,15 @@ struct PkLayout {
 
 struct ActLayout {
   int fmt, M, K, K_pad, KT, a_bits, rank;
-  uint64_t off_codes, off_tok, off_gsum, off_u, off_xt, total;
+  uint64_t off_codes, off_tok, off_gsum, off_u, off_xt, off_ct, total;
 };
+
+// ABQ with 8-bit weight codes and 16..64 tokens runs on the tensor cores, whose act buffer also
+// holds the codes tile-major (one contiguous copy per k-tile for all tokens).
+constexpr int kTcMinM = 16, kTcMaxM = 64;
+inline bool tc_layer(int fmt, int w_bits, int M) {
+  return fmt == BQ_FMT_ABQ && w_bits == 8 && M >= kTcMinM && M <= kTcMaxM;
+}
 
 inline uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
 
@@ -132,12 +139,14 @@ inline ActLayout make_act_layout(const PkLayout& L, int M) {
   uint64_t gsum = L.fmt == BQ_FMT_BVSR4 ? uint64_t(M) * (L.K_pad / 32) * 4 : 0;
   uint64_t u = uint64_t(L.KT) * M * a.rank * 4;   // LoRA partials [KT][M][r]
   uint64_t xt = uint64_t(rabit_paths(L.fmt)) * M * L.K_pad * 4;
+  uint64_t ct = tc_layer(L.fmt, L.w_bits, M) ? codes : 0;  // the same codes, [KT][M][256]
   a.off_codes = 256;
   a.off_tok = align256(a.off_codes + codes);
   a.off_gsum = align256(a.off_tok + tok);
   a.off_u = align256(a.off_gsum + gsum);
   a.off_xt = align256(a.off_u + u);
-  a.total = align256(a.off_xt + xt);
+  a.off_ct = ct ? align256(a.off_xt + xt) : 0;
+  a.total = ct ? align256(a.off_ct + ct) : align256(a.off_xt + xt);
   return a;
 }
 

@@ -94,7 +94,7 @@
  * Activation buffer (device, 256-byte aligned), version 1.
  * Header: 64 x 32-bit words: 0 magic 0x43415142 ('BQAC') 1 version 2 format 3 M 4 K 5 K_pad
  *   6 a_bits 7 lora_rank 8-9 total_bytes 10-11 off_codes 12-13 off_tok 14-15 off_gsum
- *   16-17 off_u 18-19 off_xt.
+ *   16-17 off_u 18-19 off_xt 20-21 off_ct (0 when absent).
  * codes (formats 2-5): per token m and k-tile kt, 256 bytes; byte
  *   (m*(K_pad/256) + kt)*256 + 64t + 8mu + 4h + b holds the code of k = 32(8kt+mu)+16h+4t+b
  *   (the B-operand fragment order; int8 two's complement for A8 formats, whose bits are
@@ -104,6 +104,10 @@
  * u (ternary): f32 [K_pad/256][M][r] partial dot products of the unquantized bf16 x with A
  *   over each 256-k tile (each in k order); the layer forms SiLU(sum over tiles).
  * xt (RaBiT): f32 [P][M][K_pad] = h_p * x (no activation quantization).
+ * ct (ABQ with w_bits = 8 and 16 <= M <= 64 only): the same codes tile-major, byte
+ *   (kt*M + m)*256 + 64t + 8mu + 4h + b, so that the tensor-core layer fetches a k-tile of
+ *   every token in one copy; bq_gemm on such a layer runs a tcgen05 kind::i8 GEMM (128 rows of
+ *   the weights per CTA, the tokens as the MMA's N, accumulators in tensor memory).
  */
 #ifndef BQ_H
 #define BQ_H

@@ -253,7 +253,7 @@ def read_act(buf: bytes) -> dict:
     fmt, M, K, K_pad = _u32(buf, 2), _u32(buf, 3), _u32(buf, 4), _u32(buf, 5)
     a = dict(fmt=fmt, M=M, K=K, K_pad=K_pad, a_bits=_u32(buf, 6), lora_rank=_u32(buf, 7),
              total_bytes=_u64(buf, 8), off_codes=_u64(buf, 10), off_tok=_u64(buf, 12),
-             off_gsum=_u64(buf, 14), off_u=_u64(buf, 16), off_xt=_u64(buf, 18))
+             off_gsum=_u64(buf, 14), off_u=_u64(buf, 16), off_xt=_u64(buf, 18), off_ct=_u64(buf, 20))
     KT = K_pad // 256
     if fmt in (FMT_RABIT, FMT_RABIT3):
         P = 2 if fmt == FMT_RABIT else 3
@@ -273,6 +273,12 @@ def read_act(buf: bytes) -> dict:
         codes[:, 256 * kt + kin.ravel()] = raw[:, kt].reshape(M, -1)
     a["codes"] = codes[:, :K]
     a["codes_pad"] = codes[:, K:]
+    if a["off_ct"]:  # the tile-major copy [KT][M][256] (ABQ, 8-bit weights, 16..64 tokens)
+        rt = np.frombuffer(buf, dtype=dt, count=KT * M * 256, offset=a["off_ct"]).reshape(KT, M, 4, 8, 2, 4)
+        ct = np.zeros((M, K_pad), dtype=dt)
+        for kt in range(KT):
+            ct[:, 256 * kt + kin.ravel()] = rt[kt].reshape(M, -1)
+        a["codes_t"] = ct[:, :K]
     tok = np.frombuffer(buf, dtype="<u4", count=4 * M, offset=a["off_tok"]).reshape(M, 4)
     a["scale"] = tok[:, 0].view("<f4").copy()
     a["zero"] = tok[:, 1].view("<i4").copy()

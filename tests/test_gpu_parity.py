@@ -505,3 +505,18 @@ def test_bvsr_cluster_pack_and_layer(N, K, M, rounds):
     r = O.bvsr_layer(ref["codes"], ref["sets"], ref["table"], x)
     assert np.array_equal(acc.cpu().numpy()[:, rows], r["acc"])
     assert_y_close(y.cpu().numpy()[:, rows], r["y"], f"bvsr clustered {N}x{K}")
+
+
+# ------------------------------------------------------------------ ABQ W8 on the tcgen05 tensor cores
+@pytest.mark.parametrize("N,K,M,a", [(50, 384, 16, 8), (128, 256, 17, 8), (200, 640, 33, 4), (300, 4096, 64, 8),
+                                     (16, 1280, 64, 1), (97, 640, 48, 6), (1000, 2048, 32, 8)])
+def test_abq_w8_tensor_cores(N, K, M, a):
+    """ABQ with 8-bit weight codes and 16..64 tokens runs as a tcgen05 kind::i8 GEMM (operands
+    re-laid into canonical shared-memory layouts, accumulators in tensor memory): ragged row
+    counts (a partial 128-row CTA), token counts rounded up to the MMA's N, several activation
+    widths. act + gemm and the fused call both take it and agree bit for bit (GpuLayer); the
+    integer accumulators equal the oracle's, y within tolerance."""
+    gl = GpuLayer("abq", N, K, M, seed=N + M + a, w_bits=8, a_bits=a)
+    p = _pack_parity(gl, "abq", 8)
+    check_act(gl)
+    _layer_parity(gl, p, "abq", a)
