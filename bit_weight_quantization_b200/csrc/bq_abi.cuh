@@ -393,8 +393,30 @@ inline cudaError_t launch_fmt(const PkLayout& L, const LayerArgs& g, int NW, dim
   }
 }
 
-// ABQ with 8-bit weight codes and 16..64 tokens (from an act buffer) runs on the tensor cores.
+// ABQ with 16..64 tokens (from an act buffer) runs on the tensor cores.
 inline bool tc_eligible(const PkLayout& L, int M) { return tc_layer(L.fmt, L.w_bits, M); }
+
+// One instantiation per stream layout, so the statics below track that kernel's shared-memory
+// limit in the context that raised it.
+template <int F0, int F1, int F2>
+inline bq_status launch_abq_tc_f(const PkLayout& L, const TcArgs& t, cudaStream_t s) {
+  auto k = k_abq_tc<F0, F1, F2>;
+  static std::mutex mu;
+  static unsigned long long set_ctx = 0;
+  {
+    const unsigned long long ctx = current_context_id();
+    std::lock_guard<std::mutex> lock(mu);
+    if (ctx == 0 || ctx != set_ctx) {
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return BQ_ERR_CUDA;
+      }
+      set_ctx = ctx;
+    }
+  }
+  return launch_pdl(k, dim3((L.RB + kTcRb - 1) / kTcRb), dim3(kTcThreads), kTcSmem, s, t) == cudaSuccess
+             ? BQ_OK : BQ_ERR_CUDA;
+}
 
 inline bq_status launch_abq_tc(const PkLayout& L, const void* packed, const void* act, int M, float* y,
                                int64_t* acc, cudaStream_t s) {
@@ -413,21 +435,18 @@ inline bq_status launch_abq_tc(const PkLayout& L, const void* packed, const void
   t.y = y;
   t.acc = reinterpret_cast<long long*>(acc);
   t.N = L.N; t.K = L.K; t.KT = L.KT; t.RB = L.RB; t.M = M; t.Nmma = (M + 15) / 16 * 16; t.a_bits = L.a_bits;
-  static std::mutex mu;
-  static unsigned long long set_ctx = 0;
-  {
-    const unsigned long long ctx = current_context_id();
-    std::lock_guard<std::mutex> lock(mu);
-    if (ctx == 0 || ctx != set_ctx) {
-      if (cudaFuncSetAttribute(k_abq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) != cudaSuccess) {
-        (void)cudaGetLastError();
-        return BQ_ERR_CUDA;
-      }
-      set_ctx = ctx;
-    }
+  t.tile_bytes = L.tile_bytes;
+  switch (L.w_bits) {  // the fields of 8/4/2/1 bits from the low end of the code
+    case 1: return launch_abq_tc_f<1, 0, 0>(L, t, s);
+    case 2: return launch_abq_tc_f<2, 0, 0>(L, t, s);
+    case 3: return launch_abq_tc_f<2, 1, 0>(L, t, s);
+    case 4: return launch_abq_tc_f<4, 0, 0>(L, t, s);
+    case 5: return launch_abq_tc_f<4, 1, 0>(L, t, s);
+    case 6: return launch_abq_tc_f<4, 2, 0>(L, t, s);
+    case 7: return launch_abq_tc_f<4, 2, 1>(L, t, s);
+    case 8: return launch_abq_tc_f<8, 0, 0>(L, t, s);
+    default: return BQ_ERR_UNSUPPORTED;
   }
-  return launch_pdl(k_abq_tc, dim3((L.RB + kTcRb - 1) / kTcRb), dim3(kTcThreads), kTcSmem, s, t) == cudaSuccess
-             ? BQ_OK : BQ_ERR_CUDA;
 }
 
 inline bq_status launch_layer(const PkLayout& L, LayerArgs& g, bool fused, cudaStream_t s) {

@@ -51,11 +51,11 @@ struct ActLayout {
   uint64_t off_codes, off_tok, off_gsum, off_u, off_xt, off_ct, total;
 };
 
-// ABQ with 8-bit weight codes and 16..64 tokens runs on the tensor cores, whose act buffer also
-// holds the codes tile-major (one contiguous copy per k-tile for all tokens).
+// ABQ with 16..64 tokens runs on the tensor cores, whose act buffer also holds the codes
+// tile-major (one contiguous copy per k-tile for all tokens).
 constexpr int kTcMinM = 16, kTcMaxM = 64;
 inline bool tc_layer(int fmt, int w_bits, int M) {
-  return fmt == BQ_FMT_ABQ && w_bits == 8 && M >= kTcMinM && M <= kTcMaxM;
+  return fmt == BQ_FMT_ABQ && w_bits >= 1 && w_bits <= 8 && M >= kTcMinM && M <= kTcMaxM;
 }
 
 inline uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }

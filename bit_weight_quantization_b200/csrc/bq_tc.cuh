@@ -1,16 +1,18 @@
-// ABQ layer for 16..64 tokens with 8-bit weight codes on the fifth-generation tensor cores:
-// tcgen05.mma kind::i8 (u8 x u8 -> s32) with the accumulators in tensor memory.
+// ABQ layer for 16..64 tokens on the fifth-generation tensor cores: tcgen05.mma kind::i8
+// (u8 x u8 -> s32) with the accumulators in tensor memory.
 //
-// ABQ page §3.2 eq.(3): with codes q_w (8 bits) and q_x (a bits), P = sum_k q_w q_x is a dense
+// ABQ page §3.2 eq.(3): with codes q_w (w bits) and q_x (a bits), P = sum_k q_w q_x is a dense
 // integer contraction of M tokens against N rows, the case where the tensor cores do the work
 // (the pages' binary tensor-core decomposition is the same sum taken bit-plane by bit-plane).
 //
 // One CTA computes 128 weight rows (eight 16-row blocks, the MMA's M) for all tokens (the MMA's
 // N, M rounded up to a multiple of 16). Per 256-k tile: bulk copies bring the eight packed tiles
-// (the A-fragment order of the int8 m16n8k32 MMA) and the tile's act codes of all tokens (the
-// act buffer's tile-major copy, B-fragment order per token) into one of three raw stages; the
-// eight warps re-lay both into the canonical K-major layout of the MMA operands (8-row x
-// 16-byte core matrices, no swizzle); one thread issues the tile's eight MMAs (K = 32 each) and
+// (bit-field streams in the A-fragment order of the int8 m16n8k32 MMA) and the tile's act codes
+// of all tokens (the act buffer's tile-major copy, B-fragment order per token) into one of
+// three raw stages; the eight warps re-lay both into the canonical K-major layout of the MMA
+// operands (8-row x 16-byte core matrices, no swizzle), assembling each weight code byte from
+// its streams' fields (code = sum_s field_s << shift_s); one thread issues the tile's eight MMAs
+// (K = 32 each) and
 // commits them to an mbarrier, which frees the operand buffer for the next tile. After the last
 // tile the warps read the accumulators from tensor memory (tcgen05.ld, warps w and w + 4 the
 // two column halves of lanes 32w .. 32w + 31) and run the ABQ zero-point epilogue. Every wait
@@ -29,7 +31,7 @@ constexpr int kTcThreads = 256;
 constexpr int kTcStages = 3;                 // raw stages
 constexpr int kTcColsAlloc = 64;             // tensor-memory columns (one per token)
 // shared memory carve (bytes)
-constexpr uint32_t kTcRawA = kTcRb * 4096;                 // one raw stage of weight tiles
+constexpr uint32_t kTcRawA = kTcRb * 4096;                 // one raw stage of weight tiles (8-bit at most)
 constexpr uint32_t kTcRawB = kTcMaxN * 256;                // one raw stage of act codes
 constexpr uint32_t kTcCanA = kTcRows * 256;                // canonical A of one k-tile (32 KB)
 constexpr uint32_t kTcCanB = kTcMaxN * 256;                // canonical B of one k-tile (16 KB)
@@ -44,7 +46,7 @@ constexpr uint32_t kTcSmem = kTcOffBar + 128;
 constexpr uint32_t kTcLboA = 2048, kTcSboA = 128, kTcLboB = 1024, kTcSboB = 128;
 
 struct TcArgs {
-  const uint8_t* tiles;      // packed W8 tiles [RB][KT][4096]
+  const uint8_t* tiles;      // packed tiles [RB][KT][tile_bytes]
   const float* row_delta;    // Delta_w [N_pad]
   const int* row_zero;       // z_w
   const int* row_sum;        // S_w
@@ -54,7 +56,7 @@ struct TcArgs {
   unsigned long long act_total;
   float* y;                  // [M][N]
   long long* acc;            // [M][N] or null
-  int N, K, KT, RB, M, Nmma, a_bits;
+  int N, K, KT, RB, M, Nmma, a_bits, tile_bytes;
 };
 
 __device__ __forceinline__ bool tc_header_ok(const uint32_t* h, const TcArgs& a) {
@@ -106,6 +108,23 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
 }
 
+// Field f (bits) of 32-k chunk kc for the four words of this lane's 16 bytes of a stream of width F:
+// the chunk is field kc % (8/F) of uint4 kc / (8/F); the field values land at bit offset SH.
+template <int F, int SH>
+__device__ __forceinline__ void tc_stream_fields(const uint8_t* base, int kc, int lane, uint32_t (&w4)[4]) {
+  constexpr int per = 8 / F;
+  constexpr uint32_t mask = ((1u << F) - 1u) * 0x01010101u;
+  const uint4 v = *reinterpret_cast<const uint4*>(base + ((kc / per) * 32 + lane) * 16);
+  const uint32_t sh = uint32_t(F * (kc % per));
+  w4[0] |= ((v.x >> sh) & mask) << SH;
+  w4[1] |= ((v.y >> sh) & mask) << SH;
+  w4[2] |= ((v.z >> sh) & mask) << SH;
+  w4[3] |= ((v.w >> sh) & mask) << SH;
+}
+
+// F0, F1, F2: the field widths of the layer's bit-field streams (0 = no such stream), from the
+// low end of the code: W8 [8], W4 [4], W6 [4, 2], W7 [4, 2, 1], ...
+template <int F0, int F1, int F2>
 __global__ void __launch_bounds__(kTcThreads, 1) k_abq_tc(const __grid_constant__ TcArgs a) {
   extern __shared__ __align__(128) uint8_t tc_smem[];  // operands need 16-byte alignment (no swizzle)
   uint8_t* smem = tc_smem;
@@ -115,7 +134,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_abq_tc(const __grid_constant_
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTcOffBar);  // raw stage s filled
   uint64_t* mmab = full + kTcStages;                                // the operand buffer's MMAs done
   uint32_t* words = reinterpret_cast<uint32_t*>(mmab + 1);          // [0] tmem address, [1] failure, [2] bad header
-  const uint32_t wbytes = uint32_t(nrb) * 4096u, cbytes = uint32_t(a.M) * 256u;
+  const uint32_t tb = uint32_t(a.tile_bytes);
+  const uint32_t wbytes = uint32_t(nrb) * tb, cbytes = uint32_t(a.M) * 256u;
 
   pdl_trigger();
   if (tid == 0) {
@@ -141,8 +161,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_abq_tc(const __grid_constant_
 
   auto issue_w = [&](int kt, int s) {  // weights are constant: fetched before the dependency wait too
     for (int r = 0; r < nrb; r++)
-      bulk_g2s(smem + kTcOffRawA + s * kTcRawA + r * 4096,
-               a.tiles + (size_t(rb0 + r) * a.KT + kt) * 4096, 4096, &full[s]);
+      bulk_g2s(smem + kTcOffRawA + s * kTcRawA + r * tb, a.tiles + (size_t(rb0 + r) * a.KT + kt) * tb, tb, &full[s]);
   };
   auto issue_c = [&](int kt, int s) {  // one contiguous copy: tile kt of every token
     bulk_g2s(smem + kTcOffRawB + s * kTcRawB, a.act_codes + size_t(kt) * a.M * 256, cbytes, &full[s]);
@@ -183,13 +202,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_abq_tc(const __grid_constant_
       const uint8_t* ra = smem + kTcOffRawA + s * kTcRawA;
       uint8_t* can_a = smem + kTcOffCanA;
       const int g = lane >> 2, t = lane & 3;
-      for (int rbl = 0; rbl < nrb; rbl++) {  // warp = u: its 32 lanes' 16-byte chunks
-        const int u = warp;
-        const uint4 v = *reinterpret_cast<const uint4*>(ra + rbl * 4096 + (u * 32 + lane) * 16);
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      const int kc = warp;  // this warp's 32-k chunk of the tile
+      for (int rbl = 0; rbl < nrb; rbl++) {
+        // word w of a lane holds row g + 8(w & 1) of the block at k = 32kc + 16(w >> 1) + 4t + b;
+        // stream s keeps that chunk as field kc % (8/f) of its uint4 kc / (8/f)
+        uint32_t w4[4] = {0u, 0u, 0u, 0u};
+        const uint8_t* tile = ra + rbl * tb;
+        tc_stream_fields<F0, 0>(tile, kc, lane, w4);
+        if constexpr (F1 > 0) tc_stream_fields<F1, F0>(tile + 512 * F0, kc, lane, w4);
+        if constexpr (F2 > 0) tc_stream_fields<F2, F0 + F1>(tile + 512 * (F0 + F1), kc, lane, w4);
 #pragma unroll
-        for (int w = 0; w < 4; w++) {  // row g + 8(w & 1) of the block, k = 32u + 16(w >> 1) + 4t + b
-          const uint32_t off = uint32_t(2 * u + (w >> 1)) * kTcLboA + uint32_t(2 * rbl + (w & 1)) * kTcSboA +
+        for (int w = 0; w < 4; w++) {
+          const uint32_t off = uint32_t(2 * kc + (w >> 1)) * kTcLboA + uint32_t(2 * rbl + (w & 1)) * kTcSboA +
                                uint32_t(g) * 16 + uint32_t(t) * 4;
           *reinterpret_cast<uint32_t*>(can_a + off) = w4[w];
         }

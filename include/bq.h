@@ -104,7 +104,7 @@
  * u (ternary): f32 [K_pad/256][M][r] partial dot products of the unquantized bf16 x with A
  *   over each 256-k tile (each in k order); the layer forms SiLU(sum over tiles).
  * xt (RaBiT): f32 [P][M][K_pad] = h_p * x (no activation quantization).
- * ct (ABQ with w_bits = 8 and 16 <= M <= 64 only): the same codes tile-major, byte
+ * ct (ABQ with 16 <= M <= 64 only): the same codes tile-major, byte
  *   (kt*M + m)*256 + 64t + 8mu + 4h + b, so that the tensor-core layer fetches a k-tile of
  *   every token in one copy; bq_gemm on such a layer runs a tcgen05 kind::i8 GEMM (128 rows of
  *   the weights per CTA, the tokens as the MMA's N, accumulators in tensor memory).

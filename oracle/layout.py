@@ -273,7 +273,7 @@ def read_act(buf: bytes) -> dict:
         codes[:, 256 * kt + kin.ravel()] = raw[:, kt].reshape(M, -1)
     a["codes"] = codes[:, :K]
     a["codes_pad"] = codes[:, K:]
-    if a["off_ct"]:  # the tile-major copy [KT][M][256] (ABQ, 8-bit weights, 16..64 tokens)
+    if a["off_ct"]:  # the tile-major copy [KT][M][256] (ABQ with 16..64 tokens)
         rt = np.frombuffer(buf, dtype=dt, count=KT * M * 256, offset=a["off_ct"]).reshape(KT, M, 4, 8, 2, 4)
         ct = np.zeros((M, K_pad), dtype=dt)
         for kt in range(KT):

@@ -203,7 +203,7 @@ def check_act(gl: GpuLayer):
     if gl.fmt == "abq":
         Qx, dx, zx = O.quantize_rows_asym(x, gl.a_bits)
         assert np.array_equal(a["codes"].astype(np.int32), Qx)
-        if gl.w_bits == 8 and 16 <= gl.M <= 64:   # the tile-major copy the tensor-core layer reads
+        if 16 <= gl.M <= 64:   # the tile-major copy the tensor-core layer reads
             assert np.array_equal(a["codes_t"].astype(np.int32), Qx)
         else:
             assert "codes_t" not in a
