@@ -396,26 +396,124 @@ inline cudaError_t launch_fmt(const PkLayout& L, const LayerArgs& g, int NW, dim
 // ABQ with 16..64 tokens (from an act buffer) runs on the tensor cores.
 inline bool tc_eligible(const PkLayout& L, int M) { return tc_layer(L.fmt, L.w_bits, M); }
 
+// The packed weight tiles of a layer as the tensor-core kernel's 3-D TMA map (TcTensorMap).
+// cuTensorMapEncodeTiled is a host-side encode (no device work), resolved once through the
+// runtime like the context query above.
+inline bool encode_weight_map(const PkLayout& L, const void* tiles, TcTensorMap* out) {
+  typedef CUresult (*EncodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+  static_assert(sizeof(TcTensorMap) == sizeof(CUtensorMap), "tensor map size");
+  static EncodeTiled encode = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      encode = reinterpret_cast<EncodeTiled>(f);
+    (void)cudaGetLastError();
+  });
+  if (!encode) return false;
+  const cuuint64_t dims[3] = {256u, cuuint64_t(L.KT) * L.tile_bytes / 256u, cuuint64_t(L.RB)};
+  const cuuint64_t strides[2] = {256u, cuuint64_t(L.KT) * L.tile_bytes};  // bytes, dims 1 and 2
+  const cuuint32_t box[3] = {256u, cuuint32_t(L.tile_bytes / 256), cuuint32_t(kTcRb)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUtensorMap m;
+  if (encode(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(tiles), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  std::memcpy(out, &m, sizeof(m));
+  return true;
+}
+
+// Cluster size for G row groups of 128 and KT tiles: the split of the tiles that minimises
+// waves x (tiles per CTA + kTcFixedTiles), where a wave is as many clusters as the device holds
+// at once (max_clusters[cs], from the occupancy query) and kTcFixedTiles is a CTA's fixed cost
+// (first copies, epilogue, cluster reduction) in tiles; ties go to the smaller cluster.
+constexpr int kTcFixedTiles = 4;
+inline int tc_cluster_size(int G, int KT, const int* max_clusters) {
+  int best = 1;
+  long long best_cost = -1;
+  for (int cs = 1; cs <= kTcMaxCluster && cs <= KT; cs++) {
+    if (max_clusters[cs] <= 0) continue;
+    const long long waves = (G + max_clusters[cs] - 1) / max_clusters[cs];
+    const long long cost = waves * ((KT + cs - 1) / cs + kTcFixedTiles);
+    if (best_cost < 0 || cost < best_cost) { best = cs; best_cost = cost; }
+  }
+  return best;
+}
+
 // One instantiation per stream layout, so the statics below track that kernel's shared-memory
-// limit in the context that raised it.
+// limit and cluster occupancy in the context that set them.
 template <int F0, int F1, int F2>
-inline bq_status launch_abq_tc_f(const PkLayout& L, const TcArgs& t, cudaStream_t s) {
+inline bq_status launch_abq_tc_f(const PkLayout& L, TcArgs t, cudaStream_t s) {
   auto k = k_abq_tc<F0, F1, F2>;
   static std::mutex mu;
   static unsigned long long set_ctx = 0;
+  static int max_clusters[kTcMaxN / 16 + 1][kTcMaxCluster + 1];  // [Mp / 16][cluster size]
+  const int G = (L.RB + kTcRb - 1) / kTcRb;
+  const uint32_t smem = kTcOffStages + uint32_t(t.stages) * uint32_t(t.stage_bytes) + kTcBarBytes;
+  int cs = 1;
   {
     const unsigned long long ctx = current_context_id();
     std::lock_guard<std::mutex> lock(mu);
     if (ctx == 0 || ctx != set_ctx) {
-      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem)) != cudaSuccess) {
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmemMax)) != cudaSuccess) {
         (void)cudaGetLastError();
         return BQ_ERR_CUDA;
       }
+      for (auto& r : max_clusters)
+        for (int& c : r) c = -1;
       set_ctx = ctx;
     }
+    int* mc = max_clusters[t.Mp / 16];
+    if (mc[1] < 0) {
+      int dev = 0, sms = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return BQ_ERR_CUDA;
+      }
+      for (int c = 1; c <= kTcMaxCluster; c++) {
+        cudaLaunchConfig_t q = {};
+        q.gridDim = dim3(unsigned(c));
+        q.blockDim = dim3(kTcThreads);
+        q.dynamicSmemBytes = smem;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = unsigned(c);
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        q.attrs = at;
+        q.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, k, &q) != cudaSuccess) {
+          (void)cudaGetLastError();
+          n = c == 1 ? sms : 0;  // without the query: no clusters, one CTA per SM
+        }
+        mc[c] = n;
+      }
+    }
+    cs = tc_cluster_size(G, L.KT, mc);
   }
-  return launch_pdl(k, dim3((L.RB + kTcRb - 1) / kTcRb), dim3(kTcThreads), kTcSmem, s, t) == cudaSuccess
-             ? BQ_OK : BQ_ERR_CUDA;
+  t.CS = cs;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(G * cs));
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributeClusterDimension;
+  at[1].val.clusterDim.x = unsigned(cs);
+  at[1].val.clusterDim.y = 1;
+  at[1].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = cs > 1 ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, k, t) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
 inline bq_status launch_abq_tc(const PkLayout& L, const void* packed, const void* act, int M, float* y,
@@ -424,7 +522,7 @@ inline bq_status launch_abq_tc(const PkLayout& L, const void* packed, const void
   const uint8_t* Ab = static_cast<const uint8_t*>(act);
   const ActLayout A = make_act_layout(L, M);
   TcArgs t{};
-  t.tiles = P + L.off_tiles;
+  if (!encode_weight_map(L, P + L.off_tiles, &t.wmap)) return BQ_ERR_CUDA;
   t.row_delta = reinterpret_cast<const float*>(P + L.off_rows);
   t.row_zero = reinterpret_cast<const int*>(P + L.off_rows + 4ull * L.N_pad);
   t.row_sum = reinterpret_cast<const int*>(P + L.off_rows + 8ull * L.N_pad);
@@ -434,8 +532,12 @@ inline bq_status launch_abq_tc(const PkLayout& L, const void* packed, const void
   t.act_total = A.total;
   t.y = y;
   t.acc = reinterpret_cast<long long*>(acc);
-  t.N = L.N; t.K = L.K; t.KT = L.KT; t.RB = L.RB; t.M = M; t.Nmma = (M + 15) / 16 * 16; t.a_bits = L.a_bits;
+  t.N = L.N; t.K = L.K; t.KT = L.KT; t.RB = L.RB; t.M = M; t.Mp = tc_tokens(M); t.a_bits = L.a_bits;
   t.tile_bytes = L.tile_bytes;
+  t.stages = tc_stages(L.tile_bytes, t.Mp);
+  t.stage_bytes = kTcRb * L.tile_bytes + t.Mp * 256;
+  t.CS = 1;
+  if (t.stages < 3) return BQ_ERR_UNSUPPORTED;
   switch (L.w_bits) {  // the fields of 8/4/2/1 bits from the low end of the code
     case 1: return launch_abq_tc_f<1, 0, 0>(L, t, s);
     case 2: return launch_abq_tc_f<2, 0, 0>(L, t, s);

@@ -137,8 +137,15 @@ __global__ void __launch_bounds__(1024) k_act_quant(ActArgs a) {
     }
     const int kt = k >> 8;
     codes[kt * 64 + code_word_in_tile(k & 255)] = word;
-    if (a.off_ct)  // the tile-major copy: tile kt of token m at (kt M + m) 256
-      reinterpret_cast<uint32_t*>(a.act + a.off_ct)[(size_t(kt) * a.M + m) * 64 + code_word_in_tile(k & 255)] = word;
+    if (a.off_ct) {  // the tensor-core copy: [KT][16 k-units][Mp / 8][8 tokens][16 bytes]
+      const int Mp = tc_tokens(a.M), kk = k & 255;
+      uint8_t* ct = a.act + a.off_ct + size_t(kt) * Mp * 256 + (kk >> 4) * (Mp * 16) + (kk & 15);
+      *reinterpret_cast<uint32_t*>(ct + (m >> 3) * 128 + (m & 7) * 16) = word;
+      if (m < Mp - a.M) {  // token M + m pads the MMA's N to a multiple of 16 (Mp - M < 16 <= M)
+        const int mp = a.M + m;
+        *reinterpret_cast<uint32_t*>(ct + (mp >> 3) * 128 + (mp & 7) * 16) = 0u;
+      }
+    }
     if (FMT == BQ_FMT_BVSR4) {
       // 8 consecutive threads cover one 32-element vector (blockDim and 64 are multiples of 8)
       qs += __shfl_xor_sync(0xffffffffu, qs, 1);

@@ -51,12 +51,14 @@ struct ActLayout {
   uint64_t off_codes, off_tok, off_gsum, off_u, off_xt, off_ct, total;
 };
 
-// ABQ with 16..64 tokens runs on the tensor cores, whose act buffer also holds the codes
-// tile-major (one contiguous copy per k-tile for all tokens).
+// ABQ with 16..64 tokens runs on the tensor cores, whose act buffer also holds the codes in
+// the MMA's operand layout: per k-tile one contiguous block of Mp = M rounded up to 16 tokens
+// (the padding tokens' codes zero).
 constexpr int kTcMinM = 16, kTcMaxM = 64;
 inline bool tc_layer(int fmt, int w_bits, int M) {
   return fmt == BQ_FMT_ABQ && w_bits >= 1 && w_bits <= 8 && M >= kTcMinM && M <= kTcMaxM;
 }
+__host__ __device__ inline int tc_tokens(int M) { return (M + 15) / 16 * 16; }
 
 inline uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
 
@@ -139,7 +141,8 @@ inline ActLayout make_act_layout(const PkLayout& L, int M) {
   uint64_t gsum = L.fmt == BQ_FMT_BVSR4 ? uint64_t(M) * (L.K_pad / 32) * 4 : 0;
   uint64_t u = uint64_t(L.KT) * M * a.rank * 4;   // LoRA partials [KT][M][r]
   uint64_t xt = uint64_t(rabit_paths(L.fmt)) * M * L.K_pad * 4;
-  uint64_t ct = tc_layer(L.fmt, L.w_bits, M) ? codes : 0;  // the same codes, [KT][M][256]
+  // the same codes, [KT][16 k-units][Mp / 8][8 tokens][16 bytes]
+  uint64_t ct = tc_layer(L.fmt, L.w_bits, M) ? uint64_t(tc_tokens(M)) * L.KT * 256 : 0;
   a.off_codes = 256;
   a.off_tok = align256(a.off_codes + codes);
   a.off_gsum = align256(a.off_tok + tok);

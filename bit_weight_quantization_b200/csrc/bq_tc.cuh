@@ -6,18 +6,26 @@
 // (the pages' binary tensor-core decomposition is the same sum taken bit-plane by bit-plane).
 //
 // One CTA computes 128 weight rows (eight 16-row blocks, the MMA's M) for all tokens (the MMA's
-// N, M rounded up to a multiple of 16). Per 256-k tile: bulk copies bring the eight packed tiles
-// (bit-field streams in the A-fragment order of the int8 m16n8k32 MMA) and the tile's act codes
-// of all tokens (the act buffer's tile-major copy, B-fragment order per token) into one of
-// three raw stages; the eight warps re-lay both into the canonical K-major layout of the MMA
-// operands (8-row x 16-byte core matrices, no swizzle), assembling each weight code byte from
-// its streams' fields (code = sum_s field_s << shift_s); one thread issues the tile's eight MMAs
-// (K = 32 each) and
-// commits them to an mbarrier, which frees the operand buffer for the next tile. After the last
-// tile the warps read the accumulators from tensor memory (tcgen05.ld, warps w and w + 4 the
-// two column halves of lanes 32w .. 32w + 31) and run the ABQ zero-point epilogue. Every wait
-// is bounded: on expiry the device error word is raised, no further MMA is issued, outstanding
-// copies and MMAs are waited for, and the tensor memory is freed.
+// N = Mp, M rounded up to a multiple of 16) over a range of the 256-k tiles; a cluster of CS
+// CTAs splits the tiles of one 128-row group, and each CTA then sums one slice of the tokens
+// over the cluster's partial products through distributed shared memory (integer adds: exact
+// in any order) and writes that slice's outputs.
+//
+// Warp roles, coupled only by mbarriers. The producer warp fills a ring of stages sized to the
+// shared memory: per tile one TMA tensor copy of the eight packed weight tiles (bit-field
+// streams in the A-fragment order of the int8 m16n8k32 MMA; rows past the layer read as zero)
+// and one bulk copy of the act buffer's tensor-core block of the tile (already in the
+// canonical operand layout, read by the MMA in place). Eight re-layout warps copy each weight
+// tile into one of two canonical K-major operand buffers (8-row x 16-byte core matrices, no
+// swizzle), assembling each code byte from its streams' fields (code = sum_s field_s << shift_s),
+// and arrive on the buffer's "ready" barrier. The MMA warp issues the tile's eight MMAs (K = 32
+// each) and commits them to the stage's "empty" barrier, on which the producer refills the
+// stage and the re-layout warps reuse the tile's operand buffer two tiles later. After the last tile the re-layout warps read the
+// accumulators from tensor memory (tcgen05.ld, warps w and w + 4 the two column halves of lanes
+// 32w .. 32w + 31) and run the ABQ zero-point epilogue. Every wait is bounded and also ends
+// when another role has stopped: on expiry the device error word is raised, no further MMA is
+// issued, outstanding copies and MMAs are waited for, every CTA of the cluster still takes both
+// cluster barriers, and the tensor memory is freed.
 #pragma once
 
 #include "bq_gemv.cuh"
@@ -27,37 +35,51 @@ namespace bqi {
 constexpr int kTcRows = 128;                 // weight rows per CTA
 constexpr int kTcRb = kTcRows / 16;          // row blocks per CTA
 constexpr int kTcMaxN = 64;                  // tokens (MMA N) at most
-constexpr int kTcThreads = 256;
-constexpr int kTcStages = 3;                 // raw stages
+constexpr int kTcLayoutWarps = 8;           // re-layout / epilogue warps
+constexpr int kTcProducerWarp = kTcLayoutWarps, kTcMmaWarp = kTcLayoutWarps + 1;
+constexpr int kTcThreads = (kTcLayoutWarps + 2) * 32;
+constexpr int kTcMaxStages = 8;
+constexpr int kTcMaxCluster = 8;             // portable cluster size
 constexpr int kTcColsAlloc = 64;             // tensor-memory columns (one per token)
-// shared memory carve (bytes)
-constexpr uint32_t kTcRawA = kTcRb * 4096;                 // one raw stage of weight tiles (8-bit at most)
-constexpr uint32_t kTcRawB = kTcMaxN * 256;                // one raw stage of act codes
-constexpr uint32_t kTcCanA = kTcRows * 256;                // canonical A of one k-tile (32 KB)
-constexpr uint32_t kTcCanB = kTcMaxN * 256;                // canonical B of one k-tile (16 KB)
-constexpr uint32_t kTcOffRawA = 0;
-constexpr uint32_t kTcOffRawB = kTcOffRawA + kTcStages * kTcRawA;
-constexpr uint32_t kTcOffCanA = kTcOffRawB + kTcStages * kTcRawB;
-constexpr uint32_t kTcOffCanB = kTcOffCanA + kTcCanA;
-constexpr uint32_t kTcOffBar = kTcOffCanB + kTcCanB;       // full[3], mma, then words
-constexpr uint32_t kTcSmem = kTcOffBar + 128;
-// canonical strides: A core matrix rows 16 B apart, 8-row groups 128 B apart, 16-byte k-units
-// 2048 B apart (16 row groups); B likewise with 8 token groups per k-unit (1024 B)
-constexpr uint32_t kTcLboA = 2048, kTcSboA = 128, kTcLboB = 1024, kTcSboB = 128;
+constexpr uint32_t kTcCanA = kTcRows * 256;  // canonical A of one k-tile (32 KB); two buffers
+constexpr uint32_t kTcOffStages = 2 * kTcCanA;
+// after the stages: full[8] (0), empty[8] (64), ready[2] (144), words[8] (160),
+// and the token parameters Delta_x, z_x, S_x - K z_x [3][64] (256)
+constexpr uint32_t kTcBarBytes = 1024;
+constexpr uint32_t kTcSmemMax = 227 * 1024;
+// canonical strides of A: core matrix rows 16 B apart, 8-row groups 128 B apart, 16-byte
+// k-units 2048 B apart (16 row groups); B: 8-token groups 128 B apart, k-units Mp * 16 B apart
+constexpr uint32_t kTcLboA = 2048, kTcSboA = 128, kTcSboB = 128;
+
+// The packed weight tiles as a 3-D uint8 tensor for the TMA: x = 256 bytes, y = 256-byte
+// chunks along a row block's tiles (KT tile_bytes / 256), z = row blocks; a box of
+// (256, tile_bytes / 256, 8) is one k-tile of eight row blocks, laid out in shared memory as
+// the eight tiles back to back. The map is opaque (CUtensorMap, 128 bytes, 64-byte aligned).
+struct alignas(64) TcTensorMap {
+  unsigned long long opaque[16];
+};
 
 struct TcArgs {
-  const uint8_t* tiles;      // packed tiles [RB][KT][tile_bytes]
+  TcTensorMap wmap;          // the packed weight tiles (see TcTensorMap)
   const float* row_delta;    // Delta_w [N_pad]
   const int* row_zero;       // z_w
   const int* row_sum;        // S_w
   const uint32_t* act_hdr;
-  const uint8_t* act_codes;  // tile-major [KT][M][256]
+  const uint8_t* act_codes;  // tensor-core copy [KT][16 k-units][Mp/8][8 tokens][16 B]
   const uint32_t* act_tok;   // [M][4]: Delta_x, z_x, S_x
   unsigned long long act_total;
   float* y;                  // [M][N]
   long long* acc;            // [M][N] or null
-  int N, K, KT, RB, M, Nmma, a_bits, tile_bytes;
+  int N, K, KT, RB, M, Mp, a_bits, tile_bytes;
+  int stages, stage_bytes, CS;  // ring stages, bytes per stage (weights then codes), cluster size
 };
+
+// Ring stages that fit next to the two operand buffers, for weight tiles of tile_bytes and Mp tokens.
+__host__ __device__ inline int tc_stages(int tile_bytes, int Mp) {
+  const int stage = kTcRb * tile_bytes + Mp * 256;
+  const int s = int((kTcSmemMax - kTcOffStages - kTcBarBytes) / uint32_t(stage));
+  return s < kTcMaxStages ? s : kTcMaxStages;
+}
 
 __device__ __forceinline__ bool tc_header_ok(const uint32_t* h, const TcArgs& a) {
   return h[AW_MAGIC] == kActMagic && h[AW_VERSION] == kVersion && h[AW_FMT] == uint32_t(BQ_FMT_ABQ) &&
@@ -108,6 +130,50 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
 }
 
+// one box of a 3-D tensor map into shared memory, completing bytes on bar (no multicast)
+__device__ __forceinline__ void tma_load_3d(void* dst, const TcTensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// distributed shared memory of a cluster
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t dsmem_map(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ uint32_t dsmem_ld(uint32_t raddr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];\n" : "=r"(v) : "r"(raddr) : "memory");
+  return v;
+}
+// every thread of every CTA of the cluster arrives (release) and waits (acquire); the CTAs of a
+// cluster are co-scheduled, and each one passes exactly two of these on every path
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// bounded wait that also gives up once another role of the block has stopped (*stop != 0)
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, const uint32_t* stop) {
+  for (uint32_t i = 0; i < kMaxSpin; i++) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*reinterpret_cast<const volatile uint32_t*>(stop)) return false;
+  }
+  atomicOr(&g_bq_device_error, kErrCopyTimeout);
+  return false;
+}
+
 // Field f (bits) of 32-k chunk kc for the four words of this lane's 16 bytes of a stream of width F:
 // the chunk is field kc % (8/F) of uint4 kc / (8/F); the field values land at bit offset SH.
 template <int F, int SH>
@@ -129,21 +195,34 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_abq_tc(const __grid_constant_
   extern __shared__ __align__(128) uint8_t tc_smem[];  // operands need 16-byte alignment (no swizzle)
   uint8_t* smem = tc_smem;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int rb0 = blockIdx.x * kTcRb;
-  const int nrb = min(kTcRb, a.RB - rb0);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTcOffBar);  // raw stage s filled
-  uint64_t* mmab = full + kTcStages;                                // the operand buffer's MMAs done
-  uint32_t* words = reinterpret_cast<uint32_t*>(mmab + 1);          // [0] tmem address, [1] failure, [2] bad header
+  const int CS = a.CS, S = a.stages;
+  const uint32_t rank = CS > 1 ? cluster_rank() : 0u;
+  const int rb0 = (blockIdx.x / CS) * kTcRb;
+  const int kt0 = int(rank) * a.KT / CS, nt = (int(rank) + 1) * a.KT / CS - kt0;  // this CTA's tiles
+  uint8_t* stages = smem + kTcOffStages;
+  uint8_t* region = stages + size_t(S) * a.stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(region);         // stage filled
+  uint64_t* empty = reinterpret_cast<uint64_t*>(region + 64);   // stage's MMAs done
+  uint64_t* ready = reinterpret_cast<uint64_t*>(region + 144);  // operand buffer written
+  // words: [0] tmem address, [1] a role stopped, [2] bad header, [3] this CTA failed,
+  // [4] tiles whose copies were issued, [5] tiles whose MMAs were committed
+  uint32_t* words = reinterpret_cast<uint32_t*>(region + 160);
+  float* tok_dx = reinterpret_cast<float*>(region + 256);
+  int* tok_zx = reinterpret_cast<int*>(region + 256 + 4 * kTcMaxN);
+  int* tok_t = reinterpret_cast<int*>(region + 256 + 8 * kTcMaxN);  // S_x - K z_x (mod 2^32)
   const uint32_t tb = uint32_t(a.tile_bytes);
-  const uint32_t wbytes = uint32_t(nrb) * tb, cbytes = uint32_t(a.M) * 256u;
+  const uint32_t raw_a = uint32_t(kTcRb) * tb;  // a stage: the weight box, then the codes
+  const uint32_t cbytes = uint32_t(a.Mp) * 256u;
 
   pdl_trigger();
   if (tid == 0) {
-    for (int st = 0; st < kTcStages; st++) mbar_init(&full[st], 1);
-    mbar_init(mmab, 1);
+    for (int st = 0; st < S; st++) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], 1);
+    }
+    for (int b = 0; b < 2; b++) mbar_init(&ready[b], kTcLayoutWarps);
     fence_mbar_init();
-    words[1] = 0;
-    words[2] = 0;
+    for (int i = 1; i < 8; i++) words[i] = 0;
   }
   if (warp == 0) {  // tensor-memory accumulators: 128 lanes x 64 columns
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(words)),
@@ -151,59 +230,111 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_abq_tc(const __grid_constant_
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
-  // the padding tokens' operand rows stay zero
-  for (uint32_t i = tid; i < kTcCanB / 16; i += kTcThreads)
-    reinterpret_cast<uint4*>(smem + kTcOffCanB)[i] = make_uint4(0, 0, 0, 0);
+  // the row this thread writes in the epilogue (row tid % 128 of the CTA's 128) and its
+  // constant weight parameters
+  const int row = rb0 * 16 + (tid & 127);
+  float dw = 0.f;
+  uint32_t zw = 0, sw = 0;
+  if (warp < kTcLayoutWarps && row < a.N) {
+    dw = __ldg(a.row_delta + row);
+    zw = uint32_t(__ldg(a.row_zero + row));
+    sw = uint32_t(__ldg(a.row_sum + row));
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = words[0];
 
-  auto issue_w = [&](int kt, int s) {  // weights are constant: fetched before the dependency wait too
-    for (int r = 0; r < nrb; r++)
-      bulk_g2s(smem + kTcOffRawA + s * kTcRawA + r * tb, a.tiles + (size_t(rb0 + r) * a.KT + kt) * tb, tb, &full[s]);
+  auto stage_of = [&](int j) { return stages + size_t(j % S) * a.stage_bytes; };
+  auto issue_w = [&](int j) {  // weights are constant: fetched before the dependency wait too
+    tma_load_3d(stage_of(j), &a.wmap, 0, (kt0 + j) * int(tb / 256u), rb0, &full[j % S]);
   };
-  auto issue_c = [&](int kt, int s) {  // one contiguous copy: tile kt of every token
-    bulk_g2s(smem + kTcOffRawB + s * kTcRawB, a.act_codes + size_t(kt) * a.M * 256, cbytes, &full[s]);
+  auto issue_c = [&](int j) {  // one contiguous copy: the tile's codes of every token
+    bulk_g2s(stage_of(j) + raw_a, a.act_codes + size_t(kt0 + j) * cbytes, cbytes, &full[j % S]);
   };
-  const int first = min(kTcStages, a.KT);
-  int issued = 0;  // k-tiles whose copies were issued (tile kt uses stage kt % 3)
-  if (tid == 0) {
-    for (int kt = 0; kt < first; kt++) {
-      mbar_expect_tx(&full[kt], wbytes + cbytes);
-      issue_w(kt, kt);
+  const int first = min(S, nt);
+  const bool producer = warp == kTcProducerWarp && lane == 0;
+  if (producer) {
+    for (int j = 0; j < first; j++) {
+      mbar_expect_tx(&full[j], raw_a + cbytes);
+      issue_w(j);
     }
   }
   pdl_wait();  // the act buffer may be the previous kernel's output
-  if (tid == 0) {
+  if (producer) {
     if (!tc_header_ok(a.act_hdr, a)) {
       words[2] = 1;
       atomicOr(&g_bq_device_error, kErrActHeader);
     }
     // the code copies complete the first stages' transactions even when the header is bad, so
     // that no copy is left in flight; a bad header only stops the MMAs and the outputs
-    for (int kt = 0; kt < first; kt++) issue_c(kt, kt);
-    issued = first;
+    for (int j = 0; j < first; j++) issue_c(j);
+  }
+  for (int m = tid; m < a.M; m += kTcThreads) {
+    const int zx = int(a.act_tok[4 * m + 1]);
+    tok_dx[m] = __uint_as_float(a.act_tok[4 * m]);
+    tok_zx[m] = zx;
+    tok_t[m] = int(a.act_tok[4 * m + 2] - uint32_t(a.K) * uint32_t(zx));
   }
   __syncthreads();
   const bool bad = words[2] != 0;
-  const uint32_t idesc = tc_instr_desc(a.Nmma, kTcRows);
-  const uint32_t ca = smem_u32(smem + kTcOffCanA), cb = smem_u32(smem + kTcOffCanB);
-  int committed = 0;  // tiles whose MMAs were committed (commit kt completes phase kt of mmab)
+  uint32_t* stop = &words[1];
 
-  for (int kt = 0; kt < a.KT; kt++) {
-    const int s = kt % kTcStages;
-    bool ok = mbar_wait_bounded(&full[s], uint32_t((kt / kTcStages) & 1));
-    if (kt >= 1 && ok) ok = mbar_wait_bounded(mmab, uint32_t((kt - 1) & 1));  // operand buffer free
-    if (!ok) words[1] = 1;
-    __syncthreads();
-    if (words[1]) break;
-    {  // re-layout: raw stage s -> the operand buffer
-      const uint8_t* ra = smem + kTcOffRawA + s * kTcRawA;
-      uint8_t* can_a = smem + kTcOffCanA;
-      const int g = lane >> 2, t = lane & 3;
-      const int kc = warp;  // this warp's 32-k chunk of the tile
-      for (int rbl = 0; rbl < nrb; rbl++) {
+  if (producer) {
+    int issued = first;
+    // stage j % S is free again once the MMAs of tile j - S are done (use j / S - 1 of the stage)
+    for (int j = first; j < nt; j++) {
+      if (!tc_wait(&empty[j % S], uint32_t((j / S - 1) & 1), stop)) {
+        *reinterpret_cast<volatile uint32_t*>(stop) = 1u;
+        break;
+      }
+      mbar_expect_tx(&full[j % S], raw_a + cbytes);
+      issue_w(j);
+      issue_c(j);
+      issued = j + 1;
+    }
+    words[4] = uint32_t(issued);
+  } else if (warp == kTcMmaWarp) {
+    if (lane == 0) {
+      const uint32_t idesc = tc_instr_desc(a.Mp, kTcRows);
+      const uint32_t lbo_b = uint32_t(a.Mp) * 16u;
+      int committed = 0;
+      for (int j = 0; j < nt; j++) {
+        const int buf = j & 1;
+        if (!tc_wait(&ready[buf], uint32_t((j >> 1) & 1), stop)) {
+          *reinterpret_cast<volatile uint32_t*>(stop) = 1u;
+          break;
+        }
+        tc_fence_after();
+        if (!bad) {
+          const uint32_t ca = smem_u32(smem + buf * kTcCanA), cb = smem_u32(stage_of(j) + raw_a);
+#pragma unroll
+          for (int i = 0; i < 8; i++)
+            tc_mma(tmem, tc_smem_desc(ca + i * 2 * kTcLboA, kTcLboA, kTcSboA),
+                   tc_smem_desc(cb + i * 2 * lbo_b, lbo_b, kTcSboB), idesc, j > 0 || i > 0);
+        }
+        tc_commit(&empty[j % S]);
+        committed = j + 1;
+      }
+      words[5] = uint32_t(committed);
+    }
+  } else if (warp < kTcLayoutWarps) {
+    const int g = lane >> 2, t = lane & 3;
+    const int kc = warp;  // this warp's 32-k chunk of every tile
+    for (int j = 0; j < nt; j++) {
+      const int buf = j & 1;
+      bool ok = tc_wait(&full[j % S], uint32_t((j / S) & 1), stop);
+      // operand buffer j % 2 is free once the MMAs of tile j - 2 are done (its stage's empty phase;
+      // that stage's next use needs this warp's arrival for a later tile, so the phase cannot alias)
+      if (j >= 2 && ok) ok = tc_wait(&empty[(j - 2) % S], uint32_t(((j - 2) / S) & 1), stop);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) *reinterpret_cast<volatile uint32_t*>(stop) = 1u;
+        break;
+      }
+      const uint8_t* ra = stage_of(j);
+      uint8_t* can_a = smem + buf * kTcCanA;
+#pragma unroll
+      for (int rbl = 0; rbl < kTcRb; rbl++) {
         // word w of a lane holds row g + 8(w & 1) of the block at k = 32kc + 16(w >> 1) + 4t + b;
         // stream s keeps that chunk as field kc % (8/f) of its uint4 kc / (8/f)
         uint32_t w4[4] = {0u, 0u, 0u, 0u};
@@ -218,73 +349,66 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_abq_tc(const __grid_constant_
           *reinterpret_cast<uint32_t*>(can_a + off) = w4[w];
         }
       }
-      const uint8_t* rbraw = smem + kTcOffRawB + s * kTcRawB;
-      uint8_t* can_b = smem + kTcOffCanB;
-      for (int idx = tid; idx < a.M * 16; idx += kTcThreads) {  // (token, 16-byte chunk c)
-        const int n = idx >> 4, c = idx & 15;
-        const uint4 v = *reinterpret_cast<const uint4*>(rbraw + n * 256 + c * 16);
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-        const int tt = c >> 2, cc = c & 3;
-#pragma unroll
-        for (int q = 0; q < 4; q++) {  // byte 64t + 8mu + 4h + b: mu = 2cc + q / 2, h = q % 2
-          const int j = 2 * (2 * cc + (q >> 1)) + (q & 1);
-          const uint32_t off = uint32_t(j) * kTcLboB + uint32_t(n >> 3) * kTcSboB + uint32_t(n & 7) * 16 + uint32_t(tt) * 4;
-          *reinterpret_cast<uint32_t*>(can_b + off) = w4[q];
-        }
-      }
-    }
-    fence_proxy_async();  // the operand writes become visible to the tensor cores
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      if (!bad) {
-#pragma unroll
-        for (int i = 0; i < 8; i++)
-          tc_mma(tmem, tc_smem_desc(ca + i * 2 * kTcLboA, kTcLboA, kTcSboA),
-                 tc_smem_desc(cb + i * 2 * kTcLboB, kTcLboB, kTcSboB), idesc, kt > 0 || i > 0);
-      }
-      tc_commit(mmab);
-      committed = kt + 1;
-      if (kt + kTcStages < a.KT) {  // raw stage s is free again (every thread passed the barrier)
-        fence_proxy_async();
-        mbar_expect_tx(&full[s], wbytes + cbytes);
-        issue_w(kt + kTcStages, s);
-        issue_c(kt + kTcStages, s);
-        issued = kt + kTcStages + 1;
-      }
+      fence_proxy_async();  // the operand writes become visible to the tensor cores
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ready[buf]);
     }
   }
-  // drain: every issued copy landed and the last committed MMA group completed
+  __syncthreads();  // every role has left its loop
+  // drain: the last commit of every stage (commits track all earlier MMAs) and every issued
+  // copy, so that nothing is pending on this block's shared memory or tensor memory when it exits
   if (tid == 0) {
-    if (committed > 0 && !mbar_wait_bounded(mmab, uint32_t((committed - 1) & 1))) words[1] = 1;
-    for (int kt = committed; kt < issued; kt++)
-      (void)mbar_wait_bounded(&full[kt % kTcStages], uint32_t((kt / kTcStages) & 1));
+    const int committed = int(words[5]), issued = int(words[4]);
+    bool ok = true;
+    for (int j = max(0, committed - S); j < committed; j++)
+      ok = mbar_wait_bounded(&empty[j % S], uint32_t((j / S) & 1)) && ok;
+    for (int j = max(0, issued - S); j < issued; j++)
+      ok = mbar_wait_bounded(&full[j % S], uint32_t((j / S) & 1)) && ok;
+    words[3] = (bad || !ok || words[1] != 0 || committed != nt) ? 1u : 0u;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (!bad && !words[1]) {
-    // epilogue: warp w holds rows 32 (w % 4) + lane of the CTA's 128 and tokens 32 (w / 4) ..
-    uint32_t v[32];
-    const int lq = warp & 3, half = warp >> 2;
-    tc_ld32(tmem + (uint32_t(32 * lq) << 16) + uint32_t(32 * half), v);
-    const int row = rb0 * 16 + 32 * lq + lane;
-    if (row < a.N) {
-      const float dw = __ldg(a.row_delta + row);
-      const long long zw = __ldg(a.row_zero + row), sw = __ldg(a.row_sum + row);
+  const bool layout_warp = warp < kTcLayoutWarps;
+  // re-layout warp w holds rows 32 (w % 4) + lane of the CTA's 128 and tokens 32 (w / 4) .. + 31
+  const int lq = warp & 3, half = (warp >> 2) & 1;
+  const int rl = 32 * lq + lane;
+  uint32_t v[32];
+  if (layout_warp) tc_ld32(tmem + (uint32_t(32 * lq) << 16) + uint32_t(32 * half), v);
+  // y = Delta_w Delta_x I with I = P - z_x S_w - z_w (S_x - K z_x); I fits in int32 whenever the
+  // layer's int32 accumulators do, so the wrapping 32-bit arithmetic gives it exactly
+  auto out = [&](int m, uint32_t P) {
+    const int I = int(P - uint32_t(tok_zx[m]) * sw - zw * uint32_t(tok_t[m]));
+    a.y[size_t(m) * a.N + row] = __fmul_rn(dw, tok_dx[m]) * float(I);
+    if (a.acc) a.acc[size_t(m) * a.N + row] = I;
+  };
+  if (CS == 1) {  // rl is tid % 128: this thread's row
+    if (layout_warp && words[3] == 0 && row < a.N) {
 #pragma unroll
-      for (int i = 0; i < 32; i++) {
-        const int m = 32 * half + i;
-        if (m >= a.M) break;
-        const float dx = __uint_as_float(__ldg(a.act_tok + 4 * m));
-        const long long zx = int(__ldg(a.act_tok + 4 * m + 1)), sx = int(__ldg(a.act_tok + 4 * m + 2));
-        // I = P - z_x S_w - z_w S_x + K z_w z_x
-        const long long I = (long long)int(v[i]) - zx * sw - zw * sx + (long long)a.K * zw * zx;
-        a.y[size_t(m) * a.N + row] = __fmul_rn(dw, dx) * float(I);
-        if (a.acc) a.acc[size_t(m) * a.N + row] = I;
+      for (int i = 0; i < 32; i++)
+        if (32 * half + i < a.M) out(32 * half + i, v[i]);
+    }
+  } else {
+    // reduce-scatter over the cluster: every CTA leaves its partial products in its first operand
+    // buffer, [token][128 rows]; CTA r sums tokens m = r, r + CS, ... over all CTAs and writes them
+    uint32_t* part = reinterpret_cast<uint32_t*>(smem);
+    if (layout_warp) {
+#pragma unroll
+      for (int i = 0; i < 32; i++) part[(32 * half + i) * kTcRows + rl] = v[i];
+    }
+    cluster_sync_all();
+    uint32_t failed = 0;
+    for (int c = 0; c < CS; c++) failed |= dsmem_ld(dsmem_map(smem_u32(&words[3]), uint32_t(c)));
+    if (layout_warp && failed == 0 && row < a.N) {
+      const int sub = tid >> 7;  // which of every two of this CTA's tokens
+      for (int m = int(rank) + CS * sub; m < a.M; m += 2 * CS) {
+        uint32_t P = 0;
+        const uint32_t addr = smem_u32(part + m * kTcRows + rl);
+        for (int c = 0; c < CS; c++) P += dsmem_ld(dsmem_map(addr, uint32_t(c)));
+        out(m, P);
       }
     }
+    cluster_sync_all();  // no CTA leaves while another may still read its partial products
   }
   tc_fence_before();
   __syncthreads();

@@ -104,10 +104,14 @@
  * u (ternary): f32 [K_pad/256][M][r] partial dot products of the unquantized bf16 x with A
  *   over each 256-k tile (each in k order); the layer forms SiLU(sum over tiles).
  * xt (RaBiT): f32 [P][M][K_pad] = h_p * x (no activation quantization).
- * ct (ABQ with 16 <= M <= 64 only): the same codes tile-major, byte
- *   (kt*M + m)*256 + 64t + 8mu + 4h + b, so that the tensor-core layer fetches a k-tile of
- *   every token in one copy; bq_gemm on such a layer runs a tcgen05 kind::i8 GEMM (128 rows of
- *   the weights per CTA, the tokens as the MMA's N, accumulators in tensor memory).
+ * ct (ABQ with 16 <= M <= 64 only): the same codes in the K-major operand layout of the
+ *   tensor cores' kind::i8 MMA, for Mp = M rounded up to a multiple of 16 tokens: byte
+ *   kt*Mp*256 + (kk/16)*Mp*16 + (m/8)*128 + (m%8)*16 + kk%16 holds the code of token m at
+ *   k = 256kt + kk; tokens M .. Mp-1 hold code 0. bq_gemm on such a layer runs a tcgen05
+ *   kind::i8 GEMM (128 rows of the weights per CTA, the tokens as the MMA's N, accumulators in
+ *   tensor memory) that reads each k-tile's block with one copy and feeds it to the MMA in
+ *   place; for few row groups a cluster of CTAs splits the k-tiles and sums the partial
+ *   products through distributed shared memory.
  */
 #ifndef BQ_H
 #define BQ_H

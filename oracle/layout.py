@@ -234,7 +234,7 @@ def _bf16_to_f32(u16: np.ndarray) -> np.ndarray:
 # 256-byte header of 32-bit words:
 #   0 magic 0x43415142 'BQAC'   1 version   2 format   3 M   4 K   5 K_pad
 #   6 a_bits   7 lora_rank   8-9 total_bytes   10-11 off_codes   12-13 off_tok
-#   14-15 off_gsum   16-17 off_u   18-19 off_xt
+#   14-15 off_gsum   16-17 off_u   18-19 off_xt   20-21 off_ct (0 when absent)
 # codes (formats 2-5): per token m and k-tile kt, 256 bytes; byte
 #   (m*KT + kt)*256 + 64*t + 8*mu + 4*h + b  holds the code of
 #   k = 32*(8*kt + mu) + 16*h + 4*t + b   (int8 for A8 formats, uint8 for ABQ).
@@ -243,6 +243,8 @@ def _bf16_to_f32(u16: np.ndarray) -> np.ndarray:
 # u (ternary): float32 [KT][M][lora_rank] partial dot products of x and A over each
 #   256-k tile; the layer's LoRA input is SiLU(sum over tiles)
 # xt (RaBiT): float32 [2][M][K_pad] = h_p * x
+# ct (ABQ, 16 <= M <= 64): uint8 [KT][16 k-units][Mp/8][8 tokens][16 bytes], Mp = M rounded
+#   up to 16, the codes of k = 256*kt + 16*unit + byte; tokens M .. Mp-1 hold 0
 
 
 def read_act(buf: bytes) -> dict:
@@ -273,12 +275,13 @@ def read_act(buf: bytes) -> dict:
         codes[:, 256 * kt + kin.ravel()] = raw[:, kt].reshape(M, -1)
     a["codes"] = codes[:, :K]
     a["codes_pad"] = codes[:, K:]
-    if a["off_ct"]:  # the tile-major copy [KT][M][256] (ABQ with 16..64 tokens)
-        rt = np.frombuffer(buf, dtype=dt, count=KT * M * 256, offset=a["off_ct"]).reshape(KT, M, 4, 8, 2, 4)
-        ct = np.zeros((M, K_pad), dtype=dt)
-        for kt in range(KT):
-            ct[:, 256 * kt + kin.ravel()] = rt[kt].reshape(M, -1)
-        a["codes_t"] = ct[:, :K]
+    if a["off_ct"]:  # the tensor-core copy (ABQ with 16..64 tokens)
+        Mp = (M + 15) // 16 * 16
+        rt = np.frombuffer(buf, dtype=dt, count=KT * Mp * 256, offset=a["off_ct"]).reshape(KT, 16, Mp // 8, 8, 16)
+        ct = rt.transpose(2, 3, 0, 1, 4).reshape(Mp, KT * 256)   # [n//8, n%8, kt, unit, byte]
+        a["codes_t"] = ct[:M, :K].copy()
+        a["codes_t_pad"] = ct[:M, K:].copy()
+        a["codes_t_pad_tokens"] = ct[M:].copy()
     tok = np.frombuffer(buf, dtype="<u4", count=4 * M, offset=a["off_tok"]).reshape(M, 4)
     a["scale"] = tok[:, 0].view("<f4").copy()
     a["zero"] = tok[:, 1].view("<i4").copy()

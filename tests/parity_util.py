@@ -203,8 +203,9 @@ def check_act(gl: GpuLayer):
     if gl.fmt == "abq":
         Qx, dx, zx = O.quantize_rows_asym(x, gl.a_bits)
         assert np.array_equal(a["codes"].astype(np.int32), Qx)
-        if 16 <= gl.M <= 64:   # the tile-major copy the tensor-core layer reads
+        if 16 <= gl.M <= 64:   # the copy in the operand layout the tensor-core layer reads
             assert np.array_equal(a["codes_t"].astype(np.int32), Qx)
+            assert not a["codes_t_pad"].any() and not a["codes_t_pad_tokens"].any()
         else:
             assert "codes_t" not in a
         assert np.array_equal(a["scale"], dx) and np.array_equal(a["zero"], zx)
