@@ -169,6 +169,10 @@ class ClockSampler:
     def window(self, name: str, t0: float, t1: float):
         self.windows[name] = (t0, t1)
 
+    def stats(self, t0: float, t1: float) -> dict:
+        """The samples that arrived in [t0, t1 + 0.15 s] so far, parsed."""
+        return self.parse("".join(l for t, l in list(self.lines) if t0 <= t <= t1 + 0.15))
+
     def stop(self) -> dict:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
@@ -593,6 +597,10 @@ def run_configs(args) -> None:
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)   # twice the L2 size
+    # clocks: one sampler for the whole run; every config's timed replays last >= 0.3 s so that
+    # its window holds samples (100 ms period)
+    clocks = ClockSampler(0)
+    clocks.wait_first()
     sel = config_list()
     if args.only:
         sel = [c for c in sel if c[0] == args.only]
@@ -615,17 +623,23 @@ def run_configs(args) -> None:
             with torch.cuda.graph(gi, stream=stream):
                 for L, t in zip(Ls, tim):
                     layer_call(L, t, fused=fused)
+            th0 = time.time()
             for _ in range(3):
                 g.replay()
             torch.cuda.synchronize()
+            per_replay = (time.time() - th0) / 3
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            reps = max(3, int(2000 / R))
+            reps = max(3, int(2000 / R), int(0.3 / max(per_replay, 1e-6)) + 1)
+            tw0 = time.time()
             e0.record(stream)
             for _ in range(reps):
                 g.replay()
             e1.record(stream)
             torch.cuda.synchronize()
+            tw1 = time.time()
             us_layer = e0.elapsed_time(e1) * 1e3 / (reps * R)
+            time.sleep(0.15)
+            clk = clocks.stats(tw0, tw1)
             gl = []
             for _ in range(5):
                 gi.replay()
@@ -650,10 +664,14 @@ def run_configs(args) -> None:
                     us_gemv=us_gemv, gemv_gbs=lb["gemv"] / (us_gemv * 1e-6) / 1e9,
                     gemv_frac=lb["gemv"] / (us_gemv * 1e-6) / 1e9 / peak, us_cold_single=us_cold,
                     bytes=nb, peak=peak,
-                    peak_source=peak_kind)
+                    peak_source=peak_kind, timed_replays=reps, timed_s=round(tw1 - tw0, 3),
+                    clocks={"sm_mhz": clk.get("sm_mhz"), "sm_max_mhz": clk.get("sm_max_mhz"),
+                            "reasons": clk.get("reasons", []), "samples": clk.get("samples", 0),
+                            "power_w_max": clk.get("power_w_max")})
         print(json.dumps(line), flush=True)
         del Ls, g, gi
         torch.cuda.empty_cache()
+    clocks.stop()
 
 
 def run_layer(args) -> None:

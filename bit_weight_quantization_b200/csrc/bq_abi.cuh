@@ -812,16 +812,20 @@ bq_status bq_quantize_act(const bq_layer* layer, const void* x_bf16, int32_t M, 
     return launch_pdl(k_act_rabit, dim3(blocks_for(L.K_pad, 256), M), dim3(256), 0, s, a) == cudaSuccess
                ? BQ_OK : BQ_ERR_CUDA;
   }
+  // each token's row splits over up to 148 / M blocks of 1024 threads; a row of at most 16 K
+  // elements stays in the block's shared memory after the scale pass (read from x once)
   const int slices_target = std::max(1, std::min(L.KT, (148 + M - 1) / M));
   a.tiles_per_slice = (L.KT + slices_target - 1) / slices_target;
   const int slices = (L.KT + a.tiles_per_slice - 1) / a.tiles_per_slice;
-  const dim3 grid(slices, M);
+  const dim3 grid(slices, M), block(1024);
+  a.x_smem = L.K_pad <= kActRowSmemMax ? 1 : 0;
+  const size_t xs_bytes = a.x_smem ? size_t(L.K_pad) * 2 : 0;
   cudaError_t e;
   switch (L.fmt) {
-    case BQ_FMT_BITNET_W1A8: e = launch_pdl(k_act_quant<BQ_FMT_BITNET_W1A8>, grid, dim3(1024), 0, s, a); break;
-    case BQ_FMT_TERNARY_A8: e = launch_pdl(k_act_quant<BQ_FMT_TERNARY_A8>, grid, dim3(1024), 0, s, a); break;
-    case BQ_FMT_ABQ: e = launch_pdl(k_act_quant<BQ_FMT_ABQ>, grid, dim3(1024), 0, s, a); break;
-    case BQ_FMT_BVSR4: e = launch_pdl(k_act_quant<BQ_FMT_BVSR4>, grid, dim3(1024), 0, s, a); break;
+    case BQ_FMT_BITNET_W1A8: e = launch_pdl(k_act_quant<BQ_FMT_BITNET_W1A8>, grid, block, xs_bytes, s, a); break;
+    case BQ_FMT_TERNARY_A8: e = launch_pdl(k_act_quant<BQ_FMT_TERNARY_A8>, grid, block, xs_bytes, s, a); break;
+    case BQ_FMT_ABQ: e = launch_pdl(k_act_quant<BQ_FMT_ABQ>, grid, block, xs_bytes, s, a); break;
+    case BQ_FMT_BVSR4: e = launch_pdl(k_act_quant<BQ_FMT_BVSR4>, grid, block, xs_bytes, s, a); break;
     default: return BQ_ERR_INVALID_ARG;
   }
   return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;

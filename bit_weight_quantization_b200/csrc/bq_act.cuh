@@ -1,19 +1,23 @@
 // Online activation quantization (one call per layer input).
 //
 // Grid (slices, M): every block re-reduces its token's whole row (max|x| or
-// min/max) from L2, which is cheap next to a cross-block exchange, then codes
-// its own slice of k-tiles into the B-operand fragment order. Block slice 0
-// also writes the per-token parameters, the sums and the LoRA input u.
+// min/max) from L2, which is cheap next to a cross-block exchange, keeping the
+// row in shared memory for the later passes, then codes its own slice of
+// k-tiles into the B-operand fragment order. Block slice 0 also writes the
+// per-token parameters, the sums and the LoRA input u.
 #pragma once
 
 #include "bq_internal.cuh"
 
 namespace bqi {
 
+constexpr int kActRowSmemMax = 16384;  // elements of a row kept in shared memory (32 KB, no opt-in)
+
 struct ActArgs {
   const uint16_t* x;        // bf16 [M][K]
   uint8_t* act;             // act buffer base
   int M, K, K_pad, KT, a_bits, rank, fmt, tiles_per_slice;
+  int x_smem;               // the row is kept in dynamic shared memory (K_pad * 2 bytes)
   uint64_t off_codes, off_tok, off_gsum, off_u, off_xt, off_ct, total;
   const uint16_t* lora_A;   // ternary: bf16 [K_pad][r]
   const float* h;           // RaBiT: h_p at h + p K_pad, p < rabit_paths(fmt)
@@ -65,6 +69,32 @@ __device__ __forceinline__ void load4(const uint16_t* xr, int k, int K, float v[
   }
 }
 
+// four bf16 of the row at k from the block's shared copy (filled by the scale pass) or from x
+__device__ __forceinline__ void load4_row(const uint16_t* xr, const uint2* xs, int k, int K, float v[4]) {
+  if (xs && k + 3 < K) {
+    const uint2 p = xs[k >> 2];
+    v[0] = __uint_as_float(p.x << 16);
+    v[1] = __uint_as_float(p.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(p.y << 16);
+    v[3] = __uint_as_float(p.y & 0xFFFF0000u);
+  } else {
+    load4(xr, k, K, v);
+  }
+}
+// the scale pass: four bf16 from x, also kept in the block's shared copy
+__device__ __forceinline__ void load4_keep(const uint16_t* xr, uint2* xs, int k, int K, float v[4]) {
+  if (k + 3 < K) {
+    const uint2 p = *reinterpret_cast<const uint2*>(xr + k);
+    if (xs) xs[k >> 2] = p;
+    v[0] = __uint_as_float(p.x << 16);
+    v[1] = __uint_as_float(p.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(p.y << 16);
+    v[3] = __uint_as_float(p.y & 0xFFFF0000u);
+  } else {
+    load4(xr, k, K, v);
+  }
+}
+
 // absmax int8: gamma = max|x|, s = 127/gamma, q = clamp(rn(x*s), -127, 127); gamma = 0 -> q = 0
 __device__ __forceinline__ int q_a8(float x, float s) {
   float q = rintf(__fmul_rn(x, s));
@@ -79,12 +109,15 @@ __device__ __forceinline__ int q_asym(float x, float d, int z, int qmax) {
   return int(q);
 }
 
-// 1024 threads a block: slice 0 also codes the whole row for the token's code sum, which for
-// ABQ is a correctly rounded divide per element on that block's critical path.
+// Up to 1024 threads a block. A block that codes its token's whole row (one slice) takes the
+// code sum from that pass; otherwise slice 0 codes the row once more for it (for ABQ a
+// correctly rounded divide per element on that block's critical path).
 template <int FMT>
 __global__ void __launch_bounds__(1024) k_act_quant(ActArgs a) {
-  __shared__ float shf[32];
+  __shared__ float shf[32], shf2[32];
   __shared__ int shi[32];
+  extern __shared__ uint2 act_xs[];  // the token's row (when a.x_smem): one global read of it
+  uint2* xs = a.x_smem ? act_xs : nullptr;
   const int m = blockIdx.y, slice = blockIdx.x;
   const uint16_t* xr = a.x + size_t(m) * a.K;
   pdl_trigger();
@@ -99,18 +132,28 @@ __global__ void __launch_bounds__(1024) k_act_quant(ActArgs a) {
     float lo = INFINITY, hi = -INFINITY;
     for (int k = threadIdx.x * 4; k < a.K; k += blockDim.x * 4) {
       float v[4];
-      load4(xr, k, a.K, v);
+      load4_keep(xr, xs, k, a.K, v);
       for (int b = 0; b < 4; b++) if (k + b < a.K) { lo = fminf(lo, v[b]); hi = fmaxf(hi, v[b]); }
     }
-    lo = block_min(lo, shf);
-    hi = block_max(hi, shf);
+    // one block-wide reduction for both: max of (-lo, hi)
+    {
+      float nlo = warp_max(-lo), whi = warp_max(hi);
+      const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+      __syncthreads();
+      if (lane == 0) { shf[w] = nlo; shf2[w] = whi; }
+      __syncthreads();
+      nlo = lane < nw ? shf[lane] : -INFINITY;
+      whi = lane < nw ? shf2[lane] : -INFINITY;
+      lo = -warp_max(nlo);
+      hi = warp_max(whi);
+    }
     delta = __fdiv_rn(fmaxf(__fsub_rn(hi, lo), 1e-5f), float(qmax));
     zero = int(rintf(__fdiv_rn(-lo, delta)));
   } else {
     float mx = 0.f;
     for (int k = threadIdx.x * 4; k < a.K; k += blockDim.x * 4) {
       float v[4];
-      load4(xr, k, a.K, v);
+      load4_keep(xr, xs, k, a.K, v);
       for (int b = 0; b < 4; b++) mx = fmaxf(mx, fabsf(v[b]));
     }
     mx = block_max(mx, shf);
@@ -123,10 +166,12 @@ __global__ void __launch_bounds__(1024) k_act_quant(ActArgs a) {
   int* gsum = reinterpret_cast<int*>(a.act + a.off_gsum) + size_t(m) * (a.K_pad / 32);
   const int kt0 = slice * a.tiles_per_slice;
   const int kt1 = min(a.KT, kt0 + a.tiles_per_slice);
+  const bool whole_row = kt0 == 0 && kt1 == a.KT;  // this block codes the whole row
+  int row_sum = 0;                                 // this thread's share of the code sum
   for (int q4 = kt0 * 64 + threadIdx.x; q4 < kt1 * 64; q4 += blockDim.x) {
     const int k = q4 * 4;
     float v[4];
-    load4(xr, k, a.K, v);
+    load4_row(xr, xs, k, a.K, v);
     uint32_t word = 0;
     int qs = 0;
     for (int b = 0; b < 4; b++) {
@@ -135,6 +180,7 @@ __global__ void __launch_bounds__(1024) k_act_quant(ActArgs a) {
       qs += q;
       word |= (uint32_t(q) & 0xFFu) << (8 * b);
     }
+    row_sum += qs;
     const int kt = k >> 8;
     codes[kt * 64 + code_word_in_tile(k & 255)] = word;
     if (a.off_ct) {  // the tensor-core copy: [KT][16 k-units][Mp / 8][8 tokens][16 bytes]
@@ -168,13 +214,17 @@ __global__ void __launch_bounds__(1024) k_act_quant(ActArgs a) {
   }
 
   if (slice != 0) return;
-  // --- per-token parameters: sum of codes over the whole row ---
-  int s = 0;
-  for (int k = threadIdx.x * 4; k < a.K; k += blockDim.x * 4) {
-    float v[4];
-    load4(xr, k, a.K, v);
-    for (int b = 0; b < 4; b++)
-      if (k + b < a.K) s += FMT == BQ_FMT_ABQ ? q_asym(v[b], delta, zero, qmax) : q_a8(v[b], delta);
+  // --- per-token parameters: sum of codes over the whole row (the codes pass already summed
+  //     them when this block coded the whole row; padding k hold code 0) ---
+  int s = row_sum;
+  if (!whole_row) {
+    s = 0;
+    for (int k = threadIdx.x * 4; k < a.K; k += blockDim.x * 4) {
+      float v[4];
+      load4_row(xr, xs, k, a.K, v);
+      for (int b = 0; b < 4; b++)
+        if (k + b < a.K) s += FMT == BQ_FMT_ABQ ? q_asym(v[b], delta, zero, qmax) : q_a8(v[b], delta);
+    }
   }
   s = block_sum(s, shi);
   uint32_t* tok = reinterpret_cast<uint32_t*>(a.act + a.off_tok) + 4 * m;

@@ -78,3 +78,19 @@ def test_clock_record_prefers_the_timed_window():
     assert r["reasons"] == ["sw_power_cap"] and r["sm_max_mhz"] == 1965.0
     r = bench.clock_record(dict(whole, timed={"samples": 0}, soak=soak))
     assert (r["sm_mhz"], r["window"]) == (1950.0, "soak + timed")
+
+
+def test_clock_stats_take_only_the_window():
+    """A config line's clocks are the samples that arrived during its timed replays (plus one
+    period after), parsed like the bench line's."""
+    c = bench.ClockSampler.__new__(bench.ClockSampler)
+    row = "2026/01/01 00:00:00.000, {mhz}, 1965, {w}, 0x0, Not Active, Not Active, Not Active, {cap}\n"
+    c.lines = [(10.0, row.format(mhz=1965, w=300, cap="Not Active")),
+               (20.1, row.format(mhz=1800, w=990, cap="Active")),
+               (20.2, row.format(mhz=1820, w=995, cap="Active")),
+               (20.5, row.format(mhz=1900, w=700, cap="Not Active")),
+               (30.0, row.format(mhz=1965, w=300, cap="Not Active"))]
+    s = c.stats(20.0, 20.4)
+    assert s["samples"] == 3 and s["sm_mhz"] == 1820.0 and s["reasons"] == ["sw_power_cap"]
+    assert s["power_w_max"] == 995.0
+    assert c.stats(40.0, 41.0)["samples"] == 0
