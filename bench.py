@@ -265,6 +265,15 @@ def cpu_baseline_record(all_cores: dict, one_core: dict) -> dict:
                          "best_us": one_core["best_us"]}}
 
 
+def workload_name(layers: int, no_group: bool) -> str:
+    """The bench workload's name, shared by the CUDA arm and the reference arm."""
+    return (f"BitNet W1A8 decode GEMV, M=1: {layers}-layer Llama-7B linear stack "
+            "(q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008), "
+            + ("q,k,v and gate,up each one bq_linear_group call on their shared input, "
+               "o and down one bq_linear call each" if not no_group else "one bq_linear call per projection")
+            + " (act quantization fused into the layer kernel), PDL between launches, CUDA graph per step")
+
+
 def run_reference(args) -> None:
     """The reference arm: the C++ oracle on the host cores, one BitNet W1A8 4096x4096 layer call
     (act quantization + layer) per step, on all cores; a one-core sample beside it."""
@@ -285,8 +294,10 @@ def run_reference(args) -> None:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64+f64",
         "data": "synthetic",
-        "config": {"workload": "BitNet W1A8 decode GEMV, Llama-7B shapes, M=1 (C++ CPU oracle sample: one "
-                               "4096x4096 layer call per step)", "seq_len": 1, "global_batch": 1},
+        "config": {"workload": workload_name(args.layers, args.no_group), "seq_len": 1, "global_batch": 1,
+                   "parallelism": "single",
+                   "sample": "each step one bounded sample of the workload: a BitNet W1A8 4096x4096 layer "
+                             "call (act quantization + layer) of the C++ oracle; GB/s over its algorithmic bytes"},
         "us_per_layer": el / calls * 1e6,
         "cpu_baseline": {"value": val, "unit": "GB/s", "cores": cores, "kind": "oracle (C++)", "cpu": res[0]["cpu"],
                          "nproc": res[0]["nproc"],
@@ -486,13 +497,7 @@ def run_cuda(args) -> None:
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-            "config": {"workload": "BitNet W1A8 decode GEMV, M=1: 32-layer Llama-7B linear stack "
-                                   "(q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008), "
-                                   + ("q,k,v and gate,up each one bq_linear_group call on their shared input, "
-                                      "o and down one bq_linear call each"
-                                      if not args.no_group else "one bq_linear call per projection") +
-                                   " (act quantization fused into the layer kernel), PDL between launches, "
-                                   "CUDA graph per step",
+            "config": {"workload": workload_name(args.layers, args.no_group),
                        "layers_per_step": n_layers, "launches_per_step": n_calls, "seq_len": 1,
                        "timing": "median of %d back-to-back timed regions of %d steps each (CUDA events; "
                                  "region ms min %.3f, median %.3f, max %.3f); %.1f s untimed soak before the "
