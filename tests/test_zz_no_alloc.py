@@ -15,11 +15,14 @@ def _layer(fmt, N, K, rank=32, seed=0):
     kw = {}
     if fmt == "ternary":
         kw.update(lora_rank=rank, lora_alpha=0.1, lora_A=to_dev_f32(inp["lora_A"]), lora_B=to_dev_f32(inp["lora_B"]))
+    if fmt == "abq":  # W8A8; the scratch holds the act buffer (with its tensor-core section at 16..64 tokens)
+        kw.update(w_bits=8, a_bits=8)
     return bq.QuantLinear(fmt, to_dev_f32(inp["W"]), **kw)
 
 
 @pytest.mark.parametrize("fmt,N,K,M,rank", [("ternary", 2048, 2048, 4, 32), ("ternary", 300, 1280, 16, 64),
-                                            ("bitnet", 4096, 4096, 1, 0)])
+                                            ("bitnet", 4096, 4096, 1, 0), ("abq", 300, 4096, 8, 0),
+                                            ("abq", 4096, 4096, 64, 0), ("abq", 200, 1280, 17, 0)])
 def test_static_scratch_matches_workspace_call(fmt, N, K, M, rank):
     torch, bq = torch_mods()
     ql = _layer(fmt, N, K, rank)
