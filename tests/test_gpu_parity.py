@@ -513,14 +513,16 @@ def test_bvsr_cluster_pack_and_layer(N, K, M, rounds):
                                        (1000, 2048, 32, 8, 8), (97, 640, 16, 1, 8), (200, 384, 24, 2, 8),
                                        (50, 1280, 64, 3, 5), (130, 640, 40, 4, 4), (97, 256, 64, 5, 2),
                                        (300, 2048, 33, 6, 6), (64, 640, 17, 7, 7),
-                                       (640, 2816, 64, 2, 8), (2560, 1792, 40, 4, 4)])
+                                       (640, 2816, 64, 2, 8), (2560, 1792, 40, 4, 4),
+                                       (64, 256, 16, 4, 4), (130, 20480, 20, 8, 8), (48, 16384, 32, 3, 6)])
 def test_abq_tensor_cores(N, K, M, w, a):
     """ABQ with 16..64 tokens runs as a tcgen05 kind::i8 GEMM (the weight code bytes assembled
     from their bit-field streams while the operands are re-laid into canonical shared-memory
     layouts, accumulators in tensor memory), for every weight width 1..8: ragged row counts (a
     partial 128-row CTA), token counts rounded up to the MMA's N, several activation widths,
     k-tiles split over clusters of 1..8 CTAs (evenly and raggedly) whose partial products
-    meet in distributed shared memory.
+    meet in distributed shared memory, one k-tile, and rows at and past the 16 K elements the
+    act kernel keeps in shared memory.
     act + gemm and the fused call both take it and agree bit for bit (GpuLayer); the integer
     accumulators equal the oracle's, y within tolerance."""
     gl = GpuLayer("abq", N, K, M, seed=N + M + a, w_bits=w, a_bits=a)
