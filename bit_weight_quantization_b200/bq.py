@@ -273,3 +273,30 @@ class QuantLinear:
         else:
             bq_gemm(self.layer, act, M, y, acc_dbg, stream)
         return y
+
+
+class StepGraph:
+    """A fixed sequence of this library's calls, captured once into a CUDA graph and replayed.
+
+    This is how a decode loop avoids paying the host cost of every call on every step: the
+    calls in ``issue()`` (which enqueue on torch's current stream, the default of every call
+    here) are captured on ``stream`` after ``warmup`` eager runs. The buffers they read and
+    write are fixed in the graph, so a step refreshes their contents (e.g. one copy into the
+    input buffer), calls ``replay()``, and reads the outputs. ``replay()`` enqueues the whole
+    step on torch's current stream. The library allocates nothing and never synchronizes in
+    its compute calls, which is what makes them capturable."""
+
+    def __init__(self, issue, stream=None, warmup: int = 1):
+        import torch
+        s = stream if stream is not None else torch.cuda.Stream()
+        with torch.cuda.stream(s):
+            for _ in range(warmup):
+                issue()
+        s.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=s):
+            issue()
+        s.synchronize()
+
+    def replay(self) -> None:
+        self.graph.replay()
