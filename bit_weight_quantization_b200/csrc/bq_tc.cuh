@@ -174,6 +174,59 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, const ui
   return false;
 }
 
+// The token parameters and this thread's row parameters of the epilogue.
+struct TcTok {
+  const float* dx;  // Delta_x per token (shared)
+  const int* zx;    // z_x
+  const int* t;     // S_x - K z_x (mod 2^32)
+  float dw;
+  uint32_t zw, sw;
+};
+
+// y (and the integer accumulators when asked) of tokens m0, m0 + step, ... (< M) of one row,
+// from registers.
+template <int T>
+__device__ __forceinline__ void tc_store_outputs(const TcArgs& a, int row, int m0, int step, const float (&yv)[T],
+                                                 const uint32_t (&iv)[T]) {
+#pragma unroll
+  for (int j = 0; j < T; j++) {
+    const int m = m0 + step * j;
+    if (m < a.M) {
+      a.y[size_t(m) * a.N + row] = yv[j];
+      if (a.acc) a.acc[size_t(m) * a.N + row] = (long long)int(iv[j]);
+    }
+  }
+}
+
+// Tokens m = r0, r0 + 2 CSV, ... (< M) of row rl: the cluster's CSV partial products summed in
+// CTA order, every remote load issued before the first sum (so their latencies overlap), then
+// y = Delta_w Delta_x I with I = P - z_x S_w - z_w (S_x - K z_x) in wrapping int32, then stored.
+template <int CSV>
+__device__ __forceinline__ void tc_cluster_out(const TcArgs& a, const uint32_t* part, int rl, int row, int r0,
+                                               const TcTok& tk) {
+  constexpr int T = (kTcMaxN + 2 * CSV - 1) / (2 * CSV);  // tokens one thread can hold
+  uint32_t L[T][CSV];
+#pragma unroll
+  for (int j = 0; j < T; j++) {
+    const int m = r0 + 2 * CSV * j;
+    const uint32_t addr = smem_u32(part + min(m, kTcMaxN - 1) * kTcRows + rl);
+#pragma unroll
+    for (int c = 0; c < CSV; c++) L[j][c] = m < a.M ? dsmem_ld(dsmem_map(addr, uint32_t(c))) : 0u;
+  }
+  float yv[T];
+  uint32_t iv[T];
+#pragma unroll
+  for (int j = 0; j < T; j++) {
+    const int m = min(r0 + 2 * CSV * j, kTcMaxN - 1);  // tokens past M are computed and not stored
+    uint32_t P = 0;
+#pragma unroll
+    for (int c = 0; c < CSV; c++) P += L[j][c];
+    iv[j] = uint32_t(int(P - uint32_t(tk.zx[m]) * tk.sw - tk.zw * uint32_t(tk.t[m])));
+    yv[j] = __fmul_rn(tk.dw, tk.dx[m]) * float(int(iv[j]));
+  }
+  tc_store_outputs<T>(a, row, r0, 2 * CSV, yv, iv);
+}
+
 // Field f (bits) of 32-k chunk kc for the four words of this lane's 16 bytes of a stream of width F:
 // the chunk is field kc % (8/F) of uint4 kc / (8/F); the field values land at bit offset SH.
 template <int F, int SH>
@@ -377,16 +430,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_abq_tc(const __grid_constant_
   if (layout_warp) tc_ld32(tmem + (uint32_t(32 * lq) << 16) + uint32_t(32 * half), v);
   // y = Delta_w Delta_x I with I = P - z_x S_w - z_w (S_x - K z_x); I fits in int32 whenever the
   // layer's int32 accumulators do, so the wrapping 32-bit arithmetic gives it exactly
-  auto out = [&](int m, uint32_t P) {
-    const int I = int(P - uint32_t(tok_zx[m]) * sw - zw * uint32_t(tok_t[m]));
-    a.y[size_t(m) * a.N + row] = __fmul_rn(dw, tok_dx[m]) * float(I);
-    if (a.acc) a.acc[size_t(m) * a.N + row] = I;
-  };
   if (CS == 1) {  // rl is tid % 128: this thread's row
     if (layout_warp && words[3] == 0 && row < a.N) {
+      // every output first, then every store: a store between them would keep the compiler from
+      // issuing the next token's shared loads early (it cannot tell the two pointers apart)
+      float yv[32];
 #pragma unroll
-      for (int i = 0; i < 32; i++)
-        if (32 * half + i < a.M) out(32 * half + i, v[i]);
+      for (int i = 0; i < 32; i++) {
+        const int m = 32 * half + i;  // < kTcMaxN; tokens past M are computed and not stored
+        v[i] = uint32_t(int(v[i] - uint32_t(tok_zx[m]) * sw - zw * uint32_t(tok_t[m])));
+        yv[i] = __fmul_rn(dw, tok_dx[m]) * float(int(v[i]));
+      }
+      tc_store_outputs<32>(a, row, 32 * half, 1, yv, v);
     }
   } else {
     // reduce-scatter over the cluster: every CTA leaves its partial products in its first operand
@@ -400,12 +455,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_abq_tc(const __grid_constant_
     uint32_t failed = 0;
     for (int c = 0; c < CS; c++) failed |= dsmem_ld(dsmem_map(smem_u32(&words[3]), uint32_t(c)));
     if (layout_warp && failed == 0 && row < a.N) {
-      const int sub = tid >> 7;  // which of every two of this CTA's tokens
-      for (int m = int(rank) + CS * sub; m < a.M; m += 2 * CS) {
-        uint32_t P = 0;
-        const uint32_t addr = smem_u32(part + m * kTcRows + rl);
-        for (int c = 0; c < CS; c++) P += dsmem_ld(dsmem_map(addr, uint32_t(c)));
-        out(m, P);
+      const TcTok tk{tok_dx, tok_zx, tok_t, dw, zw, sw};
+      const int r0 = int(rank) + CS * (tid >> 7);  // the first of this thread's tokens
+      switch (CS) {
+        case 2: tc_cluster_out<2>(a, part, rl, row, r0, tk); break;
+        case 3: tc_cluster_out<3>(a, part, rl, row, r0, tk); break;
+        case 4: tc_cluster_out<4>(a, part, rl, row, r0, tk); break;
+        case 5: tc_cluster_out<5>(a, part, rl, row, r0, tk); break;
+        case 6: tc_cluster_out<6>(a, part, rl, row, r0, tk); break;
+        case 7: tc_cluster_out<7>(a, part, rl, row, r0, tk); break;
+        default: tc_cluster_out<8>(a, part, rl, row, r0, tk); break;
       }
     }
     cluster_sync_all();  // no CTA leaves while another may still read its partial products

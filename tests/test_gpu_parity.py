@@ -514,7 +514,8 @@ def test_bvsr_cluster_pack_and_layer(N, K, M, rounds):
                                        (50, 1280, 64, 3, 5), (130, 640, 40, 4, 4), (97, 256, 64, 5, 2),
                                        (300, 2048, 33, 6, 6), (64, 640, 17, 7, 7),
                                        (640, 2816, 64, 2, 8), (2560, 1792, 40, 4, 4),
-                                       (64, 256, 16, 4, 4), (130, 20480, 20, 8, 8), (48, 16384, 32, 3, 6)])
+                                       (64, 256, 16, 4, 4), (130, 20480, 20, 8, 8), (48, 16384, 32, 3, 6),
+                                       (100, 1536, 24, 5, 5), (60, 1792, 48, 6, 4)])
 def test_abq_tensor_cores(N, K, M, w, a):
     """ABQ with 16..64 tokens runs as a tcgen05 kind::i8 GEMM (the weight code bytes assembled
     from their bit-field streams while the operands are re-laid into canonical shared-memory
