@@ -540,3 +540,19 @@ def test_bvsr_cluster_rounds_are_checked():
         st = bq.raw_status("bq_packed_bytes", ctypes.byref(d), 64, 256, ctypes.byref(ctypes.c_size_t()))
         assert (st == bq.BQ_OK) == ok, (fmt, r, st)
     assert layer is not None and fake
+
+
+@pytest.mark.parametrize("M", [2, 15, 16, 17, 33, 64])
+def test_abq_act_bytes_and_workspace_follow_the_documented_sections(M):
+    """The ABQ act buffer per include/bq.h: header 256, codes M x KT x 256, token words M x 16
+    (padded to 256), and for 16 <= M <= 64 the tensor-core copy Mp x KT x 256 (Mp = M rounded up
+    to 16); bq_linear's workspace for M >= 2 is that act buffer."""
+    h = _host_header("abq", 300, 1280, w_bits=8, a_bits=8)
+    layer = bq.bq_packed_validate(h.tobytes(), 1 << 30)
+    KT = 1280 // 256
+    up = lambda n: (n + 255) // 256 * 256
+    want = 256 + up(M * KT * 256) + up(M * 16)
+    if 16 <= M <= 64:
+        want += up(((M + 15) // 16 * 16) * KT * 256)
+    assert bq.bq_act_bytes(layer, M) == want
+    assert bq.bq_linear_workspace_bytes(layer, M) == want
