@@ -160,6 +160,11 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
 
+// lowers the barrier's pending transaction count by bytes that will never be copied
+__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -315,28 +320,33 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_abq_tc(const __grid_constant_
   }
   pdl_wait();  // the act buffer may be the previous kernel's output
   if (producer) {
+    // nothing past the header is read unless it matches this layer (every section then lies
+    // inside the buffer); a bad header completes the first stages' transactions without the
+    // codes, and every role skips its loop
     if (!tc_header_ok(a.act_hdr, a)) {
       words[2] = 1;
       atomicOr(&g_bq_device_error, kErrActHeader);
+      for (int j = 0; j < first; j++) mbar_complete_tx(&full[j], cbytes);
+    } else {
+      for (int j = 0; j < first; j++) issue_c(j);
     }
-    // the code copies complete the first stages' transactions even when the header is bad, so
-    // that no copy is left in flight; a bad header only stops the MMAs and the outputs
-    for (int j = 0; j < first; j++) issue_c(j);
-  }
-  for (int m = tid; m < a.M; m += kTcThreads) {
-    const int zx = int(a.act_tok[4 * m + 1]);
-    tok_dx[m] = __uint_as_float(a.act_tok[4 * m]);
-    tok_zx[m] = zx;
-    tok_t[m] = int(a.act_tok[4 * m + 2] - uint32_t(a.K) * uint32_t(zx));
   }
   __syncthreads();
   const bool bad = words[2] != 0;
+  if (!bad) {
+    for (int m = tid; m < a.M; m += kTcThreads) {
+      const int zx = int(a.act_tok[4 * m + 1]);
+      tok_dx[m] = __uint_as_float(a.act_tok[4 * m]);
+      tok_zx[m] = zx;
+      tok_t[m] = int(a.act_tok[4 * m + 2] - uint32_t(a.K) * uint32_t(zx));
+    }
+  }
   uint32_t* stop = &words[1];
 
   if (producer) {
     int issued = first;
     // stage j % S is free again once the MMAs of tile j - S are done (use j / S - 1 of the stage)
-    for (int j = first; j < nt; j++) {
+    for (int j = first; j < nt && !bad; j++) {
       if (!tc_wait(&empty[j % S], uint32_t((j / S - 1) & 1), stop)) {
         *reinterpret_cast<volatile uint32_t*>(stop) = 1u;
         break;
@@ -352,20 +362,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_abq_tc(const __grid_constant_
       const uint32_t idesc = tc_instr_desc(a.Mp, kTcRows);
       const uint32_t lbo_b = uint32_t(a.Mp) * 16u;
       int committed = 0;
-      for (int j = 0; j < nt; j++) {
+      for (int j = 0; j < nt && !bad; j++) {
         const int buf = j & 1;
         if (!tc_wait(&ready[buf], uint32_t((j >> 1) & 1), stop)) {
           *reinterpret_cast<volatile uint32_t*>(stop) = 1u;
           break;
         }
         tc_fence_after();
-        if (!bad) {
-          const uint32_t ca = smem_u32(smem + buf * kTcCanA), cb = smem_u32(stage_of(j) + raw_a);
+        const uint32_t ca = smem_u32(smem + buf * kTcCanA), cb = smem_u32(stage_of(j) + raw_a);
 #pragma unroll
-          for (int i = 0; i < 8; i++)
-            tc_mma(tmem, tc_smem_desc(ca + i * 2 * kTcLboA, kTcLboA, kTcSboA),
-                   tc_smem_desc(cb + i * 2 * lbo_b, lbo_b, kTcSboB), idesc, j > 0 || i > 0);
-        }
+        for (int i = 0; i < 8; i++)
+          tc_mma(tmem, tc_smem_desc(ca + i * 2 * kTcLboA, kTcLboA, kTcSboA),
+                 tc_smem_desc(cb + i * 2 * lbo_b, lbo_b, kTcSboB), idesc, j > 0 || i > 0);
         tc_commit(&empty[j % S]);
         committed = j + 1;
       }
@@ -374,7 +382,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_abq_tc(const __grid_constant_
   } else if (warp < kTcLayoutWarps) {
     const int g = lane >> 2, t = lane & 3;
     const int kc = warp;  // this warp's 32-k chunk of every tile
-    for (int j = 0; j < nt; j++) {
+    for (int j = 0; j < nt && !bad; j++) {
       const int buf = j & 1;
       bool ok = tc_wait(&full[j % S], uint32_t((j / S) & 1), stop);
       // operand buffer j % 2 is free once the MMAs of tile j - 2 are done (its stage's empty phase;

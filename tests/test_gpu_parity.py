@@ -312,6 +312,27 @@ def test_act_buffer_of_another_layer_config_is_refused(fmt, kw_act, kw_layer):
     bq.bq_device_check()
 
 
+@pytest.mark.parametrize("M_act,a_act", [(17, 8), (20, 4), (64, 8)])
+def test_tensor_core_gemm_refuses_a_mismatched_act_buffer(M_act, a_act):
+    """The tensor-core GEMM (ABQ, 20 tokens) given an act buffer made for fewer or more tokens
+    or another activation width: it reads nothing past the header (no code copy, no token
+    words), writes nothing and raises the device error word; the next good call is exact."""
+    from tests.parity_util import torch_mods
+    torch, bq = torch_mods()
+    src = GpuLayer("abq", 200, 512, M_act, seed=3, w_bits=8, a_bits=a_act)
+    dst = GpuLayer("abq", 200, 512, 20, seed=4, w_bits=8, a_bits=8)
+    y = torch.full((20, 200), 7.0, device="cuda")
+    bq.bq_gemm(dst.ql.layer, src.ql.act_buffer(M_act), 20, y)
+    with pytest.raises(bq.BQError) as e:
+        bq.bq_device_check()
+    assert e.value.status == bq.BQ_ERR_DEVICE_CHECK
+    assert torch.all(y == 7.0)
+    bq.bq_gemm(dst.ql.layer, dst.ql.act_buffer(20), 20, y)
+    torch.cuda.synchronize()
+    bq.bq_device_check()
+    assert np.array_equal(y.cpu().numpy(), dst.y_h)
+
+
 # ------------------------------------------------------------------ grouped layers sharing x
 @pytest.mark.parametrize("fmt,Ns,K,M,wa", [("bitnet", (64, 97, 40), 512, 1, (1, 8)),
                                            ("bitnet", (4096, 4096, 4096), 4096, 1, (1, 8)),
