@@ -184,8 +184,12 @@ __global__ void __launch_bounds__(1024) k_act_quant(ActArgs a) {
     const int kt = k >> 8;
     codes[kt * 64 + code_word_in_tile(k & 255)] = word;
     if (a.off_ct) {  // the tensor-core copy: [KT][16 k-units][Mp / 8][8 tokens][16 bytes]
-      const int Mp = tc_tokens(a.M), kk = k & 255;
-      uint8_t* ct = a.act + a.off_ct + size_t(kt) * Mp * 256 + (kk >> 4) * (Mp * 16) + (kk & 15);
+      // within each 32-k chunk a code sits at the MMA's k position p of the weight operand in
+      // tensor memory: k' = k % 32 at p = 8 ((k' % 16) / 4) + 4 (k' / 16) + k' % 4, i.e. k-unit
+      // 2 (chunk) + p / 16, byte p % 16 (a word of four codes stays together)
+      const int Mp = tc_tokens(a.M), kk = k & 255, kp = kk & 31;
+      const int p = 8 * ((kp & 15) >> 2) + 4 * (kp >> 4) + (kp & 3);
+      uint8_t* ct = a.act + a.off_ct + size_t(kt) * Mp * 256 + (2 * (kk >> 5) + (p >> 4)) * (Mp * 16) + (p & 15);
       *reinterpret_cast<uint32_t*>(ct + (m >> 3) * 128 + (m & 7) * 16) = word;
       if (m < Mp - a.M) {  // token M + m pads the MMA's N to a multiple of 16 (Mp - M < 16 <= M)
         const int mp = a.M + m;

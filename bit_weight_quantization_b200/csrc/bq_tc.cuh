@@ -15,17 +15,21 @@
 // shared memory: per tile one TMA tensor copy of the eight packed weight tiles (bit-field
 // streams in the A-fragment order of the int8 m16n8k32 MMA; rows past the layer read as zero)
 // and one bulk copy of the act buffer's tensor-core block of the tile (already in the
-// canonical operand layout, read by the MMA in place). Eight re-layout warps copy each weight
-// tile into one of two canonical K-major operand buffers (8-row x 16-byte core matrices, no
-// swizzle), assembling each code byte from its streams' fields (code = sum_s field_s << shift_s),
-// and arrive on the buffer's "ready" barrier. The MMA warp issues the tile's eight MMAs (K = 32
-// each) and commits them to the stage's "empty" barrier, on which the producer refills the
-// stage and the re-layout warps reuse the tile's operand buffer two tiles later. After the last tile the re-layout warps read the
+// canonical K-major operand layout, read by the MMA in place). Eight re-layout warps, one per
+// 16-row block, assemble each code byte from its streams' fields (code = sum_s field_s <<
+// shift_s) and store the fragment words straight into one of two weight operand buffers in
+// tensor memory (tcgen05.st 16x256b writes the m16n8 fragment pattern, so the words need no
+// shuffling; the k order this gives within each 32-k chunk is the act copy's order too), then
+// arrive on the buffer's "ready" barrier. The MMA warp issues the tile's eight MMAs (K = 32
+// each, A from tensor memory, B from shared memory) and commits them to the stage's "empty"
+// barrier, on which the producer refills the stage and the re-layout warps reuse the tile's
+// operand buffer two tiles later. After the last tile the re-layout warps read the
 // accumulators from tensor memory (tcgen05.ld, warps w and w + 4 the two column halves of lanes
 // 32w .. 32w + 31) and run the ABQ zero-point epilogue. Every wait is bounded and also ends
 // when another role has stopped: on expiry the device error word is raised, no further MMA is
 // issued, outstanding copies and MMAs are waited for, every CTA of the cluster still takes both
-// cluster barriers, and the tensor memory is freed.
+// cluster barriers, and the tensor memory is freed. An act buffer whose header does not match
+// the layer is not read past its header (no code copy, no token words, no MMA, no output).
 #pragma once
 
 #include "bq_gemv.cuh"
@@ -40,16 +44,18 @@ constexpr int kTcProducerWarp = kTcLayoutWarps, kTcMmaWarp = kTcLayoutWarps + 1;
 constexpr int kTcThreads = (kTcLayoutWarps + 2) * 32;
 constexpr int kTcMaxStages = 8;
 constexpr int kTcMaxCluster = 8;             // portable cluster size
-constexpr int kTcColsAlloc = 64;             // tensor-memory columns (one per token)
-constexpr uint32_t kTcCanA = kTcRows * 256;  // canonical A of one k-tile (32 KB); two buffers
-constexpr uint32_t kTcOffStages = 2 * kTcCanA;
+// tensor memory: the accumulators (one column per token) in columns 0..63, and two A operand
+// buffers of one k-tile each (128 rows x 256 codes, four codes a column) at columns 64 and 128
+constexpr int kTcColsAlloc = 256;
+constexpr uint32_t kTcColA = 64, kTcColsA = 64;
+constexpr uint32_t kTcOffStages = 0;
 // after the stages: full[8] (0), empty[8] (64), ready[2] (144), words[8] (160),
 // and the token parameters Delta_x, z_x, S_x - K z_x [3][64] (256)
 constexpr uint32_t kTcBarBytes = 1024;
 constexpr uint32_t kTcSmemMax = 227 * 1024;
-// canonical strides of A: core matrix rows 16 B apart, 8-row groups 128 B apart, 16-byte
-// k-units 2048 B apart (16 row groups); B: 8-token groups 128 B apart, k-units Mp * 16 B apart
-constexpr uint32_t kTcLboA = 2048, kTcSboA = 128, kTcSboB = 128;
+// canonical strides of B (K-major, no swizzle): 8-token groups 128 B apart, 16-byte k-units
+// Mp * 16 B apart
+constexpr uint32_t kTcSboB = 128;
 
 // The packed weight tiles as a 3-D uint8 tensor for the TMA: x = 256 bytes, y = 256-byte
 // chunks along a row block's tiles (KT tile_bytes / 256), z = row blocks; a box of
@@ -102,19 +108,29 @@ __host__ __device__ constexpr uint32_t tc_instr_desc(int nmma, int mmma) {
   return (2u << 4) | (uint32_t(nmma >> 3) << 17) | (uint32_t(mmma >> 4) << 24);
 }
 
-__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, int accum) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
-      : "memory");
-}
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(smem_u32(bar))
                : "memory");
 }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+
+// 16 lanes x 8 columns into tensor memory in the m16n8 fragment pattern: thread 4g + t writes
+// r0, r1 to lane g, columns 2t and 2t + 1, and r2, r3 to lane g + 8, the same columns
+__device__ __forceinline__ void tc_st16(uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("tcgen05.st.sync.aligned.16x256b.x1.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(taddr), "r"(r0), "r"(r1),
+               "r"(r2), "r"(r3)
+               : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+// the MMA with A from tensor memory (a_tmem) and B from shared memory
+__device__ __forceinline__ void tc_mma_ta(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc, int accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
 
 // 32 lanes x 32 columns of 32 bits from tensor memory (warp w reads lanes 32 (w % 4) .. + 31)
 __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&v)[32]) {
@@ -369,19 +385,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_abq_tc(const __grid_constant_
           break;
         }
         tc_fence_after();
-        const uint32_t ca = smem_u32(smem + buf * kTcCanA), cb = smem_u32(stage_of(j) + raw_a);
+        const uint32_t ta = tmem + kTcColA + uint32_t(buf) * kTcColsA, cb = smem_u32(stage_of(j) + raw_a);
 #pragma unroll
-        for (int i = 0; i < 8; i++)
-          tc_mma(tmem, tc_smem_desc(ca + i * 2 * kTcLboA, kTcLboA, kTcSboA),
-                 tc_smem_desc(cb + i * 2 * lbo_b, lbo_b, kTcSboB), idesc, j > 0 || i > 0);
+        for (int i = 0; i < 8; i++)  // chunk i: A columns 8i .. 8i + 7, B k-units 2i, 2i + 1
+          tc_mma_ta(tmem, ta + 8u * uint32_t(i), tc_smem_desc(cb + i * 2 * lbo_b, lbo_b, kTcSboB), idesc, j > 0 || i > 0);
         tc_commit(&empty[j % S]);
         committed = j + 1;
       }
       words[5] = uint32_t(committed);
     }
   } else if (warp < kTcLayoutWarps) {
-    const int g = lane >> 2, t = lane & 3;
-    const int kc = warp;  // this warp's 32-k chunk of every tile
+    // warp w takes row block b = 2 (w % 4) + w / 4 of every tile: tensor-memory lanes 16b .. 16b + 15,
+    // inside its quarter of the lanes (32 (w % 4) .. + 31)
+    const int rbl = 2 * (warp & 3) + (warp >> 2);
+    const uint32_t lane_base = uint32_t(16 * rbl) << 16;
     for (int j = 0; j < nt && !bad; j++) {
       const int buf = j & 1;
       bool ok = tc_wait(&full[j % S], uint32_t((j / S) & 1), stop);
@@ -392,25 +409,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_abq_tc(const __grid_constant_
         if (lane == 0) *reinterpret_cast<volatile uint32_t*>(stop) = 1u;
         break;
       }
-      const uint8_t* ra = stage_of(j);
-      uint8_t* can_a = smem + buf * kTcCanA;
+      tc_fence_after();
+      const uint8_t* tile = stage_of(j) + rbl * tb;
+      const uint32_t ta = tmem + lane_base + kTcColA + uint32_t(buf) * kTcColsA;
 #pragma unroll
-      for (int rbl = 0; rbl < kTcRb; rbl++) {
-        // word w of a lane holds row g + 8(w & 1) of the block at k = 32kc + 16(w >> 1) + 4t + b;
-        // stream s keeps that chunk as field kc % (8/f) of its uint4 kc / (8/f)
+      for (int kc = 0; kc < 8; kc++) {
+        // word w of lane 4g + t holds row g + 8(w & 1) of the block at k = 32kc + 16(w >> 1) + 4t + b
+        // (stream s keeps that chunk as field kc % (8/f) of its uint4 kc / (8/f)). The store puts
+        // words 0, 2 (row g) and 1, 3 (row g + 8) in columns 8kc + 2t and 8kc + 2t + 1: the MMA's
+        // k position 4c + b of column c holds k = 32kc + 16 (c & 1) + 4 (c >> 1) + b, and the act
+        // buffer's tensor-core copy orders the codes the same way
         uint32_t w4[4] = {0u, 0u, 0u, 0u};
-        const uint8_t* tile = ra + rbl * tb;
         tc_stream_fields<F0, 0>(tile, kc, lane, w4);
         if constexpr (F1 > 0) tc_stream_fields<F1, F0>(tile + 512 * F0, kc, lane, w4);
         if constexpr (F2 > 0) tc_stream_fields<F2, F0 + F1>(tile + 512 * (F0 + F1), kc, lane, w4);
-#pragma unroll
-        for (int w = 0; w < 4; w++) {
-          const uint32_t off = uint32_t(2 * kc + (w >> 1)) * kTcLboA + uint32_t(2 * rbl + (w & 1)) * kTcSboA +
-                               uint32_t(g) * 16 + uint32_t(t) * 4;
-          *reinterpret_cast<uint32_t*>(can_a + off) = w4[w];
-        }
+        tc_st16(ta + 8u * uint32_t(kc), w4[0], w4[2], w4[1], w4[3]);
       }
-      fence_proxy_async();  // the operand writes become visible to the tensor cores
+      tc_wait_st();
+      tc_fence_before();  // the operand writes become visible to the MMA issued after the arrive
       __syncwarp();
       if (lane == 0) mbar_arrive(&ready[buf]);
     }
@@ -452,8 +468,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_abq_tc(const __grid_constant_
       tc_store_outputs<32>(a, row, 32 * half, 1, yv, v);
     }
   } else {
-    // reduce-scatter over the cluster: every CTA leaves its partial products in its first operand
-    // buffer, [token][128 rows]; CTA r sums tokens m = r, r + CS, ... over all CTAs and writes them
+    // reduce-scatter over the cluster: every CTA leaves its partial products at the start of its
+    // (now idle) stage ring, [token][128 rows] (M x 512 bytes, within the ring's >= 3 stages of at
+    // least Mp x 256 bytes each); CTA r sums tokens m = r, r + CS, ... over all CTAs and writes them
     uint32_t* part = reinterpret_cast<uint32_t*>(smem);
     if (layout_warp) {
 #pragma unroll

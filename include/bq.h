@@ -106,12 +106,14 @@
  * xt (RaBiT): f32 [P][M][K_pad] = h_p * x (no activation quantization).
  * ct (ABQ with 16 <= M <= 64 only): the same codes in the K-major operand layout of the
  *   tensor cores' kind::i8 MMA, for Mp = M rounded up to a multiple of 16 tokens: byte
- *   kt*Mp*256 + (kk/16)*Mp*16 + (m/8)*128 + (m%8)*16 + kk%16 holds the code of token m at
- *   k = 256kt + kk; tokens M .. Mp-1 hold code 0. bq_gemm on such a layer runs a tcgen05
- *   kind::i8 GEMM (128 rows of the weights per CTA, the tokens as the MMA's N, accumulators in
- *   tensor memory) that reads each k-tile's block with one copy and feeds it to the MMA in
- *   place; for few row groups a cluster of CTAs splits the k-tiles and sums the partial
- *   products through distributed shared memory.
+ *   kt*Mp*256 + u*Mp*16 + (m/8)*128 + (m%8)*16 + (p%16) with u = 2i + p/16 holds the code of
+ *   token m at k = 256kt + 32i + k', p = 8((k'%16)/4) + 4(k'/16) + k'%4 (within each 32-k
+ *   chunk the order the weight operand takes in tensor memory); tokens M .. Mp-1 hold code 0.
+ *   bq_gemm on such a layer runs a tcgen05 kind::i8 GEMM (128 rows of the weights per CTA in
+ *   tensor memory, the tokens as the MMA's N from shared memory, accumulators in tensor
+ *   memory) that reads each k-tile's block with one copy and feeds it to the MMA in place; for
+ *   few row groups a cluster of CTAs splits the k-tiles and sums the partial products through
+ *   distributed shared memory.
  */
 #ifndef BQ_H
 #define BQ_H

@@ -244,7 +244,8 @@ def _bf16_to_f32(u16: np.ndarray) -> np.ndarray:
 #   256-k tile; the layer's LoRA input is SiLU(sum over tiles)
 # xt (RaBiT): float32 [2][M][K_pad] = h_p * x
 # ct (ABQ, 16 <= M <= 64): uint8 [KT][16 k-units][Mp/8][8 tokens][16 bytes], Mp = M rounded
-#   up to 16, the codes of k = 256*kt + 16*unit + byte; tokens M .. Mp-1 hold 0
+#   up to 16; k-unit 2i + p//16, byte p%16 holds the code of k = 256*kt + 32*i + k' with
+#   p = 8*((k'%16)//4) + 4*(k'//16) + k'%4; tokens M .. Mp-1 hold 0
 
 
 def read_act(buf: bytes) -> dict:
@@ -278,7 +279,13 @@ def read_act(buf: bytes) -> dict:
     if a["off_ct"]:  # the tensor-core copy (ABQ with 16..64 tokens)
         Mp = (M + 15) // 16 * 16
         rt = np.frombuffer(buf, dtype=dt, count=KT * Mp * 256, offset=a["off_ct"]).reshape(KT, 16, Mp // 8, 8, 16)
-        ct = rt.transpose(2, 3, 0, 1, 4).reshape(Mp, KT * 256)   # [n//8, n%8, kt, unit, byte]
+        pos = rt.transpose(2, 3, 0, 1, 4).reshape(Mp, KT, 256)   # [n, kt, 16*unit + byte]
+        u, byte = np.arange(256) // 16, np.arange(256) % 16
+        p = 16 * (u % 2) + byte                                  # position within the 32-k chunk
+        kk = 32 * (u // 2) + 16 * ((p >> 2) & 1) + 4 * (p >> 3) + (p & 3)
+        ct = np.zeros((Mp, KT, 256), dtype=dt)
+        ct[:, :, kk] = pos
+        ct = ct.reshape(Mp, KT * 256)
         a["codes_t"] = ct[:M, :K].copy()
         a["codes_t_pad"] = ct[:M, K:].copy()
         a["codes_t_pad_tokens"] = ct[M:].copy()
