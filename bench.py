@@ -592,6 +592,7 @@ def config_list():
     out += [("abq", N, 4096, M, w, a) for (w, a) in [(2, 8), (4, 4), (6, 6), (8, 8)]
             for N in (4096, 11008) for M in (1, 8, 64)]
     out += [("bvsr", N, K, 1, 4, 8) for N, K in [(5120, 5120), (13824, 5120), (5120, 13824)]]
+    out += [("bvsr", 5120, 5120, M, 4, 8) for M in (4, 16, 64)]  # the multi-token path
     return out
 
 

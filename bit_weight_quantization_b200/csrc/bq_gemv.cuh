@@ -734,21 +734,23 @@ struct BvsrFam {
 // holds two words: the 4-bit codes of A registers a0 (row g) and a1 (row g + 8) in the low and
 // high half of the first, a2 and a3 in the second, nibble b of a half being byte b of the
 // register. With the set's integer template, L(c) = sum_i R_i b_i(c) = L3(c & 7) + R_3 [c >= 8]
-// (at most 203, one u8 byte), and E = sum_k L(code_k) q_k comes exactly from two int8 MMAs:
-// bytes L3(c & 7) (the family table selected by the code with its bit 3 cleared) and bytes
-// R_3 [c >= 8] (R_3 selected with bit 3 flipped, so that codes below 8 copy the sign of
-// R_3 < 128, i.e. 0). Per row and vector the set s gives o and sc = span / sum R (table words
+// (at most 203, one u8 byte), and E = sum_k L(code_k) q_k comes exactly from one int8 MMA on
+// the byte sums of L3(c & 7) (the family table selected by the code with its bit 3 cleared)
+// and R_3 [c >= 8] (R_3 selected with bit 3 flipped, so that codes below 8 copy the sign of
+// R_3 < 128, i.e. 0); no byte of the sum carries, as L(c) < 256. Per row and vector the set s
+// gives o and sc = span / sum R (table words
 // 4, 5): y += sc E + o S_v, S_v the vector's code sum. TWO (warp-uniform): the CTA holds more
 // than one token, so outputs c = 1, 3 (token 2t + 1) are live too; with one token only c = 0, 2.
 // want_acc adds sum_k code_k q_k (a third MMA on the code bytes).
-// The tile is walked as a loop over its four vector pairs (the weight words and the act codes
-// of a pair are one 16-byte load each), so that the loop body stays small in the instruction
-// cache; the tile's set bytes for rows g and g + 8 are i0, i1 (byte j of the pair of words).
+// The tile's four vector pairs (the weight words and the act codes of a pair are one 16-byte
+// load each) are unrolled into one block, so that the loads and MMAs of later pairs overlap the
+// float epilogue of earlier ones; the tile's set bytes for rows g and g + 8 are i0, i1 (byte j
+// of the pair of words).
 __device__ __forceinline__ void bvsr_tile(const uint8_t* tp, const uint8_t* bp, bool has_tok, uint2 i0, uint2 i1,
                                           const float* tab, const BvsrFam* fam, const int* gs_row, int VPR,
                                           bool TWO, bool tok0, bool tok1, bool want_acc, float (&yacc)[4],
                                           long long (&cacc)[4]) {
-#pragma unroll 1
+#pragma unroll
   for (int jp = 0; jp < 4; jp++) {
     const uint4 q = lds128(tp + jp * 512);
     const uint4 bq = has_tok ? lds128(bp + jp * 16) : make_uint4(0, 0, 0, 0);
@@ -762,16 +764,14 @@ __device__ __forceinline__ void bvsr_tile(const uint8_t* tp, const uint8_t* bp, 
       const int s0 = int(__byte_perm(iw0, 0, 0x4440u | uint32_t(j & 3)));
       const int s1 = int(__byte_perm(iw1, 0, 0x4440u | uint32_t(j & 3)));
       const BvsrFam f0 = fam[s0 >> 6], f1 = fam[s1 >> 6];
-      uint32_t a1[4], a2[4];
+      uint32_t a1[4];
 #pragma unroll
       for (int r = 0; r < 4; r++) {
         const BvsrFam& f = (r & 1) ? f1 : f0;
-        a1[r] = prmt(f.lo, f.hi, sel[r] & 0x7777u);
-        a2[r] = prmt(f.r3, f.r3, sel[r] ^ 0x8888u);
+        a1[r] = prmt(f.lo, f.hi, sel[r] & 0x7777u) + prmt(f.r3, f.r3, sel[r] ^ 0x8888u);
       }
-      int d1[4] = {0, 0, 0, 0}, d2[4] = {0, 0, 0, 0};
+      int d1[4] = {0, 0, 0, 0};
       mma_u8<true>(d1, a1[0], a1[1], a1[2], a1[3], b0, b1);
-      mma_u8<true>(d2, a2[0], a2[1], a2[2], a2[3], b0, b1);
       if (want_acc) {  // the code bytes: c & 7 plus 8 [c >= 8]
         uint32_t a3[4];
 #pragma unroll
@@ -792,7 +792,7 @@ __device__ __forceinline__ void bvsr_tile(const uint8_t* tp, const uint8_t* bp, 
         for (int qq = 0; qq < 2; qq++) {
           if (qq == 1 && !TWO) break;  // warp-uniform
           const int c = 2 * h + qq;
-          yacc[c] = fmaf(os[h].y, small_int_to_float(d1[c] + d2[c]), fmaf(os[h].x, gsf[qq], yacc[c]));
+          yacc[c] = fmaf(os[h].y, small_int_to_float(d1[c]), fmaf(os[h].x, gsf[qq], yacc[c]));
         }
       }
     }
