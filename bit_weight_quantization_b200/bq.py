@@ -75,7 +75,7 @@ for _name, (_res, _args) in _SIGS.items():
 EXPORTED = tuple(_SIGS)
 
 # the struct layouts below are those of this ABI version of include/bq.h
-BQ_ABI_VERSION = 3
+BQ_ABI_VERSION = 4
 if _lib.bq_version() != BQ_ABI_VERSION:
     raise ImportError(f"{LIB_PATH} has ABI version {_lib.bq_version()}, this binding needs {BQ_ABI_VERSION}; "
                       "rebuild it with bit_weight_quantization_b200.build.build(force=True)")

@@ -141,7 +141,14 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 // workspace (an act buffer) followed by the layer from that buffer: the per-token asymmetric
 // codes take a correctly rounded divide per element, which every CTA of the fused kernel would
 // otherwise repeat for its tokens.
-inline bool linear_via_act(const PkLayout& L, int M) { return L.fmt == BQ_FMT_ABQ && M >= 2; }
+// bq_linear quantizes the activations once into an act buffer and runs the layer from it:
+// ABQ from 2 tokens (its per-element divides would otherwise repeat in every CTA), and BVSR from
+// 16 (the code image holds 8 tokens a CTA where the fused staging holds 4: 5120x5120 at M = 16
+// 32.5 -> 24.4 us, at M = 64 199 -> 116 us; at M = 4 the fused call is faster, 14.6 vs 17.7 us)
+constexpr int kBvsrViaActM = 16;
+inline bool linear_via_act(const PkLayout& L, int M) {
+  return (L.fmt == BQ_FMT_ABQ && M >= 2) || (L.fmt == BQ_FMT_BVSR4 && M >= kBvsrViaActM);
+}
 
 // bq_linear scratch: the ternary LoRA partial dot products [KT][M][r] (f32), or the act buffer
 // of an ABQ layer of more than one token
@@ -274,11 +281,13 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   // tile costs about tile_c cycles (measured: ~145 per 8-MMA stream, ~900 for a BVSR tile);
   // each row block a warp group finishes costs about epi_c cycles (split-K exchange and
   // epilogue: ~1000 measured with a split, ~300 without). Ties go to the wider split.
+  // A BVSR tile is a latency-bound chain, so groups of fewer than 4 warps leave a CTA of one row
+  // block mostly idle whatever the model says (5120x13824: 2-warp groups 38.9 us, 4-warp 28.6).
   const int ipc = (L.RB + g->CPG - 1) / g->CPG;
   const long long tile_c = bvsr ? 900 : 145ll * L.nstreams;
   int wpr = 1;
   long long best = -1;
-  for (int w = NW; w >= 1; w /= 2) {
+  for (int w = NW; w >= (bvsr ? 4 : 1); w /= 2) {
     const int G = NW / w, T = (L.KT + w - 1) / w;
     long long load[4] = {0, 0, 0, 0};
     int max_items = 0;
@@ -331,6 +340,9 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   if (per_warp < 2ull * L.tile_bytes) return false;
   g->S = int(std::min<uint64_t>(4, std::max<uint64_t>(2, per_warp / L.tile_bytes)));
   g->C = int(std::max<uint64_t>(1, std::min<uint64_t>(g->T, per_warp / (uint64_t(g->S) * L.tile_bytes))));
+  // BVSR: the same four tiles in flight as two chunks of two (half the copy issues, each of which
+  // stalls its warp for ~0.3 us behind the other warps' shared-memory traffic)
+  if (bvsr && g->S == 4 && g->C == 1 && g->T >= 2) { g->S = 2; g->C = 2; }
   g->off_ring = take(uint64_t(std::max(1, active)) * g->S * g->C * L.tile_bytes);
   g->off_bar = take(uint64_t(NW * g->S + 3) * 8 + 16);
   g->smem_bytes = uint32_t(off);

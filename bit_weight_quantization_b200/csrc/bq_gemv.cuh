@@ -964,6 +964,17 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
         if (copies_ok) waited = e + 1;
         else *fail = 1;
       }
+      // BVSR refills the previous chunk's stage here, after this chunk's wait, rather than
+      // straight after computing it: the same chunks are in flight, and the copy issue (which
+      // stalls behind the shared-memory traffic of a BVSR tile) no longer sits between a
+      // chunk's compute and the next wait
+      if (BVSR && copies_ok && e >= 1 && e - 1 + a.S < n_my) {
+        if (lane == 0) {
+          fence_proxy_async();  // the previous stage's shared reads, before the last __syncwarp, are done
+          issue(e - 1 + a.S);
+        }
+        issued = e - 1 + a.S + 1;
+      }
       if (copies_ok && ok) {
         const uint8_t* sbase = ring + size_t(st) * a.C * a.tile_bytes + lane * 16;
         const int ktc = kt_begin + ci * a.C;
@@ -1000,7 +1011,7 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
         }
       }
       __syncwarp();
-      if (copies_ok && e + a.S < n_my) {
+      if (!BVSR && copies_ok && e + a.S < n_my) {
         if (lane == 0) {
           fence_proxy_async();  // this stage's shared reads are done before the copy overwrites it
           issue(e + a.S);

@@ -213,8 +213,9 @@ typedef struct {
  * 3: bq_pack_desc gained bvsr_cluster_rounds; the BVSR tile holds 4-bit codes in nibble order
  * (one stream) and its aux section 10 KB of pack scratch after the table; bq_linear on ABQ
  * with M >= 2 takes an act buffer in its workspace. The buffer version word stays 1 (a BVSR
- * buffer of the earlier layout has 4 streams in its header and is refused). */
-#define BQ_ABI_VERSION 3
+ * buffer of the earlier layout has 4 streams in its header and is refused).
+ * 4: bq_linear on BVSR with M >= 16 also takes an act buffer in its workspace. */
+#define BQ_ABI_VERSION 4
 
 const char* bq_status_str(bq_status s);
 int32_t bq_version(void);
@@ -265,8 +266,9 @@ bq_status bq_gemm(const bq_layer* layer, const void* act, int32_t M, float* y,
  * layer kernel's prologue, so y [M][N] f32 comes from x (device bf16 [M][K], 16-byte
  * aligned) in one launch (two for the ternary format with a LoRA term, whose
  * partial dot products of x and A are computed first into `workspace`; and two for ABQ with
- * M >= 2, which quantizes the activations once into an act buffer in `workspace` and runs the
- * layer from it, since its per-element divides would otherwise be repeated by every CTA).
+ * M >= 2 and BVSR with M >= 16, which quantize the activations once into an act buffer in
+ * `workspace` and run the layer from it: ABQ's per-element divides would otherwise be repeated
+ * by every CTA, and BVSR's code image holds twice the tokens per CTA that the fused staging does).
  * Results are identical to bq_quantize_act + bq_gemm. `workspace` (device, 256-byte aligned) must hold
  * bq_linear_workspace_bytes(layer, M) bytes; it may be NULL when that is 0.
  * Launched with programmatic dependent launch: consecutive layer calls on one stream
@@ -303,7 +305,8 @@ bq_status bq_linear_group(const bq_layer* layers, int32_t n_layers, const void* 
  *    bq_linear_workspace_bytes(layer, M) > 1 MiB, returns BQ_ERR_SIZE and enqueues
  *    nothing. Two cases use scratch: the ternary format with a LoRA term, K_pad/256 * M *
  *    rank * 4 bytes (e.g. K = 16384, M = 64, rank = 64 is exactly 1 MiB), and ABQ with
- *    M >= 2, its act buffer of about M * K_pad bytes (e.g. K = 4096, M = 64: 263 KiB).
+ *    M >= 2 or BVSR with M >= 16, the act buffer of about M * K_pad bytes (e.g. ABQ K = 4096,
+ *    M = 64: 263 KiB; BVSR adds M * K_pad / 8 bytes of vector sums).
  *  - Setup: the first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current) and keeps it together with the
  *    current context's id; a failure there returns BQ_ERR_CUDA. The address belongs to

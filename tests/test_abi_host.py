@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_status_strings_and_version():
-    assert bq.bq_version() == bq.BQ_ABI_VERSION == 3
+    assert bq.bq_version() == bq.BQ_ABI_VERSION == 4
     hdr = open(os.path.join(ROOT, "include", "bq.h")).read()
     assert re.search(r"#define BQ_ABI_VERSION (\d+)", hdr).group(1) == str(bq.BQ_ABI_VERSION)
 
@@ -320,8 +320,8 @@ def test_linear_plan_invariants(fmt, N, K, kw, M, fused):
     chunks = lambda t: -(-npad // (256 // pow2(t)))
     tpc, J = p["tokens_per_cta"], p["x_chunks_per_thread"]
     assert 1 <= tpc <= min(8, M) and p["token_groups"] == -(-M // tpc)
-    if fmt == "abq" and M >= 2:   # bq_linear quantizes once into an act buffer, then the layer
-        fused = False
+    if (fmt == "abq" and M >= 2) or (fmt == "bvsr" and M >= 16):   # bq_linear quantizes once
+        fused = False                                                # into an act buffer, then the layer
     if fused:   # the most tokens whose x fits 16 chunks per thread; else one token read twice
         fits = [t for t in range(1, min(8, M) + 1) if chunks(t) <= 16]
         assert tpc == (max(fits) if fits else 1)
@@ -334,6 +334,7 @@ def test_linear_plan_invariants(fmt, N, K, kw, M, fused):
     assert CPG == max(1, min(RB, -(-cps * 148 // p["token_groups"])))
     wpr, T = p["warps_per_row_block"], p["tiles_per_warp"]
     assert wpr in (1, 2, 4, 8) and T == -(-KT // wpr)
+    assert fmt != "bvsr" or wpr >= 4   # a BVSR tile is a long chain: at least 4 warps a row block
     S, C = p["ring_stages"], p["tiles_per_stage"]
     ipc = -(-RB // CPG)
     active = min(8 // wpr, ipc) * wpr   # warps that hold row blocks share the ring
@@ -540,6 +541,18 @@ def test_bvsr_cluster_rounds_are_checked():
         st = bq.raw_status("bq_packed_bytes", ctypes.byref(d), 64, 256, ctypes.byref(ctypes.c_size_t()))
         assert (st == bq.BQ_OK) == ok, (fmt, r, st)
     assert layer is not None and fake
+
+
+@pytest.mark.parametrize("M", [1, 4, 15, 16, 17, 64])
+def test_bvsr_linear_workspace_is_the_act_buffer_from_16_tokens(M):
+    """bq_linear on BVSR runs fused (no workspace) below 16 tokens and through an act buffer
+    (its workspace) from 16 on."""
+    layer = bq.bq_packed_validate(_host_header("bvsr", 512, 1280).tobytes(), 1 << 30)
+    ws = bq.bq_linear_workspace_bytes(layer, M)
+    if M < 16:
+        assert ws == 0
+    else:
+        assert ws == bq.bq_act_bytes(layer, M) > 0
 
 
 @pytest.mark.parametrize("M", [2, 15, 16, 17, 33, 64])

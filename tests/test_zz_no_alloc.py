@@ -22,7 +22,8 @@ def _layer(fmt, N, K, rank=32, seed=0):
 
 @pytest.mark.parametrize("fmt,N,K,M,rank", [("ternary", 2048, 2048, 4, 32), ("ternary", 300, 1280, 16, 64),
                                             ("bitnet", 4096, 4096, 1, 0), ("abq", 300, 4096, 8, 0),
-                                            ("abq", 4096, 4096, 64, 0), ("abq", 200, 1280, 17, 0)])
+                                            ("abq", 4096, 4096, 64, 0), ("abq", 200, 1280, 17, 0),
+                                            ("bvsr", 512, 1280, 16, 0), ("bvsr", 300, 5120, 64, 0)])
 def test_static_scratch_matches_workspace_call(fmt, N, K, M, rank):
     torch, bq = torch_mods()
     ql = _layer(fmt, N, K, rank)
