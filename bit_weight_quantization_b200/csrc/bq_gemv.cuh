@@ -1108,21 +1108,49 @@ __global__ void __launch_bounds__(NW * 32) k_rabit(LayerArgs a) {
   const int W32 = a.K_pad / 32;
   const uint32_t* pl = a.rabit_planes + size_t(row) * W32;   // path p: + p N_pad W32
   const size_t pstride = size_t(a.N_pad) * W32;
+  // 128-k chunks: lane l owns k = 128c + 4l .. 4l + 3, i.e. bits 4(l & 7) .. + 3 of the chunk's
+  // plane word l >> 3. Per chunk and path the warp makes one 16-byte load of the four plane words
+  // (the same address for every lane), one float4 of h (or of h x, unfused) and one 8-byte load
+  // of four bf16 of x: 128-bit, coalesced loads. K is a multiple of 128, so a chunk lies wholly
+  // below K or wholly in the padding (x read as 0 there).
+  const int sh = 4 * (lane & 7), wsel = lane >> 3;
   for (int m = 0; m < a.M; m++) {
     float acc[P];
 #pragma unroll
     for (int p = 0; p < P; p++) acc[p] = 0.f;
-#pragma unroll 8
-    for (int wd = 0; wd < W32; wd++) {
-      const int k = wd * 32 + lane;
-      float xv = 0.f;
-      if (FUSED) xv = k < a.K ? bf16_bits_to_float(a.x[size_t(m) * a.K + k]) : 0.f;
+    // four chunks at a time: every load of the four issued before the first use
+    for (int c0 = 0; c0 < W32 / 4; c0 += 4) {
+      uint4 wv[4][P];
+      float4 hv[4][P];
+      uint2 xb[4];
 #pragma unroll
-      for (int p = 0; p < P; p++) {
-        const uint32_t b = __ldg(pl + p * pstride + wd);
-        const float xp = FUSED ? __fmul_rn(__ldg(a.rabit_h + size_t(p) * a.K_pad + k), xv)
-                               : __ldg(a.act_xt + (size_t(p) * a.M + m) * a.K_pad + k);
-        acc[p] += __uint_as_float(__float_as_uint(xp) ^ (((b >> lane) & 1u) << 31));
+      for (int cc = 0; cc < 4; cc++) {
+        const int c = c0 + cc, k = 128 * c + 4 * lane;
+        if (c >= W32 / 4) break;
+        xb[cc] = FUSED && 128 * c < a.K ? __ldg(reinterpret_cast<const uint2*>(a.x + size_t(m) * a.K + k)) : make_uint2(0, 0);
+#pragma unroll
+        for (int p = 0; p < P; p++) {
+          wv[cc][p] = __ldg(reinterpret_cast<const uint4*>(pl + p * pstride) + c);
+          hv[cc][p] = FUSED ? __ldg(reinterpret_cast<const float4*>(a.rabit_h + size_t(p) * a.K_pad + k))
+                            : __ldg(reinterpret_cast<const float4*>(a.act_xt + (size_t(p) * a.M + m) * a.K_pad + k));
+        }
+      }
+#pragma unroll
+      for (int cc = 0; cc < 4; cc++) {
+        if (c0 + cc >= W32 / 4) break;
+        const float xv[4] = {bf16_bits_to_float(uint16_t(xb[cc].x & 0xFFFFu)), bf16_bits_to_float(uint16_t(xb[cc].x >> 16)),
+                             bf16_bits_to_float(uint16_t(xb[cc].y & 0xFFFFu)), bf16_bits_to_float(uint16_t(xb[cc].y >> 16))};
+#pragma unroll
+        for (int p = 0; p < P; p++) {
+          const uint4 w4 = wv[cc][p];
+          const uint32_t wd = wsel == 0 ? w4.x : wsel == 1 ? w4.y : wsel == 2 ? w4.z : w4.w;
+          const float4 h4 = hv[cc][p];
+          const float xp[4] = {FUSED ? __fmul_rn(h4.x, xv[0]) : h4.x, FUSED ? __fmul_rn(h4.y, xv[1]) : h4.y,
+                               FUSED ? __fmul_rn(h4.z, xv[2]) : h4.z, FUSED ? __fmul_rn(h4.w, xv[3]) : h4.w};
+#pragma unroll
+          for (int jj = 0; jj < 4; jj++)
+            acc[p] += __uint_as_float(__float_as_uint(xp[jj]) ^ (((wd >> (sh + jj)) & 1u) << 31));
+        }
       }
     }
 #pragma unroll
