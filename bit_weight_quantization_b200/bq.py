@@ -284,7 +284,9 @@ class StepGraph:
     write are fixed in the graph, so a step refreshes their contents (e.g. one copy into the
     input buffer), calls ``replay()``, and reads the outputs. ``replay()`` enqueues the whole
     step on torch's current stream. The library allocates nothing and never synchronizes in
-    its compute calls, which is what makes them capturable."""
+    its compute calls, which is what makes them capturable. ``issue()`` may fork work onto other
+    streams and join it back before returning (e.g. read each call's outputs back to pinned host
+    memory on a copy stream while the later calls run)."""
 
     def __init__(self, issue, stream=None, warmup: int = 1):
         import torch
