@@ -259,7 +259,9 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   const int rank = L.fmt == BQ_FMT_TERNARY_A8 ? L.rank : 0;
   const int npad = L.K_pad / 8;
   g->cstride = L.KT * 256 + 16;
-  int tpc = std::min(8, M);
+  // BVSR from an act buffer takes up to 16 tokens a CTA (two MMA groups on each decoded weight
+  // fragment, so the layer is decoded once per 16 tokens); everything else at most 8
+  int tpc = std::min(bvsr && !fused ? bqi::kMaxTpc : 8, M);
   if (fused) {
     auto J = [&](int t) { return (npad + NT / pow2ceil(t) - 1) / (NT / pow2ceil(t)); };
     while (tpc > 1 && J(tpc) > kMaxXChunks) tpc--;
@@ -272,9 +274,9 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   g->TG = (M + tpc - 1) / tpc;
   // BVSR tiles are long latency-bound instruction chains (about 400 instructions a 2176-byte
   // tile): at one token per CTA, two CTAs of the same launch share each SM so that 16 warps
-  // hide each other's latency; the other formats (and multi-token BVSR, whose code image is
-  // large) keep about one CTA per SM, leaving room for the next launch's.
-  const int ctas_per_sm = bvsr && tpc == 1 ? 2 : 1;
+  // hide each other's latency; the other formats (and multi-token or act-buffer BVSR, whose code
+  // image is large and whose kernel takes more registers) keep about one CTA per SM.
+  const int ctas_per_sm = bvsr && tpc == 1 && fused ? 2 : 1;
   g->CPG = std::max(1, std::min(L.RB, (ctas_per_sm * sm_count() + g->TG - 1) / g->TG));
   // Warps sharing a row block (the k-split), a power of two: the one with the least modelled
   // time. Warp w issues on SM sub-partition w % 4, where the MMA and field-mask issue of a
@@ -317,7 +319,7 @@ inline bool plan_layer(const PkLayout& L, int M, bool fused, LayerArgs* g) {
   g->off_tab = take(bvsr ? uint64_t(kBvsrSets) * kBvsrTableStride * 4 + 4 * 16 : 16);  // + the family tables
   // split-K exchange [G][2][WPR][32][4] of int64 (+ f32 for BVSR) when warps share a row
   // block; at least the staging reductions' 3 x 32 words
-  g->off_red = take(wpr > 1 ? 2ull * NW * 32 * 4 * (bvsr ? 12 : 8) : 512);
+  g->off_red = take(wpr > 1 ? 2ull * NW * 32 * 4 * (bvsr ? 12 : 8) * (tpc > 8 ? 2 : 1) : 512);
   // ternary: the B^T rows of the CTA's row blocks (32 rank bytes each) when they fit in 32 KB
   const uint64_t lbt = uint64_t(ipc) * 32 * rank;
   g->lbt_smem = rank > 0 && lbt <= 32 * 1024;

@@ -172,9 +172,10 @@ struct LayerArgs {
 // activation staging into shared memory
 // ---------------------------------------------------------------------------
 constexpr int kMaxXChunks = 16;   // 16-byte chunks of x held in registers per thread
-// shared token area (words): [8][4] per-token parameters, then tanh(alpha) and the weight scale
-// and the group members' weight scales
-constexpr int kTokAlpha = 32, kTokWScale = 33, kTokWords = 40;
+// shared token area (words): [16][4] per-token parameters (at most 16 tokens a CTA: BVSR from
+// an act buffer; 8 otherwise), then tanh(alpha) and the group members' weight scales
+constexpr int kMaxTpc = 16;
+constexpr int kTokAlpha = 4 * kMaxTpc, kTokWScale = kTokAlpha + 1, kTokWords = kTokWScale + 8;
 
 // asymmetric a-bit code: clamp(rn(x / Delta) + z, 0, 2^a - 1)
 __device__ __forceinline__ int quant_asym(float x, float d, int z, int qmax) {
@@ -746,14 +747,21 @@ struct BvsrFam {
 // load each) are unrolled into one block, so that the loads and MMAs of later pairs overlap the
 // float epilogue of earlier ones; the tile's set bytes for rows g and g + 8 are i0, i1 (byte j
 // of the pair of words).
+// G2: the CTA holds a second group of 8 tokens (8..15, BVSR from an act buffer only): its codes
+// bp2, code sums gs_row2 and flags tok2/tok3 go through a second MMA on the same decoded A
+// operand, into yacc2 / cacc2.
+template <bool G2>
 __device__ __forceinline__ void bvsr_tile(const uint8_t* tp, const uint8_t* bp, bool has_tok, uint2 i0, uint2 i1,
                                           const float* tab, const BvsrFam* fam, const int* gs_row, int VPR,
                                           bool TWO, bool tok0, bool tok1, bool want_acc, float (&yacc)[4],
-                                          long long (&cacc)[4]) {
+                                          long long (&cacc)[4], const uint8_t* bp2, bool has_tok2,
+                                          const int* gs_row2, bool tok2, bool tok3, float (&yacc2)[4],
+                                          long long (&cacc2)[4]) {
 #pragma unroll
   for (int jp = 0; jp < 4; jp++) {
     const uint4 q = lds128(tp + jp * 512);
     const uint4 bq = has_tok ? lds128(bp + jp * 16) : make_uint4(0, 0, 0, 0);
+    const uint4 bq2 = G2 && has_tok2 ? lds128(bp2 + jp * 16) : make_uint4(0, 0, 0, 0);
     const uint32_t iw0 = jp < 2 ? i0.x : i0.y, iw1 = jp < 2 ? i1.x : i1.y;
 #pragma unroll
     for (int v = 0; v < 2; v++) {
@@ -772,6 +780,8 @@ __device__ __forceinline__ void bvsr_tile(const uint8_t* tp, const uint8_t* bp, 
       }
       int d1[4] = {0, 0, 0, 0};
       mma_u8<true>(d1, a1[0], a1[1], a1[2], a1[3], b0, b1);
+      int e1[4] = {0, 0, 0, 0};
+      if (G2) mma_u8<true>(e1, a1[0], a1[1], a1[2], a1[3], v ? bq2.z : bq2.x, v ? bq2.w : bq2.y);
       if (want_acc) {  // the code bytes: c & 7 plus 8 [c >= 8]
         uint32_t a3[4];
 #pragma unroll
@@ -781,6 +791,12 @@ __device__ __forceinline__ void bvsr_tile(const uint8_t* tp, const uint8_t* bp, 
         mma_u8<true>(d3, a3[0], a3[1], a3[2], a3[3], b0, b1);
 #pragma unroll
         for (int c = 0; c < 4; c++) cacc[c] += d3[c];
+        if (G2) {
+          int e3[4] = {0, 0, 0, 0};
+          mma_u8<true>(e3, a3[0], a3[1], a3[2], a3[3], v ? bq2.z : bq2.x, v ? bq2.w : bq2.y);
+#pragma unroll
+          for (int c = 0; c < 4; c++) cacc2[c] += e3[c];
+        }
       }
       const float2 os[2] = {*reinterpret_cast<const float2*>(tab + s0 * kBvsrTableStride + 4),
                             *reinterpret_cast<const float2*>(tab + s1 * kBvsrTableStride + 4)};
@@ -794,6 +810,12 @@ __device__ __forceinline__ void bvsr_tile(const uint8_t* tp, const uint8_t* bp, 
           const int c = 2 * h + qq;
           yacc[c] = fmaf(os[h].y, small_int_to_float(d1[c]), fmaf(os[h].x, gsf[qq], yacc[c]));
         }
+      }
+      if (G2) {
+        const float gsf2[2] = {tok2 ? small_int_to_float(gs_row2[j]) : 0.f, tok3 ? small_int_to_float(gs_row2[VPR + j]) : 0.f};
+#pragma unroll
+        for (int c = 0; c < 4; c++)
+          yacc2[c] = fmaf(os[c >> 1].y, small_int_to_float(e1[c]), fmaf(os[c >> 1].x, gsf2[c & 1], yacc2[c]));
       }
     }
   }
@@ -810,10 +832,11 @@ __device__ __forceinline__ void bvsr_tile(const uint8_t* tp, const uint8_t* bp, 
 // epilogue: after the prologue there is no block-wide synchronization.
 // ---------------------------------------------------------------------------
 // Two CTAs per SM (at most 128 registers a thread): the next launch's CTA must fit beside
-// this one to prefetch its weights.
+// this one to prefetch its weights. BVSR from an act buffer (up to 16 tokens, two MMA groups)
+// runs one CTA per SM and takes the registers of a whole half of the file.
 // T1: every CTA holds one token (tpc = 1); the kernel then carries only the one-token staging.
 template <int FMT, int F0, int F1, int F2, int NW, bool FUSED, bool T1>
-__global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ LayerArgs a) {
+__global__ void __launch_bounds__(NW * 32, (FMT == BQ_FMT_BVSR4 && !FUSED) ? 1 : 2) k_layer(const __grid_constant__ LayerArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr bool BSIGNED = FMT != BQ_FMT_ABQ;
   constexpr bool BVSR = FMT == BQ_FMT_BVSR4;
@@ -927,6 +950,11 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
 
   const bool has_tok = g < mg;
   const uint8_t* bsrc = smem + a.off_codes + size_t(has_tok ? g : 0) * a.cstride + t * 64;
+  // BVSR with more than 8 tokens in the CTA (from an act buffer): tokens 8..15 are a second MMA
+  // group on the same decoded weights (warp-uniform)
+  const bool TG2 = BVSR && !FUSED && mg > 8;
+  const bool has_tok2 = TG2 && 8 + g < mg;
+  const uint8_t* bsrc2 = smem + a.off_codes + size_t(has_tok2 ? 8 + g : 0) * a.cstride + t * 64;
   const int VPR = a.K_pad / 32;
   const int* gsum = reinterpret_cast<const int*>(smem + a.off_gsum);
   const float* tab = reinterpret_cast<const float*>(smem + a.off_tab);
@@ -934,6 +962,9 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
   const bool want_acc = a.gl[0].acc != nullptr;  // BVSR (never grouped)
   long long* redl = reinterpret_cast<long long*>(smem + a.off_red);                // [G][2][WPR][32][4]
   float* redf = reinterpret_cast<float*>(smem + a.off_red + 2 * NW * 32 * 4 * 8);  // same shape
+  // the second token group's exchange (BVSR, more than 8 tokens) follows, in the same layout
+  long long* redl2 = reinterpret_cast<long long*>(smem + a.off_red + 2 * NW * 32 * 4 * 12);
+  float* redf2 = reinterpret_cast<float*>(smem + a.off_red + 2 * NW * 32 * 4 * 20);
   bool copies_ok = true;
   int waited = 0, issued = first;  // chunks this warp has waited for / has issued
 
@@ -941,8 +972,8 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
   constexpr int W1 = F1 > 0 ? F1 : 1, A1 = F1 > 0 ? 8 / F1 : 1;
   constexpr int W2 = F2 > 0 ? F2 : 1, A2 = F2 > 0 ? 8 / F2 : 1;
   int c0[A0][4], c1[A1][4], c2[A2][4];
-  float yacc[4];
-  long long cacc[4];
+  float yacc[4], yacc2[4];
+  long long cacc[4], cacc2[4];
 
   for (int gi = 0; gi < n_gitems; gi++) {
     if (gi > 0) load_rowp<FMT>(a, rb_of(gi), lane, rp);
@@ -953,7 +984,7 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
 #pragma unroll
     for (int j = 0; j < A2; j++) c2[j][0] = c2[j][1] = c2[j][2] = c2[j][3] = 0;
 #pragma unroll
-    for (int c = 0; c < 4; c++) { yacc[c] = 0.f; cacc[c] = 0; }
+    for (int c = 0; c < 4; c++) { yacc[c] = 0.f; cacc[c] = 0; yacc2[c] = 0.f; cacc2[c] = 0; }
     for (int ci = 0; ci < cpw; ci++) {
       const int e = gi * cpw + ci;
       const int cnt = chunk_tiles(e);
@@ -1005,8 +1036,14 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
             const uint8_t* tidx = tp - lane * 16 + 2048;
             const uint2 i0 = *reinterpret_cast<const uint2*>(tidx + g * 8);
             const uint2 i1 = *reinterpret_cast<const uint2*>(tidx + (g + 8) * 8);
-            bvsr_tile(tp, bsrc + kt * 256, has_tok, i0, i1, tab, fam, gsum + size_t(2 * t) * VPR + kt * 8, VPR, mg > 1, 2 * t < mg,
-                      2 * t + 1 < mg, want_acc, yacc, cacc);
+            const int* gs0 = gsum + size_t(2 * t) * VPR + kt * 8;
+            if (!FUSED && TG2)
+              bvsr_tile<true>(tp, bsrc + kt * 256, has_tok, i0, i1, tab, fam, gs0, VPR, true, 2 * t < mg, 2 * t + 1 < mg,
+                              want_acc, yacc, cacc, bsrc2 + kt * 256, has_tok2, gs0 + size_t(8) * VPR, 8 + 2 * t < mg,
+                              9 + 2 * t < mg, yacc2, cacc2);
+            else
+              bvsr_tile<false>(tp, bsrc + kt * 256, has_tok, i0, i1, tab, fam, gs0, VPR, mg > 1, 2 * t < mg,
+                               2 * t + 1 < mg, want_acc, yacc, cacc, bsrc2, false, gs0, false, false, yacc2, cacc2);
           }
         }
       }
@@ -1034,8 +1071,14 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
       for (int c = 0; c < 4; c++) p[c] = cacc[c];
     }
     const int rb = rb_of(gi);
+    long long p2[4];
+#pragma unroll
+    for (int c = 0; c < 4; c++) p2[c] = cacc2[c];
     if (WPR == 1) {
-      if (ok && !*fail) layer_epilogue<FMT>(a, smem, tokp, rb, m0, mg, lane, rp, lbt_of(gi), p, yacc);
+      if (ok && !*fail) {
+        layer_epilogue<FMT>(a, smem, tokp, rb, m0, mg, lane, rp, lbt_of(gi), p, yacc);
+        if (TG2) layer_epilogue<FMT>(a, smem, tokp + 32, rb, m0 + 8, mg - 8, lane, rp, lbt_of(gi), p2, yacc2);
+      }
       continue;
     }
     const int buf = gi & 1;
@@ -1046,10 +1089,14 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
 #pragma unroll
       for (int c = 0; c < 4; c++) redf[slot * 4 + c] = yacc[c];
     }
+    if (TG2) {
+#pragma unroll
+      for (int c = 0; c < 4; c++) { redl2[slot * 4 + c] = p2[c]; redf2[slot * 4 + c] = yacc2[c]; }
+    }
     asm volatile("bar.sync %0, %1;\n" ::"r"(1 + grp), "r"(WPR * 32) : "memory");
     if (wg != gi % WPR || !ok || *fail) continue;
-    long long pl[4] = {0, 0, 0, 0};
-    float yl[4] = {0.f, 0.f, 0.f, 0.f};
+    long long pl[4] = {0, 0, 0, 0}, pl2[4] = {0, 0, 0, 0};
+    float yl[4] = {0.f, 0.f, 0.f, 0.f}, yl2[4] = {0.f, 0.f, 0.f, 0.f};
     for (int w = 0; w < WPR; w++) {  // in warp order
       const size_t s2 = ((size_t(grp) * 2 + buf) * WPR + w) * 32 + lane;
       const longlong2 v0 = *reinterpret_cast<const longlong2*>(redl + s2 * 4);
@@ -1059,8 +1106,13 @@ __global__ void __launch_bounds__(NW * 32, 2) k_layer(const __grid_constant__ La
         const float4 f = *reinterpret_cast<const float4*>(redf + s2 * 4);
         yl[0] += f.x; yl[1] += f.y; yl[2] += f.z; yl[3] += f.w;
       }
+      if (TG2) {
+#pragma unroll
+        for (int c = 0; c < 4; c++) { pl2[c] += redl2[s2 * 4 + c]; yl2[c] += redf2[s2 * 4 + c]; }
+      }
     }
     layer_epilogue<FMT>(a, smem, tokp, rb, m0, mg, lane, rp, lbt_of(gi), pl, yl);
+    if (TG2) layer_epilogue<FMT>(a, smem, tokp + 32, rb, m0 + 8, mg - 8, lane, rp, lbt_of(gi), pl2, yl2);
   }
   // copies issued but never waited for (an abandoned wait) must land before the block exits
   if (!copies_ok)

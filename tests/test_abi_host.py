@@ -307,6 +307,12 @@ def _plan_cases():
             ("bvsr", 5120, 13824, {}), ("bvsr", 64, 256, {})]
 
 
+def fused_call(fmt, M, fused):
+    """Whether bq_linear runs the fused kernel (ABQ from 2 tokens and BVSR from 16 go through
+    an act buffer), or fused is False (bq_gemm)."""
+    return fused and not ((fmt == "abq" and M >= 2) or (fmt == "bvsr" and M >= 16))
+
+
 @pytest.mark.parametrize("fmt,N,K,kw", _plan_cases())
 @pytest.mark.parametrize("M", [1, 3, 8, 9, 64])
 @pytest.mark.parametrize("fused", [True, False])
@@ -319,7 +325,8 @@ def test_linear_plan_invariants(fmt, N, K, kw, M, fused):
     pow2 = lambda t: 1 << (t - 1).bit_length()
     chunks = lambda t: -(-npad // (256 // pow2(t)))
     tpc, J = p["tokens_per_cta"], p["x_chunks_per_thread"]
-    assert 1 <= tpc <= min(8, M) and p["token_groups"] == -(-M // tpc)
+    tmax = 16 if fmt == "bvsr" and not fused_call(fmt, M, fused) else 8   # BVSR from an act buffer: two MMA groups
+    assert 1 <= tpc <= min(tmax, M) and p["token_groups"] == -(-M // tpc)
     if (fmt == "abq" and M >= 2) or (fmt == "bvsr" and M >= 16):   # bq_linear quantizes once
         fused = False                                                # into an act buffer, then the layer
     if fused:   # the most tokens whose x fits 16 chunks per thread; else one token read twice
@@ -328,8 +335,8 @@ def test_linear_plan_invariants(fmt, N, K, kw, M, fused):
         assert J == (chunks(tpc) if fits else 0)
     else:       # the most tokens whose int8 codes fit 96 KB
         cstride = KT * 256 + 16
-        assert J == 0 and tpc == max([t for t in range(1, min(8, M) + 1) if t * cstride <= 96 * 1024] + [1])
-    cps = 2 if fmt == "bvsr" and tpc == 1 else 1   # CTAs of one launch per SM (148 SMs when no device)
+        assert J == 0 and tpc == max([t for t in range(1, min(tmax, M) + 1) if t * cstride <= 96 * 1024] + [1])
+    cps = 2 if fmt == "bvsr" and tpc == 1 and fused else 1   # CTAs of one launch per SM (148 SMs when no device)
     CPG = p["ctas_per_group"]
     assert CPG == max(1, min(RB, -(-cps * 148 // p["token_groups"])))
     wpr, T = p["warps_per_row_block"], p["tiles_per_warp"]

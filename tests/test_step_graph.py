@@ -35,3 +35,39 @@ def test_step_graph_replays_the_eager_calls():
         bq.bq_device_check()
         for a, b in zip(got, (ya, yb, yc)):
             assert np.array_equal(a, b.cpu().numpy())
+
+
+def test_step_graph_with_readbacks_forked_onto_a_copy_stream():
+    """The pattern of the bench's end-to-end step: each call's output is read back to pinned
+    host memory on a copy stream as soon as the call is done, inside the captured step, and
+    the copy stream joins before the step ends. Every replay's host copies equal the eager
+    results of the same inputs."""
+    torch, bq = torch_mods()
+    layers = [bq.QuantLinear("bitnet", to_dev_f32(I.weights(n, 1280, seed=5 + i))) for i, n in enumerate((300, 200, 150))]
+    x = torch.empty((1, 1280), dtype=torch.bfloat16, device="cuda")
+    ys = [torch.empty((1, L.N), device="cuda") for L in layers]
+    hs = [torch.empty((1, L.N)).pin_memory() for L in layers]
+    copy_stream = torch.cuda.Stream()
+
+    def issue():
+        for L, y, h in zip(layers, ys, hs):
+            L.linear(x, y)
+            done = torch.cuda.Event()
+            done.record()
+            copy_stream.wait_event(done)
+            with torch.cuda.stream(copy_stream):
+                h.copy_(y, non_blocking=True)
+        torch.cuda.current_stream().wait_stream(copy_stream)
+
+    g = bq.StepGraph(issue)
+    for step in range(3):
+        x.copy_(to_dev_bf16(I.activations(1, 1280, seed=30 + step)))
+        g.replay()
+        torch.cuda.synchronize()
+        got = [h.numpy().copy() for h in hs]
+        for L, y in zip(layers, ys):
+            L.linear(x, y)
+        torch.cuda.synchronize()
+        bq.bq_device_check()
+        for a, y in zip(got, ys):
+            assert np.array_equal(a, y.cpu().numpy())
