@@ -268,7 +268,8 @@ bq_status bq_gemm(const bq_layer* layer, const void* act, int32_t M, float* y,
  * partial dot products of x and A are computed first into `workspace`; and two for ABQ with
  * M >= 2 and BVSR with M >= 16, which quantize the activations once into an act buffer in
  * `workspace` and run the layer from it: ABQ's per-element divides would otherwise be repeated
- * by every CTA, and BVSR's code image holds twice the tokens per CTA that the fused staging does).
+ * by every CTA, and BVSR's code image holds up to 16 tokens a CTA where the fused staging holds
+ * 4 at K = 5120).
  * Results are identical to bq_quantize_act + bq_gemm. `workspace` (device, 256-byte aligned) must hold
  * bq_linear_workspace_bytes(layer, M) bytes; it may be NULL when that is 0.
  * Launched with programmatic dependent launch: consecutive layer calls on one stream
@@ -329,7 +330,8 @@ bq_status bq_linear_static_scratch(const bq_layer* layer, const void* x_bf16, in
  * enqueued. BQ_ERR_UNSUPPORTED if the layer does not fit the tiled kernel, or for RaBiT
  * (not tiled). The SM count is the current device's (148 when no device is visible). */
 typedef struct {
-  int32_t tokens_per_cta;         /* tokens sharing a CTA's MMA columns (<= 8) */
+  int32_t tokens_per_cta;         /* tokens sharing a CTA's MMA columns (<= 8; BVSR from an act
+                                     buffer <= 16, two MMA groups) */
   int32_t token_groups;           /* CTA groups, one per tokens_per_cta tokens */
   int32_t ctas_per_group;         /* persistent CTAs per token group (grid = product) */
   int32_t warps_per_row_block;    /* warps splitting K over one 16-row block (power of two) */
