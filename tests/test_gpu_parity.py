@@ -11,7 +11,8 @@ import pytest
 import bq_inputs as I
 from oracle import cref as O
 from tests.parity_util import (GpuLayer, assert_codes_near_tie, assert_y_close, check_act, oracle_layer,
-                               oracle_pack, rabit_near, ternary_near, to_dev_bf16, to_dev_f32, ulp_diff)
+                               oracle_pack, rabit_near, ternary_near, to_dev_bf16, to_dev_f32, torch_mods,
+                               ulp_diff)
 
 pytestmark = pytest.mark.gpu
 
@@ -127,6 +128,20 @@ def test_max_tokens(fmt, N, K):
     p = _pack_parity(gl, fmt)
     check_act(gl)
     _layer_parity(gl, p, fmt)
+
+
+@pytest.mark.parametrize("N,K,M", [(97, 640, 12), (50, 2560, 16), (40, 5120, 13), (33, 128, 16)])
+def test_bvsr_two_token_groups(N, K, M):
+    """BVSR from an act buffer holds up to 16 tokens a CTA as two 8-token MMA groups on each
+    decoded weight fragment: second groups partly and fully filled, ragged N. Below 16 tokens
+    the fused call (at most 8 tokens a CTA) equals act + gemm (two groups) bit for bit, which
+    GpuLayer checks; both match the oracle."""
+    torch, bq = torch_mods()
+    gl = GpuLayer("bvsr", N, K, M, seed=N + K + M)
+    assert bq.bq_linear_plan(gl.ql.layer, M, False)["tokens_per_cta"] == M
+    p = _pack_parity(gl, "bvsr")
+    check_act(gl)
+    _layer_parity(gl, p, "bvsr")
 
 
 @pytest.mark.parametrize("N,K", SMALL)
